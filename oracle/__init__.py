@@ -1,0 +1,151 @@
+"""TEST INFRASTRUCTURE ONLY: fp64 CPU oracle for the Finch-C2 / RWKV-6 WKV recurrence.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import this package.  The product library (libgoldwkv) never
+links, loads or calls it, and the two share no code.
+
+The arithmetic lives in ``wkv6_oracle.c`` (plain sequential loops, fp64), which follows
+the GoldFinch review page, section 3.4 "Finch-C2 Time Mixing": decay
+``w_t = exp(-exp(d_t))`` ("Data-dependent decay"), the state sum
+``wkv_t = sum_{i<t} diag(prod_{j=i+1}^{t-1} w_j) k_i^T v_i`` ("Recurrent state update and
+output"), readout ``r_t . wkv_t`` plus the base-Finch static bonus ``r_t . diag(u) k_t^T v_t``,
+and LayerNorm over the concatenated heads.  This module only builds/loads the shared
+object and marshals numpy arrays.
+
+Pins: every entry point is checked by ``tests/test_oracle_pins.py`` against brute-force
+sums, closed forms and invariants that do not call this code (see that file's header).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "wkv6_oracle.c"
+_BUILD = _HERE / "_build"
+_SO = _BUILD / "libwkv6_oracle.so"
+
+
+def build(src: Path = _SRC, out: Path = _SO, extra_flags=()) -> Path:
+    """Compile the oracle C source with gcc into a shared object (no -march tuning)."""
+    out.parent.mkdir(parents=True, exist_ok=True)
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread", *extra_flags,
+           str(src), "-o", str(out), "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build(so: Path, src: Path) -> bool:
+    return (not so.exists()) or so.stat().st_mtime < src.stat().st_mtime
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+class Oracle:
+    """ctypes front end of one compiled oracle shared object."""
+
+    def __init__(self, so_path: Path | str | None = None):
+        if so_path is None:
+            if _needs_build(_SO, _SRC):
+                build()
+            so_path = _SO
+        self.path = Path(so_path)
+        lib = ctypes.CDLL(str(self.path))
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.wkv6_oracle_prefill.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                            dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.wkv6_oracle_prefill.restype = ctypes.c_int
+        lib.wkv6_oracle_decode_step.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.wkv6_oracle_decode_step.restype = ctypes.c_int
+        lib.wkv6_oracle_layernorm.argtypes = [ctypes.c_long, ctypes.c_int, dp, dp, dp,
+                                              ctypes.c_double, dp]
+        lib.wkv6_oracle_layernorm.restype = ctypes.c_int
+        self._lib = lib
+
+    @staticmethod
+    def _f64(a):
+        if a is None:
+            return None
+        return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+    @staticmethod
+    def _ptr(a):
+        if a is None:
+            return None
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+    def prefill(self, r, k, v, omega, u, state_in=None, nthreads: int | None = None):
+        """r,k,v,omega: [B,T,H,D]; u: [H,D]; state_in: [B,H,D,D] or None.
+
+        Returns (y [B,T,H,D], state_out [B,H,D,D]) as float64 arrays.
+        """
+        r, k, v, omega, u = (self._f64(x) for x in (r, k, v, omega, u))
+        s_in = self._f64(state_in)
+        B, T, H, D = r.shape
+        assert k.shape == v.shape == omega.shape == r.shape and u.shape == (H, D)
+        if s_in is not None:
+            assert s_in.shape == (B, H, D, D)
+        y = np.empty_like(r)
+        s_out = np.empty((B, H, D, D), dtype=np.float64)
+        rc = self._lib.wkv6_oracle_prefill(B, T, H, D, self._ptr(r), self._ptr(k), self._ptr(v),
+                                           self._ptr(omega), self._ptr(u), self._ptr(s_in),
+                                           self._ptr(y), self._ptr(s_out),
+                                           nthreads or default_threads())
+        if rc != 0:
+            raise RuntimeError(f"oracle prefill failed rc={rc}")
+        return y, s_out
+
+    def decode_step(self, r, k, v, omega, u, state, nthreads: int | None = None):
+        """r,k,v,omega: [B,H,D]; state [B,H,D,D] (not modified). Returns (y, new_state)."""
+        r, k, v, omega, u = (self._f64(x) for x in (r, k, v, omega, u))
+        st = np.array(state, dtype=np.float64, copy=True, order="C")
+        B, H, D = r.shape
+        y = np.empty_like(r)
+        rc = self._lib.wkv6_oracle_decode_step(B, H, D, self._ptr(r), self._ptr(k), self._ptr(v),
+                                               self._ptr(omega), self._ptr(u), self._ptr(st),
+                                               self._ptr(y), nthreads or default_threads())
+        if rc != 0:
+            raise RuntimeError(f"oracle decode failed rc={rc}")
+        return y, st
+
+    def layernorm(self, x, gamma=None, beta=None, eps: float = 1e-5):
+        """LayerNorm over the last axis of x (any leading shape), fp64."""
+        x = self._f64(x)
+        C = x.shape[-1]
+        N = x.size // C
+        g = self._f64(gamma)
+        b = self._f64(beta)
+        out = np.empty_like(x)
+        rc = self._lib.wkv6_oracle_layernorm(N, C, self._ptr(x), self._ptr(g), self._ptr(b),
+                                             float(eps), self._ptr(out))
+        if rc != 0:
+            raise RuntimeError(f"oracle layernorm failed rc={rc}")
+        return out
+
+    def prefill_ln(self, r, k, v, omega, u, state_in, gamma, beta, eps=1e-5, nthreads=None):
+        """Prefill followed by LayerNorm over the concatenated heads (H*D) of each token."""
+        y, s = self.prefill(r, k, v, omega, u, state_in, nthreads)
+        B, T, H, D = y.shape
+        yl = self.layernorm(y.reshape(B, T, H * D), gamma, beta, eps).reshape(B, T, H, D)
+        return yl, s, y
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle built from ``wkv6_oracle.c`` (compiled on first use if missing or stale)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

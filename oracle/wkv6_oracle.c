@@ -1,0 +1,199 @@
+/*
+ * TEST INFRASTRUCTURE ONLY.  Plain, slow, obviously-correct fp64 CPU oracle for the
+ * Finch-C2 / RWKV-6 time-mix WKV recurrence.  Only the test suite, the smoke check and
+ * the benchmark's CPU-baseline leg may load this file; the product path (libgoldwkv)
+ * shares no code, header or constant with it.
+ *
+ * Source of the definition: "GoldFinch: High Performance RWKV/Transformer Hybrid ..."
+ * (paper-graph-ui review page), section 3.4, "Finch-C2 Time Mixing":
+ *   - data-dependent decay        w_t = exp(-exp(d_t))             ("Data-dependent decay")
+ *   - recurrent state             wkv_t = sum_{i<t} diag(prod_{j=i+1}^{t-1} w_j) k_i^T v_i
+ *                                                                 ("Recurrent state update and output")
+ *   - readout                     r_t . wkv_t  plus the base-Finch static bonus u
+ *                                 (the bonus enters as r_t . diag(u) k_t^T v_t)
+ *   - LayerNorm over the concatenation of all heads                ("... full concatenated dimension")
+ * Written in recursive form: with S_{-1} = state_in (zero if absent),
+ *   y_t[j] = sum_i r_t[i] S_{t-1}[i][j] + (sum_i r_t[i] u[i] k_t[i]) v_t[j]
+ *   S_t[i][j] = w_t[i] S_{t-1}[i][j] + k_t[i] v_t[j]
+ * so wkv_t of the page is S_{t-1} here: the newest outer product enters undecayed and
+ * w_t first touches the state when S_t is formed.  Rows of S (index i) are key/decay
+ * channels, columns (index j) value channels.
+ *
+ * Every function here is pinned by tests/test_oracle_pins.py against brute-force sums,
+ * closed forms and invariants that do not reuse this code.
+ *
+ * Layouts (row-major, fp64):
+ *   r, k, v, omega, y : [B][T][H][D]
+ *   u                 : [H][D]
+ *   state_in/out      : [B][H][D][D]   (state[b][h][i][j])
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* One (b,h) sequence, tokens t0..t0+T-1, element (t,c) of a token-major tensor at
+ * base[t*tstride + c]. */
+static void wkv6_one_head(long T, int D, long tstride,
+                          const double *r, const double *k, const double *v,
+                          const double *omega, const double *u,
+                          const double *s_in, double *y, double *s_out, double *S,
+                          double *w)
+{
+    for (int i = 0; i < D; ++i)
+        for (int j = 0; j < D; ++j)
+            S[i * D + j] = s_in ? s_in[i * D + j] : 0.0;
+
+    for (long t = 0; t < T; ++t) {
+        const double *rt = r + t * tstride;
+        const double *kt = k + t * tstride;
+        const double *vt = v + t * tstride;
+        const double *ot = omega + t * tstride;
+        double *yt = y + t * tstride;
+
+        /* decay of this token: w_t = exp(-exp(omega_t)) */
+        for (int i = 0; i < D; ++i)
+            w[i] = exp(-exp(ot[i]));
+
+        /* bonus coefficient sum_i r_t[i] u[i] k_t[i] */
+        double bonus = 0.0;
+        for (int i = 0; i < D; ++i)
+            bonus += rt[i] * u[i] * kt[i];
+
+        /* readout from the state before this token */
+        for (int j = 0; j < D; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < D; ++i)
+                acc += rt[i] * S[i * D + j];
+            yt[j] = acc + bonus * vt[j];
+        }
+
+        /* state update: decay rows, add the outer product k_t^T v_t */
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                S[i * D + j] = w[i] * S[i * D + j] + kt[i] * vt[j];
+    }
+
+    if (s_out)
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                s_out[i * D + j] = S[i * D + j];
+}
+
+typedef struct {
+    int B, H, D;
+    long T;
+    const double *r, *k, *v, *omega, *u, *s_in;
+    double *y, *s_out;
+    int next;               /* next (b*H+h) unit to take */
+    pthread_mutex_t lock;
+} job_t;
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const int D = J->D;
+    double *S = (double *)malloc(sizeof(double) * (size_t)D * D);
+    double *w = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!S || !w) {
+        free(S);
+        free(w);
+        return (void *)1;
+    }
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int unit = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (unit >= J->B * J->H)
+            break;
+        int b = unit / J->H, h = unit % J->H;
+        long tstride = (long)J->H * D;
+        size_t x0 = ((size_t)b * J->T * J->H + h) * D;      /* element (b, t=0, h, 0) */
+        size_t s0 = ((size_t)b * J->H + h) * D * D;
+        wkv6_one_head(J->T, D, tstride, J->r + x0, J->k + x0, J->v + x0, J->omega + x0,
+                      J->u + (size_t)h * D, J->s_in ? J->s_in + s0 : NULL, J->y + x0,
+                      J->s_out ? J->s_out + s0 : NULL, S, w);
+    }
+    free(S);
+    free(w);
+    return NULL;
+}
+
+/* Full prefill over [B][T][H][D] inputs.  state_in may be NULL (zeros); state_out may be
+ * NULL (not written) or equal state_in.  Runs the (b,h) units on nthreads POSIX threads.
+ * Returns 0 on success, -1 on bad arguments, -2 if a thread could not be started. */
+int wkv6_oracle_prefill(int B, long T, int H, int D,
+                        const double *r, const double *k, const double *v,
+                        const double *omega, const double *u, const double *state_in,
+                        double *y, double *state_out, int nthreads)
+{
+    if (B < 0 || T < 0 || H < 0 || D <= 0 || nthreads <= 0)
+        return -1;
+    if (B == 0 || H == 0)
+        return 0;
+    job_t J;
+    J.B = B; J.T = T; J.H = H; J.D = D;
+    J.r = r; J.k = k; J.v = v; J.omega = omega; J.u = u; J.s_in = state_in;
+    J.y = y; J.s_out = state_out;
+    J.next = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads > B * H)
+        nthreads = B * H;
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    int started = 0, rc = 0;
+    for (int n = 0; n < nthreads; ++n) {
+        if (pthread_create(&tid[n], NULL, worker, &J) != 0) {
+            rc = -2;
+            break;
+        }
+        ++started;
+    }
+    for (int n = 0; n < started; ++n) {
+        void *ret = NULL;
+        pthread_join(tid[n], &ret);
+        if (ret)
+            rc = -2;
+    }
+    free(tid);
+    pthread_mutex_destroy(&J.lock);
+    return rc;
+}
+
+/* One autoregressive step (T = 1) for every (b,h), state updated in place.
+ * r, k, v, omega, y : [B][H][D];  state : [B][H][D][D]. */
+int wkv6_oracle_decode_step(int B, int H, int D,
+                            const double *r, const double *k, const double *v,
+                            const double *omega, const double *u, double *state,
+                            double *y, int nthreads)
+{
+    return wkv6_oracle_prefill(B, 1, H, D, r, k, v, omega, u, state, y, state, nthreads);
+}
+
+/* LayerNorm of each of the N rows of x[N][C] over its C entries:
+ *   out = (x - mean) / sqrt(var + eps) * gamma + beta,  var the biased (1/C) variance.
+ * gamma/beta may be NULL (1 and 0).  out may equal x. */
+int wkv6_oracle_layernorm(long N, int C, const double *x, const double *gamma,
+                          const double *beta, double eps, double *out)
+{
+    if (N < 0 || C <= 0)
+        return -1;
+    for (long n = 0; n < N; ++n) {
+        const double *xr = x + n * (long)C;
+        double *orow = out + n * (long)C;
+        double mean = 0.0;
+        for (int c = 0; c < C; ++c)
+            mean += xr[c];
+        mean /= (double)C;
+        double var = 0.0;
+        for (int c = 0; c < C; ++c)
+            var += (xr[c] - mean) * (xr[c] - mean);
+        var /= (double)C;
+        double inv = 1.0 / sqrt(var + eps);
+        for (int c = 0; c < C; ++c) {
+            double g = gamma ? gamma[c] : 1.0;
+            double bb = beta ? beta[c] : 0.0;
+            orow[c] = (xr[c] - mean) * inv * g + bb;
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,261 @@
+"""Independent checks ("pins") of the fp64 oracle.
+
+None of these reuses the oracle's loop: each computes the expected result from another
+statement of the method on the GoldFinch review page, section 3.4 "Finch-C2 Time Mixing",
+or from mathematics that the definition fixes:
+
+* explicit_sum      - the page's state as an explicit sum over past tokens of
+                      diag(prod_{j=i+1}^{t-1} w_j) k_i^T v_i ("Recurrent state update and
+                      output"), products formed one by one, O(T^3 D) brute force;
+* t1_closed_form    - a single token: y = (r.(u*k)) v + r S0, S1 = diag(w) S0 + k^T v;
+* decode_closed_form- the same closed form through the decode entry point;
+* linear_attention  - w == 1 and u = 0 is strictly causal linear attention
+                      ("Transformers are RNNs", cited on the citation-graph page):
+                      y = tril(R K^T, -1) V + R S0;
+* zero_decay        - w == 0 keeps one token of memory:
+                      y_t = (r_t.(u*k_t)) v_t + (r_t.k_{t-1}) v_{t-1},  S_T = k_{T-1}^T v_{T-1};
+* geometric         - per-channel constant decay with constant k, v from zero state:
+                      S_t[i][j] = k_i v_j (1 - w_i^t) / (1 - w_i)  (geometric series);
+* split_carry       - O(1)-per-token state passing: running [0, t1) then [t1, T) from the
+                      carried state equals the full run, for several t1;
+* linearity         - y and S are jointly linear in (v, S0), y is linear in r;
+* ln_moments        - LayerNorm output has mean 0 and variance var/(var+eps);
+* ln_torch          - LayerNorm equals torch.nn.functional.layer_norm in fp64;
+* ln_shift          - LayerNorm is invariant to adding a constant to every channel.
+
+``run_all(oracle)`` returns the list of failing pin names; the mutation test uses it to
+show that plausible mistakes planted in the oracle are caught.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+RTOL = 1e-11
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _inputs(seed, B, T, H, D, omega=(-6.0, 1.0), s0=True):
+    g = _rng(seed)
+    r = g.normal(0, 0.3, (B, T, H, D))
+    k = g.normal(0, 0.3, (B, T, H, D))
+    v = g.normal(0, 0.3, (B, T, H, D))
+    om = g.uniform(omega[0], omega[1], (B, T, H, D))
+    u = g.normal(0, 0.5, (H, D))
+    S0 = g.normal(0, 0.1, (B, H, D, D)) if s0 else np.zeros((B, H, D, D))
+    return r, k, v, om, u, S0
+
+
+def _close(a, b, rtol=RTOL):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    scale = max(1e-300, float(np.max(np.abs(b))) if b.size else 1.0)
+    return a.shape == b.shape and float(np.max(np.abs(a - b))) <= rtol * scale if a.size else True
+
+
+def brute_force_explicit(r, k, v, om, u, S0):
+    """y and final state from the explicit-sum form, every product taken one by one."""
+    B, T, H, D = r.shape
+    w = np.exp(-np.exp(om))
+    y = np.zeros_like(r)
+    S_fin = np.zeros((B, H, D, D))
+    for b in range(B):
+        for h in range(H):
+            for t in range(T + 1):
+                # wkv_t: state seen by token t (t == T gives the final state)
+                wkv = np.zeros((D, D))
+                decay0 = np.ones(D)
+                for j in range(0, t):
+                    decay0 = decay0 * w[b, j, h]
+                wkv = wkv + decay0[:, None] * S0[b, h]
+                for i in range(0, t):
+                    dec = np.ones(D)
+                    for j in range(i + 1, t):
+                        dec = dec * w[b, j, h]
+                    wkv = wkv + (dec * k[b, i, h])[:, None] * v[b, i, h][None, :]
+                if t < T:
+                    rt = r[b, t, h]
+                    bonus = float(np.sum(rt * u[h] * k[b, t, h]))
+                    y[b, t, h] = rt @ wkv + bonus * v[b, t, h]
+                else:
+                    S_fin[b, h] = wkv
+    return y, S_fin
+
+
+def pin_explicit_sum(o):
+    ok = True
+    for seed, (B, T, H, D), s0 in [(1, (2, 9, 2, 8), True), (2, (1, 6, 1, 64), True),
+                                   (3, (1, 12, 3, 4), False)]:
+        r, k, v, om, u, S0 = _inputs(seed, B, T, H, D, s0=s0)
+        y, S = o.prefill(r, k, v, om, u, S0)
+        ye, Se = brute_force_explicit(r, k, v, om, u, S0)
+        ok &= _close(y, ye) and _close(S, Se)
+    return ok
+
+
+def pin_t1_closed_form(o):
+    r, k, v, om, u, S0 = _inputs(4, 3, 1, 2, 16)
+    y, S = o.prefill(r, k, v, om, u, S0)
+    w = np.exp(-np.exp(om[:, 0]))
+    ok = True
+    for b in range(3):
+        for h in range(2):
+            rr, kk, vv = r[b, 0, h], k[b, 0, h], v[b, 0, h]
+            y_ref = np.dot(rr * u[h], kk) * vv + rr @ S0[b, h]
+            S_ref = np.diag(w[b, h]) @ S0[b, h] + np.outer(kk, vv)
+            ok &= _close(y[b, 0, h], y_ref) and _close(S[b, h], S_ref)
+    return ok
+
+
+def pin_decode_closed_form(o):
+    g = _rng(5)
+    B, H, D = 4, 3, 64
+    r, k, v = (g.normal(0, 0.3, (B, H, D)) for _ in range(3))
+    om = g.uniform(-6, 1, (B, H, D))
+    u = g.normal(0, 0.5, (H, D))
+    S0 = g.normal(0, 0.1, (B, H, D, D))
+    y, S = o.decode_step(r, k, v, om, u, S0)
+    w = np.exp(-np.exp(om))
+    y_ref = np.einsum("bhi,hi,bhi->bh", r, u, k)[..., None] * v + np.einsum("bhi,bhij->bhj", r, S0)
+    S_ref = w[..., None] * S0 + k[..., :, None] * v[..., None, :]
+    return _close(y, y_ref) and _close(S, S_ref)
+
+
+def pin_linear_attention(o):
+    r, k, v, _, _, S0 = _inputs(6, 2, 33, 2, 16)
+    om = np.full_like(r, -60.0)          # exp(-exp(-60)) == 1.0 in fp64
+    assert np.all(np.exp(-np.exp(om)) == 1.0)
+    u = np.zeros((2, 16))
+    y, S = o.prefill(r, k, v, om, u, S0)
+    ok = True
+    for b in range(2):
+        for h in range(2):
+            R, K, V = r[b, :, h], k[b, :, h], v[b, :, h]
+            y_ref = np.tril(R @ K.T, -1) @ V + R @ S0[b, h]
+            S_ref = S0[b, h] + K.T @ V
+            ok &= _close(y[b, :, h], y_ref) and _close(S[b, h], S_ref)
+    return ok
+
+
+def pin_zero_decay(o):
+    r, k, v, _, u, S0 = _inputs(7, 2, 20, 2, 16)
+    om = np.full_like(r, 8.0)            # exp(-exp(8)) == 0.0 in fp64
+    assert np.all(np.exp(-np.exp(om)) == 0.0)
+    y, S = o.prefill(r, k, v, om, u, S0)
+    ok = True
+    for b in range(2):
+        for h in range(2):
+            R, K, V = r[b, :, h], k[b, :, h], v[b, :, h]
+            bonus = np.sum(R * u[h] * K, axis=1)
+            y_ref = bonus[:, None] * V
+            y_ref[0] += R[0] @ S0[b, h]
+            y_ref[1:] += np.sum(R[1:] * K[:-1], axis=1)[:, None] * V[:-1]
+            ok &= _close(y[b, :, h], y_ref) and _close(S[b, h], np.outer(K[-1], V[-1]))
+    return ok
+
+
+def pin_geometric(o):
+    g = _rng(8)
+    T, H, D = 50, 2, 16
+    om_c = g.uniform(-3, 0.5, (H, D))
+    k_c = g.normal(0, 0.3, (H, D))
+    v_c = g.normal(0, 0.3, (H, D))
+    r = g.normal(0, 0.3, (1, T, H, D))
+    u = g.normal(0, 0.5, (H, D))
+    om = np.broadcast_to(om_c, (1, T, H, D)).copy()
+    k = np.broadcast_to(k_c, (1, T, H, D)).copy()
+    v = np.broadcast_to(v_c, (1, T, H, D)).copy()
+    y, S = o.prefill(r, k, v, om, u, None)
+    w = np.exp(-np.exp(om_c))
+    ok = True
+    for h in range(H):
+        geo_T = (1 - w[h] ** T) / (1 - w[h])
+        ok &= _close(S[0, h], (k_c[h] * geo_T)[:, None] * v_c[h][None, :])
+        for t in range(T):
+            geo_t = (1 - w[h] ** t) / (1 - w[h])
+            y_ref = np.dot(r[0, t, h], k_c[h] * geo_t) * v_c[h] + np.dot(r[0, t, h] * u[h], k_c[h]) * v_c[h]
+            ok &= _close(y[0, t, h], y_ref)
+    return ok
+
+
+def pin_split_carry(o):
+    r, k, v, om, u, S0 = _inputs(9, 2, 40, 2, 16)
+    y, S = o.prefill(r, k, v, om, u, S0)
+    ok = True
+    for t1 in (1, 17, 20, 39):
+        y1, S1 = o.prefill(r[:, :t1], k[:, :t1], v[:, :t1], om[:, :t1], u, S0)
+        y2, S2 = o.prefill(r[:, t1:], k[:, t1:], v[:, t1:], om[:, t1:], u, S1)
+        ok &= _close(np.concatenate([y1, y2], axis=1), y, 1e-12) and _close(S2, S, 1e-12)
+    return ok
+
+
+def pin_linearity(o):
+    r, k, v1, om, u, S1 = _inputs(10, 2, 25, 2, 16)
+    _, _, v2, _, _, S2 = _inputs(11, 2, 25, 2, 16)
+    ya, Sa = o.prefill(r, k, v1, om, u, S1)
+    yb, Sb = o.prefill(r, k, v2, om, u, S2)
+    yc, Sc = o.prefill(r, k, v1 + v2, om, u, S1 + S2)
+    yd, _ = o.prefill(2.5 * r, k, v1, om, u, S1)
+    return _close(yc, ya + yb, 1e-12) and _close(Sc, Sa + Sb, 1e-12) and _close(yd, 2.5 * ya, 1e-12)
+
+
+def pin_ln_moments(o):
+    g = _rng(12)
+    x = g.normal(0.3, 2.0, (7, 96))
+    eps = 1e-5
+    out = o.layernorm(x, None, None, eps)
+    var_x = x.var(axis=1)
+    return (float(np.max(np.abs(out.mean(axis=1)))) < 1e-12 and
+            _close(out.var(axis=1), var_x / (var_x + eps), 1e-12))
+
+
+def pin_ln_torch(o):
+    g = _rng(13)
+    x = g.normal(0.0, 1.5, (5, 3, 64))
+    gam = 1.0 + 0.1 * g.normal(size=64)
+    bet = 0.1 * g.normal(size=64)
+    out = o.layernorm(x, gam, bet, 1e-5)
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (64,), torch.from_numpy(gam),
+                                         torch.from_numpy(bet), 1e-5).numpy()
+    return _close(out, ref, 1e-12)
+
+
+def pin_ln_shift(o):
+    g = _rng(14)
+    x = g.normal(0.0, 1.0, (6, 128))
+    gam = 1.0 + 0.1 * g.normal(size=128)
+    bet = 0.1 * g.normal(size=128)
+    a = o.layernorm(x, gam, bet, 1e-5)
+    b = o.layernorm(x + 3.25, gam, bet, 1e-5)
+    return _close(a, b, 1e-10)
+
+
+PINS = {
+    "explicit_sum": pin_explicit_sum,
+    "t1_closed_form": pin_t1_closed_form,
+    "decode_closed_form": pin_decode_closed_form,
+    "linear_attention": pin_linear_attention,
+    "zero_decay": pin_zero_decay,
+    "geometric": pin_geometric,
+    "split_carry": pin_split_carry,
+    "linearity": pin_linearity,
+    "ln_moments": pin_ln_moments,
+    "ln_torch": pin_ln_torch,
+    "ln_shift": pin_ln_shift,
+}
+
+
+def run_all(o):
+    """Names of the pins that the given oracle fails."""
+    failed = []
+    for name, fn in PINS.items():
+        try:
+            ok = bool(fn(o))
+        except Exception:  # a crash counts as a failure
+            ok = False
+        if not ok:
+            failed.append(name)
+    return failed

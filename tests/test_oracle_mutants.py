@@ -1,0 +1,60 @@
+"""Plant plausible mistakes in (copies of) the oracle and check that the pins catch each.
+
+Each mutant replaces one exact statement of ``oracle/wkv6_oracle.c`` (the statement must
+occur exactly once, so the test tracks the source), is compiled to a temporary shared
+object with gcc, and must fail at least one pin of ``tests/pins.py``.  CPU only.
+"""
+import pathlib
+
+import pytest
+
+import oracle as oracle_pkg
+from tests import pins
+
+SRC = pathlib.Path(oracle_pkg.__file__).parent / "wkv6_oracle.c"
+
+MUTANTS = {
+    # decay transform wrong: single exponential, or sign flipped inside
+    "decay_single_exp": ("w[i] = exp(-exp(ot[i]));", "w[i] = exp(-ot[i]);"),
+    "decay_sign": ("w[i] = exp(-exp(ot[i]));", "w[i] = exp(-exp(-ot[i]));"),
+    # bonus term: u dropped, or the whole bonus dropped
+    "bonus_without_u": ("bonus += rt[i] * u[i] * kt[i];", "bonus += rt[i] * kt[i];"),
+    "bonus_dropped": ("yt[j] = acc + bonus * vt[j];", "yt[j] = acc;"),
+    # decay applied to value columns instead of key rows
+    "decay_on_columns": ("S[i * D + j] = w[i] * S[i * D + j] + kt[i] * vt[j];",
+                         "S[i * D + j] = w[j] * S[i * D + j] + kt[i] * vt[j];"),
+    # outer product transposed
+    "outer_transposed": ("S[i * D + j] = w[i] * S[i * D + j] + kt[i] * vt[j];",
+                         "S[i * D + j] = w[i] * S[i * D + j] + kt[j] * vt[i];"),
+    # new outer product decayed by the current token
+    "decay_after_add": ("S[i * D + j] = w[i] * S[i * D + j] + kt[i] * vt[j];",
+                        "S[i * D + j] = w[i] * (S[i * D + j] + kt[i] * vt[j]);"),
+    # readout through the transposed state
+    "readout_transposed": ("acc += rt[i] * S[i * D + j];", "acc += rt[i] * S[j * D + i];"),
+    # readout from the state after this token's update (off by one in time)
+    "readout_after_update": ("acc += rt[i] * S[i * D + j];",
+                             "acc += rt[i] * (w[i] * S[i * D + j] + kt[i] * vt[j]);"),
+    # initial state ignored
+    "state_in_ignored": ("S[i * D + j] = s_in ? s_in[i * D + j] : 0.0;", "S[i * D + j] = 0.0;"),
+    # LayerNorm: unbiased variance, eps outside the square root, beta dropped, mean not removed
+    "ln_unbiased_var": ("var /= (double)C;", "var /= (double)(C - 1);"),
+    "ln_eps_outside": ("double inv = 1.0 / sqrt(var + eps);", "double inv = 1.0 / (sqrt(var) + eps);"),
+    "ln_beta_dropped": ("orow[c] = (xr[c] - mean) * inv * g + bb;", "orow[c] = (xr[c] - mean) * inv * g;"),
+    "ln_mean_kept": ("orow[c] = (xr[c] - mean) * inv * g + bb;", "orow[c] = xr[c] * inv * g + bb;"),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    before, after = MUTANTS[name]
+    text = SRC.read_text()
+    assert text.count(before) == 1, f"mutant {name}: statement not found exactly once"
+    mutated = tmp_path / f"{name}.c"
+    mutated.write_text(text.replace(before, after))
+    so = oracle_pkg.build(mutated, tmp_path / f"lib{name}.so")
+    failed = pins.run_all(oracle_pkg.Oracle(so))
+    assert failed, f"mutant {name} passes every pin"
+
+
+def test_unmutated_oracle_passes_all_pins(oracle):
+    assert pins.run_all(oracle) == []
