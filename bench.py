@@ -1,0 +1,429 @@
+#!/usr/bin/env python3
+"""Benchmark of the WKV6 hot path on B200: prefill tokens/s (+ decode GB/s), one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step): one wkv6_prefill call over the 1.5B-class layer shape,
+B=8, T=4096, H=32, D=64, bf16 r/k/v/omega/y, fp32 u and state, initial state ~N(0,0.1)
+(seeded synthetic data).  The inputs (537 MB) exceed the 126 MB L2, so no flush is needed
+between timed steps.  For N > 1 (torchrun, one rank per GPU) every rank runs its own
+independent batch of that shape (weak scaling; the path has no collective) and `value` is
+all tokens of all ranks over the slowest rank's device time.
+
+The line also reports: the dominant kernel's roofline fraction (algorithmic bytes per
+launch / CUDA-event launch time vs. the measured HBM copy bandwidth), SM clocks sampled
+with nvidia-smi during the timed region, an end-to-end figure through the public API with
+host buffers (pinned host -> device inputs, prefill, device -> host y and state inside the
+timed region), the fp64 oracle timed on the host cores on a bounded sample, and the decode
+step (B=256, H=32, 100 steps, state updated in place) in GB/s against the same roofline.
+
+`--impl reference` times the oracle (the only reference implementation of this path) on the
+host cores on the same workload, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from linear_attention_rnn_finch_b200 import workloads as W  # noqa: E402
+
+METRIC = "WKV prefill tokens/s (H=32, D=64) and decode GB/s; fraction of roofline"
+PREFILL_CFG = W.CONFIGS[1]
+DECODE_CFG = W.CONFIGS[3]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def prefill_bytes(B, T, H, D=64, esz=2):
+    """Algorithmic HBM bytes of one prefill launch: r, k, v, omega in, y out (per
+    token-head 5*D*esz), fp32 state in and out (2*D*D*4 per head), u."""
+    return 5 * D * esz * B * T * H + 2 * D * D * 4 * B * H + H * D * 4
+
+
+def decode_bytes(B, H, D=64, esz=2):
+    """Algorithmic bytes of one decode step: state read + written, r/k/v/omega in, y out."""
+    return B * H * (2 * D * D * 4 + 5 * D * esz) + H * D * 4
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------------ clock sampler
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.marks = {}
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, name):
+        self.marks[name] = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]),
+                                 reasons={n: ("Active" in v) for n, v in zip(self.REASONS, f[5:9])}))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({n for r in rows for n, a in r["reasons"].items() if a})
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ oracle timing
+def oracle_sample(cfg, b_rows: int, t_tokens: int, seed_offset: int = 0):
+    """Inputs of the oracle's bounded sample: b_rows batch rows x t_tokens tokens of cfg,
+    drawn by the same seeded generator on the host."""
+    import numpy as np
+    inp = W.make_prefill_inputs(cfg, "cpu", B=b_rows, T=t_tokens, seed=cfg.seed + seed_offset)
+    a = [inp[n].to(torch.float64).numpy() for n in ("r", "k", "v", "omega")]
+    return a, inp["u"].double().numpy(), inp["state0"].double().numpy(), np
+
+
+def time_oracle(cfg, b_rows, t_tokens, reps=1):
+    import oracle as oracle_pkg
+    orc = oracle_pkg.get()
+    a, u, s0, _ = oracle_sample(cfg, b_rows, t_tokens)
+    nthreads = oracle_pkg.default_threads()
+    best = None
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        orc.prefill(*a, u, s0, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        best = dt if best is None else min(best, dt)
+    return b_rows * t_tokens / best, nthreads, best
+
+
+def sized_sample(cfg, seconds: float):
+    """(batch rows, tokens) of a sample the oracle finishes in about `seconds`, from a
+    short calibration run on 1 row x 128 tokens."""
+    tps, _, _ = time_oracle(cfg, 1, 128)
+    tokens = max(64, int(tps * seconds))
+    rows = max(1, min(cfg.B, tokens // cfg.T))
+    t_tok = cfg.T if rows > 1 else max(64, min(cfg.T, tokens))
+    return rows, t_tok
+
+
+# ------------------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    import linear_attention_rnn_finch_b200 as gw
+    from linear_attention_rnn_finch_b200 import binding
+
+    binding.load()
+    dev = torch.device("cuda", local)
+    cfg = PREFILL_CFG
+    B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
+    inp = W.make_prefill_inputs(cfg, dev, seed=cfg.seed + 17 * rank)
+    y = torch.empty_like(inp["r"])
+    s_out = torch.empty_like(inp["state0"])
+    stream = torch.cuda.current_stream(dev)
+    args_p = [inp[n] for n in ("r", "k", "v", "omega")]
+    algo = args.algo
+
+    def step():
+        gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], y=y, state_out=s_out, algo=algo)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # untimed warm-up: W steps, then ~1 s of steps so clocks settle and the sampler sees load
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark("t0")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    ev[-1].synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler.mark("t1")
+    launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms_max = max_over_ranks(total_ms, world)
+    tokens_all = sum_over_ranks(float(B * T * args.steps), world)
+    value = tokens_all / (total_ms_max / 1e3)
+    ms_per_step = total_ms_max / args.steps
+
+    hbm, peak_kind = peaks()
+    bytes_launch = prefill_bytes(B, T, H, D)
+    avg_launch_ms = statistics.mean(launch_ms)
+    achieved = bytes_launch / (avg_launch_ms / 1e3) / 1e9
+    launches_per_step = 1  # one prefill kernel per call (no LayerNorm in this workload)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "wkv6_prefill_1p5b_layer", "B": B, "T": T, "H": H, "D": D,
+                   "io": "bf16", "state": "fp32", "algo": algo,
+                   "parallelism": f"dp{world} (independent batches, no collective)",
+                   "l2": "inputs larger than L2 (537 MB in, 134 MB out per step)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                     "algorithmic_bytes_per_launch": bytes_launch,
+                     "kernel": "wkv6 prefill (algo=%s)" % algo},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+
+    # decode: 100 steps back to back, state in place; GB/s of algorithmic bytes
+    if not args.no_decode:
+        dcfg = DECODE_CFG
+        dinp = W.make_decode_inputs(dcfg, dev, seed=dcfg.seed + 17 * rank)
+        state = dinp["state0"].clone()
+        ybuf = torch.empty_like(dinp["r"][0])
+        dsteps = dcfg.steps
+        dargs = [[dinp[n][s] for n in ("r", "k", "v", "omega")] for s in range(dsteps)]
+
+        def dstep(s):
+            gw.wkv6_decode_step(*dargs[s], dinp["u"], state, y=ybuf)
+
+        for s in range(dsteps):
+            dstep(s)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(dsteps):
+            dstep(s)
+        e1.record(stream)
+        e1.synchronize()
+        barrier(world)
+        dms = max_over_ranks(e0.elapsed_time(e1), world) / dsteps
+        dbytes = decode_bytes(dcfg.B, dcfg.H, dcfg.D)
+        dgbs = dbytes / (dms / 1e3) / 1e9
+        out["decode"] = {"metric": "decode GB/s", "value": dgbs * world, "unit": "GB/s",
+                         "per_gpu_gbs": dgbs, "ms_per_step": dms, "steps": dsteps,
+                         "config": {"workload": "wkv6_decode_step", "B": dcfg.B, "H": dcfg.H,
+                                    "D": dcfg.D, "io": "bf16", "state": "fp32 in place",
+                                    "l2": "state 134 MB > L2"},
+                         "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm,
+                                      "unit": "GB/s", "frac": dgbs / hbm, "traffic": None,
+                                      "algorithmic_bytes_per_launch": dbytes}}
+        del dinp, dargs, state
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        host = {n: inp[n].cpu().pin_memory() for n in ("r", "k", "v", "omega", "u", "state0")}
+        dbuf = {n: torch.empty_like(inp[n]) for n in host}
+        y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        s_h = torch.empty(s_out.shape, dtype=s_out.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = y_h.numel() * y_h.element_size() + s_h.numel() * s_h.element_size()
+
+        def e2e_step():
+            for n in host:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            gw.wkv6_prefill(dbuf["r"], dbuf["k"], dbuf["v"], dbuf["omega"], dbuf["u"],
+                            dbuf["state0"], y=y, state_out=s_out, algo=algo)
+            y_h.copy_(y, non_blocking=True)
+            s_h.copy_(s_out, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        etok = sum_over_ranks(float(B * T * e2e_steps), world)
+        out["e2e"] = {"value": etok / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    sampler.stop()
+    out["clocks"] = sampler.summary(sampler.marks.get("t0", 0) - 1.0, sampler.marks.get("t1", 0))
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b_rows, t_tok = sized_sample(cfg, 12.0)
+        tps, cores, secs = time_oracle(cfg, b_rows, t_tok)
+        out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{b_rows} batch row x {t_tok} tokens x {H} heads of "
+                                         f"the same workload ({secs:.1f} s, fp64)"}
+    return out
+
+
+# ------------------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores; each step one bounded sample."""
+    if rank != 0:
+        return None
+    import oracle as oracle_pkg
+    cfg = PREFILL_CFG
+    orc = oracle_pkg.get()
+    # each step about 1.5 s of oracle work, so K + W steps end within a few minutes
+    b_rows, t_tok = sized_sample(cfg, 1.5)
+    a, u, s0, _ = oracle_sample(cfg, b_rows, t_tok)
+    nthreads = oracle_pkg.default_threads()
+    for _ in range(args.warmup):
+        orc.prefill(*a, u, s0, nthreads=nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.prefill(*a, u, s0, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    value = b_rows * t_tok * args.steps / dt
+    sample = f"{b_rows} batch row x {t_tok} tokens x {cfg.H} heads per step, fp64"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "wkv6_prefill_1p5b_layer", "B": cfg.B, "T": cfg.T, "H": cfg.H,
+                   "D": cfg.D, "io": "bf16 inputs, fp64 arithmetic"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--algo", choices=["auto", "recurrent", "chunked"], default="auto")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        # host-only arm: rank 0 runs the oracle and prints; other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    world, rank, local = dist_setup()
+    try:
+        out = run_ours(args, world, rank, local)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

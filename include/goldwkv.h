@@ -1,0 +1,136 @@
+/*
+ * libgoldwkv -- the Finch-C2 / RWKV-6 time-mix WKV recurrence on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (GoldFinch review page, section 3.4 "Finch-C2 Time Mixing"): per batch
+ * row b and head h, with head size D = 64, a D x D fp32 state S whose rows i are key /
+ * decay channels and whose columns j are value channels.  For each token t:
+ *
+ *     w_t[i]  = exp(-exp(omega_t[i]))                    ("Data-dependent decay")
+ *     y_t[j]  = sum_i r_t[i] * S[i][j]
+ *             + (sum_i r_t[i] * u[i] * k_t[i]) * v_t[j]   (base-Finch static bonus u)
+ *     S[i][j] = w_t[i] * S[i][j] + k_t[i] * v_t[j]        ("Recurrent state update and output":
+ *                                                          the state is the decayed sum of
+ *                                                          past outer products k_i^T v_i)
+ *
+ * Optionally y is passed through LayerNorm over the concatenation of all H heads of a
+ * token (d_model = H*D), as Finch-C2 uses in place of per-head GroupNorm:
+ *     y <- (y - mean) / sqrt(var + eps) * gamma + beta,  var the biased variance.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers r, k, v, omega, u, state*, y, gamma, beta, workspace are DEVICE pointers on
+ *    the current CUDA device; the caller owns every buffer.  The library never allocates
+ *    device memory, never synchronises and keeps no global mutable state, so calls on
+ *    different streams are independent.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously; a device-side fault surfaces as a CUDA error at the caller's
+ *    next synchronisation.
+ *  - Arguments are validated before anything is launched; on any error nothing is
+ *    launched and no output is touched.
+ *  - Layouts are row-major and dense:
+ *        r, k, v, omega, y : [B][T][H][D] (prefill) or [B][H][D] (decode), dtype `io`
+ *        u                 : [H][D] fp32
+ *        state             : [B][H][D][D] fp32, state[b][h][i][j]
+ *        gamma, beta       : [H*D] fp32
+ *  - All pointers must be 16-byte aligned.  y must not overlap r, k, v, omega, u or the
+ *    states.  state_out may equal state_in (in-place), but may not partially overlap it.
+ *  - omega is the decay logit d_t; the library forms w = exp(-exp(omega)) itself.
+ */
+#ifndef GOLDWKV_H
+#define GOLDWKV_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum wkv_status {
+    WKV_OK = 0,
+    WKV_ERR_INVALID_ARG = 1,   /* null / misaligned / overlapping pointer, negative size   */
+    WKV_ERR_UNSUPPORTED = 2,   /* D != 64, or a dtype / option combination not built      */
+    WKV_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed             */
+    WKV_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired                       */
+    WKV_ERR_WORKSPACE = 5      /* workspace missing or smaller than *_workspace_bytes()   */
+} wkv_status;
+
+typedef enum wkv_dtype {
+    WKV_F32 = 0,               /* fp32 r, k, v, omega and y                                */
+    WKV_BF16 = 1               /* bf16 r, k, v, omega and y                                */
+} wkv_dtype;
+
+typedef enum wkv_algo {
+    WKV_ALGO_AUTO = 0,         /* library picks (chunked tensor-core path where it applies) */
+    WKV_ALGO_RECURRENT = 1,    /* token-by-token fp32 recurrence on CUDA cores             */
+    WKV_ALGO_CHUNKED = 2       /* chunked prefill on tcgen05 tensor cores (bf16 I/O only)  */
+} wkv_algo;
+
+/* LayerNorm over the H*D concatenated head outputs of each token. */
+typedef struct wkv_ln {
+    const float *gamma;        /* [H*D] device, fp32, required                             */
+    const float *beta;         /* [H*D] device, fp32, required                             */
+    float eps;                 /* added to the variance inside the square root; > 0      */
+} wkv_ln;
+
+/* Bytes of device workspace wkv6_prefill needs for these sizes (0: none).  Depends only
+ * on its arguments. */
+size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
+                                    wkv_algo algo);
+
+/*
+ * Prefill: run the recurrence over T tokens for every (b,h), starting from state_in.
+ * Defined by the page's state sum and readout (section 3.4, "Recurrent state update and
+ * output"); the pre-fill procedure it serves is section 3.4 "Training and Inference
+ * Procedures" (tokens fed through the recurrence one by one or in parallel chunks).
+ *   r, k, v, omega  [B][T][H][D] io     inputs
+ *   u               [H][D] fp32         bonus
+ *   state_in        [B][H][D][D] fp32   or NULL for a zero initial state
+ *   state_out       [B][H][D][D] fp32   final state, or NULL (not written); may == state_in
+ *   y               [B][T][H][D] io     output (LayerNorm-ed when ln != NULL)
+ *   B, T, H >= 0 (B, H or T == 0 is an empty problem: with T == 0 state_out receives
+ *   state_in, or zeros), D == 64.
+ *   ln              NULL, or LayerNorm parameters
+ *   workspace       device scratch of at least wkv6_prefill_workspace_bytes(...) bytes
+ *                   (may be NULL when that is 0); contents on entry are ignored.
+ * Returns WKV_OK, or an error with nothing launched (INVALID_ARG, UNSUPPORTED, WORKSPACE)
+ * or WKV_ERR_CUDA if a launch failed.
+ */
+wkv_status wkv6_prefill(const void *r, const void *k, const void *v, const void *omega,
+                        const float *u, const float *state_in, float *state_out, void *y,
+                        int B, int T, int H, int D, wkv_dtype io, const wkv_ln *ln,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* As wkv6_prefill, with the algorithm chosen by the caller (WKV_ALGO_CHUNKED on fp32 I/O
+ * returns WKV_ERR_UNSUPPORTED). */
+wkv_status wkv6_prefill_algo(const void *r, const void *k, const void *v, const void *omega,
+                             const float *u, const float *state_in, float *state_out, void *y,
+                             int B, int T, int H, int D, wkv_dtype io, const wkv_ln *ln,
+                             wkv_algo algo, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/* Bytes of device workspace wkv6_decode_step needs (non-zero only with LayerNorm). */
+size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln);
+
+/*
+ * One autoregressive step (T = 1) for every (b,h), the state updated IN PLACE: the O(1)
+ * per-token recurrent update of section 3.4 "Training and Inference Procedures"
+ * (autoregressive generation) applied to the recurrence above.
+ *   r, k, v, omega  [B][H][D] io;  u [H][D] fp32;  state [B][H][D][D] fp32 (read, then
+ *   overwritten with the new state);  y [B][H][D] io (LayerNorm-ed when ln != NULL).
+ *   workspace: at least wkv6_decode_workspace_bytes(...) bytes.
+ */
+wkv_status wkv6_decode_step(const void *r, const void *k, const void *v, const void *omega,
+                            const float *u, float *state, void *y, int B, int H, int D,
+                            wkv_dtype io, const wkv_ln *ln, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *wkv6_status_string(wkv_status s);
+
+/* Version of this ABI (incremented on any signature change). */
+int wkv6_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GOLDWKV_H */

@@ -1,1 +1,11 @@
-"""B200 (sm_100a) WKV6 recurrence: chunked prefill and decode step behind a C ABI."""
+"""B200 (sm_100a) WKV6 recurrence: chunked prefill and decode step behind a C ABI.
+
+The compute lives in ``libgoldwkv.so`` (see ``include/goldwkv.h``); ``binding`` marshals
+torch tensors into it.  Importing this package does not load the library; the first call
+does, and raises if it was not built.
+"""
+from .binding import (WkvError, decode_workspace_bytes, load, prefill_workspace_bytes,
+                      wkv6_decode_step, wkv6_prefill)
+
+__all__ = ["WkvError", "decode_workspace_bytes", "load", "prefill_workspace_bytes",
+           "wkv6_decode_step", "wkv6_prefill"]

@@ -1,0 +1,195 @@
+"""Thin ctypes binding of libgoldwkv (include/goldwkv.h): argument marshalling only.
+
+Every step of the recurrence runs in the library's CUDA kernels; this module checks
+tensor placement / dtype / contiguity, allocates outputs and workspace with torch on the
+tensors' device, passes raw device pointers and the current CUDA stream, and turns a
+non-OK status into an exception.  There is no CPU fallback: if the library is missing or
+was not built, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libgoldwkv.so"
+
+WKV_OK, WKV_ERR_INVALID_ARG, WKV_ERR_UNSUPPORTED, WKV_ERR_CUDA, WKV_ERR_TIMEOUT, WKV_ERR_WORKSPACE = range(6)
+WKV_F32, WKV_BF16 = 0, 1
+ALGOS = {"auto": 0, "recurrent": 1, "chunked": 2}
+HEAD_SIZE = 64
+
+_lib = None
+
+
+class WkvError(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn}: {message} (status {status})")
+        self.status = status
+
+
+class _LN(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
+def load(path: Path | str | None = None):
+    """Load libgoldwkv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = Path(path) if path is not None else LIB_PATH
+    if not p.exists():
+        raise RuntimeError(
+            f"{p} not found: build it with `python -m linear_attention_rnn_finch_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(str(p))
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.wkv6_prefill_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    L.wkv6_prefill_workspace_bytes.restype = sz
+    L.wkv6_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.wkv6_decode_workspace_bytes.restype = sz
+    L.wkv6_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+    L.wkv6_prefill.restype = i
+    L.wkv6_prefill_algo.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, sz, vp]
+    L.wkv6_prefill_algo.restype = i
+    L.wkv6_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
+    L.wkv6_decode_step.restype = i
+    L.wkv6_status_string.argtypes = [i]
+    L.wkv6_status_string.restype = ctypes.c_char_p
+    L.wkv6_abi_version.argtypes = []
+    L.wkv6_abi_version.restype = i
+    if path is None:
+        _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().wkv6_status_string(status).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _io(dtype) -> int:
+    if dtype == torch.float32:
+        return WKV_F32
+    if dtype == torch.bfloat16:
+        return WKV_BF16
+    raise ValueError(f"unsupported I/O dtype {dtype}; expected float32 or bfloat16")
+
+
+def _check(name, t, device, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(device, stream):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ln_struct(ln, H, D, device):
+    if ln is None:
+        return None, None
+    gamma, beta, eps = ln
+    _check("ln.gamma", gamma, device, torch.float32, (H * D,))
+    _check("ln.beta", beta, device, torch.float32, (H * D,))
+    s = _LN(gamma.data_ptr(), beta.data_ptr(), float(eps))
+    return s, ctypes.byref(s)
+
+
+def _raise(fn, status):
+    if status != WKV_OK:
+        raise WkvError(fn, status, status_string(status))
+
+
+def prefill_workspace_bytes(B, T, H, D, io_dtype, with_ln, algo="auto") -> int:
+    return int(load().wkv6_prefill_workspace_bytes(B, T, H, D, _io(io_dtype), int(bool(with_ln)),
+                                                   ALGOS[algo]))
+
+
+def decode_workspace_bytes(B, H, D, io_dtype, with_ln) -> int:
+    return int(load().wkv6_decode_workspace_bytes(B, H, D, _io(io_dtype), int(bool(with_ln))))
+
+
+def wkv6_prefill(r, k, v, omega, u, state_in=None, *, ln=None, algo="auto", y=None,
+                 state_out=None, want_state=True, workspace=None, stream=None):
+    """Prefill over [B, T, H, D] inputs (fp32 or bf16), fp32 u [H, D] and optional fp32
+    state_in [B, H, D, D].  ``ln`` = (gamma, beta, eps) applies LayerNorm over H*D.
+
+    Returns (y, state_out); state_out is None when ``want_state`` is False and no
+    ``state_out`` tensor was given.  ``state_out`` may be ``state_in`` (in-place update).
+    """
+    L = load()
+    if r.dim() != 4:
+        raise ValueError("r must be [B, T, H, D]")
+    B, T, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega)):
+        _check(name, t, dev, dt, (B, T, H, D))
+    _check("u", u, dev, torch.float32, (H, D))
+    if state_in is not None:
+        _check("state_in", state_in, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, T, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, T, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _check("state_out", state_out, dev, torch.float32, (B, H, D, D))
+    ln_s, ln_p = _ln_struct(ln, H, D, dev)
+    need = int(L.wkv6_prefill_workspace_bytes(B, T, H, D, _io(dt), int(ln is not None), ALGOS[algo]))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6_prefill_algo(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state_in),
+                                 _ptr(state_out), _ptr(y), B, T, H, D, _io(dt), ln_p, ALGOS[algo],
+                                 _ptr(workspace), ws_bytes, _stream_ptr(dev, stream))
+    del ln_s
+    _raise("wkv6_prefill", st)
+    return y, state_out
+
+
+def wkv6_decode_step(r, k, v, omega, u, state, *, ln=None, y=None, workspace=None, stream=None):
+    """One step over [B, H, D] inputs; ``state`` [B, H, D, D] fp32 is updated in place.
+    Returns y [B, H, D]."""
+    L = load()
+    if r.dim() != 3:
+        raise ValueError("r must be [B, H, D]")
+    B, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega)):
+        _check(name, t, dev, dt, (B, H, D))
+    _check("u", u, dev, torch.float32, (H, D))
+    _check("state", state, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, H, D))
+    ln_s, ln_p = _ln_struct(ln, H, D, dev)
+    need = int(L.wkv6_decode_workspace_bytes(B, H, D, _io(dt), int(ln is not None)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6_decode_step(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state),
+                                _ptr(y), B, H, D, _io(dt), ln_p, _ptr(workspace), ws_bytes,
+                                _stream_ptr(dev, stream))
+    del ln_s
+    _raise("wkv6_decode_step", st)
+    return y

@@ -1,0 +1,250 @@
+// libgoldwkv C ABI: argument validation and dispatch to the kernels.  Declarations and
+// the contract of each entry point are in include/goldwkv.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "goldwkv.h"
+#include "internal.h"
+
+namespace {
+
+constexpr int kHeadSizeApi = 64;  // D: the only head size the kernels are built for
+
+struct Span {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Span span(const void* p, size_t bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Span{a, a + bytes};
+}
+
+bool overlaps(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host-side fault injection for tests of the error paths: GOLDWKV_FAULT=launch makes the
+// entry points report a failed launch without launching anything.
+bool injected(const char* what) {
+    const char* f = getenv("GOLDWKV_FAULT");
+    return f != nullptr && strcmp(f, what) == 0;
+}
+
+// p must be memory the current device can address as device memory.
+bool on_current_device(const void* p, int dev) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    if (a.type == cudaMemoryTypeDevice) return a.device == dev;
+    if (a.type == cudaMemoryTypeManaged) return true;
+    return false;
+}
+
+struct Buf {
+    const void* p;
+    size_t bytes;
+    bool required;
+};
+
+// Common pointer checks: required non-null, 16-byte aligned, on the current device.
+wkv_status check_bufs(const Buf* bufs, int n) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return WKV_ERR_CUDA;
+    }
+    for (int i = 0; i < n; ++i) {
+        if (bufs[i].p == nullptr) {
+            if (bufs[i].required) return WKV_ERR_INVALID_ARG;
+            continue;
+        }
+        if (!aligned16(bufs[i].p)) return WKV_ERR_INVALID_ARG;
+        if (!on_current_device(bufs[i].p, dev)) return WKV_ERR_INVALID_ARG;
+    }
+    return WKV_OK;
+}
+
+wkv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA; }
+
+size_t io_size(wkv_dtype io) { return io == WKV_BF16 ? 2 : 4; }
+
+bool valid_io(wkv_dtype io) { return io == WKV_F32 || io == WKV_BF16; }
+
+wkv_status check_ln(const wkv_ln* ln, int H, int D, int dev_check) {
+    if (ln == nullptr) return WKV_OK;
+    if (!(ln->eps > 0.f) || ln->eps != ln->eps || ln->eps > 1e30f) return WKV_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)H * D * sizeof(float);
+    Buf b[2] = {{ln->gamma, bytes, true}, {ln->beta, bytes, true}};
+    (void)dev_check;
+    return check_bufs(b, 2);
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv6_abi_version(void) { return 1; }
+
+const char* wkv6_status_string(wkv_status s) {
+    switch (s) {
+        case WKV_OK: return "ok";
+        case WKV_ERR_INVALID_ARG: return "invalid argument";
+        case WKV_ERR_UNSUPPORTED: return "unsupported (head size must be 64; chunked path needs bf16 I/O)";
+        case WKV_ERR_CUDA: return "CUDA launch or runtime error";
+        case WKV_ERR_TIMEOUT: return "bounded device wait expired";
+        case WKV_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
+                                    wkv_algo algo) {
+    (void)algo;
+    if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
+    if (with_ln && io == WKV_BF16) return (size_t)B * T * H * D * sizeof(float);
+    return 0;
+}
+
+size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln) {
+    if (B <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
+    if (with_ln && io == WKV_BF16) return (size_t)B * H * D * sizeof(float);
+    return 0;
+}
+
+wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const void* omega,
+                             const float* u, const float* state_in, float* state_out, void* y,
+                             int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
+                             wkv_algo algo, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
+    if (algo != WKV_ALGO_AUTO && algo != WKV_ALGO_RECURRENT && algo != WKV_ALGO_CHUNKED)
+        return WKV_ERR_INVALID_ARG;
+    if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
+    if (algo == WKV_ALGO_CHUNKED && io != WKV_BF16) return WKV_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (B == 0 || H == 0) return WKV_OK;
+
+    const size_t esz = io_size(io);
+    const size_t xbytes = (size_t)B * T * H * D * esz;
+    const size_t sbytes = (size_t)B * H * D * D * sizeof(float);
+    const size_t ubytes = (size_t)H * D * sizeof(float);
+    const bool tokens = T > 0;
+    Buf bufs[] = {{r, xbytes, tokens},        {k, xbytes, tokens},      {v, xbytes, tokens},
+                  {omega, xbytes, tokens},    {u, ubytes, tokens},      {y, xbytes, tokens},
+                  {state_in, sbytes, false},  {state_out, sbytes, false},
+                  {workspace, workspace_bytes, false}};
+    wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
+    if (s != WKV_OK) return s;
+    if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
+
+    // aliasing: state_out may equal state_in, nothing else may overlap an output
+    const Span sy = span(y, tokens ? xbytes : 0), sso = span(state_out, state_out ? sbytes : 0);
+    const Span ins[] = {span(r, tokens ? xbytes : 0), span(k, tokens ? xbytes : 0),
+                        span(v, tokens ? xbytes : 0), span(omega, tokens ? xbytes : 0),
+                        span(u, tokens ? ubytes : 0), span(state_in, state_in ? sbytes : 0),
+                        span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
+                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0)};
+    for (const Span& in : ins)
+        if (overlaps(sy, in)) return WKV_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(sso, ins[i])) return WKV_ERR_INVALID_ARG;
+    if (overlaps(sso, ins[6]) || overlaps(sso, ins[7]) || overlaps(sso, sy))
+        return WKV_ERR_INVALID_ARG;
+    if (state_in && state_out && state_in != state_out && overlaps(sso, ins[5]))
+        return WKV_ERR_INVALID_ARG;
+
+    const size_t need = wkv6_prefill_workspace_bytes(B, T, H, D, io, ln != nullptr, algo);
+    if (need > 0) {
+        if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+        const Span sw = span(workspace, need);
+        if (overlaps(sw, sy) || overlaps(sw, sso)) return WKV_ERR_INVALID_ARG;
+        for (const Span& in : ins)
+            if (overlaps(sw, in)) return WKV_ERR_INVALID_ARG;
+    }
+
+    if (injected("launch")) return WKV_ERR_CUDA;
+
+    if (!tokens) {  // empty sequence: the state passes through unchanged
+        if (state_out == nullptr || state_out == state_in) return WKV_OK;
+        if (state_in) return from_cuda(cudaMemcpyAsync(state_out, state_in, sbytes,
+                                                       cudaMemcpyDeviceToDevice, st));
+        return from_cuda(cudaMemsetAsync(state_out, 0, sbytes, st));
+    }
+
+    const bool bf16 = io == WKV_BF16;
+    float* y_raw = nullptr;
+    if (ln) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
+    cudaError_t e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw,
+                                              B, T, H, bf16, st);
+    if (e != cudaSuccess) return WKV_ERR_CUDA;
+    if (ln) {
+        e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y,
+                                           (long)B * T, H * D, bf16, st);
+        if (e != cudaSuccess) return WKV_ERR_CUDA;
+    }
+    return WKV_OK;
+}
+
+wkv_status wkv6_prefill(const void* r, const void* k, const void* v, const void* omega,
+                        const float* u, const float* state_in, float* state_out, void* y,
+                        int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    return wkv6_prefill_algo(r, k, v, omega, u, state_in, state_out, y, B, T, H, D, io, ln,
+                             WKV_ALGO_AUTO, workspace, workspace_bytes, stream);
+}
+
+wkv_status wkv6_decode_step(const void* r, const void* k, const void* v, const void* omega,
+                            const float* u, float* state, void* y, int B, int H, int D,
+                            wkv_dtype io, const wkv_ln* ln, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    if (B < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
+    if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return WKV_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t esz = io_size(io);
+    const size_t xbytes = (size_t)B * H * D * esz;
+    const size_t sbytes = (size_t)B * H * D * D * sizeof(float);
+    const size_t ubytes = (size_t)H * D * sizeof(float);
+    Buf bufs[] = {{r, xbytes, true}, {k, xbytes, true},     {v, xbytes, true},
+                  {omega, xbytes, true}, {u, ubytes, true}, {state, sbytes, true},
+                  {y, xbytes, true}, {workspace, workspace_bytes, false}};
+    wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
+    if (s != WKV_OK) return s;
+    if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
+
+    const Span sy = span(y, xbytes), ss = span(state, sbytes);
+    const Span ins[] = {span(r, xbytes), span(k, xbytes), span(v, xbytes), span(omega, xbytes),
+                        span(u, ubytes), span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
+                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0)};
+    if (overlaps(sy, ss)) return WKV_ERR_INVALID_ARG;
+    for (const Span& in : ins)
+        if (overlaps(sy, in) || overlaps(ss, in)) return WKV_ERR_INVALID_ARG;
+
+    const size_t need = wkv6_decode_workspace_bytes(B, H, D, io, ln != nullptr);
+    if (need > 0) {
+        if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+        const Span sw = span(workspace, need);
+        if (overlaps(sw, sy) || overlaps(sw, ss)) return WKV_ERR_INVALID_ARG;
+        for (const Span& in : ins)
+            if (overlaps(sw, in)) return WKV_ERR_INVALID_ARG;
+    }
+    if (injected("launch")) return WKV_ERR_CUDA;
+
+    const bool bf16 = io == WKV_BF16;
+    float* y_raw = nullptr;
+    if (ln) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
+    cudaError_t e = goldwkv::launch_decode(r, k, v, omega, u, state, y, y_raw, B, H, bf16, st);
+    if (e != cudaSuccess) return WKV_ERR_CUDA;
+    if (ln) {
+        e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y, (long)B,
+                                           H * D, bf16, st);
+        if (e != cudaSuccess) return WKV_ERR_CUDA;
+    }
+    return WKV_OK;
+}
+
+}  // extern "C"

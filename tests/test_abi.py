@@ -1,0 +1,69 @@
+"""The C-ABI library builds, loads and exports every entry point the headers declare.
+
+CPU only: no compute call is made (there is no GPU here); workspace queries and status
+strings are pure host functions.
+"""
+import ctypes
+import pathlib
+import re
+
+import pytest
+
+from linear_attention_rnn_finch_b200 import binding, build
+
+ROOT = pathlib.Path(__file__).resolve().parents[1]
+DECL = re.compile(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(wkv6_\w+)\s*\(", re.M)
+
+
+def declared_functions():
+    names = []
+    for h in sorted((ROOT / "include").glob("*.h")):
+        text = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
+        names += DECL.findall(text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ctypes.CDLL(str(binding.LIB_PATH))
+
+
+def test_headers_declare_entry_points():
+    names = declared_functions()
+    for must in ("wkv6_prefill", "wkv6_prefill_algo", "wkv6_decode_step",
+                 "wkv6_prefill_workspace_bytes", "wkv6_decode_workspace_bytes",
+                 "wkv6_status_string", "wkv6_abi_version"):
+        assert must in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_symbol_exported(lib, name):
+    assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings_and_version():
+    L = binding.load()
+    assert L.wkv6_abi_version() == 1
+    for s in range(6):
+        assert binding.status_string(s)
+    assert binding.status_string(0) == "ok"
+
+
+def test_workspace_queries():
+    import torch
+    # LayerNorm with bf16 output needs an fp32 staging buffer of y; nothing else does
+    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False) == 0
+    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.float32, True) == 0
+    assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True) == 2 * 10 * 3 * 64 * 4
+    assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, True) == 256 * 32 * 64 * 4
+    assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, False) == 0
+    # invalid sizes report zero
+    assert binding.prefill_workspace_bytes(2, 10, 3, 32, torch.bfloat16, True) == 0
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 2, 1, 64)
+    with pytest.raises(ValueError):
+        binding.wkv6_prefill(x, x, x, x, torch.zeros(1, 64))
