@@ -19,8 +19,9 @@
  * Conventions shared by every entry point
  *  - Pointers r, k, v, omega, u, state*, y, gamma, beta, workspace are DEVICE pointers on
  *    the current CUDA device; the caller owns every buffer.  The library never allocates
- *    device memory, never synchronises and keeps no global mutable state, so calls on
- *    different streams are independent.
+ *    device memory, keeps no global mutable state and, apart from wkv6_workspace_status,
+ *    never synchronises, so calls on different streams with different workspaces are
+ *    independent.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
  *    enqueued asynchronously; a device-side fault surfaces as a CUDA error at the caller's
  *    next synchronisation.
@@ -72,7 +73,9 @@ typedef struct wkv_ln {
 } wkv_ln;
 
 /* Bytes of device workspace wkv6_prefill needs for these sizes (0: none).  Depends only
- * on its arguments. */
+ * on its arguments.  Layout: the chunked path keeps a 4-byte device status word at offset
+ * 0 (256 bytes reserved); LayerNorm with bf16 output adds an fp32 [B][T][H][D] staging
+ * buffer after it. */
 size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
                                     wkv_algo algo);
 
@@ -90,7 +93,11 @@ size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, in
  *   state_in, or zeros), D == 64.
  *   ln              NULL, or LayerNorm parameters
  *   workspace       device scratch of at least wkv6_prefill_workspace_bytes(...) bytes
- *                   (may be NULL when that is 0); contents on entry are ignored.
+ *                   (may be NULL when that is 0).  On the chunked path its first 4 bytes
+ *                   are a status word that must be zero before the first call (zero-fill
+ *                   new workspace; see wkv6_workspace_status); other bytes are scratch.
+ *   Algorithm: WKV_ALGO_AUTO takes the chunked tensor-core kernel for bf16 I/O and the
+ *   fp32 recurrence for fp32 I/O.
  * Returns WKV_OK, or an error with nothing launched (INVALID_ARG, UNSUPPORTED, WORKSPACE)
  * or WKV_ERR_CUDA if a launch failed.
  */
@@ -106,6 +113,15 @@ wkv_status wkv6_prefill_algo(const void *r, const void *k, const void *v, const 
                              int B, int T, int H, int D, wkv_dtype io, const wkv_ln *ln,
                              wkv_algo algo, void *workspace, size_t workspace_bytes,
                              void *stream);
+
+/*
+ * Device status word of a workspace used by wkv6_prefill on the chunked path.  The chunked
+ * kernel bounds every wait on its own copies and tensor-core work; if one expires, the CTA
+ * drains its in-flight work, frees its tensor memory, returns early and sets this word.
+ * Synchronises `stream`, returns WKV_ERR_TIMEOUT (and clears the word) if it was set,
+ * WKV_OK otherwise.  The word must be zero before first use (zero-fill new workspace).
+ */
+wkv_status wkv6_workspace_status(void *workspace, void *stream);
 
 /* Bytes of device workspace wkv6_decode_step needs (non-zero only with LayerNorm). */
 size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln);

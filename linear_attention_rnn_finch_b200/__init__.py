@@ -4,8 +4,8 @@ The compute lives in ``libgoldwkv.so`` (see ``include/goldwkv.h``); ``binding`` 
 torch tensors into it.  Importing this package does not load the library; the first call
 does, and raises if it was not built.
 """
-from .binding import (WkvError, decode_workspace_bytes, load, prefill_workspace_bytes,
-                      wkv6_decode_step, wkv6_prefill)
+from .binding import (WkvError, decode_workspace_bytes, load, new_workspace,
+                      prefill_workspace_bytes, wkv6_decode_step, wkv6_prefill, workspace_status)
 
-__all__ = ["WkvError", "decode_workspace_bytes", "load", "prefill_workspace_bytes",
-           "wkv6_decode_step", "wkv6_prefill"]
+__all__ = ["WkvError", "decode_workspace_bytes", "load", "new_workspace",
+           "prefill_workspace_bytes", "wkv6_decode_step", "wkv6_prefill", "workspace_status"]

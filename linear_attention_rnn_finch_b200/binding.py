@@ -56,6 +56,8 @@ def load(path: Path | str | None = None):
     L.wkv6_prefill_algo.restype = i
     L.wkv6_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
     L.wkv6_decode_step.restype = i
+    L.wkv6_workspace_status.argtypes = [vp, vp]
+    L.wkv6_workspace_status.restype = i
     L.wkv6_status_string.argtypes = [i]
     L.wkv6_status_string.restype = ctypes.c_char_p
     L.wkv6_abi_version.argtypes = []
@@ -153,7 +155,7 @@ def wkv6_prefill(r, k, v, omega, u, state_in=None, *, ln=None, algo="auto", y=No
     ln_s, ln_p = _ln_struct(ln, H, D, dev)
     need = int(L.wkv6_prefill_workspace_bytes(B, T, H, D, _io(dt), int(ln is not None), ALGOS[algo]))
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = new_workspace(need, dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         st = L.wkv6_prefill_algo(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state_in),
@@ -162,6 +164,19 @@ def wkv6_prefill(r, k, v, omega, u, state_in=None, *, ln=None, algo="auto", y=No
     del ln_s
     _raise("wkv6_prefill", st)
     return y, state_out
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """Zero-filled device workspace (its leading status word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream and read (then clear) the workspace's device status word:
+    WKV_OK, or WKV_ERR_TIMEOUT if a bounded wait in the chunked kernel expired."""
+    dev = workspace.device
+    with torch.cuda.device(dev):
+        return int(load().wkv6_workspace_status(_ptr(workspace), _stream_ptr(dev, stream)))
 
 
 def wkv6_decode_step(r, k, v, omega, u, state, *, ln=None, y=None, workspace=None, stream=None):

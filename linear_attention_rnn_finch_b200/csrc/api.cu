@@ -11,6 +11,9 @@
 namespace {
 
 constexpr int kHeadSizeApi = 64;  // D: the only head size the kernels are built for
+constexpr size_t kStatusBytes = 256;  // device status word at the start of the workspace
+// Bounded waits inside the chunked kernel: SM cycles (about a second at 1.9 GHz).
+constexpr long long kSpinBudget = 2000000000LL;
 
 struct Span {
     uintptr_t lo, hi;  // [lo, hi)
@@ -83,6 +86,13 @@ wkv_status check_ln(const wkv_ln* ln, int H, int D, int dev_check) {
     return check_bufs(b, 2);
 }
 
+// Which kernel serves a prefill call.
+bool use_chunked(wkv_dtype io, wkv_algo algo) {
+    if (algo == WKV_ALGO_CHUNKED) return true;
+    if (algo == WKV_ALGO_RECURRENT) return false;
+    return io == WKV_BF16;
+}
+
 }  // namespace
 
 extern "C" {
@@ -103,10 +113,12 @@ const char* wkv6_status_string(wkv_status s) {
 
 size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
                                     wkv_algo algo) {
-    (void)algo;
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
-    if (with_ln && io == WKV_BF16) return (size_t)B * T * H * D * sizeof(float);
-    return 0;
+    const bool chunked = use_chunked(io, algo);
+    size_t bytes = chunked ? kStatusBytes : 0;
+    // LayerNorm with bf16 output stages the fp32 rows; with fp32 output y itself does
+    if (with_ln && io == WKV_BF16) bytes += (size_t)B * T * H * D * sizeof(float);
+    return bytes;
 }
 
 size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln) {
@@ -176,10 +188,20 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
     }
 
     const bool bf16 = io == WKV_BF16;
+    const bool chunked = use_chunked(io, algo);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
-    if (ln) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
-    cudaError_t e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw,
-                                              B, T, H, bf16, st);
+    if (ln) y_raw = bf16 ? reinterpret_cast<float*>(ws + (chunked ? kStatusBytes : 0))
+                         : static_cast<float*>(y);
+    cudaError_t e;
+    if (chunked) {
+        const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+        e = goldwkv::launch_chunked(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T, H,
+                                    reinterpret_cast<int*>(ws), budget, st);
+    } else {
+        e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,
+                                      H, bf16, st);
+    }
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     if (ln) {
         e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y,
@@ -187,6 +209,21 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
         if (e != cudaSuccess) return WKV_ERR_CUDA;
     }
     return WKV_OK;
+}
+
+wkv_status wkv6_workspace_status(void* workspace, void* stream) {
+    if (workspace == nullptr || !aligned16(workspace)) return WKV_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    if (word == 0) return WKV_OK;
+    const int zero = 0;
+    if (cudaMemcpyAsync(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    return WKV_ERR_TIMEOUT;
 }
 
 wkv_status wkv6_prefill(const void* r, const void* k, const void* v, const void* omega,

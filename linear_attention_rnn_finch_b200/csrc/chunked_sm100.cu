@@ -1,0 +1,571 @@
+// Chunked WKV6 prefill on sm_100a: TMA-fed tcgen05 tensor-core contractions.
+//
+// What is computed (GoldFinch review page, section 3.4, "Recurrent state update and
+// output" and "Data-dependent decay"): per (b,h) with D = 64,
+//     y_t = r_t . (diag(u) k_t^T v_t + S_{t-1}),   S_t = diag(w_t) S_{t-1} + k_t^T v_t,
+//     w_t = exp(-exp(omega_t)).
+// The page's pre-fill runs the recurrence "in parallel chunks" (section 3.4, "Training and
+// Inference Procedures"); this kernel is that chunked form.  For a chunk of C = 64 tokens
+// with incoming state S (rows i: key/decay channels, columns j: value channels):
+//
+//   y_t   = Rt_t . S  +  sum_{s<t} A[t][s] v_s  +  A[t][t] v_t
+//   S_out = diag(gamma) S + Kt^T V
+// with  Rt_t = r_t * prod_{tau<t} w_tau,  Kt_s = k_s * prod_{tau>s} w_tau,
+//       gamma = prod_{tau<C} w_tau,  A[t][t] = sum_i r_t[i] u[i] k_t[i]  (the bonus),
+//       A[t][s] = sum_i r_t[i] k_s[i] prod_{s<tau<t} w_tau[i]   (s < t).
+//
+// Overflow-free decay factorisation of A.  Every decay factor is a product of w's over a
+// range, i.e. <= 1.  Split the pairs (t, s), s < t, by the highest bit in which t and s
+// differ, l in 0..5: both lie in one 2^(l+1)-aligned block, t in its upper 2^l half and s
+// in the lower half, so
+//     prod_{s<tau<t} w = [prod of w from the start of t's 2^l block to t-1]
+//                      * [prod of w from s+1 to the end of s's 2^l block].
+// With Q^l_t = r_t * (first bracket) and K^l_s = k_s * (second bracket) -- both <= |r|, |k|
+// -- the pairs of level l are entries of the product Q^l (K^l)^T.  Level 0 needs no decay
+// at all (Q^0 = r, K^0 = k: the raw TMA tiles).  Each level is one 64x64x64 tcgen05 MMA
+// into its own TMEM accumulator; A is assembled by picking, for every (t, s), the entry of
+// its level.  No exponential of a positive number is ever formed, so nothing overflows
+// for any decay, and no clamp is needed.
+//
+// Precision: operands are bf16 with fp32 accumulation.  S and A, whose rounding would sit
+// directly on y, are split into bf16 hi + lo parts (two MMAs each); the fp32 state chain
+// S <- gamma*S + U stays in registers across chunks.
+//
+// Schedule (one CTA per (b,h), 256 threads, chunks in order, all warps in lockstep):
+//   TMA loads of r, k, v, omega run two chunks ahead (2-stage ring, mbarrier tx-count);
+//   prep    : warp = 8 channels, lane = 2 tokens; w, block products (shuffle butterfly),
+//             operands Q^1..5, K^1..5, Rt, Kt^T written to 128B-swizzled smem;
+//   MMA 1   : L^0..L^5, U = Kt^T V, Y = Rt S_hi + Rt S_lo (thread 0 issues, commit);
+//   state   : S <- gamma S + U in registers; S_hi/S_lo for the next chunk;
+//   assemble: A from the level accumulators, hi/lo to smem;
+//   MMA 2   : Y += A_hi V + A_lo V;
+//   epilogue: Y -> bf16 -> smem -> TMA store (double-buffered).
+// An M=64 accumulator occupies TMEM lanes 16q..16q+15 of sub-partition q, so warp w reads
+// rows 16(w%4)..+15 with its lanes 0..15, columns split between warps w and w+4.
+//
+// Every mbarrier wait is bounded (spin budget in SM cycles); on expiry the CTA records
+// an error word, drains its in-flight copies and MMAs with a second bounded wait, frees
+// its TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace goldwkv {
+
+namespace {
+
+constexpr int C = 64;                 // tokens per chunk
+constexpr int kThreads = 256;
+constexpr int kStages = 2;
+constexpr int kTile = 64 * 64 * 2;    // one 64 x 64 bf16 tile, bytes
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t COL_L0 = 0;        // level accumulators at 64*l
+constexpr uint32_t COL_U = 384;
+constexpr uint32_t COL_Y = 448;
+constexpr uint32_t IDESC_KK = ptx::idesc_bf16(64, 64, 0, 0);
+constexpr uint32_t IDESC_KM = ptx::idesc_bf16(64, 64, 0, 1);
+
+struct __align__(1024) Smem {
+    uint8_t in[kStages][4][kTile];   // r, k, v, omega tiles per stage (TMA, 128B swizzle)
+    uint8_t q[5][kTile];             // Q^1..Q^5; q[0], q[1] are reused for A_hi, A_lo
+    uint8_t kk[5][kTile];            // K^1..K^5
+    uint8_t rt[kTile];               // Rt  [t][i]
+    uint8_t ktT[kTile];              // Kt^T [i][s]
+    uint8_t s_hi[kTile];             // S as bf16 [i][j], high part
+    uint8_t s_lo[kTile];             // low part
+    uint8_t ystage[2][kTile];        // y tiles for the TMA store
+    float u[64];
+    float gamma[64];
+    float bonus_part[8][64];         // per channel group partial of sum_i r u k
+    uint64_t full[kStages];
+    uint64_t mma1, mma2;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// byte offset of element (row, col) in a 64 x 64 bf16 tile with 128-byte rows, swizzled
+__device__ __forceinline__ uint32_t sw_chunk(int row, int chunk) {
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
+// hi = bf16(x), lo = bf16(x - hi): x ~= hi + lo to about 16 significant bits
+__device__ __forceinline__ void split8(const float (&f)[8], uint4& hi, uint4& lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = __bfloat162float(__float2bfloat16_rn(f[i]));
+        l[i] = f[i] - h[i];
+    }
+    hi = pack8(h);
+    lo = pack8(l);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4*>(base + off) = v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
+                    const float* s_in, float* s_out, float* __restrict__ y_raw, int T, int H,
+                    int* status, long long spin_budget, long long drain_budget) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                       ~uintptr_t(1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x, b = bh / H, h = bh - (bh / H) * H;
+    const int NC = (T + C - 1) / C;
+
+    // ------------------------------------------------------------ set-up
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) ptx::mbar_init(&s.full[i], 1);
+        ptx::mbar_init(&s.mma1, 1);
+        ptx::mbar_init(&s.mma2, 1);
+        ptx::fence_mbar_init();
+        s.abort = 0;
+        ptx::prefetch_tensormap(&tm_r);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_w);
+        ptx::prefetch_tensormap(&tm_y);
+    }
+    if (tid < 64) s.u[tid] = u[h * 64 + tid];
+    if (warp == 0) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
+    // zero the operand tiles once, so that rows an MMA reads but never uses hold finite data
+    for (int i = tid; i < (int)(sizeof(s.q) + sizeof(s.kk)) / 16; i += kThreads)
+        reinterpret_cast<uint4*>(s.q)[i] = make_uint4(0, 0, 0, 0);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+
+    auto issue_load = [&](int chunk) {
+        const int st = chunk % kStages;
+        ptx::mbar_arrive_expect_tx(&s.full[st], 4 * kTile);
+        const int t0 = chunk * C;
+        ptx::tma_load_4d(s.in[st][0], &tm_r, &s.full[st], 0, h, t0, b);
+        ptx::tma_load_4d(s.in[st][1], &tm_k, &s.full[st], 0, h, t0, b);
+        ptx::tma_load_4d(s.in[st][2], &tm_v, &s.full[st], 0, h, t0, b);
+        ptx::tma_load_4d(s.in[st][3], &tm_w, &s.full[st], 0, h, t0, b);
+    };
+    if (tid == 0)
+        for (int c = 0; c < kStages && c < NC; ++c) issue_load(c);
+
+    // ------------------------------------------------------------ state in registers
+    // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in lanes 0..15), column half hh
+    const int q = warp & 3, hh = warp >> 2;
+    const bool row_lane = lane < 16;
+    const int row = 16 * q + (lane & 15);          // state row i / token row t of this lane
+    const uint32_t tlane = (uint32_t)(32 * q) << 16;
+    float S[32];
+    {
+        const float* src = s_in ? s_in + (size_t)bh * 4096 + row * 64 + 32 * hh : nullptr;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (src && row_lane) x = *reinterpret_cast<const float4*>(src + j);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        if (row_lane) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                uint4 hi, lo;
+                split8(f, hi, lo);
+                st_shared_v4(s.s_hi, sw_chunk(row, 4 * hh + cc), hi);
+                st_shared_v4(s.s_lo, sw_chunk(row, 4 * hh + cc), lo);
+            }
+        }
+    }
+
+    bool failed = false;
+    int n = 0;
+    int issued1 = -1, issued2 = -1;   // last chunk whose MMA group 1 / 2 thread 0 issued
+    for (; n < NC; ++n) {
+        const int st = n % kStages;
+        const int t0 = n * C;
+        const int valid = min(C, T - t0);
+        uint8_t* r_tile = s.in[st][0];
+        uint8_t* k_tile = s.in[st][1];
+        uint8_t* v_tile = s.in[st][2];
+        uint8_t* w_tile = s.in[st][3];
+        uint8_t* y_tile = s.ystage[n & 1];
+        if (tid == 0) ptx::bulk_wait_read<1>();    // the store that last used y_tile has read it
+
+        if (!ptx::mbar_wait(&s.full[st], (uint32_t)((n / kStages) & 1), spin_budget)) s.abort = 1;
+
+        // -------------------------------------------------------- prep
+        {
+            const int cg = warp;                      // channels 8cg .. 8cg+7
+            const int ta = 2 * lane, tb = ta + 1;     // tokens of this lane
+            float rv[2][8], kv[2][8], wv[2][8];
+            {
+                float om[2][8];
+                unpack8(*reinterpret_cast<const uint4*>(r_tile + sw_chunk(ta, cg)), rv[0]);
+                unpack8(*reinterpret_cast<const uint4*>(r_tile + sw_chunk(tb, cg)), rv[1]);
+                unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(ta, cg)), kv[0]);
+                unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(tb, cg)), kv[1]);
+                unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(ta, cg)), om[0]);
+                unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(tb, cg)), om[1]);
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        wv[p][c] = (ta + p < valid) ? __expf(-__expf(om[p][c])) : 1.f;
+            }
+            // bonus partials: sum over this lane's 8 channels of r u k
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float acc = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc = fmaf(rv[p][c] * s.u[8 * cg + c], kv[p][c], acc);
+                s.bonus_part[cg][ta + p] = acc;
+            }
+            // level 1: blocks of 2 tokens, both in this lane
+            float E[2][8], F[2][8], BP[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                E[0][c] = 1.f;
+                E[1][c] = wv[0][c];
+                F[0][c] = wv[1][c];
+                F[1][c] = 1.f;
+                BP[c] = wv[0][c] * wv[1][c];
+            }
+            auto write_level = [&](uint8_t* qtile, uint8_t* ktile, bool upper) {
+                // rows of t's upper half use Q^l = r * E, rows of the lower half K^l = k * F
+                float f[8];
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) f[c] = upper ? rv[p][c] * E[p][c] : kv[p][c] * F[p][c];
+                    st_shared_v4(upper ? qtile : ktile, sw_chunk(ta + p, cg), pack8(f));
+                }
+            };
+            write_level(s.q[0], s.kk[0], (lane & 1) != 0);
+#pragma unroll
+            for (int l = 2; l <= 6; ++l) {
+                const int sh = 1 << (l - 2);
+                const bool upper = (lane & sh) != 0;  // t in the upper 2^(l-1) half of its block
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float sib = __shfl_xor_sync(0xffffffffu, BP[c], sh);
+                    const float mE = upper ? sib : 1.f;
+                    const float mF = upper ? 1.f : sib;
+                    E[0][c] *= mE;
+                    E[1][c] *= mE;
+                    F[0][c] *= mF;
+                    F[1][c] *= mF;
+                    BP[c] *= sib;
+                }
+                if (l <= 5) write_level(s.q[l - 1], s.kk[l - 1], (lane & (1 << (l - 1))) != 0);
+            }
+            // level 6 = the whole chunk: Rt = r * E6 (all rows), Kt^T = (k * F6)^T, gamma
+            {
+                float f[8];
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) f[c] = rv[p][c] * E[p][c];
+                    st_shared_v4(s.rt, sw_chunk(ta + p, cg), pack8(f));
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int i = 8 * cg + c;
+                    const uint32_t off = (uint32_t)(i * 128 + ((((lane >> 2)) ^ (i & 7)) << 4) + (lane & 3) * 4);
+                    *reinterpret_cast<uint32_t*>(s.ktT + off) = pack2(kv[0][c] * F[0][c], kv[1][c] * F[1][c]);
+                }
+                if (lane == 0)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) s.gamma[8 * cg + c] = BP[c];
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+        if (s.abort) { failed = true; break; }
+
+        // -------------------------------------------------------- MMA 1
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            const uint32_t a_r = ptx::smem_addr(r_tile), b_k = ptx::smem_addr(k_tile);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_L0, ptx::desc_kmajor(a_r + 32 * kq),
+                              ptx::desc_kmajor(b_k + 32 * kq), IDESC_KK, kq > 0);
+#pragma unroll
+            for (int l = 1; l <= 5; ++l) {
+                const uint32_t a = ptx::smem_addr(s.q[l - 1]), bb = ptx::smem_addr(s.kk[l - 1]);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)
+                    ptx::mma_bf16(tmem + 64 * l, ptx::desc_kmajor(a + 32 * kq),
+                                  ptx::desc_kmajor(bb + 32 * kq), IDESC_KK, kq > 0);
+            }
+            const uint32_t a_kt = ptx::smem_addr(s.ktT), b_v = ptx::smem_addr(v_tile);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kt + 32 * kq),
+                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, kq > 0);
+            const uint32_t a_rt = ptx::smem_addr(s.rt);
+            const uint32_t b_hi = ptx::smem_addr(s.s_hi), b_lo = ptx::smem_addr(s.s_lo);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(a_rt + 32 * kq),
+                              ptx::desc_mnmajor(b_hi + 2048 * kq), IDESC_KM, kq > 0);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(a_rt + 32 * kq),
+                              ptx::desc_mnmajor(b_lo + 2048 * kq), IDESC_KM, 1);
+            ptx::mma_commit(&s.mma1);
+            issued1 = n;
+        }
+        if (!ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), spin_budget)) s.abort = 1;
+        ptx::tc_fence_after();
+
+        // -------------------------------------------------------- state chain
+        {
+            uint32_t U[32];
+            ptx::tmem_ld32(tmem + tlane + COL_U + 32 * hh, U);
+            ptx::tmem_wait_ld();
+            if (row_lane) {
+                const float g = s.gamma[row];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                    uint4 hi, lo;
+                    split8(f, hi, lo);
+                    st_shared_v4(s.s_hi, sw_chunk(row, 4 * hh + cc), hi);
+                    st_shared_v4(s.s_lo, sw_chunk(row, 4 * hh + cc), lo);
+                }
+            }
+        }
+
+        // -------------------------------------------------------- assemble A
+        {
+            const int t = row;               // token row (lanes 0..15)
+            const int p = t & 7;
+            const bool upper8 = (lane & 15) >= 8;  // t in block 2q+1 (else 2q)
+            float bonus = 0.f;
+            if (row_lane) {
+#pragma unroll
+                for (int g = 0; g < 8; ++g) bonus += s.bonus_part[g][t];
+            }
+#pragma unroll
+            for (int gg = 0; gg < 4; ++gg) {
+                const int g = 4 * hh + gg;   // key block of 8 columns
+                float a[8];
+                if (g < 2 * q) {
+                    const int lvl = 3 + (31 - __clz((2 * q) ^ g));
+                    uint32_t v[8];
+                    ptx::tmem_ld8(tmem + tlane + 64 * lvl + 8 * g, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) a[c] = __uint_as_float(v[c]);
+                } else if (g <= 2 * q + 1) {
+                    uint32_t v0[8], v1[8], v2[8], v3[8];
+                    ptx::tmem_ld8(tmem + tlane + 0 + 8 * g, v0);
+                    ptx::tmem_ld8(tmem + tlane + 64 + 8 * g, v1);
+                    ptx::tmem_ld8(tmem + tlane + 128 + 8 * g, v2);
+                    ptx::tmem_ld8(tmem + tlane + 192 + 8 * g, v3);
+                    ptx::tmem_wait_ld();
+                    const bool diag = (g == 2 * q) ? !upper8 : upper8;  // s in t's own 8-block
+                    const bool below = (g == 2 * q) && upper8;           // whole block before t
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float x = 0.f;
+                        if (below) {
+                            x = __uint_as_float(v3[c]);
+                        } else if (diag) {
+                            if (c == p) {
+                                x = bonus;
+                            } else if (c < p) {
+                                const int lvl = 31 - __clz(p ^ c);
+                                x = __uint_as_float(lvl == 0 ? v0[c] : (lvl == 1 ? v1[c] : v2[c]));
+                            }
+                        }
+                        a[c] = x;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) a[c] = 0.f;
+                }
+                if (row_lane) {
+                    uint4 hi, lo;
+                    split8(a, hi, lo);
+                    st_shared_v4(s.q[0], sw_chunk(t, g), hi);
+                    st_shared_v4(s.q[1], sw_chunk(t, g), lo);
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+        if (s.abort) { failed = true; break; }
+
+        // -------------------------------------------------------- MMA 2: Y += A V
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            const uint32_t a_hi = ptx::smem_addr(s.q[0]), a_lo = ptx::smem_addr(s.q[1]);
+            const uint32_t b_v = ptx::smem_addr(v_tile);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(a_hi + 32 * kq),
+                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, 1);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(a_lo + 32 * kq),
+                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, 1);
+            ptx::mma_commit(&s.mma2);
+            issued2 = n;
+        }
+        if (!ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), spin_budget)) s.abort = 1;
+        ptx::tc_fence_after();
+
+        // -------------------------------------------------------- epilogue
+        {
+            uint32_t Y[32];
+            ptx::tmem_ld32(tmem + tlane + COL_Y + 32 * hh, Y);
+            ptx::tmem_wait_ld();
+            if (row_lane && y_raw != nullptr) {
+                // fp32 rows for the LayerNorm pass: 128 contiguous bytes per lane
+                if (row < valid) {
+                    float* dst = y_raw + (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(dst + j) =
+                            make_float4(__uint_as_float(Y[j]), __uint_as_float(Y[j + 1]),
+                                        __uint_as_float(Y[j + 2]), __uint_as_float(Y[j + 3]));
+                }
+            } else if (row_lane) {
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(Y[8 * cc + e]);
+                    st_shared_v4(y_tile, sw_chunk(row, 4 * hh + cc), pack8(f));
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+        if (s.abort) { failed = true; break; }
+        if (tid == 0) {
+            if (y_raw == nullptr) {
+                ptx::tma_store_4d(&tm_y, y_tile, 0, h, t0, b);
+                ptx::bulk_commit();
+            }
+            // every thread is past its reads of this stage and the MMAs that read it are done
+            if (n + kStages < NC) {
+                ptx::fence_proxy_async_smem();
+                issue_load(n + kStages);
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ finish / drain
+    if (failed) {
+        if (tid == 0) {
+            atomicExch(status, 1);
+            // copies still in flight: chunks n .. min(NC, n + kStages) - 1 may have been issued
+            for (int c = n; c < NC && c < n + kStages; ++c)
+                ptx::mbar_wait(&s.full[c % kStages], (uint32_t)((c / kStages) & 1), drain_budget);
+            if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), drain_budget);
+            if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), drain_budget);
+        }
+    } else if (s_out != nullptr && row_lane) {
+        float* dst = s_out + (size_t)bh * 4096 + row * 64 + 32 * hh;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+    if (tid == 0) ptx::bulk_wait<0>();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+    static EncodeTiled fn = []() -> EncodeTiled {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiled>(p);
+    }();
+    return fn;
+}
+
+// [B][T][H][64] bf16 viewed as 4-D (D, H, T, B); box = 64 channels x 1 head x 64 tokens.
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {64, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {64 * 2, (cuuint64_t)H * 64 * 2, (cuuint64_t)T * H * 64 * 2};
+    const cuuint32_t box[4] = {64, 1, C, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t chunked_smem_bytes() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_chunked(const void* r, const void* k, const void* v, const void* omega,
+                           const float* u, const float* s_in, float* s_out, void* y,
+                           float* y_raw, int B, int T, int H, int* status, long long spin_budget,
+                           cudaStream_t st) {
+    CUtensorMap mr, mk, mv, mw, my;
+    if (!make_map(&mr, r, B, T, H) || !make_map(&mk, k, B, T, H) || !make_map(&mv, v, B, T, H) ||
+        !make_map(&mw, omega, B, T, H) || !make_map(&my, y, B, T, H))
+        return cudaErrorInvalidValue;
+    const size_t smem = chunked_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long drain = 4000000000LL;
+    wkv6_chunked_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
+        mr, mk, mv, mw, my, u, s_in, s_out, y_raw, T, H, status, spin_budget, drain);
+    return cudaGetLastError();
+}
+
+}  // namespace goldwkv

@@ -22,4 +22,13 @@ cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const floa
                                   float eps, void* out, long rows, int C, bool bf16,
                                   cudaStream_t st);
 
+// Chunked tensor-core prefill (bf16 I/O).  y_raw != nullptr: fp32 y rows go there (for a
+// LayerNorm pass) instead of bf16 y.  status: device word set to 1 if a bounded wait
+// expired.  spin_budget: SM cycles each wait may spin.
+cudaError_t launch_chunked(const void* r, const void* k, const void* v, const void* omega,
+                           const float* u, const float* s_in, float* s_out, void* y,
+                           float* y_raw, int B, int T, int H, int* status, long long spin_budget,
+                           cudaStream_t st);
+size_t chunked_smem_bytes();
+
 }  // namespace goldwkv

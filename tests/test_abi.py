@@ -33,7 +33,7 @@ def test_headers_declare_entry_points():
     names = declared_functions()
     for must in ("wkv6_prefill", "wkv6_prefill_algo", "wkv6_decode_step",
                  "wkv6_prefill_workspace_bytes", "wkv6_decode_workspace_bytes",
-                 "wkv6_status_string", "wkv6_abi_version"):
+                 "wkv6_status_string", "wkv6_abi_version", "wkv6_workspace_status"):
         assert must in names
 
 
@@ -52,10 +52,13 @@ def test_status_strings_and_version():
 
 def test_workspace_queries():
     import torch
-    # LayerNorm with bf16 output needs an fp32 staging buffer of y; nothing else does
-    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False) == 0
+    # the chunked path keeps a 256-byte status block; LayerNorm with bf16 output adds an
+    # fp32 staging buffer of y; the fp32 recurrence needs nothing
+    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False) == 256
+    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False, "recurrent") == 0
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.float32, True) == 0
-    assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True) == 2 * 10 * 3 * 64 * 4
+    assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True) == 256 + 2 * 10 * 3 * 64 * 4
+    assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True, "recurrent") == 2 * 10 * 3 * 64 * 4
     assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, True) == 256 * 32 * 64 * 4
     assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, False) == 0
     # invalid sizes report zero

@@ -46,8 +46,14 @@ def untouched(d):
 
 
 def test_valid_call_ok(bufs):
-    assert call(bufs) == bd.WKV_OK
+    ws = bd.new_workspace(bd.prefill_workspace_bytes(B, T, H, D, torch.bfloat16, False), "cuda")
+    assert call(bufs, ws=vp(ws), ws_bytes=ws.numel()) == bd.WKV_OK
     assert not untouched(bufs)
+
+
+def test_chunked_needs_workspace(bufs):
+    assert call(bufs) == bd.WKV_ERR_WORKSPACE and untouched(bufs)
+    assert call(bufs, algo=1) == bd.WKV_OK   # the recurrence needs none
 
 
 def test_head_size_unsupported(bufs):
@@ -90,9 +96,9 @@ def test_layernorm_needs_workspace(bufs):
     ln = bd._LN(bufs["gamma"].data_ptr(), bufs["beta"].data_ptr(), 1e-5)
     assert call(bufs, ln=ctypes.byref(ln)) == bd.WKV_ERR_WORKSPACE and untouched(bufs)
     need = bd.prefill_workspace_bytes(B, T, H, D, torch.bfloat16, True)
-    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    ws = bd.new_workspace(need - 16, "cuda")
     assert call(bufs, ln=ctypes.byref(ln), ws=vp(ws), ws_bytes=need - 16) == bd.WKV_ERR_WORKSPACE
-    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ws = bd.new_workspace(need, "cuda")
     assert call(bufs, ln=ctypes.byref(ln), ws=vp(ws), ws_bytes=need) == bd.WKV_OK
 
 
@@ -129,3 +135,23 @@ def test_decode_validation(bufs):
     assert st == bd.WKV_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert torch.equal(state, bufs["s_in"]) and bool((y == 5.0).all())
+
+
+def test_chunked_wait_timeout_is_reported_and_context_survives(oracle, monkeypatch):
+    """A zero spin budget makes the chunked kernel's first bounded wait expire: every CTA
+    drains its in-flight copies, frees its tensor memory and returns; the workspace status
+    word reports the timeout and the next call on the same context is correct."""
+    from linear_attention_rnn_finch_b200 import workloads as W
+    from tests.parity import TOL, f64, rel_err
+    cfg = W.CONFIGS[1].with_(seed=9100)
+    inp = W.make_prefill_inputs(cfg, "cuda", B=2, T=200)
+    args = [inp[n] for n in ("r", "k", "v", "omega")]
+    ws = bd.new_workspace(bd.prefill_workspace_bytes(2, 200, cfg.H, 64, torch.bfloat16, False), "cuda")
+    monkeypatch.setenv("GOLDWKV_FAULT", "timeout0")
+    bd.wkv6_prefill(*args, inp["u"], inp["state0"], algo="chunked", workspace=ws)
+    assert bd.workspace_status(ws) == bd.WKV_ERR_TIMEOUT
+    monkeypatch.delenv("GOLDWKV_FAULT")
+    y, s = bd.wkv6_prefill(*args, inp["u"], inp["state0"], algo="chunked", workspace=ws)
+    assert bd.workspace_status(ws) == bd.WKV_OK
+    yo, so = oracle.prefill(*[f64(a) for a in args], f64(inp["u"]), f64(inp["state0"]))
+    assert rel_err(y, yo) <= TOL[torch.bfloat16] and rel_err(s, so) <= TOL[torch.bfloat16]

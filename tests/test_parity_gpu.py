@@ -16,7 +16,7 @@ from tests.parity import TOL, f64, oracle_heads, rel_err
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-BF16_ALGOS = ["auto", "recurrent"]
+BF16_ALGOS = ["chunked", "recurrent"]
 
 
 def _run(inp, algo="auto", T=None, ln=False, state=True):
