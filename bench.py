@@ -217,9 +217,10 @@ def run_ours(args, world, rank, local):
 
     binding.load()
     dev = torch.device("cuda", local)
-    cfg = PREFILL_CFG
+    cfg = PREFILL_CFG if args.batch is None else PREFILL_CFG.with_(B=args.batch)
     B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
     inp = W.make_prefill_inputs(cfg, dev, seed=cfg.seed + 17 * rank)
+    ws = gw.new_workspace(gw.prefill_workspace_bytes(B, T, H, D, cfg.dtype, False, args.algo), dev)
     y = torch.empty_like(inp["r"])
     s_out = torch.empty_like(inp["state0"])
     stream = torch.cuda.current_stream(dev)
@@ -227,7 +228,8 @@ def run_ours(args, world, rank, local):
     algo = args.algo
 
     def step():
-        gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], y=y, state_out=s_out, algo=algo)
+        gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], y=y, state_out=s_out, algo=algo,
+                        workspace=ws)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -235,7 +237,7 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    t_end = time.time() + 1.0
+    t_end = time.time() + (0.0 if args.no_clock_warm else 1.0)
     while time.time() < t_end:
         for _ in range(20):
             step()
@@ -271,7 +273,8 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "wkv6_prefill_1p5b_layer", "B": B, "T": T, "H": H, "D": D,
+        "config": {"workload": "wkv6_prefill_1p5b_layer" + ("" if args.batch is None else f"_B{B}"),
+                   "B": B, "T": T, "H": H, "D": D,
                    "io": "bf16", "state": "fp32", "algo": algo,
                    "parallelism": f"dp{world} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (537 MB in, 134 MB out per step)"},
@@ -332,7 +335,7 @@ def run_ours(args, world, rank, local):
             for n in host:
                 dbuf[n].copy_(host[n], non_blocking=True)
             gw.wkv6_prefill(dbuf["r"], dbuf["k"], dbuf["v"], dbuf["omega"], dbuf["u"],
-                            dbuf["state0"], y=y, state_out=s_out, algo=algo)
+                            dbuf["state0"], y=y, state_out=s_out, algo=algo, workspace=ws)
             y_h.copy_(y, non_blocking=True)
             s_h.copy_(s_out, non_blocking=True)
 
@@ -416,6 +419,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clock-warm", action="store_true",
+                    help="skip the ~1 s untimed warm-up loop (for profiler runs)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the prefill batch size (smaller profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

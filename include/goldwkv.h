@@ -62,7 +62,10 @@ typedef enum wkv_dtype {
 typedef enum wkv_algo {
     WKV_ALGO_AUTO = 0,         /* library picks (chunked tensor-core path where it applies) */
     WKV_ALGO_RECURRENT = 1,    /* token-by-token fp32 recurrence on CUDA cores             */
-    WKV_ALGO_CHUNKED = 2       /* chunked prefill on tcgen05 tensor cores (bf16 I/O only)  */
+    WKV_ALGO_CHUNKED = 2,      /* chunked prefill on tcgen05 tensor cores (bf16 I/O only)  */
+    WKV_ALGO_CHUNKED_LEVELS = 3 /* chunked, every chunk through the level factorisation that
+                                   takes any decay (the path WKV_ALGO_CHUNKED falls back to
+                                   per sequence); bf16 I/O only, slower, for testing      */
 } wkv_algo;
 
 /* LayerNorm over the H*D concatenated head outputs of each token. */
@@ -73,9 +76,10 @@ typedef struct wkv_ln {
 } wkv_ln;
 
 /* Bytes of device workspace wkv6_prefill needs for these sizes (0: none).  Depends only
- * on its arguments.  Layout: the chunked path keeps a 4-byte device status word at offset
- * 0 (256 bytes reserved); LayerNorm with bf16 output adds an fp32 [B][T][H][D] staging
- * buffer after it. */
+ * on its arguments.  Layout on the chunked path: a 4-byte device status word at offset 0
+ * (256 bytes reserved), then per (b,h) a hand-off record (chunk index, and a D x D fp32
+ * state) used when a sequence moves from the fast to the level-factorised kernel;
+ * LayerNorm with bf16 output adds an fp32 [B][T][H][D] staging buffer at the end. */
 size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
                                     wkv_algo algo);
 

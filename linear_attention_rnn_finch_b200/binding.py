@@ -18,7 +18,7 @@ LIB_PATH = _PKG / "libgoldwkv.so"
 
 WKV_OK, WKV_ERR_INVALID_ARG, WKV_ERR_UNSUPPORTED, WKV_ERR_CUDA, WKV_ERR_TIMEOUT, WKV_ERR_WORKSPACE = range(6)
 WKV_F32, WKV_BF16 = 0, 1
-ALGOS = {"auto": 0, "recurrent": 1, "chunked": 2}
+ALGOS = {"auto": 0, "recurrent": 1, "chunked": 2, "chunked_levels": 3}
 HEAD_SIZE = 64
 
 _lib = None

@@ -88,10 +88,16 @@ wkv_status check_ln(const wkv_ln* ln, int H, int D, int dev_check) {
 
 // Which kernel serves a prefill call.
 bool use_chunked(wkv_dtype io, wkv_algo algo) {
-    if (algo == WKV_ALGO_CHUNKED) return true;
+    if (algo == WKV_ALGO_CHUNKED || algo == WKV_ALGO_CHUNKED_LEVELS) return true;
     if (algo == WKV_ALGO_RECURRENT) return false;
     return io == WKV_BF16;
 }
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// chunked-path workspace: status | hand-off chunk per (b,h) | hand-off state per (b,h)
+size_t handoff_ints_bytes(int B, int H) { return round256((size_t)B * H * sizeof(int)); }
+size_t handoff_state_bytes(int B, int H) { return (size_t)B * H * 64 * 64 * sizeof(float); }
 
 }  // namespace
 
@@ -115,7 +121,7 @@ size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, in
                                     wkv_algo algo) {
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
     const bool chunked = use_chunked(io, algo);
-    size_t bytes = chunked ? kStatusBytes : 0;
+    size_t bytes = chunked ? kStatusBytes + handoff_ints_bytes(B, H) + handoff_state_bytes(B, H) : 0;
     // LayerNorm with bf16 output stages the fp32 rows; with fp32 output y itself does
     if (with_ln && io == WKV_BF16) bytes += (size_t)B * T * H * D * sizeof(float);
     return bytes;
@@ -133,10 +139,12 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
                              wkv_algo algo, void* workspace, size_t workspace_bytes,
                              void* stream) {
     if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
-    if (algo != WKV_ALGO_AUTO && algo != WKV_ALGO_RECURRENT && algo != WKV_ALGO_CHUNKED)
+    if (algo != WKV_ALGO_AUTO && algo != WKV_ALGO_RECURRENT && algo != WKV_ALGO_CHUNKED &&
+        algo != WKV_ALGO_CHUNKED_LEVELS)
         return WKV_ERR_INVALID_ARG;
     if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
-    if (algo == WKV_ALGO_CHUNKED && io != WKV_BF16) return WKV_ERR_UNSUPPORTED;
+    if ((algo == WKV_ALGO_CHUNKED || algo == WKV_ALGO_CHUNKED_LEVELS) && io != WKV_BF16)
+        return WKV_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (B == 0 || H == 0) return WKV_OK;
 
@@ -191,13 +199,33 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
     const bool chunked = use_chunked(io, algo);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
-    if (ln) y_raw = bf16 ? reinterpret_cast<float*>(ws + (chunked ? kStatusBytes : 0))
-                         : static_cast<float*>(y);
+    const size_t hand_i = chunked ? kStatusBytes : 0;
+    const size_t hand_s = hand_i + (chunked ? handoff_ints_bytes(B, H) : 0);
+    const size_t raw_at = hand_s + (chunked ? handoff_state_bytes(B, H) : 0);
+    if (ln) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
     if (chunked) {
         const long long budget = injected("timeout0") ? 0 : kSpinBudget;
-        e = goldwkv::launch_chunked(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T, H,
-                                    reinterpret_cast<int*>(ws), budget, st);
+        CUtensorMap maps[5];
+        if (!goldwkv::make_token_map(&maps[0], r, B, T, H) ||
+            !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
+            !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
+            !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
+            !goldwkv::make_token_map(&maps[4], y, B, T, H))
+            return WKV_ERR_CUDA;
+        int* status = reinterpret_cast<int*>(ws);
+        int* h_chunk = reinterpret_cast<int*>(ws + hand_i);
+        float* h_state = reinterpret_cast<float*>(ws + hand_s);
+        if (algo == WKV_ALGO_CHUNKED_LEVELS) {
+            e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
+                                               status, nullptr, nullptr, budget, st);
+        } else {
+            e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y_raw, B, T, H,
+                                             status, h_chunk, h_state, budget, st);
+            if (e == cudaSuccess)
+                e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
+                                                   status, h_chunk, h_state, budget, st);
+        }
     } else {
         e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,
                                       H, bf16, st);

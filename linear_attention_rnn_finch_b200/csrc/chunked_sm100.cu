@@ -130,13 +130,18 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
                     const float* s_in, float* s_out, float* __restrict__ y_raw, int T, int H,
-                    int* status, long long spin_budget, long long drain_budget) {
+                    int* status, const int* start_chunk, const float* handoff_state,
+                    long long spin_budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.x, b = bh / H, h = bh - (bh / H) * H;
     const int NC = (T + C - 1) / C;
+    // resume point: chunks before n0 (and the state entering n0) came from the fast kernel
+    const int n0 = start_chunk ? start_chunk[bh] : 0;
+    if (n0 < 0 || n0 >= NC) return;       // this (b,h) is already complete
+    if (start_chunk) s_in = handoff_state;
 
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
@@ -162,7 +167,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     const uint32_t tmem = s.tmem_base;
 
     auto issue_load = [&](int chunk) {
-        const int st = chunk % kStages;
+        const int st = (chunk - n0) % kStages;
         ptx::mbar_arrive_expect_tx(&s.full[st], 4 * kTile);
         const int t0 = chunk * C;
         ptx::tma_load_4d(s.in[st][0], &tm_r, &s.full[st], 0, h, t0, b);
@@ -171,7 +176,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
         ptx::tma_load_4d(s.in[st][3], &tm_w, &s.full[st], 0, h, t0, b);
     };
     if (tid == 0)
-        for (int c = 0; c < kStages && c < NC; ++c) issue_load(c);
+        for (int c = n0; c < n0 + kStages && c < NC; ++c) issue_load(c);
 
     // ------------------------------------------------------------ state in registers
     // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in lanes 0..15), column half hh
@@ -203,20 +208,21 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     }
 
     bool failed = false;
-    int n = 0;
+    int n = n0;
     int issued1 = -1, issued2 = -1;   // last chunk whose MMA group 1 / 2 thread 0 issued
     for (; n < NC; ++n) {
-        const int st = n % kStages;
+        const int m = n - n0;             // position since the start: stage and phase parity
+        const int st = m % kStages;
         const int t0 = n * C;
         const int valid = min(C, T - t0);
         uint8_t* r_tile = s.in[st][0];
         uint8_t* k_tile = s.in[st][1];
         uint8_t* v_tile = s.in[st][2];
         uint8_t* w_tile = s.in[st][3];
-        uint8_t* y_tile = s.ystage[n & 1];
+        uint8_t* y_tile = s.ystage[m & 1];
         if (tid == 0) ptx::bulk_wait_read<1>();    // the store that last used y_tile has read it
 
-        if (!ptx::mbar_wait(&s.full[st], (uint32_t)((n / kStages) & 1), spin_budget)) s.abort = 1;
+        if (!ptx::mbar_wait(&s.full[st], (uint32_t)((m / kStages) & 1), spin_budget)) s.abort = 1;
 
         // -------------------------------------------------------- prep
         {
@@ -341,7 +347,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             ptx::mma_commit(&s.mma1);
             issued1 = n;
         }
-        if (!ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), spin_budget)) s.abort = 1;
+        if (!ptx::mbar_wait(&s.mma1, (uint32_t)(m & 1), spin_budget)) s.abort = 1;
         ptx::tc_fence_after();
 
         // -------------------------------------------------------- state chain
@@ -444,7 +450,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             ptx::mma_commit(&s.mma2);
             issued2 = n;
         }
-        if (!ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), spin_budget)) s.abort = 1;
+        if (!ptx::mbar_wait(&s.mma2, (uint32_t)(m & 1), spin_budget)) s.abort = 1;
         ptx::tc_fence_after();
 
         // -------------------------------------------------------- epilogue
@@ -495,9 +501,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             atomicExch(status, 1);
             // copies still in flight: chunks n .. min(NC, n + kStages) - 1 may have been issued
             for (int c = n; c < NC && c < n + kStages; ++c)
-                ptx::mbar_wait(&s.full[c % kStages], (uint32_t)((c / kStages) & 1), drain_budget);
-            if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), drain_budget);
-            if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), drain_budget);
+                ptx::mbar_wait(&s.full[(c - n0) % kStages], (uint32_t)(((c - n0) / kStages) & 1),
+                               drain_budget);
+            if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)((n - n0) & 1), drain_budget);
+            if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)((n - n0) & 1), drain_budget);
         }
     } else if (s_out != nullptr && row_lane) {
         float* dst = s_out + (size_t)bh * 4096 + row * 64 + 32 * hh;
@@ -514,12 +521,14 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     }
 }
 
+}  // namespace
+
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiled encode_fn() {
+static EncodeTiled encode_fn() {
     static EncodeTiled fn = []() -> EncodeTiled {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -532,8 +541,9 @@ EncodeTiled encode_fn() {
     return fn;
 }
 
-// [B][T][H][64] bf16 viewed as 4-D (D, H, T, B); box = 64 channels x 1 head x 64 tokens.
-bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
+// [B][T][H][64] bf16 viewed as 4-D (D, H, T, B); box = 64 channels x 1 head x 64 tokens,
+// 128-byte swizzle.  Rows past T read as zeros and are not written by stores.
+bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H) {
     EncodeTiled enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[4] = {64, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -546,25 +556,20 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
            CUDA_SUCCESS;
 }
 
-}  // namespace
-
 size_t chunked_smem_bytes() { return sizeof(Smem) + 1024; }
 
-cudaError_t launch_chunked(const void* r, const void* k, const void* v, const void* omega,
-                           const float* u, const float* s_in, float* s_out, void* y,
-                           float* y_raw, int B, int T, int H, int* status, long long spin_budget,
-                           cudaStream_t st) {
-    CUtensorMap mr, mk, mv, mw, my;
-    if (!make_map(&mr, r, B, T, H) || !make_map(&mk, k, B, T, H) || !make_map(&mv, v, B, T, H) ||
-        !make_map(&mw, omega, B, T, H) || !make_map(&my, y, B, T, H))
-        return cudaErrorInvalidValue;
+cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
+                                  float* s_out, float* y_raw, int B, int T, int H, int* status,
+                                  const int* start_chunk, const float* handoff_state,
+                                  long long spin_budget, cudaStream_t st) {
     const size_t smem = chunked_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long drain = 4000000000LL;
     wkv6_chunked_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
-        mr, mk, mv, mw, my, u, s_in, s_out, y_raw, T, H, status, spin_budget, drain);
+        maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw, T, H, status,
+        start_chunk, handoff_state, spin_budget, drain);
     return cudaGetLastError();
 }
 

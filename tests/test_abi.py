@@ -52,12 +52,14 @@ def test_status_strings_and_version():
 
 def test_workspace_queries():
     import torch
-    # the chunked path keeps a 256-byte status block; LayerNorm with bf16 output adds an
-    # fp32 staging buffer of y; the fp32 recurrence needs nothing
-    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False) == 256
+    # the chunked path keeps a 256-byte status block and a hand-off record per (b,h)
+    # (chunk index, rounded up to 256 bytes in total, and a 16 KB state); LayerNorm with bf16
+    # output adds an fp32 staging buffer of y; the fp32 recurrence needs nothing
+    hand = lambda B, H: 256 + ((B * H * 4 + 255) // 256) * 256 + B * H * 64 * 64 * 4
+    assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False) == hand(4, 32)
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False, "recurrent") == 0
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.float32, True) == 0
-    assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True) == 256 + 2 * 10 * 3 * 64 * 4
+    assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True) == hand(2, 3) + 2 * 10 * 3 * 64 * 4
     assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True, "recurrent") == 2 * 10 * 3 * 64 * 4
     assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, True) == 256 * 32 * 64 * 4
     assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, False) == 0

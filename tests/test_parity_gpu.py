@@ -16,7 +16,7 @@ from tests.parity import TOL, f64, oracle_heads, rel_err
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-BF16_ALGOS = ["chunked", "recurrent"]
+BF16_ALGOS = ["chunked", "chunked_levels", "recurrent"]
 
 
 def _run(inp, algo="auto", T=None, ln=False, state=True):
@@ -120,6 +120,41 @@ def test_decay_saturated(oracle, algo, omega_value):
     yo, so = _oracle_full(oracle, inp)
     assert rel_err(y, yo) <= TOL[torch.bfloat16]
     assert rel_err(s, so) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("extreme_from", [0, 64, 130, 300])
+def test_handoff_mid_sequence(oracle, extreme_from):
+    """Mild decays up to token `extreme_from`, then some channels with w ~ 0: the fast
+    kernel takes the first chunks and hands the rest (and its state) to the level kernel."""
+    cfg = W.CONFIGS[1].with_(seed=7550 + extreme_from)
+    inp = W.make_prefill_inputs(cfg, DEV, B=2, T=400)
+    for n in ("r", "k", "v", "omega"):
+        inp[n] = inp[n][:, :, :4].contiguous()
+    inp["u"], inp["state0"] = inp["u"][:4].contiguous(), inp["state0"][:, :4].contiguous()
+    om = inp["omega"].float()
+    om[:, extreme_from:, :, ::3] = 3.5          # exp(-exp(3.5)) ~ 4e-15 per token
+    inp["omega"] = om.to(torch.bfloat16)
+    y, s = _run(inp, "chunked")
+    yo, so = _oracle_full(oracle, inp)
+    assert rel_err(y, yo) <= TOL[torch.bfloat16]
+    assert rel_err(s, so) <= TOL[torch.bfloat16]
+
+
+def test_isolated_extreme_chunk(oracle):
+    """A single chunk with an extreme decay in the middle of a mild sequence."""
+    cfg = W.CONFIGS[1].with_(seed=7560)
+    inp = W.make_prefill_inputs(cfg, DEV, B=1, T=320)
+    for n in ("r", "k", "v", "omega"):
+        inp[n] = inp[n][:, :, :2].contiguous()
+    inp["u"], inp["state0"] = inp["u"][:2].contiguous(), inp["state0"][:, :2].contiguous()
+    om = inp["omega"].float()
+    om[:, 128:192, 1, 5] = 6.0
+    inp["omega"] = om.to(torch.bfloat16)
+    for algo in ("chunked", "chunked_levels"):
+        y, s = _run(inp, algo)
+        yo, so = _oracle_full(oracle, inp)
+        assert rel_err(y, yo) <= TOL[torch.bfloat16], algo
+        assert rel_err(s, so) <= TOL[torch.bfloat16], algo
 
 
 def test_deterministic():
