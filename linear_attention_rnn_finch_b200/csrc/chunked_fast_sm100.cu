@@ -24,10 +24,10 @@
 // the combination is one add in registers.  With all parts split the arithmetic is as
 // accurate as fp32; the only bf16 rounding left is that of the output y.
 //
-// Per chunk three MMA groups (K = 64, four K16 instructions each):
-//   G1: [Rt_hi ; Rt_lo] (M=128) x [S_hi^T ; S_lo^T ; Kh_hi ; Kh_lo]^T (N=256) -> D1
-//       columns   0..127: readout Rt . S (hi and lo parts of S)
-//       columns 128..255: intra-chunk scores Rt . Kh (hi and lo parts of Kh)
+// Per chunk three MMA groups (K = 64, four K16 instructions per chain):
+//   G1: [Rt_hi ; Rt_lo] (M=128) x [S_hi^T ; Kh_hi]^T, then x [S_lo^T ; Kh_lo]^T accumulated
+//       into the same columns (N=128) -> D1: columns 0..63 readout Rt . S, columns 64..127
+//       intra-chunk scores Rt . Kh (hi and lo parts of S and Kh summed by the MMA)
 //   GU: V^T (M=64) x [Kh_hi | Kh_lo] (N=128) -> DU = (Kh^T V)^T, the state increment
 //   GA: [A_hi ; A_lo] (M=128) x V (N=64) -> DA, the intra-chunk output A . V
 //
@@ -53,18 +53,18 @@ constexpr int kThreads = 448;
 constexpr int kPrepWarp0 = 2, kEpiWarp0 = 6;
 constexpr int kEpiThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t COL_D1 = 0, COL_DU = 256, COL_DA = 384;
+constexpr uint32_t COL_D1 = 0, COL_DU = 128, COL_DA = 256;
 // log2 of the largest factor exp(-L_s) allowed: ln range 60 -> log2 range 86.56
 constexpr float kMaxLog2Range = 86.5617f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr uint32_t IDESC_G1 = ptx::idesc_bf16(128, 256, 0, 0);
+constexpr uint32_t IDESC_G1 = ptx::idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t IDESC_GU = ptx::idesc_bf16(64, 128, 1, 1);
 constexpr uint32_t IDESC_GA = ptx::idesc_bf16(128, 64, 0, 1);
 
 struct __align__(1024) Smem {
     uint8_t in[kStages][4][kTile];   // r, k, v, omega tiles (TMA, 128B swizzle)
-    uint8_t bblk[2][4][kTile];       // per parity: S_hi^T, S_lo^T, Kh_hi, Kh_lo (G1 operand B)
+    uint8_t bblk[2][4][kTile];       // per parity: S_hi^T, Kh_hi, S_lo^T, Kh_lo (G1 operand B)
     uint8_t rt[2][2 * kTile];        // per parity: Rt hi/lo, 128 stacked rows (G1 operand A)
     uint8_t at[2 * kTile];           // A hi/lo, 128 stacked rows (GA operand A)
     uint8_t ystage[kTile];           // y tile for the TMA store
@@ -86,20 +86,21 @@ __device__ __forceinline__ uint32_t sw_off(int row, int chunk) {
 // stacked hi/lo row of token t: hi parts in rows 0-7 of each 16-row group, lo in rows 8-15
 __device__ __forceinline__ int hi_row(int t) { return 32 * (t >> 4) + 16 * ((t >> 3) & 1) + (t & 7); }
 
-__device__ __forceinline__ float bf16_lo(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
-
+// bf16x2 of (a, b): a in the low half (lower address), b in the high half
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-// hi / lo pairs of two floats
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const float ah = bf16_lo(a), bh = bf16_lo(b);
-    hi = pack2(ah, bh);
-    lo = pack2(a - ah, b - bh);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
 }
 __device__ __forceinline__ float2 unpack2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// hi = bf16(x), lo = bf16(x - hi) for a pair: two conversions and one packed subtract
+__device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
+    hi = pack2(x.x, x.y);
+    const float2 d = __fadd2_rn(x, make_float2(-__uint_as_float(hi << 16),
+                                               -__uint_as_float(hi & 0xFFFF0000u)));
+    lo = pack2(d.x, d.y);
 }
 __device__ __forceinline__ void sts32(uint8_t* base, uint32_t off, uint32_t v) {
     *reinterpret_cast<uint32_t*>(base + off) = v;
@@ -240,17 +241,22 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 if (n > 0 && !ptx::mbar_wait(&s.epi_mid, (uint32_t)((n - 1) & 1), budget)) { s.abort = 1; break; }
                 ptx::tc_fence_after();
                 const uint32_t v_tile = ptx::smem_addr(s.in[st][2]);
-                const uint32_t bblk = ptx::smem_addr(s.bblk[pb][0]);
-                const uint32_t kh = ptx::smem_addr(s.bblk[pb][2]);
+                const uint32_t bhi = ptx::smem_addr(s.bblk[pb][0]);   // [S_hi^T ; Kh_hi]
+                const uint32_t blo = ptx::smem_addr(s.bblk[pb][2]);   // [S_lo^T ; Kh_lo]
+                const uint32_t kh = ptx::smem_addr(s.bblk[pb][1]);
                 const uint32_t rt = ptx::smem_addr(s.rt[pb]);
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // GU: V^T x [Kh_hi | Kh_lo]
+                for (int kq = 0; kq < 4; ++kq)   // GU: V^T x [Kh_hi | Kh_lo] (N atoms 16 KB apart)
                     ptx::mma_bf16(tmem + COL_DU, ptx::desc_sw128(v_tile + 2048 * kq, 1024),
-                                  ptx::desc_sw128(kh + 2048 * kq, kTile), IDESC_GU, kq > 0);
+                                  ptx::desc_sw128(kh + 2048 * kq, 2 * kTile), IDESC_GU, kq > 0);
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // G1: [Rt] x [S^T ; Kh]
+                for (int kq = 0; kq < 4; ++kq)   // G1: [Rt] x [S_hi^T ; Kh_hi]
                     ptx::mma_bf16(tmem + COL_D1, ptx::desc_kmajor(rt + 32 * kq),
-                                  ptx::desc_kmajor(bblk + 32 * kq), IDESC_G1, kq > 0);
+                                  ptx::desc_kmajor(bhi + 32 * kq), IDESC_G1, kq > 0);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)   //   + [Rt] x [S_lo^T ; Kh_lo]
+                    ptx::mma_bf16(tmem + COL_D1, ptx::desc_kmajor(rt + 32 * kq),
+                                  ptx::desc_kmajor(blo + 32 * kq), IDESC_G1, 1);
                 ptx::mma_commit(&s.g1_done);
                 last_g1 = n;
                 // GA needs A (assembly of n) and DA free (output of n-1 read)
@@ -273,11 +279,14 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------ prep (4 warps)
-        const int qw = warp - kPrepWarp0;     // token quarter: tokens 16qw .. 16qw+15
-        const int c0 = 2 * lane;              // channels c0, c0+1
-        const float u0 = u[h * 64 + c0], u1 = u[h * 64 + c0 + 1];
-        const int chunk = lane >> 2;          // 16-byte chunk of channels c0, c0+1
+        // lane = channel pair (2l, 2l+1), warp = token quarter (16 tokens); log2 units
+        const int qw = warp - kPrepWarp0;
+        const int c0 = 2 * lane;
+        const float2 uu = make_float2(u[h * 64 + c0], u[h * 64 + c0 + 1]);
+        const int chunk = lane >> 2;          // 16-byte chunk holding channels c0, c0+1
         const uint32_t cbyte = (uint32_t)(lane & 3) * 4;
+        const float2 l2e = make_float2(kLog2e, kLog2e);
+        const float2 nl2e = make_float2(-kLog2e, -kLog2e);
         for (int n = 0; n < NC; ++n) {
             const int pb = n & 1, st = n % kStages;
             const int valid = min(C, T - n * C);
@@ -288,64 +297,61 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             const uint8_t* r_tile = s.in[st][0];
             const uint8_t* k_tile = s.in[st][1];
             const uint8_t* w_tile = s.in[st][3];
-            // pass 1: log2 decay, local inclusive prefix; bonus partials
-            float L0[16], L1[16], bon[16];
-            float a0 = 0.f, a1 = 0.f;
+            // pass 1: local inclusive prefix of log2 w = -exp(omega) log2(e)
+            float2 L[16];
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int p = 0; p < 16; ++p) {
                 const int t = 16 * qw + p;
-                const uint32_t off = sw_off(t, chunk) + cbyte;
-                const float2 om = unpack2(lds32(w_tile, off));
-                const float2 rr = unpack2(lds32(r_tile, off));
-                const float2 kk = unpack2(lds32(k_tile, off));
-                const bool live = t < valid;
-                // log2 w = -exp(omega) * log2(e)
-                const float e0 = live ? fast_exp2(om.x * kLog2e) : 0.f;
-                const float e1 = live ? fast_exp2(om.y * kLog2e) : 0.f;
-                a0 = fmaf(-e0, kLog2e, a0);
-                a1 = fmaf(-e1, kLog2e, a1);
-                L0[p] = a0;
-                L1[p] = a1;
-                bon[p] = fmaf(rr.x * u0, kk.x, rr.y * u1 * kk.y);
+                const float2 om = __fmul2_rn(unpack2(lds32(w_tile, sw_off(t, chunk) + cbyte)), l2e);
+                float2 e = make_float2(fast_exp2(om.x), fast_exp2(om.y));
+                if (t >= valid) e = make_float2(0.f, 0.f);
+                acc = __ffma2_rn(e, nl2e, acc);
+                L[p] = acc;
             }
-            s.qtot[qw][c0] = a0;
-            s.qtot[qw][c0 + 1] = a1;
+            s.qtot[qw][c0] = acc.x;
+            s.qtot[qw][c0 + 1] = acc.y;
             named_bar(1, 128);
-            float o0 = 0.f, o1 = 0.f, tot0 = 0.f, tot1 = 0.f;
+            float2 off = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const float q0 = s.qtot[w][c0], q1 = s.qtot[w][c0 + 1];
-                if (w < qw) { o0 += q0; o1 += q1; }
-                tot0 += q0;
-                tot1 += q1;
+                const float2 qv = make_float2(s.qtot[w][c0], s.qtot[w][c0 + 1]);
+                if (w < qw) off = __fadd2_rn(off, qv);
+                tot = __fadd2_rn(tot, qv);
             }
-            const bool ok = __all_sync(0xffffffffu, (tot0 >= -kMaxLog2Range) && (tot1 >= -kMaxLog2Range));
+            const bool ok = __all_sync(0xffffffffu, (tot.x >= -kMaxLog2Range) && (tot.y >= -kMaxLog2Range));
             if (!ok) {
                 if (qw == 0 && lane == 0) s.unsafe[pb] = 1;
                 named_bar(1, 128);           // qtot is reused by the next chunk
                 mbar_arrive(&s.prep_done[pb]);
                 break;                        // this (b,h) continues in the level kernel
             }
-            // pass 2: Rt = r * 2^(L excl), Kh = k * 2^(-L incl), hi / lo parts
+            // pass 2: Rt = r 2^(L_{t-1}), Kh = k 2^(-L_t) as bf16 hi / lo; bonus partials
             uint8_t* rt = s.rt[pb];
-            uint8_t* kh_hi = s.bblk[pb][2];
+            uint8_t* kh_hi = s.bblk[pb][1];
             uint8_t* kh_lo = s.bblk[pb][3];
+            float bon[16];
+            float2 fr = make_float2(fast_exp2(off.x), fast_exp2(off.y));   // 2^(L_{t-1})
 #pragma unroll
             for (int p = 0; p < 16; ++p) {
                 const int t = 16 * qw + p;
-                const uint32_t off = sw_off(t, chunk) + cbyte;
-                const float2 rr = unpack2(lds32(r_tile, off));
-                const float2 kk = unpack2(lds32(k_tile, off));
-                const float le0 = o0 + (p ? L0[p - 1] : 0.f), le1 = o1 + (p ? L1[p - 1] : 0.f);
-                const float li0 = o0 + L0[p], li1 = o1 + L1[p];
+                const uint32_t o = sw_off(t, chunk) + cbyte;
+                const float2 rr = unpack2(lds32(r_tile, o));
+                const float2 kk = unpack2(lds32(k_tile, o));
+                const float2 li = __fadd2_rn(off, L[p]);
+                const float2 fk = make_float2(fast_exp2(-li.x), fast_exp2(-li.y));
                 uint32_t hi, lo;
-                split2(rr.x * fast_exp2(le0), rr.y * fast_exp2(le1), hi, lo);
+                split2(__fmul2_rn(rr, fr), hi, lo);
                 const int hr = hi_row(t);
-                sts32(rt, sw_off(hr, chunk) + cbyte, hi);
-                sts32(rt, sw_off(hr + 8, chunk) + cbyte, lo);
-                split2(kk.x * fast_exp2(-li0), kk.y * fast_exp2(-li1), hi, lo);
-                sts32(kh_hi, off, hi);
-                sts32(kh_lo, off, lo);
+                const uint32_t cb = (uint32_t)(chunk ^ (t & 7)) << 4;
+                sts32(rt, (uint32_t)hr * 128 + cb + cbyte, hi);
+                sts32(rt, (uint32_t)(hr + 8) * 128 + cb + cbyte, lo);
+                split2(__fmul2_rn(kk, fk), hi, lo);
+                sts32(kh_hi, o, hi);
+                sts32(kh_lo, o, lo);
+                const float2 ru = __fmul2_rn(rr, uu);
+                bon[p] = fmaf(ru.x, kk.x, ru.y * kk.y);
+                if (p < 15) fr = make_float2(fast_exp2(li.x), fast_exp2(li.y));
             }
             // bonus: reduce the 16 per-token partials over the 32 lanes (reduce-scatter)
 #pragma unroll
@@ -382,8 +388,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 s.bonus[pb][16 * qw + p] = bon[0];
             }
             if (qw == 0) {
-                s.gamma[pb][c0] = fast_exp2(tot0);
-                s.gamma[pb][c0 + 1] = fast_exp2(tot1);
+                s.gamma[pb][c0] = fast_exp2(tot.x);
+                s.gamma[pb][c0 + 1] = fast_exp2(tot.y);
                 if (lane == 0) s.unsafe[pb] = 0;
             }
             ptx::fence_proxy_async_smem();
@@ -392,41 +398,60 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ epilogue (8 warps)
-        const int q = warp & 3;               // TMEM sub-partition: rows 32q .. 32q+31
-        const int ch = (warp - kEpiWarp0) >> 2;  // column half of every 64-wide block
+        // warp (q, ch): TMEM sub-partition q, columns 32ch .. 32ch+31 of each 64-wide block.
+        // Thread: token / state rows r0 = 16q + l/4 and r1 = r0 + 8; column pairs
+        // cbase + 8k + {0,1}, k = 0..3.
+        const int q = warp & 3;
+        const int ch = (warp - kEpiWarp0) >> 2;
         const int et = tid - kEpiWarp0 * 32;  // 0 .. 255
-        const int r0 = 16 * q + (lane >> 2), r1 = r0 + 8;   // token rows / state rows
-        const int cbase = 32 * ch + 2 * (lane & 3);          // + 8k + {0,1}, k = 0..3
+        const int r0 = 16 * q + (lane >> 2), r1 = r0 + 8;
+        const int cbase = 32 * ch + 2 * (lane & 3);
+        const uint32_t cb = (uint32_t)(lane & 3) * 4;
         const uint32_t lane_m64 = (uint32_t)(32 * q) << 16;
         const uint32_t lane_h0 = (uint32_t)(32 * q) << 16, lane_h1 = (uint32_t)(32 * q + 16) << 16;
-        // state S[j][i] held transposed: rows j = r0, r1; columns i = cbase + 8k + {0,1}
-        float S0[8], S1[8];
+        // A block of this warp: rows 16q..16q+15, columns 32ch..32ch+31
+        const bool a_zero = 16 * q + 15 < 32 * ch;      // entirely above the diagonal
+        const bool a_full = 16 * q >= 32 * ch + 32;     // entirely below the diagonal
+        const int hr0 = hi_row(r0), hr1 = hi_row(r1);
+        // state S[i][j] held transposed: rows j = r0, r1; columns i = cbase + 8k + {0,1}
+        float2 S0[4], S1[4];
         {
             const float* src = s_in ? s_in + (size_t)bh * 4096 : nullptr;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int i = cbase + 8 * k + e;
-                    S0[2 * k + e] = src ? src[i * 64 + r0] : 0.f;
-                    S1[2 * k + e] = src ? src[i * 64 + r1] : 0.f;
-                }
-            // S_0 into parity 0: S_hi^T / S_lo^T rows j, K index i
+            for (int k = 0; k < 4; ++k) {
+                const int i = cbase + 8 * k;
+                S0[k] = src ? make_float2(src[i * 64 + r0], src[(i + 1) * 64 + r0]) : make_float2(0.f, 0.f);
+                S1[k] = src ? make_float2(src[i * 64 + r1], src[(i + 1) * 64 + r1]) : make_float2(0.f, 0.f);
+            }
+            // S_0 into parity 0: S_hi^T (tile 0) / S_lo^T (tile 2), rows j, K index i
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const uint32_t o0 = sw_off(r0, 4 * ch + k) + (uint32_t)(lane & 3) * 4;
-                const uint32_t o1 = sw_off(r1, 4 * ch + k) + (uint32_t)(lane & 3) * 4;
                 uint32_t hi, lo;
-                split2(S0[2 * k], S0[2 * k + 1], hi, lo);
-                sts32(s.bblk[0][0], o0, hi);
-                sts32(s.bblk[0][1], o0, lo);
-                split2(S1[2 * k], S1[2 * k + 1], hi, lo);
-                sts32(s.bblk[0][0], o1, hi);
-                sts32(s.bblk[0][1], o1, lo);
+                split2(S0[k], hi, lo);
+                sts32(s.bblk[0][0], sw_off(r0, 4 * ch + k) + cb, hi);
+                sts32(s.bblk[0][2], sw_off(r0, 4 * ch + k) + cb, lo);
+                split2(S1[k], hi, lo);
+                sts32(s.bblk[0][0], sw_off(r1, 4 * ch + k) + cb, hi);
+                sts32(s.bblk[0][2], sw_off(r1, 4 * ch + k) + cb, lo);
+            }
+            // blocks of A that are always zero are written once here
+            if (a_zero) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    sts32(s.at, sw_off(hr0, 4 * ch + k) + cb, 0u);
+                    sts32(s.at, sw_off(hr0 + 8, 4 * ch + k) + cb, 0u);
+                    sts32(s.at, sw_off(hr1, 4 * ch + k) + cb, 0u);
+                    sts32(s.at, sw_off(hr1 + 8, 4 * ch + k) + cb, 0u);
+                }
             }
             ptx::fence_proxy_async_smem();
             mbar_arrive(&s.s_init);
         }
+        // sum of the hi row (regs 4k, 4k+1) and lo row (regs 4k+2, 4k+3) of a 16x256b load
+        auto rows_sum = [](const uint32_t (&v)[16], int k) {
+            return __fadd2_rn(make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1])),
+                              make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+        };
         int n = 0;
         for (; n < NC; ++n) {
             const int pb = n & 1;
@@ -444,78 +469,63 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             // ---- state: S <- gamma (S + U), U^T[j][i] = DU[j][i] + DU[j][64+i]
             {
                 uint32_t ua[16], ub[16];
-                ptx::tmem_wait_ld();
                 tmem_ld16x4(tmem + lane_m64 + COL_DU + 32 * ch, ua);
                 tmem_ld16x4(tmem + lane_m64 + COL_DU + 64 + 32 * ch, ub);
                 ptx::tmem_wait_ld();
                 uint8_t* sh = s.bblk[pb ^ 1][0];
-                uint8_t* sl = s.bblk[pb ^ 1][1];
+                uint8_t* sl = s.bblk[pb ^ 1][2];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    float nv0[2], nv1[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int i = cbase + 8 * k + e;
-                        const float g = s.gamma[pb][i];
-                        const float du0 = __uint_as_float(ua[4 * k + e]) + __uint_as_float(ub[4 * k + e]);
-                        const float du1 = __uint_as_float(ua[4 * k + 2 + e]) + __uint_as_float(ub[4 * k + 2 + e]);
-                        S0[2 * k + e] = g * (S0[2 * k + e] + du0);
-                        S1[2 * k + e] = g * (S1[2 * k + e] + du1);
-                        nv0[e] = S0[2 * k + e];
-                        nv1[e] = S1[2 * k + e];
-                    }
+                    const float2 g = *reinterpret_cast<const float2*>(&s.gamma[pb][cbase + 8 * k]);
+                    const float2 du0 = __fadd2_rn(make_float2(__uint_as_float(ua[4 * k]), __uint_as_float(ua[4 * k + 1])),
+                                                  make_float2(__uint_as_float(ub[4 * k]), __uint_as_float(ub[4 * k + 1])));
+                    const float2 du1 = __fadd2_rn(make_float2(__uint_as_float(ua[4 * k + 2]), __uint_as_float(ua[4 * k + 3])),
+                                                  make_float2(__uint_as_float(ub[4 * k + 2]), __uint_as_float(ub[4 * k + 3])));
+                    S0[k] = __fmul2_rn(g, __fadd2_rn(S0[k], du0));
+                    S1[k] = __fmul2_rn(g, __fadd2_rn(S1[k], du1));
                     uint32_t hi, lo;
-                    const uint32_t o0 = sw_off(r0, 4 * ch + k) + (uint32_t)(lane & 3) * 4;
-                    const uint32_t o1 = sw_off(r1, 4 * ch + k) + (uint32_t)(lane & 3) * 4;
-                    split2(nv0[0], nv0[1], hi, lo);
-                    sts32(sh, o0, hi);
-                    sts32(sl, o0, lo);
-                    split2(nv1[0], nv1[1], hi, lo);
-                    sts32(sh, o1, hi);
-                    sts32(sl, o1, lo);
+                    split2(S0[k], hi, lo);
+                    sts32(sh, sw_off(r0, 4 * ch + k) + cb, hi);
+                    sts32(sl, sw_off(r0, 4 * ch + k) + cb, lo);
+                    split2(S1[k], hi, lo);
+                    sts32(sh, sw_off(r1, 4 * ch + k) + cb, hi);
+                    sts32(sl, sw_off(r1, 4 * ch + k) + cb, lo);
                 }
             }
             // ---- readout part Yi (kept in registers) and scores A -> A_hi / A_lo tiles
-            float Y0[8], Y1[8], A0[8], A1[8];
+            float2 Y0[4], Y1[4];
             {
-                // hi and lo rows of one (token half, column block) pair, summed in registers
-                auto load_pair = [&](uint32_t lane_base, uint32_t col_a, uint32_t col_b, float (&out)[8]) {
-                    uint32_t pa[16], pq[16];
-                    tmem_ld16x4(tmem + lane_base + col_a + 32 * ch, pa);
-                    tmem_ld16x4(tmem + lane_base + col_b + 32 * ch, pq);
-                    ptx::tmem_wait_ld();
+                uint32_t p0[16], p1[16];
+                tmem_ld16x4(tmem + lane_h0 + COL_D1 + 32 * ch, p0);
+                tmem_ld16x4(tmem + lane_h1 + COL_D1 + 32 * ch, p1);
+                ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int x = 4 * k + e;       // hi row; x + 2 is the lo row
-                            out[2 * k + e] = (__uint_as_float(pa[x]) + __uint_as_float(pa[x + 2])) +
-                                             (__uint_as_float(pq[x]) + __uint_as_float(pq[x + 2]));
-                        }
-                };
-                load_pair(lane_h0, COL_D1 + 0, COL_D1 + 64, Y0);     // Rt . (S_hi + S_lo)
-                load_pair(lane_h1, COL_D1 + 0, COL_D1 + 64, Y1);
-                load_pair(lane_h0, COL_D1 + 128, COL_D1 + 192, A0);  // Rt . (Kh_hi + Kh_lo)
-                load_pair(lane_h1, COL_D1 + 128, COL_D1 + 192, A1);
-                // mask: strictly causal scores, bonus on the diagonal
+                for (int k = 0; k < 4; ++k) {
+                    Y0[k] = rows_sum(p0, k);
+                    Y1[k] = rows_sum(p1, k);
+                }
+            }
+            if (!a_zero) {
+                uint32_t p0[16], p1[16];
+                tmem_ld16x4(tmem + lane_h0 + COL_D1 + 64 + 32 * ch, p0);
+                tmem_ld16x4(tmem + lane_h1 + COL_D1 + 64 + 32 * ch, p1);
+                ptx::tmem_wait_ld();
                 const float b0 = s.bonus[pb][r0], b1 = s.bonus[pb][r1];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    float m0[2], m1[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int sidx = cbase + 8 * k + e;
-                        const float a0v = A0[2 * k + e], a1v = A1[2 * k + e];
-                        m0[e] = sidx < r0 ? a0v : (sidx == r0 ? b0 : 0.f);
-                        m1[e] = sidx < r1 ? a1v : (sidx == r1 ? b1 : 0.f);
+                    float2 a0 = rows_sum(p0, k), a1 = rows_sum(p1, k);
+                    if (!a_full) {   // strictly causal scores, bonus on the diagonal
+                        const int sx = cbase + 8 * k;
+                        a0.x = sx < r0 ? a0.x : (sx == r0 ? b0 : 0.f);
+                        a0.y = sx + 1 < r0 ? a0.y : (sx + 1 == r0 ? b0 : 0.f);
+                        a1.x = sx < r1 ? a1.x : (sx == r1 ? b1 : 0.f);
+                        a1.y = sx + 1 < r1 ? a1.y : (sx + 1 == r1 ? b1 : 0.f);
                     }
                     uint32_t hi, lo;
-                    const int hr0 = hi_row(r0), hr1 = hi_row(r1);
-                    const uint32_t cb = (uint32_t)(lane & 3) * 4;
-                    split2(m0[0], m0[1], hi, lo);
+                    split2(a0, hi, lo);
                     sts32(s.at, sw_off(hr0, 4 * ch + k) + cb, hi);
                     sts32(s.at, sw_off(hr0 + 8, 4 * ch + k) + cb, lo);
-                    split2(m1[0], m1[1], hi, lo);
+                    split2(a1, hi, lo);
                     sts32(s.at, sw_off(hr1, 4 * ch + k) + cb, hi);
                     sts32(s.at, sw_off(hr1 + 8, 4 * ch + k) + cb, lo);
                 }
@@ -530,18 +540,17 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 if (named_bar_any(3, kEpiThreads, bad || ld_volatile(&s.abort))) break;
             }
             ptx::tc_fence_after();
-            uint32_t d0[16], d1[16];
-            tmem_ld16x4(tmem + lane_h0 + COL_DA + 32 * ch, d0);
-            tmem_ld16x4(tmem + lane_h1 + COL_DA + 32 * ch, d1);
-            ptx::tmem_wait_ld();
+            {
+                uint32_t d0[16], d1[16];
+                tmem_ld16x4(tmem + lane_h0 + COL_DA + 32 * ch, d0);
+                tmem_ld16x4(tmem + lane_h1 + COL_DA + 32 * ch, d1);
+                ptx::tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int x = 4 * k + e;
-                    Y0[2 * k + e] += __uint_as_float(d0[x]) + __uint_as_float(d0[x + 2]);
-                    Y1[2 * k + e] += __uint_as_float(d1[x]) + __uint_as_float(d1[x + 2]);
+                for (int k = 0; k < 4; ++k) {
+                    Y0[k] = __fadd2_rn(Y0[k], rows_sum(d0, k));
+                    Y1[k] = __fadd2_rn(Y1[k], rows_sum(d1, k));
                 }
+            }
             ptx::tc_fence_before();
             mbar_arrive(&s.epi_end);    // DA read: GA of the next chunk may overwrite it
             if (y_raw != nullptr) {
@@ -549,21 +558,18 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 for (int k = 0; k < 4; ++k) {
                     const int j = cbase + 8 * k;
                     if (r0 < valid)
-                        *reinterpret_cast<float2*>(y_raw + (((size_t)b * T + n * C + r0) * H + h) * 64 + j) =
-                            make_float2(Y0[2 * k], Y0[2 * k + 1]);
+                        *reinterpret_cast<float2*>(y_raw + (((size_t)b * T + n * C + r0) * H + h) * 64 + j) = Y0[k];
                     if (r1 < valid)
-                        *reinterpret_cast<float2*>(y_raw + (((size_t)b * T + n * C + r1) * H + h) * 64 + j) =
-                            make_float2(Y1[2 * k], Y1[2 * k + 1]);
+                        *reinterpret_cast<float2*>(y_raw + (((size_t)b * T + n * C + r1) * H + h) * 64 + j) = Y1[k];
                 }
             } else {
                 // the previous chunk's store must have read the staging tile
                 if (et == 0) ptx::bulk_wait_read<0>();
                 named_bar(2, kEpiThreads);
-                const uint32_t cb = (uint32_t)(lane & 3) * 4;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    sts32(s.ystage, sw_off(r0, 4 * ch + k) + cb, pack2(Y0[2 * k], Y0[2 * k + 1]));
-                    sts32(s.ystage, sw_off(r1, 4 * ch + k) + cb, pack2(Y1[2 * k], Y1[2 * k + 1]));
+                    sts32(s.ystage, sw_off(r0, 4 * ch + k) + cb, pack2(Y0[k].x, Y0[k].y));
+                    sts32(s.ystage, sw_off(r1, 4 * ch + k) + cb, pack2(Y1[k].x, Y1[k].y));
                 }
                 ptx::fence_proxy_async_smem();
                 named_bar(2, kEpiThreads);
@@ -580,13 +586,13 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             float* dst = stopped ? handoff_state + (size_t)bh * 4096 : s_out ? s_out + (size_t)bh * 4096 : nullptr;
             if (dst) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int i = cbase + 8 * k + e;
-                        dst[i * 64 + r0] = S0[2 * k + e];
-                        dst[i * 64 + r1] = S1[2 * k + e];
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    const int i = cbase + 8 * k;
+                    dst[i * 64 + r0] = S0[k].x;
+                    dst[(i + 1) * 64 + r0] = S0[k].y;
+                    dst[i * 64 + r1] = S1[k].x;
+                    dst[(i + 1) * 64 + r1] = S1[k].y;
+                }
             }
             if (et == 0) handoff_chunk[bh] = stopped ? n : -1;
         }
