@@ -19,9 +19,9 @@
  * Conventions shared by every entry point
  *  - Pointers r, k, v, omega, u, state*, y, gamma, beta, workspace are DEVICE pointers on
  *    the current CUDA device; the caller owns every buffer.  The library never allocates
- *    device memory, keeps no global mutable state and, apart from wkv6_workspace_status,
- *    never synchronises, so calls on different streams with different workspaces are
- *    independent.
+ *    device memory, keeps no global mutable state (one exception: the built-in scratch of
+ *    wkv6_prefill_static) and, apart from wkv6_workspace_status, never synchronises, so
+ *    calls on different streams with different workspaces are independent.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
  *    enqueued asynchronously; a device-side fault surfaces as a CUDA error at the caller's
  *    next synchronisation.
@@ -142,6 +142,47 @@ wkv_status wkv6_decode_step(const void *r, const void *k, const void *v, const v
                             const float *u, float *state, void *y, int B, int H, int D,
                             wkv_dtype io, const wkv_ln *ln, void *workspace,
                             size_t workspace_bytes, void *stream);
+
+/* Size of the scratch array built into the library for wkv6_prefill_static, per device. */
+#define WKV6_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * Prefill that allocates nothing and takes no workspace argument.  The pages have no
+ * counterpart: this is a calling convention of this library, not part of the method.
+ *
+ * Who it is for: callers that cannot hand the library device memory at call time, for
+ * example code that runs where allocating is not allowed or not safe (a runtime that
+ * forbids allocation once it is running, a region whose memory is owned by someone else,
+ * a latency-bound loop where an allocation might block or fail), and which also cannot
+ * keep a workspace of its own alive between calls.
+ *
+ * Same arguments, results and errors as wkv6_prefill (WKV_ALGO_AUTO) without the two
+ * workspace arguments.  The workspace wkv6_prefill would need is taken instead from a
+ * scratch array of WKV6_STATIC_SCRATCH_BYTES bytes compiled into the library (one per
+ * device).  Neither this call nor anything it calls allocates memory.
+ *   - Limit: sizes for which wkv6_prefill_workspace_bytes(B, T, H, D, io, ln != NULL,
+ *     WKV_ALGO_AUTO) exceeds WKV6_STATIC_SCRATCH_BYTES return WKV_ERR_WORKSPACE with
+ *     nothing launched.  On the chunked path (bf16 I/O) that is 16 KB per (b,h) plus a
+ *     little, so up to 511 (b,h) pairs without LayerNorm; bf16 with LayerNorm also needs
+ *     4 * B*T*H*D bytes and fits only for small problems.  fp32 I/O needs no scratch.
+ *   - Set-up: the first call on each device, with that device current, looks up the
+ *     scratch's device address (cudaGetSymbolAddress, which may load the library's device
+ *     code) and caches it; a failed lookup returns WKV_ERR_CUDA.  Make that first call, on
+ *     every device that will use it, before capturing a stream that will contain it.
+ *   - Zero state: the scratch's first 4 bytes are the chunked path's status word, zero
+ *     when the library's device code is loaded.  Nothing else in it has to start at zero:
+ *     every other byte a call reads was written earlier in the same call.  A wait that
+ *     expires sets the word; this entry point does not report it (there is no
+ *     wkv6_workspace_status for it), and the word has no effect on any result.
+ *   - Concurrency: all calls on one device share the one scratch.  Calls whose execution
+ *     may overlap (different streams, or different host threads without ordering between
+ *     them) race on it and can corrupt each other's outputs; order them (one stream, or
+ *     events), or use wkv6_prefill with a workspace per stream.
+ */
+wkv_status wkv6_prefill_static(const void *r, const void *k, const void *v, const void *omega,
+                               const float *u, const float *state_in, float *state_out, void *y,
+                               int B, int T, int H, int D, wkv_dtype io, const wkv_ln *ln,
+                               void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *wkv6_status_string(wkv_status s);

@@ -5,7 +5,9 @@ torch tensors into it.  Importing this package does not load the library; the fi
 does, and raises if it was not built.
 """
 from .binding import (WkvError, decode_workspace_bytes, load, new_workspace,
-                      prefill_workspace_bytes, wkv6_decode_step, wkv6_prefill, workspace_status)
+                      prefill_workspace_bytes, wkv6_decode_step, wkv6_prefill, wkv6_prefill_static,
+                      workspace_status)
 
 __all__ = ["WkvError", "decode_workspace_bytes", "load", "new_workspace",
-           "prefill_workspace_bytes", "wkv6_decode_step", "wkv6_prefill", "workspace_status"]
+           "prefill_workspace_bytes", "wkv6_decode_step", "wkv6_prefill", "wkv6_prefill_static",
+           "workspace_status"]

@@ -54,6 +54,8 @@ def load(path: Path | str | None = None):
     L.wkv6_prefill.restype = i
     L.wkv6_prefill_algo.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, sz, vp]
     L.wkv6_prefill_algo.restype = i
+    L.wkv6_prefill_static.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp]
+    L.wkv6_prefill_static.restype = i
     L.wkv6_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
     L.wkv6_decode_step.restype = i
     L.wkv6_workspace_status.argtypes = [vp, vp]
@@ -163,6 +165,44 @@ def wkv6_prefill(r, k, v, omega, u, state_in=None, *, ln=None, algo="auto", y=No
                                  _ptr(workspace), ws_bytes, _stream_ptr(dev, stream))
     del ln_s
     _raise("wkv6_prefill", st)
+    return y, state_out
+
+
+STATIC_SCRATCH_BYTES = 8 << 20   # WKV6_STATIC_SCRATCH_BYTES
+
+
+def wkv6_prefill_static(r, k, v, omega, u, state_in=None, *, ln=None, y=None, state_out=None,
+                        want_state=True, stream=None):
+    """wkv6_prefill without a workspace: the library serves it from its built-in scratch
+    (include/goldwkv.h, wkv6_prefill_static).  The library allocates nothing; this wrapper
+    still allocates y / state_out with torch when they are not given.  Calls that may
+    overlap in time on one device race on the shared scratch."""
+    L = load()
+    if r.dim() != 4:
+        raise ValueError("r must be [B, T, H, D]")
+    B, T, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega)):
+        _check(name, t, dev, dt, (B, T, H, D))
+    _check("u", u, dev, torch.float32, (H, D))
+    if state_in is not None:
+        _check("state_in", state_in, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, T, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, T, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _check("state_out", state_out, dev, torch.float32, (B, H, D, D))
+    ln_s, ln_p = _ln_struct(ln, H, D, dev)
+    with torch.cuda.device(dev):
+        st = L.wkv6_prefill_static(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state_in),
+                                   _ptr(state_out), _ptr(y), B, T, H, D, _io(dt), ln_p,
+                                   _stream_ptr(dev, stream))
+    del ln_s
+    _raise("wkv6_prefill_static", st)
     return y, state_out
 
 
