@@ -56,6 +56,33 @@ def decode_bytes(B, H, D=64, esz=2):
     return B * H * (2 * D * D * 4 + 5 * D * esz) + H * D * 4
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture of each dominant kernel, with the hash of the sources the captured build came
+# from; reported only while the sources still hash to that value (else null).
+CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
+NCU_TRAFFIC = {
+    "prefill": {"sources": ("chunked_fast_sm100.cu", "sm100_ptx.cuh", "common.cuh", "internal.h"),
+                "sha256_16": "4e8cad9ac8f94f62", "bytes": 541151232 + 122149632,
+                "workload": (8, 4096, 32),
+                "profile": "profiles/wkv6_fast_kernel_prefill_B8_T4096_H32_bf16.md"},
+    "decode": {"sources": ("decode.cu", "common.cuh"),
+               "sha256_16": "c68942cec925238b", "bytes": 138428672 + 80250624,
+               "workload": (256, 32),
+               "profile": "profiles/wkv6_decode_kernel_B256_H32_bf16.md"},
+}
+
+
+def ncu_traffic(kind: str, workload: tuple):
+    import hashlib
+    rec = NCU_TRAFFIC[kind]
+    h = hashlib.sha256()
+    for name in rec["sources"]:
+        h.update((CSRC / name).read_bytes())
+    if h.hexdigest()[:16] != rec["sha256_16"] or tuple(workload) != rec["workload"]:
+        return None
+    return rec["bytes"]
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -219,7 +246,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     cfg = PREFILL_CFG if args.batch is None else PREFILL_CFG.with_(B=args.batch)
     B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
-    inp = W.make_prefill_inputs(cfg, dev, seed=cfg.seed + 17 * rank)
+    inp = W.make_prefill_shard(cfg, dev, rank)
     ws = gw.new_workspace(gw.prefill_workspace_bytes(B, T, H, D, cfg.dtype, False, args.algo), dev)
     y = torch.empty_like(inp["r"])
     s_out = torch.empty_like(inp["state0"])
@@ -266,7 +293,10 @@ def run_ours(args, world, rank, local):
     bytes_launch = prefill_bytes(B, T, H, D)
     avg_launch_ms = statistics.mean(launch_ms)
     achieved = bytes_launch / (avg_launch_ms / 1e3) / 1e9
-    launches_per_step = 1  # one prefill kernel per call (no LayerNorm in this workload)
+    # the chunked path launches the fast kernel and the level kernel (which finishes any
+    # sequence handed over to it); the fp32 recurrence is one kernel; no LayerNorm here
+    chunked = algo == "chunked" or (algo == "auto" and cfg.dtype == torch.bfloat16)
+    launches_per_step = 2 if chunked else 1
 
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -279,17 +309,19 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"dp{world} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (537 MB in, 134 MB out per step)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm,
+                     "traffic": ncu_traffic("prefill", (B, T, H)) if chunked else None,
                      "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "algorithmic_bytes_per_launch": bytes_launch,
-                     "kernel": "wkv6 prefill (algo=%s)" % algo},
+                     "kernel": "wkv6 prefill (algo=%s): wkv6_fast_kernel + level kernel, "
+                               "timed together per call" % algo},
         "gpu_launches": launches_per_step * args.steps,
     }
 
     # decode: 100 steps back to back, state in place; GB/s of algorithmic bytes
     if not args.no_decode:
         dcfg = DECODE_CFG
-        dinp = W.make_decode_inputs(dcfg, dev, seed=dcfg.seed + 17 * rank)
+        dinp = W.make_decode_shard(dcfg, dev, rank)
         state = dinp["state0"].clone()
         ybuf = torch.empty_like(dinp["r"][0])
         dsteps = dcfg.steps
@@ -318,8 +350,10 @@ def run_ours(args, world, rank, local):
                                     "D": dcfg.D, "io": "bf16", "state": "fp32 in place",
                                     "l2": "state 134 MB > L2"},
                          "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm,
-                                      "unit": "GB/s", "frac": dgbs / hbm, "traffic": None,
-                                      "algorithmic_bytes_per_launch": dbytes}}
+                                      "unit": "GB/s", "frac": dgbs / hbm,
+                                      "traffic": ncu_traffic("decode", (dcfg.B, dcfg.H)),
+                                      "algorithmic_bytes_per_launch": dbytes},
+                         "gpu_launches": dsteps}
         del dinp, dargs, state
 
     # end to end through the public API with host buffers

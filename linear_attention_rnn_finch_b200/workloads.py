@@ -135,6 +135,27 @@ def make_prefill_inputs(cfg: WkvConfig, device="cpu", *, B=None, T=None, seed=No
     return out
 
 
+def _share_params(out, base):
+    for n in ("u", "gamma", "beta"):
+        if n in base:
+            out[n] = base[n]
+    return out
+
+
+def make_prefill_shard(cfg: WkvConfig, device, rank: int, **kw):
+    """Rank `rank`'s batch in a data-parallel run: its own tokens and initial state (seed
+    cfg.seed + 17 * rank), the layer's parameters u (and LayerNorm gamma, beta) those of
+    rank 0, as every rank holds the same layer."""
+    out = make_prefill_inputs(cfg, device, seed=cfg.seed + 17 * rank, **kw)
+    return _share_params(out, make_prefill_inputs(cfg, device, **kw)) if rank else out
+
+
+def make_decode_shard(cfg: WkvConfig, device, rank: int, **kw):
+    """As make_prefill_shard, for the decode inputs."""
+    out = make_decode_inputs(cfg, device, seed=cfg.seed + 17 * rank, **kw)
+    return _share_params(out, make_decode_inputs(cfg, device, **kw)) if rank else out
+
+
 def make_decode_inputs(cfg: WkvConfig, device="cpu", *, B=None, steps=None, seed=None):
     """Seeded decode inputs: per-step r,k,v,omega [steps, B, H, D], u, initial state."""
     B = cfg.B if B is None else B
