@@ -62,7 +62,7 @@ def decode_bytes(B, H, D=64, esz=2):
 CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "sm100_ptx.cuh", "common.cuh", "internal.h"),
-                "sha256_16": "4e8cad9ac8f94f62", "bytes": 541151232 + 122149632,
+                "sha256_16": "05b71e9b6aaf3768", "bytes": 541236224 + 120360704,
                 "workload": (8, 4096, 32),
                 "profile": "profiles/wkv6_fast_kernel_prefill_B8_T4096_H32_bf16.md"},
     "decode": {"sources": ("decode.cu", "common.cuh"),

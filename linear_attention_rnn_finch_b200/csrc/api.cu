@@ -220,7 +220,7 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
             e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
                                                status, nullptr, nullptr, budget, st);
         } else {
-            e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y_raw, B, T, H,
+            e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H,
                                              status, h_chunk, h_state, budget, st);
             if (e == cudaSuccess)
                 e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,

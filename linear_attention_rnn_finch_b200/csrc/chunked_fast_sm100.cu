@@ -16,24 +16,32 @@
 // chunk and the chunk index are handed (through the workspace) to the level-factorised
 // kernel, which finishes the sequence.  Nothing is clamped.
 //
-// Precision.  Every operand that is rounded to bf16 -- Rt, Kh, S and A -- is split into
-// hi = bf16(x) and lo = bf16(x - hi).  The lo parts cost no extra MMA instructions: hi and
-// lo rows are stacked into M = 128 (rows 0-7 of every 16-row group hold hi parts of 8
-// tokens, rows 8-15 the lo parts of the same tokens), and a 16x256b TMEM load hands each
-// thread the hi and lo element of the same (token, column) in registers {0,1} / {2,3}, so
-// the combination is one add in registers.  With all parts split the arithmetic is as
-// accurate as fp32; the only bf16 rounding left is that of the output y.
+// Precision.  Rt, S and A are split into hi = bf16(x) and lo = bf16(x - hi), and Kh is
+// split for the state increment.  The lo parts cost no extra MMA instructions: hi and lo
+// rows are stacked into M = 128 (rows 0-7 of every 16-row group hold hi parts of 8 tokens,
+// rows 8-15 the lo parts of the same tokens), and a 16x256b TMEM load hands each thread the
+// hi and lo element of the same (token, column) in registers {0,1} / {2,3}, so the
+// combination is one add in registers.
 //
-// Per chunk three MMA groups (K = 64, four K16 instructions per chain):
-//   G1: [Rt_hi ; Rt_lo] (M=128) x [S_hi^T ; Kh_hi]^T, then x [S_lo^T ; Kh_lo]^T accumulated
-//       into the same columns (N=128) -> D1: columns 0..63 readout Rt . S, columns 64..127
-//       intra-chunk scores Rt . Kh (hi and lo parts of S and Kh summed by the MMA)
-//   GU: V^T (M=64) x [Kh_hi | Kh_lo] (N=128) -> DU = (Kh^T V)^T, the state increment
-//   GA: [A_hi ; A_lo] (M=128) x V (N=64) -> DA, the intra-chunk output A . V
+// The recurrence and the output are separate pipelines.  The state only needs
+//   GU(n): V^T (M=64) x [Kh_hi | Kh_lo] (N=128) -> DU = (Kh^T V)^T, the increment of chunk n,
+// which depends on the chunk's own operands, not on S; the epilogue folds it into the fp32
+// state it keeps in registers.  The output of chunk n needs three more products:
+//   SC(n): [Rt_hi ; Rt_lo] (M=128) x Kh_hi^T (N=64)           intra-chunk scores
+//   RO(n): [Rt_hi ; Rt_lo] x [S_hi^T ; S_lo^T] (N=128)        readout of S_{n-1} -> Y
+//   GA(n): [A_hi ; A_lo] x V (N=64), accumulated into Y        A = masked scores + bonus
+// None of them feeds back into S, so they trail the state by a chunk without stalling it.
 //
-// Warp roles (448 threads): warp 0 TMA producer (3-stage ring of r, k, v, omega tiles);
-// warp 1 MMA issuer (and TMEM owner); warps 2-5 prep (log-decay scan, Rt / Kh operands,
-// bonus, gamma, range test); warps 6-13 epilogue (state update, assembly of A, output).
+// Warp roles (608 threads):
+//   warp 0, one thread: TMA loads (3-stage rings: r/k/omega released by prep, v by GU and GA);
+//     TMEM owner.
+//   warp 1, one thread: GU(n), SC(n) in chunk order.  warp 2, one thread: RO(n), GA(n).  Each
+//     blocks on the one barrier it needs next; two issuers let the state stream run ahead
+//     of the output stream.  Buffers read by both are released by one commit from each.
+//   warps 3-10 (prep): 8 tokens each of the same chunk -- log-decay prefix, Rt / Kh hi/lo
+//     operands, bonus, gamma, range test.
+//   warps 11-18 (epilogue): per chunk n, state(n) = gamma (S + DU) and S_n hi/lo for RO(n+1);
+//     the output of chunk n-1 (Y -> y); A(n) for GA(n).
 // Handshakes are mbarriers; every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -49,32 +57,40 @@ namespace {
 constexpr int C = 64;
 constexpr int kStages = 3;
 constexpr int kTile = 64 * 64 * 2;            // 64 rows x 128 B
-constexpr int kThreads = 448;
-constexpr int kPrepWarp0 = 2, kEpiWarp0 = 6;
-constexpr int kEpiThreads = 256;
+constexpr int kPrepWarps = 8, kEpiWarps = 8;
+constexpr int kTmaWarp = 0, kMmaUWarp = 1, kMmaYWarp = 2;
+constexpr int kPrepWarp0 = 3, kEpiWarp0 = kPrepWarp0 + kPrepWarps;
+constexpr int kPrepThreads = 32 * kPrepWarps, kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 32 * kPrepWarp0 + kPrepThreads + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t COL_D1 = 0, COL_DU = 128, COL_DA = 256;
+// DU: 2 buffers x 128 columns (M=64); SC: 2 x 64 (M=128); Y: 128 (M=128)
+constexpr uint32_t COL_DU = 0, COL_SC = 256, COL_Y = 384;
 // log2 of the largest factor exp(-L_s) allowed: ln range 60 -> log2 range 86.56
 constexpr float kMaxLog2Range = 86.5617f;
 constexpr float kLog2e = 1.4426950408889634f;
+// named barriers (id 0 is __syncthreads)
+constexpr int kBarPrep = 1, kBarEpi = 2;
 
-constexpr uint32_t IDESC_G1 = ptx::idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t IDESC_GU = ptx::idesc_bf16(64, 128, 1, 1);
+constexpr uint32_t IDESC_SC = ptx::idesc_bf16(128, 64, 0, 0);
+constexpr uint32_t IDESC_RO = ptx::idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t IDESC_GA = ptx::idesc_bf16(128, 64, 0, 1);
 
 struct __align__(1024) Smem {
-    uint8_t in[kStages][4][kTile];   // r, k, v, omega tiles (TMA, 128B swizzle)
-    uint8_t bblk[2][4][kTile];       // per parity: S_hi^T, Kh_hi, S_lo^T, Kh_lo (G1 operand B)
-    uint8_t rt[2][2 * kTile];        // per parity: Rt hi/lo, 128 stacked rows (G1 operand A)
-    uint8_t at[2 * kTile];           // A hi/lo, 128 stacked rows (GA operand A)
-    uint8_t ystage[kTile];           // y tile for the TMA store
-    float qtot[4][64];               // prep: per-quarter sums of log2 w
+    uint8_t rkw[kStages][3][kTile];  // r, k, omega tiles (TMA, 128B swizzle)
+    uint8_t vt[kStages][kTile];      // v tiles
+    uint8_t rt[2][2 * kTile];        // per parity: Rt hi/lo, 128 stacked rows
+    uint8_t kh[2][2 * kTile];        // per parity: Kh_hi tile, then Kh_lo tile
+    uint8_t sb[2][2 * kTile];        // S_hi^T tile, then S_lo^T tile; sb[m & 1] feeds RO(m)
+    uint8_t at[2 * kTile];           // A hi/lo, 128 stacked rows
+    float qtot[2][kPrepWarps][64];   // prep: per-warp sums of log2 w
     float gamma[2][64];
     float bonus[2][64];
     int unsafe[2];
-    uint64_t full[kStages], empty[kStages];
-    uint64_t prep_done[2], op_free[2];
-    uint64_t g1_done, ga_done, epi_mid, epi_end, s_init;
+    uint64_t full_rkw[kStages], empty_rkw[kStages], full_v[kStages], empty_v[kStages];
+    uint64_t prep_done[2], op_free[2], ep_free[2];
+    uint64_t gu_done[2], sc_done[2], du_free[2], sc_free[2], s_ready[2], s_free[2];
+    uint64_t a_ready, ya_done, y_free;
     uint32_t tmem_base;
     int abort;
     int stop_at;                     // chunk at which this (b,h) leaves for the level kernel
@@ -125,6 +141,17 @@ __device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, uint32_t (&v)[16]) {
           "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
 }
+// the (hi row + lo row) pair k of a 16x256b load: registers 4k, 4k+1 plus 4k+2, 4k+3
+__device__ __forceinline__ float2 rows_sum(const uint32_t (&v)[16], int k) {
+    return __fadd2_rn(make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1])),
+                      make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+}
+__device__ __forceinline__ float2 lo_pair(const uint32_t (&v)[16], int k) {
+    return make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]));
+}
+__device__ __forceinline__ float2 hi_pair(const uint32_t (&v)[16], int k) {
+    return make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+}
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -150,11 +177,92 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 __device__ __forceinline__ int ld_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
 
+// Bounded wait that gives up early once the CTA has aborted; on expiry it aborts the CTA.
+// Returns false if the caller should treat its data as invalid (abort).
+// With `or_stop`, also gives up (without aborting) once this (b,h) has been handed over.
+__device__ __forceinline__ bool wait_soft(Smem& s, uint64_t* bar, uint32_t parity, long long budget,
+                                          bool or_stop = false) {
+    if (ptx::mbar_test_wait(bar, parity)) return true;
+    if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
+    if (budget <= 0) {
+        s.abort = 1;
+        return false;
+    }
+    const long long t0 = clock64();
+    for (;;) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ld_volatile(&s.abort)) return false;
+        if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
+        if (clock64() - t0 > budget) {
+            s.abort = 1;
+            return false;
+        }
+    }
+}
+
+// Output of chunk m: y = Y[:, 0:64] + Y[:, 64:128] (hi and lo rows each), stored as bf16 (or
+// fp32 rows to y_raw).  Frees the Y accumulator for RO(m+1).
+__device__ __forceinline__ void output_chunk(Smem& s, int m, uint32_t tmem, uint32_t lane_h0,
+                                             uint32_t lane_h1, int ch, int cbase, int r0, int r1,
+                                             int b, int h, int T, int H, __nv_bfloat16* y,
+                                             float* y_raw, long long budget) {
+    wait_soft(s, &s.ya_done, (uint32_t)(m & 1), budget);
+    ptx::tc_fence_after();
+    float2 Y0[4], Y1[4];
+    {
+        uint32_t a[16], c[16];
+        tmem_ld16x4(tmem + lane_h0 + COL_Y + 32 * ch, a);
+        tmem_ld16x4(tmem + lane_h0 + COL_Y + 64 + 32 * ch, c);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Y0[k] = __fadd2_rn(rows_sum(a, k), rows_sum(c, k));
+    }
+    {
+        uint32_t a[16], c[16];
+        tmem_ld16x4(tmem + lane_h1 + COL_Y + 32 * ch, a);
+        tmem_ld16x4(tmem + lane_h1 + COL_Y + 64 + 32 * ch, c);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Y1[k] = __fadd2_rn(rows_sum(a, k), rows_sum(c, k));
+    }
+    ptx::tc_fence_before();
+    mbar_arrive(&s.y_free);
+    const int valid = min(C, T - m * C);
+    const size_t row0 = ((size_t)b * T + (size_t)m * C + r0) * H + h;
+    const size_t row1 = ((size_t)b * T + (size_t)m * C + r1) * H + h;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int j = cbase + 8 * k;
+        if (y_raw != nullptr) {
+            if (r0 < valid) *reinterpret_cast<float2*>(y_raw + row0 * 64 + j) = Y0[k];
+            if (r1 < valid) *reinterpret_cast<float2*>(y_raw + row1 * 64 + j) = Y1[k];
+        } else {
+            if (r0 < valid) *reinterpret_cast<uint32_t*>(y + row0 * 64 + j) = pack2(Y0[k].x, Y0[k].y);
+            if (r1 < valid) *reinterpret_cast<uint32_t*>(y + row1 * 64 + j) = pack2(Y1[k].x, Y1[k].y);
+        }
+    }
+}
+
+// S_hi^T at tile, S_lo^T at tile + kTile: this thread's rows j = r0, r1, columns i of its pairs
+__device__ __forceinline__ void store_state(uint8_t* tile, const float2 (&S0)[4], const float2 (&S1)[4],
+                                            int r0, int r1, int ch, uint32_t cb) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t hi, lo;
+        split2(S0[k], hi, lo);
+        sts32(tile, sw_off(r0, 4 * ch + k) + cb, hi);
+        sts32(tile + kTile, sw_off(r0, 4 * ch + k) + cb, lo);
+        split2(S1[k], hi, lo);
+        sts32(tile, sw_off(r1, 4 * ch + k) + cb, hi);
+        sts32(tile + kTile, sw_off(r1, 4 * ch + k) + cb, lo);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
-                 const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
-                 const float* s_in, float* s_out, float* __restrict__ y_raw, int T, int H,
+                 const float* __restrict__ u, const float* s_in, float* s_out,
+                 __nv_bfloat16* __restrict__ y, float* __restrict__ y_raw, int T, int H,
                  int* status, int* handoff_chunk, float* handoff_state, long long budget,
                  long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
@@ -166,121 +274,142 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
-            ptx::mbar_init(&s.full[i], 1);
-            ptx::mbar_init(&s.empty[i], 1);
+            ptx::mbar_init(&s.full_rkw[i], 1);
+            ptx::mbar_init(&s.empty_rkw[i], kPrepThreads);
+            ptx::mbar_init(&s.full_v[i], 1);
+            ptx::mbar_init(&s.empty_v[i], 2);      // GU (warp 1) and GA (warp 2)
         }
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&s.prep_done[i], 128);
-            ptx::mbar_init(&s.op_free[i], 1);
+            ptx::mbar_init(&s.prep_done[i], kPrepThreads);
+            ptx::mbar_init(&s.op_free[i], 2);      // GU/SC (warp 1) and RO (warp 2)
+            ptx::mbar_init(&s.ep_free[i], kEpiThreads);
+            ptx::mbar_init(&s.gu_done[i], 1);
+            ptx::mbar_init(&s.sc_done[i], 1);
+            ptx::mbar_init(&s.du_free[i], kEpiThreads);
+            ptx::mbar_init(&s.sc_free[i], kEpiThreads);
+            ptx::mbar_init(&s.s_ready[i], kEpiThreads);
+            ptx::mbar_init(&s.s_free[i], 1);
         }
-        ptx::mbar_init(&s.g1_done, 1);
-        ptx::mbar_init(&s.ga_done, 1);
-        ptx::mbar_init(&s.epi_mid, kEpiThreads);
-        ptx::mbar_init(&s.epi_end, kEpiThreads);
-        ptx::mbar_init(&s.s_init, kEpiThreads);
+        ptx::mbar_init(&s.a_ready, kEpiThreads);
+        ptx::mbar_init(&s.ya_done, 1);
+        ptx::mbar_init(&s.y_free, kEpiThreads);
         ptx::fence_mbar_init();
         s.abort = 0;
         s.stop_at = -1;
     }
-    if (warp == 1) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
+    if (warp == kTmaWarp) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = s.tmem_base;
 
-    if (warp == 0) {
+    if (warp == kTmaWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ptx::prefetch_tensormap(&tm_r);
             ptx::prefetch_tensormap(&tm_k);
             ptx::prefetch_tensormap(&tm_v);
             ptx::prefetch_tensormap(&tm_w);
-            int last[kStages] = {-1, -1, -1};
+            int last_rkw[kStages] = {-1, -1, -1}, last_v[kStages] = {-1, -1, -1};
             for (int n = 0; n < NC; ++n) {
                 const int st = n % kStages;
-                if (n >= kStages) {
-                    // wait for the stage to be released; give up if this head stopped
-                    const uint32_t par = (uint32_t)(((n - kStages) / kStages) & 1);
-                    bool ok = false;
-                    const long long t0 = clock64();
-                    for (;;) {
-                        if (ptx::mbar_try_wait(&s.empty[st], par)) { ok = true; break; }
-                        if (ld_volatile(&s.stop_at) >= 0 || ld_volatile(&s.abort)) break;
-                        if (clock64() - t0 > budget) { s.abort = 1; break; }
-                    }
-                    if (!ok) break;
-                }
-                ptx::mbar_arrive_expect_tx(&s.full[st], 4 * kTile);
-                const int t0 = n * C;
-                ptx::tma_load_4d(s.in[st][0], &tm_r, &s.full[st], 0, h, t0, b);
-                ptx::tma_load_4d(s.in[st][1], &tm_k, &s.full[st], 0, h, t0, b);
-                ptx::tma_load_4d(s.in[st][2], &tm_v, &s.full[st], 0, h, t0, b);
-                ptx::tma_load_4d(s.in[st][3], &tm_w, &s.full[st], 0, h, t0, b);
-                last[st] = n;
+                const uint32_t par = (uint32_t)((n / kStages - 1) & 1);   // release of chunk n-3
+                if (n >= kStages && !wait_soft(s, &s.empty_rkw[st], par, budget, true)) break;
+                ptx::mbar_arrive_expect_tx(&s.full_rkw[st], 3 * kTile);
+                ptx::tma_load_4d(s.rkw[st][0], &tm_r, &s.full_rkw[st], 0, h, n * C, b);
+                ptx::tma_load_4d(s.rkw[st][1], &tm_k, &s.full_rkw[st], 0, h, n * C, b);
+                ptx::tma_load_4d(s.rkw[st][2], &tm_w, &s.full_rkw[st], 0, h, n * C, b);
+                last_rkw[st] = n;
+                if (n >= kStages && !wait_soft(s, &s.empty_v[st], par, budget, true)) break;
+                ptx::mbar_arrive_expect_tx(&s.full_v[st], kTile);
+                ptx::tma_load_4d(s.vt[st], &tm_v, &s.full_v[st], 0, h, n * C, b);
+                last_v[st] = n;
             }
             // every issued copy must land before the CTA may exit
-            for (int st = 0; st < kStages; ++st)
-                if (last[st] >= 0)
-                    ptx::mbar_wait(&s.full[st], (uint32_t)((last[st] / kStages) & 1), drain_budget);
+            for (int st = 0; st < kStages; ++st) {
+                if (last_rkw[st] >= 0)
+                    ptx::mbar_wait(&s.full_rkw[st], (uint32_t)((last_rkw[st] / kStages) & 1), drain_budget);
+                if (last_v[st] >= 0)
+                    ptx::mbar_wait(&s.full_v[st], (uint32_t)((last_v[st] / kStages) & 1), drain_budget);
+            }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kMmaUWarp) {
+        // ------------------------------------------------------------ GU, SC issue
         if (lane == 0) {
-            int last_g1 = -1, last_ga = -1;
+            int last = -1;
             for (int n = 0; n < NC; ++n) {
                 const int pb = n & 1, st = n % kStages;
-                if (!ptx::mbar_wait(&s.prep_done[pb], (uint32_t)((n >> 1) & 1), budget)) { s.abort = 1; break; }
-                if (s.unsafe[pb]) {          // hand this (b,h) to the level kernel from chunk n
+                if (!wait_soft(s, &s.prep_done[pb], (uint32_t)((n >> 1) & 1), budget)) break;
+                if (ld_volatile(&s.unsafe[pb])) {   // hand this (b,h) to the level kernel
                     s.stop_at = n;
-                    mbar_arrive(&s.g1_done);  // wakes the epilogue, which saves the state
+                    mbar_arrive(&s.gu_done[pb]);    // wakes the epilogue, which hands off
                     break;
                 }
-                // D1 / DU free and S_n written: the epilogue finished state + assembly of n-1
-                // (for n = 0: the initial state is in shared memory)
-                if (n == 0 && !ptx::mbar_wait(&s.s_init, 0, budget)) { s.abort = 1; break; }
-                if (n > 0 && !ptx::mbar_wait(&s.epi_mid, (uint32_t)((n - 1) & 1), budget)) { s.abort = 1; break; }
+                if (!wait_soft(s, &s.full_v[st], (uint32_t)((n / kStages) & 1), budget)) break;
+                if (n >= 2 && !wait_soft(s, &s.du_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget)) break;
+                if (n >= 2 && !wait_soft(s, &s.sc_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget)) break;
                 ptx::tc_fence_after();
-                const uint32_t v_tile = ptx::smem_addr(s.in[st][2]);
-                const uint32_t bhi = ptx::smem_addr(s.bblk[pb][0]);   // [S_hi^T ; Kh_hi]
-                const uint32_t blo = ptx::smem_addr(s.bblk[pb][2]);   // [S_lo^T ; Kh_lo]
-                const uint32_t kh = ptx::smem_addr(s.bblk[pb][1]);
+                const uint32_t v_tile = ptx::smem_addr(s.vt[st]);
+                const uint32_t kh = ptx::smem_addr(s.kh[pb]);
                 const uint32_t rt = ptx::smem_addr(s.rt[pb]);
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // GU: V^T x [Kh_hi | Kh_lo] (N atoms 16 KB apart)
-                    ptx::mma_bf16(tmem + COL_DU, ptx::desc_sw128(v_tile + 2048 * kq, 1024),
-                                  ptx::desc_sw128(kh + 2048 * kq, 2 * kTile), IDESC_GU, kq > 0);
+                for (int kq = 0; kq < 4; ++kq)   // DU = V^T x [Kh_hi | Kh_lo]
+                    ptx::mma_bf16(tmem + COL_DU + 128 * pb, ptx::desc_sw128(v_tile + 2048 * kq, 1024),
+                                  ptx::desc_sw128(kh + 2048 * kq, kTile), IDESC_GU, kq > 0);
+                ptx::mma_commit(&s.gu_done[pb]);
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // G1: [Rt] x [S_hi^T ; Kh_hi]
-                    ptx::mma_bf16(tmem + COL_D1, ptx::desc_kmajor(rt + 32 * kq),
-                                  ptx::desc_kmajor(bhi + 32 * kq), IDESC_G1, kq > 0);
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   //   + [Rt] x [S_lo^T ; Kh_lo]
-                    ptx::mma_bf16(tmem + COL_D1, ptx::desc_kmajor(rt + 32 * kq),
-                                  ptx::desc_kmajor(blo + 32 * kq), IDESC_G1, 1);
-                ptx::mma_commit(&s.g1_done);
-                last_g1 = n;
-                // GA needs A (assembly of n) and DA free (output of n-1 read)
-                if (!ptx::mbar_wait(&s.epi_mid, (uint32_t)(n & 1), budget)) { s.abort = 1; break; }
-                if (n > 0 && !ptx::mbar_wait(&s.epi_end, (uint32_t)((n - 1) & 1), budget)) { s.abort = 1; break; }
+                for (int kq = 0; kq < 4; ++kq)   // SC = [Rt] x Kh_hi^T
+                    ptx::mma_bf16(tmem + COL_SC + 64 * pb, ptx::desc_kmajor(rt + 32 * kq),
+                                  ptx::desc_kmajor(kh + 32 * kq), IDESC_SC, kq > 0);
+                ptx::mma_commit(&s.sc_done[pb]);
+                ptx::mma_commit(&s.op_free[pb]);
+                ptx::mma_commit(&s.empty_v[st]);
+                last = n;
+            }
+            // drain: our tensor-core work must be complete before TMEM is freed
+            if (last >= 0) ptx::mbar_wait(&s.sc_done[last & 1], (uint32_t)((last >> 1) & 1), drain_budget);
+        }
+    } else if (warp == kMmaYWarp) {
+        // ------------------------------------------------------------ RO, GA issue
+        if (lane == 0) {
+            uint64_t* last_bar = nullptr;   // the latest commit covers all earlier MMAs
+            uint32_t last_par = 0;
+            for (int n = 0; n < NC; ++n) {
+                const int pb = n & 1, st = n % kStages;
+                if (!wait_soft(s, &s.prep_done[pb], (uint32_t)((n >> 1) & 1), budget)) break;
+                if (ld_volatile(&s.unsafe[pb])) break;   // chunks before n are complete
+                if (!wait_soft(s, &s.s_ready[pb], (uint32_t)((n >> 1) & 1), budget)) break;
+                if (n >= 1 && !wait_soft(s, &s.y_free, (uint32_t)((n - 1) & 1), budget)) break;
                 ptx::tc_fence_after();
+                const uint32_t rt = ptx::smem_addr(s.rt[pb]);
+                const uint32_t sbuf = ptx::smem_addr(s.sb[pb]);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)   // Y = [Rt] x [S_hi^T ; S_lo^T]
+                    ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(rt + 32 * kq),
+                                  ptx::desc_kmajor(sbuf + 32 * kq), IDESC_RO, kq > 0);
+                ptx::mma_commit(&s.s_free[pb]);    // sb[pb] read
+                ptx::mma_commit(&s.op_free[pb]);   // Rt of parity pb read
+                last_bar = &s.s_free[pb];
+                last_par = (uint32_t)((n >> 1) & 1);
+                if (!wait_soft(s, &s.a_ready, (uint32_t)(n & 1), budget)) break;
+                ptx::tc_fence_after();
+                const uint32_t v_tile = ptx::smem_addr(s.vt[st]);
                 const uint32_t at = ptx::smem_addr(s.at);
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)
-                    ptx::mma_bf16(tmem + COL_DA, ptx::desc_kmajor(at + 32 * kq),
-                                  ptx::desc_mnmajor(v_tile + 2048 * kq), IDESC_GA, kq > 0);
-                ptx::mma_commit(&s.ga_done);
-                ptx::mma_commit(&s.empty[st]);     // stage read by GU / GA (prep read it before)
-                ptx::mma_commit(&s.op_free[pb]);   // Rt / Kh / gamma / bonus of parity pb
-                last_ga = n;
+                for (int kq = 0; kq < 4; ++kq)   // Y[:, 0:64] += [A] x V
+                    ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(at + 32 * kq),
+                                  ptx::desc_mnmajor(v_tile + 2048 * kq), IDESC_GA, 1);
+                ptx::mma_commit(&s.ya_done);
+                ptx::mma_commit(&s.empty_v[st]);
+                last_bar = &s.ya_done;
+                last_par = (uint32_t)(n & 1);
             }
-            // drain: our own tensor-core work must be complete before TMEM is freed
-            if (last_g1 >= 0) ptx::mbar_wait(&s.g1_done, (uint32_t)(last_g1 & 1), drain_budget);
-            if (last_ga >= 0) ptx::mbar_wait(&s.ga_done, (uint32_t)(last_ga & 1), drain_budget);
+            if (last_bar != nullptr) ptx::mbar_wait(last_bar, last_par, drain_budget);
         }
     } else if (warp < kEpiWarp0) {
-        // ------------------------------------------------------------ prep (4 warps)
-        // lane = channel pair (2l, 2l+1), warp = token quarter (16 tokens); log2 units
-        const int qw = warp - kPrepWarp0;
+        // ------------------------------------------------------------ prep (8 warps)
+        // warp g: tokens 8g .. 8g+7 of every chunk; lane = channel pair (2l, 2l+1); log2 units
+        const int g = warp - kPrepWarp0;
         const int c0 = 2 * lane;
         const float2 uu = make_float2(u[h * 64 + c0], u[h * 64 + c0 + 1]);
         const int chunk = lane >> 2;          // 16-byte chunk holding channels c0, c0+1
@@ -290,124 +419,127 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         for (int n = 0; n < NC; ++n) {
             const int pb = n & 1, st = n % kStages;
             const int valid = min(C, T - n * C);
-            bool bad = !ptx::mbar_wait(&s.full[st], (uint32_t)((n / kStages) & 1), budget);
-            if (n >= 2) bad |= !ptx::mbar_wait(&s.op_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget);
-            if (bad) s.abort = 1;
-            if (named_bar_any(1, 128, bad || ld_volatile(&s.abort))) break;   // uniform over prep
-            const uint8_t* r_tile = s.in[st][0];
-            const uint8_t* k_tile = s.in[st][1];
-            const uint8_t* w_tile = s.in[st][3];
+            bool ok_wait = wait_soft(s, &s.full_rkw[st], (uint32_t)((n / kStages) & 1), budget);
+            if (n >= 2) {
+                ok_wait = ok_wait && wait_soft(s, &s.op_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget);
+                ok_wait = ok_wait && wait_soft(s, &s.ep_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget);
+            }
+            if (named_bar_any(kBarPrep, kPrepThreads, !ok_wait || ld_volatile(&s.abort))) break;
+            const uint8_t* r_tile = s.rkw[st][0];
+            const uint8_t* k_tile = s.rkw[st][1];
+            const uint8_t* w_tile = s.rkw[st][2];
             // pass 1: local inclusive prefix of log2 w = -exp(omega) log2(e)
-            float2 L[16];
+            float2 L[8];
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const int t = 16 * qw + p;
+            for (int p = 0; p < 8; ++p) {
+                const int t = 8 * g + p;
                 const float2 om = __fmul2_rn(unpack2(lds32(w_tile, sw_off(t, chunk) + cbyte)), l2e);
                 float2 e = make_float2(fast_exp2(om.x), fast_exp2(om.y));
                 if (t >= valid) e = make_float2(0.f, 0.f);
                 acc = __ffma2_rn(e, nl2e, acc);
                 L[p] = acc;
             }
-            s.qtot[qw][c0] = acc.x;
-            s.qtot[qw][c0 + 1] = acc.y;
-            named_bar(1, 128);
+            *reinterpret_cast<float2*>(&s.qtot[pb][g][c0]) = acc;
+            named_bar(kBarPrep, kPrepThreads);
             float2 off = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float2 qv = make_float2(s.qtot[w][c0], s.qtot[w][c0 + 1]);
-                if (w < qw) off = __fadd2_rn(off, qv);
+            for (int w = 0; w < kPrepWarps; ++w) {
+                const float2 qv = *reinterpret_cast<const float2*>(&s.qtot[pb][w][c0]);
+                if (w < g) off = __fadd2_rn(off, qv);
                 tot = __fadd2_rn(tot, qv);
             }
+            // every warp sees the same totals, so all take the same branch
             const bool ok = __all_sync(0xffffffffu, (tot.x >= -kMaxLog2Range) && (tot.y >= -kMaxLog2Range));
             if (!ok) {
-                if (qw == 0 && lane == 0) s.unsafe[pb] = 1;
-                named_bar(1, 128);           // qtot is reused by the next chunk
+                if (g == 0 && lane == 0) s.unsafe[pb] = 1;
                 mbar_arrive(&s.prep_done[pb]);
                 break;                        // this (b,h) continues in the level kernel
             }
             // pass 2: Rt = r 2^(L_{t-1}), Kh = k 2^(-L_t) as bf16 hi / lo; bonus partials
-            uint8_t* rt = s.rt[pb];
-            uint8_t* kh_hi = s.bblk[pb][1];
-            uint8_t* kh_lo = s.bblk[pb][3];
-            float bon[16];
-            float2 fr = make_float2(fast_exp2(off.x), fast_exp2(off.y));   // 2^(L_{t-1})
+            uint32_t rw[8], kw[8];
 #pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const int t = 16 * qw + p;
-                const uint32_t o = sw_off(t, chunk) + cbyte;
-                const float2 rr = unpack2(lds32(r_tile, o));
-                const float2 kk = unpack2(lds32(k_tile, o));
+            for (int p = 0; p < 8; ++p) {
+                const uint32_t o = sw_off(8 * g + p, chunk) + cbyte;
+                rw[p] = lds32(r_tile, o);
+                kw[p] = lds32(k_tile, o);
+            }
+            mbar_arrive(&s.empty_rkw[st]);   // r, k, omega of this stage read
+            uint8_t* rt = s.rt[pb];
+            uint8_t* kh_hi = s.kh[pb];
+            uint8_t* kh_lo = s.kh[pb] + kTile;
+            // all exponentials first (independent of each other), then products and stores
+            float2 fr[8], fk[8];   // 2^(L_{t-1}), 2^(-L_t)
+            fr[0] = make_float2(fast_exp2(off.x), fast_exp2(off.y));
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
                 const float2 li = __fadd2_rn(off, L[p]);
-                const float2 fk = make_float2(fast_exp2(-li.x), fast_exp2(-li.y));
+                fk[p] = make_float2(fast_exp2(-li.x), fast_exp2(-li.y));
+                if (p < 7) fr[p + 1] = make_float2(fast_exp2(li.x), fast_exp2(li.y));
+            }
+            float bon[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const int t = 8 * g + p;
+                const uint32_t o = sw_off(t, chunk) + cbyte;
+                const float2 rr = unpack2(rw[p]);
+                const float2 kk = unpack2(kw[p]);
                 uint32_t hi, lo;
-                split2(__fmul2_rn(rr, fr), hi, lo);
+                split2(__fmul2_rn(rr, fr[p]), hi, lo);
                 const int hr = hi_row(t);
                 const uint32_t cb = (uint32_t)(chunk ^ (t & 7)) << 4;
                 sts32(rt, (uint32_t)hr * 128 + cb + cbyte, hi);
                 sts32(rt, (uint32_t)(hr + 8) * 128 + cb + cbyte, lo);
-                split2(__fmul2_rn(kk, fk), hi, lo);
+                split2(__fmul2_rn(kk, fk[p]), hi, lo);
                 sts32(kh_hi, o, hi);
                 sts32(kh_lo, o, lo);
                 const float2 ru = __fmul2_rn(rr, uu);
                 bon[p] = fmaf(ru.x, kk.x, ru.y * kk.y);
-                if (p < 15) fr = make_float2(fast_exp2(li.x), fast_exp2(li.y));
             }
-            // bonus: reduce the 16 per-token partials over the 32 lanes (reduce-scatter)
+            // bonus: reduce the 8 per-token partials over the 32 lanes (reduce-scatter)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const bool up = lane & 16;
-                const float send = up ? bon[i] : bon[i + 8];
-                const float keep = up ? bon[i + 8] : bon[i];
+                const float send = up ? bon[i] : bon[i + 4];
+                const float keep = up ? bon[i + 4] : bon[i];
                 bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const bool up = lane & 8;
-                const float send = up ? bon[i] : bon[i + 4];
-                const float keep = up ? bon[i + 4] : bon[i];
-                bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-            }
-#pragma unroll
             for (int i = 0; i < 2; ++i) {
-                const bool up = lane & 4;
+                const bool up = lane & 8;
                 const float send = up ? bon[i] : bon[i + 2];
                 const float keep = up ? bon[i + 2] : bon[i];
-                bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
             }
             {
-                const bool up = lane & 2;
+                const bool up = lane & 4;
                 const float send = up ? bon[0] : bon[1];
                 const float keep = up ? bon[1] : bon[0];
-                bon[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                bon[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
             }
+            bon[0] += __shfl_xor_sync(0xffffffffu, bon[0], 2);
             bon[0] += __shfl_xor_sync(0xffffffffu, bon[0], 1);
-            if ((lane & 1) == 0) {
-                const int p = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-                              ((lane >> 1) & 1);
-                s.bonus[pb][16 * qw + p] = bon[0];
+            if ((lane & 3) == 0) {
+                const int p = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+                s.bonus[pb][8 * g + p] = bon[0];
             }
-            if (qw == 0) {
-                s.gamma[pb][c0] = fast_exp2(tot.x);
-                s.gamma[pb][c0 + 1] = fast_exp2(tot.y);
+            if (g == 0) {
+                *reinterpret_cast<float2*>(&s.gamma[pb][c0]) = make_float2(fast_exp2(tot.x), fast_exp2(tot.y));
                 if (lane == 0) s.unsafe[pb] = 0;
             }
             ptx::fence_proxy_async_smem();
-            named_bar(1, 128);               // qtot reads done before the next chunk writes it
             mbar_arrive(&s.prep_done[pb]);
         }
     } else {
         // ------------------------------------------------------------ epilogue (8 warps)
-        // warp (q, ch): TMEM sub-partition q, columns 32ch .. 32ch+31 of each 64-wide block.
-        // Thread: token / state rows r0 = 16q + l/4 and r1 = r0 + 8; column pairs
-        // cbase + 8k + {0,1}, k = 0..3.
+        // warp (q, ch): TMEM sub-partition q = warp % 4, columns 32ch .. 32ch+31 of each
+        // 64-wide block.  Thread: token / state rows r0 = 16q + l/4 and r1 = r0 + 8; column
+        // pairs cbase + 8k + {0,1}, k = 0..3.
         const int q = warp & 3;
         const int ch = (warp - kEpiWarp0) >> 2;
-        const int et = tid - kEpiWarp0 * 32;  // 0 .. 255
         const int r0 = 16 * q + (lane >> 2), r1 = r0 + 8;
         const int cbase = 32 * ch + 2 * (lane & 3);
         const uint32_t cb = (uint32_t)(lane & 3) * 4;
-        const uint32_t lane_m64 = (uint32_t)(32 * q) << 16;
         const uint32_t lane_h0 = (uint32_t)(32 * q) << 16, lane_h1 = (uint32_t)(32 * q + 16) << 16;
         // A block of this warp: rows 16q..16q+15, columns 32ch..32ch+31
         const bool a_zero = 16 * q + 15 < 32 * ch;      // entirely above the diagonal
@@ -423,19 +555,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 S0[k] = src ? make_float2(src[i * 64 + r0], src[(i + 1) * 64 + r0]) : make_float2(0.f, 0.f);
                 S1[k] = src ? make_float2(src[i * 64 + r1], src[(i + 1) * 64 + r1]) : make_float2(0.f, 0.f);
             }
-            // S_0 into parity 0: S_hi^T (tile 0) / S_lo^T (tile 2), rows j, K index i
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                uint32_t hi, lo;
-                split2(S0[k], hi, lo);
-                sts32(s.bblk[0][0], sw_off(r0, 4 * ch + k) + cb, hi);
-                sts32(s.bblk[0][2], sw_off(r0, 4 * ch + k) + cb, lo);
-                split2(S1[k], hi, lo);
-                sts32(s.bblk[0][0], sw_off(r1, 4 * ch + k) + cb, hi);
-                sts32(s.bblk[0][2], sw_off(r1, 4 * ch + k) + cb, lo);
-            }
-            // blocks of A that are always zero are written once here
-            if (a_zero) {
+            store_state(s.sb[0], S0, S1, r0, r1, ch, cb);   // S entering chunk 0, read by RO(0)
+            if (a_zero) {                     // blocks of A that are always zero: once, here
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     sts32(s.at, sw_off(hr0, 4 * ch + k) + cb, 0u);
@@ -445,72 +566,57 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 }
             }
             ptx::fence_proxy_async_smem();
-            mbar_arrive(&s.s_init);
+            mbar_arrive(&s.s_ready[0]);
         }
-        // sum of the hi row (regs 4k, 4k+1) and lo row (regs 4k+2, 4k+3) of a 16x256b load
-        auto rows_sum = [](const uint32_t (&v)[16], int k) {
-            return __fadd2_rn(make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1])),
-                              make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
-        };
         int n = 0;
         for (; n < NC; ++n) {
             const int pb = n & 1;
-            const int valid = min(C, T - n * C);
+            // ---- state(n): S <- gamma (S + U), U^T[j][i] = DU[j][i] + DU[j][64+i]
             {
-                bool bad = !ptx::mbar_wait(&s.g1_done, (uint32_t)(n & 1), budget);
-                // gamma / bonus of this chunk were written by prep before prep_done
-                if (!bad && ld_volatile(&s.stop_at) != n)
-                    bad = !ptx::mbar_wait(&s.prep_done[pb], (uint32_t)((n >> 1) & 1), budget);
-                if (bad) s.abort = 1;
-                // uniform over the epilogue group: stop (hand-off) or abort
-                if (named_bar_any(3, kEpiThreads, bad || ld_volatile(&s.abort) || ld_volatile(&s.stop_at) == n)) break;
+                const bool ok = wait_soft(s, &s.gu_done[pb], (uint32_t)((n >> 1) & 1), budget);
+                // uniform over the epilogue: stop (hand-off) or abort
+                if (named_bar_any(kBarEpi, kEpiThreads, !ok || ld_volatile(&s.abort) || ld_volatile(&s.stop_at) == n)) break;
             }
             ptx::tc_fence_after();
-            // ---- state: S <- gamma (S + U), U^T[j][i] = DU[j][i] + DU[j][64+i]
             {
                 uint32_t ua[16], ub[16];
-                tmem_ld16x4(tmem + lane_m64 + COL_DU + 32 * ch, ua);
-                tmem_ld16x4(tmem + lane_m64 + COL_DU + 64 + 32 * ch, ub);
+                tmem_ld16x4(tmem + lane_h0 + COL_DU + 128 * pb + 32 * ch, ua);
+                tmem_ld16x4(tmem + lane_h0 + COL_DU + 128 * pb + 64 + 32 * ch, ub);
                 ptx::tmem_wait_ld();
-                uint8_t* sh = s.bblk[pb ^ 1][0];
-                uint8_t* sl = s.bblk[pb ^ 1][2];
+                ptx::tc_fence_before();
+                mbar_arrive(&s.du_free[pb]);
+                float2 gv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) gv[k] = *reinterpret_cast<const float2*>(&s.gamma[pb][cbase + 8 * k]);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const float2 g = *reinterpret_cast<const float2*>(&s.gamma[pb][cbase + 8 * k]);
-                    const float2 du0 = __fadd2_rn(make_float2(__uint_as_float(ua[4 * k]), __uint_as_float(ua[4 * k + 1])),
-                                                  make_float2(__uint_as_float(ub[4 * k]), __uint_as_float(ub[4 * k + 1])));
-                    const float2 du1 = __fadd2_rn(make_float2(__uint_as_float(ua[4 * k + 2]), __uint_as_float(ua[4 * k + 3])),
-                                                  make_float2(__uint_as_float(ub[4 * k + 2]), __uint_as_float(ub[4 * k + 3])));
-                    S0[k] = __fmul2_rn(g, __fadd2_rn(S0[k], du0));
-                    S1[k] = __fmul2_rn(g, __fadd2_rn(S1[k], du1));
-                    uint32_t hi, lo;
-                    split2(S0[k], hi, lo);
-                    sts32(sh, sw_off(r0, 4 * ch + k) + cb, hi);
-                    sts32(sl, sw_off(r0, 4 * ch + k) + cb, lo);
-                    split2(S1[k], hi, lo);
-                    sts32(sh, sw_off(r1, 4 * ch + k) + cb, hi);
-                    sts32(sl, sw_off(r1, 4 * ch + k) + cb, lo);
+                    const float2 du0 = __fadd2_rn(lo_pair(ua, k), lo_pair(ub, k));
+                    const float2 du1 = __fadd2_rn(hi_pair(ua, k), hi_pair(ub, k));
+                    S0[k] = __fmul2_rn(gv[k], __fadd2_rn(S0[k], du0));
+                    S1[k] = __fmul2_rn(gv[k], __fadd2_rn(S1[k], du1));
                 }
             }
-            // ---- readout part Yi (kept in registers) and scores A -> A_hi / A_lo tiles
-            float2 Y0[4], Y1[4];
-            {
-                uint32_t p0[16], p1[16];
-                tmem_ld16x4(tmem + lane_h0 + COL_D1 + 32 * ch, p0);
-                tmem_ld16x4(tmem + lane_h1 + COL_D1 + 32 * ch, p1);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    Y0[k] = rows_sum(p0, k);
-                    Y1[k] = rows_sum(p1, k);
-                }
+            if (n + 1 < NC) {
+                // S_n feeds RO(n+1) from sb[(n+1) & 1], whose S_{n-2} RO(n-1) has read
+                if (n >= 1) wait_soft(s, &s.s_free[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), budget);
+                store_state(s.sb[(n + 1) & 1], S0, S1, r0, r1, ch, cb);
+                ptx::fence_proxy_async_smem();
+                mbar_arrive(&s.s_ready[(n + 1) & 1]);
             }
+            // ---- output of chunk n-1 (its GA was issued at the end of the previous round)
+            if (n >= 1) output_chunk(s, n - 1, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
+            // ---- A(n): masked scores with the bonus on the diagonal, hi / lo, for GA(n)
+            wait_soft(s, &s.sc_done[pb], (uint32_t)((n >> 1) & 1), budget);
+            ptx::tc_fence_after();
             if (!a_zero) {
                 uint32_t p0[16], p1[16];
-                tmem_ld16x4(tmem + lane_h0 + COL_D1 + 64 + 32 * ch, p0);
-                tmem_ld16x4(tmem + lane_h1 + COL_D1 + 64 + 32 * ch, p1);
+                tmem_ld16x4(tmem + lane_h0 + COL_SC + 64 * pb + 32 * ch, p0);
+                tmem_ld16x4(tmem + lane_h1 + COL_SC + 64 * pb + 32 * ch, p1);
                 ptx::tmem_wait_ld();
+                ptx::tc_fence_before();
+                mbar_arrive(&s.sc_free[pb]);
                 const float b0 = s.bonus[pb][r0], b1 = s.bonus[pb][r1];
+                // the A tile is free: GA(n-1) completed before output(n-1) read Y
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     float2 a0 = rows_sum(p0, k), a1 = rows_sum(p1, k);
@@ -529,57 +635,18 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     sts32(s.at, sw_off(hr1, 4 * ch + k) + cb, hi);
                     sts32(s.at, sw_off(hr1 + 8, 4 * ch + k) + cb, lo);
                 }
+            } else {
+                ptx::tc_fence_before();
+                mbar_arrive(&s.sc_free[pb]);
             }
             ptx::fence_proxy_async_smem();
-            ptx::tc_fence_before();
-            mbar_arrive(&s.epi_mid);
-            // ---- output: y = Yi + A.V
-            {
-                const bool bad = !ptx::mbar_wait(&s.ga_done, (uint32_t)(n & 1), budget);
-                if (bad) s.abort = 1;
-                if (named_bar_any(3, kEpiThreads, bad || ld_volatile(&s.abort))) break;
-            }
-            ptx::tc_fence_after();
-            {
-                uint32_t d0[16], d1[16];
-                tmem_ld16x4(tmem + lane_h0 + COL_DA + 32 * ch, d0);
-                tmem_ld16x4(tmem + lane_h1 + COL_DA + 32 * ch, d1);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    Y0[k] = __fadd2_rn(Y0[k], rows_sum(d0, k));
-                    Y1[k] = __fadd2_rn(Y1[k], rows_sum(d1, k));
-                }
-            }
-            ptx::tc_fence_before();
-            mbar_arrive(&s.epi_end);    // DA read: GA of the next chunk may overwrite it
-            if (y_raw != nullptr) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int j = cbase + 8 * k;
-                    if (r0 < valid)
-                        *reinterpret_cast<float2*>(y_raw + (((size_t)b * T + n * C + r0) * H + h) * 64 + j) = Y0[k];
-                    if (r1 < valid)
-                        *reinterpret_cast<float2*>(y_raw + (((size_t)b * T + n * C + r1) * H + h) * 64 + j) = Y1[k];
-                }
-            } else {
-                // the previous chunk's store must have read the staging tile
-                if (et == 0) ptx::bulk_wait_read<0>();
-                named_bar(2, kEpiThreads);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    sts32(s.ystage, sw_off(r0, 4 * ch + k) + cb, pack2(Y0[k].x, Y0[k].y));
-                    sts32(s.ystage, sw_off(r1, 4 * ch + k) + cb, pack2(Y1[k].x, Y1[k].y));
-                }
-                ptx::fence_proxy_async_smem();
-                named_bar(2, kEpiThreads);
-                if (et == 0) {
-                    ptx::tma_store_4d(&tm_y, s.ystage, 0, h, n * C, b);
-                    ptx::bulk_commit();
-                }
-            }
+            mbar_arrive(&s.a_ready);
+            mbar_arrive(&s.ep_free[pb]);      // gamma / bonus of parity pb read
         }
-        // ---- leave: final state, or the state entering the chunk handed to the level kernel
+        // ---- leave: output of the last chunk done, final state (or the state entering the
+        // chunk handed to the level kernel)
+        if (!ld_volatile(&s.abort) && n >= 1)
+            output_chunk(s, n - 1, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
         const bool aborted = ld_volatile(&s.abort) != 0;
         if (!aborted) {
             const bool stopped = (n < NC);
@@ -594,9 +661,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     dst[(i + 1) * 64 + r1] = S1[k].y;
                 }
             }
-            if (et == 0) handoff_chunk[bh] = stopped ? n : -1;
+            if (tid == kEpiWarp0 * 32) handoff_chunk[bh] = stopped ? n : -1;
         }
-        if (et == 0) ptx::bulk_wait<0>();
     }
 
     ptx::tc_fence_before();
@@ -605,7 +671,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         atomicExch(status, 1);
         handoff_chunk[bh] = -1;
     }
-    if (warp == 1) {
+    if (warp == kTmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
@@ -616,16 +682,16 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
 size_t fast_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
-                                float* s_out, float* y_raw, int B, int T, int H, int* status,
-                                int* handoff_chunk, float* handoff_state, long long budget,
-                                cudaStream_t st) {
+                                float* s_out, void* y, float* y_raw, int B, int T, int H,
+                                int* status, int* handoff_chunk, float* handoff_state,
+                                long long budget, cudaStream_t st) {
     const size_t smem = fast_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(wkv6_fast_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     wkv6_fast_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw, T, H, status,
-        handoff_chunk, handoff_state, budget, 4000000000LL);
+        maps[0], maps[1], maps[2], maps[3], u, s_in, s_out, static_cast<__nv_bfloat16*>(y),
+        y_raw, T, H, status, handoff_chunk, handoff_state, budget, 4000000000LL);
     return cudaGetLastError();
 }
 

@@ -32,7 +32,7 @@ bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H);
 // whose decay range it cannot take and records that chunk in handoff_chunk[bh] (-1: done)
 // with the state entering it in handoff_state[bh].  y_raw != nullptr: fp32 y rows there.
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
-                                float* s_out, float* y_raw, int B, int T, int H, int* status,
+                                float* s_out, void* y, float* y_raw, int B, int T, int H, int* status,
                                 int* handoff_chunk, float* handoff_state, long long budget,
                                 cudaStream_t st);
 
