@@ -195,6 +195,52 @@ def sum_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def other_prefill(cfg, dev, world, hbm, algo, steps):
+    """Device-timed prefill calls of another workload shape: one line of its own (tokens/s and
+    the fraction of the HBM roofline), inputs resident in HBM and larger than L2."""
+    import linear_attention_rnn_finch_b200 as gw
+    inp = W.make_prefill_inputs(cfg, dev)
+    B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
+    ln = (inp["gamma"], inp["beta"], inp["eps"]) if cfg.ln else None
+    ws = gw.new_workspace(gw.prefill_workspace_bytes(B, T, H, D, cfg.dtype, ln is not None, algo), dev)
+    y = torch.empty_like(inp["r"])
+    s_out = torch.empty_like(inp["state0"])
+    args_p = [inp[n] for n in ("r", "k", "v", "omega")]
+
+    def call():
+        gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], ln=ln, y=y, state_out=s_out,
+                        algo=algo, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    nbytes = prefill_bytes(B, T, H, D)
+    # with LayerNorm the library also writes and re-reads an fp32 copy of y; the roofline
+    # counts only the bytes the operation itself must move
+    nbytes_note = ("LayerNorm runs as a second pass over an fp32 copy of y, not counted in the "
+                   "algorithmic bytes") if cfg.ln else None
+    line = {"workload": cfg.name, "B": B, "T": T, "H": H, "D": D, "io": "bf16",
+            "ln": bool(cfg.ln), "steps": steps, "ms_per_call": ms,
+            "tokens_per_s": world * B * T / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm,
+                         "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm,
+                         "algorithmic_bytes_per_call": nbytes}}
+    if nbytes_note:
+        line["note"] = nbytes_note
+    del inp, y, s_out, ws
+    torch.cuda.empty_cache()
+    return line
+
+
 # ------------------------------------------------------------------------------ oracle timing
 def oracle_sample(cfg, b_rows: int, t_tokens: int, seed_offset: int = 0):
     """Inputs of the oracle's bounded sample: b_rows batch rows x t_tokens tokens of cfg,
@@ -356,6 +402,12 @@ def run_ours(args, world, rank, local):
                          "gpu_launches": dsteps}
         del dinp, dargs, state
 
+    # the other prefill shapes: long context (one sequence per head; the library splits it
+    # into segments across SMs) and the decay-extreme stress with fused LayerNorm
+    if not args.no_other:
+        out["other_prefill"] = [other_prefill(W.CONFIGS[2], dev, world, hbm, args.algo, steps=5),
+                                other_prefill(W.CONFIGS[4], dev, world, hbm, args.algo, steps=5)]
+
     # end to end through the public API with host buffers
     if not args.no_e2e:
         host = {n: inp[n].cpu().pin_memory() for n in ("r", "k", "v", "omega", "u", "state0")}
@@ -452,6 +504,8 @@ def main():
     ap.add_argument("--algo", choices=["auto", "recurrent", "chunked"], default="auto")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-other", action="store_true",
+                    help="skip the long-context and decay-extreme prefill lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clock-warm", action="store_true",
                     help="skip the ~1 s untimed warm-up loop (for profiler runs)")

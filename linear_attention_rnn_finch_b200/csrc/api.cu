@@ -95,9 +95,55 @@ bool use_chunked(wkv_dtype io, wkv_algo algo) {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// chunked-path workspace: status | hand-off chunk per (b,h) | hand-off state per (b,h)
-size_t handoff_ints_bytes(int B, int H) { return round256((size_t)B * H * sizeof(int)); }
-size_t handoff_state_bytes(int B, int H) { return (size_t)B * H * 64 * 64 * sizeof(float); }
+constexpr int kChunk = 64;          // tokens per chunk of the chunked kernels
+constexpr int kSmCount = 148;       // SMs of a B200: the unit of a wave of CTAs
+constexpr int kMinSegChunks = 16;   // shortest segment worth a CTA
+// Cost of the state pre-pass per chunk relative to the full prefill per chunk (it reads
+// k, v, omega and runs the state update only).
+constexpr double kPrePassCost = 0.5;
+
+long waves(long ctas) { return (ctas + kSmCount - 1) / kSmCount; }
+
+// Segments per sequence on the chunked path.  One CTA runs each (b,h) segment; the split
+// pays when B*H alone leaves SMs idle: estimated time = waves of the main pass x chunks per
+// segment + the pre-pass over the first P-1 segments.  Every segment must be non-empty.
+// GOLDWKV_SEGMENTS=n forces n (tests of the split on small problems).
+int choose_segments(int B, int T, int H) {
+    const long nbh = (long)B * H;
+    const int nc = (T + kChunk - 1) / kChunk;
+    auto feasible = [&](int P) { return P >= 1 && (long)(P - 1) * ((nc + P - 1) / P) < nc; };
+    if (const char* f = getenv("GOLDWKV_SEGMENTS")) {
+        int P = atoi(f);
+        while (P > 1 && !feasible(P)) --P;
+        return P < 1 ? 1 : P;
+    }
+    double best = (double)waves(nbh) * nc;
+    int best_p = 1;
+    for (int P = 2; P <= 64; ++P) {
+        const int seg = (nc + P - 1) / P;
+        if (seg < kMinSegChunks) break;
+        if (!feasible(P)) continue;
+        const double t = (double)waves(nbh * P) * seg + kPrePassCost * (double)waves(nbh * (P - 1)) * seg;
+        if (t < 0.9 * best) {
+            best = t;
+            best_p = P;
+        }
+    }
+    return best_p;
+}
+
+// chunked-path workspace: status | hand-off chunk per unit | hand-off state per unit |
+// segment states (B*H*(P-1) x D*D fp32) | segment log2 decays (B*H*(P-1) x D fp32)
+size_t handoff_ints_bytes(long units) { return round256((size_t)units * sizeof(int)); }
+size_t handoff_state_bytes(long units) { return (size_t)units * 64 * 64 * sizeof(float); }
+size_t segment_bytes(int B, int H, int P) {
+    return (size_t)B * H * (P - 1) * (64 * 64 + 64) * sizeof(float);
+}
+size_t chunked_bytes(int B, int H, int P) {
+    const long units = (long)B * H * P;
+    return kStatusBytes + handoff_ints_bytes(units) + handoff_state_bytes(units) +
+           segment_bytes(B, H, P);
+}
 
 }  // namespace
 
@@ -121,7 +167,8 @@ size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, in
                                     wkv_algo algo) {
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
     const bool chunked = use_chunked(io, algo);
-    size_t bytes = chunked ? kStatusBytes + handoff_ints_bytes(B, H) + handoff_state_bytes(B, H) : 0;
+    const int P = algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
+    size_t bytes = chunked ? chunked_bytes(B, H, P) : 0;
     // LayerNorm with bf16 output stages the fp32 rows; with fp32 output y itself does
     if (with_ln && io == WKV_BF16) bytes += (size_t)B * T * H * D * sizeof(float);
     return bytes;
@@ -199,9 +246,12 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
     const bool chunked = use_chunked(io, algo);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
+    const int P = !chunked || algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
+    const long units = (long)B * H * P;
     const size_t hand_i = chunked ? kStatusBytes : 0;
-    const size_t hand_s = hand_i + (chunked ? handoff_ints_bytes(B, H) : 0);
-    const size_t raw_at = hand_s + (chunked ? handoff_state_bytes(B, H) : 0);
+    const size_t hand_s = hand_i + (chunked ? handoff_ints_bytes(units) : 0);
+    const size_t seg_at = hand_s + (chunked ? handoff_state_bytes(units) : 0);
+    const size_t raw_at = chunked ? chunked_bytes(B, H, P) : 0;
     if (ln) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
     if (chunked) {
@@ -216,15 +266,27 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
         int* status = reinterpret_cast<int*>(ws);
         int* h_chunk = reinterpret_cast<int*>(ws + hand_i);
         float* h_state = reinterpret_cast<float*>(ws + hand_s);
+        float* s_mid = reinterpret_cast<float*>(ws + seg_at);
+        float* log2g = s_mid + (size_t)B * H * (P - 1) * 64 * 64;
+        const int nc = (T + kChunk - 1) / kChunk;
+        const goldwkv::Segments seg{P, (nc + P - 1) / P, s_mid};
         if (algo == WKV_ALGO_CHUNKED_LEVELS) {
-            e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
+            e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg,
                                                status, nullptr, nullptr, budget, st);
         } else {
-            e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H,
-                                             status, h_chunk, h_state, budget, st);
+            e = cudaSuccess;
+            if (P > 1) {   // states entering segments 1 .. P-1 (computed in place in s_mid)
+                e = goldwkv::launch_segment_states(maps, s_mid, log2g, B, T, H, seg, status,
+                                                   budget, st);
+                if (e == cudaSuccess)
+                    e = goldwkv::launch_segment_carry(state_in, s_mid, log2g, s_mid, B, H, P, st);
+            }
+            if (e == cudaSuccess)
+                e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H,
+                                                 seg, status, h_chunk, h_state, budget, st);
             if (e == cudaSuccess)
                 e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
-                                                   status, h_chunk, h_state, budget, st);
+                                                   seg, status, h_chunk, h_state, budget, st);
         }
     } else {
         e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,

@@ -1,0 +1,125 @@
+// Device helpers shared by the tcgen05 chunk kernels: 128B-swizzled tile addressing, bf16
+// pair packing and hi/lo splitting, 16x256b TMEM loads, named barriers and bounded
+// mbarrier waits.  Include only from CUDA sources compiled for sm_100a.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "sm100_ptx.cuh"
+
+namespace goldwkv {
+namespace tiles {
+
+constexpr int kTile = 64 * 64 * 2;   // one 64-row x 128-byte tile (64 x 64 bf16)
+
+__device__ __forceinline__ uint32_t sw_off(int row, int chunk) {
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+// stacked hi/lo row of token t: hi parts in rows 0-7 of each 16-row group, lo in rows 8-15
+__device__ __forceinline__ int hi_row(int t) { return 32 * (t >> 4) + 16 * ((t >> 3) & 1) + (t & 7); }
+
+// bf16x2 of (a, b): a in the low half (lower address), b in the high half
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// hi = bf16(x), lo = bf16(x - hi) for a pair: two conversions and one packed subtract
+__device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
+    hi = pack2(x.x, x.y);
+    const float2 d = __fadd2_rn(x, make_float2(-__uint_as_float(hi << 16),
+                                               -__uint_as_float(hi & 0xFFFF0000u)));
+    lo = pack2(d.x, d.y);
+}
+__device__ __forceinline__ void sts32(uint8_t* base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t*>(base + off) = v;
+}
+__device__ __forceinline__ uint32_t lds32(const uint8_t* base, uint32_t off) {
+    return *reinterpret_cast<const uint32_t*>(base + off);
+}
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 16 lanes x 256 bits x 4: thread l gets lanes base + l/4 (regs 4k, 4k+1) and
+// base + 8 + l/4 (regs 4k+2, 4k+3), columns col + 8k + 2(l%4) + {0,1}, k = 0..3.
+__device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+// the (hi row + lo row) pair k of a 16x256b load: registers 4k, 4k+1 plus 4k+2, 4k+3
+__device__ __forceinline__ float2 rows_sum(const uint32_t (&v)[16], int k) {
+    return __fadd2_rn(make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1])),
+                      make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+}
+__device__ __forceinline__ float2 lo_pair(const uint32_t (&v)[16], int k) {
+    return make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]));
+}
+__device__ __forceinline__ float2 hi_pair(const uint32_t (&v)[16], int k) {
+    return make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// barrier over `nthreads` threads that also ORs a predicate across them (uniform decision)
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ int ld_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+
+// Bounded wait on an mbarrier phase.  `s` is the CTA's shared state with `abort` and
+// `stop_at` words: the wait gives up early once the CTA has aborted, and on expiry it aborts
+// the CTA.
+// Returns false if the caller should treat its data as invalid (abort).
+// With `or_stop`, also gives up (without aborting) once this (b,h) has been handed over.
+template <class Sm>
+__device__ __forceinline__ bool wait_soft(Sm& s, uint64_t* bar, uint32_t parity, long long budget,
+                                          bool or_stop = false) {
+    if (ptx::mbar_test_wait(bar, parity)) return true;
+    if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
+    if (budget <= 0) {
+        s.abort = 1;
+        return false;
+    }
+    const long long t0 = clock64();
+    for (;;) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ld_volatile(&s.abort)) return false;
+        if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
+        if (clock64() - t0 > budget) {
+            s.abort = 1;
+            return false;
+        }
+    }
+}
+
+
+}  // namespace tiles
+}  // namespace goldwkv

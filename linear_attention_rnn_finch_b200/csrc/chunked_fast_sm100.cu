@@ -48,15 +48,17 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "chunk_tiles.cuh"
 #include "sm100_ptx.cuh"
 
 namespace goldwkv {
 
 namespace {
 
+using namespace tiles;
+
 constexpr int C = 64;
 constexpr int kStages = 3;
-constexpr int kTile = 64 * 64 * 2;            // 64 rows x 128 B
 constexpr int kPrepWarps = 8, kEpiWarps = 8;
 constexpr int kTmaWarp = 0, kMmaUWarp = 1, kMmaYWarp = 2;
 constexpr int kPrepWarp0 = 3, kEpiWarp0 = kPrepWarp0 + kPrepWarps;
@@ -96,116 +98,13 @@ struct __align__(1024) Smem {
     int stop_at;                     // chunk at which this (b,h) leaves for the level kernel
 };
 
-__device__ __forceinline__ uint32_t sw_off(int row, int chunk) {
-    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-// stacked hi/lo row of token t: hi parts in rows 0-7 of each 16-row group, lo in rows 8-15
-__device__ __forceinline__ int hi_row(int t) { return 32 * (t >> 4) + 16 * ((t >> 3) & 1) + (t & 7); }
-
-// bf16x2 of (a, b): a in the low half (lower address), b in the high half
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-    return r;
-}
-__device__ __forceinline__ float2 unpack2(uint32_t w) {
-    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-// hi = bf16(x), lo = bf16(x - hi) for a pair: two conversions and one packed subtract
-__device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
-    hi = pack2(x.x, x.y);
-    const float2 d = __fadd2_rn(x, make_float2(-__uint_as_float(hi << 16),
-                                               -__uint_as_float(hi & 0xFFFF0000u)));
-    lo = pack2(d.x, d.y);
-}
-__device__ __forceinline__ void sts32(uint8_t* base, uint32_t off, uint32_t v) {
-    *reinterpret_cast<uint32_t*>(base + off) = v;
-}
-__device__ __forceinline__ uint32_t lds32(const uint8_t* base, uint32_t off) {
-    return *reinterpret_cast<const uint32_t*>(base + off);
-}
-__device__ __forceinline__ float fast_exp2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// 16 lanes x 256 bits x 4: thread l gets lanes base + l/4 (regs 4k, 4k+1) and
-// base + 8 + l/4 (regs 4k+2, 4k+3), columns col + 8k + 2(l%4) + {0,1}, k = 0..3.
-__device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
-}
-// the (hi row + lo row) pair k of a 16x256b load: registers 4k, 4k+1 plus 4k+2, 4k+3
-__device__ __forceinline__ float2 rows_sum(const uint32_t (&v)[16], int k) {
-    return __fadd2_rn(make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1])),
-                      make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
-}
-__device__ __forceinline__ float2 lo_pair(const uint32_t (&v)[16], int k) {
-    return make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]));
-}
-__device__ __forceinline__ float2 hi_pair(const uint32_t (&v)[16], int k) {
-    return make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
-}
-
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// barrier over `nthreads` threads that also ORs a predicate across them (uniform decision)
-__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ int ld_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
-
-// Bounded wait that gives up early once the CTA has aborted; on expiry it aborts the CTA.
-// Returns false if the caller should treat its data as invalid (abort).
-// With `or_stop`, also gives up (without aborting) once this (b,h) has been handed over.
-__device__ __forceinline__ bool wait_soft(Smem& s, uint64_t* bar, uint32_t parity, long long budget,
-                                          bool or_stop = false) {
-    if (ptx::mbar_test_wait(bar, parity)) return true;
-    if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
-    if (budget <= 0) {
-        s.abort = 1;
-        return false;
-    }
-    const long long t0 = clock64();
-    for (;;) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
-        if (ld_volatile(&s.abort)) return false;
-        if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
-        if (clock64() - t0 > budget) {
-            s.abort = 1;
-            return false;
-        }
-    }
-}
-
 // Output of chunk m: y = Y[:, 0:64] + Y[:, 64:128] (hi and lo rows each), stored as bf16 (or
 // fp32 rows to y_raw).  Frees the Y accumulator for RO(m+1).
-__device__ __forceinline__ void output_chunk(Smem& s, int m, uint32_t tmem, uint32_t lane_h0,
+__device__ __forceinline__ void output_chunk(Smem& s, int m, int c0, uint32_t tmem, uint32_t lane_h0,
                                              uint32_t lane_h1, int ch, int cbase, int r0, int r1,
                                              int b, int h, int T, int H, __nv_bfloat16* y,
                                              float* y_raw, long long budget) {
+    // m: chunk index within the unit (GA(m) is the (m+1)-th ya_done phase); c0 + m: absolute
     wait_soft(s, &s.ya_done, (uint32_t)(m & 1), budget);
     ptx::tc_fence_after();
     float2 Y0[4], Y1[4];
@@ -227,9 +126,10 @@ __device__ __forceinline__ void output_chunk(Smem& s, int m, uint32_t tmem, uint
     }
     ptx::tc_fence_before();
     mbar_arrive(&s.y_free);
-    const int valid = min(C, T - m * C);
-    const size_t row0 = ((size_t)b * T + (size_t)m * C + r0) * H + h;
-    const size_t row1 = ((size_t)b * T + (size_t)m * C + r1) * H + h;
+    const int tc = (c0 + m) * C;
+    const int valid = min(C, T - tc);
+    const size_t row0 = ((size_t)b * T + (size_t)tc + r0) * H + h;
+    const size_t row1 = ((size_t)b * T + (size_t)tc + r1) * H + h;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int j = cbase + 8 * k;
@@ -263,14 +163,17 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                  const float* __restrict__ u, const float* s_in, float* s_out,
                  __nv_bfloat16* __restrict__ y, float* __restrict__ y_raw, int T, int H,
-                 int* status, int* handoff_chunk, float* handoff_state, long long budget,
-                 long long drain_budget) {
+                 Segments seg, int* status, int* handoff_chunk, float* handoff_state,
+                 long long budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, b = bh / H, h = bh - (bh / H) * H;
-    const int NC = (T + C - 1) / C;
+    // unit: segment pseg of sequence bh; chunks cseg .. cseg + NC - 1 (absolute indices)
+    const int unit = blockIdx.x, nbh = gridDim.x / seg.P;
+    const int bh = unit % nbh, pseg = unit / nbh, b = bh / H, h = bh - (bh / H) * H;
+    const int cseg = pseg * seg.seg_chunks;
+    const int NC = min((T + C - 1) / C, cseg + seg.seg_chunks) - cseg;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -316,13 +219,13 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 const uint32_t par = (uint32_t)((n / kStages - 1) & 1);   // release of chunk n-3
                 if (n >= kStages && !wait_soft(s, &s.empty_rkw[st], par, budget, true)) break;
                 ptx::mbar_arrive_expect_tx(&s.full_rkw[st], 3 * kTile);
-                ptx::tma_load_4d(s.rkw[st][0], &tm_r, &s.full_rkw[st], 0, h, n * C, b);
-                ptx::tma_load_4d(s.rkw[st][1], &tm_k, &s.full_rkw[st], 0, h, n * C, b);
-                ptx::tma_load_4d(s.rkw[st][2], &tm_w, &s.full_rkw[st], 0, h, n * C, b);
+                ptx::tma_load_4d(s.rkw[st][0], &tm_r, &s.full_rkw[st], 0, h, (cseg + n) * C, b);
+                ptx::tma_load_4d(s.rkw[st][1], &tm_k, &s.full_rkw[st], 0, h, (cseg + n) * C, b);
+                ptx::tma_load_4d(s.rkw[st][2], &tm_w, &s.full_rkw[st], 0, h, (cseg + n) * C, b);
                 last_rkw[st] = n;
                 if (n >= kStages && !wait_soft(s, &s.empty_v[st], par, budget, true)) break;
                 ptx::mbar_arrive_expect_tx(&s.full_v[st], kTile);
-                ptx::tma_load_4d(s.vt[st], &tm_v, &s.full_v[st], 0, h, n * C, b);
+                ptx::tma_load_4d(s.vt[st], &tm_v, &s.full_v[st], 0, h, (cseg + n) * C, b);
                 last_v[st] = n;
             }
             // every issued copy must land before the CTA may exit
@@ -418,7 +321,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         const float2 nl2e = make_float2(-kLog2e, -kLog2e);
         for (int n = 0; n < NC; ++n) {
             const int pb = n & 1, st = n % kStages;
-            const int valid = min(C, T - n * C);
+            const int valid = min(C, T - (cseg + n) * C);
             bool ok_wait = wait_soft(s, &s.full_rkw[st], (uint32_t)((n / kStages) & 1), budget);
             if (n >= 2) {
                 ok_wait = ok_wait && wait_soft(s, &s.op_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget);
@@ -548,7 +451,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         // state S[i][j] held transposed: rows j = r0, r1; columns i = cbase + 8k + {0,1}
         float2 S0[4], S1[4];
         {
-            const float* src = s_in ? s_in + (size_t)bh * 4096 : nullptr;
+            const float* src = pseg > 0 ? seg.s_mid + ((size_t)bh * (seg.P - 1) + (pseg - 1)) * 4096
+                                     : s_in ? s_in + (size_t)bh * 4096 : nullptr;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int i = cbase + 8 * k;
@@ -573,6 +477,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             const int pb = n & 1;
             // ---- state(n): S <- gamma (S + U), U^T[j][i] = DU[j][i] + DU[j][64+i]
             {
+                // gamma and bonus of chunk n reach us from prep through the chain prep's
+                // release-arrive on prep_done -> the GU issuer's acquire -> its commit on gu_done
                 const bool ok = wait_soft(s, &s.gu_done[pb], (uint32_t)((n >> 1) & 1), budget);
                 // uniform over the epilogue: stop (hand-off) or abort
                 if (named_bar_any(kBarEpi, kEpiThreads, !ok || ld_volatile(&s.abort) || ld_volatile(&s.stop_at) == n)) break;
@@ -604,7 +510,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 mbar_arrive(&s.s_ready[(n + 1) & 1]);
             }
             // ---- output of chunk n-1 (its GA was issued at the end of the previous round)
-            if (n >= 1) output_chunk(s, n - 1, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
+            if (n >= 1) output_chunk(s, n - 1, cseg, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
             // ---- A(n): masked scores with the bonus on the diagonal, hi / lo, for GA(n)
             wait_soft(s, &s.sc_done[pb], (uint32_t)((n >> 1) & 1), budget);
             ptx::tc_fence_after();
@@ -646,11 +552,13 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         // ---- leave: output of the last chunk done, final state (or the state entering the
         // chunk handed to the level kernel)
         if (!ld_volatile(&s.abort) && n >= 1)
-            output_chunk(s, n - 1, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
+            output_chunk(s, n - 1, cseg, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
         const bool aborted = ld_volatile(&s.abort) != 0;
         if (!aborted) {
             const bool stopped = (n < NC);
-            float* dst = stopped ? handoff_state + (size_t)bh * 4096 : s_out ? s_out + (size_t)bh * 4096 : nullptr;
+            float* dst = stopped                       ? handoff_state + (size_t)unit * 4096
+                         : (s_out && pseg == seg.P - 1) ? s_out + (size_t)bh * 4096
+                                                     : nullptr;
             if (dst) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -661,7 +569,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     dst[(i + 1) * 64 + r1] = S1[k].y;
                 }
             }
-            if (tid == kEpiWarp0 * 32) handoff_chunk[bh] = stopped ? n : -1;
+            if (tid == kEpiWarp0 * 32) handoff_chunk[unit] = stopped ? cseg + n : -1;
         }
     }
 
@@ -669,7 +577,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
     __syncthreads();
     if (s.abort && tid == 0) {
         atomicExch(status, 1);
-        handoff_chunk[bh] = -1;
+        handoff_chunk[unit] = -1;
     }
     if (warp == kTmaWarp) {
         ptx::tc_fence_after();
@@ -683,15 +591,15 @@ size_t fast_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
                                 float* s_out, void* y, float* y_raw, int B, int T, int H,
-                                int* status, int* handoff_chunk, float* handoff_state,
-                                long long budget, cudaStream_t st) {
+                                Segments seg, int* status, int* handoff_chunk,
+                                float* handoff_state, long long budget, cudaStream_t st) {
     const size_t smem = fast_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(wkv6_fast_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_fast_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
+    wkv6_fast_kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], u, s_in, s_out, static_cast<__nv_bfloat16*>(y),
-        y_raw, T, H, status, handoff_chunk, handoff_state, budget, 4000000000LL);
+        y_raw, T, H, seg, status, handoff_chunk, handoff_state, budget, 4000000000LL);
     return cudaGetLastError();
 }
 

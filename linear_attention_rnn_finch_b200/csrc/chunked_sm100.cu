@@ -130,18 +130,25 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
                     const float* s_in, float* s_out, float* __restrict__ y_raw, int T, int H,
-                    int* status, const int* start_chunk, const float* handoff_state,
-                    long long spin_budget, long long drain_budget) {
+                    Segments seg, int* status, const int* start_chunk,
+                    const float* handoff_state, long long spin_budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, b = bh / H, h = bh - (bh / H) * H;
-    const int NC = (T + C - 1) / C;
+    // unit: segment pseg of sequence bh, absolute chunks c_begin .. NC - 1
+    const int unit = blockIdx.x, nbh = gridDim.x / seg.P;
+    const int bh = unit % nbh, pseg = unit / nbh, b = bh / H, h = bh - (bh / H) * H;
+    const int c_begin = pseg * seg.seg_chunks;
+    const int NC = min((T + C - 1) / C, c_begin + seg.seg_chunks);
     // resume point: chunks before n0 (and the state entering n0) came from the fast kernel
-    const int n0 = start_chunk ? start_chunk[bh] : 0;
-    if (n0 < 0 || n0 >= NC) return;       // this (b,h) is already complete
-    if (start_chunk) s_in = handoff_state;
+    const int n0 = start_chunk ? start_chunk[unit] : c_begin;
+    if (n0 < 0 || n0 >= NC) return;       // this unit is already complete
+    const float* state0 = start_chunk ? handoff_state + (size_t)unit * 4096
+                        : pseg > 0    ? seg.s_mid + ((size_t)bh * (seg.P - 1) + (pseg - 1)) * 4096
+                        : s_in        ? s_in + (size_t)bh * 4096
+                                      : nullptr;
+    if (pseg < seg.P - 1) s_out = nullptr;   // only the last segment's final state is the output
 
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
@@ -186,7 +193,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     const uint32_t tlane = (uint32_t)(32 * q) << 16;
     float S[32];
     {
-        const float* src = s_in ? s_in + (size_t)bh * 4096 + row * 64 + 32 * hh : nullptr;
+        const float* src = state0 ? state0 + row * 64 + 32 * hh : nullptr;
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -559,16 +566,17 @@ bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H) {
 size_t chunked_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
-                                  float* s_out, float* y_raw, int B, int T, int H, int* status,
-                                  const int* start_chunk, const float* handoff_state,
-                                  long long spin_budget, cudaStream_t st) {
+                                  float* s_out, float* y_raw, int B, int T, int H, Segments seg,
+                                  int* status, const int* start_chunk,
+                                  const float* handoff_state, long long spin_budget,
+                                  cudaStream_t st) {
     const size_t smem = chunked_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long drain = 4000000000LL;
-    wkv6_chunked_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw, T, H, status,
+    wkv6_chunked_kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw, T, H, seg, status,
         start_chunk, handoff_state, spin_budget, drain);
     return cudaGetLastError();
 }

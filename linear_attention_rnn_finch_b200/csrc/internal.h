@@ -27,23 +27,47 @@ cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const floa
 // TMA descriptor of a [B][T][H][64] bf16 tensor: box 64 channels x 1 head x 64 tokens.
 bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H);
 
-// Fast path (one-sided decay factorisation, warp-specialised pipeline).  maps: r, k, v,
-// omega, y.  For each (b,h) it writes y and the final state, or stops at the first chunk
-// whose decay range it cannot take and records that chunk in handoff_chunk[bh] (-1: done)
-// with the state entering it in handoff_state[bh].  y_raw != nullptr: fp32 y rows there.
-cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
-                                float* s_out, void* y, float* y_raw, int B, int T, int H, int* status,
-                                int* handoff_chunk, float* handoff_state, long long budget,
-                                cudaStream_t st);
+// Sequence split.  Every (b,h) sequence is cut into P segments of seg_chunks 64-token
+// chunks (the last one may be shorter); the kernels below run one CTA per unit
+// u = p * (B*H) + bh.  The state entering segment p > 0 is s_mid[bh][p-1] ([D][D] fp32),
+// computed beforehand by launch_segment_states + launch_segment_carry.  P = 1: no split.
+struct Segments {
+    int P;
+    int seg_chunks;
+    const float* s_mid;
+};
 
-// Level-factorised path (any decay).  start_chunk == nullptr: every (b,h) from chunk 0 with
-// state s_in; otherwise (b,h) resumes at start_chunk[bh] (skipped if < 0) from
-// handoff_state.  status: device word set to 1 if a bounded wait expired.
+// State of each segment p < P-1 from a zero initial state, s_loc[bh][p] ([D][D]), and its
+// log2 decay sum[bh][p][i] = log2 prod_{t in segment} w_t[i]; chunked on tcgen05 with the
+// suffix factorisation (factors <= 1: no overflow for any decay).  maps: r, k, v, omega.
+cudaError_t launch_segment_states(const CUtensorMap* maps, float* s_loc, float* log2g, int B,
+                                  int T, int H, Segments seg, int* status, long long budget,
+                                  cudaStream_t st);
+// s_mid[bh][p] = 2^log2g[bh][p] (rows) * s_in(p) + s_loc[bh][p], p = 0 .. P-2, in order, where
+// s_in(0) = state_in (zero if null) and s_in(p) = s_mid[bh][p-1]; s_mid may alias s_loc.
+cudaError_t launch_segment_carry(const float* state_in, const float* s_loc, const float* log2g,
+                                 float* s_mid, int B, int H, int P, cudaStream_t st);
+
+// Fast path (one-sided decay factorisation, warp-specialised pipeline).  maps: r, k, v,
+// omega.  For each unit it writes y (and, in the last segment, the final state), or stops at
+// the first chunk whose decay range it cannot take and records that chunk (absolute index)
+// in handoff_chunk[u] (-1: done) with the state entering it in handoff_state[u].
+// y_raw != nullptr: fp32 y rows there instead of y.
+cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
+                                float* s_out, void* y, float* y_raw, int B, int T, int H,
+                                Segments seg, int* status, int* handoff_chunk,
+                                float* handoff_state, long long budget, cudaStream_t st);
+
+// Level-factorised path (any decay).  start_chunk == nullptr: every unit from its first
+// chunk with its incoming state; otherwise unit u resumes at chunk start_chunk[u] (skipped if
+// < 0) from handoff_state[u].  status: device word set to 1 if a bounded wait expired.
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
-                                  float* s_out, float* y_raw, int B, int T, int H, int* status,
-                                  const int* start_chunk, const float* handoff_state,
-                                  long long spin_budget, cudaStream_t st);
+                                  float* s_out, float* y_raw, int B, int T, int H, Segments seg,
+                                  int* status, const int* start_chunk,
+                                  const float* handoff_state, long long spin_budget,
+                                  cudaStream_t st);
 size_t chunked_smem_bytes();
 size_t fast_smem_bytes();
+size_t segment_smem_bytes();
 
 }  // namespace goldwkv

@@ -157,6 +157,65 @@ def test_isolated_extreme_chunk(oracle):
         assert rel_err(s, so) <= TOL[torch.bfloat16], algo
 
 
+# ----------------------------------------------------------------------------- sequence split
+def _small(seed, B, T, H):
+    inp = W.make_prefill_inputs(W.CONFIGS[1].with_(seed=seed), DEV, B=B, T=T)
+    for n in ("r", "k", "v", "omega"):
+        inp[n] = inp[n][:, :, :H].contiguous()
+    inp["u"], inp["state0"] = inp["u"][:H].contiguous(), inp["state0"][:, :H].contiguous()
+    return inp
+
+
+@pytest.mark.parametrize("P", [2, 3, 6])
+@pytest.mark.parametrize("case", ["mild", "zero_state", "handoff_late", "ragged"])
+def test_sequence_split(oracle, monkeypatch, P, case):
+    """Segments of one sequence on different CTAs: the state pre-pass and carry give each
+    segment its incoming state; the result must match the unsplit oracle run."""
+    monkeypatch.setenv("GOLDWKV_SEGMENTS", str(P))
+    T = {"ragged": 1001}.get(case, 1024)
+    inp = _small(7700 + P, B=2, T=T, H=3)
+    if case == "handoff_late":   # an extreme chunk inside a later segment
+        om = inp["omega"].float()
+        om[:, 830:900, 1, 5] = 6.0
+        inp["omega"] = om.to(torch.bfloat16)
+    state = case != "zero_state"
+    nc = (T + 63) // 64
+    seg = (nc + P - 1) // P
+    hand = lambda units: 256 + ((units * 4 + 255) // 256) * 256 + units * 16384
+    assert gw.prefill_workspace_bytes(2, T, 3, 64, torch.bfloat16, False) == \
+        hand(6 * P) + 6 * (P - 1) * (4096 + 64) * 4, "the split was not taken"
+    assert (P - 1) * seg < nc
+    y, s = _run(inp, "chunked", state=state)
+    yo, so = _oracle_full(oracle, inp, state=state)
+    assert rel_err(y, yo) <= TOL[torch.bfloat16]
+    assert rel_err(s, so) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("omega_value", [-60.0, 30.0])
+def test_sequence_split_saturated_decay(oracle, monkeypatch, omega_value):
+    """w = 1 everywhere (segment decay product 1: the whole state carries) and w = 0 (the
+    product underflows to 0: nothing carries)."""
+    monkeypatch.setenv("GOLDWKV_SEGMENTS", "4")
+    inp = _small(7800, B=1, T=1280, H=2)
+    inp["omega"] = torch.full_like(inp["v"], omega_value)
+    y, s = _run(inp, "chunked")
+    yo, so = _oracle_full(oracle, inp)
+    assert rel_err(y, yo) <= TOL[torch.bfloat16]
+    assert rel_err(s, so) <= TOL[torch.bfloat16]
+
+
+def test_sequence_split_matches_unsplit(monkeypatch):
+    """Split and unsplit runs of the same problem agree to the tolerance (they differ only
+    in rounding order)."""
+    inp = _small(7810, B=2, T=2048, H=4)
+    y1, s1 = _run(inp, "chunked")
+    monkeypatch.setenv("GOLDWKV_SEGMENTS", "4")
+    y4, s4 = _run(inp, "chunked")
+    dy = (y1.float() - y4.float()).abs().max().item() / y1.float().abs().max().item()
+    ds = (s1 - s4).abs().max().item() / s1.abs().max().item()
+    assert dy <= TOL[torch.bfloat16] and ds <= TOL[torch.bfloat16], (dy, ds)
+
+
 def test_deterministic():
     cfg = W.CONFIGS[1].with_(seed=7600)
     inp = W.make_prefill_inputs(cfg, DEV, B=2, T=300)
