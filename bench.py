@@ -61,8 +61,9 @@ def decode_bytes(B, H, D=64, esz=2):
 # from; reported only while the sources still hash to that value (else null).
 CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
-    "prefill": {"sources": ("chunked_fast_sm100.cu", "sm100_ptx.cuh", "common.cuh", "internal.h"),
-                "sha256_16": "05b71e9b6aaf3768", "bytes": 541236224 + 120360704,
+    "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
+                            "internal.h"),
+                "sha256_16": "c4103f1785484646", "bytes": 541242368 + 121432320,
                 "workload": (8, 4096, 32),
                 "profile": "profiles/wkv6_fast_kernel_prefill_B8_T4096_H32_bf16.md"},
     "decode": {"sources": ("decode.cu", "common.cuh"),
