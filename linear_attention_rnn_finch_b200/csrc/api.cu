@@ -98,11 +98,15 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kChunk = 64;          // tokens per chunk of the chunked kernels
 constexpr int kSmCount = 148;       // SMs of a B200: the unit of a wave of CTAs
 constexpr int kMinSegChunks = 16;   // shortest segment worth a CTA
-// Cost of the state pre-pass per chunk relative to the full prefill per chunk (it reads
-// k, v, omega and runs the state update only).
-constexpr double kPrePassCost = 0.5;
+// The state pre-pass runs two CTAs per SM; its time per chunk and wave of those slots,
+// relative to the main prefill's per chunk and wave (one CTA per SM), measured on B200.
+constexpr int kPrePassCtasPerSm = 2;
+constexpr double kPrePassCost = 0.62;
 
-long waves(long ctas) { return (ctas + kSmCount - 1) / kSmCount; }
+long waves(long ctas, int per_sm = 1) {
+    const long slots = (long)kSmCount * per_sm;
+    return (ctas + slots - 1) / slots;
+}
 
 // Segments per sequence on the chunked path.  One CTA runs each (b,h) segment; the split
 // pays when B*H alone leaves SMs idle: estimated time = waves of the main pass x chunks per
@@ -123,7 +127,8 @@ int choose_segments(int B, int T, int H) {
         const int seg = (nc + P - 1) / P;
         if (seg < kMinSegChunks) break;
         if (!feasible(P)) continue;
-        const double t = (double)waves(nbh * P) * seg + kPrePassCost * (double)waves(nbh * (P - 1)) * seg;
+        const double t = (double)waves(nbh * P) * seg +
+                         kPrePassCost * (double)waves(nbh * (P - 1), kPrePassCtasPerSm) * seg;
         if (t < 0.9 * best) {
             best = t;
             best_p = P;

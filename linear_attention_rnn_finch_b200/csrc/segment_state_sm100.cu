@@ -14,11 +14,12 @@
 //     S <- diag(gamma) S + Kt^T V,  gamma = prod_{tau in chunk} w_tau,
 // with the suffix sums accumulated directly (a sum of terms of one sign, not a difference
 // of prefix sums), so any decay -- down to w = 0 -- is exact to fp32 rounding.  Kt is split
-// into bf16 hi + lo parts; Kt^T V runs on tcgen05 as V^T (M=64) x [Kt_hi | Kt_lo] (N=128).
+// into bf16 hi + lo parts; Kt^T V runs on tcgen05 as V^T (M=64) x Kt_hi + V^T x Kt_lo
+// (N=64 each, accumulated in TMEM).
 //
-// Warp roles (576 threads): warp 0 TMA (k, v, omega; 3-stage ring) and TMEM owner;
-// warp 1 one MMA thread; warps 2-9 prep (8 tokens each); warps 10-17 the state update in
-// registers.  Every wait is bounded.
+// Warp roles (320 threads, two CTAs per SM): warp 0 TMA (k, v, omega; 3-stage ring) and TMEM
+// owner; warp 1 one MMA thread; warps 2-5 prep (16 tokens each); warps 6-9 the state update
+// in registers, one warp per TMEM sub-partition.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -35,14 +36,15 @@ using namespace tiles;
 
 constexpr int C = 64;
 constexpr int kStages = 3;
-constexpr int kPrepWarps = 8, kEpiWarps = 8;
+constexpr int kPrepWarps = 4, kEpiWarps = 4;
+constexpr int kTokPerWarp = C / kPrepWarps;   // 16
 constexpr int kTmaWarp = 0, kMmaWarp = 1, kPrepWarp0 = 2, kEpiWarp0 = kPrepWarp0 + kPrepWarps;
 constexpr int kPrepThreads = 32 * kPrepWarps, kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 32 * kPrepWarp0 + kPrepThreads + kEpiThreads;
-constexpr uint32_t kTmemCols = 256;   // DU: 2 buffers x 128 columns (M = 64)
+constexpr uint32_t kTmemCols = 128;   // DU: 2 buffers x 64 columns (M = 64)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kBarPrep = 1;
-constexpr uint32_t IDESC_GU = ptx::idesc_bf16(64, 128, 1, 1);
+constexpr uint32_t IDESC_GU = ptx::idesc_bf16(64, 64, 1, 1);
 
 struct __align__(1024) Smem {
     uint8_t in[kStages][3][kTile];   // k, v, omega tiles (TMA, 128B swizzle)
@@ -56,7 +58,7 @@ struct __align__(1024) Smem {
     int stop_at;                     // unused here (no hand-over); read by wait_soft
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_w, float* s_loc, float* log2g, int H,
                           int P, int seg_chunks, int* status, long long budget, long long drain_budget) {
@@ -125,9 +127,13 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 const uint32_t v_tile = ptx::smem_addr(s.in[st][1]);
                 const uint32_t kt = ptx::smem_addr(s.kt[pb]);
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // DU = V^T x [Kt_hi | Kt_lo]
-                    ptx::mma_bf16(tmem + 128 * pb, ptx::desc_sw128(v_tile + 2048 * kq, 1024),
-                                  ptx::desc_sw128(kt + 2048 * kq, kTile), IDESC_GU, kq > 0);
+                for (int kq = 0; kq < 4; ++kq)   // DU = V^T x Kt_hi + V^T x Kt_lo
+                    ptx::mma_bf16(tmem + 64 * pb, ptx::desc_mnmajor(v_tile + 2048 * kq),
+                                  ptx::desc_mnmajor(kt + 2048 * kq), IDESC_GU, kq > 0);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)
+                    ptx::mma_bf16(tmem + 64 * pb, ptx::desc_mnmajor(v_tile + 2048 * kq),
+                                  ptx::desc_mnmajor(kt + kTile + 2048 * kq), IDESC_GU, 1);
                 ptx::mma_commit(&s.gu_done[pb]);
                 ptx::mma_commit(&s.op_free[pb]);
                 ptx::mma_commit(&s.empty[st]);
@@ -136,14 +142,14 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             if (last >= 0) ptx::mbar_wait(&s.gu_done[last & 1], (uint32_t)((last >> 1) & 1), drain_budget);
         }
     } else if (warp < kEpiWarp0) {
-        // ------------------------------------------------------------ prep (8 warps)
-        // warp g: tokens 8g .. 8g+7; lane = channel pair (2l, 2l+1); log2 units
+        // ------------------------------------------------------------ prep (4 warps)
+        // warp g: tokens 16g .. 16g+15; lane = channel pair (2l, 2l+1); log2 units
         const int g = warp - kPrepWarp0;
         const int c2 = 2 * lane;
         const int chunk = lane >> 2;
         const uint32_t cbyte = (uint32_t)(lane & 3) * 4;
         const float2 l2e = make_float2(kLog2e, kLog2e);
-        float2 lg = make_float2(0.f, 0.f);   // sum of log2 w over the segment (warp 0)
+        float2 lg = make_float2(0.f, 0.f);   // -sum of log2 w over the segment (warp 0)
         for (int n = 0; n < NC; ++n) {
             const int pb = n & 1, st = n % kStages;
             bool ok = wait_soft(s, &s.full[st], (uint32_t)((n / kStages) & 1), budget);
@@ -154,25 +160,17 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             if (named_bar_any(kBarPrep, kPrepThreads, !ok || ld_volatile(&s.abort))) break;
             const uint8_t* k_tile = s.in[st][0];
             const uint8_t* w_tile = s.in[st][2];
-            // -log2 w = exp(omega) log2(e) per token; suffix sums inside the warp's 8 tokens
-            float2 e[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float2 om = __fmul2_rn(unpack2(lds32(w_tile, sw_off(8 * g + q, chunk) + cbyte)), l2e);
-                e[q] = __fmul2_rn(make_float2(fast_exp2(om.x), fast_exp2(om.y)), l2e);
-            }
-            float2 suf[8];                    // -sum_{q' > q} (log2 w) within the warp
+            // -log2 w = exp(omega) log2(e); exclusive suffix sums inside the warp's tokens,
+            // accumulated from the last token down (terms of one sign)
+            float2 suf[kTokPerWarp];
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int q = 7; q >= 0; --q) {
+            for (int q = kTokPerWarp - 1; q >= 0; --q) {
+                const float2 om = __fmul2_rn(unpack2(lds32(w_tile, sw_off(kTokPerWarp * g + q, chunk) + cbyte)), l2e);
                 suf[q] = acc;
-                acc = __fadd2_rn(acc, e[q]);
+                acc = __ffma2_rn(make_float2(fast_exp2(om.x), fast_exp2(om.y)), l2e, acc);
             }
             *reinterpret_cast<float2*>(&s.qtot[pb][g][c2]) = acc;   // -sum of the warp's log2 w
-            uint32_t kw[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) kw[q] = lds32(k_tile, sw_off(8 * g + q, chunk) + cbyte);
-            mbar_arrive(&s.empty[st]);       // k and omega of this stage read
             named_bar(kBarPrep, kPrepThreads);
             float2 after = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
 #pragma unroll
@@ -184,15 +182,16 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             uint8_t* kt_hi = s.kt[pb];
             uint8_t* kt_lo = s.kt[pb] + kTile;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < kTokPerWarp; ++q) {
+                const uint32_t o = sw_off(kTokPerWarp * g + q, chunk) + cbyte;
                 const float2 x = __fadd2_rn(after, suf[q]);          // >= 0
                 const float2 f = make_float2(fast_exp2(-x.x), fast_exp2(-x.y));
                 uint32_t hi, lo;
-                split2(__fmul2_rn(unpack2(kw[q]), f), hi, lo);
-                const uint32_t o = sw_off(8 * g + q, chunk) + cbyte;
+                split2(__fmul2_rn(unpack2(lds32(k_tile, o)), f), hi, lo);
                 sts32(kt_hi, o, hi);
                 sts32(kt_lo, o, lo);
             }
+            mbar_arrive(&s.empty[st]);       // k and omega of this stage read
             if (g == 0) {
                 *reinterpret_cast<float2*>(&s.gamma[pb][c2]) = make_float2(fast_exp2(-tot.x), fast_exp2(-tot.y));
                 lg = __fadd2_rn(lg, tot);
@@ -203,16 +202,16 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         if (g == 0 && !ld_volatile(&s.abort))
             *reinterpret_cast<float2*>(log2g + out_idx * 64 + c2) = make_float2(-lg.x, -lg.y);
     } else {
-        // ------------------------------------------------------------ state (8 warps)
-        // warp (q, ch): rows j = 16q + l/4 and +8 of S^T, columns i = 32ch + 8k + 2(l%4) + {0,1}
+        // ------------------------------------------------------------ state (4 warps)
+        // warp q = warp % 4 (its TMEM sub-partition): rows j = 16q + l/4 and +8 of S^T,
+        // columns i = 32h + 8k + 2(l%4) + {0,1} for column halves h = 0, 1
         const int q = warp & 3;
-        const int ch = (warp - kEpiWarp0) >> 2;
         const int r0 = 16 * q + (lane >> 2), r1 = r0 + 8;
-        const int cbase = 32 * ch + 2 * (lane & 3);
+        const int cl = 2 * (lane & 3);
         const uint32_t lane_h0 = (uint32_t)(32 * q) << 16;
-        float2 S0[4], S1[4];
+        float2 S0[8], S1[8];   // index 4h + k
 #pragma unroll
-        for (int k = 0; k < 4; ++k) S0[k] = S1[k] = make_float2(0.f, 0.f);
+        for (int k = 0; k < 8; ++k) S0[k] = S1[k] = make_float2(0.f, 0.f);
         int n = 0;
         for (; n < NC; ++n) {
             const int pb = n & 1;
@@ -222,28 +221,27 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 break;   // abort: every later wait returns at once as well
             ptx::tc_fence_after();
             uint32_t ua[16], ub[16];
-            tmem_ld16x4(tmem + lane_h0 + 128 * pb + 32 * ch, ua);
-            tmem_ld16x4(tmem + lane_h0 + 128 * pb + 64 + 32 * ch, ub);
+            tmem_ld16x4(tmem + lane_h0 + 64 * pb, ua);
+            tmem_ld16x4(tmem + lane_h0 + 64 * pb + 32, ub);
             ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             mbar_arrive(&s.du_free[pb]);
-            float2 gv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) gv[k] = *reinterpret_cast<const float2*>(&s.gamma[pb][cbase + 8 * k]);
-            mbar_arrive(&s.ep_free[pb]);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float2 du0 = __fadd2_rn(lo_pair(ua, k), lo_pair(ub, k));
-                const float2 du1 = __fadd2_rn(hi_pair(ua, k), hi_pair(ub, k));
-                S0[k] = __ffma2_rn(gv[k], S0[k], du0);
-                S1[k] = __ffma2_rn(gv[k], S1[k], du1);
+                const float2 g0 = *reinterpret_cast<const float2*>(&s.gamma[pb][cl + 8 * k]);
+                const float2 g1 = *reinterpret_cast<const float2*>(&s.gamma[pb][32 + cl + 8 * k]);
+                S0[k] = __ffma2_rn(g0, S0[k], lo_pair(ua, k));
+                S1[k] = __ffma2_rn(g0, S1[k], hi_pair(ua, k));
+                S0[4 + k] = __ffma2_rn(g1, S0[4 + k], lo_pair(ub, k));
+                S1[4 + k] = __ffma2_rn(g1, S1[4 + k], hi_pair(ub, k));
             }
+            mbar_arrive(&s.ep_free[pb]);
         }
         if (n == NC && !ld_volatile(&s.abort)) {
             float* dst = s_loc + out_idx * 4096;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = cbase + 8 * k;
+            for (int k = 0; k < 8; ++k) {
+                const int i = 32 * (k >> 2) + cl + 8 * (k & 3);
                 dst[i * 64 + r0] = S0[k].x;
                 dst[(i + 1) * 64 + r0] = S0[k].y;
                 dst[i * 64 + r1] = S1[k].x;
