@@ -67,6 +67,10 @@ class Oracle:
         lib.wkv6_oracle_decode_step.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                 dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
         lib.wkv6_oracle_decode_step.restype = ctypes.c_int
+        lib.wkv6c2_oracle_prefill.argtypes = lib.wkv6_oracle_prefill.argtypes
+        lib.wkv6c2_oracle_prefill.restype = ctypes.c_int
+        lib.wkv6c2_oracle_decode_step.argtypes = lib.wkv6_oracle_decode_step.argtypes
+        lib.wkv6c2_oracle_decode_step.restype = ctypes.c_int
         lib.wkv6_oracle_layernorm.argtypes = [ctypes.c_long, ctypes.c_int, dp, dp, dp,
                                               ctypes.c_double, dp]
         lib.wkv6_oracle_layernorm.restype = ctypes.c_int
@@ -117,6 +121,42 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle decode failed rc={rc}")
         return y, st
+
+    def prefill_c2(self, r, k, v, omega, uprime, state_in=None, nthreads: int | None = None):
+        """Finch-C2 exact form: key k (1 - w), second value uprime [B,T,H,D] added to the
+        readout (no static bonus).  Same shapes and returns as prefill."""
+        r, k, v, omega, up = (self._f64(x) for x in (r, k, v, omega, uprime))
+        B, T, H, D = r.shape
+        s_in = None if state_in is None else self._f64(state_in)
+        y = np.empty_like(r)
+        s_out = np.empty((B, H, D, D), dtype=np.float64)
+        rc = self._lib.wkv6c2_oracle_prefill(B, T, H, D, self._ptr(r), self._ptr(k), self._ptr(v),
+                                             self._ptr(omega), self._ptr(up), self._ptr(s_in),
+                                             self._ptr(y), self._ptr(s_out),
+                                             nthreads or default_threads())
+        if rc != 0:
+            raise RuntimeError(f"oracle C2 prefill failed rc={rc}")
+        return y, s_out
+
+    def decode_step_c2(self, r, k, v, omega, uprime, state, nthreads: int | None = None):
+        """Finch-C2 step: r,k,v,omega,uprime [B,H,D]; state [B,H,D,D] (not modified)."""
+        r, k, v, omega, up = (self._f64(x) for x in (r, k, v, omega, uprime))
+        st = np.array(state, dtype=np.float64, copy=True, order="C")
+        B, H, D = r.shape
+        y = np.empty_like(r)
+        rc = self._lib.wkv6c2_oracle_decode_step(B, H, D, self._ptr(r), self._ptr(k), self._ptr(v),
+                                                 self._ptr(omega), self._ptr(up), self._ptr(st),
+                                                 self._ptr(y), nthreads or default_threads())
+        if rc != 0:
+            raise RuntimeError(f"oracle C2 decode failed rc={rc}")
+        return y, st
+
+    def prefill_c2_ln(self, r, k, v, omega, uprime, state_in, gamma, beta, eps=1e-5, nthreads=None):
+        """Finch-C2 prefill followed by LayerNorm over the concatenated heads."""
+        y, s = self.prefill_c2(r, k, v, omega, uprime, state_in, nthreads)
+        B, T, H, D = y.shape
+        yl = self.layernorm(y.reshape(B, T, H * D), gamma, beta, eps).reshape(B, T, H, D)
+        return yl, s, y
 
     def layernorm(self, x, gamma=None, beta=None, eps: float = 1e-5):
         """LayerNorm over the last axis of x (any leading shape), fp64."""

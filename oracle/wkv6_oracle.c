@@ -5,13 +5,16 @@
  * shares no code, header or constant with it.
  *
  * Source of the definition: "GoldFinch: High Performance RWKV/Transformer Hybrid ..."
- * (paper-graph-ui review page), section 3.4, "Finch-C2 Time Mixing":
+ * review page (mlsanity.com), section 3.4, "Finch-C2 Time Mixing":
  *   - data-dependent decay        w_t = exp(-exp(d_t))             ("Data-dependent decay")
  *   - recurrent state             wkv_t = sum_{i<t} diag(prod_{j=i+1}^{t-1} w_j) k_i^T v_i
  *                                                                 ("Recurrent state update and output")
  *   - readout                     r_t . wkv_t  plus the base-Finch static bonus u
  *                                 (the bonus enters as r_t . diag(u) k_t^T v_t)
  *   - LayerNorm over the concatenation of all heads                ("... full concatenated dimension")
+ *   - Finch-C2's exact form (wkv6c2_*): key k_t (1 - w_t), second value u'_t added to the
+ *     readout instead of the static bonus              ("Key computation with normalization
+ *                                                        property", "the new second value")
  * Written in recursive form: with S_{-1} = state_in (zero if absent),
  *   y_t[j] = sum_i r_t[i] S_{t-1}[i][j] + (sum_i r_t[i] u[i] k_t[i]) v_t[j]
  *   S_t[i][j] = w_t[i] S_{t-1}[i][j] + k_t[i] v_t[j]
@@ -80,10 +83,63 @@ static void wkv6_one_head(long T, int D, long tstride,
                 s_out[i * D + j] = S[i * D + j];
 }
 
+/* Finch-C2 exact time mixing, one (b,h) sequence.  Same state and decay as above, with the
+ * two changes of the page's Finch-C2 ("Key computation with normalization property" and
+ * "Receptance, value, and the new second value"):
+ *   - the key enters the state multiplied by (1 - w_t):  S_t = diag(w_t) S_{t-1} + (k_t (1 - w_t))^T v_t
+ *   - no static bonus; a data-dependent second value u'_t is added to the readout:
+ *     y_t = r_t . S_{t-1} + u'_t
+ * u'_t (uprime) is token-major like y. */
+static void wkv6c2_one_head(long T, int D, long tstride,
+                            const double *r, const double *k, const double *v,
+                            const double *omega, const double *uprime,
+                            const double *s_in, double *y, double *s_out, double *S,
+                            double *w)
+{
+    for (int i = 0; i < D; ++i)
+        for (int j = 0; j < D; ++j)
+            S[i * D + j] = (s_in != NULL) ? s_in[i * D + j] : 0.0;
+
+    for (long t = 0; t < T; ++t) {
+        const double *rt = r + t * tstride;
+        const double *kt = k + t * tstride;
+        const double *vt = v + t * tstride;
+        const double *ot = omega + t * tstride;
+        const double *ut = uprime + t * tstride;
+        double *yt = y + t * tstride;
+
+        for (int i = 0; i < D; ++i) {
+            const double decay = exp(-exp(ot[i]));   /* w_t of this token */
+            w[i] = decay;
+        }
+
+        /* readout from the state before this token, plus the second value */
+        for (int j = 0; j < D; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < D; ++i)
+                acc += S[i * D + j] * rt[i];
+            yt[j] = acc + ut[j];
+        }
+
+        /* state update with the normalised key k_t (1 - w_t) */
+        for (int i = 0; i < D; ++i) {
+            const double kn = kt[i] * (1.0 - w[i]);
+            for (int j = 0; j < D; ++j)
+                S[i * D + j] = w[i] * S[i * D + j] + kn * vt[j];
+        }
+    }
+
+    if (s_out)
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                s_out[i * D + j] = S[i * D + j];
+}
+
 typedef struct {
     int B, H, D;
     long T;
     const double *r, *k, *v, *omega, *u, *s_in;
+    const double *uprime;   /* Finch-C2 second value [B][T][H][D], or NULL (base Finch) */
     double *y, *s_out;
     int next;               /* next (b*H+h) unit to take */
     pthread_mutex_t lock;
@@ -110,13 +166,44 @@ static void *worker(void *arg)
         long tstride = (long)J->H * D;
         size_t x0 = ((size_t)b * J->T * J->H + h) * D;      /* element (b, t=0, h, 0) */
         size_t s0 = ((size_t)b * J->H + h) * D * D;
-        wkv6_one_head(J->T, D, tstride, J->r + x0, J->k + x0, J->v + x0, J->omega + x0,
-                      J->u + (size_t)h * D, J->s_in ? J->s_in + s0 : NULL, J->y + x0,
-                      J->s_out ? J->s_out + s0 : NULL, S, w);
+        if (J->uprime)
+            wkv6c2_one_head(J->T, D, tstride, J->r + x0, J->k + x0, J->v + x0, J->omega + x0,
+                            J->uprime + x0, J->s_in ? J->s_in + s0 : NULL, J->y + x0,
+                            J->s_out ? J->s_out + s0 : NULL, S, w);
+        else
+            wkv6_one_head(J->T, D, tstride, J->r + x0, J->k + x0, J->v + x0, J->omega + x0,
+                          J->u + (size_t)h * D, J->s_in ? J->s_in + s0 : NULL, J->y + x0,
+                          J->s_out ? J->s_out + s0 : NULL, S, w);
     }
     free(S);
     free(w);
     return NULL;
+}
+
+static int run_units(job_t *J, int nthreads)
+{
+    J->next = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    if (nthreads > J->B * J->H)
+        nthreads = J->B * J->H;
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    int started = 0, rc = 0;
+    for (int n = 0; n < nthreads; ++n) {
+        if (pthread_create(&tid[n], NULL, worker, J) != 0) {
+            rc = -2;
+            break;
+        }
+        ++started;
+    }
+    for (int n = 0; n < started; ++n) {
+        void *ret = NULL;
+        pthread_join(tid[n], &ret);
+        if (ret)
+            rc = -2;
+    }
+    free(tid);
+    pthread_mutex_destroy(&J->lock);
+    return rc;
 }
 
 /* Full prefill over [B][T][H][D] inputs.  state_in may be NULL (zeros); state_out may be
@@ -134,29 +221,27 @@ int wkv6_oracle_prefill(int B, long T, int H, int D,
     job_t J;
     J.B = B; J.T = T; J.H = H; J.D = D;
     J.r = r; J.k = k; J.v = v; J.omega = omega; J.u = u; J.s_in = state_in;
+    J.uprime = NULL;
     J.y = y; J.s_out = state_out;
-    J.next = 0;
-    pthread_mutex_init(&J.lock, NULL);
-    if (nthreads > B * H)
-        nthreads = B * H;
-    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
-    int started = 0, rc = 0;
-    for (int n = 0; n < nthreads; ++n) {
-        if (pthread_create(&tid[n], NULL, worker, &J) != 0) {
-            rc = -2;
-            break;
-        }
-        ++started;
-    }
-    for (int n = 0; n < started; ++n) {
-        void *ret = NULL;
-        pthread_join(tid[n], &ret);
-        if (ret)
-            rc = -2;
-    }
-    free(tid);
-    pthread_mutex_destroy(&J.lock);
-    return rc;
+    return run_units(&J, nthreads);
+}
+
+/* Finch-C2 prefill (see wkv6c2_one_head): uprime [B][T][H][D] replaces u. */
+int wkv6c2_oracle_prefill(int B, long T, int H, int D,
+                          const double *r, const double *k, const double *v,
+                          const double *omega, const double *uprime, const double *state_in,
+                          double *y, double *state_out, int nthreads)
+{
+    if (B < 0 || T < 0 || H < 0 || D <= 0 || nthreads <= 0 || (!uprime && T > 0 && B > 0 && H > 0))
+        return -1;
+    if (B == 0 || H == 0)
+        return 0;
+    job_t J;
+    J.B = B; J.T = T; J.H = H; J.D = D;
+    J.r = r; J.k = k; J.v = v; J.omega = omega; J.u = NULL; J.s_in = state_in;
+    J.uprime = uprime;
+    J.y = y; J.s_out = state_out;
+    return run_units(&J, nthreads);
 }
 
 /* One autoregressive step (T = 1) for every (b,h), state updated in place.
@@ -167,6 +252,15 @@ int wkv6_oracle_decode_step(int B, int H, int D,
                             double *y, int nthreads)
 {
     return wkv6_oracle_prefill(B, 1, H, D, r, k, v, omega, u, state, y, state, nthreads);
+}
+
+/* Finch-C2 autoregressive step, state updated in place. */
+int wkv6c2_oracle_decode_step(int B, int H, int D,
+                              const double *r, const double *k, const double *v,
+                              const double *omega, const double *uprime, double *state,
+                              double *y, int nthreads)
+{
+    return wkv6c2_oracle_prefill(B, 1, H, D, r, k, v, omega, uprime, state, y, state, nthreads);
 }
 
 /* LayerNorm of each of the N rows of x[N][C] over its C entries:

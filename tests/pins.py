@@ -23,6 +23,16 @@ or from mathematics that the definition fixes:
 * ln_torch          - LayerNorm equals torch.nn.functional.layer_norm in fp64;
 * ln_shift          - LayerNorm is invariant to adding a constant to every channel.
 
+Finch-C2's exact form (key k_t (1 - w_t), second value u'_t instead of the static bonus;
+section 3.4 "Key computation with normalization property" and "the new second value"):
+
+* c2_explicit_sum   - the explicit sum with the normalised keys, brute force, plus u'_t;
+* c2_normalised_rows- the property the page gives for k (1 - w): with k = v = 1 and every
+                      state row starting at 1, each row stays exactly 1 for any decays
+                      (S_t = w S_{t-1} + (1 - w) 1), so y_t = sum_i r_t[i] + u'_t;
+* c2_second_value   - y is affine in u' with unit slope and the state does not see u';
+* c2_decode         - the decode step's closed form with the normalised key.
+
 ``run_all(oracle)`` returns the list of failing pin names; the mutation test uses it to
 show that plausible mistakes planted in the oracle are caught.
 """
@@ -233,6 +243,53 @@ def pin_ln_shift(o):
     return _close(a, b, 1e-10)
 
 
+def pin_c2_explicit_sum(o):
+    ok = True
+    for seed, (B, T, H, D), s0 in [(11, (2, 8, 2, 8), True), (12, (1, 6, 1, 64), False)]:
+        r, k, v, om, _, S0 = _inputs(seed, B, T, H, D, s0=s0)
+        up = _rng(seed + 100).normal(0, 0.3, r.shape)
+        y, S = o.prefill_c2(r, k, v, om, up, S0)
+        w = np.exp(-np.exp(om))
+        kn = k * (1.0 - w)                       # the normalised key of each token
+        ye, Se = brute_force_explicit(r, kn, v, om, np.zeros((H, D)), S0)
+        ok &= _close(y, ye + up) and _close(S, Se)
+    return ok
+
+
+def pin_c2_normalised_rows(o):
+    g = _rng(13)
+    B, T, H, D = 1, 40, 2, 16
+    r = g.normal(0, 0.3, (B, T, H, D))
+    om = g.uniform(-8.0, 3.0, (B, T, H, D))
+    ones = np.ones((B, T, H, D))
+    up = g.normal(0, 0.3, (B, T, H, D))
+    S0 = np.ones((B, H, D, D))
+    y, S = o.prefill_c2(r, ones, ones, om, up, S0)
+    y_ref = r.sum(axis=-1, keepdims=True) + up
+    return _close(S, np.ones_like(S), 1e-13) and _close(y, y_ref, 1e-12)
+
+
+def pin_c2_second_value(o):
+    r, k, v, om, _, S0 = _inputs(14, 2, 20, 2, 8)
+    up = _rng(15).normal(0, 1.0, r.shape)
+    y0, S0_ = o.prefill_c2(r, k, v, om, np.zeros_like(r), S0)
+    y1, S1_ = o.prefill_c2(r, k, v, om, up, S0)
+    return _close(y1 - y0, up) and np.array_equal(S0_, S1_)
+
+
+def pin_c2_decode(o):
+    g = _rng(16)
+    B, H, D = 3, 2, 64
+    r, k, v, up = (g.normal(0, 0.3, (B, H, D)) for _ in range(4))
+    om = g.uniform(-6, 2, (B, H, D))
+    S0 = g.normal(0, 0.1, (B, H, D, D))
+    y, S = o.decode_step_c2(r, k, v, om, up, S0)
+    w = np.exp(-np.exp(om))
+    y_ref = np.einsum("bhi,bhij->bhj", r, S0) + up
+    S_ref = w[..., None] * S0 + (k * (1.0 - w))[..., :, None] * v[..., None, :]
+    return _close(y, y_ref) and _close(S, S_ref)
+
+
 PINS = {
     "explicit_sum": pin_explicit_sum,
     "t1_closed_form": pin_t1_closed_form,
@@ -245,6 +302,10 @@ PINS = {
     "ln_moments": pin_ln_moments,
     "ln_torch": pin_ln_torch,
     "ln_shift": pin_ln_shift,
+    "c2_explicit_sum": pin_c2_explicit_sum,
+    "c2_normalised_rows": pin_c2_normalised_rows,
+    "c2_second_value": pin_c2_second_value,
+    "c2_decode": pin_c2_decode,
 }
 
 

@@ -41,6 +41,14 @@ MUTANTS = {
     "ln_eps_outside": ("double inv = 1.0 / sqrt(var + eps);", "double inv = 1.0 / (sqrt(var) + eps);"),
     "ln_beta_dropped": ("orow[c] = (xr[c] - mean) * inv * g + bb;", "orow[c] = (xr[c] - mean) * inv * g;"),
     "ln_mean_kept": ("orow[c] = (xr[c] - mean) * inv * g + bb;", "orow[c] = xr[c] * inv * g + bb;"),
+    # Finch-C2 exact form
+    "c2_key_not_normalised": ("const double kn = kt[i] * (1.0 - w[i]);", "const double kn = kt[i];"),
+    "c2_key_scaled_by_w": ("const double kn = kt[i] * (1.0 - w[i]);", "const double kn = kt[i] * w[i];"),
+    "c2_second_value_dropped": ("yt[j] = acc + ut[j];", "yt[j] = acc;"),
+    "c2_second_value_on_state": ("S[i * D + j] = w[i] * S[i * D + j] + kn * vt[j];",
+                                 "S[i * D + j] = w[i] * S[i * D + j] + kn * vt[j] + ut[j];"),
+    "c2_decay_after_update": ("S[i * D + j] = w[i] * S[i * D + j] + kn * vt[j];",
+                              "S[i * D + j] = w[i] * (S[i * D + j] + kn * vt[j]);"),
 }
 
 
