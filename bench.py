@@ -196,11 +196,15 @@ def sum_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def other_prefill(cfg, dev, world, hbm, algo, steps):
+def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False):
     """Device-timed prefill calls of another workload shape: one line of its own (tokens/s and
-    the fraction of the HBM roofline), inputs resident in HBM and larger than L2."""
+    the fraction of the HBM roofline), inputs resident in HBM and larger than L2.  c2: the
+    Finch-C2 entry point (normalised key, second value u' read in place of the bonus)."""
     import linear_attention_rnn_finch_b200 as gw
     inp = W.make_prefill_inputs(cfg, dev)
+    if c2:
+        g = torch.Generator(device=dev).manual_seed(cfg.seed + 5)
+        inp["uprime"] = (torch.randn(inp["r"].shape, generator=g, device=dev) * 0.125).to(cfg.dtype)
     B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
     ln = (inp["gamma"], inp["beta"], inp["eps"]) if cfg.ln else None
     ws = gw.new_workspace(gw.prefill_workspace_bytes(B, T, H, D, cfg.dtype, ln is not None, algo), dev)
@@ -209,8 +213,12 @@ def other_prefill(cfg, dev, world, hbm, algo, steps):
     args_p = [inp[n] for n in ("r", "k", "v", "omega")]
 
     def call():
-        gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], ln=ln, y=y, state_out=s_out,
-                        algo=algo, workspace=ws)
+        if c2:
+            gw.wkv6c2_prefill(*args_p, inp["uprime"], inp["state0"], ln=ln, y=y, state_out=s_out,
+                              workspace=ws)
+        else:
+            gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], ln=ln, y=y, state_out=s_out,
+                            algo=algo, workspace=ws)
 
     for _ in range(3):
         call()
@@ -224,12 +232,14 @@ def other_prefill(cfg, dev, world, hbm, algo, steps):
     e1.record(stream)
     e1.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
-    nbytes = prefill_bytes(B, T, H, D)
+    nbytes = prefill_bytes(B, T, H, D) + (B * T * H * D * 2 if c2 else 0)   # + u' read
     # with LayerNorm the library also writes and re-reads an fp32 copy of y; the roofline
     # counts only the bytes the operation itself must move
     nbytes_note = ("LayerNorm runs as a second pass over an fp32 copy of y, not counted in the "
                    "algorithmic bytes") if cfg.ln else None
-    line = {"workload": cfg.name, "B": B, "T": T, "H": H, "D": D, "io": "bf16",
+    line = {"workload": ("wkv6c2_" + cfg.name[5:]) if c2 else cfg.name, "B": B, "T": T, "H": H,
+            "D": D, "io": "bf16", "form": "Finch-C2 (normalised key, second value)" if c2 else
+            "base Finch (static bonus)",
             "ln": bool(cfg.ln), "steps": steps, "ms_per_call": ms,
             "tokens_per_s": world * B * T / (ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm,
@@ -407,7 +417,9 @@ def run_ours(args, world, rank, local):
     # into segments across SMs) and the decay-extreme stress with fused LayerNorm
     if not args.no_other:
         out["other_prefill"] = [other_prefill(W.CONFIGS[2], dev, world, hbm, args.algo, steps=5),
-                                other_prefill(W.CONFIGS[4], dev, world, hbm, args.algo, steps=5)]
+                                other_prefill(W.CONFIGS[4], dev, world, hbm, args.algo, steps=5),
+                                other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
+                                              c2=True)]
 
     # end to end through the public API with host buffers
     if not args.no_e2e:

@@ -143,6 +143,33 @@ wkv_status wkv6_decode_step(const void *r, const void *k, const void *v, const v
                             wkv_dtype io, const wkv_ln *ln, void *workspace,
                             size_t workspace_bytes, void *stream);
 
+/*
+ * Finch-C2's exact time mixing (GoldFinch review page, section 3.4: "Key computation with
+ * normalization property" and "Receptance, value, and the new second value"; final output
+ * "LayerNorm(concat(r_t . wkv_t + u'_t))").  Against the recurrence at the top of this file,
+ * two things change:
+ *     S[i][j] = w_t[i] S[i][j] + k_t[i] (1 - w_t[i]) v_t[j]   (the key is normalised by 1 - w)
+ *     y_t[j]  = sum_i r_t[i] S[i][j] + u'_t[j]                  (no static bonus u; the second
+ *                                                                value u' is added instead)
+ * and LayerNorm, when requested, applies to that sum.  k is the key before the (1 - w)
+ * factor; the library forms 1 - w = -expm1(-exp(omega)) itself.
+ *
+ * wkv6c2_prefill: as wkv6_prefill (WKV_ALGO_AUTO, same workspace query, same layouts and
+ * errors) with `uprime` in place of `u`:
+ *   uprime  [B][T][H][D] io  the second value u'_t of every token; required when B, T, H > 0;
+ *           must not overlap y or the states.
+ */
+wkv_status wkv6c2_prefill(const void *r, const void *k, const void *v, const void *omega,
+                          const void *uprime, const float *state_in, float *state_out, void *y,
+                          int B, int T, int H, int D, wkv_dtype io, const wkv_ln *ln,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* wkv6c2_decode_step: as wkv6_decode_step with uprime [B][H][D] io in place of u. */
+wkv_status wkv6c2_decode_step(const void *r, const void *k, const void *v, const void *omega,
+                              const void *uprime, float *state, void *y, int B, int H, int D,
+                              wkv_dtype io, const wkv_ln *ln, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
 /* Size of the scratch array built into the library for wkv6_prefill_static, per device. */
 #define WKV6_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 

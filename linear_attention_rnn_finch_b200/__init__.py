@@ -6,8 +6,8 @@ does, and raises if it was not built.
 """
 from .binding import (WkvError, decode_workspace_bytes, load, new_workspace,
                       prefill_workspace_bytes, wkv6_decode_step, wkv6_prefill, wkv6_prefill_static,
-                      workspace_status)
+                      wkv6c2_decode_step, wkv6c2_prefill, workspace_status)
 
 __all__ = ["WkvError", "decode_workspace_bytes", "load", "new_workspace",
            "prefill_workspace_bytes", "wkv6_decode_step", "wkv6_prefill", "wkv6_prefill_static",
-           "workspace_status"]
+           "wkv6c2_decode_step", "wkv6c2_prefill", "workspace_status"]

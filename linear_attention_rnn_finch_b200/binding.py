@@ -56,6 +56,10 @@ def load(path: Path | str | None = None):
     L.wkv6_prefill_algo.restype = i
     L.wkv6_prefill_static.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp]
     L.wkv6_prefill_static.restype = i
+    L.wkv6c2_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+    L.wkv6c2_prefill.restype = i
+    L.wkv6c2_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
+    L.wkv6c2_decode_step.restype = i
     L.wkv6_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
     L.wkv6_decode_step.restype = i
     L.wkv6_workspace_status.argtypes = [vp, vp]
@@ -204,6 +208,74 @@ def wkv6_prefill_static(r, k, v, omega, u, state_in=None, *, ln=None, y=None, st
     del ln_s
     _raise("wkv6_prefill_static", st)
     return y, state_out
+
+
+def wkv6c2_prefill(r, k, v, omega, uprime, state_in=None, *, ln=None, y=None, state_out=None,
+                   want_state=True, workspace=None, stream=None):
+    """Finch-C2 exact form (include/goldwkv.h, wkv6c2_prefill): the key is normalised by
+    1 - w inside the library and the second value ``uprime`` [B, T, H, D] (dtype of r) is
+    added to the readout in place of the static bonus.  Returns (y, state_out)."""
+    L = load()
+    if r.dim() != 4:
+        raise ValueError("r must be [B, T, H, D]")
+    B, T, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega), ("uprime", uprime)):
+        _check(name, t, dev, dt, (B, T, H, D))
+    if state_in is not None:
+        _check("state_in", state_in, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, T, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, T, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _check("state_out", state_out, dev, torch.float32, (B, H, D, D))
+    ln_s, ln_p = _ln_struct(ln, H, D, dev)
+    need = int(L.wkv6_prefill_workspace_bytes(B, T, H, D, _io(dt), int(ln is not None), 0))
+    if workspace is None and need > 0:
+        workspace = new_workspace(need, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6c2_prefill(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(uprime), _ptr(state_in),
+                              _ptr(state_out), _ptr(y), B, T, H, D, _io(dt), ln_p, _ptr(workspace),
+                              ws_bytes, _stream_ptr(dev, stream))
+    del ln_s
+    _raise("wkv6c2_prefill", st)
+    return y, state_out
+
+
+def wkv6c2_decode_step(r, k, v, omega, uprime, state, *, ln=None, y=None, workspace=None,
+                       stream=None):
+    """Finch-C2 step over [B, H, D] inputs with second value ``uprime`` [B, H, D]; ``state``
+    is updated in place.  Returns y."""
+    L = load()
+    if r.dim() != 3:
+        raise ValueError("r must be [B, H, D]")
+    B, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega), ("uprime", uprime)):
+        _check(name, t, dev, dt, (B, H, D))
+    _check("state", state, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, H, D))
+    ln_s, ln_p = _ln_struct(ln, H, D, dev)
+    need = int(L.wkv6_decode_workspace_bytes(B, H, D, _io(dt), int(ln is not None)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6c2_decode_step(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(uprime), _ptr(state),
+                                  _ptr(y), B, H, D, _io(dt), ln_p, _ptr(workspace), ws_bytes,
+                                  _stream_ptr(dev, stream))
+    del ln_s
+    _raise("wkv6c2_decode_step", st)
+    return y
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:

@@ -185,11 +185,18 @@ size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_l
     return 0;
 }
 
-wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const void* omega,
-                             const float* u, const float* state_in, float* state_out, void* y,
-                             int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
-                             wkv_algo algo, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by the base (static bonus u) and the Finch-C2 (second value uprime) entry points:
+// exactly one of u / uprime is used, selected by uprime != nullptr.
+wkv_status prefill_impl(const void* r, const void* k, const void* v, const void* omega,
+                        const float* u, const void* uprime, const float* state_in,
+                        float* state_out, void* y, int B, int T, int H, int D, wkv_dtype io,
+                        const wkv_ln* ln, wkv_algo algo, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    const bool c2 = uprime != nullptr;
     if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
     if (algo != WKV_ALGO_AUTO && algo != WKV_ALGO_RECURRENT && algo != WKV_ALGO_CHUNKED &&
         algo != WKV_ALGO_CHUNKED_LEVELS)
@@ -206,9 +213,9 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
     const size_t ubytes = (size_t)H * D * sizeof(float);
     const bool tokens = T > 0;
     Buf bufs[] = {{r, xbytes, tokens},        {k, xbytes, tokens},      {v, xbytes, tokens},
-                  {omega, xbytes, tokens},    {u, ubytes, tokens},      {y, xbytes, tokens},
+                  {omega, xbytes, tokens},    {u, ubytes, tokens && !c2}, {y, xbytes, tokens},
                   {state_in, sbytes, false},  {state_out, sbytes, false},
-                  {workspace, workspace_bytes, false}};
+                  {workspace, workspace_bytes, false}, {uprime, xbytes, false}};
     wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
     if (s != WKV_OK) return s;
     if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
@@ -217,13 +224,16 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
     const Span sy = span(y, tokens ? xbytes : 0), sso = span(state_out, state_out ? sbytes : 0);
     const Span ins[] = {span(r, tokens ? xbytes : 0), span(k, tokens ? xbytes : 0),
                         span(v, tokens ? xbytes : 0), span(omega, tokens ? xbytes : 0),
-                        span(u, tokens ? ubytes : 0), span(state_in, state_in ? sbytes : 0),
+                        span(c2 ? nullptr : u, tokens && !c2 ? ubytes : 0),
+                        span(state_in, state_in ? sbytes : 0),
                         span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
-                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0)};
+                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0),
+                        span(uprime, c2 && tokens ? xbytes : 0)};
     for (const Span& in : ins)
         if (overlaps(sy, in)) return WKV_ERR_INVALID_ARG;
     for (int i = 0; i < 5; ++i)
         if (overlaps(sso, ins[i])) return WKV_ERR_INVALID_ARG;
+    if (overlaps(sso, ins[8])) return WKV_ERR_INVALID_ARG;
     if (overlaps(sso, ins[6]) || overlaps(sso, ins[7]) || overlaps(sso, sy))
         return WKV_ERR_INVALID_ARG;
     if (state_in && state_out && state_in != state_out && overlaps(sso, ins[5]))
@@ -249,6 +259,7 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
 
     const bool bf16 = io == WKV_BF16;
     const bool chunked = use_chunked(io, algo);
+    const goldwkv::Variant var{uprime};
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
     const int P = !chunked || algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
@@ -277,25 +288,25 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
         const goldwkv::Segments seg{P, (nc + P - 1) / P, s_mid};
         if (algo == WKV_ALGO_CHUNKED_LEVELS) {
             e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg,
-                                               status, nullptr, nullptr, budget, st);
+                                               var, status, nullptr, nullptr, budget, st);
         } else {
             e = cudaSuccess;
             if (P > 1) {   // states entering segments 1 .. P-1 (computed in place in s_mid)
-                e = goldwkv::launch_segment_states(maps, s_mid, log2g, B, T, H, seg, status,
+                e = goldwkv::launch_segment_states(maps, s_mid, log2g, B, T, H, seg, var, status,
                                                    budget, st);
                 if (e == cudaSuccess)
                     e = goldwkv::launch_segment_carry(state_in, s_mid, log2g, s_mid, B, H, P, st);
             }
             if (e == cudaSuccess)
                 e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H,
-                                                 seg, status, h_chunk, h_state, budget, st);
+                                                 seg, var, status, h_chunk, h_state, budget, st);
             if (e == cudaSuccess)
                 e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
-                                                   seg, status, h_chunk, h_state, budget, st);
+                                                   seg, var, status, h_chunk, h_state, budget, st);
         }
     } else {
         e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,
-                                      H, bf16, st);
+                                      H, bf16, var, st);
     }
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     if (ln) {
@@ -304,6 +315,85 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
         if (e != cudaSuccess) return WKV_ERR_CUDA;
     }
     return WKV_OK;
+}
+
+
+wkv_status decode_impl(const void* r, const void* k, const void* v, const void* omega,
+                       const float* u, const void* uprime, float* state, void* y, int B, int H,
+                       int D, wkv_dtype io, const wkv_ln* ln, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    const bool c2 = uprime != nullptr;
+    if (B < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
+    if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return WKV_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t esz = io_size(io);
+    const size_t xbytes = (size_t)B * H * D * esz;
+    const size_t sbytes = (size_t)B * H * D * D * sizeof(float);
+    const size_t ubytes = (size_t)H * D * sizeof(float);
+    Buf bufs[] = {{r, xbytes, true}, {k, xbytes, true},     {v, xbytes, true},
+                  {omega, xbytes, true}, {u, ubytes, !c2}, {state, sbytes, true},
+                  {y, xbytes, true}, {workspace, workspace_bytes, false},
+                  {uprime, xbytes, false}};
+    wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
+    if (s != WKV_OK) return s;
+    if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
+
+    const Span sy = span(y, xbytes), ss = span(state, sbytes);
+    const Span ins[] = {span(r, xbytes), span(k, xbytes), span(v, xbytes), span(omega, xbytes),
+                        span(c2 ? nullptr : u, c2 ? 0 : ubytes),
+                        span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
+                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0),
+                        span(uprime, c2 ? xbytes : 0)};
+    if (overlaps(sy, ss)) return WKV_ERR_INVALID_ARG;
+    for (const Span& in : ins)
+        if (overlaps(sy, in) || overlaps(ss, in)) return WKV_ERR_INVALID_ARG;
+
+    const size_t need = wkv6_decode_workspace_bytes(B, H, D, io, ln != nullptr);
+    if (need > 0) {
+        if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+        const Span sw = span(workspace, need);
+        if (overlaps(sw, sy) || overlaps(sw, ss)) return WKV_ERR_INVALID_ARG;
+        for (const Span& in : ins)
+            if (overlaps(sw, in)) return WKV_ERR_INVALID_ARG;
+    }
+    if (injected("launch")) return WKV_ERR_CUDA;
+
+    const bool bf16 = io == WKV_BF16;
+    float* y_raw = nullptr;
+    if (ln) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
+    cudaError_t e = goldwkv::launch_decode(r, k, v, omega, u, state, y, y_raw, B, H, bf16,
+                                           goldwkv::Variant{uprime}, st);
+    if (e != cudaSuccess) return WKV_ERR_CUDA;
+    if (ln) {
+        e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y, (long)B,
+                                           H * D, bf16, st);
+        if (e != cudaSuccess) return WKV_ERR_CUDA;
+    }
+    return WKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const void* omega,
+                             const float* u, const float* state_in, float* state_out, void* y,
+                             int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
+                             wkv_algo algo, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    return prefill_impl(r, k, v, omega, u, nullptr, state_in, state_out, y, B, T, H, D, io, ln,
+                        algo, workspace, workspace_bytes, stream);
+}
+
+wkv_status wkv6c2_prefill(const void* r, const void* k, const void* v, const void* omega,
+                          const void* uprime, const float* state_in, float* state_out, void* y,
+                          int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    // uprime may be null only for an empty problem, where only the state passes through
+    if (B > 0 && T > 0 && H > 0 && uprime == nullptr) return WKV_ERR_INVALID_ARG;
+    return prefill_impl(r, k, v, omega, nullptr, uprime, state_in, state_out, y, B, T, H, D, io,
+                        ln, WKV_ALGO_AUTO, workspace, workspace_bytes, stream);
 }
 
 wkv_status wkv6_workspace_status(void* workspace, void* stream) {
@@ -333,50 +423,17 @@ wkv_status wkv6_decode_step(const void* r, const void* k, const void* v, const v
                             const float* u, float* state, void* y, int B, int H, int D,
                             wkv_dtype io, const wkv_ln* ln, void* workspace,
                             size_t workspace_bytes, void* stream) {
-    if (B < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
-    if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
-    if (B == 0 || H == 0) return WKV_OK;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const size_t esz = io_size(io);
-    const size_t xbytes = (size_t)B * H * D * esz;
-    const size_t sbytes = (size_t)B * H * D * D * sizeof(float);
-    const size_t ubytes = (size_t)H * D * sizeof(float);
-    Buf bufs[] = {{r, xbytes, true}, {k, xbytes, true},     {v, xbytes, true},
-                  {omega, xbytes, true}, {u, ubytes, true}, {state, sbytes, true},
-                  {y, xbytes, true}, {workspace, workspace_bytes, false}};
-    wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
-    if (s != WKV_OK) return s;
-    if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
+    return decode_impl(r, k, v, omega, u, nullptr, state, y, B, H, D, io, ln, workspace,
+                       workspace_bytes, stream);
+}
 
-    const Span sy = span(y, xbytes), ss = span(state, sbytes);
-    const Span ins[] = {span(r, xbytes), span(k, xbytes), span(v, xbytes), span(omega, xbytes),
-                        span(u, ubytes), span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
-                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0)};
-    if (overlaps(sy, ss)) return WKV_ERR_INVALID_ARG;
-    for (const Span& in : ins)
-        if (overlaps(sy, in) || overlaps(ss, in)) return WKV_ERR_INVALID_ARG;
-
-    const size_t need = wkv6_decode_workspace_bytes(B, H, D, io, ln != nullptr);
-    if (need > 0) {
-        if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
-        const Span sw = span(workspace, need);
-        if (overlaps(sw, sy) || overlaps(sw, ss)) return WKV_ERR_INVALID_ARG;
-        for (const Span& in : ins)
-            if (overlaps(sw, in)) return WKV_ERR_INVALID_ARG;
-    }
-    if (injected("launch")) return WKV_ERR_CUDA;
-
-    const bool bf16 = io == WKV_BF16;
-    float* y_raw = nullptr;
-    if (ln) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
-    cudaError_t e = goldwkv::launch_decode(r, k, v, omega, u, state, y, y_raw, B, H, bf16, st);
-    if (e != cudaSuccess) return WKV_ERR_CUDA;
-    if (ln) {
-        e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y, (long)B,
-                                           H * D, bf16, st);
-        if (e != cudaSuccess) return WKV_ERR_CUDA;
-    }
-    return WKV_OK;
+wkv_status wkv6c2_decode_step(const void* r, const void* k, const void* v, const void* omega,
+                              const void* uprime, float* state, void* y, int B, int H, int D,
+                              wkv_dtype io, const wkv_ln* ln, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    if (B > 0 && H > 0 && uprime == nullptr) return WKV_ERR_INVALID_ARG;
+    return decode_impl(r, k, v, omega, nullptr, uprime, state, y, B, H, D, io, ln, workspace,
+                       workspace_bytes, stream);
 }
 
 }  // extern "C"

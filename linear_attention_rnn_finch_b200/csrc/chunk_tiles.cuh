@@ -94,6 +94,22 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 __device__ __forceinline__ int ld_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
 
+// 1 - exp(-x) for x = exp(omega) >= 0 (the Finch-C2 key factor 1 - w), without the
+// cancellation of 1 - w for small x: below 1/4 the series x (1 - x/2 (1 - x/3 (1 - x/4
+// (1 - x/5)))), whose first omitted term is x^6/720 (relative error < 1.5e-6 there);
+// from 1/4 up, 1 - 2^(-x log2 e) directly (w <= 0.78, so the subtraction loses < 3 bits).
+__device__ __forceinline__ float2 one_minus_exp_neg2(float2 x) {
+    const float2 one = make_float2(1.f, 1.f);
+    float2 p = __ffma2_rn(x, make_float2(-0.2f, -0.2f), one);
+    p = __ffma2_rn(__fmul2_rn(x, make_float2(-0.25f, -0.25f)), p, one);
+    p = __ffma2_rn(__fmul2_rn(x, make_float2(-1.f / 3.f, -1.f / 3.f)), p, one);
+    p = __ffma2_rn(__fmul2_rn(x, make_float2(-0.5f, -0.5f)), p, one);
+    p = __fmul2_rn(x, p);
+    constexpr float kNegLog2e = -1.4426950408889634f;
+    const float2 d = make_float2(1.f - fast_exp2(x.x * kNegLog2e), 1.f - fast_exp2(x.y * kNegLog2e));
+    return make_float2(x.x < 0.25f ? p.x : d.x, x.y < 0.25f ? p.y : d.y);
+}
+
 // Bounded wait on an mbarrier phase.  `s` is the CTA's shared state with `abort` and
 // `stop_at` words: the wait gives up early once the CTA has aborted, and on expiry it aborts
 // the CTA.

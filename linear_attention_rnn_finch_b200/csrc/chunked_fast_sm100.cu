@@ -98,12 +98,15 @@ struct __align__(1024) Smem {
     int stop_at;                     // chunk at which this (b,h) leaves for the level kernel
 };
 
-// Output of chunk m: y = Y[:, 0:64] + Y[:, 64:128] (hi and lo rows each), stored as bf16 (or
+// Output of chunk m (plus the second value u' of Finch-C2, whose words up0 / up1 for rows
+// r0 / r1 the caller loaded ahead of time): y = Y[:, 0:64] + Y[:, 64:128] (hi and lo rows each), stored as bf16 (or
 // fp32 rows to y_raw).  Frees the Y accumulator for RO(m+1).
+template <bool kC2>
 __device__ __forceinline__ void output_chunk(Smem& s, int m, int c0, uint32_t tmem, uint32_t lane_h0,
                                              uint32_t lane_h1, int ch, int cbase, int r0, int r1,
                                              int b, int h, int T, int H, __nv_bfloat16* y,
-                                             float* y_raw, long long budget) {
+                                             float* y_raw, const uint32_t (&up0)[4],
+                                             const uint32_t (&up1)[4], long long budget) {
     // m: chunk index within the unit (GA(m) is the (m+1)-th ya_done phase); c0 + m: absolute
     wait_soft(s, &s.ya_done, (uint32_t)(m & 1), budget);
     ptx::tc_fence_after();
@@ -133,6 +136,10 @@ __device__ __forceinline__ void output_chunk(Smem& s, int m, int c0, uint32_t tm
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int j = cbase + 8 * k;
+        if (kC2) {   // Finch-C2: the second value u'_t joins the readout (loaded beforehand)
+            Y0[k] = __fadd2_rn(Y0[k], unpack2(up0[k]));
+            Y1[k] = __fadd2_rn(Y1[k], unpack2(up1[k]));
+        }
         if (y_raw != nullptr) {
             if (r0 < valid) *reinterpret_cast<float2*>(y_raw + row0 * 64 + j) = Y0[k];
             if (r1 < valid) *reinterpret_cast<float2*>(y_raw + row1 * 64 + j) = Y1[k];
@@ -140,6 +147,23 @@ __device__ __forceinline__ void output_chunk(Smem& s, int m, int c0, uint32_t tm
             if (r0 < valid) *reinterpret_cast<uint32_t*>(y + row0 * 64 + j) = pack2(Y0[k].x, Y0[k].y);
             if (r1 < valid) *reinterpret_cast<uint32_t*>(y + row1 * 64 + j) = pack2(Y1[k].x, Y1[k].y);
         }
+    }
+}
+
+// u' words of chunk (c0 + m) for this thread's rows r0, r1 and column pairs cbase + 8k;
+// rows past T read as zero.  Issued well before output_chunk needs them.
+__device__ __forceinline__ void load_uprime(const __nv_bfloat16* __restrict__ uprime, int m, int c0,
+                                            int b, int h, int T, int H, int cbase, int r0, int r1,
+                                            uint32_t (&up0)[4], uint32_t (&up1)[4]) {
+    const int tc = (c0 + m) * C;
+    const int valid = min(C, T - tc);
+    const size_t row0 = ((size_t)b * T + (size_t)tc + r0) * H + h;
+    const size_t row1 = ((size_t)b * T + (size_t)tc + r1) * H + h;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int j = cbase + 8 * k;
+        up0[k] = r0 < valid ? __ldg(reinterpret_cast<const unsigned int*>(uprime + row0 * 64 + j)) : 0u;
+        up1[k] = r1 < valid ? __ldg(reinterpret_cast<const unsigned int*>(uprime + row1 * 64 + j)) : 0u;
     }
 }
 
@@ -158,11 +182,14 @@ __device__ __forceinline__ void store_state(uint8_t* tile, const float2 (&S0)[4]
     }
 }
 
+// kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
+template <bool kC2>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                  const float* __restrict__ u, const float* s_in, float* s_out,
-                 __nv_bfloat16* __restrict__ y, float* __restrict__ y_raw, int T, int H,
+                 __nv_bfloat16* __restrict__ y, float* __restrict__ y_raw,
+                 const __nv_bfloat16* __restrict__ uprime, int T, int H,
                  Segments seg, int* status, int* handoff_chunk, float* handoff_state,
                  long long budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
@@ -314,7 +341,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         // warp g: tokens 8g .. 8g+7 of every chunk; lane = channel pair (2l, 2l+1); log2 units
         const int g = warp - kPrepWarp0;
         const int c0 = 2 * lane;
-        const float2 uu = make_float2(u[h * 64 + c0], u[h * 64 + c0 + 1]);
+        const float2 uu = kC2 ? make_float2(0.f, 0.f) : make_float2(u[h * 64 + c0], u[h * 64 + c0 + 1]);
         const int chunk = lane >> 2;          // 16-byte chunk holding channels c0, c0+1
         const uint32_t cbyte = (uint32_t)(lane & 3) * 4;
         const float2 l2e = make_float2(kLog2e, kLog2e);
@@ -333,6 +360,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             const uint8_t* w_tile = s.rkw[st][2];
             // pass 1: local inclusive prefix of log2 w = -exp(omega) log2(e)
             float2 L[8];
+            float2 ex[8];   // exp(omega) of each token (Finch-C2 normalises the key with it)
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
@@ -342,6 +370,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 if (t >= valid) e = make_float2(0.f, 0.f);
                 acc = __ffma2_rn(e, nl2e, acc);
                 L[p] = acc;
+                ex[p] = e;
             }
             *reinterpret_cast<float2*>(&s.qtot[pb][g][c0]) = acc;
             named_bar(kBarPrep, kPrepThreads);
@@ -386,7 +415,9 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 const int t = 8 * g + p;
                 const uint32_t o = sw_off(t, chunk) + cbyte;
                 const float2 rr = unpack2(rw[p]);
-                const float2 kk = unpack2(kw[p]);
+                float2 kk = unpack2(kw[p]);
+                if (kC2)   // k (1 - w), 1 - w = 1 - exp(-exp(omega)) without cancellation
+                    kk = __fmul2_rn(kk, one_minus_exp_neg2(ex[p]));
                 uint32_t hi, lo;
                 split2(__fmul2_rn(rr, fr[p]), hi, lo);
                 const int hr = hi_row(t);
@@ -396,10 +427,13 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 split2(__fmul2_rn(kk, fk[p]), hi, lo);
                 sts32(kh_hi, o, hi);
                 sts32(kh_lo, o, lo);
-                const float2 ru = __fmul2_rn(rr, uu);
-                bon[p] = fmaf(ru.x, kk.x, ru.y * kk.y);
+                if (!kC2) {
+                    const float2 ru = __fmul2_rn(rr, uu);
+                    bon[p] = fmaf(ru.x, kk.x, ru.y * kk.y);
+                }
             }
             // bonus: reduce the 8 per-token partials over the 32 lanes (reduce-scatter)
+            if (!kC2) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const bool up = lane & 16;
@@ -425,6 +459,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             if ((lane & 3) == 0) {
                 const int p = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
                 s.bonus[pb][8 * g + p] = bon[0];
+            }
             }
             if (g == 0) {
                 *reinterpret_cast<float2*>(&s.gamma[pb][c0]) = make_float2(fast_exp2(tot.x), fast_exp2(tot.y));
@@ -472,9 +507,12 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             ptx::fence_proxy_async_smem();
             mbar_arrive(&s.s_ready[0]);
         }
+        uint32_t up0[4] = {0u, 0u, 0u, 0u}, up1[4] = {0u, 0u, 0u, 0u};   // u' of the next output
         int n = 0;
         for (; n < NC; ++n) {
             const int pb = n & 1;
+            // Finch-C2: u' of chunk n-1 is read from HBM now and used by output(n-1) below
+            if (kC2 && n >= 1) load_uprime(uprime, n - 1, cseg, b, h, T, H, cbase, r0, r1, up0, up1);
             // ---- state(n): S <- gamma (S + U), U^T[j][i] = DU[j][i] + DU[j][64+i]
             {
                 // gamma and bonus of chunk n reach us from prep through the chain prep's
@@ -510,7 +548,9 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 mbar_arrive(&s.s_ready[(n + 1) & 1]);
             }
             // ---- output of chunk n-1 (its GA was issued at the end of the previous round)
-            if (n >= 1) output_chunk(s, n - 1, cseg, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
+            if (n >= 1)
+                output_chunk<kC2>(s, n - 1, cseg, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw,
+                                  up0, up1, budget);
             // ---- A(n): masked scores with the bonus on the diagonal, hi / lo, for GA(n)
             wait_soft(s, &s.sc_done[pb], (uint32_t)((n >> 1) & 1), budget);
             ptx::tc_fence_after();
@@ -521,7 +561,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 ptx::tmem_wait_ld();
                 ptx::tc_fence_before();
                 mbar_arrive(&s.sc_free[pb]);
-                const float b0 = s.bonus[pb][r0], b1 = s.bonus[pb][r1];
+                const float b0 = kC2 ? 0.f : s.bonus[pb][r0], b1 = kC2 ? 0.f : s.bonus[pb][r1];
                 // the A tile is free: GA(n-1) completed before output(n-1) read Y
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -551,8 +591,11 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         }
         // ---- leave: output of the last chunk done, final state (or the state entering the
         // chunk handed to the level kernel)
-        if (!ld_volatile(&s.abort) && n >= 1)
-            output_chunk(s, n - 1, cseg, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw, budget);
+        if (!ld_volatile(&s.abort) && n >= 1) {
+            if (kC2) load_uprime(uprime, n - 1, cseg, b, h, T, H, cbase, r0, r1, up0, up1);
+            output_chunk<kC2>(s, n - 1, cseg, tmem, lane_h0, lane_h1, ch, cbase, r0, r1, b, h, T, H, y, y_raw,
+                              up0, up1, budget);
+        }
         const bool aborted = ld_volatile(&s.abort) != 0;
         if (!aborted) {
             const bool stopped = (n < NC);
@@ -591,15 +634,16 @@ size_t fast_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
                                 float* s_out, void* y, float* y_raw, int B, int T, int H,
-                                Segments seg, int* status, int* handoff_chunk,
+                                Segments seg, Variant var, int* status, int* handoff_chunk,
                                 float* handoff_state, long long budget, cudaStream_t st) {
     const size_t smem = fast_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(wkv6_fast_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kernel = var.uprime ? wkv6_fast_kernel<true> : wkv6_fast_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_fast_kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
+    kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], u, s_in, s_out, static_cast<__nv_bfloat16*>(y),
-        y_raw, T, H, seg, status, handoff_chunk, handoff_state, budget, 4000000000LL);
+        y_raw, static_cast<const __nv_bfloat16*>(var.uprime), T, H, seg, status, handoff_chunk,
+        handoff_state, budget, 4000000000LL);
     return cudaGetLastError();
 }
 

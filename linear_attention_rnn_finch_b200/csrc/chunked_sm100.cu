@@ -125,12 +125,14 @@ __device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 
     *reinterpret_cast<uint4*>(base + off) = v;
 }
 
+// kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
+template <bool kC2>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
-                    const float* s_in, float* s_out, float* __restrict__ y_raw, int T, int H,
-                    Segments seg, int* status, const int* start_chunk,
+                    const float* s_in, float* s_out, float* __restrict__ y_raw,
+                    const __nv_bfloat16* __restrict__ uprime, int T, int H, Segments seg, int* status, const int* start_chunk,
                     const float* handoff_state, long long spin_budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -163,7 +165,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
         ptx::prefetch_tensormap(&tm_w);
         ptx::prefetch_tensormap(&tm_y);
     }
-    if (tid < 64) s.u[tid] = u[h * 64 + tid];
+    if (tid < 64) s.u[tid] = kC2 ? 0.f : u[h * 64 + tid];
     if (warp == 0) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     // zero the operand tiles once, so that rows an MMA reads but never uses hold finite data
     for (int i = tid; i < (int)(sizeof(s.q) + sizeof(s.kk)) / 16; i += kThreads)
@@ -249,6 +251,17 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         wv[p][c] = (ta + p < valid) ? __expf(-__expf(om[p][c])) : 1.f;
+                if (kC2) {
+                    // normalised key k (1 - w), 1 - w = -expm1(-exp(omega)); level 0 reads the
+                    // k tile itself, so it is rewritten in place (bf16, as the other levels)
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            kv[p][c] *= (ta + p < valid) ? -expm1f(-__expf(om[p][c])) : 0.f;
+                    st_shared_v4(k_tile, sw_chunk(ta, cg), pack8(kv[0]));
+                    st_shared_v4(k_tile, sw_chunk(tb, cg), pack8(kv[1]));
+                }
             }
             // bonus partials: sum over this lane's 8 channels of r u k
 #pragma unroll
@@ -465,6 +478,16 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             uint32_t Y[32];
             ptx::tmem_ld32(tmem + tlane + COL_Y + 32 * hh, Y);
             ptx::tmem_wait_ld();
+            if (kC2 && row_lane && row < valid) {   // the second value u'_t joins the readout
+                const __nv_bfloat16* up = uprime + (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float f[8];
+                    unpack8(*reinterpret_cast<const uint4*>(up + 8 * cc), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) Y[8 * cc + e] = __float_as_uint(__uint_as_float(Y[8 * cc + e]) + f[e]);
+                }
+            }
             if (row_lane && y_raw != nullptr) {
                 // fp32 rows for the LayerNorm pass: 128 contiguous bytes per lane
                 if (row < valid) {
@@ -567,17 +590,18 @@ size_t chunked_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
                                   float* s_out, float* y_raw, int B, int T, int H, Segments seg,
-                                  int* status, const int* start_chunk,
+                                  Variant var, int* status, const int* start_chunk,
                                   const float* handoff_state, long long spin_budget,
                                   cudaStream_t st) {
     const size_t smem = chunked_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kernel = var.uprime ? wkv6_chunked_kernel<true> : wkv6_chunked_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long drain = 4000000000LL;
-    wkv6_chunked_kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw, T, H, seg, status,
-        start_chunk, handoff_state, spin_budget, drain);
+    kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw,
+        static_cast<const __nv_bfloat16*>(var.uprime), T, H, seg, status, start_chunk,
+        handoff_state, spin_budget, drain);
     return cudaGetLastError();
 }
 

@@ -20,12 +20,15 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// uprime != nullptr: Finch-C2 exact form -- key k (1 - w), no static bonus, second value
+// u' ([B][H][D], dtype IO) added to y.
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
 wkv6_decode_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                    const IO* __restrict__ v, const IO* __restrict__ omega,
-                   const float* __restrict__ u, float* __restrict__ state,
-                   IO* __restrict__ y, float* __restrict__ y_raw, int H) {
+                   const float* __restrict__ u, const IO* __restrict__ uprime,
+                   float* __restrict__ state, IO* __restrict__ y, float* __restrict__ y_raw,
+                   int H) {
     constexpr int D = kHeadSize;
     __shared__ float sr[D], sk[D], sv[D], sw[D];
     __shared__ float4 red[kThreads / 32][D / 4];
@@ -44,12 +47,14 @@ wkv6_decode_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
 
     if (tid < D) {
         const size_t g = (size_t)bh * D + tid;
-        const float rv = to_f32(r[g]), kv = to_f32(k[g]);
+        const float rv = to_f32(r[g]), om = to_f32(omega[g]);
+        float kv = to_f32(k[g]);
+        if (uprime) kv *= -expm1f(-expf(om));   // k (1 - w)
         sr[tid] = rv;
         sk[tid] = kv;
         sv[tid] = to_f32(v[g]);
-        sw[tid] = decay_from_logit(to_f32(omega[g]));
-        const float p = warp_sum(rv * u[h * D + tid] * kv);
+        sw[tid] = decay_from_logit(om);
+        const float p = uprime ? 0.f : warp_sum(rv * u[h * D + tid] * kv);
         if ((tid & 31) == 0) sbonus[tid >> 5] = p;
     }
     __syncthreads();
@@ -85,6 +90,7 @@ wkv6_decode_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
         for (int w = 0; w < kThreads / 32; ++w) yv += redf[w * D + tid];
         yv = fmaf(sbonus[0] + sbonus[1], sv[tid], yv);
         const size_t g = (size_t)bh * D + tid;
+        if (uprime) yv += to_f32(uprime[g]);
         if (y_raw) y_raw[g] = yv;
         else y[g] = from_f32<IO>(yv);
     }
@@ -94,17 +100,17 @@ wkv6_decode_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
 
 cudaError_t launch_decode(const void* r, const void* k, const void* v, const void* omega,
                           const float* u, float* state, void* y, float* y_raw, int B, int H,
-                          bool bf16, cudaStream_t st) {
+                          bool bf16, Variant var, cudaStream_t st) {
     const unsigned grid = (unsigned)(B * H);
     if (bf16) {
         using T16 = __nv_bfloat16;
         wkv6_decode_kernel<T16><<<grid, kThreads, 0, st>>>(
-            (const T16*)r, (const T16*)k, (const T16*)v, (const T16*)omega, u, state,
-            (T16*)y, y_raw, H);
+            (const T16*)r, (const T16*)k, (const T16*)v, (const T16*)omega, u,
+            (const T16*)var.uprime, state, (T16*)y, y_raw, H);
     } else {
         wkv6_decode_kernel<float><<<grid, kThreads, 0, st>>>(
-            (const float*)r, (const float*)k, (const float*)v, (const float*)omega, u, state,
-            (float*)y, y_raw, H);
+            (const float*)r, (const float*)k, (const float*)v, (const float*)omega, u,
+            (const float*)var.uprime, state, (float*)y, y_raw, H);
     }
     return cudaGetLastError();
 }

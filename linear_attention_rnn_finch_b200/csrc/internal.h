@@ -7,16 +7,25 @@
 
 namespace goldwkv {
 
+// Which form of the time mixing: base Finch / RWKV-6 (static bonus u) when uprime is null;
+// otherwise Finch-C2's exact form -- the key enters the state as k_t (1 - w_t), there is no
+// static bonus, and the second value uprime (same layout and dtype as y) is added to the
+// readout before LayerNorm.
+struct Variant {
+    const void* uprime;
+};
+
 // Token-by-token recurrence (fp32 math).  y_raw != nullptr: write fp32 un-normalised y
 // there instead of y.
 cudaError_t launch_recurrent(const void* r, const void* k, const void* v, const void* omega,
                              const float* u, const float* s_in, float* s_out, void* y,
-                             float* y_raw, int B, int T, int H, bool bf16, cudaStream_t st);
+                             float* y_raw, int B, int T, int H, bool bf16, Variant var,
+                             cudaStream_t st);
 
 // One decode step, state in place.  y_raw as above.
 cudaError_t launch_decode(const void* r, const void* k, const void* v, const void* omega,
                           const float* u, float* state, void* y, float* y_raw, int B, int H,
-                          bool bf16, cudaStream_t st);
+                          bool bf16, Variant var, cudaStream_t st);
 
 // LayerNorm of `rows` rows of C fp32 values into `out` (fp32 or bf16); out may equal x.
 cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const float* beta,
@@ -41,8 +50,8 @@ struct Segments {
 // log2 decay sum[bh][p][i] = log2 prod_{t in segment} w_t[i]; chunked on tcgen05 with the
 // suffix factorisation (factors <= 1: no overflow for any decay).  maps: r, k, v, omega.
 cudaError_t launch_segment_states(const CUtensorMap* maps, float* s_loc, float* log2g, int B,
-                                  int T, int H, Segments seg, int* status, long long budget,
-                                  cudaStream_t st);
+                                  int T, int H, Segments seg, Variant var, int* status,
+                                  long long budget, cudaStream_t st);
 // s_mid[bh][p] = 2^log2g[bh][p] (rows) * s_in(p) + s_loc[bh][p], p = 0 .. P-2, in order, where
 // s_in(0) = state_in (zero if null) and s_in(p) = s_mid[bh][p-1]; s_mid may alias s_loc.
 cudaError_t launch_segment_carry(const float* state_in, const float* s_loc, const float* log2g,
@@ -55,7 +64,7 @@ cudaError_t launch_segment_carry(const float* state_in, const float* s_loc, cons
 // y_raw != nullptr: fp32 y rows there instead of y.
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
                                 float* s_out, void* y, float* y_raw, int B, int T, int H,
-                                Segments seg, int* status, int* handoff_chunk,
+                                Segments seg, Variant var, int* status, int* handoff_chunk,
                                 float* handoff_state, long long budget, cudaStream_t st);
 
 // Level-factorised path (any decay).  start_chunk == nullptr: every unit from its first
@@ -63,7 +72,7 @@ cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const f
 // < 0) from handoff_state[u].  status: device word set to 1 if a bounded wait expired.
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
                                   float* s_out, float* y_raw, int B, int T, int H, Segments seg,
-                                  int* status, const int* start_chunk,
+                                  Variant var, int* status, const int* start_chunk,
                                   const float* handoff_state, long long spin_budget,
                                   cudaStream_t st);
 size_t chunked_smem_bytes();

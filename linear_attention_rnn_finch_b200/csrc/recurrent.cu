@@ -23,12 +23,15 @@ constexpr int kTile = 32;          // tokens staged per shared-memory tile
 constexpr int kCols = 32;          // value columns per CTA
 constexpr int kThreads = 128;      // 32 columns x 4 row quarters
 
+// uprime != nullptr: Finch-C2 exact form -- key k (1 - w), no static bonus, and the second
+// value u'_t (same layout as y) added to the readout.
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
 wkv6_recurrent_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                       const IO* __restrict__ v, const IO* __restrict__ omega,
-                      const float* __restrict__ u, const float* s_in, float* s_out,
-                      IO* __restrict__ y, float* __restrict__ y_raw, int T, int H) {
+                      const float* __restrict__ u, const IO* __restrict__ uprime,
+                      const float* s_in, float* s_out, IO* __restrict__ y,
+                      float* __restrict__ y_raw, int T, int H) {
     constexpr int D = kHeadSize;
     __shared__ __align__(16) float sr[kTile][D];
     __shared__ __align__(16) float sk[kTile][D];
@@ -45,7 +48,7 @@ wkv6_recurrent_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
     const int jl = warp * 8 + (lane >> 2);     // local column 0..31
     const int j = blockIdx.y * kCols + jl;     // global value column
 
-    if (tid < D) su[tid] = u[h * D + tid];
+    if (tid < D) su[tid] = uprime ? 0.f : u[h * D + tid];
 
     // state rows 16q..16q+15 of column j
     float S[16];
@@ -67,6 +70,7 @@ wkv6_recurrent_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                 rv = to_f32(r[g]);
                 kv = to_f32(k[g]);
                 wv = decay_from_logit(to_f32(omega[g]));
+                if (uprime) kv *= -expm1f(-expf(to_f32(omega[g])));   // k (1 - w)
             }
             sr[tt][c] = rv;
             sk[tt][c] = kv;
@@ -110,8 +114,8 @@ wkv6_recurrent_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             if (q == 0) {
-                const float yv = fmaf(sbonus[tt], vj, acc);
                 const size_t g = xbase + (size_t)(t0 + tt) * tstride + j;
+                const float yv = fmaf(sbonus[tt], vj, acc) + (uprime ? to_f32(uprime[g]) : 0.f);
                 if (y_raw) y_raw[g] = yv;
                 else y[g] = from_f32<IO>(yv);
             }
@@ -128,17 +132,18 @@ wkv6_recurrent_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
 
 cudaError_t launch_recurrent(const void* r, const void* k, const void* v, const void* omega,
                              const float* u, const float* s_in, float* s_out, void* y,
-                             float* y_raw, int B, int T, int H, bool bf16, cudaStream_t st) {
+                             float* y_raw, int B, int T, int H, bool bf16, Variant var,
+                             cudaStream_t st) {
     dim3 grid((unsigned)(B * H), kHeadSize / kCols);
     if (bf16) {
         using T16 = __nv_bfloat16;
         wkv6_recurrent_kernel<T16><<<grid, kThreads, 0, st>>>(
-            (const T16*)r, (const T16*)k, (const T16*)v, (const T16*)omega, u, s_in, s_out,
-            (T16*)y, y_raw, T, H);
+            (const T16*)r, (const T16*)k, (const T16*)v, (const T16*)omega, u,
+            (const T16*)var.uprime, s_in, s_out, (T16*)y, y_raw, T, H);
     } else {
         wkv6_recurrent_kernel<float><<<grid, kThreads, 0, st>>>(
-            (const float*)r, (const float*)k, (const float*)v, (const float*)omega, u, s_in,
-            s_out, (float*)y, y_raw, T, H);
+            (const float*)r, (const float*)k, (const float*)v, (const float*)omega, u,
+            (const float*)var.uprime, s_in, s_out, (float*)y, y_raw, T, H);
     }
     return cudaGetLastError();
 }

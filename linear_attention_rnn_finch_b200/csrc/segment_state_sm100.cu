@@ -58,6 +58,8 @@ struct __align__(1024) Smem {
     int stop_at;                     // unused here (no hand-over); read by wait_soft
 };
 
+// kC2: Finch-C2's normalised key k (1 - w) enters the state.
+template <bool kC2>
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_w, float* s_loc, float* log2g, int H,
@@ -185,7 +187,11 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             for (int q = 0; q < kTokPerWarp; ++q) {
                 const uint32_t o = sw_off(kTokPerWarp * g + q, chunk) + cbyte;
                 const float2 x = __fadd2_rn(after, suf[q]);          // >= 0
-                const float2 f = make_float2(fast_exp2(-x.x), fast_exp2(-x.y));
+                float2 f = make_float2(fast_exp2(-x.x), fast_exp2(-x.y));
+                if (kC2) {   // times 1 - w = 1 - exp(-exp(omega)) of this token
+                    const float2 om = __fmul2_rn(unpack2(lds32(w_tile, o)), l2e);
+                    f = __fmul2_rn(f, one_minus_exp_neg2(make_float2(fast_exp2(om.x), fast_exp2(om.y))));
+                }
                 uint32_t hi, lo;
                 split2(__fmul2_rn(unpack2(lds32(k_tile, o)), f), hi, lo);
                 sts32(kt_hi, o, hi);
@@ -293,15 +299,15 @@ wkv6_segment_carry_kernel(const float* state_in, const float* s_loc, const float
 size_t segment_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_segment_states(const CUtensorMap* maps, float* s_loc, float* log2g, int B,
-                                  int T, int H, Segments seg, int* status, long long budget,
-                                  cudaStream_t st) {
+                                  int T, int H, Segments seg, Variant var, int* status,
+                                  long long budget, cudaStream_t st) {
     (void)T;
     if (seg.P < 2) return cudaSuccess;
     const size_t smem = segment_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(wkv6_segment_state_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kernel = var.uprime ? wkv6_segment_state_kernel<true> : wkv6_segment_state_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_segment_state_kernel<<<(unsigned)(B * H * (seg.P - 1)), kThreads, smem, st>>>(
+    kernel<<<(unsigned)(B * H * (seg.P - 1)), kThreads, smem, st>>>(
         maps[1], maps[2], maps[3], s_loc, log2g, H, seg.P, seg.seg_chunks, status, budget,
         4000000000LL);
     return cudaGetLastError();
