@@ -63,11 +63,11 @@ CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
                             "internal.h"),
-                "sha256_16": "c4103f1785484646", "bytes": 541242368 + 121432320,
+                "sha256_16": "8b33ec275d194be7", "bytes": 541247232 + 120351744,
                 "workload": (8, 4096, 32),
                 "profile": "profiles/wkv6_fast_kernel_prefill_B8_T4096_H32_bf16.md"},
     "decode": {"sources": ("decode.cu", "common.cuh"),
-               "sha256_16": "c68942cec925238b", "bytes": 138428672 + 80250624,
+               "sha256_16": "8fb24cf16874f036", "bytes": 138433536 + 78408192,
                "workload": (256, 32),
                "profile": "profiles/wkv6_decode_kernel_B256_H32_bf16.md"},
 }
