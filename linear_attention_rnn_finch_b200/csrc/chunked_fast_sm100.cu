@@ -60,6 +60,7 @@ using namespace tiles;
 constexpr int C = 64;
 constexpr int kStages = 3;
 constexpr int kPrepWarps = 8, kEpiWarps = 8;
+constexpr int kTok = C / kPrepWarps;   // tokens per prep warp (a power of two <= 32)
 constexpr int kTmaWarp = 0, kMmaUWarp = 1, kMmaYWarp = 2;
 constexpr int kPrepWarp0 = 3, kEpiWarp0 = kPrepWarp0 + kPrepWarps;
 constexpr int kPrepThreads = 32 * kPrepWarps, kEpiThreads = 32 * kEpiWarps;
@@ -359,12 +360,12 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             const uint8_t* k_tile = s.rkw[st][1];
             const uint8_t* w_tile = s.rkw[st][2];
             // pass 1: local inclusive prefix of log2 w = -exp(omega) log2(e)
-            float2 L[8];
-            float2 ex[8];   // exp(omega) of each token (Finch-C2 normalises the key with it)
+            float2 L[kTok];
+            float2 ex[kTok];   // exp(omega) of each token (Finch-C2 normalises the key with it)
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int t = 8 * g + p;
+            for (int p = 0; p < kTok; ++p) {
+                const int t = kTok * g + p;
                 const float2 om = __fmul2_rn(unpack2(lds32(w_tile, sw_off(t, chunk) + cbyte)), l2e);
                 float2 e = make_float2(fast_exp2(om.x), fast_exp2(om.y));
                 if (t >= valid) e = make_float2(0.f, 0.f);
@@ -389,10 +390,10 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 break;                        // this (b,h) continues in the level kernel
             }
             // pass 2: Rt = r 2^(L_{t-1}), Kh = k 2^(-L_t) as bf16 hi / lo; bonus partials
-            uint32_t rw[8], kw[8];
+            uint32_t rw[kTok], kw[kTok];
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const uint32_t o = sw_off(8 * g + p, chunk) + cbyte;
+            for (int p = 0; p < kTok; ++p) {
+                const uint32_t o = sw_off(kTok * g + p, chunk) + cbyte;
                 rw[p] = lds32(r_tile, o);
                 kw[p] = lds32(k_tile, o);
             }
@@ -401,18 +402,18 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             uint8_t* kh_hi = s.kh[pb];
             uint8_t* kh_lo = s.kh[pb] + kTile;
             // all exponentials first (independent of each other), then products and stores
-            float2 fr[8], fk[8];   // 2^(L_{t-1}), 2^(-L_t)
+            float2 fr[kTok], fk[kTok];   // 2^(L_{t-1}), 2^(-L_t)
             fr[0] = make_float2(fast_exp2(off.x), fast_exp2(off.y));
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
+            for (int p = 0; p < kTok; ++p) {
                 const float2 li = __fadd2_rn(off, L[p]);
                 fk[p] = make_float2(fast_exp2(-li.x), fast_exp2(-li.y));
-                if (p < 7) fr[p + 1] = make_float2(fast_exp2(li.x), fast_exp2(li.y));
+                if (p < kTok - 1) fr[p + 1] = make_float2(fast_exp2(li.x), fast_exp2(li.y));
             }
-            float bon[8];
+            float bon[kTok];
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int t = 8 * g + p;
+            for (int p = 0; p < kTok; ++p) {
+                const int t = kTok * g + p;
                 const uint32_t o = sw_off(t, chunk) + cbyte;
                 const float2 rr = unpack2(rw[p]);
                 float2 kk = unpack2(kw[p]);
@@ -432,34 +433,30 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     bon[p] = fmaf(ru.x, kk.x, ru.y * kk.y);
                 }
             }
-            // bonus: reduce the 8 per-token partials over the 32 lanes (reduce-scatter)
+            // bonus: reduce the kTok per-token partials over the 32 lanes (reduce-scatter: each
+            // halving step keeps half of the tokens on each side of a lane-bit split)
             if (!kC2) {
+                constexpr int kSteps = kTok == 8 ? 3 : kTok == 4 ? 2 : kTok == 2 ? 1 : 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const bool up = lane & 16;
-                const float send = up ? bon[i] : bon[i + 4];
-                const float keep = up ? bon[i + 4] : bon[i];
-                bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-            }
+                for (int stp = 0; stp < kSteps; ++stp) {
+                    const int mask = 16 >> stp, half = kTok >> (stp + 1);
+                    const bool up = lane & mask;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const bool up = lane & 8;
-                const float send = up ? bon[i] : bon[i + 2];
-                const float keep = up ? bon[i + 2] : bon[i];
-                bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-            }
-            {
-                const bool up = lane & 4;
-                const float send = up ? bon[0] : bon[1];
-                const float keep = up ? bon[1] : bon[0];
-                bon[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-            }
-            bon[0] += __shfl_xor_sync(0xffffffffu, bon[0], 2);
-            bon[0] += __shfl_xor_sync(0xffffffffu, bon[0], 1);
-            if ((lane & 3) == 0) {
-                const int p = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-                s.bonus[pb][8 * g + p] = bon[0];
-            }
+                    for (int i = 0; i < half; ++i) {
+                        const float send = up ? bon[i] : bon[i + half];
+                        const float keep = up ? bon[i + half] : bon[i];
+                        bon[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                    }
+                }
+#pragma unroll
+                for (int mask = 16 >> kSteps; mask >= 1; mask >>= 1)
+                    bon[0] += __shfl_xor_sync(0xffffffffu, bon[0], mask);
+                if ((lane & ((32 >> kSteps) - 1)) == 0) {
+                    int p = 0;   // token index: lane bits 4, 3, ... of the halving steps
+#pragma unroll
+                    for (int stp = 0; stp < kSteps; ++stp) p = 2 * p + ((lane >> (4 - stp)) & 1);
+                    s.bonus[pb][kTok * g + p] = bon[0];
+                }
             }
             if (g == 0) {
                 *reinterpret_cast<float2*>(&s.gamma[pb][c0]) = make_float2(fast_exp2(tot.x), fast_exp2(tot.y));
