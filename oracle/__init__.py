@@ -74,6 +74,9 @@ class Oracle:
         lib.wkv6_oracle_layernorm.argtypes = [ctypes.c_long, ctypes.c_int, dp, dp, dp,
                                               ctypes.c_double, dp]
         lib.wkv6_oracle_layernorm.restype = ctypes.c_int
+        lib.wkv6_oracle_groupnorm_gate.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp,
+                                                   dp, ctypes.c_double, dp, dp]
+        lib.wkv6_oracle_groupnorm_gate.restype = ctypes.c_int
         self._lib = lib
 
     @staticmethod
@@ -171,6 +174,25 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle layernorm failed rc={rc}")
         return out
+
+    def groupnorm_gate(self, x, gamma=None, beta=None, eps: float = 1e-5, gate=None):
+        """Per-head GroupNorm of x [..., H, D] (each head's D channels), affine gamma/beta
+        [H*D], then times gate [..., H, D] (or 1), fp64."""
+        x = self._f64(x)
+        H, D = x.shape[-2], x.shape[-1]
+        N = x.size // (H * D)
+        g, b, gt = self._f64(gamma), self._f64(beta), self._f64(gate)
+        out = np.empty_like(x)
+        rc = self._lib.wkv6_oracle_groupnorm_gate(N, H, D, self._ptr(x), self._ptr(g), self._ptr(b),
+                                                  float(eps), self._ptr(gt), self._ptr(out))
+        if rc != 0:
+            raise RuntimeError(f"oracle groupnorm failed rc={rc}")
+        return out
+
+    def prefill_gn(self, r, k, v, omega, u, state_in, gamma, beta, eps=1e-5, gate=None, nthreads=None):
+        """Base-Finch output: prefill, then per-head GroupNorm and the gate."""
+        y, s = self.prefill(r, k, v, omega, u, state_in, nthreads)
+        return self.groupnorm_gate(y, gamma, beta, eps, gate), s, y
 
     def prefill_ln(self, r, k, v, omega, u, state_in, gamma, beta, eps=1e-5, nthreads=None):
         """Prefill followed by LayerNorm over the concatenated heads (H*D) of each token."""

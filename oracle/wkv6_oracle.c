@@ -291,3 +291,38 @@ int wkv6_oracle_layernorm(long N, int C, const double *x, const double *gamma,
     }
     return 0;
 }
+
+/* Base Finch's output normalisation, per head (the page's "per-head GroupNorm" that
+ * Finch-C2 replaces by LayerNorm), followed by the output gate:
+ *   out[n][h][c] = ((x[n][h][c] - mean_nh) / sqrt(var_nh + eps) * gamma[h*D + c] + beta[h*D + c])
+ *                  * gate[n][h][c]
+ * mean_nh / var_nh (biased) over the D channels of head h of row n; x, gate, out [N][H][D];
+ * gamma / beta [H*D] may be NULL (1 / 0); gate may be NULL (1).  out may equal x. */
+int wkv6_oracle_groupnorm_gate(long N, int H, int D, const double *x, const double *gamma,
+                               const double *beta, double eps, const double *gate, double *out)
+{
+    if (N < 0 || H <= 0 || D <= 0)
+        return -1;
+    for (long n = 0; n < N; ++n) {
+        for (int h = 0; h < H; ++h) {
+            const long base = (n * H + h) * (long)D;
+            double mu = 0.0;
+            for (int c = 0; c < D; ++c)
+                mu += x[base + c];
+            mu /= (double)D;
+            double s2 = 0.0;
+            for (int c = 0; c < D; ++c)
+                s2 += (x[base + c] - mu) * (x[base + c] - mu);
+            s2 /= (double)D;
+            const double rs = 1.0 / sqrt(s2 + eps);
+            for (int c = 0; c < D; ++c) {
+                const double ga = gamma ? gamma[h * D + c] : 1.0;
+                const double be = beta ? beta[h * D + c] : 0.0;
+                const double gt = gate ? gate[base + c] : 1.0;
+                out[base + c] = ((x[base + c] - mu) * rs * ga + be) * gt;
+            }
+        }
+    }
+    return 0;
+}
+

@@ -33,6 +33,16 @@ section 3.4 "Key computation with normalization property" and "the new second va
 * c2_second_value   - y is affine in u' with unit slope and the state does not see u';
 * c2_decode         - the decode step's closed form with the normalised key.
 
+Base Finch's per-head GroupNorm and output gate:
+
+* gn_moments        - every head of every row has mean 0 and variance var/(var+eps) before
+                      the affine part;
+* gn_torch          - GroupNorm equals torch.nn.functional.group_norm (H groups over H*D
+                      channels) in fp64;
+* gn_gate           - the gate multiplies the normalised output elementwise (gate 1 and
+                      gate 2x give x and 2x, a random gate gives the product);
+* gn_head_local     - changing one head's inputs changes only that head's outputs.
+
 ``run_all(oracle)`` returns the list of failing pin names; the mutation test uses it to
 show that plausible mistakes planted in the oracle are caught.
 """
@@ -290,6 +300,48 @@ def pin_c2_decode(o):
     return _close(y, y_ref) and _close(S, S_ref)
 
 
+def pin_gn_moments(o):
+    g = _rng(21)
+    x = g.normal(0.4, 2.0, (5, 3, 64))
+    y = o.groupnorm_gate(x, None, None, 1e-5)
+    var = x.var(axis=-1, keepdims=True)
+    ok = float(np.max(np.abs(y.mean(axis=-1)))) <= 1e-13   # absolute: the reference is 0
+    return ok and _close(y.var(axis=-1, keepdims=True), var / (var + 1e-5), 1e-10)
+
+
+def pin_gn_torch(o):
+    g = _rng(22)
+    N, H, D = 7, 4, 64
+    x = g.normal(0, 1.0, (N, H, D))
+    gam = 1 + 0.1 * g.normal(size=H * D)
+    bet = 0.1 * g.normal(size=H * D)
+    y = o.groupnorm_gate(x, gam, bet, 1e-5)
+    ref = torch.nn.functional.group_norm(torch.from_numpy(x.reshape(N, H * D)), H,
+                                         torch.from_numpy(gam), torch.from_numpy(bet), 1e-5)
+    return _close(y.reshape(N, H * D), ref.numpy(), 1e-12)
+
+
+def pin_gn_gate(o):
+    g = _rng(23)
+    x = g.normal(0, 1.0, (4, 2, 64))
+    gam = 1 + 0.1 * g.normal(size=128)
+    bet = 0.1 * g.normal(size=128)
+    gate = g.normal(0, 1.0, x.shape)
+    base = o.groupnorm_gate(x, gam, bet, 1e-5)
+    ok = _close(o.groupnorm_gate(x, gam, bet, 1e-5, np.ones_like(x)), base)
+    ok &= _close(o.groupnorm_gate(x, gam, bet, 1e-5, 2.0 * np.ones_like(x)), 2.0 * base)
+    return ok and _close(o.groupnorm_gate(x, gam, bet, 1e-5, gate), base * gate)
+
+
+def pin_gn_head_local(o):
+    g = _rng(24)
+    x = g.normal(0, 1.0, (3, 4, 64))
+    x2 = x.copy()
+    x2[:, 2] = g.normal(5.0, 3.0, (3, 64))
+    a, b = o.groupnorm_gate(x, None, None, 1e-5), o.groupnorm_gate(x2, None, None, 1e-5)
+    return np.array_equal(a[:, [0, 1, 3]], b[:, [0, 1, 3]]) and not np.allclose(a[:, 2], b[:, 2])
+
+
 PINS = {
     "explicit_sum": pin_explicit_sum,
     "t1_closed_form": pin_t1_closed_form,
@@ -306,6 +358,10 @@ PINS = {
     "c2_normalised_rows": pin_c2_normalised_rows,
     "c2_second_value": pin_c2_second_value,
     "c2_decode": pin_c2_decode,
+    "gn_moments": pin_gn_moments,
+    "gn_torch": pin_gn_torch,
+    "gn_gate": pin_gn_gate,
+    "gn_head_local": pin_gn_head_local,
 }
 
 

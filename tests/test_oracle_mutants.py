@@ -49,6 +49,14 @@ MUTANTS = {
                                  "S[i * D + j] = w[i] * S[i * D + j] + kn * vt[j] + ut[j];"),
     "c2_decay_after_update": ("S[i * D + j] = w[i] * S[i * D + j] + kn * vt[j];",
                               "S[i * D + j] = w[i] * (S[i * D + j] + kn * vt[j]);"),
+    # per-head GroupNorm and gate
+    "gn_unbiased_var": ("s2 /= (double)D;", "s2 /= (double)(D - 1);"),
+    "gn_gamma_not_per_head": ("const double ga = gamma ? gamma[h * D + c] : 1.0;",
+                              "const double ga = gamma ? gamma[c] : 1.0;"),
+    "gn_gate_on_input": ("out[base + c] = ((x[base + c] - mu) * rs * ga + be) * gt;",
+                         "out[base + c] = ((x[base + c] * gt - mu) * rs * ga + be);"),
+    "gn_gate_before_beta": ("out[base + c] = ((x[base + c] - mu) * rs * ga + be) * gt;",
+                            "out[base + c] = (x[base + c] - mu) * rs * ga * gt + be;"),
 }
 
 
