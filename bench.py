@@ -63,7 +63,7 @@ CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
                             "internal.h"),
-                "sha256_16": "8b33ec275d194be7", "bytes": 541247232 + 120351744,
+                "sha256_16": "70892a82047ac1bf", "bytes": 541468160 + 120561920,
                 "workload": (8, 4096, 32),
                 "profile": "profiles/wkv6_fast_kernel_prefill_B8_T4096_H32_bf16.md"},
     "decode": {"sources": ("decode.cu", "common.cuh"),

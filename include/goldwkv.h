@@ -170,6 +170,46 @@ wkv_status wkv6c2_decode_step(const void *r, const void *k, const void *v, const
                               wkv_dtype io, const wkv_ln *ln, void *workspace,
                               size_t workspace_bytes, void *stream);
 
+/*
+ * Base Finch's own output stage, which Finch-C2 removes (GoldFinch review page, section 3.4
+ * "Finch-C2 Time Mixing": modification (1) removes the gate, (2) replaces the per-head
+ * GroupNorm with the full-width LayerNorm).  After the base recurrence at the top of this
+ * file, each head's D outputs of each token are normalised on their own and then multiplied
+ * by the gate:
+ *     y[b][t][h][c] <- ((y - mean_bth) / sqrt(var_bth + eps) * gamma[h*D + c]
+ *                       + beta[h*D + c]) * gate[b][t][h][c]
+ * mean / var (biased) over the D = 64 channels of head h of token (b,t).  The gate is an
+ * input: whatever activation produced it (the pages do not print the gate's form) is
+ * applied by the caller.
+ */
+typedef struct wkv_gn {
+    const float *gamma;        /* [H*D] device, fp32, required                             */
+    const float *beta;         /* [H*D] device, fp32, required                             */
+    float eps;                 /* added to the variance inside the square root; > 0      */
+    const void *gate;          /* device, dtype `io`, layout of y ([B][T][H][D] prefill,
+                                  [B][H][D] decode); NULL = no gate.  Must not overlap y,
+                                  the states or the workspace.                            */
+} wkv_gn;
+
+/*
+ * wkv6_prefill_gn: as wkv6_prefill (WKV_ALGO_AUTO; same layouts, aliasing rules and errors)
+ * with the GroupNorm + gate output stage above in place of LayerNorm.  gn is required.
+ * Workspace: wkv6_prefill_workspace_bytes(B, T, H, D, io, 1, WKV_ALGO_AUTO) -- the same as
+ * with LayerNorm (an fp32 staging copy of y when io is bf16).
+ */
+wkv_status wkv6_prefill_gn(const void *r, const void *k, const void *v, const void *omega,
+                           const float *u, const float *state_in, float *state_out, void *y,
+                           int B, int T, int H, int D, wkv_dtype io, const wkv_gn *gn,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* wkv6_decode_step_gn: as wkv6_decode_step with the GroupNorm + gate output stage (gn
+ * required; gate [B][H][D] io or NULL).  Workspace: wkv6_decode_workspace_bytes(B, H, D,
+ * io, 1). */
+wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, const void *omega,
+                               const float *u, float *state, void *y, int B, int H, int D,
+                               wkv_dtype io, const wkv_gn *gn, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
 /* Size of the scratch array built into the library for wkv6_prefill_static, per device. */
 #define WKV6_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 

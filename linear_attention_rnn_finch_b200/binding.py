@@ -34,6 +34,11 @@ class _LN(ctypes.Structure):
     _fields_ = [("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
+class _GN(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("eps", ctypes.c_float),
+                ("gate", ctypes.c_void_p)]
+
+
 def load(path: Path | str | None = None):
     """Load libgoldwkv.so (raises if it has not been built)."""
     global _lib
@@ -62,6 +67,10 @@ def load(path: Path | str | None = None):
     L.wkv6c2_decode_step.restype = i
     L.wkv6_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
     L.wkv6_decode_step.restype = i
+    L.wkv6_prefill_gn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+    L.wkv6_prefill_gn.restype = i
+    L.wkv6_decode_step_gn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
+    L.wkv6_decode_step_gn.restype = i
     L.wkv6_workspace_status.argtypes = [vp, vp]
     L.wkv6_workspace_status.restype = i
     L.wkv6_status_string.argtypes = [i]
@@ -319,4 +328,84 @@ def wkv6_decode_step(r, k, v, omega, u, state, *, ln=None, y=None, workspace=Non
                                 _stream_ptr(dev, stream))
     del ln_s
     _raise("wkv6_decode_step", st)
+    return y
+
+
+def _gn_struct(gn, H, D, device, dtype, gate_shape):
+    gamma, beta, eps, gate = gn
+    _check("gn.gamma", gamma, device, torch.float32, (H * D,))
+    _check("gn.beta", beta, device, torch.float32, (H * D,))
+    if gate is not None:
+        _check("gn.gate", gate, device, dtype, gate_shape)
+    s = _GN(gamma.data_ptr(), beta.data_ptr(), float(eps),
+            None if gate is None else gate.data_ptr())
+    return s, ctypes.byref(s)
+
+
+def wkv6_prefill_gn(r, k, v, omega, u, state_in=None, *, gn, y=None, state_out=None,
+                    want_state=True, workspace=None, stream=None):
+    """Base Finch prefill with its per-head GroupNorm and output gate (include/goldwkv.h,
+    wkv6_prefill_gn).  ``gn`` = (gamma [H*D], beta [H*D], eps, gate [B, T, H, D] or None).
+    Returns (y, state_out)."""
+    L = load()
+    if r.dim() != 4:
+        raise ValueError("r must be [B, T, H, D]")
+    B, T, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega)):
+        _check(name, t, dev, dt, (B, T, H, D))
+    _check("u", u, dev, torch.float32, (H, D))
+    if state_in is not None:
+        _check("state_in", state_in, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, T, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, T, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _check("state_out", state_out, dev, torch.float32, (B, H, D, D))
+    gn_s, gn_p = _gn_struct(gn, H, D, dev, dt, (B, T, H, D))
+    need = int(L.wkv6_prefill_workspace_bytes(B, T, H, D, _io(dt), 1, 0))
+    if workspace is None and need > 0:
+        workspace = new_workspace(need, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6_prefill_gn(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state_in),
+                               _ptr(state_out), _ptr(y), B, T, H, D, _io(dt), gn_p,
+                               _ptr(workspace), ws_bytes, _stream_ptr(dev, stream))
+    del gn_s
+    _raise("wkv6_prefill_gn", st)
+    return y, state_out
+
+
+def wkv6_decode_step_gn(r, k, v, omega, u, state, *, gn, y=None, workspace=None, stream=None):
+    """Base Finch step with per-head GroupNorm and gate; ``gn`` = (gamma, beta, eps,
+    gate [B, H, D] or None).  ``state`` is updated in place.  Returns y."""
+    L = load()
+    if r.dim() != 3:
+        raise ValueError("r must be [B, H, D]")
+    B, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega)):
+        _check(name, t, dev, dt, (B, H, D))
+    _check("u", u, dev, torch.float32, (H, D))
+    _check("state", state, dev, torch.float32, (B, H, D, D))
+    if y is None:
+        y = torch.empty((B, H, D), dtype=dt, device=dev)
+    _check("y", y, dev, dt, (B, H, D))
+    gn_s, gn_p = _gn_struct(gn, H, D, dev, dt, (B, H, D))
+    need = int(L.wkv6_decode_workspace_bytes(B, H, D, _io(dt), 1))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6_decode_step_gn(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state),
+                                   _ptr(y), B, H, D, _io(dt), gn_p, _ptr(workspace), ws_bytes,
+                                   _stream_ptr(dev, stream))
+    del gn_s
+    _raise("wkv6_decode_step_gn", st)
     return y

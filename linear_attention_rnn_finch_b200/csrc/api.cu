@@ -77,13 +77,55 @@ size_t io_size(wkv_dtype io) { return io == WKV_BF16 ? 2 : 4; }
 
 bool valid_io(wkv_dtype io) { return io == WKV_F32 || io == WKV_BF16; }
 
-wkv_status check_ln(const wkv_ln* ln, int H, int D, int dev_check) {
-    if (ln == nullptr) return WKV_OK;
-    if (!(ln->eps > 0.f) || ln->eps != ln->eps || ln->eps > 1e30f) return WKV_ERR_INVALID_ARG;
+// Output stage after the recurrence: none, LayerNorm over a token's H*D channels, or
+// base Finch's per-head GroupNorm times an optional gate.
+struct Norm {
+    enum Kind { kNone, kLayer, kGroup } kind = kNone;
+    const float* gamma = nullptr;
+    const float* beta = nullptr;
+    float eps = 0.f;
+    const void* gate = nullptr;   // GroupNorm only; dtype io, layout of y
+    bool on() const { return kind != kNone; }
+};
+
+Norm layer_norm(const wkv_ln* ln) {
+    Norm n;
+    if (ln) {
+        n.kind = Norm::kLayer;
+        n.gamma = ln->gamma;
+        n.beta = ln->beta;
+        n.eps = ln->eps;
+    }
+    return n;
+}
+
+Norm group_norm(const wkv_gn* gn) {
+    Norm n;
+    n.kind = Norm::kGroup;
+    n.gamma = gn->gamma;
+    n.beta = gn->beta;
+    n.eps = gn->eps;
+    n.gate = gn->gate;
+    return n;
+}
+
+// gamma / beta [H*D] fp32 required, eps finite and > 0, gate (xbytes) optional
+wkv_status check_norm(const Norm& n, int H, int D, size_t xbytes) {
+    if (!n.on()) return WKV_OK;
+    if (!(n.eps > 0.f) || n.eps != n.eps || n.eps > 1e30f) return WKV_ERR_INVALID_ARG;
     const size_t bytes = (size_t)H * D * sizeof(float);
-    Buf b[2] = {{ln->gamma, bytes, true}, {ln->beta, bytes, true}};
-    (void)dev_check;
-    return check_bufs(b, 2);
+    Buf b[3] = {{n.gamma, bytes, true}, {n.beta, bytes, true}, {n.gate, xbytes, false}};
+    return check_bufs(b, 3);
+}
+
+// Launch the output stage: y_raw (fp32 [rows][H*D]) -> y (io)
+cudaError_t launch_norm(const Norm& n, const float* y_raw, void* y, long tokens, int H, int D,
+                        bool bf16, cudaStream_t st) {
+    if (n.kind == Norm::kLayer)
+        return goldwkv::launch_layernorm_rows(y_raw, n.gamma, n.beta, n.eps, y, tokens, H * D,
+                                              bf16, st);
+    return goldwkv::launch_groupnorm_gate(y_raw, n.gamma, n.beta, n.eps, n.gate, y, tokens * H,
+                                          H, bf16, st);
 }
 
 // Which kernel serves a prefill call.
@@ -194,7 +236,7 @@ namespace {
 wkv_status prefill_impl(const void* r, const void* k, const void* v, const void* omega,
                         const float* u, const void* uprime, const float* state_in,
                         float* state_out, void* y, int B, int T, int H, int D, wkv_dtype io,
-                        const wkv_ln* ln, wkv_algo algo, void* workspace,
+                        const Norm& nm, wkv_algo algo, void* workspace,
                         size_t workspace_bytes, void* stream) {
     const bool c2 = uprime != nullptr;
     if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
@@ -218,7 +260,7 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
                   {workspace, workspace_bytes, false}, {uprime, xbytes, false}};
     wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
     if (s != WKV_OK) return s;
-    if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
+    if ((s = check_norm(nm, H, D, tokens ? xbytes : 0)) != WKV_OK) return s;
 
     // aliasing: state_out may equal state_in, nothing else may overlap an output
     const Span sy = span(y, tokens ? xbytes : 0), sso = span(state_out, state_out ? sbytes : 0);
@@ -226,20 +268,21 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
                         span(v, tokens ? xbytes : 0), span(omega, tokens ? xbytes : 0),
                         span(c2 ? nullptr : u, tokens && !c2 ? ubytes : 0),
                         span(state_in, state_in ? sbytes : 0),
-                        span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
-                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0),
-                        span(uprime, c2 && tokens ? xbytes : 0)};
+                        span(nm.gamma, nm.on() ? ubytes : 0),
+                        span(nm.beta, nm.on() ? ubytes : 0),
+                        span(uprime, c2 && tokens ? xbytes : 0),
+                        span(nm.gate, nm.gate && tokens ? xbytes : 0)};
     for (const Span& in : ins)
         if (overlaps(sy, in)) return WKV_ERR_INVALID_ARG;
     for (int i = 0; i < 5; ++i)
         if (overlaps(sso, ins[i])) return WKV_ERR_INVALID_ARG;
-    if (overlaps(sso, ins[8])) return WKV_ERR_INVALID_ARG;
+    if (overlaps(sso, ins[8]) || overlaps(sso, ins[9])) return WKV_ERR_INVALID_ARG;
     if (overlaps(sso, ins[6]) || overlaps(sso, ins[7]) || overlaps(sso, sy))
         return WKV_ERR_INVALID_ARG;
     if (state_in && state_out && state_in != state_out && overlaps(sso, ins[5]))
         return WKV_ERR_INVALID_ARG;
 
-    const size_t need = wkv6_prefill_workspace_bytes(B, T, H, D, io, ln != nullptr, algo);
+    const size_t need = wkv6_prefill_workspace_bytes(B, T, H, D, io, nm.on(), algo);
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
         const Span sw = span(workspace, need);
@@ -268,7 +311,7 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     const size_t hand_s = hand_i + (chunked ? handoff_ints_bytes(units) : 0);
     const size_t seg_at = hand_s + (chunked ? handoff_state_bytes(units) : 0);
     const size_t raw_at = chunked ? chunked_bytes(B, H, P) : 0;
-    if (ln) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
+    if (nm.on()) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
     if (chunked) {
         const long long budget = injected("timeout0") ? 0 : kSpinBudget;
@@ -309,18 +352,15 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
                                       H, bf16, var, st);
     }
     if (e != cudaSuccess) return WKV_ERR_CUDA;
-    if (ln) {
-        e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y,
-                                           (long)B * T, H * D, bf16, st);
-        if (e != cudaSuccess) return WKV_ERR_CUDA;
-    }
+    if (nm.on() && launch_norm(nm, y_raw, y, (long)B * T, H, D, bf16, st) != cudaSuccess)
+        return WKV_ERR_CUDA;
     return WKV_OK;
 }
 
 
 wkv_status decode_impl(const void* r, const void* k, const void* v, const void* omega,
                        const float* u, const void* uprime, float* state, void* y, int B, int H,
-                       int D, wkv_dtype io, const wkv_ln* ln, void* workspace,
+                       int D, wkv_dtype io, const Norm& nm, void* workspace,
                        size_t workspace_bytes, void* stream) {
     const bool c2 = uprime != nullptr;
     if (B < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
@@ -337,19 +377,20 @@ wkv_status decode_impl(const void* r, const void* k, const void* v, const void* 
                   {uprime, xbytes, false}};
     wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
     if (s != WKV_OK) return s;
-    if ((s = check_ln(ln, H, D, 1)) != WKV_OK) return s;
+    if ((s = check_norm(nm, H, D, xbytes)) != WKV_OK) return s;
 
     const Span sy = span(y, xbytes), ss = span(state, sbytes);
     const Span ins[] = {span(r, xbytes), span(k, xbytes), span(v, xbytes), span(omega, xbytes),
                         span(c2 ? nullptr : u, c2 ? 0 : ubytes),
-                        span(ln ? ln->gamma : nullptr, ln ? ubytes : 0),
-                        span(ln ? ln->beta : nullptr, ln ? ubytes : 0),
-                        span(uprime, c2 ? xbytes : 0)};
+                        span(nm.gamma, nm.on() ? ubytes : 0),
+                        span(nm.beta, nm.on() ? ubytes : 0),
+                        span(uprime, c2 ? xbytes : 0),
+                        span(nm.gate, nm.gate ? xbytes : 0)};
     if (overlaps(sy, ss)) return WKV_ERR_INVALID_ARG;
     for (const Span& in : ins)
         if (overlaps(sy, in) || overlaps(ss, in)) return WKV_ERR_INVALID_ARG;
 
-    const size_t need = wkv6_decode_workspace_bytes(B, H, D, io, ln != nullptr);
+    const size_t need = wkv6_decode_workspace_bytes(B, H, D, io, nm.on());
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
         const Span sw = span(workspace, need);
@@ -361,15 +402,12 @@ wkv_status decode_impl(const void* r, const void* k, const void* v, const void* 
 
     const bool bf16 = io == WKV_BF16;
     float* y_raw = nullptr;
-    if (ln) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
+    if (nm.on()) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
     cudaError_t e = goldwkv::launch_decode(r, k, v, omega, u, state, y, y_raw, B, H, bf16,
                                            goldwkv::Variant{uprime}, st);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
-    if (ln) {
-        e = goldwkv::launch_layernorm_rows(y_raw, ln->gamma, ln->beta, ln->eps, y, (long)B,
-                                           H * D, bf16, st);
-        if (e != cudaSuccess) return WKV_ERR_CUDA;
-    }
+    if (nm.on() && launch_norm(nm, y_raw, y, (long)B, H, D, bf16, st) != cudaSuccess)
+        return WKV_ERR_CUDA;
     return WKV_OK;
 }
 
@@ -382,8 +420,8 @@ wkv_status wkv6_prefill_algo(const void* r, const void* k, const void* v, const 
                              int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
                              wkv_algo algo, void* workspace, size_t workspace_bytes,
                              void* stream) {
-    return prefill_impl(r, k, v, omega, u, nullptr, state_in, state_out, y, B, T, H, D, io, ln,
-                        algo, workspace, workspace_bytes, stream);
+    return prefill_impl(r, k, v, omega, u, nullptr, state_in, state_out, y, B, T, H, D, io,
+                        layer_norm(ln), algo, workspace, workspace_bytes, stream);
 }
 
 wkv_status wkv6c2_prefill(const void* r, const void* k, const void* v, const void* omega,
@@ -393,7 +431,7 @@ wkv_status wkv6c2_prefill(const void* r, const void* k, const void* v, const voi
     // uprime may be null only for an empty problem, where only the state passes through
     if (B > 0 && T > 0 && H > 0 && uprime == nullptr) return WKV_ERR_INVALID_ARG;
     return prefill_impl(r, k, v, omega, nullptr, uprime, state_in, state_out, y, B, T, H, D, io,
-                        ln, WKV_ALGO_AUTO, workspace, workspace_bytes, stream);
+                        layer_norm(ln), WKV_ALGO_AUTO, workspace, workspace_bytes, stream);
 }
 
 wkv_status wkv6_workspace_status(void* workspace, void* stream) {
@@ -423,8 +461,8 @@ wkv_status wkv6_decode_step(const void* r, const void* k, const void* v, const v
                             const float* u, float* state, void* y, int B, int H, int D,
                             wkv_dtype io, const wkv_ln* ln, void* workspace,
                             size_t workspace_bytes, void* stream) {
-    return decode_impl(r, k, v, omega, u, nullptr, state, y, B, H, D, io, ln, workspace,
-                       workspace_bytes, stream);
+    return decode_impl(r, k, v, omega, u, nullptr, state, y, B, H, D, io, layer_norm(ln),
+                       workspace, workspace_bytes, stream);
 }
 
 wkv_status wkv6c2_decode_step(const void* r, const void* k, const void* v, const void* omega,
@@ -432,8 +470,26 @@ wkv_status wkv6c2_decode_step(const void* r, const void* k, const void* v, const
                               wkv_dtype io, const wkv_ln* ln, void* workspace,
                               size_t workspace_bytes, void* stream) {
     if (B > 0 && H > 0 && uprime == nullptr) return WKV_ERR_INVALID_ARG;
-    return decode_impl(r, k, v, omega, nullptr, uprime, state, y, B, H, D, io, ln, workspace,
-                       workspace_bytes, stream);
+    return decode_impl(r, k, v, omega, nullptr, uprime, state, y, B, H, D, io, layer_norm(ln),
+                       workspace, workspace_bytes, stream);
+}
+
+wkv_status wkv6_prefill_gn(const void* r, const void* k, const void* v, const void* omega,
+                           const float* u, const float* state_in, float* state_out, void* y,
+                           int B, int T, int H, int D, wkv_dtype io, const wkv_gn* gn,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (gn == nullptr) return WKV_ERR_INVALID_ARG;
+    return prefill_impl(r, k, v, omega, u, nullptr, state_in, state_out, y, B, T, H, D, io,
+                        group_norm(gn), WKV_ALGO_AUTO, workspace, workspace_bytes, stream);
+}
+
+wkv_status wkv6_decode_step_gn(const void* r, const void* k, const void* v, const void* omega,
+                               const float* u, float* state, void* y, int B, int H, int D,
+                               wkv_dtype io, const wkv_gn* gn, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    if (gn == nullptr) return WKV_ERR_INVALID_ARG;
+    return decode_impl(r, k, v, omega, u, nullptr, state, y, B, H, D, io, group_norm(gn),
+                       workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

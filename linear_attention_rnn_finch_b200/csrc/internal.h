@@ -32,6 +32,12 @@ cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const floa
                                   float eps, void* out, long rows, int C, bool bf16,
                                   cudaStream_t st);
 
+// Per-head GroupNorm (rows of 64 = one head of one token; gamma/beta [H*64], head = row % H)
+// then times gate (same layout as out, or null).  out may equal x (fp32).
+cudaError_t launch_groupnorm_gate(const float* x, const float* gamma, const float* beta, float eps,
+                                  const void* gate, void* out, long rows, int H, bool bf16,
+                                  cudaStream_t st);
+
 // ---- chunked tensor-core prefill (bf16 I/O)
 // TMA descriptor of a [B][T][H][64] bf16 tensor: box 64 channels x 1 head x 64 tokens.
 bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H);
