@@ -196,24 +196,33 @@ def sum_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False):
+def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False, gn=False):
     """Device-timed prefill calls of another workload shape: one line of its own (tokens/s and
     the fraction of the HBM roofline), inputs resident in HBM and larger than L2.  c2: the
-    Finch-C2 entry point (normalised key, second value u' read in place of the bonus)."""
+    Finch-C2 entry point (normalised key, second value u' read in place of the bonus).  gn:
+    base Finch's output stage (per-head GroupNorm, then a gate tensor read from HBM)."""
     import linear_attention_rnn_finch_b200 as gw
     inp = W.make_prefill_inputs(cfg, dev)
+    g = torch.Generator(device=dev).manual_seed(cfg.seed + 5)
     if c2:
-        g = torch.Generator(device=dev).manual_seed(cfg.seed + 5)
         inp["uprime"] = (torch.randn(inp["r"].shape, generator=g, device=dev) * 0.125).to(cfg.dtype)
     B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
+    if gn:
+        gn_args = (1.0 + 0.1 * torch.randn(H * D, generator=g, device=dev),
+                   0.1 * torch.randn(H * D, generator=g, device=dev), 64e-5,
+                   (2.0 * torch.rand(inp["r"].shape, generator=g, device=dev)).to(cfg.dtype))
     ln = (inp["gamma"], inp["beta"], inp["eps"]) if cfg.ln else None
-    ws = gw.new_workspace(gw.prefill_workspace_bytes(B, T, H, D, cfg.dtype, ln is not None, algo), dev)
+    ws = gw.new_workspace(gw.prefill_workspace_bytes(B, T, H, D, cfg.dtype, ln is not None or gn,
+                                                     algo), dev)
     y = torch.empty_like(inp["r"])
     s_out = torch.empty_like(inp["state0"])
     args_p = [inp[n] for n in ("r", "k", "v", "omega")]
 
     def call():
-        if c2:
+        if gn:
+            gw.wkv6_prefill_gn(*args_p, inp["u"], inp["state0"], gn=gn_args, y=y, state_out=s_out,
+                               workspace=ws)
+        elif c2:
             gw.wkv6c2_prefill(*args_p, inp["uprime"], inp["state0"], ln=ln, y=y, state_out=s_out,
                               workspace=ws)
         else:
@@ -232,14 +241,17 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False):
     e1.record(stream)
     e1.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
-    nbytes = prefill_bytes(B, T, H, D) + (B * T * H * D * 2 if c2 else 0)   # + u' read
-    # with LayerNorm the library also writes and re-reads an fp32 copy of y; the roofline
-    # counts only the bytes the operation itself must move
-    nbytes_note = ("LayerNorm runs as a second pass over an fp32 copy of y, not counted in the "
-                   "algorithmic bytes") if cfg.ln else None
-    line = {"workload": ("wkv6c2_" + cfg.name[5:]) if c2 else cfg.name, "B": B, "T": T, "H": H,
-            "D": D, "io": "bf16", "form": "Finch-C2 (normalised key, second value)" if c2 else
-            "base Finch (static bonus)",
+    # + u' read (C2) or + gate read (GroupNorm)
+    nbytes = prefill_bytes(B, T, H, D) + (B * T * H * D * 2 if c2 or gn else 0)
+    # with LayerNorm / GroupNorm the library also writes and re-reads an fp32 copy of y; the
+    # roofline counts only the bytes the operation itself must move
+    nbytes_note = (("GroupNorm + gate" if gn else "LayerNorm") + " runs as a second pass over an "
+                   "fp32 copy of y, not counted in the algorithmic bytes") if cfg.ln or gn else None
+    name = ("wkv6c2_" + cfg.name[5:]) if c2 else (cfg.name + "_groupnorm_gate") if gn else cfg.name
+    form = ("Finch-C2 (normalised key, second value)" if c2 else
+            "base Finch (static bonus), per-head GroupNorm and gate" if gn else
+            "base Finch (static bonus)")
+    line = {"workload": name, "B": B, "T": T, "H": H, "D": D, "io": "bf16", "form": form,
             "ln": bool(cfg.ln), "steps": steps, "ms_per_call": ms,
             "tokens_per_s": world * B * T / (ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm,
@@ -248,6 +260,8 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False):
     if nbytes_note:
         line["note"] = nbytes_note
     del inp, y, s_out, ws
+    if gn:
+        del gn_args
     torch.cuda.empty_cache()
     return line
 
@@ -414,12 +428,15 @@ def run_ours(args, world, rank, local):
         del dinp, dargs, state
 
     # the other prefill shapes: long context (one sequence per head; the library splits it
-    # into segments across SMs) and the decay-extreme stress with fused LayerNorm
+    # into segments across SMs), the decay-extreme stress with LayerNorm, and the 1.5B layer
+    # in Finch-C2's form and with base Finch's GroupNorm + gate
     if not args.no_other:
         out["other_prefill"] = [other_prefill(W.CONFIGS[2], dev, world, hbm, args.algo, steps=5),
                                 other_prefill(W.CONFIGS[4], dev, world, hbm, args.algo, steps=5),
                                 other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
-                                              c2=True)]
+                                              c2=True),
+                                other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
+                                              gn=True)]
 
     # end to end through the public API with host buffers: every step copies its inputs in
     # from pinned host memory and reads y and the final state back.  Steps are pipelined over

@@ -77,6 +77,9 @@ class Oracle:
         lib.wkv6_oracle_groupnorm_gate.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp,
                                                    dp, ctypes.c_double, dp, dp]
         lib.wkv6_oracle_groupnorm_gate.restype = ctypes.c_int
+        lib.wkv6_oracle_backward.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                             dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.wkv6_oracle_backward.restype = ctypes.c_int
         self._lib = lib
 
     @staticmethod
@@ -124,6 +127,26 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle decode failed rc={rc}")
         return y, st
+
+    def backward(self, r, k, v, omega, u, state_in, dy, dstate_out=None):
+        """Gradients of prefill: given dy = dL/dy [B,T,H,D] and dstate_out = dL/dstate_out
+        [B,H,D,D] (None: zero), returns (dr, dk, dv, domega [B,T,H,D], du [H,D] summed over
+        b and t, dstate_in [B,H,D,D]) as float64 arrays.  state_in None means zeros."""
+        r, k, v, omega, u, dy = (self._f64(x) for x in (r, k, v, omega, u, dy))
+        s_in, ds_out = self._f64(state_in), self._f64(dstate_out)
+        B, T, H, D = r.shape
+        assert k.shape == v.shape == omega.shape == dy.shape == r.shape and u.shape == (H, D)
+        dr, dk, dv, dom = (np.empty_like(r) for _ in range(4))
+        du = np.empty((H, D), dtype=np.float64)
+        ds_in = np.empty((B, H, D, D), dtype=np.float64)
+        rc = self._lib.wkv6_oracle_backward(B, T, H, D, self._ptr(r), self._ptr(k), self._ptr(v),
+                                            self._ptr(omega), self._ptr(u), self._ptr(s_in),
+                                            self._ptr(dy), self._ptr(ds_out), self._ptr(dr),
+                                            self._ptr(dk), self._ptr(dv), self._ptr(dom),
+                                            self._ptr(du), self._ptr(ds_in))
+        if rc != 0:
+            raise RuntimeError(f"oracle backward failed rc={rc}")
+        return dr, dk, dv, dom, du, ds_in
 
     def prefill_c2(self, r, k, v, omega, uprime, state_in=None, nthreads: int | None = None):
         """Finch-C2 exact form: key k (1 - w), second value uprime [B,T,H,D] added to the

@@ -326,3 +326,125 @@ int wkv6_oracle_groupnorm_gate(long N, int H, int D, const double *x, const doub
     return 0;
 }
 
+
+/* Backward pass of the base recurrence (wkv6_one_head) for one (b,h) sequence: the adjoint
+ * of the recursion written out by the chain rule, token by token in reverse.  The forward
+ * states are recomputed first and kept (Sall[t] = state before token t, t = 0..T).
+ * With G the gradient with respect to the state after token t (G = dstate_out, or zero, at
+ * the end of the sequence):
+ *   dv_t[j]  = sum_i G[i][j] k_t[i] + (sum_i r_t[i] u[i] k_t[i]) dy_t[j]
+ *   dk_t[i]  = sum_j G[i][j] v_t[j] + r_t[i] u[i] (v_t . dy_t)
+ *   dr_t[i]  = sum_j Sall[t][i][j] dy_t[j] + u[i] k_t[i] (v_t . dy_t)
+ *   dw_t[i]  = sum_j G[i][j] Sall[t][i][j]
+ *   domega_t = dw_t * dw/domega = dw_t * (-exp(omega_t) w_t)
+ *   du[i]   += r_t[i] k_t[i] (v_t . dy_t)
+ *   G[i][j]  = w_t[i] G[i][j] + r_t[i] dy_t[j]   (now the gradient of the state before t)
+ * and dstate_in = G at the start.  du_acc accumulates (summed over all calls). */
+static void wkv6_one_head_backward(long T, int D, long tstride,
+                                   const double *r, const double *k, const double *v,
+                                   const double *omega, const double *u, const double *s_in,
+                                   const double *dy, const double *ds_out,
+                                   double *dr, double *dk, double *dv, double *domega,
+                                   double *du_acc, double *ds_in, double *Sall, double *G)
+{
+    const long DD = (long)D * D;
+    for (long e = 0; e < DD; ++e)
+        Sall[e] = s_in ? s_in[e] : 0.0;
+    for (long t = 0; t < T; ++t) {
+        const double *kt = k + t * tstride, *vt = v + t * tstride, *ot = omega + t * tstride;
+        const double *Sb = Sall + t * DD;
+        double *Sa = Sall + (t + 1) * DD;
+        for (int i = 0; i < D; ++i) {
+            const double wi = exp(-exp(ot[i]));
+            for (int j = 0; j < D; ++j)
+                Sa[i * D + j] = wi * Sb[i * D + j] + kt[i] * vt[j];
+        }
+    }
+
+    for (long e = 0; e < DD; ++e)
+        G[e] = ds_out ? ds_out[e] : 0.0;
+    for (long t = T - 1; t >= 0; --t) {
+        const double *rt = r + t * tstride, *kt = k + t * tstride, *vt = v + t * tstride;
+        const double *ot = omega + t * tstride, *dyt = dy + t * tstride;
+        const double *Sprev = Sall + t * DD;          /* state before token t */
+        double *drt = dr + t * tstride, *dkt = dk + t * tstride, *dvt = dv + t * tstride;
+        double *dot = domega + t * tstride;
+
+        double vdy = 0.0, rku = 0.0;
+        for (int j = 0; j < D; ++j)
+            vdy += vt[j] * dyt[j];
+        for (int i = 0; i < D; ++i)
+            rku += rt[i] * u[i] * kt[i];
+
+        for (int j = 0; j < D; ++j) {
+            double g = 0.0;
+            for (int i = 0; i < D; ++i)
+                g += G[i * D + j] * kt[i];
+            dvt[j] = g + rku * dyt[j];
+        }
+        for (int i = 0; i < D; ++i) {
+            const double wi = exp(-exp(ot[i]));
+            double gk = 0.0, gr = 0.0, gw = 0.0;
+            for (int j = 0; j < D; ++j) {
+                gk += G[i * D + j] * vt[j];
+                gr += Sprev[i * D + j] * dyt[j];
+                gw += G[i * D + j] * Sprev[i * D + j];
+            }
+            dkt[i] = gk + rt[i] * u[i] * vdy;
+            drt[i] = gr + u[i] * kt[i] * vdy;
+            dot[i] = gw * (-exp(ot[i]) * wi);
+            du_acc[i] += rt[i] * kt[i] * vdy;
+        }
+        /* carry the gradient to the state before token t */
+        for (int i = 0; i < D; ++i) {
+            const double wi = exp(-exp(ot[i]));
+            for (int j = 0; j < D; ++j)
+                G[i * D + j] = wi * G[i * D + j] + rt[i] * dyt[j];
+        }
+    }
+    if (ds_in)
+        for (long e = 0; e < DD; ++e)
+            ds_in[e] = G[e];
+}
+
+/* Gradients of a loss L(y, state_out) with respect to every input of wkv6_oracle_prefill,
+ * given dy = dL/dy [B][T][H][D] and dstate_out = dL/dstate_out [B][H][D][D] (NULL: zero).
+ * Outputs dr, dk, dv, domega [B][T][H][D]; du [H][D] (summed over b and t); dstate_in
+ * [B][H][D][D] (NULL: not written).  state_in NULL means zeros.  Sequential over (b,h).
+ * Returns 0, -1 on bad arguments, -3 if memory for the kept states cannot be had. */
+int wkv6_oracle_backward(int B, long T, int H, int D,
+                         const double *r, const double *k, const double *v,
+                         const double *omega, const double *u, const double *state_in,
+                         const double *dy, const double *dstate_out,
+                         double *dr, double *dk, double *dv, double *domega,
+                         double *du, double *dstate_in)
+{
+    if (B < 0 || T < 0 || H < 0 || D <= 0)
+        return -1;
+    for (long e = 0; e < (long)H * D; ++e)
+        du[e] = 0.0;
+    if (B == 0 || H == 0)
+        return 0;
+    const long DD = (long)D * D;
+    double *Sall = (double *)malloc(sizeof(double) * (size_t)(T + 1) * (size_t)DD);
+    double *G = (double *)malloc(sizeof(double) * (size_t)DD);
+    if (!Sall || !G) {
+        free(Sall);
+        free(G);
+        return -3;
+    }
+    const long tstride = (long)H * D;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const size_t x0 = ((size_t)b * T * H + h) * D;
+            const size_t s0 = ((size_t)b * H + h) * DD;
+            wkv6_one_head_backward(T, D, tstride, r + x0, k + x0, v + x0, omega + x0,
+                                   u + (size_t)h * D, state_in ? state_in + s0 : NULL, dy + x0,
+                                   dstate_out ? dstate_out + s0 : NULL, dr + x0, dk + x0,
+                                   dv + x0, domega + x0, du + (size_t)h * D,
+                                   dstate_in ? dstate_in + s0 : NULL, Sall, G);
+        }
+    free(Sall);
+    free(G);
+    return 0;
+}

@@ -43,6 +43,19 @@ Base Finch's per-head GroupNorm and output gate:
                       gate 2x give x and 2x, a random gate gives the product);
 * gn_head_local     - changing one head's inputs changes only that head's outputs.
 
+The backward pass (gradients of a loss sum(y * dy) + sum(S_T * dS_T) with respect to r, k,
+v, omega, u and the initial state):
+
+* bwd_finite_diff   - central finite differences of that loss through the (pinned) forward
+                      entry point, every input element one by one, on tiny sizes;
+* bwd_autograd      - torch autograd through an independent torch statement of the
+                      explicit-sum form (products formed one by one), fp64;
+* bwd_decay_identity- the decay gradient equals the sum of the pair terms that straddle the
+                      token, which rearranges to
+                      dlog w_t = <S_T, dS_T>_row + sum_{s>t} r_s dr_s' - sum_{s>=t} k_s dk_s'
+                      (dr', dk' without their bonus parts): a relation between outputs;
+* bwd_empty         - T = 0: dS_0 = dS_T and every other gradient is zero.
+
 ``run_all(oracle)`` returns the list of failing pin names; the mutation test uses it to
 show that plausible mistakes planted in the oracle are caught.
 """
@@ -342,6 +355,101 @@ def pin_gn_head_local(o):
     return np.array_equal(a[:, [0, 1, 3]], b[:, [0, 1, 3]]) and not np.allclose(a[:, 2], b[:, 2])
 
 
+def _bwd_inputs(seed, B, T, H, D):
+    r, k, v, om, u, S0 = _inputs(seed, B, T, H, D, omega=(-3.0, 1.0))
+    g = _rng(seed + 100)
+    return r, k, v, om, u, S0, g.normal(0, 1.0, r.shape), g.normal(0, 1.0, S0.shape)
+
+
+def pin_bwd_finite_diff(o):
+    r, k, v, om, u, S0, dy, dS = _bwd_inputs(30, 2, 4, 2, 3)
+    got = o.backward(r, k, v, om, u, S0, dy, dS)
+
+    def loss(*a):
+        y, S = o.prefill(*a)
+        return float(np.sum(y * dy) + np.sum(S * dS))
+
+    base = [r, k, v, om, u, S0]
+    h = 1e-6
+    ok = True
+    for idx in range(6):          # got: dr, dk, dv, domega, du, dS0 -- the order of base
+        x = base[idx]
+        num = np.zeros_like(x)
+        for e in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[e] += h
+            xm[e] -= h
+            ap, am = list(base), list(base)
+            ap[idx], am[idx] = xp, xm
+            num[e] = (loss(*ap) - loss(*am)) / (2 * h)
+        ok &= _close(got[idx], num, rtol=1e-6)
+    return ok
+
+
+def _torch_explicit(r, k, v, om, u, S0):
+    """y and final state, explicit-sum form in torch (differentiable), products one by one."""
+    B, T, H, D = r.shape
+    w = torch.exp(-torch.exp(om))
+    ys, finals = [], []
+    for b in range(B):
+        yb, fb = [], []
+        for h in range(H):
+            rows = []
+            for t in range(T + 1):
+                wkv = S0[b, h]
+                for j in range(t):
+                    wkv = w[b, j, h][:, None] * wkv     # S0 decayed by every earlier token
+                for i in range(t):
+                    dec = torch.ones(D, dtype=r.dtype)
+                    for j in range(i + 1, t):
+                        dec = dec * w[b, j, h]
+                    wkv = wkv + (dec * k[b, i, h])[:, None] * v[b, i, h][None, :]
+                if t < T:
+                    rt = r[b, t, h]
+                    rows.append(rt @ wkv + torch.sum(rt * u[h] * k[b, t, h]) * v[b, t, h])
+                else:
+                    fb.append(wkv)
+            yb.append(torch.stack(rows))
+        ys.append(torch.stack(yb, dim=1))
+        finals.append(torch.stack(fb))
+    return torch.stack(ys), torch.stack(finals)
+
+
+def pin_bwd_autograd(o):
+    ok = True
+    for seed, (B, T, H, D) in [(31, (1, 5, 2, 4)), (32, (2, 3, 1, 6))]:
+        r, k, v, om, u, S0, dy, dS = _bwd_inputs(seed, B, T, H, D)
+        ts = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (r, k, v, om, u, S0)]
+        y, S = _torch_explicit(*ts)
+        (torch.sum(y * torch.tensor(dy)) + torch.sum(S * torch.tensor(dS))).backward()
+        got = o.backward(r, k, v, om, u, S0, dy, dS)
+        for g_or, t in zip(got, ts):
+            ok &= _close(g_or, t.grad.numpy(), rtol=1e-10)
+    return ok
+
+
+def pin_bwd_decay_identity(o):
+    r, k, v, om, u, S0, dy, dS = _bwd_inputs(33, 2, 7, 2, 5)
+    dr, dk, dv, dom, du, dS0 = o.backward(r, k, v, om, u, S0, dy, dS)
+    _, S_T = o.prefill(r, k, v, om, u, S0)
+    vdy = np.sum(v * dy, axis=-1, keepdims=True)
+    bonus = r * u[None, None] * k * vdy                  # r_t u k_t (v_t . dy_t), per channel
+    P = r * dr - bonus                                   # r_s dr_s without the bonus part
+    Q = k * dk - bonus                                   # k_s dk_s without the bonus part
+    E = np.einsum("bhij,bhij->bhi", S_T, dS)             # <S_T, dS_T> per row
+    T = r.shape[1]
+    dlog = np.empty_like(r)
+    for t in range(T):
+        dlog[:, t] = E + P[:, t + 1:].sum(axis=1) - Q[:, t:].sum(axis=1)
+    return _close(dom, dlog * (-np.exp(om)), rtol=1e-11)
+
+
+def pin_bwd_empty(o):
+    r, k, v, om, u, S0, dy, dS = _bwd_inputs(34, 2, 0, 3, 4)
+    dr, dk, dv, dom, du, dS0 = o.backward(r, k, v, om, u, S0, dy, dS)
+    return np.array_equal(dS0, dS) and not np.any(du) and dr.size == 0
+
+
 PINS = {
     "explicit_sum": pin_explicit_sum,
     "t1_closed_form": pin_t1_closed_form,
@@ -362,6 +470,10 @@ PINS = {
     "gn_torch": pin_gn_torch,
     "gn_gate": pin_gn_gate,
     "gn_head_local": pin_gn_head_local,
+    "bwd_finite_diff": pin_bwd_finite_diff,
+    "bwd_autograd": pin_bwd_autograd,
+    "bwd_decay_identity": pin_bwd_decay_identity,
+    "bwd_empty": pin_bwd_empty,
 }
 
 

@@ -57,6 +57,17 @@ MUTANTS = {
                          "out[base + c] = ((x[base + c] * gt - mu) * rs * ga + be);"),
     "gn_gate_before_beta": ("out[base + c] = ((x[base + c] - mu) * rs * ga + be) * gt;",
                             "out[base + c] = (x[base + c] - mu) * rs * ga * gt + be;"),
+    # backward pass
+    "bwd_dr_from_state_after": ("gr += Sprev[i * D + j] * dyt[j];",
+                                "gr += Sall[(t + 1) * DD + i * D + j] * dyt[j];"),
+    "bwd_dk_bonus_dropped": ("dkt[i] = gk + rt[i] * u[i] * vdy;", "dkt[i] = gk;"),
+    "bwd_domega_without_w": ("dot[i] = gw * (-exp(ot[i]) * wi);", "dot[i] = gw * (-exp(ot[i]));"),
+    "bwd_carry_on_columns": ("G[i * D + j] = wi * G[i * D + j] + rt[i] * dyt[j];",
+                             "G[i * D + j] = exp(-exp(ot[j])) * G[i * D + j] + rt[i] * dyt[j];"),
+    "bwd_carry_without_readout": ("G[i * D + j] = wi * G[i * D + j] + rt[i] * dyt[j];",
+                                  "G[i * D + j] = wi * G[i * D + j];"),
+    "bwd_dv_transposed": ("g += G[i * D + j] * kt[i];", "g += G[j * D + i] * kt[i];"),
+    "bwd_du_without_r": ("du_acc[i] += rt[i] * kt[i] * vdy;", "du_acc[i] += kt[i] * vdy;"),
 }
 
 
