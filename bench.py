@@ -51,6 +51,24 @@ def prefill_bytes(B, T, H, D=64, esz=2):
     return 5 * D * esz * B * T * H + 2 * D * D * 4 * B * H + H * D * 4
 
 
+def backward_flops(B, T, H, D=64):
+    """Algorithmic fp32 FLOPs of one backward call: three scans over every (b,h), each per
+    token a readout (D*D fused multiply-adds) and a state update w*X + a*b (D*D multiplies
+    and D*D fused multiply-adds): 2 + 1 + 2 = 5 FLOPs per state entry per scan."""
+    return 3 * 5 * D * D * B * T * H
+
+
+def backward_bytes(B, T, H, D=64, esz=2):
+    """Algorithmic HBM bytes of one backward call: r, k, v, omega, dy in and dr, dk, dv,
+    domega out (9*D*esz per token-head), state_in and dS_T in, dS_0 out (3*D*D*4 per head)."""
+    return 9 * D * esz * B * T * H + 3 * D * D * 4 * B * H + 2 * H * D * 4
+
+
+# FP32 CUDA-core peak of a B200 from its unit counts and clock: 148 SMs x 128 FP32 lanes x
+# 2 FLOPs per fused multiply-add x 1.965 GHz (clocks.max.sm).
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def decode_bytes(B, H, D=64, esz=2):
     """Algorithmic bytes of one decode step: state read + written, r/k/v/omega in, y out."""
     return B * H * (2 * D * D * 4 + 5 * D * esz) + H * D * 4
@@ -266,6 +284,50 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False, gn=False):
     return line
 
 
+def backward_line(cfg, dev, world, steps):
+    """Device-timed wkv6_backward on the prefill workload's shape (bf16 I/O): gradients of
+    r, k, v, omega, u and the initial state for a random dy and final-state gradient."""
+    import linear_attention_rnn_finch_b200 as gw
+    inp = W.make_prefill_inputs(cfg, dev)
+    g = torch.Generator(device=dev).manual_seed(cfg.seed + 7)
+    dy = torch.randn(inp["r"].shape, generator=g, device=dev).to(cfg.dtype)
+    dS = torch.randn(inp["state0"].shape, generator=g, device=dev) * 0.1
+    B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
+    ws = torch.empty(gw.backward_workspace_bytes(B, T, H, D, cfg.dtype), dtype=torch.uint8,
+                     device=dev)
+    args_b = [inp[n] for n in ("r", "k", "v", "omega", "u", "state0")]
+
+    def call():
+        return gw.wkv6_backward(*args_b, dy, dS, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    flops, nbytes = backward_flops(B, T, H, D), backward_bytes(B, T, H, D)
+    line = {"workload": "wkv6_backward_1p5b_layer", "B": B, "T": T, "H": H, "D": D, "io": "bf16",
+            "steps": steps, "ms_per_call": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+            "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
+                         "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
+                         "frac": flops / (ms / 1e3) / 1e12 / ALU_FP32_TFLOPS,
+                         "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                         "algorithmic_flops_per_call": flops},
+            "hbm": {"achieved_gbs": nbytes / (ms / 1e3) / 1e9, "algorithmic_bytes_per_call": nbytes},
+            "gpu_launches": 3 * steps,
+            "kernels": "wkv6_bwd_dr_dv_kernel, wkv6_bwd_dk_domega_kernel, wkv6_bwd_du_kernel"}
+    del inp, dy, dS, ws, args_b
+    torch.cuda.empty_cache()
+    return line
+
+
 # ------------------------------------------------------------------------------ oracle timing
 def oracle_sample(cfg, b_rows: int, t_tokens: int, seed_offset: int = 0):
     """Inputs of the oracle's bounded sample: b_rows batch rows x t_tokens tokens of cfg,
@@ -437,6 +499,7 @@ def run_ours(args, world, rank, local):
                                               c2=True),
                                 other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
                                               gn=True)]
+        out["backward"] = backward_line(W.CONFIGS[1], dev, world, steps=5)
 
     # end to end through the public API with host buffers: every step copies its inputs in
     # from pinned host memory and reads y and the final state back.  Steps are pipelined over

@@ -210,6 +210,37 @@ wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, cons
                                wkv_dtype io, const wkv_gn *gn, void *workspace,
                                size_t workspace_bytes, void *stream);
 
+/*
+ * Backward pass of the base recurrence (wkv6_prefill without LayerNorm) for training: the
+ * gradients of a loss L with respect to every input, given dy = dL/dy and, optionally,
+ * dstate_out = dL/dstate_out.  Training with all tokens in parallel is section 3.4
+ * "Training and Inference Procedures" of the GoldFinch review page; the gradients are
+ * the chain rule applied to the recurrence at the top of this file (G the gradient of the
+ * state after token t, G = dstate_out after the last token):
+ *     dr_t = S_{t-1} dy_t + u * k_t (v_t . dy_t)        dk_t = G v_t + u * r_t (v_t . dy_t)
+ *     dv_t = G^T k_t + (r_t . (u * k_t)) dy_t           du   = sum_{b,t} r_t * k_t (v_t . dy_t)
+ *     domega_t[i] = (sum_j G[i][j] S_{t-1}[i][j]) * w_t[i] * (-exp(omega_t[i]))
+ *     G <- diag(w_t) G + r_t^T dy_t,   dstate_in = G before the first token.
+ * The three scans run on CUDA cores in fp32 (the decay gradient through the equivalent sum
+ * of the pair terms that straddle each token).
+ *   r, k, v, omega, u, state_in   the forward call's inputs (state_in NULL = zeros)
+ *   dy          [B][T][H][D] io   gradient of y
+ *   dstate_out  [B][H][D][D] fp32 gradient of the final state, or NULL (zero)
+ *   dr, dk, dv, domega [B][T][H][D] io   outputs
+ *   du          [H][D] fp32       output, summed over batch and tokens (overwritten)
+ *   dstate_in   [B][H][D][D] fp32 output, or NULL (not computed)
+ *   workspace   at least wkv6_backward_workspace_bytes(...) bytes; no initial contents needed.
+ * No output may overlap an input, another output or the workspace.  T = 0: du = 0 and
+ * dstate_in = dstate_out (or zero).
+ */
+size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io);
+
+wkv_status wkv6_backward(const void *r, const void *k, const void *v, const void *omega,
+                         const float *u, const float *state_in, const void *dy,
+                         const float *dstate_out, void *dr, void *dk, void *dv, void *domega,
+                         float *du, float *dstate_in, int B, int T, int H, int D, wkv_dtype io,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
 /* Size of the scratch array built into the library for wkv6_prefill_static, per device. */
 #define WKV6_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 

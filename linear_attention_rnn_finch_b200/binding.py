@@ -71,6 +71,10 @@ def load(path: Path | str | None = None):
     L.wkv6_prefill_gn.restype = i
     L.wkv6_decode_step_gn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
     L.wkv6_decode_step_gn.restype = i
+    L.wkv6_backward_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.wkv6_backward_workspace_bytes.restype = sz
+    L.wkv6_backward.argtypes = [vp] * 14 + [i, i, i, i, i, vp, sz, vp]
+    L.wkv6_backward.restype = i
     L.wkv6_workspace_status.argtypes = [vp, vp]
     L.wkv6_workspace_status.restype = i
     L.wkv6_status_string.argtypes = [i]
@@ -409,3 +413,41 @@ def wkv6_decode_step_gn(r, k, v, omega, u, state, *, gn, y=None, workspace=None,
     del gn_s
     _raise("wkv6_decode_step_gn", st)
     return y
+
+
+def wkv6_backward(r, k, v, omega, u, state_in, dy, dstate_out=None, *, want_dstate_in=True,
+                  workspace=None, stream=None):
+    """Gradients of wkv6_prefill (no LayerNorm) given dy [B, T, H, D] (dtype of r) and the
+    final-state gradient dstate_out [B, H, D, D] fp32 (None: zero).  Returns
+    (dr, dk, dv, domega, du [H, D] fp32, dstate_in [B, H, D, D] fp32 or None)."""
+    L = load()
+    if r.dim() != 4:
+        raise ValueError("r must be [B, T, H, D]")
+    B, T, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega), ("dy", dy)):
+        _check(name, t, dev, dt, (B, T, H, D))
+    _check("u", u, dev, torch.float32, (H, D))
+    for name, t in (("state_in", state_in), ("dstate_out", dstate_out)):
+        if t is not None:
+            _check(name, t, dev, torch.float32, (B, H, D, D))
+    dr, dk, dv, dom = (torch.empty((B, T, H, D), dtype=dt, device=dev) for _ in range(4))
+    du = torch.empty((H, D), dtype=torch.float32, device=dev)
+    ds_in = torch.empty((B, H, D, D), dtype=torch.float32, device=dev) if want_dstate_in else None
+    need = int(L.wkv6_backward_workspace_bytes(B, T, H, D, _io(dt)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6_backward(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state_in),
+                             _ptr(dy), _ptr(dstate_out), _ptr(dr), _ptr(dk), _ptr(dv), _ptr(dom),
+                             _ptr(du), _ptr(ds_in), B, T, H, D, _io(dt), _ptr(workspace),
+                             ws_bytes, _stream_ptr(dev, stream))
+    _raise("wkv6_backward", st)
+    return dr, dk, dv, dom, du, ds_in
+
+
+def backward_workspace_bytes(B, T, H, D, io_dtype) -> int:
+    return int(load().wkv6_backward_workspace_bytes(B, T, H, D, _io(io_dtype)))

@@ -7,6 +7,7 @@
 
 #include "goldwkv.h"
 #include "internal.h"
+#include "backward.h"
 
 namespace {
 
@@ -490,6 +491,79 @@ wkv_status wkv6_decode_step_gn(const void* r, const void* k, const void* v, cons
     if (gn == nullptr) return WKV_ERR_INVALID_ARG;
     return decode_impl(r, k, v, omega, u, nullptr, state, y, B, H, D, io, group_norm(gn),
                        workspace, workspace_bytes, stream);
+}
+
+
+size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
+    if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
+    // P and E in the row scans' accumulation type: fp64 for fp32 I/O, fp32 for bf16 I/O
+    const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
+    const size_t x = (size_t)B * T * H * D, bh = (size_t)B * H * D;
+    return round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
+}
+
+wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void* omega,
+                         const float* u, const float* state_in, const void* dy,
+                         const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
+                         float* du, float* dstate_in, int B, int T, int H, int D, wkv_dtype io,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
+    if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
+    if (H == 0) return WKV_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t xbytes = (size_t)B * T * H * D * io_size(io);
+    const size_t sbytes = (size_t)B * H * D * D * sizeof(float);
+    const size_t ubytes = (size_t)H * D * sizeof(float);
+    const bool tokens = B > 0 && T > 0;
+    Buf bufs[] = {{r, xbytes, tokens},      {k, xbytes, tokens},         {v, xbytes, tokens},
+                  {omega, xbytes, tokens},  {dy, xbytes, tokens},        {u, ubytes, tokens},
+                  {dr, xbytes, tokens},     {dk, xbytes, tokens},        {dv, xbytes, tokens},
+                  {domega, xbytes, tokens}, {du, ubytes, true},          {state_in, sbytes, false},
+                  {dstate_out, sbytes, false}, {dstate_in, sbytes, false},
+                  {workspace, workspace_bytes, false}};
+    wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
+    if (s != WKV_OK) return s;
+
+    // no output may overlap an input, another output or the workspace
+    const size_t xb = tokens ? xbytes : 0, sb = B > 0 ? sbytes : 0;
+    const Span ins[] = {span(r, xb), span(k, xb), span(v, xb), span(omega, xb), span(dy, xb),
+                        span(u, tokens ? ubytes : 0), span(state_in, state_in ? sb : 0),
+                        span(dstate_out, dstate_out ? sb : 0)};
+    const Span outs[] = {span(dr, xb), span(dk, xb), span(dv, xb), span(domega, xb),
+                         span(du, ubytes), span(dstate_in, dstate_in ? sb : 0)};
+    const int n_outs = (int)(sizeof(outs) / sizeof(outs[0]));
+    for (int a = 0; a < n_outs; ++a) {
+        for (const Span& in : ins)
+            if (overlaps(outs[a], in)) return WKV_ERR_INVALID_ARG;
+        for (int b2 = a + 1; b2 < n_outs; ++b2)
+            if (overlaps(outs[a], outs[b2])) return WKV_ERR_INVALID_ARG;
+    }
+    const size_t need = wkv6_backward_workspace_bytes(B, T, H, D, io);
+    if (need > 0) {
+        if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+        const Span sw = span(workspace, need);
+        for (const Span& in : ins)
+            if (overlaps(sw, in)) return WKV_ERR_INVALID_ARG;
+        for (const Span& o : outs)
+            if (overlaps(sw, o)) return WKV_ERR_INVALID_ARG;
+    }
+    if (injected("launch")) return WKV_ERR_CUDA;
+
+    if (!tokens) {   // no token: du = 0, and the state gradient passes through unchanged
+        if (cudaMemsetAsync(du, 0, ubytes, st) != cudaSuccess) return WKV_ERR_CUDA;
+        if (dstate_in == nullptr || B == 0) return WKV_OK;
+        if (dstate_out) return from_cuda(cudaMemcpyAsync(dstate_in, dstate_out, sbytes,
+                                                         cudaMemcpyDeviceToDevice, st));
+        return from_cuda(cudaMemsetAsync(dstate_in, 0, sbytes, st));
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
+    void* P = ws;
+    uint8_t* E = ws + round256((size_t)B * T * H * D * acc);
+    float* du_part = reinterpret_cast<float*>(E + round256((size_t)B * H * D * acc));
+    return from_cuda(goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr,
+                                              dk, dv, domega, du, dstate_in, P, E, du_part, B,
+                                              T, H, io == WKV_BF16, st));
 }
 
 }  // extern "C"

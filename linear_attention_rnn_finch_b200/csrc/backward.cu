@@ -1,0 +1,404 @@
+// Backward pass of the WKV6 recurrence on CUDA cores, fp32 state and arithmetic.
+//
+// Forward (GoldFinch review page, section 3.4 "Recurrent state update and output", with the
+// base-Finch bonus u): per (b,h)
+//     y_t[j]  = sum_i r_t[i] S[i][j] + (sum_i r_t[i] u[i] k_t[i]) v_t[j]
+//     S[i][j] = w_t[i] S[i][j] + k_t[i] v_t[j],     w_t = exp(-exp(omega_t)),
+// S the state before token t.  Given dy and dS_T (the gradient of the final state), the
+// chain rule gives, with G_t the gradient of the state after token t
+// (G_{t-1} = diag(w_t) G_t + r_t^T dy_t, G_{T-1} = dS_T):
+//     dr_t[i] = sum_j S_{t-1}[i][j] dy_t[j] + u[i] k_t[i] (v_t . dy_t)
+//     dk_t[i] = sum_j G_t[i][j] v_t[j]      + u[i] r_t[i] (v_t . dy_t)
+//     dv_t[j] = sum_i k_t[i] G_t[i][j]      + (sum_i r_t[i] u[i] k_t[i]) dy_t[j]
+//     du[i]   = sum_{b,t} r_t[i] k_t[i] (v_t . dy_t),     dS_0 = G before the first token.
+// The decay gradient is the sum of the pair terms (source token tau, reading token s) whose
+// decay product contains w_t, i.e. tau < t < s.  Writing P_s = r_s * (dr_s without bonus)
+// and Q_s = k_s * (dk_s without bonus) -- each the sum of the pair terms ending / starting at
+// s -- and E = sum_j S_T[i][j] dS_T[i][j] for the pairs that end in the final state,
+//     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,     domega_t = dlog w_t * (-exp(omega_t)).
+//
+// Three sweeps, each a token-by-token scan like the forward recurrent kernel:
+//   dr  rows of S (reduce over j), forward in time; also writes P, E and per-(b,h) du parts
+//   dv  columns of G (reduce over i), reverse in time -- the forward recurrence with the
+//       roles r <-> k, v -> dy run backwards
+//   dk  rows of G, reverse in time, with the decay-gradient scan fused (needs P and E).
+// The dr and dv sweeps run as one launch (blockIdx.z); the dk sweep follows; a small kernel
+// sums du over the batch.
+//
+// Work split: a CTA owns one (b,h) and 32 of the 64 rows (or columns); thread (row, q)
+// keeps 16 state entries in registers, the sum over the other index is finished with two
+// xor-shuffles across the four q-threads of a row.  Tokens are staged through shared memory
+// in tiles of kTile; per-token outputs are staged too and written coalesced per tile.
+//
+// Precision.  The identity subtracts, at every token, the pair terms that start at or after
+// it; where w_t is tiny the result is tiny too and what is left is the rounding of those
+// terms, times exp(omega_t).  With bf16 I/O that residue is far below the output rounding,
+// and the row scans run in fp32.  With fp32 I/O (the precision path) the two row scans, P
+// and E keep fp64, so the residue stays at fp64 rounding; the dv scan stays fp32.
+#include "common.cuh"
+#include "backward.h"
+
+namespace goldwkv {
+
+namespace {
+
+constexpr int kHalf = 32;        // rows (or columns) per CTA
+constexpr int kThreads = 128;    // 32 rows x 4 column quarters
+
+// Accumulation type of the row scans and tokens per shared-memory tile, per I/O type.
+template <typename IO> struct Prec {
+    using Acc = float;
+    static constexpr int kTile = 32;
+};
+template <> struct Prec<float> {
+    using Acc = double;
+    static constexpr int kTile = 16;
+};
+
+template <typename Acc, int kTile>
+struct RowSmem {
+    float b[kTile][kHeadSize];   // right factor of the update (v: dr sweep, dy: dk sweep)
+    float q[kTile][kHeadSize];   // readout vector (dy: dr sweep, v: dk sweep)
+    float a[kTile][kHalf];       // left factor of the update, this CTA's rows (k | r)
+    float m[kTile][kHalf];       // the other of r / k, this CTA's rows (P or Q product)
+    float w[kTile][kHalf];       // decay
+    float ne[kTile][kHalf];      // -exp(omega): d w / d omega = w * ne  (dk sweep)
+    Acc p[kTile][kHalf];         // P of the dr sweep (dk sweep)
+    Acc o2[kTile][kHalf];        // staged P (dr sweep) / domega (dk sweep)
+    float o1[kTile][kHalf];      // staged dr / dk
+    float vdy[kTile];            // v_t . dy_t
+    float u[kHalf];
+};
+
+template <int kTile>
+struct ColSmem {
+    float k[kTile][kHeadSize];
+    float r[kTile][kHeadSize];
+    float w[kTile][kHeadSize];
+    float dy[kTile][kHalf];      // this CTA's columns
+    float o[kTile][kHalf];       // staged dv
+    float rku[kTile];            // sum_i r_t[i] u[i] k_t[i]
+    float u[kHeadSize];
+};
+
+// Token-major element (b, t, h, c): ((b*T + t)*H + h)*64 + c.
+__device__ __forceinline__ size_t tok_index(size_t xbase, int t, size_t tstride, int c) {
+    return xbase + (size_t)t * tstride + c;
+}
+
+// kRev == false: the dr sweep (a = k, m = r, b = v, q = dy, X0 = state_in), forward in time.
+// kRev == true : the dk sweep (a = r, m = k, b = dy, q = v, X0 = dS_T), reverse in time, with
+//                the decay-gradient scan (reads P and E written by the dr sweep).
+template <typename IO, bool kRev, typename Acc = typename Prec<IO>::Acc,
+          int kTile = Prec<IO>::kTile>
+__device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __restrict__ a_src,
+                                          const IO* __restrict__ m_src,
+                                          const IO* __restrict__ b_src,
+                                          const IO* __restrict__ q_src,
+                                          const IO* __restrict__ omega,
+                                          const float* __restrict__ u, const float* x0,
+                                          IO* __restrict__ out, Acc* __restrict__ P,
+                                          IO* __restrict__ domega, Acc* __restrict__ E,
+                                          const float* __restrict__ dS_T,
+                                          float* __restrict__ du_part, float* x_final, int T,
+                                          int H) {
+    constexpr int D = kHeadSize;
+    const int bh = blockIdx.x;
+    const int b = bh / H, h = bh - (bh / H) * H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int qq = lane & 3;                    // column quarter: columns 16qq .. 16qq+15
+    const int rl = warp * 8 + (lane >> 2);      // local row 0..31
+    const int rowbase = blockIdx.y * kHalf;
+    const int i = rowbase + rl;
+
+    if (tid < kHalf) s.u[tid] = u[h * D + rowbase + tid];
+
+    const size_t sbase = (size_t)bh * D * D + (size_t)i * D + 16 * qq;
+    Acc X[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) X[m] = x0 ? (Acc)x0[sbase + m] : Acc(0);
+
+    const size_t tstride = (size_t)H * D;
+    const size_t xbase = ((size_t)b * T * H + h) * D;
+    const int ntile = (T + kTile - 1) / kTile;
+    Acc du_acc = 0, accP = 0, accQ = 0;
+    const Acc Ei = kRev ? E[(size_t)bh * D + i] : Acc(0);
+
+    for (int it = 0; it < ntile; ++it) {
+        const int tile = kRev ? ntile - 1 - it : it;
+        const int t0 = tile * kTile;
+        const int nt = min(kTile, T - t0);
+        __syncthreads();   // previous tile consumed and flushed
+        for (int idx = tid; idx < kTile * D; idx += kThreads) {
+            const int tt = idx / D, c = idx - (idx / D) * D;
+            float bv = 0.f, qv = 0.f;
+            if (tt < nt) {
+                const size_t g = tok_index(xbase, t0 + tt, tstride, c);
+                bv = to_f32(b_src[g]);
+                qv = to_f32(q_src[g]);
+            }
+            s.b[tt][c] = bv;
+            s.q[tt][c] = qv;
+        }
+        for (int idx = tid; idx < kTile * kHalf; idx += kThreads) {
+            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
+            float av = 0.f, mv = 0.f, ne = 0.f;
+            Acc pv = 0;
+            if (tt < nt) {
+                const size_t g = tok_index(xbase, t0 + tt, tstride, rowbase + c);
+                av = to_f32(a_src[g]);
+                mv = to_f32(m_src[g]);
+                ne = -expf(to_f32(omega[g]));
+                if (kRev) pv = P[g];
+            }
+            s.a[tt][c] = av;
+            s.m[tt][c] = mv;
+            s.ne[tt][c] = ne;
+            s.w[tt][c] = expf(ne);
+            s.p[tt][c] = pv;
+        }
+        __syncthreads();
+        for (int tt = warp * (kTile / 4); tt < (warp + 1) * (kTile / 4); ++tt) {
+            const float p = warp_sum(s.b[tt][lane] * s.q[tt][lane] +
+                                     s.b[tt][lane + 32] * s.q[tt][lane + 32]);
+            if (lane == 0) s.vdy[tt] = p;
+        }
+        __syncthreads();
+
+        for (int st = 0; st < nt; ++st) {
+            const int tt = kRev ? nt - 1 - st : st;
+            const float4* q4 = reinterpret_cast<const float4*>(&s.q[tt][16 * qq]);
+            const float4* b4 = reinterpret_cast<const float4*>(&s.b[tt][16 * qq]);
+            const Acc ai = s.a[tt][rl], wi = s.w[tt][rl];
+            Acc acc0 = 0, acc1 = 0;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 qv = q4[m4], bv = b4[m4];
+                Acc* x = &X[4 * m4];
+                acc0 += x[0] * (Acc)qv.x;
+                acc1 += x[1] * (Acc)qv.y;
+                acc0 += x[2] * (Acc)qv.z;
+                acc1 += x[3] * (Acc)qv.w;
+                x[0] = wi * x[0] + ai * (Acc)bv.x;
+                x[1] = wi * x[1] + ai * (Acc)bv.y;
+                x[2] = wi * x[2] + ai * (Acc)bv.z;
+                x[3] = wi * x[3] + ai * (Acc)bv.w;
+            }
+            Acc acc = acc0 + acc1;
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (qq == 0) {
+                const Acc vdy = s.vdy[tt], mi = s.m[tt][rl];
+                const Acc bonus = (Acc)s.u[rl] * ai * vdy;
+                s.o1[tt][rl] = (float)(acc + bonus);
+                if (!kRev) {
+                    s.o2[tt][rl] = mi * acc;          // P_t: pair terms ending at t
+                    du_acc += mi * ai * vdy;
+                } else {
+                    accQ += mi * acc;                 // Q_t: pair terms starting at t
+                    s.o2[tt][rl] = (Ei + accP - accQ) * (Acc)s.ne[tt][rl];
+                    accP += s.p[tt][rl];
+                }
+            }
+        }
+        __syncthreads();
+        for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
+            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
+            const size_t g = tok_index(xbase, t0 + tt, tstride, rowbase + c);
+            out[g] = from_f32<IO>(s.o1[tt][c]);
+            if (!kRev) P[g] = s.o2[tt][c];
+            else domega[g] = from_f32<IO>((float)s.o2[tt][c]);
+        }
+    }
+
+    if (!kRev) {
+        Acc e = 0;
+        if (dS_T) {
+#pragma unroll
+            for (int m = 0; m < 16; ++m) e += X[m] * (Acc)dS_T[sbase + m];
+        }
+        e += __shfl_xor_sync(0xffffffffu, e, 1);
+        e += __shfl_xor_sync(0xffffffffu, e, 2);
+        if (qq == 0) {
+            E[(size_t)bh * D + i] = e;
+            du_part[(size_t)bh * D + i] = (float)du_acc;
+        }
+    } else if (x_final) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) x_final[sbase + m] = (float)X[m];
+    }
+}
+
+// The dv sweep: columns of G, reverse in time (the forward recurrence with r <-> k, v -> dy).
+template <typename IO, int kTile = Prec<IO>::kTile>
+__device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restrict__ r,
+                                          const IO* __restrict__ k, const IO* __restrict__ omega,
+                                          const IO* __restrict__ dy, const float* __restrict__ u,
+                                          const float* __restrict__ dS_T, IO* __restrict__ dv,
+                                          int T, int H) {
+    constexpr int D = kHeadSize;
+    const int bh = blockIdx.x;
+    const int b = bh / H, h = bh - (bh / H) * H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int qq = lane & 3;                    // row quarter: rows 16qq .. 16qq+15
+    const int jl = warp * 8 + (lane >> 2);      // local column 0..31
+    const int colbase = blockIdx.y * kHalf;
+    const int j = colbase + jl;
+
+    if (tid < D) s.u[tid] = u[h * D + tid];
+
+    const size_t sbase = (size_t)bh * D * D;
+    float G[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) G[m] = dS_T ? dS_T[sbase + (size_t)(16 * qq + m) * D + j] : 0.f;
+
+    const size_t tstride = (size_t)H * D;
+    const size_t xbase = ((size_t)b * T * H + h) * D;
+    const int ntile = (T + kTile - 1) / kTile;
+    for (int it = 0; it < ntile; ++it) {
+        const int t0 = (ntile - 1 - it) * kTile;
+        const int nt = min(kTile, T - t0);
+        __syncthreads();
+        for (int idx = tid; idx < kTile * D; idx += kThreads) {
+            const int tt = idx / D, c = idx - (idx / D) * D;
+            float rv = 0.f, kv = 0.f, wv = 1.f;
+            if (tt < nt) {
+                const size_t g = tok_index(xbase, t0 + tt, tstride, c);
+                rv = to_f32(r[g]);
+                kv = to_f32(k[g]);
+                wv = decay_from_logit(to_f32(omega[g]));
+            }
+            s.r[tt][c] = rv;
+            s.k[tt][c] = kv;
+            s.w[tt][c] = wv;
+        }
+        for (int idx = tid; idx < kTile * kHalf; idx += kThreads) {
+            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
+            s.dy[tt][c] = tt < nt ? to_f32(dy[tok_index(xbase, t0 + tt, tstride, colbase + c)]) : 0.f;
+        }
+        __syncthreads();
+        for (int tt = warp * (kTile / 4); tt < (warp + 1) * (kTile / 4); ++tt) {
+            const float p = warp_sum(s.r[tt][lane] * s.u[lane] * s.k[tt][lane] +
+                                     s.r[tt][lane + 32] * s.u[lane + 32] * s.k[tt][lane + 32]);
+            if (lane == 0) s.rku[tt] = p;
+        }
+        __syncthreads();
+
+        for (int st = 0; st < nt; ++st) {
+            const int tt = nt - 1 - st;
+            const float4* k4 = reinterpret_cast<const float4*>(&s.k[tt][16 * qq]);
+            const float4* r4 = reinterpret_cast<const float4*>(&s.r[tt][16 * qq]);
+            const float4* w4 = reinterpret_cast<const float4*>(&s.w[tt][16 * qq]);
+            const float dyj = s.dy[tt][jl];
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 kk = k4[m4], rr = r4[m4], ww = w4[m4];
+                float* g = &G[4 * m4];
+                acc0 = fmaf(kk.x, g[0], acc0);
+                acc1 = fmaf(kk.y, g[1], acc1);
+                acc0 = fmaf(kk.z, g[2], acc0);
+                acc1 = fmaf(kk.w, g[3], acc1);
+                g[0] = fmaf(ww.x, g[0], rr.x * dyj);
+                g[1] = fmaf(ww.y, g[1], rr.y * dyj);
+                g[2] = fmaf(ww.z, g[2], rr.z * dyj);
+                g[3] = fmaf(ww.w, g[3], rr.w * dyj);
+            }
+            float acc = acc0 + acc1;
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (qq == 0) s.o[tt][jl] = fmaf(s.rku[tt], dyj, acc);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
+            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
+            dv[tok_index(xbase, t0 + tt, tstride, colbase + c)] = from_f32<IO>(s.o[tt][c]);
+        }
+    }
+}
+
+template <typename IO>
+struct SweepSmem {
+    using Row = RowSmem<typename Prec<IO>::Acc, Prec<IO>::kTile>;
+    using Col = ColSmem<Prec<IO>::kTile>;
+    static constexpr size_t kBytes = sizeof(Row) > sizeof(Col) ? sizeof(Row) : sizeof(Col);
+};
+
+// blockIdx.z == 0: dr sweep; blockIdx.z == 1: dv sweep.
+template <typename IO>
+__global__ void __launch_bounds__(kThreads)
+wkv6_bwd_dr_dv_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
+                      const IO* __restrict__ v, const IO* __restrict__ omega,
+                      const float* __restrict__ u, const float* state_in, const IO* __restrict__ dy,
+                      const float* __restrict__ dS_T, IO* __restrict__ dr, IO* __restrict__ dv,
+                      typename Prec<IO>::Acc* __restrict__ P, typename Prec<IO>::Acc* __restrict__ E,
+                      float* __restrict__ du_part, int T, int H) {
+    using Sm = SweepSmem<IO>;
+    __shared__ __align__(16) unsigned char smem[Sm::kBytes];
+    if (blockIdx.z == 0)
+        row_sweep<IO, false>(*reinterpret_cast<typename Sm::Row*>(smem), k, r, v, dy, omega, u,
+                             state_in, dr, P, nullptr, E, dS_T, du_part, nullptr, T, H);
+    else
+        col_sweep<IO>(*reinterpret_cast<typename Sm::Col*>(smem), r, k, omega, dy, u, dS_T, dv,
+                      T, H);
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(kThreads)
+wkv6_bwd_dk_domega_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
+                          const IO* __restrict__ v, const IO* __restrict__ omega,
+                          const float* __restrict__ u, const IO* __restrict__ dy,
+                          const float* __restrict__ dS_T, IO* __restrict__ dk,
+                          IO* __restrict__ domega, typename Prec<IO>::Acc* __restrict__ P,
+                          typename Prec<IO>::Acc* __restrict__ E, float* dS_0, int T, int H) {
+    __shared__ __align__(16) typename SweepSmem<IO>::Row s;
+    row_sweep<IO, true>(s, r, k, dy, v, omega, u, dS_T, dk, P, domega, E, nullptr, nullptr, dS_0,
+                        T, H);
+}
+
+// du[h][i] = sum_b du_part[b][h][i]  (fixed order: deterministic)
+__global__ void wkv6_bwd_du_kernel(const float* __restrict__ du_part, float* __restrict__ du,
+                                   int B, int H) {
+    const int h = blockIdx.x, i = threadIdx.x;
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b) acc += du_part[((size_t)b * H + h) * kHeadSize + i];
+    du[(size_t)h * kHeadSize + i] = acc;
+}
+
+template <typename IO>
+cudaError_t launch_typed(const void* r, const void* k, const void* v, const void* omega,
+                         const float* u, const float* state_in, const void* dy,
+                         const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
+                         float* du, float* dstate_in, void* P_, void* E_, float* du_part, int B,
+                         int T, int H, cudaStream_t st) {
+    using Acc = typename Prec<IO>::Acc;
+    const IO *r_ = (const IO*)r, *k_ = (const IO*)k, *v_ = (const IO*)v, *o_ = (const IO*)omega,
+             *dy_ = (const IO*)dy;
+    Acc *P = static_cast<Acc*>(P_), *E = static_cast<Acc*>(E_);
+    const unsigned bh = (unsigned)(B * H);
+    wkv6_bwd_dr_dv_kernel<IO><<<dim3(bh, kHeadSize / kHalf, 2), kThreads, 0, st>>>(
+        r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    wkv6_bwd_dk_domega_kernel<IO><<<dim3(bh, kHeadSize / kHalf), kThreads, 0, st>>>(
+        r_, k_, v_, o_, u, dy_, dstate_out, (IO*)dk, (IO*)domega, P, E, dstate_in, T, H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    wkv6_bwd_du_kernel<<<H, kHeadSize, 0, st>>>(du_part, du, B, H);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const void* r, const void* k, const void* v, const void* omega,
+                            const float* u, const float* state_in, const void* dy,
+                            const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
+                            float* du, float* dstate_in, void* P, void* E, float* du_part,
+                            int B, int T, int H, bool bf16, cudaStream_t st) {
+    if (bf16)
+        return launch_typed<__nv_bfloat16>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
+                                           dv, domega, du, dstate_in, P, E, du_part, B, T, H, st);
+    return launch_typed<float>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv, domega,
+                               du, dstate_in, P, E, du_part, B, T, H, st);
+}
+
+}  // namespace goldwkv

@@ -1,0 +1,18 @@
+// Launcher of the WKV6 backward kernels (csrc/backward.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace goldwkv {
+
+// Backward of the base recurrence: three token-by-token sweeps and a reduction of du over
+// the batch.  Scratch the caller provides: P [B][T][H][64] and E [B*H][64] of the scans
+// accumulation type (fp64 for fp32 I/O, fp32 for bf16 I/O), du_part [B*H][64] fp32.
+// dstate_out / state_in may be null (zero); dstate_in may be null (not written).
+cudaError_t launch_backward(const void* r, const void* k, const void* v, const void* omega,
+                            const float* u, const float* state_in, const void* dy,
+                            const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
+                            float* du, float* dstate_in, void* P, void* E, float* du_part,
+                            int B, int T, int H, bool bf16, cudaStream_t st);
+
+}  // namespace goldwkv
