@@ -86,6 +86,73 @@ __device__ __forceinline__ size_t tok_index(size_t xbase, int t, size_t tstride,
     return xbase + (size_t)t * tstride + c;
 }
 
+// Tiles move as 16-byte chunks: a thread loads its chunks of the NEXT tile into registers
+// before computing the current one, and converts them into shared memory afterwards, so the
+// global-memory latency hides behind a tile of work.  A tile of W channels x kTile tokens of
+// type X has kTile * W * sizeof(X) / 16 chunks; chunk c covers elements
+// [c * n, c * n + n) of the tile in token-major order, n = 16 / sizeof(X).  Every row of W
+// channels is a whole number of chunks and starts 16-byte aligned in global memory.
+template <typename X>
+__device__ __forceinline__ uint4 load_chunk(const X* __restrict__ src, size_t xbase, size_t tstride,
+                                            int t0, int nt, int colbase, int W, int c) {
+    constexpr int n = 16 / sizeof(X);
+    const int e = c * n, tt = e / W, col = e - (e / W) * W;
+    if (tt >= nt) return make_uint4(0u, 0u, 0u, 0u);
+    return __ldg(reinterpret_cast<const uint4*>(src + tok_index(xbase, t0 + tt, tstride,
+                                                                  colbase + col)));
+}
+
+// The elements of a chunk as fp32 (bf16 / fp32 chunks) or as they are (fp64 chunks).
+__device__ __forceinline__ void unpack(uint4 c, float (&f)[8]) {   // 8 bf16
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        f[2 * e] = __uint_as_float(w[e] << 16);
+        f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void unpack(uint4 c, float (&f)[4]) {   // 4 fp32
+    f[0] = __uint_as_float(c.x);
+    f[1] = __uint_as_float(c.y);
+    f[2] = __uint_as_float(c.z);
+    f[3] = __uint_as_float(c.w);
+}
+__device__ __forceinline__ void unpack(uint4 c, double (&f)[2]) {  // 2 fp64
+    f[0] = __hiloint2double((int)c.y, (int)c.x);
+    f[1] = __hiloint2double((int)c.w, (int)c.z);
+}
+
+template <typename X> struct ChunkOf;
+template <> struct ChunkOf<__nv_bfloat16> { using Elem = float; static constexpr int n = 8; };
+template <> struct ChunkOf<float> { using Elem = float; static constexpr int n = 4; };
+template <> struct ChunkOf<double> { using Elem = double; static constexpr int n = 2; };
+
+// n fp32 values to dst (16-byte aligned) as 16-byte stores.
+template <int n>
+__device__ __forceinline__ void store_f32(float* dst, const float (&f)[n]) {
+    static_assert(n % 4 == 0, "whole float4s");
+#pragma unroll
+    for (int j = 0; j < n; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
+}
+
+// Store chunk c of a token-major tile into dst (the tile flattened, same element order).
+template <typename X>
+__device__ __forceinline__ void put_chunk(uint4 raw, float* dst, int c) {
+    float f[ChunkOf<X>::n];
+    unpack(raw, f);
+    store_f32(dst + c * ChunkOf<X>::n, f);
+}
+__device__ __forceinline__ void put_chunk_f64(uint4 raw, double* dst, int c) {
+    *reinterpret_cast<uint4*>(dst + 2 * c) = raw;   // 2 fp64 values, bit for bit
+}
+__device__ __forceinline__ void put_chunk_acc(uint4 raw, float* dst, int c) {
+    put_chunk<float>(raw, dst, c);
+}
+__device__ __forceinline__ void put_chunk_acc(uint4 raw, double* dst, int c) {
+    put_chunk_f64(raw, dst, c);
+}
+
 // kRev == false: the dr sweep (a = k, m = r, b = v, q = dy, X0 = state_in), forward in time.
 // kRev == true : the dk sweep (a = r, m = k, b = dy, q = v, X0 = dS_T), reverse in time, with
 //                the decay-gradient scan (reads P and E written by the dr sweep).
@@ -113,10 +180,15 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
 
     if (tid < kHalf) s.u[tid] = u[h * D + rowbase + tid];
 
-    const size_t sbase = (size_t)bh * D * D + (size_t)i * D + 16 * qq;
+    // X[4*m4 + j] is entry (i, col(m4, j)): the four threads of a row interleave in blocks
+    // of 4 columns, so their 16-byte shared-memory reads fall in distinct banks
+    const size_t sbase = (size_t)bh * D * D + (size_t)i * D + 4 * qq;
+    auto col = [](int m4, int j) { return 16 * m4 + j; };   // + 4*qq, folded into sbase
     Acc X[16];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) X[m] = x0 ? (Acc)x0[sbase + m] : Acc(0);
+    for (int m4 = 0; m4 < 4; ++m4)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) X[4 * m4 + j] = x0 ? (Acc)x0[sbase + col(m4, j)] : Acc(0);
 
     const size_t tstride = (size_t)H * D;
     const size_t xbase = ((size_t)b * T * H + h) * D;
@@ -124,40 +196,68 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
     Acc du_acc = 0, accP = 0, accQ = 0;
     const Acc Ei = kRev ? E[(size_t)bh * D + i] : Acc(0);
 
+    // chunk counts per thread: [kTile][64] and [kTile][32] tiles of IO, [kTile][32] of Acc
+    constexpr int kFull = kTile * D * (int)sizeof(IO) / 16 / kThreads;
+    constexpr int kRows = kTile * kHalf * (int)sizeof(IO) / 16 / kThreads;
+    constexpr int kAcc = kTile * kHalf * (int)sizeof(Acc) / 16 / kThreads;
+    static_assert(kFull * kThreads * 16 == kTile * D * (int)sizeof(IO) && kRows >= 1 &&
+                      kRows * kThreads * 16 == kTile * kHalf * (int)sizeof(IO) &&
+                      kAcc * kThreads * 16 == kTile * kHalf * (int)sizeof(Acc),
+                  "tiles must split into whole chunks per thread");
+    uint4 rb[kFull], rq[kFull], ra[kRows], rm[kRows], ro[kRows], rp[kAcc];
+    auto fetch = [&](int it) {   // chunks of tile `it` (in sweep order) into registers
+        const int t0 = (kRev ? ntile - 1 - it : it) * kTile, nt = min(kTile, T - t0);
+#pragma unroll
+        for (int c = 0; c < kFull; ++c) {
+            rb[c] = load_chunk(b_src, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+            rq[c] = load_chunk(q_src, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+        }
+#pragma unroll
+        for (int c = 0; c < kRows; ++c) {
+            ra[c] = load_chunk(a_src, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
+            rm[c] = load_chunk(m_src, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
+            ro[c] = load_chunk(omega, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
+        }
+        if (kRev) {
+#pragma unroll
+            for (int c = 0; c < kAcc; ++c)
+                rp[c] = load_chunk(P, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
+        }
+    };
+    if (ntile > 0) fetch(0);
+
     for (int it = 0; it < ntile; ++it) {
         const int tile = kRev ? ntile - 1 - it : it;
         const int t0 = tile * kTile;
         const int nt = min(kTile, T - t0);
         __syncthreads();   // previous tile consumed and flushed
-        for (int idx = tid; idx < kTile * D; idx += kThreads) {
-            const int tt = idx / D, c = idx - (idx / D) * D;
-            float bv = 0.f, qv = 0.f;
-            if (tt < nt) {
-                const size_t g = tok_index(xbase, t0 + tt, tstride, c);
-                bv = to_f32(b_src[g]);
-                qv = to_f32(q_src[g]);
-            }
-            s.b[tt][c] = bv;
-            s.q[tt][c] = qv;
+#pragma unroll
+        for (int c = 0; c < kFull; ++c) {
+            put_chunk<IO>(rb[c], &s.b[0][0], tid + c * kThreads);
+            put_chunk<IO>(rq[c], &s.q[0][0], tid + c * kThreads);
         }
-        for (int idx = tid; idx < kTile * kHalf; idx += kThreads) {
-            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
-            float av = 0.f, mv = 0.f, ne = 0.f;
-            Acc pv = 0;
-            if (tt < nt) {
-                const size_t g = tok_index(xbase, t0 + tt, tstride, rowbase + c);
-                av = to_f32(a_src[g]);
-                mv = to_f32(m_src[g]);
-                ne = -expf(to_f32(omega[g]));
-                if (kRev) pv = P[g];
+#pragma unroll
+        for (int c = 0; c < kRows; ++c) {
+            constexpr int n = ChunkOf<IO>::n;
+            put_chunk<IO>(ra[c], &s.a[0][0], tid + c * kThreads);
+            put_chunk<IO>(rm[c], &s.m[0][0], tid + c * kThreads);
+            float om[n], ne[n], w[n];
+            unpack(ro[c], om);
+#pragma unroll
+            for (int j = 0; j < n; ++j) {   // (padding tokens past T are never read)
+                ne[j] = -expf(om[j]);
+                w[j] = expf(ne[j]);
             }
-            s.a[tt][c] = av;
-            s.m[tt][c] = mv;
-            s.ne[tt][c] = ne;
-            s.w[tt][c] = expf(ne);
-            s.p[tt][c] = pv;
+            const int e = (tid + c * kThreads) * n;
+            store_f32(&s.ne[0][0] + e, ne);
+            store_f32(&s.w[0][0] + e, w);
+        }
+        if (kRev) {
+#pragma unroll
+            for (int c = 0; c < kAcc; ++c) put_chunk_acc(rp[c], &s.p[0][0], tid + c * kThreads);
         }
         __syncthreads();
+        if (it + 1 < ntile) fetch(it + 1);   // in flight while this tile is computed
         for (int tt = warp * (kTile / 4); tt < (warp + 1) * (kTile / 4); ++tt) {
             const float p = warp_sum(s.b[tt][lane] * s.q[tt][lane] +
                                      s.b[tt][lane + 32] * s.q[tt][lane + 32]);
@@ -165,15 +265,32 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
         }
         __syncthreads();
 
+        // operands of token `st` (in sweep order) from shared memory; the next token's are
+        // read while the current one is computed
+        float4 qc[4], bc[4];
+        float ac = 0.f, wc = 0.f;
+        auto operands = [&](int st, float4 (&qv)[4], float4 (&bv)[4], float& a, float& w) {
+            const int tt = kRev ? nt - 1 - st : st;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                qv[m4] = *reinterpret_cast<const float4*>(&s.q[tt][16 * m4 + 4 * qq]);
+                bv[m4] = *reinterpret_cast<const float4*>(&s.b[tt][16 * m4 + 4 * qq]);
+            }
+            a = s.a[tt][rl];
+            w = s.w[tt][rl];
+        };
+        if (nt > 0) operands(0, qc, bc, ac, wc);
+#pragma unroll 2
         for (int st = 0; st < nt; ++st) {
             const int tt = kRev ? nt - 1 - st : st;
-            const float4* q4 = reinterpret_cast<const float4*>(&s.q[tt][16 * qq]);
-            const float4* b4 = reinterpret_cast<const float4*>(&s.b[tt][16 * qq]);
-            const Acc ai = s.a[tt][rl], wi = s.w[tt][rl];
+            float4 qn[4], bn[4];
+            float an, wn;
+            operands(min(st + 1, nt - 1), qn, bn, an, wn);
+            const Acc ai = ac, wi = wc;
             Acc acc0 = 0, acc1 = 0;
 #pragma unroll
             for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 qv = q4[m4], bv = b4[m4];
+                const float4 qv = qc[m4], bv = bc[m4];
                 Acc* x = &X[4 * m4];
                 acc0 += x[0] * (Acc)qv.x;
                 acc1 += x[1] * (Acc)qv.y;
@@ -200,6 +317,13 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
                     accP += s.p[tt][rl];
                 }
             }
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                qc[m4] = qn[m4];
+                bc[m4] = bn[m4];
+            }
+            ac = an;
+            wc = wn;
         }
         __syncthreads();
         for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
@@ -215,7 +339,9 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
         Acc e = 0;
         if (dS_T) {
 #pragma unroll
-            for (int m = 0; m < 16; ++m) e += X[m] * (Acc)dS_T[sbase + m];
+            for (int m4 = 0; m4 < 4; ++m4)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) e += X[4 * m4 + j] * (Acc)dS_T[sbase + col(m4, j)];
         }
         e += __shfl_xor_sync(0xffffffffu, e, 1);
         e += __shfl_xor_sync(0xffffffffu, e, 2);
@@ -225,7 +351,9 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
         }
     } else if (x_final) {
 #pragma unroll
-        for (int m = 0; m < 16; ++m) x_final[sbase + m] = (float)X[m];
+        for (int m4 = 0; m4 < 4; ++m4)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x_final[sbase + col(m4, j)] = (float)X[4 * m4 + j];
     }
 }
 
@@ -247,36 +375,57 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
 
     if (tid < D) s.u[tid] = u[h * D + tid];
 
+    // G[4*m4 + e] is entry (row 16*m4 + 4*qq + e, column j): rows interleave in blocks of 4
+    // across the four threads of a column (bank-conflict-free 16-byte reads)
     const size_t sbase = (size_t)bh * D * D;
     float G[16];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) G[m] = dS_T ? dS_T[sbase + (size_t)(16 * qq + m) * D + j] : 0.f;
+    for (int m4 = 0; m4 < 4; ++m4)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            G[4 * m4 + e] = dS_T ? dS_T[sbase + (size_t)(16 * m4 + 4 * qq + e) * D + j] : 0.f;
 
     const size_t tstride = (size_t)H * D;
     const size_t xbase = ((size_t)b * T * H + h) * D;
     const int ntile = (T + kTile - 1) / kTile;
+    constexpr int kFull = kTile * D * (int)sizeof(IO) / 16 / kThreads;
+    constexpr int kCols = kTile * kHalf * (int)sizeof(IO) / 16 / kThreads;
+    static_assert(kFull * kThreads * 16 == kTile * D * (int)sizeof(IO) && kCols >= 1 &&
+                      kCols * kThreads * 16 == kTile * kHalf * (int)sizeof(IO),
+                  "tiles must split into whole chunks per thread");
+    uint4 rr[kFull], rk[kFull], ro[kFull], rd[kCols];
+    auto fetch = [&](int it) {   // chunks of tile `it` (reverse order) into registers
+        const int t0 = (ntile - 1 - it) * kTile, nt = min(kTile, T - t0);
+#pragma unroll
+        for (int c = 0; c < kFull; ++c) {
+            rr[c] = load_chunk(r, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+            rk[c] = load_chunk(k, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+            ro[c] = load_chunk(omega, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+        }
+#pragma unroll
+        for (int c = 0; c < kCols; ++c)
+            rd[c] = load_chunk(dy, xbase, tstride, t0, nt, colbase, kHalf, tid + c * kThreads);
+    };
+    if (ntile > 0) fetch(0);
     for (int it = 0; it < ntile; ++it) {
         const int t0 = (ntile - 1 - it) * kTile;
         const int nt = min(kTile, T - t0);
         __syncthreads();
-        for (int idx = tid; idx < kTile * D; idx += kThreads) {
-            const int tt = idx / D, c = idx - (idx / D) * D;
-            float rv = 0.f, kv = 0.f, wv = 1.f;
-            if (tt < nt) {
-                const size_t g = tok_index(xbase, t0 + tt, tstride, c);
-                rv = to_f32(r[g]);
-                kv = to_f32(k[g]);
-                wv = decay_from_logit(to_f32(omega[g]));
-            }
-            s.r[tt][c] = rv;
-            s.k[tt][c] = kv;
-            s.w[tt][c] = wv;
+#pragma unroll
+        for (int c = 0; c < kFull; ++c) {
+            constexpr int n = ChunkOf<IO>::n;
+            put_chunk<IO>(rr[c], &s.r[0][0], tid + c * kThreads);
+            put_chunk<IO>(rk[c], &s.k[0][0], tid + c * kThreads);
+            float om[n], w[n];
+            unpack(ro[c], om);
+#pragma unroll
+            for (int j = 0; j < n; ++j) w[j] = decay_from_logit(om[j]);
+            store_f32(&s.w[0][0] + (tid + c * kThreads) * n, w);
         }
-        for (int idx = tid; idx < kTile * kHalf; idx += kThreads) {
-            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
-            s.dy[tt][c] = tt < nt ? to_f32(dy[tok_index(xbase, t0 + tt, tstride, colbase + c)]) : 0.f;
-        }
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) put_chunk<IO>(rd[c], &s.dy[0][0], tid + c * kThreads);
         __syncthreads();
+        if (it + 1 < ntile) fetch(it + 1);
         for (int tt = warp * (kTile / 4); tt < (warp + 1) * (kTile / 4); ++tt) {
             const float p = warp_sum(s.r[tt][lane] * s.u[lane] * s.k[tt][lane] +
                                      s.r[tt][lane + 32] * s.u[lane + 32] * s.k[tt][lane + 32]);
@@ -284,16 +433,30 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
         }
         __syncthreads();
 
+        float4 kc[4], rc[4], wc[4];
+        float dc = 0.f;
+        auto operands = [&](int st, float4 (&kv)[4], float4 (&rv)[4], float4 (&wv)[4], float& d) {
+            const int tt = nt - 1 - st;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                kv[m4] = *reinterpret_cast<const float4*>(&s.k[tt][16 * m4 + 4 * qq]);
+                rv[m4] = *reinterpret_cast<const float4*>(&s.r[tt][16 * m4 + 4 * qq]);
+                wv[m4] = *reinterpret_cast<const float4*>(&s.w[tt][16 * m4 + 4 * qq]);
+            }
+            d = s.dy[tt][jl];
+        };
+        if (nt > 0) operands(0, kc, rc, wc, dc);
+#pragma unroll 2
         for (int st = 0; st < nt; ++st) {
             const int tt = nt - 1 - st;
-            const float4* k4 = reinterpret_cast<const float4*>(&s.k[tt][16 * qq]);
-            const float4* r4 = reinterpret_cast<const float4*>(&s.r[tt][16 * qq]);
-            const float4* w4 = reinterpret_cast<const float4*>(&s.w[tt][16 * qq]);
-            const float dyj = s.dy[tt][jl];
+            float4 kn[4], rn[4], wn[4];
+            float dn;
+            operands(min(st + 1, nt - 1), kn, rn, wn, dn);
+            const float dyj = dc;
             float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
             for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 kk = k4[m4], rr = r4[m4], ww = w4[m4];
+                const float4 kk = kc[m4], rr = rc[m4], ww = wc[m4];
                 float* g = &G[4 * m4];
                 acc0 = fmaf(kk.x, g[0], acc0);
                 acc1 = fmaf(kk.y, g[1], acc1);
@@ -308,6 +471,13 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             if (qq == 0) s.o[tt][jl] = fmaf(s.rku[tt], dyj, acc);
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                kc[m4] = kn[m4];
+                rc[m4] = rn[m4];
+                wc[m4] = wn[m4];
+            }
+            dc = dn;
         }
         __syncthreads();
         for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
@@ -326,7 +496,7 @@ struct SweepSmem {
 
 // blockIdx.z == 0: dr sweep; blockIdx.z == 1: dv sweep.
 template <typename IO>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)   // 4 CTAs (16 warps) per SM
 wkv6_bwd_dr_dv_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                       const IO* __restrict__ v, const IO* __restrict__ omega,
                       const float* __restrict__ u, const float* state_in, const IO* __restrict__ dy,
@@ -344,7 +514,7 @@ wkv6_bwd_dr_dv_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)   // 4 CTAs (16 warps) per SM
 wkv6_bwd_dk_domega_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                           const IO* __restrict__ v, const IO* __restrict__ omega,
                           const float* __restrict__ u, const IO* __restrict__ dy,
