@@ -9,8 +9,10 @@ the GoldFinch review page, section 3.4 "Finch-C2 Time Mixing": decay
 ``w_t = exp(-exp(d_t))`` ("Data-dependent decay"), the state sum
 ``wkv_t = sum_{i<t} diag(prod_{j=i+1}^{t-1} w_j) k_i^T v_i`` ("Recurrent state update and
 output"), readout ``r_t . wkv_t`` plus the base-Finch static bonus ``r_t . diag(u) k_t^T v_t``,
-and LayerNorm over the concatenated heads.  This module only builds/loads the shared
-object and marshals numpy arrays.
+and LayerNorm over the concatenated heads; base Finch's per-head GroupNorm and gate; the
+backward pass of the base recurrence; GOLD key compression and TokenCat decompression
+(section 3.4 "GOLD Key Compression and TokenCat Decompression").  This module only
+builds/loads the shared object and marshals numpy arrays.
 
 Pins: every entry point is checked by ``tests/test_oracle_pins.py`` against brute-force
 sums, closed forms and invariants that do not call this code (see that file's header).
@@ -80,6 +82,11 @@ class Oracle:
         lib.wkv6_oracle_backward.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                              dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
         lib.wkv6_oracle_backward.restype = ctypes.c_int
+        lib.gold_oracle_compress.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp, dp]
+        lib.gold_oracle_compress.restype = ctypes.c_int
+        lib.gold_oracle_decompress.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp, dp,
+                                               dp, ctypes.c_double, dp]
+        lib.gold_oracle_decompress.restype = ctypes.c_int
         self._lib = lib
 
     @staticmethod
@@ -224,6 +231,34 @@ class Oracle:
         yl = self.layernorm(y.reshape(B, T, H * D), gamma, beta, eps).reshape(B, T, H, D)
         return yl, s, y
 
+    def gold_compress(self, x, w_kd):
+        """GOLD compression c = x W_KD; x [..., D], w_kd [Dc, D] (rows of the map). fp64."""
+        x, w = self._f64(x), self._f64(w_kd)
+        D, Dc = x.shape[-1], w.shape[0]
+        assert w.shape == (Dc, D)
+        xs = np.ascontiguousarray(x.reshape(-1, D))
+        c = np.empty((xs.shape[0], Dc))
+        rc = self._lib.gold_oracle_compress(xs.shape[0], D, Dc, self._ptr(xs), self._ptr(w),
+                                            self._ptr(c))
+        if rc != 0:
+            raise RuntimeError(f"oracle gold_compress failed rc={rc}")
+        return c.reshape(*x.shape[:-1], Dc)
+
+    def gold_decompress(self, x0, c, w_ku, gamma=None, eps: float = 1e-6):
+        """TokenCat decompression RMSNorm(concat(x0, c) W_KU); x0 [..., D], c [..., Dc], w_ku
+        [D, D + Dc] (rows of the map), gamma [D] or None. fp64."""
+        x0, c, w, g = self._f64(x0), self._f64(c), self._f64(w_ku), self._f64(gamma)
+        D, Dc = x0.shape[-1], c.shape[-1]
+        assert w.shape == (D, D + Dc) and x0.shape[:-1] == c.shape[:-1]
+        xs = np.ascontiguousarray(x0.reshape(-1, D))
+        cs = np.ascontiguousarray(c.reshape(-1, Dc))
+        kd = np.empty_like(xs)
+        rc = self._lib.gold_oracle_decompress(xs.shape[0], D, Dc, self._ptr(xs), self._ptr(cs),
+                                              self._ptr(w), self._ptr(g), float(eps), self._ptr(kd))
+        if rc != 0:
+            raise RuntimeError(f"oracle gold_decompress failed rc={rc}")
+        return kd.reshape(x0.shape)
+
 
 _default: Oracle | None = None
 
@@ -234,3 +269,4 @@ def get() -> Oracle:
     if _default is None:
         _default = Oracle()
     return _default
+

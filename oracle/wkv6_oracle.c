@@ -15,6 +15,12 @@
  *   - Finch-C2's exact form (wkv6c2_*): key k_t (1 - w_t), second value u'_t added to the
  *     readout instead of the static bonus              ("Key computation with normalization
  *                                                        property", "the new second value")
+ *   - base Finch's per-head GroupNorm and output gate, which Finch-C2 removes
+ *   - the backward pass of the base recurrence (the chain rule through the recursion; the
+ *     page's "Training and Inference Procedures" trains all tokens in parallel)
+ *   - GOLD key compression c_t = x_t W_KD and TokenCat decompression
+ *     RMSNorm(concat(x0_t, c_t) W_KU)            ("GOLD Key Compression and TokenCat
+ *                                                  Decompression")
  * Written in recursive form: with S_{-1} = state_in (zero if absent),
  *   y_t[j] = sum_i r_t[i] S_{t-1}[i][j] + (sum_i r_t[i] u[i] k_t[i]) v_t[j]
  *   S_t[i][j] = w_t[i] S_{t-1}[i][j] + k_t[i] v_t[j]
@@ -446,5 +452,64 @@ int wkv6_oracle_backward(int B, long T, int H, int D,
         }
     free(Sall);
     free(G);
+    return 0;
+}
+
+/* GOLD key compression (GoldFinch review page, section 3.4 "GOLD Key Compression and
+ * TokenCat Decompression", compression step): c_t = x_t W_KD, W_KD a D x Dc matrix
+ * (Dc = D/16 in the page's model).  W_KD is passed transposed, as the rows of the linear
+ * map: w_kd[j][i] = W_KD[i][j], [Dc][D].  x [N][D], c [N][Dc]. */
+int gold_oracle_compress(long N, int D, int Dc, const double *x, const double *w_kd, double *c)
+{
+    if (N < 0 || D <= 0 || Dc <= 0)
+        return -1;
+    for (long n = 0; n < N; ++n)
+        for (int j = 0; j < Dc; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < D; ++i)
+                acc += x[n * D + i] * w_kd[(long)j * D + i];
+            c[n * Dc + j] = acc;
+        }
+    return 0;
+}
+
+/* TokenCat decompression (same section): k^D_t = RMSNorm(concat(x0_t, c_t) W_KU), W_KU a
+ * (D + Dc) x D matrix passed transposed as w_ku[o][i] = W_KU[i][o], [D][D + Dc].  RMSNorm of
+ * a row z of D values: z[o] / sqrt(mean_o z[o]^2 + eps) * gamma[o] (gamma NULL = 1).
+ * x0 [N][D], c [N][Dc], kd [N][D]. */
+int gold_oracle_decompress(long N, int D, int Dc, const double *x0, const double *c,
+                           const double *w_ku, const double *gamma, double eps, double *kd)
+{
+    if (N < 0 || D <= 0 || Dc <= 0 || !(eps >= 0.0))
+        return -1;
+    const int K = D + Dc;
+    double *z = (double *)malloc(sizeof(double) * (size_t)D);
+    double *cat = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!z || !cat) {
+        free(z);
+        free(cat);
+        return -3;
+    }
+    for (long n = 0; n < N; ++n) {
+        /* the concatenation [x0_t, c_t] */
+        for (int i = 0; i < D; ++i)
+            cat[i] = x0[n * D + i];
+        for (int j = 0; j < Dc; ++j)
+            cat[D + j] = c[n * Dc + j];
+        double ms = 0.0;
+        for (int o = 0; o < D; ++o) {
+            double acc = 0.0;
+            for (int i = 0; i < K; ++i)
+                acc += cat[i] * w_ku[(long)o * K + i];
+            z[o] = acc;
+            ms += acc * acc;
+        }
+        ms /= (double)D;
+        const double inv_rms = 1.0 / sqrt(ms + eps);
+        for (int o = 0; o < D; ++o)
+            kd[n * D + o] = z[o] * inv_rms * (gamma ? gamma[o] : 1.0);
+    }
+    free(z);
+    free(cat);
     return 0;
 }

@@ -56,6 +56,16 @@ v, omega, u and the initial state):
                       (dr', dk' without their bonus parts): a relation between outputs;
 * bwd_empty         - T = 0: dS_0 = dS_T and every other gradient is zero.
 
+GOLD key compression and TokenCat decompression (section 3.4 "GOLD Key Compression and
+TokenCat Decompression"):
+
+* gold_compress_matmul  - c = x W_KD equals numpy's matrix product;
+* gold_decompress_blocks- concat(x0, c) W_KU equals x0 W_KU[:D] + c W_KU[D:] (numpy), then
+                          an RMSNorm written out in numpy;
+* gold_rmsnorm_torch    - the same through torch.nn.functional.rms_norm, with a large eps;
+* gold_scale_invariance - with eps = 0, scaling x0 and c by any a > 0 leaves the output
+                          unchanged, and every row of output / gamma has mean square 1.
+
 ``run_all(oracle)`` returns the list of failing pin names; the mutation test uses it to
 show that plausible mistakes planted in the oracle are caught.
 """
@@ -450,6 +460,41 @@ def pin_bwd_empty(o):
     return np.array_equal(dS0, dS) and not np.any(du) and dr.size == 0
 
 
+def _gold_inputs(seed, N=7, D=48, Dc=8):
+    g = _rng(seed)
+    return (g.normal(0, 1.0, (N, D)), g.normal(0, 1.0, (N, Dc)), g.normal(0, 0.2, (Dc, D)),
+            g.normal(0, 0.2, (D, D + Dc)), g.normal(1.0, 0.3, D))
+
+
+def pin_gold_compress_matmul(o):
+    x, _, w_kd, _, _ = _gold_inputs(40)
+    return _close(o.gold_compress(x, w_kd), x @ w_kd.T, rtol=1e-12)
+
+
+def pin_gold_decompress_blocks(o):
+    x0, c, _, w_ku, gam = _gold_inputs(41)
+    D = x0.shape[1]
+    z = x0 @ w_ku[:, :D].T + c @ w_ku[:, D:].T
+    want = z / np.sqrt(np.mean(z * z, axis=1, keepdims=True) + 1e-3) * gam
+    return _close(o.gold_decompress(x0, c, w_ku, gam, 1e-3), want, rtol=1e-12)
+
+
+def pin_gold_rmsnorm_torch(o):
+    x0, c, _, w_ku, gam = _gold_inputs(42)
+    x0, c = 0.3 * x0, 0.3 * c          # row mean squares near 0.2, so eps = 0.5 matters
+    z = torch.cat([torch.tensor(x0), torch.tensor(c)], dim=1) @ torch.tensor(w_ku).T
+    want = torch.nn.functional.rms_norm(z, (z.shape[1],), weight=torch.tensor(gam), eps=0.5)
+    return _close(o.gold_decompress(x0, c, w_ku, gam, 0.5), want.numpy(), rtol=1e-12)
+
+
+def pin_gold_scale_invariance(o):
+    x0, c, _, w_ku, gam = _gold_inputs(43)
+    a = o.gold_decompress(x0, c, w_ku, gam, 0.0)
+    b = o.gold_decompress(7.5 * x0, 7.5 * c, w_ku, gam, 0.0)
+    ms = np.mean((a / gam) ** 2, axis=1)
+    return _close(a, b, rtol=1e-12) and bool(np.all(np.abs(ms - 1.0) < 1e-12))
+
+
 PINS = {
     "explicit_sum": pin_explicit_sum,
     "t1_closed_form": pin_t1_closed_form,
@@ -474,6 +519,10 @@ PINS = {
     "bwd_autograd": pin_bwd_autograd,
     "bwd_decay_identity": pin_bwd_decay_identity,
     "bwd_empty": pin_bwd_empty,
+    "gold_compress_matmul": pin_gold_compress_matmul,
+    "gold_decompress_blocks": pin_gold_decompress_blocks,
+    "gold_rmsnorm_torch": pin_gold_rmsnorm_torch,
+    "gold_scale_invariance": pin_gold_scale_invariance,
 }
 
 

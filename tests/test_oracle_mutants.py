@@ -68,6 +68,15 @@ MUTANTS = {
                                   "G[i * D + j] = wi * G[i * D + j];"),
     "bwd_dv_transposed": ("g += G[i * D + j] * kt[i];", "g += G[j * D + i] * kt[i];"),
     "bwd_du_without_r": ("du_acc[i] += rt[i] * kt[i] * vdy;", "du_acc[i] += kt[i] * vdy;"),
+    # GOLD compression and TokenCat decompression
+    "gold_compress_transposed": ("acc += x[n * D + i] * w_kd[(long)j * D + i];",
+                                 "acc += x[n * D + i] * w_kd[(long)i * Dc + j];"),
+    "gold_cat_drops_c": ("cat[D + j] = c[n * Dc + j];", "cat[D + j] = 0.0;"),
+    "gold_rms_eps_outside": ("const double inv_rms = 1.0 / sqrt(ms + eps);",
+                             "const double inv_rms = 1.0 / (sqrt(ms) + eps);"),
+    "gold_rms_mean_over_cat": ("ms /= (double)D;", "ms /= (double)K;"),
+    "gold_gamma_ignored": ("kd[n * D + o] = z[o] * inv_rms * (gamma ? gamma[o] : 1.0);",
+                           "kd[n * D + o] = z[o] * inv_rms;"),
 }
 
 
