@@ -43,6 +43,7 @@ METRIC = "WKV prefill tokens/s (H=32, D=64) and decode GB/s; fraction of rooflin
 PREFILL_CFG = W.CONFIGS[1]
 DECODE_CFG = W.CONFIGS[3]
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0   # an earlier dense bf16 GEMM measurement on B200 (burst)
 
 
 def prefill_bytes(B, T, H, D=64, esz=2):
@@ -328,6 +329,63 @@ def backward_line(cfg, dev, world, steps):
     return line
 
 
+def gold_line(dev, world, steps, B=8, T=4096, D=2048, Dc=128):
+    """Device-timed GOLD compression + TokenCat decompression of every token of the 1.5B-layer
+    shape (D = H*64 = 2048, Dc = D/16): one step = gold_compress then gold_decompress."""
+    import linear_attention_rnn_finch_b200 as gw
+    N = B * T
+    g = torch.Generator(device=dev).manual_seed(1005)
+    x = torch.randn((N, D), generator=g, device=dev).to(torch.bfloat16)
+    x0 = torch.randn((N, D), generator=g, device=dev).to(torch.bfloat16)
+    w_kd = (torch.randn((Dc, D), generator=g, device=dev) / D ** 0.5).to(torch.bfloat16)
+    w_ku = (torch.randn((D, D + Dc), generator=g, device=dev) / (D + Dc) ** 0.5).to(torch.bfloat16)
+    gamma = 1.0 + 0.1 * torch.randn(D, generator=g, device=dev)
+    c = torch.empty((N, Dc), dtype=torch.bfloat16, device=dev)
+    kd = torch.empty_like(x0)
+    L = gw.load()
+    ws_c = torch.empty(L.gold_compress_workspace_bytes(N, D, Dc), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(L.gold_decompress_workspace_bytes(N, D, Dc), dtype=torch.uint8, device=dev)
+
+    def call():
+        gw.gold_compress(x, w_kd, c=c, workspace=ws_c)
+        gw.gold_decompress(x0, c, w_ku, gamma, 1e-6, kd=kd, workspace=ws_d)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    flops = 2 * N * D * Dc + 2 * N * (D + Dc) * D
+    peak = bf16_peak()
+    line = {"workload": "gold_compress_decompress_1p5b", "N_tokens": N, "D": D, "Dc": Dc,
+            "io": "bf16", "steps": steps, "ms_per_call": ms,
+            "tokens_per_s": world * N / (ms / 1e3),
+            "roofline": {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": flops / (ms / 1e3) / 1e12 / peak,
+                         "peak_source": "measured bf16_tflops (cuBLAS burst)",
+                         "algorithmic_flops_per_call": flops},
+            "gpu_launches": steps,
+            "note": "the three GEMMs run in cuBLASLt (library kernels); rmsnorm_rows_kernel "
+                    "is the one kernel of ours per call"}
+    del x, x0, w_kd, w_ku, gamma, c, kd, ws_c, ws_d
+    torch.cuda.empty_cache()
+    return line
+
+
+def bf16_peak():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        return float(json.loads(p.read_text())["bf16_tflops"])
+    return FALLBACK_BF16_TFLOPS
+
+
 # ------------------------------------------------------------------------------ oracle timing
 def oracle_sample(cfg, b_rows: int, t_tokens: int, seed_offset: int = 0):
     """Inputs of the oracle's bounded sample: b_rows batch rows x t_tokens tokens of cfg,
@@ -500,6 +558,7 @@ def run_ours(args, world, rank, local):
                                 other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
                                               gn=True)]
         out["backward"] = backward_line(W.CONFIGS[1], dev, world, steps=5)
+        out["gold"] = gold_line(dev, world, steps=10)
 
     # end to end through the public API with host buffers: every step copies its inputs in
     # from pinned host memory and reads y and the final state back.  Steps are pipelined over

@@ -241,6 +241,32 @@ wkv_status wkv6_backward(const void *r, const void *k, const void *v, const void
                          float *du, float *dstate_in, int B, int T, int H, int D, wkv_dtype io,
                          void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * GOLD key compression and TokenCat decompression (GoldFinch review page, section 3.4
+ * "GOLD Key Compression and TokenCat Decompression"): the output x_t of the last Finch-C2
+ * layer is compressed by one global matrix W_KD (D x Dc, Dc = D/16 in the page's model)
+ * into the cache entry c_t = x_t W_KD; a GOLD layer rebuilds the proto-key
+ *     k^D_t = RMSNorm(concat(x0_t, c_t) W_KU),   W_KU (D + Dc) x D,
+ * x0_t the token's input embedding, RMSNorm(z) = z / sqrt(mean(z^2) + eps) * gamma.
+ * All tensors bf16 row-major except gamma (fp32); the weights are passed as the rows of
+ * each linear map (the layout of a linear layer's weight, [out][in]):
+ *   x, x0 [N][D];  c [N][Dc];  kd [N][D];  w_kd [Dc][D] (w_kd[j][i] = W_KD[i][j]);
+ *   w_ku [D][D + Dc] (w_ku[o][i] = W_KU[i][o]);  gamma [D] fp32 or NULL (= 1).
+ * The products run on the tensor cores through cuBLASLt with fp32 accumulation (c is
+ * rounded to bf16 once); the concatenation is never formed (W_KU splits into its x0 and c
+ * blocks).  D and Dc must be multiples of 8 (else WKV_ERR_UNSUPPORTED), N <= 2^31 - 1.
+ * Outputs may not overlap inputs or the workspace.  Workspace: at least
+ * gold_*_workspace_bytes(...) bytes, any contents; for decompression it holds the fp32
+ * product before RMSNorm.  eps must be > 0.
+ */
+size_t gold_compress_workspace_bytes(long N, int D, int Dc);
+wkv_status gold_compress(const void *x, const void *w_kd, void *c, long N, int D, int Dc,
+                         void *workspace, size_t workspace_bytes, void *stream);
+size_t gold_decompress_workspace_bytes(long N, int D, int Dc);
+wkv_status gold_decompress(const void *x0, const void *c, const void *w_ku, const float *gamma,
+                           float eps, void *kd, long N, int D, int Dc, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
 /* Size of the scratch array built into the library for wkv6_prefill_static, per device. */
 #define WKV6_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 

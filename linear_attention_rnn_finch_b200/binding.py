@@ -75,6 +75,14 @@ def load(path: Path | str | None = None):
     L.wkv6_backward_workspace_bytes.restype = sz
     L.wkv6_backward.argtypes = [vp] * 14 + [i, i, i, i, i, vp, sz, vp]
     L.wkv6_backward.restype = i
+    L.gold_compress_workspace_bytes.argtypes = [ctypes.c_long, i, i]
+    L.gold_compress_workspace_bytes.restype = sz
+    L.gold_decompress_workspace_bytes.argtypes = [ctypes.c_long, i, i]
+    L.gold_decompress_workspace_bytes.restype = sz
+    L.gold_compress.argtypes = [vp, vp, vp, ctypes.c_long, i, i, vp, sz, vp]
+    L.gold_compress.restype = i
+    L.gold_decompress.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp, ctypes.c_long, i, i, vp, sz, vp]
+    L.gold_decompress.restype = i
     L.wkv6_workspace_status.argtypes = [vp, vp]
     L.wkv6_workspace_status.restype = i
     L.wkv6_status_string.argtypes = [i]
@@ -451,3 +459,57 @@ def wkv6_backward(r, k, v, omega, u, state_in, dy, dstate_out=None, *, want_dsta
 
 def backward_workspace_bytes(B, T, H, D, io_dtype) -> int:
     return int(load().wkv6_backward_workspace_bytes(B, T, H, D, _io(io_dtype)))
+
+
+def gold_compress(x, w_kd, *, c=None, workspace=None, stream=None):
+    """GOLD compression c = x W_KD (include/goldwkv.h): x [..., D] bf16, w_kd [Dc, D] bf16
+    (the rows of the map).  Returns c [..., Dc] bf16."""
+    L = load()
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    D, Dc = x.shape[-1], w_kd.shape[0]
+    N = x.numel() // D if D else 0
+    _check("x", x, dev, torch.bfloat16)
+    _check("w_kd", w_kd, dev, torch.bfloat16, (Dc, D))
+    if c is None:
+        c = torch.empty((*x.shape[:-1], Dc), dtype=torch.bfloat16, device=dev)
+    _check("c", c, dev, torch.bfloat16, (*x.shape[:-1], Dc))
+    need = int(L.gold_compress_workspace_bytes(N, D, Dc))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.gold_compress(_ptr(x), _ptr(w_kd), _ptr(c), N, D, Dc, _ptr(workspace), ws_bytes,
+                             _stream_ptr(dev, stream))
+    _raise("gold_compress", st)
+    return c
+
+
+def gold_decompress(x0, c, w_ku, gamma=None, eps=1e-6, *, kd=None, workspace=None, stream=None):
+    """TokenCat decompression RMSNorm(concat(x0, c) W_KU) (include/goldwkv.h): x0 [..., D]
+    and c [..., Dc] bf16, w_ku [D, D + Dc] bf16 (the rows of the map), gamma [D] fp32 or
+    None.  Returns kd [..., D] bf16."""
+    L = load()
+    dev = x0.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    D, Dc = x0.shape[-1], c.shape[-1]
+    N = x0.numel() // D if D else 0
+    _check("x0", x0, dev, torch.bfloat16)
+    _check("c", c, dev, torch.bfloat16, (*x0.shape[:-1], Dc))
+    _check("w_ku", w_ku, dev, torch.bfloat16, (D, D + Dc))
+    if gamma is not None:
+        _check("gamma", gamma, dev, torch.float32, (D,))
+    if kd is None:
+        kd = torch.empty_like(x0)
+    _check("kd", kd, dev, torch.bfloat16, tuple(x0.shape))
+    need = int(L.gold_decompress_workspace_bytes(N, D, Dc))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.gold_decompress(_ptr(x0), _ptr(c), _ptr(w_ku), _ptr(gamma), float(eps), _ptr(kd),
+                               N, D, Dc, _ptr(workspace), ws_bytes, _stream_ptr(dev, stream))
+    _raise("gold_decompress", st)
+    return kd

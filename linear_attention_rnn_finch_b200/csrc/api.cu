@@ -8,6 +8,7 @@
 #include "goldwkv.h"
 #include "internal.h"
 #include "backward.h"
+#include "gold.h"
 
 namespace {
 
@@ -564,6 +565,89 @@ wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void
     return from_cuda(goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr,
                                               dk, dv, domega, du, dstate_in, P, E, du_part, B,
                                               T, H, io == WKV_BF16, st));
+}
+
+
+}  // extern "C"
+
+// ---- GOLD key compression and TokenCat decompression (bf16)
+
+namespace {
+
+constexpr size_t kLtWorkspace = (size_t)32 << 20;   // cuBLASLt workspace per call
+
+// Sizes the GOLD entry points take: 16-byte rows of bf16 (D, Dc multiples of 8), N within
+// the GEMMs' int range.
+wkv_status check_gold_sizes(long N, int D, int Dc) {
+    if (N < 0 || D <= 0 || Dc <= 0) return WKV_ERR_INVALID_ARG;
+    if (D % 8 != 0 || Dc % 8 != 0 || N > 0x7fffffffL) return WKV_ERR_UNSUPPORTED;
+    return WKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gold_compress_workspace_bytes(long N, int D, int Dc) {
+    if (check_gold_sizes(N, D, Dc) != WKV_OK || N == 0) return 0;
+    return kLtWorkspace;
+}
+
+size_t gold_decompress_workspace_bytes(long N, int D, int Dc) {
+    if (check_gold_sizes(N, D, Dc) != WKV_OK || N == 0) return 0;
+    return round256((size_t)N * D * sizeof(float)) + kLtWorkspace;
+}
+
+wkv_status gold_compress(const void* x, const void* w_kd, void* c, long N, int D, int Dc,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    wkv_status s = check_gold_sizes(N, D, Dc);
+    if (s != WKV_OK) return s;
+    if (N == 0) return WKV_OK;
+    const size_t xb = (size_t)N * D * 2, wb = (size_t)Dc * D * 2, cb = (size_t)N * Dc * 2;
+    Buf bufs[] = {{x, xb, true}, {w_kd, wb, true}, {c, cb, true},
+                  {workspace, workspace_bytes, false}};
+    if ((s = check_bufs(bufs, 4)) != WKV_OK) return s;
+    const size_t need = gold_compress_workspace_bytes(N, D, Dc);
+    if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+    const Span sc = span(c, cb), sw = span(workspace, need);
+    if (overlaps(sc, span(x, xb)) || overlaps(sc, span(w_kd, wb)) || overlaps(sw, sc) ||
+        overlaps(sw, span(x, xb)) || overlaps(sw, span(w_kd, wb)))
+        return WKV_ERR_INVALID_ARG;
+    if (injected("launch")) return WKV_ERR_CUDA;
+    return goldwkv::gold_gemm_compress(x, w_kd, c, N, D, Dc, workspace, need,
+                                       reinterpret_cast<cudaStream_t>(stream))
+               ? WKV_OK
+               : WKV_ERR_CUDA;
+}
+
+wkv_status gold_decompress(const void* x0, const void* c, const void* w_ku, const float* gamma,
+                           float eps, void* kd, long N, int D, int Dc, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    wkv_status s = check_gold_sizes(N, D, Dc);
+    if (s != WKV_OK) return s;
+    if (!(eps > 0.f) || eps > 1e30f) return WKV_ERR_INVALID_ARG;
+    if (N == 0) return WKV_OK;
+    const size_t xb = (size_t)N * D * 2, cb = (size_t)N * Dc * 2;
+    const size_t wb = (size_t)D * (D + Dc) * 2, gb = (size_t)D * sizeof(float);
+    Buf bufs[] = {{x0, xb, true}, {c, cb, true}, {w_ku, wb, true}, {gamma, gb, false},
+                  {kd, xb, true}, {workspace, workspace_bytes, false}};
+    if ((s = check_bufs(bufs, 6)) != WKV_OK) return s;
+    const size_t need = gold_decompress_workspace_bytes(N, D, Dc);
+    if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+    const Span outs[] = {span(kd, xb), span(workspace, need)};
+    const Span ins[] = {span(x0, xb), span(c, cb), span(w_ku, wb), span(gamma, gamma ? gb : 0)};
+    if (overlaps(outs[0], outs[1])) return WKV_ERR_INVALID_ARG;
+    for (const Span& o : outs)
+        for (const Span& in : ins)
+            if (overlaps(o, in)) return WKV_ERR_INVALID_ARG;
+    if (injected("launch")) return WKV_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* z = reinterpret_cast<float*>(ws);
+    void* lt = ws + round256((size_t)N * D * sizeof(float));
+    if (!goldwkv::gold_gemm_decompress(x0, c, w_ku, z, N, D, Dc, lt, kLtWorkspace, st))
+        return WKV_ERR_CUDA;
+    return from_cuda(goldwkv::launch_rmsnorm_rows(z, gamma, eps, kd, N, D, st));
 }
 
 }  // extern "C"

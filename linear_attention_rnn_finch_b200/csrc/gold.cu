@@ -1,0 +1,144 @@
+// GOLD key compression and TokenCat decompression (GoldFinch review page, section 3.4 "GOLD
+// Key Compression and TokenCat Decompression"):
+//     c_t   = x_t W_KD                                   (D -> Dc = D/16)
+//     k^D_t = RMSNorm(concat(x0_t, c_t) W_KU)            (D + Dc -> D)
+// Both products are plain dense GEMMs and run through cuBLASLt on the tensor cores (bf16
+// operands, fp32 accumulation).  The concatenation is never formed: W_KU splits into the
+// block that multiplies x0 and the block that multiplies c, and the second GEMM accumulates
+// into the first one's fp32 output.  RMSNorm over the D outputs of a token is our kernel.
+//
+// Row-major [rows][cols] matrices are cuBLAS column-major [cols x rows] matrices, so with
+// the weights given as the rows of each map (w[out][in]) every product is a "TN" GEMM:
+// C^T (out x N) = W (in x out, transposed) . X^T (in x N).
+#include <cublasLt.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "gold.h"
+
+namespace goldwkv {
+
+namespace {
+
+// One cuBLASLt handle for the process, created on first use (host state only).
+cublasLtHandle_t lt_handle() {
+    static std::once_flag once;
+    static cublasLtHandle_t h = nullptr;
+    std::call_once(once, [] {
+        if (cublasLtCreate(&h) != CUBLAS_STATUS_SUCCESS) h = nullptr;
+    });
+    return h;
+}
+
+// D (m x n, ldd, type dtype) = alpha * op_T(A) . B + beta * D, A stored (k x m, lda), B
+// (k x n, ldb), both bf16; fp32 compute.
+bool gemm_tn(int m, int n, int k, const void* A, int lda, const void* B, int ldb, float beta,
+             void* Dm, cudaDataType_t dtype, int ldd, void* ws, size_t ws_bytes, cudaStream_t st) {
+    cublasLtHandle_t h = lt_handle();
+    if (h == nullptr) return false;
+    cublasLtMatmulDesc_t op = nullptr;
+    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
+    cublasLtMatmulPreference_t pref = nullptr;
+    bool ok = false;
+    do {
+        if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS)
+            break;
+        const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
+        if (cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)) !=
+                CUBLAS_STATUS_SUCCESS ||
+            cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)) !=
+                CUBLAS_STATUS_SUCCESS)
+            break;
+        if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, k, m, lda) != CUBLAS_STATUS_SUCCESS ||
+            cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, k, n, ldb) != CUBLAS_STATUS_SUCCESS ||
+            cublasLtMatrixLayoutCreate(&ld, dtype, m, n, ldd) != CUBLAS_STATUS_SUCCESS)
+            break;
+        if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
+        if (cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
+                                                 &ws_bytes, sizeof(ws_bytes)) !=
+            CUBLAS_STATUS_SUCCESS)
+            break;
+        cublasLtMatmulHeuristicResult_t res{};
+        int found = 0;
+        if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, ld, ld, pref, 1, &res, &found) !=
+                CUBLAS_STATUS_SUCCESS ||
+            found < 1)
+            break;
+        const float alpha = 1.f;
+        ok = cublasLtMatmul(h, op, &alpha, A, la, B, lb, &beta, Dm, ld, Dm, ld, &res.algo, ws,
+                            ws_bytes, st) == CUBLAS_STATUS_SUCCESS;
+    } while (false);
+    if (pref) cublasLtMatmulPreferenceDestroy(pref);
+    if (ld) cublasLtMatrixLayoutDestroy(ld);
+    if (lb) cublasLtMatrixLayoutDestroy(lb);
+    if (la) cublasLtMatrixLayoutDestroy(la);
+    if (op) cublasLtMatmulDescDestroy(op);
+    return ok;
+}
+
+constexpr int kRmsThreads = 256;
+
+// One CTA per row: sum of squares over the D fp32 values (16-byte loads), then the scale.
+__global__ void __launch_bounds__(kRmsThreads)
+rmsnorm_rows_kernel(const float* __restrict__ z, const float* __restrict__ gamma, float eps,
+                    __nv_bfloat16* __restrict__ out, int D) {
+    __shared__ float part[kRmsThreads / 32];
+    const size_t row = blockIdx.x;
+    const float4* z4 = reinterpret_cast<const float4*>(z + row * D);
+    const int n4 = D / 4;
+    float ss = 0.f;
+    for (int q = threadIdx.x; q < n4; q += kRmsThreads) {
+        const float4 a = z4[q];
+        ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, ss))));
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRmsThreads / 32; ++w) tot += part[w];
+    const float inv = rsqrtf(tot / (float)D + eps);
+    for (int q = threadIdx.x; q < n4; q += kRmsThreads) {
+        const float4 a = z4[q];
+        float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (gamma) g = reinterpret_cast<const float4*>(gamma)[q];
+        __nv_bfloat162 lo = __floats2bfloat162_rn(a.x * inv * g.x, a.y * inv * g.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(a.z * inv * g.z, a.w * inv * g.w);
+        uint2 packed;
+        packed.x = *reinterpret_cast<uint32_t*>(&lo);
+        packed.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(out + row * D)[q] = packed;
+    }
+}
+
+}  // namespace
+
+bool gold_gemm_compress(const void* x, const void* w_kd, void* c, long N, int D, int Dc,
+                        void* lt_workspace, size_t lt_bytes, cudaStream_t st) {
+    // c^T (Dc x N) = w_kd (D x Dc col-major, transposed) . x^T (D x N)
+    return gemm_tn(Dc, (int)N, D, w_kd, D, x, D, 0.f, c, CUDA_R_16BF, Dc, lt_workspace,
+                   lt_bytes, st);
+}
+
+bool gold_gemm_decompress(const void* x0, const void* c, const void* w_ku, float* z, long N,
+                          int D, int Dc, void* lt_workspace, size_t lt_bytes, cudaStream_t st) {
+    const int K = D + Dc;
+    const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(w_ku);
+    // z^T = w_ku[:, :D] . x0^T, then += w_ku[:, D:] . c^T
+    return gemm_tn(D, (int)N, D, w, K, x0, D, 0.f, z, CUDA_R_32F, D, lt_workspace, lt_bytes,
+                   st) &&
+           gemm_tn(D, (int)N, Dc, w + D, K, c, Dc, 1.f, z, CUDA_R_32F, D, lt_workspace, lt_bytes,
+                   st);
+}
+
+cudaError_t launch_rmsnorm_rows(const float* z, const float* gamma, float eps, void* out, long N,
+                                int D, cudaStream_t st) {
+    if (N <= 0) return cudaSuccess;
+    rmsnorm_rows_kernel<<<(unsigned)N, kRmsThreads, 0, st>>>(z, gamma, eps,
+                                                             static_cast<__nv_bfloat16*>(out), D);
+    return cudaGetLastError();
+}
+
+}  // namespace goldwkv

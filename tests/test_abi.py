@@ -12,7 +12,7 @@ import pytest
 from linear_attention_rnn_finch_b200 import binding, build
 
 ROOT = pathlib.Path(__file__).resolve().parents[1]
-DECL = re.compile(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(wkv6(?:c2)?_\w+)\s*\(", re.M)
+DECL = re.compile(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b((?:wkv6(?:c2)?|gold)_\w+)\s*\(", re.M)
 
 
 def declared_functions():
@@ -36,7 +36,8 @@ def test_headers_declare_entry_points():
                  "wkv6_status_string", "wkv6_abi_version", "wkv6_workspace_status",
                  "wkv6_prefill_static", "wkv6c2_prefill", "wkv6c2_decode_step",
                  "wkv6_prefill_gn", "wkv6_decode_step_gn", "wkv6_backward",
-                 "wkv6_backward_workspace_bytes"):
+                 "wkv6_backward_workspace_bytes", "gold_compress", "gold_decompress",
+                 "gold_compress_workspace_bytes", "gold_decompress_workspace_bytes"):
         assert must in names
 
 
