@@ -51,31 +51,82 @@ layernorm_rows_kernel(const float* x, const float* __restrict__ gamma,
 // Base Finch's output normalisation per head, then the output gate (GoldFinch review page,
 // section 3.4: Finch-C2 replaces this per-head GroupNorm -- and drops the gate):
 //     out = ((x - mean_h) / sqrt(var_h + eps) * gamma + beta) * gate,
-// statistics over the D = 64 channels of one head of one token.  One warp per (token, head)
-// row, two channels per lane; x may equal out (fp32): a warp reads its row before writing.
+// statistics over the D = 64 channels of one head of one token.  Eight lanes per (token,
+// head) row, eight channels per lane in 16-byte accesses, four rows per warp: short
+// per-row dependency chains, so many rows are in flight per SM.  x may equal out (fp32):
+// each lane reads its eight values before writing them.
+constexpr int kGnLanes = 8;                      // lanes per row
+constexpr int kGnRowsPerCta = kThreads / kGnLanes;
+
+__device__ __forceinline__ float gn_sum(float v) {   // over the 8 lanes of a row
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    return v;
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(w[e] << 16);
+        v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        w[e] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
 groupnorm_gate_kernel(const float* x, const float* __restrict__ gamma,
                       const float* __restrict__ beta, float eps, const IO* __restrict__ gate,
                       IO* out, long rows, int H) {
-    const long row = (long)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const int lane = threadIdx.x & 31, c = 2 * lane;
-    const size_t base = (size_t)row * 64;
-    const float2 v = *reinterpret_cast<const float2*>(x + base + c);
-    const float mean = warp_sum(v.x + v.y) * (1.f / 64.f);
-    const float d0 = v.x - mean, d1 = v.y - mean;
-    const float var = warp_sum(fmaf(d0, d0, d1 * d1)) * (1.f / 64.f);
-    const float inv = rsqrtf(var + eps);
+    // every lane of the warp stays for the shuffles; a group past the last row works on the
+    // last row again and does not store
+    const long row_id = (long)blockIdx.x * kGnRowsPerCta + (threadIdx.x / kGnLanes);
+    const bool valid = row_id < rows;
+    const long row = valid ? row_id : rows - 1;
+    const int c = 8 * (threadIdx.x % kGnLanes);
+    const size_t base = (size_t)row * 64 + c;
+    float v[8], g[8], bt[8], gt[8];
+    load8(x + base, v);
     const int hc = (int)(row % H) * 64 + c;
-    float o0 = fmaf(d0 * inv, gamma[hc], beta[hc]);
-    float o1 = fmaf(d1 * inv, gamma[hc + 1], beta[hc + 1]);
-    if (gate) {
-        o0 *= to_f32(gate[base + c]);
-        o1 *= to_f32(gate[base + c + 1]);
+    load8(gamma + hc, g);
+    load8(beta + hc, bt);
+    if (gate) load8(gate + base, gt);
+    float sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sum += v[e];
+    const float mean = gn_sum(sum) * (1.f / 64.f);
+    float sq = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        v[e] -= mean;
+        sq = fmaf(v[e], v[e], sq);
     }
-    out[base + c] = from_f32<IO>(o0);
-    out[base + c + 1] = from_f32<IO>(o1);
+    const float inv = rsqrtf(gn_sum(sq) * (1.f / 64.f) + eps);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        v[e] = fmaf(v[e] * inv, g[e], bt[e]);
+        if (gate) v[e] *= gt[e];
+    }
+    if (valid) store8(out + base, v);
 }
 
 }  // namespace
@@ -84,7 +135,7 @@ cudaError_t launch_groupnorm_gate(const float* x, const float* gamma, const floa
                                   const void* gate, void* out, long rows, int H, bool bf16,
                                   cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((rows + kThreads / 32 - 1) / (kThreads / 32));
+    const unsigned grid = (unsigned)((rows + kGnRowsPerCta - 1) / kGnRowsPerCta);
     if (bf16)
         groupnorm_gate_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
             x, gamma, beta, eps, (const __nv_bfloat16*)gate, (__nv_bfloat16*)out, rows, H);
