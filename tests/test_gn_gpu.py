@@ -2,8 +2,9 @@
 the fp64 oracle: the base recurrence, then GroupNorm over each head's 64 channels of each
 token with a per-channel affine, then the output gate -- the two pieces Finch-C2 removes.
 
-Covered: the chunked bf16 path (fast kernel, level kernel, sequence split), the fp32
-recurrence, the gate absent, the decode step in both dtypes, and the argument checks.
+Covered: the chunked bf16 path (fast kernel, level kernel after a hand-over, the sequence
+split with and without a hand-over), the fp32 recurrence, the gate absent, the decode step
+in both dtypes, and the argument checks.
 """
 import ctypes
 
@@ -69,6 +70,21 @@ def test_gn_level_kernel_hand_over(oracle):
     inp = _problem(9530, B=2, T=300, H=3)
     om = inp["omega"].float()
     om[:, 140:, 1, ::3] = 3.5     # decay range the fast kernel hands to the level kernel
+    inp["omega"] = om.to(torch.bfloat16)
+    y, s = _run(inp)
+    yo, so = _oracle(oracle, inp)
+    assert rel_err(y, yo) <= TOL[torch.bfloat16]
+    assert rel_err(s, so) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("extreme_from", [0, 700])
+def test_gn_split_with_hand_over(oracle, monkeypatch, extreme_from):
+    """Sequence split into 3 segments with a hand-over to the level kernel in the first or
+    the last segment: the GroupNorm pass sees rows from both kernels."""
+    monkeypatch.setenv("GOLDWKV_SEGMENTS", "3")
+    inp = _problem(9545 + extreme_from, B=1, T=1100, H=2)
+    om = inp["omega"].float()
+    om[:, extreme_from:extreme_from + 90, 1, ::4] = 3.5
     inp["omega"] = om.to(torch.bfloat16)
     y, s = _run(inp)
     yo, so = _oracle(oracle, inp)
