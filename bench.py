@@ -695,10 +695,11 @@ def main():
                     help="skip the ~1 s untimed warm-up loop (for profiler runs)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the prefill batch size (smaller profiler captures)")
-    ap.add_argument("--backward-only", action="store_true",
-                    help="print only the backward line (wkv6_backward on the 1.5B-layer shape, "
-                         "--batch and --seq-len override B and T), for profiler runs")
-    ap.add_argument("--seq-len", type=int, default=None, help="T of --backward-only")
+    ap.add_argument("--only", choices=["backward", "gold"], default=None,
+                    help="print only that line (wkv6_backward, or GOLD compression + "
+                         "decompression, on the 1.5B-layer shape; --batch and --seq-len "
+                         "override B and T), for profiler runs")
+    ap.add_argument("--seq-len", type=int, default=None, help="T of --only")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -714,12 +715,14 @@ def main():
 
     world, rank, local = dist_setup()
     try:
-        if args.backward_only:
+        if args.only is not None:
             from linear_attention_rnn_finch_b200 import binding
             binding.load()
             cfg = PREFILL_CFG.with_(**{k: v for k, v in (("B", args.batch), ("T", args.seq_len))
                                        if v is not None})
-            out = backward_line(cfg, torch.device("cuda", local), world, steps=args.steps)
+            dev = torch.device("cuda", local)
+            out = (backward_line(cfg, dev, world, steps=args.steps) if args.only == "backward"
+                   else gold_line(dev, world, steps=args.steps, B=cfg.B, T=cfg.T))
         else:
             out = run_ours(args, world, rank, local)
         if rank == 0 and out is not None:

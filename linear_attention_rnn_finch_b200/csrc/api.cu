@@ -595,7 +595,9 @@ size_t gold_compress_workspace_bytes(long N, int D, int Dc) {
 
 size_t gold_decompress_workspace_bytes(long N, int D, int Dc) {
     if (check_gold_sizes(N, D, Dc) != WKV_OK || N == 0) return 0;
-    return round256((size_t)N * D * sizeof(float)) + kLtWorkspace;
+    // fp32 product, the bf16 concatenation [x0 | c], cuBLASLt's workspace
+    return round256((size_t)N * D * sizeof(float)) + round256((size_t)N * (D + Dc) * 2) +
+           kLtWorkspace;
 }
 
 wkv_status gold_compress(const void* x, const void* w_kd, void* c, long N, int D, int Dc,
@@ -644,8 +646,9 @@ wkv_status gold_decompress(const void* x0, const void* c, const void* w_ku, cons
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* z = reinterpret_cast<float*>(ws);
-    void* lt = ws + round256((size_t)N * D * sizeof(float));
-    if (!goldwkv::gold_gemm_decompress(x0, c, w_ku, z, N, D, Dc, lt, kLtWorkspace, st))
+    uint8_t* cat = ws + round256((size_t)N * D * sizeof(float));
+    void* lt = cat + round256((size_t)N * (D + Dc) * 2);
+    if (!goldwkv::gold_gemm_decompress(x0, c, w_ku, cat, z, N, D, Dc, lt, kLtWorkspace, st))
         return WKV_ERR_CUDA;
     return from_cuda(goldwkv::launch_rmsnorm_rows(z, gamma, eps, kd, N, D, st));
 }

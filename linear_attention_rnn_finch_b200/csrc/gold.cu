@@ -3,9 +3,10 @@
 //     c_t   = x_t W_KD                                   (D -> Dc = D/16)
 //     k^D_t = RMSNorm(concat(x0_t, c_t) W_KU)            (D + Dc -> D)
 // Both products are plain dense GEMMs and run through cuBLASLt on the tensor cores (bf16
-// operands, fp32 accumulation).  The concatenation is never formed: W_KU splits into the
-// block that multiplies x0 and the block that multiplies c, and the second GEMM accumulates
-// into the first one's fp32 output.  RMSNorm over the D outputs of a token is our kernel.
+// operands, fp32 accumulation).  The concatenation [x0 | c] is copied into the workspace
+// by a kernel of ours (16-byte moves) so that the decompression is one GEMM over
+// K = D + Dc, its fp32 output written once; RMSNorm over the D outputs of a token is our
+// kernel too.
 //
 // Row-major [rows][cols] matrices are cuBLAS column-major [cols x rows] matrices, so with
 // the weights given as the rows of each map (w[out][in]) every product is a "TN" GEMM:
@@ -78,6 +79,18 @@ bool gemm_tn(int m, int n, int k, const void* A, int lda, const void* B, int ldb
     return ok;
 }
 
+// cat [N][D + Dc] = [x0 | c], rows of bf16 moved as 16-byte chunks (D, Dc multiples of 8)
+__global__ void concat_rows_kernel(const uint4* __restrict__ x0, const uint4* __restrict__ c,
+                                   uint4* __restrict__ cat, long N, int dq, int cq) {
+    const long total = N * (dq + cq);
+    for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long)gridDim.x * blockDim.x) {
+        const long n = e / (dq + cq);
+        const int j = (int)(e - n * (dq + cq));
+        cat[e] = j < dq ? x0[n * dq + j] : c[n * cq + (j - dq)];
+    }
+}
+
 constexpr int kRmsThreads = 256;
 
 // One CTA per row: sum of squares over the D fp32 values (16-byte loads), then the scale.
@@ -122,14 +135,19 @@ bool gold_gemm_compress(const void* x, const void* w_kd, void* c, long N, int D,
                    lt_bytes, st);
 }
 
-bool gold_gemm_decompress(const void* x0, const void* c, const void* w_ku, float* z, long N,
-                          int D, int Dc, void* lt_workspace, size_t lt_bytes, cudaStream_t st) {
-    const int K = D + Dc;
-    const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(w_ku);
-    // z^T = w_ku[:, :D] . x0^T, then += w_ku[:, D:] . c^T
-    return gemm_tn(D, (int)N, D, w, K, x0, D, 0.f, z, CUDA_R_32F, D, lt_workspace, lt_bytes,
-                   st) &&
-           gemm_tn(D, (int)N, Dc, w + D, K, c, Dc, 1.f, z, CUDA_R_32F, D, lt_workspace, lt_bytes,
+bool gold_gemm_decompress(const void* x0, const void* c, const void* w_ku, void* cat, float* z,
+                          long N, int D, int Dc, void* lt_workspace, size_t lt_bytes,
+                          cudaStream_t st) {
+    const int K = D + Dc, dq = D / 8, cq = Dc / 8;
+    const long chunks = N * (dq + cq);
+    const unsigned grid = (unsigned)((chunks + 255) / 256 < 148L * 16 ? (chunks + 255) / 256
+                                                                       : 148L * 16);
+    concat_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x0),
+                                             static_cast<const uint4*>(c),
+                                             static_cast<uint4*>(cat), N, dq, cq);
+    if (cudaGetLastError() != cudaSuccess) return false;
+    // z^T (D x N) = w_ku (K x D col-major, transposed) . cat^T (K x N)
+    return gemm_tn(D, (int)N, K, w_ku, K, cat, K, 0.f, z, CUDA_R_32F, D, lt_workspace, lt_bytes,
                    st);
 }
 
