@@ -314,6 +314,9 @@ def backward_line(cfg, dev, world, steps):
     e1.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
     flops, nbytes = backward_flops(B, T, H, D), backward_bytes(B, T, H, D)
+    # dr scan, dk scan, du sum; 2 reversals + fast + level kernels for dv (+ 2 segment
+    # kernels when the sequence is split)
+    launches_per_call = 3 + 4
     line = {"workload": "wkv6_backward_1p5b_layer", "B": B, "T": T, "H": H, "D": D, "io": "bf16",
             "steps": steps, "ms_per_call": ms, "tokens_per_s": world * B * T / (ms / 1e3),
             "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
@@ -322,8 +325,13 @@ def backward_line(cfg, dev, world, steps):
                          "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
                          "algorithmic_flops_per_call": flops},
             "hbm": {"achieved_gbs": nbytes / (ms / 1e3) / 1e9, "algorithmic_bytes_per_call": nbytes},
-            "gpu_launches": 3 * steps,
-            "kernels": "wkv6_bwd_dr_dv_kernel, wkv6_bwd_dk_domega_kernel, wkv6_bwd_du_kernel"}
+            "gpu_launches": launches_per_call * steps,
+            "kernels": "dr scan (wkv6_bwd_dr_dv_kernel), dk + decay-gradient scan "
+                       "(wkv6_bwd_dk_domega_kernel), du sum; dv through the chunked tensor-core "
+                       "prefill on time-reversed copies (reverse_tokens_kernel x2, "
+                       "wkv6_fast_kernel, wkv6_chunked_kernel)",
+            "note": "algorithmic FLOPs are the three recurrences (dr, dk, dv) at 5 FLOPs per "
+                    "state entry per token; dv runs on the tensor cores"}
     del inp, dy, dS, ws, args_b
     torch.cuda.empty_cache()
     return line

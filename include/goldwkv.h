@@ -221,8 +221,11 @@ wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, cons
  *     dv_t = G^T k_t + (r_t . (u * k_t)) dy_t           du   = sum_{b,t} r_t * k_t (v_t . dy_t)
  *     domega_t[i] = (sum_j G[i][j] S_{t-1}[i][j]) * w_t[i] * (-exp(omega_t[i]))
  *     G <- diag(w_t) G + r_t^T dy_t,   dstate_in = G before the first token.
- * The three scans run on CUDA cores in fp32 (the decay gradient through the equivalent sum
- * of the pair terms that straddle each token).
+ * dr and dk (with the decay gradient, through the equivalent sum of the pair terms that
+ * straddle each token) are token-by-token scans on CUDA cores in fp32.  dv is the forward
+ * recurrence run in reversed time with r and k swapped and dy as the value; with bf16 I/O
+ * it runs through the chunked tensor-core prefill on time-reversed copies, with fp32 I/O
+ * as a third scan.
  *   r, k, v, omega, u, state_in   the forward call's inputs (state_in NULL = zeros)
  *   dy          [B][T][H][D] io   gradient of y
  *   dstate_out  [B][H][D][D] fp32 gradient of the final state, or NULL (zero)

@@ -233,6 +233,55 @@ size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_l
 
 namespace {
 
+// The chunked tensor-core path of a bf16 prefill: for P > 1 the segment pre-pass and carry,
+// then the fast kernel and the level-factorised kernel (which resumes any (b,h) the fast one
+// handed over), or the level kernel alone (levels_only).  ws: a workspace laid out as
+// chunked_bytes(B, H, P) describes.  Returns false if a tensor map cannot be made; *e holds
+// the first launch error.
+bool launch_chunked_path(const void* r, const void* k, const void* v, const void* omega,
+                         const float* u, const goldwkv::Variant& var, const float* state_in,
+                         float* state_out, void* y, float* y_raw, int B, int T, int H, int P,
+                         bool levels_only, uint8_t* ws, cudaStream_t st, cudaError_t* e) {
+    const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+    CUtensorMap maps[5];
+    if (!goldwkv::make_token_map(&maps[0], r, B, T, H) ||
+        !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
+        !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
+        !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
+        !goldwkv::make_token_map(&maps[4], y, B, T, H))
+        return false;
+    const long units = (long)B * H * P;
+    const size_t hand_i = kStatusBytes;
+    const size_t hand_s = hand_i + handoff_ints_bytes(units);
+    const size_t seg_at = hand_s + handoff_state_bytes(units);
+    int* status = reinterpret_cast<int*>(ws);
+    int* h_chunk = reinterpret_cast<int*>(ws + hand_i);
+    float* h_state = reinterpret_cast<float*>(ws + hand_s);
+    float* s_mid = reinterpret_cast<float*>(ws + seg_at);
+    float* log2g = s_mid + (size_t)B * H * (P - 1) * 64 * 64;
+    const int nc = (T + kChunk - 1) / kChunk;
+    const goldwkv::Segments seg{P, (nc + P - 1) / P, s_mid};
+    if (levels_only) {
+        *e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg,
+                                            var, status, nullptr, nullptr, budget, st);
+        return true;
+    }
+    *e = cudaSuccess;
+    if (P > 1) {   // states entering segments 1 .. P-1 (computed in place in s_mid)
+        *e = goldwkv::launch_segment_states(maps, s_mid, log2g, B, T, H, seg, var, status, budget,
+                                            st);
+        if (*e == cudaSuccess)
+            *e = goldwkv::launch_segment_carry(state_in, s_mid, log2g, s_mid, B, H, P, st);
+    }
+    if (*e == cudaSuccess)
+        *e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H, seg,
+                                          var, status, h_chunk, h_state, budget, st);
+    if (*e == cudaSuccess)
+        *e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg, var,
+                                            status, h_chunk, h_state, budget, st);
+    return true;
+}
+
 // Shared by the base (static bonus u) and the Finch-C2 (second value uprime) entry points:
 // exactly one of u / uprime is used, selected by uprime != nullptr.
 wkv_status prefill_impl(const void* r, const void* k, const void* v, const void* omega,
@@ -308,47 +357,13 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
     const int P = !chunked || algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
-    const long units = (long)B * H * P;
-    const size_t hand_i = chunked ? kStatusBytes : 0;
-    const size_t hand_s = hand_i + (chunked ? handoff_ints_bytes(units) : 0);
-    const size_t seg_at = hand_s + (chunked ? handoff_state_bytes(units) : 0);
     const size_t raw_at = chunked ? chunked_bytes(B, H, P) : 0;
     if (nm.on()) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
     if (chunked) {
-        const long long budget = injected("timeout0") ? 0 : kSpinBudget;
-        CUtensorMap maps[5];
-        if (!goldwkv::make_token_map(&maps[0], r, B, T, H) ||
-            !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
-            !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
-            !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
-            !goldwkv::make_token_map(&maps[4], y, B, T, H))
+        if (!launch_chunked_path(r, k, v, omega, u, var, state_in, state_out, y, y_raw, B, T, H,
+                                 P, algo == WKV_ALGO_CHUNKED_LEVELS, ws, st, &e))
             return WKV_ERR_CUDA;
-        int* status = reinterpret_cast<int*>(ws);
-        int* h_chunk = reinterpret_cast<int*>(ws + hand_i);
-        float* h_state = reinterpret_cast<float*>(ws + hand_s);
-        float* s_mid = reinterpret_cast<float*>(ws + seg_at);
-        float* log2g = s_mid + (size_t)B * H * (P - 1) * 64 * 64;
-        const int nc = (T + kChunk - 1) / kChunk;
-        const goldwkv::Segments seg{P, (nc + P - 1) / P, s_mid};
-        if (algo == WKV_ALGO_CHUNKED_LEVELS) {
-            e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg,
-                                               var, status, nullptr, nullptr, budget, st);
-        } else {
-            e = cudaSuccess;
-            if (P > 1) {   // states entering segments 1 .. P-1 (computed in place in s_mid)
-                e = goldwkv::launch_segment_states(maps, s_mid, log2g, B, T, H, seg, var, status,
-                                                   budget, st);
-                if (e == cudaSuccess)
-                    e = goldwkv::launch_segment_carry(state_in, s_mid, log2g, s_mid, B, H, P, st);
-            }
-            if (e == cudaSuccess)
-                e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H,
-                                                 seg, var, status, h_chunk, h_state, budget, st);
-            if (e == cudaSuccess)
-                e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H,
-                                                   seg, var, status, h_chunk, h_state, budget, st);
-        }
     } else {
         e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,
                                       H, bf16, var, st);
@@ -500,7 +515,10 @@ size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
     // P and E in the row scans' accumulation type: fp64 for fp32 I/O, fp32 for bf16 I/O
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     const size_t x = (size_t)B * T * H * D, bh = (size_t)B * H * D;
-    return round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
+    size_t bytes = round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
+    // bf16: time-reversed k, r, dy, omega and dv, and the chunked prefill's own workspace
+    if (io == WKV_BF16) bytes += 5 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H));
+    return bytes;
 }
 
 wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void* omega,
@@ -561,10 +579,39 @@ wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     void* P = ws;
     uint8_t* E = ws + round256((size_t)B * T * H * D * acc);
-    float* du_part = reinterpret_cast<float*>(E + round256((size_t)B * H * D * acc));
+    uint8_t* dpart = E + round256((size_t)B * H * D * acc);
+    float* du_part = reinterpret_cast<float*>(dpart);
+    const bool bf16 = io == WKV_BF16;
+    if (bf16) {
+        // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
+        // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.
+        // It runs through the chunked tensor-core prefill on time-reversed copies.
+        const size_t xr = round256(xbytes);
+        uint8_t* rev = dpart + round256((size_t)B * H * D * sizeof(float));
+        void* rk = rev;
+        void* rr = rev + xr;
+        void* rdy = rev + 2 * xr;
+        void* rom = rev + 3 * xr;
+        void* rdv = rev + 4 * xr;
+        uint8_t* cws = rev + 5 * xr;
+        const void* src[4] = {k, r, dy, omega};
+        void* dst[4] = {rk, rr, rdy, rom};
+        if (goldwkv::launch_reverse_tokens(src, dst, 4, B, T, H, st) != cudaSuccess)
+            return WKV_ERR_CUDA;
+        cudaError_t e = cudaSuccess;
+        if (!launch_chunked_path(rk, rr, rdy, rom, u, goldwkv::Variant{nullptr}, dstate_out,
+                                 nullptr, rdv, nullptr, B, T, H, choose_segments(B, T, H), false,
+                                 cws, st, &e) ||
+            e != cudaSuccess)
+            return WKV_ERR_CUDA;
+        const void* src_dv[1] = {rdv};
+        void* dst_dv[1] = {dv};
+        if (goldwkv::launch_reverse_tokens(src_dv, dst_dv, 1, B, T, H, st) != cudaSuccess)
+            return WKV_ERR_CUDA;
+    }
     return from_cuda(goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr,
                                               dk, dv, domega, du, dstate_in, P, E, du_part, B,
-                                              T, H, io == WKV_BF16, st));
+                                              T, H, bf16, /*with_dv=*/!bf16, st));
 }
 
 

@@ -23,7 +23,9 @@
 //       roles r <-> k, v -> dy run backwards
 //   dk  rows of G, reverse in time, with the decay-gradient scan fused (needs P and E).
 // The dr and dv sweeps run as one launch (blockIdx.z); the dk sweep follows; a small kernel
-// sums du over the batch.
+// sums du over the batch.  Because dv is exactly a forward recurrence in reversed time, the
+// bf16 path leaves it out of these scans and runs it through the chunked tensor-core
+// prefill on time-reversed copies (reverse_tokens_kernel moves them).
 //
 // Work split: a CTA owns one (b,h) and 32 of the 64 rows (or columns); thread (row, q)
 // keeps 16 state entries in registers, the sum over the other index is finished with two
@@ -526,6 +528,25 @@ wkv6_bwd_dk_domega_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                         T, H);
 }
 
+// dst[i][b][t][h][:] = src[i][b][T-1-t][h][:] for n bf16 tensors [B][T][H][64]: 16-byte moves
+struct ReverseArgs {
+    const uint4* src[kMaxReverse];
+    uint4* dst[kMaxReverse];
+};
+
+__global__ void reverse_tokens_kernel(ReverseArgs a, int n, long B, int T, int H) {
+    const long per = (long)T * H * 8;               // 16-byte chunks per batch row
+    const long total = B * per;
+    for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long)gridDim.x * blockDim.x) {
+        const long b = e / per;
+        const long rem = e - b * per;
+        const long t = rem / ((long)H * 8);
+        const long src_e = b * per + ((long)(T - 1 - t) * H * 8) + (rem - t * H * 8);
+        for (int i = 0; i < n; ++i) a.dst[i][e] = a.src[i][src_e];
+    }
+}
+
 // du[h][i] = sum_b du_part[b][h][i]  (fixed order: deterministic)
 __global__ void wkv6_bwd_du_kernel(const float* __restrict__ du_part, float* __restrict__ du,
                                    int B, int H) {
@@ -540,13 +561,13 @@ cudaError_t launch_typed(const void* r, const void* k, const void* v, const void
                          const float* u, const float* state_in, const void* dy,
                          const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                          float* du, float* dstate_in, void* P_, void* E_, float* du_part, int B,
-                         int T, int H, cudaStream_t st) {
+                         int T, int H, bool with_dv, cudaStream_t st) {
     using Acc = typename Prec<IO>::Acc;
     const IO *r_ = (const IO*)r, *k_ = (const IO*)k, *v_ = (const IO*)v, *o_ = (const IO*)omega,
              *dy_ = (const IO*)dy;
     Acc *P = static_cast<Acc*>(P_), *E = static_cast<Acc*>(E_);
     const unsigned bh = (unsigned)(B * H);
-    wkv6_bwd_dr_dv_kernel<IO><<<dim3(bh, kHeadSize / kHalf, 2), kThreads, 0, st>>>(
+    wkv6_bwd_dr_dv_kernel<IO><<<dim3(bh, kHeadSize / kHalf, with_dv ? 2 : 1), kThreads, 0, st>>>(
         r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -563,12 +584,29 @@ cudaError_t launch_backward(const void* r, const void* k, const void* v, const v
                             const float* u, const float* state_in, const void* dy,
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
-                            int B, int T, int H, bool bf16, cudaStream_t st) {
+                            int B, int T, int H, bool bf16, bool with_dv, cudaStream_t st) {
     if (bf16)
         return launch_typed<__nv_bfloat16>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
-                                           dv, domega, du, dstate_in, P, E, du_part, B, T, H, st);
+                                           dv, domega, du, dstate_in, P, E, du_part, B, T, H,
+                                           with_dv, st);
     return launch_typed<float>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv, domega,
-                               du, dstate_in, P, E, du_part, B, T, H, st);
+                               du, dstate_in, P, E, du_part, B, T, H, with_dv, st);
+}
+
+cudaError_t launch_reverse_tokens(const void* const* src, void* const* dst, int n, int B, int T,
+                                  int H, cudaStream_t st) {
+    if (n < 1 || n > kMaxReverse) return cudaErrorInvalidValue;
+    if (B <= 0 || T <= 0 || H <= 0) return cudaSuccess;
+    ReverseArgs a{};
+    for (int i = 0; i < n; ++i) {
+        a.src[i] = static_cast<const uint4*>(src[i]);
+        a.dst[i] = static_cast<uint4*>(dst[i]);
+    }
+    const long total = (long)B * T * H * 8;
+    const long blocks = (total + 255) / 256;
+    reverse_tokens_kernel<<<(unsigned)(blocks < 148L * 16 ? blocks : 148L * 16), 256, 0, st>>>(
+        a, n, B, T, H);
+    return cudaGetLastError();
 }
 
 }  // namespace goldwkv

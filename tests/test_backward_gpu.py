@@ -3,7 +3,10 @@
 Every gradient (dr, dk, dv, domega, du, dS0) is compared element by element at sizes that
 span several 32-token tiles and a ragged tail, for fp32 and bf16 I/O, with and without an
 initial state and a final-state gradient; the 1.5B-layer shape (B8 T4096 H32, bf16) is
-checked on sampled heads.  Also: the empty sequence, determinism and argument checks.
+checked on sampled heads.  With bf16 I/O dv comes from the chunked tensor-core prefill run
+on time-reversed copies: extreme decays (hand-over to the level kernel) and a forced
+sequence split cover that path.  Also: the empty sequence, determinism and argument
+checks.
 """
 import ctypes
 
@@ -76,6 +79,20 @@ def test_backward_strong_decay(oracle):
     g = torch.Generator(device=DEV).manual_seed(9881)
     inp["omega"] = -9.0 + 13.0 * torch.rand(inp["omega"].shape, generator=g, device=DEV)
     _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.float32])
+
+
+@pytest.mark.parametrize("segments", [None, "3"])
+def test_backward_bf16_extreme_decay_and_split(oracle, monkeypatch, segments):
+    """bf16: dv runs through the chunked prefill on time-reversed copies; decays near zero
+    make it hand sequences to the level kernel, and a forced 3-way sequence split runs the
+    segment pre-pass on the reversed sequence."""
+    if segments:
+        monkeypatch.setenv("GOLDWKV_SEGMENTS", segments)
+    inp = _problem(9895, B=2, T=1100, H=2, dtype=torch.bfloat16)
+    om = inp["omega"].float()
+    om[:, 300:420, 1, ::3] = 3.5
+    inp["omega"] = om.to(torch.bfloat16)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
 
 
 def test_backward_empty_sequence():
