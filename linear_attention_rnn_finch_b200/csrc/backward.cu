@@ -267,32 +267,14 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
         }
         __syncthreads();
 
-        // operands of token `st` (in sweep order) from shared memory; the next token's are
-        // read while the current one is computed
-        float4 qc[4], bc[4];
-        float ac = 0.f, wc = 0.f;
-        auto operands = [&](int st, float4 (&qv)[4], float4 (&bv)[4], float& a, float& w) {
-            const int tt = kRev ? nt - 1 - st : st;
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                qv[m4] = *reinterpret_cast<const float4*>(&s.q[tt][16 * m4 + 4 * qq]);
-                bv[m4] = *reinterpret_cast<const float4*>(&s.b[tt][16 * m4 + 4 * qq]);
-            }
-            a = s.a[tt][rl];
-            w = s.w[tt][rl];
-        };
-        if (nt > 0) operands(0, qc, bc, ac, wc);
-#pragma unroll 2
         for (int st = 0; st < nt; ++st) {
             const int tt = kRev ? nt - 1 - st : st;
-            float4 qn[4], bn[4];
-            float an, wn;
-            operands(min(st + 1, nt - 1), qn, bn, an, wn);
-            const Acc ai = ac, wi = wc;
+            const Acc ai = s.a[tt][rl], wi = s.w[tt][rl];
             Acc acc0 = 0, acc1 = 0;
 #pragma unroll
             for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 qv = qc[m4], bv = bc[m4];
+                const float4 qv = *reinterpret_cast<const float4*>(&s.q[tt][16 * m4 + 4 * qq]);
+                const float4 bv = *reinterpret_cast<const float4*>(&s.b[tt][16 * m4 + 4 * qq]);
                 Acc* x = &X[4 * m4];
                 acc0 += x[0] * (Acc)qv.x;
                 acc1 += x[1] * (Acc)qv.y;
@@ -319,13 +301,6 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
                     accP += s.p[tt][rl];
                 }
             }
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                qc[m4] = qn[m4];
-                bc[m4] = bn[m4];
-            }
-            ac = an;
-            wc = wn;
         }
         __syncthreads();
         for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
@@ -435,30 +410,15 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
         }
         __syncthreads();
 
-        float4 kc[4], rc[4], wc[4];
-        float dc = 0.f;
-        auto operands = [&](int st, float4 (&kv)[4], float4 (&rv)[4], float4 (&wv)[4], float& d) {
-            const int tt = nt - 1 - st;
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                kv[m4] = *reinterpret_cast<const float4*>(&s.k[tt][16 * m4 + 4 * qq]);
-                rv[m4] = *reinterpret_cast<const float4*>(&s.r[tt][16 * m4 + 4 * qq]);
-                wv[m4] = *reinterpret_cast<const float4*>(&s.w[tt][16 * m4 + 4 * qq]);
-            }
-            d = s.dy[tt][jl];
-        };
-        if (nt > 0) operands(0, kc, rc, wc, dc);
-#pragma unroll 2
         for (int st = 0; st < nt; ++st) {
             const int tt = nt - 1 - st;
-            float4 kn[4], rn[4], wn[4];
-            float dn;
-            operands(min(st + 1, nt - 1), kn, rn, wn, dn);
-            const float dyj = dc;
+            const float dyj = s.dy[tt][jl];
             float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
             for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 kk = kc[m4], rr = rc[m4], ww = wc[m4];
+                const float4 kk = *reinterpret_cast<const float4*>(&s.k[tt][16 * m4 + 4 * qq]);
+                const float4 rr = *reinterpret_cast<const float4*>(&s.r[tt][16 * m4 + 4 * qq]);
+                const float4 ww = *reinterpret_cast<const float4*>(&s.w[tt][16 * m4 + 4 * qq]);
                 float* g = &G[4 * m4];
                 acc0 = fmaf(kk.x, g[0], acc0);
                 acc1 = fmaf(kk.y, g[1], acc1);
@@ -473,13 +433,6 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             if (qq == 0) s.o[tt][jl] = fmaf(s.rku[tt], dyj, acc);
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                kc[m4] = kn[m4];
-                rc[m4] = rn[m4];
-                wc[m4] = wn[m4];
-            }
-            dc = dn;
         }
         __syncthreads();
         for (int idx = tid; idx < nt * kHalf; idx += kThreads) {

@@ -25,6 +25,82 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
     return t;
 }
 
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(w[e] << 16);
+        v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        w[e] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Rows of C = 8 * n channels, n <= kMax * kThreads: each thread holds up to kMax chunks of
+// 8 values in registers (16-byte loads and stores), so the row is read from memory once.
+template <typename IO, int kMax>
+__global__ void __launch_bounds__(kThreads)
+layernorm_rows_vec_kernel(const float* x, const float* __restrict__ gamma,
+                          const float* __restrict__ beta, float eps, IO* out, int C) {
+    __shared__ float red[kThreads / 32];
+    const float* row = x + (size_t)blockIdx.x * C;
+    IO* orow = out + (size_t)blockIdx.x * C;
+    const int nch = C / 8;
+    float v[kMax][8];
+    float s = 0.f;
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+        const int ch = threadIdx.x + m * kThreads;
+        if (ch < nch) {
+            load8(row + 8 * ch, v[m]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += v[m][e];
+        }
+    }
+    const float mean = block_sum(s, red) / (float)C;
+    float q = 0.f;
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+        if (threadIdx.x + m * kThreads < nch) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[m][e] -= mean;
+                q = fmaf(v[m][e], v[m][e], q);
+            }
+        }
+    }
+    const float inv = rsqrtf(block_sum(q, red) / (float)C + eps);
+    // x and out may alias (fp32 in place): the row was read before the barriers above
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+        const int ch = threadIdx.x + m * kThreads;
+        if (ch < nch) {
+            float g[8], b[8];
+            load8(gamma + 8 * ch, g);
+            load8(beta + 8 * ch, b);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[m][e] = fmaf(v[m][e] * inv, g[e], b[e]);
+            store8(orow + 8 * ch, v[m]);
+        }
+    }
+}
+
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
 layernorm_rows_kernel(const float* x, const float* __restrict__ gamma,
@@ -63,33 +139,6 @@ __device__ __forceinline__ float gn_sum(float v) {   // over the 8 lanes of a ro
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 4);
     return v;
-}
-
-__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 a = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        v[2 * e] = __uint_as_float(w[e] << 16);
-        v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-    }
-}
-__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
-    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
-__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-        w[e] = *reinterpret_cast<uint32_t*>(&t);
-    }
-    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 template <typename IO>
@@ -149,11 +198,28 @@ cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const floa
                                   float eps, void* out, long rows, int C, bool bf16,
                                   cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
+    // C = H * 64: whole 8-value chunks; rows of up to 8192 channels stay in registers
+    const int per = (C / 8 + kThreads - 1) / kThreads;
+    const unsigned grid = (unsigned)rows;
+    if (C % 8 == 0 && per <= 4) {
+        if (bf16) {
+            auto* o = (__nv_bfloat16*)out;
+            if (per == 1) layernorm_rows_vec_kernel<__nv_bfloat16, 1><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, o, C);
+            else if (per == 2) layernorm_rows_vec_kernel<__nv_bfloat16, 2><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, o, C);
+            else layernorm_rows_vec_kernel<__nv_bfloat16, 4><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, o, C);
+        } else {
+            auto* o = (float*)out;
+            if (per == 1) layernorm_rows_vec_kernel<float, 1><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, o, C);
+            else if (per == 2) layernorm_rows_vec_kernel<float, 2><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, o, C);
+            else layernorm_rows_vec_kernel<float, 4><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, o, C);
+        }
+        return cudaGetLastError();
+    }
     if (bf16)
-        layernorm_rows_kernel<__nv_bfloat16><<<(unsigned)rows, kThreads, 0, st>>>(
+        layernorm_rows_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
             x, gamma, beta, eps, (__nv_bfloat16*)out, C);
     else
-        layernorm_rows_kernel<float><<<(unsigned)rows, kThreads, 0, st>>>(
+        layernorm_rows_kernel<float><<<grid, kThreads, 0, st>>>(
             x, gamma, beta, eps, (float*)out, C);
     return cudaGetLastError();
 }
