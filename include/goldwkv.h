@@ -256,8 +256,8 @@ wkv_status wkv6_backward(const void *r, const void *k, const void *v, const void
  *   x, x0 [N][D];  c [N][Dc];  kd [N][D];  w_kd [Dc][D] (w_kd[j][i] = W_KD[i][j]);
  *   w_ku [D][D + Dc] (w_ku[o][i] = W_KU[i][o]);  gamma [D] fp32 or NULL (= 1).
  * The products run on the tensor cores through cuBLASLt with fp32 accumulation (c is
- * rounded to bf16 once).  D and Dc must be multiples of 8 (else WKV_ERR_UNSUPPORTED),
- * N <= 2^31 - 1.  Outputs may not overlap inputs or the workspace.  Workspace: at least
+ * rounded to bf16 once).  D and Dc must be multiples of 8 and D <= 16384 (else
+ * WKV_ERR_UNSUPPORTED), N <= 2^31 - 1.  Outputs may not overlap inputs or the workspace.  Workspace: at least
  * gold_*_workspace_bytes(...) bytes, any contents; for decompression it holds the
  * concatenation [x0 | c] (bf16) and the fp32 product before RMSNorm.  eps must be > 0.
  */

@@ -627,7 +627,7 @@ constexpr size_t kLtWorkspace = (size_t)32 << 20;   // cuBLASLt workspace per ca
 // the GEMMs' int range.
 wkv_status check_gold_sizes(long N, int D, int Dc) {
     if (N < 0 || D <= 0 || Dc <= 0) return WKV_ERR_INVALID_ARG;
-    if (D % 8 != 0 || Dc % 8 != 0 || N > 0x7fffffffL) return WKV_ERR_UNSUPPORTED;
+    if (D % 8 != 0 || Dc % 8 != 0 || D > 16384 || N > 0x7fffffffL) return WKV_ERR_UNSUPPORTED;
     return WKV_OK;
 }
 
