@@ -155,9 +155,31 @@ __device__ __forceinline__ void put_chunk_acc(uint4 raw, double* dst, int c) {
     put_chunk_f64(raw, dst, c);
 }
 
+// Sum of v over the 16 lanes of a half-warp for 4 rows at once (reduce-scatter): on return
+// the lane holds the total of row 2*bit3 + bit2 of its lane index in v[0].
+template <typename Acc>
+__device__ __forceinline__ void reduce16x4(Acc (&v)[4], int lane) {
+    const bool hi8 = lane & 8, hi4 = lane & 4;
+    // lanes with bit 3 set keep rows 2, 3; the others rows 0, 1
+    const Acc s0 = hi8 ? v[0] : v[2], s1 = hi8 ? v[1] : v[3];
+    const Acc k0 = hi8 ? v[2] : v[0], k1 = hi8 ? v[3] : v[1];
+    v[0] = k0 + __shfl_xor_sync(0xffffffffu, s0, 8);
+    v[1] = k1 + __shfl_xor_sync(0xffffffffu, s1, 8);
+    // bit 2 picks one of the two
+    const Acc s2 = hi4 ? v[0] : v[1], k2 = hi4 ? v[1] : v[0];
+    v[0] = k2 + __shfl_xor_sync(0xffffffffu, s2, 4);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
 // kRev == false: the dr sweep (a = k, m = r, b = v, q = dy, X0 = state_in), forward in time.
 // kRev == true : the dk sweep (a = r, m = k, b = dy, q = v, X0 = dS_T), reverse in time, with
 //                the decay-gradient scan (reads P and E written by the dr sweep).
+// Thread (g, c) = (tid / 16, tid % 16) keeps the 4 x 4 block of rows 4g..4g+3 (of the CTA's
+// 32) and columns 4c..4c+3: per token one 16-byte read each of the readout and update
+// vectors (its 4 columns) and of the rows' a and w, the row sums finished over the 16 lanes
+// of a half-warp by a reduce-scatter (5 shuffles for 4 rows).  Lane c % 4 == 0 of each
+// group of four then owns row e = c / 4 (its outputs and running sums).
 template <typename IO, bool kRev, typename Acc = typename Prec<IO>::Acc,
           int kTile = Prec<IO>::kTile>
 __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __restrict__ a_src,
@@ -175,28 +197,27 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh - (bh / H) * H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int qq = lane & 3;                    // column quarter: columns 16qq .. 16qq+15
-    const int rl = warp * 8 + (lane >> 2);      // local row 0..31
+    const int g = tid >> 4, c = tid & 15;
     const int rowbase = blockIdx.y * kHalf;
-    const int i = rowbase + rl;
+    const int er = 2 * ((c >> 3) & 1) + ((c >> 2) & 1);   // row (of 4) this lane owns after
+    const bool owner = (c & 3) == 0;                      // reduce16x4; one writer per row
+    const int rl_own = 4 * g + er;                        // its local row 0..31
 
     if (tid < kHalf) s.u[tid] = u[h * D + rowbase + tid];
 
-    // X[4*m4 + j] is entry (i, col(m4, j)): the four threads of a row interleave in blocks
-    // of 4 columns, so their 16-byte shared-memory reads fall in distinct banks
-    const size_t sbase = (size_t)bh * D * D + (size_t)i * D + 4 * qq;
-    auto col = [](int m4, int j) { return 16 * m4 + j; };   // + 4*qq, folded into sbase
-    Acc X[16];
+    // X[e][f]: entry (rowbase + 4g + e, 4c + f)
+    const size_t sbase = (size_t)bh * D * D + (size_t)(rowbase + 4 * g) * D + 4 * c;
+    Acc X[4][4];
 #pragma unroll
-    for (int m4 = 0; m4 < 4; ++m4)
+    for (int e = 0; e < 4; ++e)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) X[4 * m4 + j] = x0 ? (Acc)x0[sbase + col(m4, j)] : Acc(0);
+        for (int f = 0; f < 4; ++f) X[e][f] = x0 ? (Acc)x0[sbase + (size_t)e * D + f] : Acc(0);
 
     const size_t tstride = (size_t)H * D;
     const size_t xbase = ((size_t)b * T * H + h) * D;
     const int ntile = (T + kTile - 1) / kTile;
     Acc du_acc = 0, accP = 0, accQ = 0;
-    const Acc Ei = kRev ? E[(size_t)bh * D + i] : Acc(0);
+    const Acc Ei = kRev ? E[(size_t)bh * D + rowbase + rl_own] : Acc(0);
 
     // chunk counts per thread: [kTile][64] and [kTile][32] tiles of IO, [kTile][32] of Acc
     constexpr int kFull = kTile * D * (int)sizeof(IO) / 16 / kThreads;
@@ -210,20 +231,20 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
     auto fetch = [&](int it) {   // chunks of tile `it` (in sweep order) into registers
         const int t0 = (kRev ? ntile - 1 - it : it) * kTile, nt = min(kTile, T - t0);
 #pragma unroll
-        for (int c = 0; c < kFull; ++c) {
-            rb[c] = load_chunk(b_src, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
-            rq[c] = load_chunk(q_src, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+        for (int k = 0; k < kFull; ++k) {
+            rb[k] = load_chunk(b_src, xbase, tstride, t0, nt, 0, D, tid + k * kThreads);
+            rq[k] = load_chunk(q_src, xbase, tstride, t0, nt, 0, D, tid + k * kThreads);
         }
 #pragma unroll
-        for (int c = 0; c < kRows; ++c) {
-            ra[c] = load_chunk(a_src, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
-            rm[c] = load_chunk(m_src, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
-            ro[c] = load_chunk(omega, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
+        for (int k = 0; k < kRows; ++k) {
+            ra[k] = load_chunk(a_src, xbase, tstride, t0, nt, rowbase, kHalf, tid + k * kThreads);
+            rm[k] = load_chunk(m_src, xbase, tstride, t0, nt, rowbase, kHalf, tid + k * kThreads);
+            ro[k] = load_chunk(omega, xbase, tstride, t0, nt, rowbase, kHalf, tid + k * kThreads);
         }
         if (kRev) {
 #pragma unroll
-            for (int c = 0; c < kAcc; ++c)
-                rp[c] = load_chunk(P, xbase, tstride, t0, nt, rowbase, kHalf, tid + c * kThreads);
+            for (int k = 0; k < kAcc; ++k)
+                rp[k] = load_chunk(P, xbase, tstride, t0, nt, rowbase, kHalf, tid + k * kThreads);
         }
     };
     if (ntile > 0) fetch(0);
@@ -234,29 +255,29 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
         const int nt = min(kTile, T - t0);
         __syncthreads();   // previous tile consumed and flushed
 #pragma unroll
-        for (int c = 0; c < kFull; ++c) {
-            put_chunk<IO>(rb[c], &s.b[0][0], tid + c * kThreads);
-            put_chunk<IO>(rq[c], &s.q[0][0], tid + c * kThreads);
+        for (int k = 0; k < kFull; ++k) {
+            put_chunk<IO>(rb[k], &s.b[0][0], tid + k * kThreads);
+            put_chunk<IO>(rq[k], &s.q[0][0], tid + k * kThreads);
         }
 #pragma unroll
-        for (int c = 0; c < kRows; ++c) {
+        for (int k = 0; k < kRows; ++k) {
             constexpr int n = ChunkOf<IO>::n;
-            put_chunk<IO>(ra[c], &s.a[0][0], tid + c * kThreads);
-            put_chunk<IO>(rm[c], &s.m[0][0], tid + c * kThreads);
+            put_chunk<IO>(ra[k], &s.a[0][0], tid + k * kThreads);
+            put_chunk<IO>(rm[k], &s.m[0][0], tid + k * kThreads);
             float om[n], ne[n], w[n];
-            unpack(ro[c], om);
+            unpack(ro[k], om);
 #pragma unroll
             for (int j = 0; j < n; ++j) {   // (padding tokens past T are never read)
                 ne[j] = -expf(om[j]);
                 w[j] = expf(ne[j]);
             }
-            const int e = (tid + c * kThreads) * n;
-            store_f32(&s.ne[0][0] + e, ne);
-            store_f32(&s.w[0][0] + e, w);
+            const int e0 = (tid + k * kThreads) * n;
+            store_f32(&s.ne[0][0] + e0, ne);
+            store_f32(&s.w[0][0] + e0, w);
         }
         if (kRev) {
 #pragma unroll
-            for (int c = 0; c < kAcc; ++c) put_chunk_acc(rp[c], &s.p[0][0], tid + c * kThreads);
+            for (int k = 0; k < kAcc; ++k) put_chunk_acc(rp[k], &s.p[0][0], tid + k * kThreads);
         }
         __syncthreads();
         if (it + 1 < ntile) fetch(it + 1);   // in flight while this tile is computed
@@ -269,68 +290,66 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
 
         for (int st = 0; st < nt; ++st) {
             const int tt = kRev ? nt - 1 - st : st;
-            const Acc ai = s.a[tt][rl], wi = s.w[tt][rl];
-            Acc acc0 = 0, acc1 = 0;
+            const float4 qv = *reinterpret_cast<const float4*>(&s.q[tt][4 * c]);
+            const float4 bv = *reinterpret_cast<const float4*>(&s.b[tt][4 * c]);
+            const float4 av = *reinterpret_cast<const float4*>(&s.a[tt][4 * g]);
+            const float4 wv = *reinterpret_cast<const float4*>(&s.w[tt][4 * g]);
+            const Acc qf[4] = {qv.x, qv.y, qv.z, qv.w}, bf[4] = {bv.x, bv.y, bv.z, bv.w};
+            const Acc ae[4] = {av.x, av.y, av.z, av.w}, we[4] = {wv.x, wv.y, wv.z, wv.w};
+            Acc part[4];
 #pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 qv = *reinterpret_cast<const float4*>(&s.q[tt][16 * m4 + 4 * qq]);
-                const float4 bv = *reinterpret_cast<const float4*>(&s.b[tt][16 * m4 + 4 * qq]);
-                Acc* x = &X[4 * m4];
-                acc0 += x[0] * (Acc)qv.x;
-                acc1 += x[1] * (Acc)qv.y;
-                acc0 += x[2] * (Acc)qv.z;
-                acc1 += x[3] * (Acc)qv.w;
-                x[0] = wi * x[0] + ai * (Acc)bv.x;
-                x[1] = wi * x[1] + ai * (Acc)bv.y;
-                x[2] = wi * x[2] + ai * (Acc)bv.z;
-                x[3] = wi * x[3] + ai * (Acc)bv.w;
+            for (int e = 0; e < 4; ++e) {
+                Acc a0 = X[e][0] * qf[0], a1 = X[e][1] * qf[1];
+                a0 += X[e][2] * qf[2];
+                a1 += X[e][3] * qf[3];
+                part[e] = a0 + a1;
+#pragma unroll
+                for (int f = 0; f < 4; ++f) X[e][f] = we[e] * X[e][f] + ae[e] * bf[f];
             }
-            Acc acc = acc0 + acc1;
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (qq == 0) {
-                const Acc vdy = s.vdy[tt], mi = s.m[tt][rl];
-                const Acc bonus = (Acc)s.u[rl] * ai * vdy;
-                s.o1[tt][rl] = (float)(acc + bonus);
+            reduce16x4(part, lane);
+            if (owner) {
+                const Acc acc = part[0];
+                const Acc vdy = s.vdy[tt], mi = s.m[tt][rl_own], ai = s.a[tt][rl_own];
+                const Acc bonus = (Acc)s.u[rl_own] * ai * vdy;
+                s.o1[tt][rl_own] = (float)(acc + bonus);
                 if (!kRev) {
-                    s.o2[tt][rl] = mi * acc;          // P_t: pair terms ending at t
+                    s.o2[tt][rl_own] = mi * acc;          // P_t: pair terms ending at t
                     du_acc += mi * ai * vdy;
                 } else {
-                    accQ += mi * acc;                 // Q_t: pair terms starting at t
-                    s.o2[tt][rl] = (Ei + accP - accQ) * (Acc)s.ne[tt][rl];
-                    accP += s.p[tt][rl];
+                    accQ += mi * acc;                     // Q_t: pair terms starting at t
+                    s.o2[tt][rl_own] = (Ei + accP - accQ) * (Acc)s.ne[tt][rl_own];
+                    accP += s.p[tt][rl_own];
                 }
             }
         }
         __syncthreads();
         for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
-            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
-            const size_t g = tok_index(xbase, t0 + tt, tstride, rowbase + c);
-            out[g] = from_f32<IO>(s.o1[tt][c]);
-            if (!kRev) P[g] = s.o2[tt][c];
-            else domega[g] = from_f32<IO>((float)s.o2[tt][c]);
+            const int tt = idx / kHalf, cc = idx - (idx / kHalf) * kHalf;
+            const size_t gi = tok_index(xbase, t0 + tt, tstride, rowbase + cc);
+            out[gi] = from_f32<IO>(s.o1[tt][cc]);
+            if (!kRev) P[gi] = s.o2[tt][cc];
+            else domega[gi] = from_f32<IO>((float)s.o2[tt][cc]);
         }
     }
 
     if (!kRev) {
-        Acc e = 0;
+        Acc ev[4] = {0, 0, 0, 0};
         if (dS_T) {
 #pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4)
+            for (int e = 0; e < 4; ++e)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) e += X[4 * m4 + j] * (Acc)dS_T[sbase + col(m4, j)];
+                for (int f = 0; f < 4; ++f) ev[e] += X[e][f] * (Acc)dS_T[sbase + (size_t)e * D + f];
         }
-        e += __shfl_xor_sync(0xffffffffu, e, 1);
-        e += __shfl_xor_sync(0xffffffffu, e, 2);
-        if (qq == 0) {
-            E[(size_t)bh * D + i] = e;
-            du_part[(size_t)bh * D + i] = (float)du_acc;
+        reduce16x4(ev, lane);
+        if (owner) {
+            E[(size_t)bh * D + rowbase + rl_own] = ev[0];
+            du_part[(size_t)bh * D + rowbase + rl_own] = (float)du_acc;
         }
     } else if (x_final) {
 #pragma unroll
-        for (int m4 = 0; m4 < 4; ++m4)
+        for (int e = 0; e < 4; ++e)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) x_final[sbase + col(m4, j)] = (float)X[4 * m4 + j];
+            for (int f = 0; f < 4; ++f) x_final[sbase + (size_t)e * D + f] = (float)X[e][f];
     }
 }
 
