@@ -82,6 +82,9 @@ class Oracle:
         lib.wkv6_oracle_backward.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                              dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
         lib.wkv6_oracle_backward.restype = ctypes.c_int
+        lib.wkv6c2_oracle_backward.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int,
+                                               ctypes.c_int] + [dp] * 13
+        lib.wkv6c2_oracle_backward.restype = ctypes.c_int
         lib.gold_oracle_compress.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp, dp]
         lib.gold_oracle_compress.restype = ctypes.c_int
         lib.gold_oracle_decompress.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp, dp,
@@ -154,6 +157,24 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle backward failed rc={rc}")
         return dr, dk, dv, dom, du, ds_in
+
+    def backward_c2(self, r, k, v, omega, state_in, dy, dstate_out=None):
+        """Gradients of prefill_c2: (dr, dk, dv, domega, duprime [B,T,H,D], dstate_in
+        [B,H,D,D]) for dy [B,T,H,D] and dstate_out [B,H,D,D] (None: zero); fp64."""
+        r, k, v, omega, dy = (self._f64(x) for x in (r, k, v, omega, dy))
+        s_in, ds_out = self._f64(state_in), self._f64(dstate_out)
+        B, T, H, D = r.shape
+        assert k.shape == v.shape == omega.shape == dy.shape == r.shape
+        dr, dk, dv, dom, dup = (np.empty_like(r) for _ in range(5))
+        ds_in = np.empty((B, H, D, D), dtype=np.float64)
+        rc = self._lib.wkv6c2_oracle_backward(B, T, H, D, self._ptr(r), self._ptr(k), self._ptr(v),
+                                              self._ptr(omega), self._ptr(s_in), self._ptr(dy),
+                                              self._ptr(ds_out), self._ptr(dr), self._ptr(dk),
+                                              self._ptr(dv), self._ptr(dom), self._ptr(dup),
+                                              self._ptr(ds_in))
+        if rc != 0:
+            raise RuntimeError(f"oracle backward_c2 failed rc={rc}")
+        return dr, dk, dv, dom, dup, ds_in
 
     def prefill_c2(self, r, k, v, omega, uprime, state_in=None, nthreads: int | None = None):
         """Finch-C2 exact form: key k (1 - w), second value uprime [B,T,H,D] added to the

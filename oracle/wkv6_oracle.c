@@ -513,3 +513,114 @@ int gold_oracle_decompress(long N, int D, int Dc, const double *x0, const double
     free(cat);
     return 0;
 }
+
+/* Backward pass of Finch-C2's exact form (wkv6c2_one_head) for one (b,h) sequence, the
+ * adjoint written out as for the base form.  With kn_t = k_t (1 - w_t) the normalised key
+ * and G the gradient of the state after token t (dstate_out, or zero, at the end):
+ *   dv_t[j]   = sum_i G[i][j] kn_t[i]                    (no bonus in this form)
+ *   dkn[i]    = sum_j G[i][j] v_t[j];   dk_t[i] = dkn[i] (1 - w_t[i])
+ *   dr_t[i]   = sum_j Sall[t][i][j] dy_t[j]
+ *   dw_t[i]   = sum_j G[i][j] Sall[t][i][j] - dkn[i] k_t[i]    (kn depends on w too)
+ *   domega_t  = dw_t (-exp(omega_t) w_t)
+ *   duprime_t = dy_t                                      (u'_t is added to y_t)
+ *   G[i][j]   = w_t[i] G[i][j] + r_t[i] dy_t[j]
+ * and dstate_in = G at the start. */
+static void wkv6c2_one_head_backward(long T, int D, long tstride,
+                                     const double *r, const double *k, const double *v,
+                                     const double *omega, const double *s_in,
+                                     const double *dy, const double *ds_out,
+                                     double *dr, double *dk, double *dv, double *domega,
+                                     double *duprime, double *ds_in, double *Sall, double *G)
+{
+    const long DD = (long)D * D;
+    for (long e = 0; e < DD; ++e)
+        Sall[e] = s_in ? s_in[e] : 0.0;
+    for (long t = 0; t < T; ++t) {
+        const double *kt = k + t * tstride, *vt = v + t * tstride, *ot = omega + t * tstride;
+        const double *Sb = Sall + t * DD;
+        double *Sa = Sall + (t + 1) * DD;
+        for (int i = 0; i < D; ++i) {
+            const double wi = exp(-exp(ot[i]));
+            const double kni = kt[i] * (1.0 - wi);
+            for (int j = 0; j < D; ++j)
+                Sa[i * D + j] = wi * Sb[i * D + j] + kni * vt[j];
+        }
+    }
+
+    for (long e = 0; e < DD; ++e)
+        G[e] = ds_out ? ds_out[e] : 0.0;
+    for (long t = T - 1; t >= 0; --t) {
+        const double *rt = r + t * tstride, *kt = k + t * tstride, *vt = v + t * tstride;
+        const double *ot = omega + t * tstride, *dyt = dy + t * tstride;
+        const double *Sprev = Sall + t * DD;
+        double *drt = dr + t * tstride, *dkt = dk + t * tstride, *dvt = dv + t * tstride;
+        double *dot = domega + t * tstride, *dut = duprime + t * tstride;
+
+        for (int j = 0; j < D; ++j) {
+            double g = 0.0;
+            for (int i = 0; i < D; ++i)
+                g += G[i * D + j] * (kt[i] * (1.0 - exp(-exp(ot[i]))));
+            dvt[j] = g;
+            dut[j] = dyt[j];
+        }
+        for (int i = 0; i < D; ++i) {
+            const double wi = exp(-exp(ot[i]));
+            double gkn = 0.0, gr = 0.0, gw = 0.0;
+            for (int j = 0; j < D; ++j) {
+                gkn += G[i * D + j] * vt[j];
+                gr += dyt[j] * Sprev[i * D + j];
+                gw += Sprev[i * D + j] * G[i * D + j];
+            }
+            dkt[i] = gkn * (1.0 - wi);
+            drt[i] = gr;
+            dot[i] = (gw - gkn * kt[i]) * (-exp(ot[i]) * wi);
+        }
+        for (int i = 0; i < D; ++i) {
+            const double wi = exp(-exp(ot[i]));
+            for (int j = 0; j < D; ++j)
+                G[i * D + j] = G[i * D + j] * wi + rt[i] * dyt[j];
+        }
+    }
+    if (ds_in)
+        for (long e = 0; e < DD; ++e)
+            ds_in[e] = G[e];
+}
+
+/* Gradients of a loss L(y, state_out) with respect to every input of wkv6c2_oracle_prefill
+ * (r, k, v, omega, uprime, state_in), given dy and dstate_out (NULL: zero).  Outputs
+ * dr, dk, dv, domega, duprime [B][T][H][D]; dstate_in [B][H][D][D] (NULL: not written).
+ * Returns 0, -1 on bad arguments, -3 if memory for the kept states cannot be had. */
+int wkv6c2_oracle_backward(int B, long T, int H, int D,
+                           const double *r, const double *k, const double *v,
+                           const double *omega, const double *state_in,
+                           const double *dy, const double *dstate_out,
+                           double *dr, double *dk, double *dv, double *domega,
+                           double *duprime, double *dstate_in)
+{
+    if (B < 0 || T < 0 || H < 0 || D <= 0)
+        return -1;
+    if (B == 0 || H == 0)
+        return 0;
+    const long DD = (long)D * D;
+    double *Sall = (double *)malloc(sizeof(double) * (size_t)(T + 1) * (size_t)DD);
+    double *G = (double *)malloc(sizeof(double) * (size_t)DD);
+    if (!Sall || !G) {
+        free(Sall);
+        free(G);
+        return -3;
+    }
+    const long tstride = (long)H * D;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const size_t x0 = ((size_t)b * T * H + h) * D;
+            const size_t s0 = ((size_t)b * H + h) * DD;
+            wkv6c2_one_head_backward(T, D, tstride, r + x0, k + x0, v + x0, omega + x0,
+                                     state_in ? state_in + s0 : NULL, dy + x0,
+                                     dstate_out ? dstate_out + s0 : NULL, dr + x0, dk + x0,
+                                     dv + x0, domega + x0, duprime + x0,
+                                     dstate_in ? dstate_in + s0 : NULL, Sall, G);
+        }
+    free(Sall);
+    free(G);
+    return 0;
+}

@@ -55,6 +55,10 @@ v, omega, u and the initial state):
                       dlog w_t = <S_T, dS_T>_row + sum_{s>t} r_s dr_s' - sum_{s>=t} k_s dk_s'
                       (dr', dk' without their bonus parts): a relation between outputs;
 * bwd_empty         - T = 0: dS_0 = dS_T and every other gradient is zero.
+* c2_bwd_finite_diff- Finch-C2's backward against central differences through the C2
+                      forward entry point (inputs r, k, v, omega, u', S_0);
+* c2_bwd_autograd   - Finch-C2's backward against torch autograd through an independent
+                      torch statement of the C2 explicit sum.
 
 GOLD key compression and TokenCat decompression (section 3.4 "GOLD Key Compression and
 TokenCat Decompression"):
@@ -454,6 +458,77 @@ def pin_bwd_decay_identity(o):
     return _close(dom, dlog * (-np.exp(om)), rtol=1e-11)
 
 
+def pin_c2_bwd_finite_diff(o):
+    r, k, v, om, _, S0, dy, dS = _bwd_inputs(35, 2, 4, 1, 3)
+    up = _rng(36).normal(0, 0.5, r.shape)
+    got = o.backward_c2(r, k, v, om, S0, dy, dS)
+
+    def loss(*a):
+        y, S = o.prefill_c2(*a)
+        return float(np.sum(y * dy) + np.sum(S * dS))
+
+    base = [r, k, v, om, up, S0]       # got: dr, dk, dv, domega, du', dS0 -- this order
+    h = 1e-6
+    ok = True
+    for idx in range(6):
+        x = base[idx]
+        num = np.zeros_like(x)
+        for e in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[e] += h
+            xm[e] -= h
+            ap, am = list(base), list(base)
+            ap[idx], am[idx] = xp, xm
+            num[e] = (loss(*ap) - loss(*am)) / (2 * h)
+        ok &= _close(got[idx], num, rtol=1e-6)
+    return ok
+
+
+def _torch_c2_explicit(r, k, v, om, up, S0):
+    """Finch-C2: y_t = r_t . sum_{s<t} diag(prod w) (k_s (1 - w_s))^T v_s + decayed S0, plus
+    u'_t; final state likewise; products formed one by one (torch, differentiable)."""
+    B, T, H, D = r.shape
+    w = torch.exp(-torch.exp(om))
+    ys, finals = [], []
+    for b in range(B):
+        yb, fb = [], []
+        for h in range(H):
+            rows = []
+            for t in range(T + 1):
+                wkv = S0[b, h]
+                for j in range(t):
+                    wkv = w[b, j, h][:, None] * wkv
+                for i in range(t):
+                    dec = torch.ones(D, dtype=r.dtype)
+                    for j in range(i + 1, t):
+                        dec = dec * w[b, j, h]
+                    kn = k[b, i, h] * (1.0 - w[b, i, h])
+                    wkv = wkv + (dec * kn)[:, None] * v[b, i, h][None, :]
+                if t < T:
+                    rows.append(r[b, t, h] @ wkv + up[b, t, h])
+                else:
+                    fb.append(wkv)
+            yb.append(torch.stack(rows))
+        ys.append(torch.stack(yb, dim=1))
+        finals.append(torch.stack(fb))
+    return torch.stack(ys), torch.stack(finals)
+
+
+def pin_c2_bwd_autograd(o):
+    ok = True
+    for seed, (B, T, H, D) in [(37, (1, 5, 2, 4)), (38, (2, 3, 1, 5))]:
+        r, k, v, om, _, S0, dy, dS = _bwd_inputs(seed, B, T, H, D)
+        up = _rng(seed + 1).normal(0, 0.5, r.shape)
+        ts = [torch.tensor(a, dtype=torch.float64, requires_grad=True)
+              for a in (r, k, v, om, up, S0)]
+        y, S = _torch_c2_explicit(*ts)
+        (torch.sum(y * torch.tensor(dy)) + torch.sum(S * torch.tensor(dS))).backward()
+        got = o.backward_c2(r, k, v, om, S0, dy, dS)
+        for g_or, t in zip(got, ts):
+            ok &= _close(g_or, t.grad.numpy(), rtol=1e-10)
+    return ok
+
+
 def pin_bwd_empty(o):
     r, k, v, om, u, S0, dy, dS = _bwd_inputs(34, 2, 0, 3, 4)
     dr, dk, dv, dom, du, dS0 = o.backward(r, k, v, om, u, S0, dy, dS)
@@ -519,6 +594,8 @@ PINS = {
     "bwd_autograd": pin_bwd_autograd,
     "bwd_decay_identity": pin_bwd_decay_identity,
     "bwd_empty": pin_bwd_empty,
+    "c2_bwd_finite_diff": pin_c2_bwd_finite_diff,
+    "c2_bwd_autograd": pin_c2_bwd_autograd,
     "gold_compress_matmul": pin_gold_compress_matmul,
     "gold_decompress_blocks": pin_gold_decompress_blocks,
     "gold_rmsnorm_torch": pin_gold_rmsnorm_torch,

@@ -101,6 +101,24 @@ def test_gn_sequence_split(oracle, monkeypatch):
     assert rel_err(s, so) <= TOL[torch.bfloat16]
 
 
+def test_gn_full_layer_shape_sampled_heads(oracle):
+    """B8 T4096 H32 bf16 with the gate, as bench.py times it; three heads through the oracle
+    (the GroupNorm is local to a head, so a head's rows check on their own)."""
+    cfg = W.CONFIGS[1]
+    inp = _problem(cfg.seed, B=cfg.B, T=cfg.T, H=cfg.H)
+    y, s = _run(inp)
+    for b, h in ((0, 0), (3, 17), (7, 31)):
+        one = {n: inp[n][b:b + 1, :, h:h + 1] for n in ("r", "k", "v", "omega", "gate")}
+        a = [f64(one[n]) for n in ("r", "k", "v", "omega")]
+        hs = slice(64 * h, 64 * h + 64)
+        yo, so, _ = oracle.prefill_gn(*a, f64(inp["u"][h:h + 1]),
+                                      f64(inp["state0"][b:b + 1, h:h + 1]),
+                                      f64(inp["gamma"][hs]), f64(inp["beta"][hs]), GN_EPS,
+                                      f64(one["gate"]))
+        assert rel_err(y[b:b + 1, :, h:h + 1], yo) <= TOL[torch.bfloat16]
+        assert rel_err(s[b:b + 1, h:h + 1], so) <= TOL[torch.bfloat16]
+
+
 def test_gn_fp32_recurrence(oracle):
     inp = _problem(9550, B=2, T=150, H=2, dtype=torch.float32, cfg=0)
     y, s = _run(inp)

@@ -68,6 +68,12 @@ MUTANTS = {
                                   "G[i * D + j] = wi * G[i * D + j];"),
     "bwd_dv_transposed": ("g += G[i * D + j] * kt[i];", "g += G[j * D + i] * kt[i];"),
     "bwd_du_without_r": ("du_acc[i] += rt[i] * kt[i] * vdy;", "du_acc[i] += kt[i] * vdy;"),
+    # Finch-C2 backward
+    "c2bwd_dk_without_1mw": ("dkt[i] = gkn * (1.0 - wi);", "dkt[i] = gkn;"),
+    "c2bwd_domega_without_key_term": ("dot[i] = (gw - gkn * kt[i]) * (-exp(ot[i]) * wi);",
+                                      "dot[i] = gw * (-exp(ot[i]) * wi);"),
+    "c2bwd_dv_raw_key": ("g += G[i * D + j] * (kt[i] * (1.0 - exp(-exp(ot[i]))));",
+                         "g += G[i * D + j] * kt[i];"),
     # GOLD compression and TokenCat decompression
     "gold_compress_transposed": ("acc += x[n * D + i] * w_kd[(long)j * D + i];",
                                  "acc += x[n * D + i] * w_kd[(long)i * Dc + j];"),
