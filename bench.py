@@ -285,20 +285,25 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False, gn=False):
     return line
 
 
-def backward_line(cfg, dev, world, steps):
-    """Device-timed wkv6_backward on the prefill workload's shape (bf16 I/O): gradients of
-    r, k, v, omega, u and the initial state for a random dy and final-state gradient."""
+def backward_line(cfg, dev, world, steps, c2=False):
+    """Device-timed wkv6_backward (or, c2, wkv6c2_backward) on the prefill workload's shape
+    (bf16 I/O): gradients of every input for a random dy and final-state gradient."""
     import linear_attention_rnn_finch_b200 as gw
     inp = W.make_prefill_inputs(cfg, dev)
     g = torch.Generator(device=dev).manual_seed(cfg.seed + 7)
     dy = torch.randn(inp["r"].shape, generator=g, device=dev).to(cfg.dtype)
     dS = torch.randn(inp["state0"].shape, generator=g, device=dev) * 0.1
     B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
-    ws = torch.empty(gw.backward_workspace_bytes(B, T, H, D, cfg.dtype), dtype=torch.uint8,
-                     device=dev)
-    args_b = [inp[n] for n in ("r", "k", "v", "omega", "u", "state0")]
+    L = gw.load()
+    nbytes_ws = (L.wkv6c2_backward_workspace_bytes if c2 else L.wkv6_backward_workspace_bytes)(
+        B, T, H, D, 1)
+    ws = torch.empty(nbytes_ws, dtype=torch.uint8, device=dev)
+    names = ("r", "k", "v", "omega", "state0") if c2 else ("r", "k", "v", "omega", "u", "state0")
+    args_b = [inp[n] for n in names]
 
     def call():
+        if c2:
+            return gw.wkv6c2_backward(*args_b, dy, dS, workspace=ws)
         return gw.wkv6_backward(*args_b, dy, dS, workspace=ws)
 
     for _ in range(3):
@@ -315,9 +320,10 @@ def backward_line(cfg, dev, world, steps):
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
     flops, nbytes = backward_flops(B, T, H, D), backward_bytes(B, T, H, D)
     # dr scan, dk scan, du sum; 2 reversals + fast + level kernels for dv (+ 2 segment
-    # kernels when the sequence is split)
-    launches_per_call = 3 + 4
-    line = {"workload": "wkv6_backward_1p5b_layer", "B": B, "T": T, "H": H, "D": D, "io": "bf16",
+    # kernels when the sequence is split).  Finch-C2: the dr + dv scan launch and the dk scan
+    launches_per_call = 2 if c2 else 3 + 4
+    line = {"workload": "wkv6c2_backward_1p5b_layer" if c2 else "wkv6_backward_1p5b_layer",
+            "B": B, "T": T, "H": H, "D": D, "io": "bf16",
             "steps": steps, "ms_per_call": ms, "tokens_per_s": world * B * T / (ms / 1e3),
             "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
                          "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
@@ -326,12 +332,14 @@ def backward_line(cfg, dev, world, steps):
                          "algorithmic_flops_per_call": flops},
             "hbm": {"achieved_gbs": nbytes / (ms / 1e3) / 1e9, "algorithmic_bytes_per_call": nbytes},
             "gpu_launches": launches_per_call * steps,
-            "kernels": "dr scan (wkv6_bwd_dr_dv_kernel), dk + decay-gradient scan "
-                       "(wkv6_bwd_dk_domega_kernel), du sum; dv through the chunked tensor-core "
-                       "prefill on time-reversed copies (reverse_tokens_kernel x2, "
-                       "wkv6_fast_kernel, wkv6_chunked_kernel)",
+            "kernels": ("dr and dv scans (wkv6_bwd_dr_dv_kernel), dk + decay-gradient scan "
+                        "(wkv6_bwd_dk_domega_kernel), all on CUDA cores") if c2 else
+                       ("dr scan (wkv6_bwd_dr_dv_kernel), dk + decay-gradient scan "
+                        "(wkv6_bwd_dk_domega_kernel), du sum; dv through the chunked tensor-core "
+                        "prefill on time-reversed copies (reverse_tokens_kernel x2, "
+                        "wkv6_fast_kernel, wkv6_chunked_kernel)"),
             "note": "algorithmic FLOPs are the three recurrences (dr, dk, dv) at 5 FLOPs per "
-                    "state entry per token; dv runs on the tensor cores"}
+                    "state entry per token" + ("" if c2 else "; dv runs on the tensor cores")}
     del inp, dy, dS, ws, args_b
     torch.cuda.empty_cache()
     return line
@@ -566,6 +574,7 @@ def run_ours(args, world, rank, local):
                                 other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
                                               gn=True)]
         out["backward"] = backward_line(W.CONFIGS[1], dev, world, steps=5)
+        out["backward_c2"] = backward_line(W.CONFIGS[1], dev, world, steps=5, c2=True)
         out["gold"] = gold_line(dev, world, steps=10)
 
     # end to end through the public API with host buffers: every step copies its inputs in
@@ -703,7 +712,7 @@ def main():
                     help="skip the ~1 s untimed warm-up loop (for profiler runs)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the prefill batch size (smaller profiler captures)")
-    ap.add_argument("--only", choices=["backward", "gold"], default=None,
+    ap.add_argument("--only", choices=["backward", "backward_c2", "gold"], default=None,
                     help="print only that line (wkv6_backward, or GOLD compression + "
                          "decompression, on the 1.5B-layer shape; --batch and --seq-len "
                          "override B and T), for profiler runs")
@@ -729,8 +738,10 @@ def main():
             cfg = PREFILL_CFG.with_(**{k: v for k, v in (("B", args.batch), ("T", args.seq_len))
                                        if v is not None})
             dev = torch.device("cuda", local)
-            out = (backward_line(cfg, dev, world, steps=args.steps) if args.only == "backward"
-                   else gold_line(dev, world, steps=args.steps, B=cfg.B, T=cfg.T))
+            out = (gold_line(dev, world, steps=args.steps, B=cfg.B, T=cfg.T)
+                   if args.only == "gold" else
+                   backward_line(cfg, dev, world, steps=args.steps,
+                                 c2=args.only == "backward_c2"))
         else:
             out = run_ours(args, world, rank, local)
         if rank == 0 and out is not None:

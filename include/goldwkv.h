@@ -245,6 +245,27 @@ wkv_status wkv6_backward(const void *r, const void *k, const void *v, const void
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Backward pass of Finch-C2's exact form (wkv6c2_prefill without LayerNorm): gradients of a
+ * loss with respect to r, k, v, omega, u' and state_in, given dy and (optionally)
+ * dstate_out.  With kn_t = k_t (1 - w_t) and G as for wkv6_backward:
+ *     dr_t = S_{t-1} dy_t;   dkn = G v_t, dk_t = dkn (1 - w_t);   dv_t = G^T kn_t;
+ *     domega_t = (sum_j G[i][j] S_{t-1}[i][j] - dkn k_t) w_t (-exp(omega_t));   du'_t = dy_t
+ * (no bonus; u' enters y additively).  All three are token-by-token scans on CUDA cores
+ * (fp32, fp64 row scans with fp32 I/O); the decay gradient goes through the pair identity
+ * with the normalised keys.
+ *   duprime  [B][T][H][D] io: output (a copy of dy), or NULL (not written).
+ * Other arguments, layouts and errors as wkv6_backward; workspace: at least
+ * wkv6c2_backward_workspace_bytes(...) bytes.
+ */
+size_t wkv6c2_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io);
+
+wkv_status wkv6c2_backward(const void *r, const void *k, const void *v, const void *omega,
+                           const float *state_in, const void *dy, const float *dstate_out,
+                           void *dr, void *dk, void *dv, void *domega, void *duprime,
+                           float *dstate_in, int B, int T, int H, int D, wkv_dtype io,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * GOLD key compression and TokenCat decompression (GoldFinch review page, section 3.4
  * "GOLD Key Compression and TokenCat Decompression"): the output x_t of the last Finch-C2
  * layer is compressed by one global matrix W_KD (D x Dc, Dc = D/16 in the page's model)

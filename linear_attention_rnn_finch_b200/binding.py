@@ -75,6 +75,10 @@ def load(path: Path | str | None = None):
     L.wkv6_backward_workspace_bytes.restype = sz
     L.wkv6_backward.argtypes = [vp] * 14 + [i, i, i, i, i, vp, sz, vp]
     L.wkv6_backward.restype = i
+    L.wkv6c2_backward_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.wkv6c2_backward_workspace_bytes.restype = sz
+    L.wkv6c2_backward.argtypes = [vp] * 13 + [i, i, i, i, i, vp, sz, vp]
+    L.wkv6c2_backward.restype = i
     L.gold_compress_workspace_bytes.argtypes = [ctypes.c_long, i, i]
     L.gold_compress_workspace_bytes.restype = sz
     L.gold_decompress_workspace_bytes.argtypes = [ctypes.c_long, i, i]
@@ -513,3 +517,36 @@ def gold_decompress(x0, c, w_ku, gamma=None, eps=1e-6, *, kd=None, workspace=Non
                                N, D, Dc, _ptr(workspace), ws_bytes, _stream_ptr(dev, stream))
     _raise("gold_decompress", st)
     return kd
+
+
+def wkv6c2_backward(r, k, v, omega, state_in, dy, dstate_out=None, *, want_dstate_in=True,
+                    want_duprime=True, workspace=None, stream=None):
+    """Gradients of wkv6c2_prefill (no LayerNorm) for dy [B, T, H, D] and dstate_out
+    [B, H, D, D] fp32 (None: zero).  Returns (dr, dk, dv, domega, duprime or None,
+    dstate_in or None)."""
+    L = load()
+    if r.dim() != 4:
+        raise ValueError("r must be [B, T, H, D]")
+    B, T, H, D = r.shape
+    dev, dt = r.device, r.dtype
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("r", r), ("k", k), ("v", v), ("omega", omega), ("dy", dy)):
+        _check(name, t, dev, dt, (B, T, H, D))
+    for name, t in (("state_in", state_in), ("dstate_out", dstate_out)):
+        if t is not None:
+            _check(name, t, dev, torch.float32, (B, H, D, D))
+    dr, dk, dv, dom = (torch.empty((B, T, H, D), dtype=dt, device=dev) for _ in range(4))
+    dup = torch.empty((B, T, H, D), dtype=dt, device=dev) if want_duprime else None
+    ds_in = torch.empty((B, H, D, D), dtype=torch.float32, device=dev) if want_dstate_in else None
+    need = int(L.wkv6c2_backward_workspace_bytes(B, T, H, D, _io(dt)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6c2_backward(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(state_in), _ptr(dy),
+                               _ptr(dstate_out), _ptr(dr), _ptr(dk), _ptr(dv), _ptr(dom),
+                               _ptr(dup), _ptr(ds_in), B, T, H, D, _io(dt), _ptr(workspace),
+                               ws_bytes, _stream_ptr(dev, stream))
+    _raise("wkv6c2_backward", st)
+    return dr, dk, dv, dom, dup, ds_in

@@ -510,22 +510,30 @@ wkv_status wkv6_decode_step_gn(const void* r, const void* k, const void* v, cons
 }
 
 
-size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
+}  // extern "C"
+
+namespace {
+
+// Workspace of the backward: P and E in the row scans' accumulation type (fp64 for fp32
+// I/O, fp32 for bf16 I/O) and the per-(b,h) du parts; with tc_dv, also the time-reversed
+// k, r, dy, omega and dv and the chunked prefill's own workspace.
+size_t backward_bytes(int B, int T, int H, int D, wkv_dtype io, bool tc_dv) {
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
-    // P and E in the row scans' accumulation type: fp64 for fp32 I/O, fp32 for bf16 I/O
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     const size_t x = (size_t)B * T * H * D, bh = (size_t)B * H * D;
     size_t bytes = round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
-    // bf16: time-reversed k, r, dy, omega and dv, and the chunked prefill's own workspace
-    if (io == WKV_BF16) bytes += 5 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H));
+    if (tc_dv) bytes += 5 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H));
     return bytes;
 }
 
-wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void* omega,
+// Shared by the base (static bonus u; du out) and the Finch-C2 (key k (1 - w), second
+// value; du' = dy out) backward entry points.
+wkv_status backward_impl(const void* r, const void* k, const void* v, const void* omega,
                          const float* u, const float* state_in, const void* dy,
                          const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
-                         float* du, float* dstate_in, int B, int T, int H, int D, wkv_dtype io,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+                         float* du, void* duprime, float* dstate_in, int B, int T, int H, int D,
+                         wkv_dtype io, bool c2, void* workspace, size_t workspace_bytes,
+                         void* stream) {
     if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
     if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
     if (H == 0) return WKV_OK;
@@ -535,21 +543,22 @@ wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void
     const size_t ubytes = (size_t)H * D * sizeof(float);
     const bool tokens = B > 0 && T > 0;
     Buf bufs[] = {{r, xbytes, tokens},      {k, xbytes, tokens},         {v, xbytes, tokens},
-                  {omega, xbytes, tokens},  {dy, xbytes, tokens},        {u, ubytes, tokens},
+                  {omega, xbytes, tokens},  {dy, xbytes, tokens},        {u, ubytes, tokens && !c2},
                   {dr, xbytes, tokens},     {dk, xbytes, tokens},        {dv, xbytes, tokens},
-                  {domega, xbytes, tokens}, {du, ubytes, true},          {state_in, sbytes, false},
+                  {domega, xbytes, tokens}, {du, ubytes, !c2},           {state_in, sbytes, false},
                   {dstate_out, sbytes, false}, {dstate_in, sbytes, false},
-                  {workspace, workspace_bytes, false}};
+                  {workspace, workspace_bytes, false}, {duprime, xbytes, false}};
     wkv_status s = check_bufs(bufs, (int)(sizeof(bufs) / sizeof(bufs[0])));
     if (s != WKV_OK) return s;
 
     // no output may overlap an input, another output or the workspace
     const size_t xb = tokens ? xbytes : 0, sb = B > 0 ? sbytes : 0;
     const Span ins[] = {span(r, xb), span(k, xb), span(v, xb), span(omega, xb), span(dy, xb),
-                        span(u, tokens ? ubytes : 0), span(state_in, state_in ? sb : 0),
-                        span(dstate_out, dstate_out ? sb : 0)};
+                        span(c2 ? nullptr : u, tokens && !c2 ? ubytes : 0),
+                        span(state_in, state_in ? sb : 0), span(dstate_out, dstate_out ? sb : 0)};
     const Span outs[] = {span(dr, xb), span(dk, xb), span(dv, xb), span(domega, xb),
-                         span(du, ubytes), span(dstate_in, dstate_in ? sb : 0)};
+                         span(c2 ? nullptr : du, c2 ? 0 : ubytes),
+                         span(dstate_in, dstate_in ? sb : 0), span(duprime, duprime ? xb : 0)};
     const int n_outs = (int)(sizeof(outs) / sizeof(outs[0]));
     for (int a = 0; a < n_outs; ++a) {
         for (const Span& in : ins)
@@ -557,7 +566,9 @@ wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void
         for (int b2 = a + 1; b2 < n_outs; ++b2)
             if (overlaps(outs[a], outs[b2])) return WKV_ERR_INVALID_ARG;
     }
-    const size_t need = wkv6_backward_workspace_bytes(B, T, H, D, io);
+    const bool bf16 = io == WKV_BF16;
+    const bool tc_dv = bf16 && !c2;   // dv through the chunked tensor-core prefill
+    const size_t need = backward_bytes(B, T, H, D, io, tc_dv);
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
         const Span sw = span(workspace, need);
@@ -569,20 +580,22 @@ wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void
     if (injected("launch")) return WKV_ERR_CUDA;
 
     if (!tokens) {   // no token: du = 0, and the state gradient passes through unchanged
-        if (cudaMemsetAsync(du, 0, ubytes, st) != cudaSuccess) return WKV_ERR_CUDA;
+        if (!c2 && cudaMemsetAsync(du, 0, ubytes, st) != cudaSuccess) return WKV_ERR_CUDA;
         if (dstate_in == nullptr || B == 0) return WKV_OK;
         if (dstate_out) return from_cuda(cudaMemcpyAsync(dstate_in, dstate_out, sbytes,
                                                          cudaMemcpyDeviceToDevice, st));
         return from_cuda(cudaMemsetAsync(dstate_in, 0, sbytes, st));
     }
+    if (c2 && duprime &&   // u'_t is added to y_t as it is: its gradient is dy_t
+        cudaMemcpyAsync(duprime, dy, xbytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return WKV_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     void* P = ws;
     uint8_t* E = ws + round256((size_t)B * T * H * D * acc);
     uint8_t* dpart = E + round256((size_t)B * H * D * acc);
     float* du_part = reinterpret_cast<float*>(dpart);
-    const bool bf16 = io == WKV_BF16;
-    if (bf16) {
+    if (tc_dv) {
         // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
         // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.
         // It runs through the chunked tensor-core prefill on time-reversed copies.
@@ -609,11 +622,43 @@ wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void
         if (goldwkv::launch_reverse_tokens(src_dv, dst_dv, 1, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
-    return from_cuda(goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr,
-                                              dk, dv, domega, du, dstate_in, P, E, du_part, B,
-                                              T, H, bf16, /*with_dv=*/!bf16, st));
+    return from_cuda(goldwkv::launch_backward(r, k, v, omega, c2 ? nullptr : u, state_in, dy,
+                                              dstate_out, dr, dk, dv, domega, du, dstate_in, P,
+                                              E, du_part, B, T, H, bf16, /*with_dv=*/!tc_dv, c2,
+                                              st));
 }
 
+}  // namespace
+
+extern "C" {
+
+size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
+    return backward_bytes(B, T, H, D, io, io == WKV_BF16);
+}
+
+size_t wkv6c2_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
+    return backward_bytes(B, T, H, D, io, false);
+}
+
+wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void* omega,
+                         const float* u, const float* state_in, const void* dy,
+                         const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
+                         float* du, float* dstate_in, int B, int T, int H, int D, wkv_dtype io,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    return backward_impl(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv, domega, du,
+                         nullptr, dstate_in, B, T, H, D, io, false, workspace, workspace_bytes,
+                         stream);
+}
+
+wkv_status wkv6c2_backward(const void* r, const void* k, const void* v, const void* omega,
+                           const float* state_in, const void* dy, const float* dstate_out,
+                           void* dr, void* dk, void* dv, void* domega, void* duprime,
+                           float* dstate_in, int B, int T, int H, int D, wkv_dtype io,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    return backward_impl(r, k, v, omega, nullptr, state_in, dy, dstate_out, dr, dk, dv, domega,
+                         nullptr, duprime, dstate_in, B, T, H, D, io, true, workspace,
+                         workspace_bytes, stream);
+}
 
 }  // extern "C"
 

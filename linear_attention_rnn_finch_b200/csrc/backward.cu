@@ -32,6 +32,12 @@
 // xor-shuffles across the four q-threads of a row.  Tokens are staged through shared memory
 // in tiles of kTile; per-token outputs are staged too and written coalesced per tile.
 //
+// Finch-C2's exact form (kC2): the key enters the state as kn_t = k_t (1 - w_t) and there
+// is no bonus, so the dr and dv scans use kn in place of k (formed while staging), the dk
+// scan yields dkn and returns dk = dkn (1 - w) with Q_t = kn_t dkn_t, and the decay gradient
+// gains the direct term of kn on w: domega += dkn k w exp(omega).  du' = dy is the caller's
+// copy.  dv stays a CUDA-core scan in this form (the chunked prefill would need kn in bf16).
+//
 // Precision.  The identity subtracts, at every token, the pair terms that start at or after
 // it; where w_t is tiny the result is tiny too and what is left is the rounding of those
 // terms, times exp(omega_t).  With bf16 I/O that residue is far below the output rounding,
@@ -180,7 +186,7 @@ __device__ __forceinline__ void reduce16x4(Acc (&v)[4], int lane) {
 // vectors (its 4 columns) and of the rows' a and w, the row sums finished over the 16 lanes
 // of a half-warp by a reduce-scatter (5 shuffles for 4 rows).  Lane c % 4 == 0 of each
 // group of four then owns row e = c / 4 (its outputs and running sums).
-template <typename IO, bool kRev, typename Acc = typename Prec<IO>::Acc,
+template <typename IO, bool kRev, bool kC2, typename Acc = typename Prec<IO>::Acc,
           int kTile = Prec<IO>::kTile>
 __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __restrict__ a_src,
                                           const IO* __restrict__ m_src,
@@ -203,7 +209,7 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
     const bool owner = (c & 3) == 0;                      // reduce16x4; one writer per row
     const int rl_own = 4 * g + er;                        // its local row 0..31
 
-    if (tid < kHalf) s.u[tid] = u[h * D + rowbase + tid];
+    if (tid < kHalf) s.u[tid] = kC2 ? 0.f : u[h * D + rowbase + tid];
 
     // X[e][f]: entry (rowbase + 4g + e, 4c + f)
     const size_t sbase = (size_t)bh * D * D + (size_t)(rowbase + 4 * g) * D + 4 * c;
@@ -262,16 +268,18 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
 #pragma unroll
         for (int k = 0; k < kRows; ++k) {
             constexpr int n = ChunkOf<IO>::n;
-            put_chunk<IO>(ra[k], &s.a[0][0], tid + k * kThreads);
             put_chunk<IO>(rm[k], &s.m[0][0], tid + k * kThreads);
-            float om[n], ne[n], w[n];
+            float om[n], ne[n], w[n], av[n];
             unpack(ro[k], om);
+            unpack(ra[k], av);
 #pragma unroll
             for (int j = 0; j < n; ++j) {   // (padding tokens past T are never read)
                 ne[j] = -expf(om[j]);
                 w[j] = expf(ne[j]);
+                if (kC2 && !kRev) av[j] *= -expm1f(ne[j]);   // the dr scan's kn = k (1 - w)
             }
             const int e0 = (tid + k * kThreads) * n;
+            store_f32(&s.a[0][0] + e0, av);
             store_f32(&s.ne[0][0] + e0, ne);
             store_f32(&s.w[0][0] + e0, w);
         }
@@ -310,15 +318,27 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
             if (owner) {
                 const Acc acc = part[0];
                 const Acc vdy = s.vdy[tt], mi = s.m[tt][rl_own], ai = s.a[tt][rl_own];
-                const Acc bonus = (Acc)s.u[rl_own] * ai * vdy;
-                s.o1[tt][rl_own] = (float)(acc + bonus);
-                if (!kRev) {
-                    s.o2[tt][rl_own] = mi * acc;          // P_t: pair terms ending at t
-                    du_acc += mi * ai * vdy;
-                } else {
-                    accQ += mi * acc;                     // Q_t: pair terms starting at t
-                    s.o2[tt][rl_own] = (Ei + accP - accQ) * (Acc)s.ne[tt][rl_own];
+                if (kC2 && kRev) {
+                    // acc = dkn; m = k: kn = k (1 - w), dk = dkn (1 - w), and kn's own
+                    // dependence on w adds -dkn k w to the gradient of w (before the chain
+                    // factor d w / d omega = w ne)
+                    const float ne = s.ne[tt][rl_own];
+                    const Acc omw = (Acc)(-expm1f(ne)), wv = s.w[tt][rl_own];
+                    s.o1[tt][rl_own] = (float)(acc * omw);
+                    accQ += mi * omw * acc;               // Q_t with the source value kn_t
+                    s.o2[tt][rl_own] = (Ei + accP - accQ - acc * mi * wv) * (Acc)ne;
                     accP += s.p[tt][rl_own];
+                } else {
+                    const Acc bonus = (Acc)s.u[rl_own] * ai * vdy;
+                    s.o1[tt][rl_own] = (float)(acc + bonus);
+                    if (!kRev) {
+                        s.o2[tt][rl_own] = mi * acc;      // P_t: pair terms ending at t
+                        du_acc += mi * ai * vdy;
+                    } else {
+                        accQ += mi * acc;                 // Q_t: pair terms starting at t
+                        s.o2[tt][rl_own] = (Ei + accP - accQ) * (Acc)s.ne[tt][rl_own];
+                        accP += s.p[tt][rl_own];
+                    }
                 }
             }
         }
@@ -354,7 +374,7 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
 }
 
 // The dv sweep: columns of G, reverse in time (the forward recurrence with r <-> k, v -> dy).
-template <typename IO, int kTile = Prec<IO>::kTile>
+template <typename IO, bool kC2, int kTile = Prec<IO>::kTile>
 __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restrict__ r,
                                           const IO* __restrict__ k, const IO* __restrict__ omega,
                                           const IO* __restrict__ dy, const float* __restrict__ u,
@@ -369,7 +389,7 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
     const int colbase = blockIdx.y * kHalf;
     const int j = colbase + jl;
 
-    if (tid < D) s.u[tid] = u[h * D + tid];
+    if (tid < D) s.u[tid] = kC2 ? 0.f : u[h * D + tid];
 
     // G[4*m4 + e] is entry (row 16*m4 + 4*qq + e, column j): rows interleave in blocks of 4
     // across the four threads of a column (bank-conflict-free 16-byte reads)
@@ -411,12 +431,16 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
         for (int c = 0; c < kFull; ++c) {
             constexpr int n = ChunkOf<IO>::n;
             put_chunk<IO>(rr[c], &s.r[0][0], tid + c * kThreads);
-            put_chunk<IO>(rk[c], &s.k[0][0], tid + c * kThreads);
-            float om[n], w[n];
+            float om[n], w[n], kv[n];
             unpack(ro[c], om);
+            unpack(rk[c], kv);
 #pragma unroll
-            for (int j = 0; j < n; ++j) w[j] = decay_from_logit(om[j]);
+            for (int j = 0; j < n; ++j) {
+                w[j] = decay_from_logit(om[j]);
+                if (kC2) kv[j] *= -expm1f(-expf(om[j]));   // kn = k (1 - w)
+            }
             store_f32(&s.w[0][0] + (tid + c * kThreads) * n, w);
+            store_f32(&s.k[0][0] + (tid + c * kThreads) * n, kv);
         }
 #pragma unroll
         for (int c = 0; c < kCols; ++c) put_chunk<IO>(rd[c], &s.dy[0][0], tid + c * kThreads);
@@ -469,7 +493,7 @@ struct SweepSmem {
 };
 
 // blockIdx.z == 0: dr sweep; blockIdx.z == 1: dv sweep.
-template <typename IO>
+template <typename IO, bool kC2>
 __global__ void __launch_bounds__(kThreads, 4)   // 4 CTAs (16 warps) per SM
 wkv6_bwd_dr_dv_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                       const IO* __restrict__ v, const IO* __restrict__ omega,
@@ -480,14 +504,14 @@ wkv6_bwd_dr_dv_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
     using Sm = SweepSmem<IO>;
     __shared__ __align__(16) unsigned char smem[Sm::kBytes];
     if (blockIdx.z == 0)
-        row_sweep<IO, false>(*reinterpret_cast<typename Sm::Row*>(smem), k, r, v, dy, omega, u,
+        row_sweep<IO, false, kC2>(*reinterpret_cast<typename Sm::Row*>(smem), k, r, v, dy, omega, u,
                              state_in, dr, P, nullptr, E, dS_T, du_part, nullptr, T, H);
     else
-        col_sweep<IO>(*reinterpret_cast<typename Sm::Col*>(smem), r, k, omega, dy, u, dS_T, dv,
+        col_sweep<IO, kC2>(*reinterpret_cast<typename Sm::Col*>(smem), r, k, omega, dy, u, dS_T, dv,
                       T, H);
 }
 
-template <typename IO>
+template <typename IO, bool kC2>
 __global__ void __launch_bounds__(kThreads, 4)   // 4 CTAs (16 warps) per SM
 wkv6_bwd_dk_domega_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                           const IO* __restrict__ v, const IO* __restrict__ omega,
@@ -496,7 +520,7 @@ wkv6_bwd_dk_domega_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                           IO* __restrict__ domega, typename Prec<IO>::Acc* __restrict__ P,
                           typename Prec<IO>::Acc* __restrict__ E, float* dS_0, int T, int H) {
     __shared__ __align__(16) typename SweepSmem<IO>::Row s;
-    row_sweep<IO, true>(s, r, k, dy, v, omega, u, dS_T, dk, P, domega, E, nullptr, nullptr, dS_0,
+    row_sweep<IO, true, kC2>(s, r, k, dy, v, omega, u, dS_T, dk, P, domega, E, nullptr, nullptr, dS_0,
                         T, H);
 }
 
@@ -528,7 +552,7 @@ __global__ void wkv6_bwd_du_kernel(const float* __restrict__ du_part, float* __r
     du[(size_t)h * kHeadSize + i] = acc;
 }
 
-template <typename IO>
+template <typename IO, bool kC2>
 cudaError_t launch_typed(const void* r, const void* k, const void* v, const void* omega,
                          const float* u, const float* state_in, const void* dy,
                          const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
@@ -539,13 +563,14 @@ cudaError_t launch_typed(const void* r, const void* k, const void* v, const void
              *dy_ = (const IO*)dy;
     Acc *P = static_cast<Acc*>(P_), *E = static_cast<Acc*>(E_);
     const unsigned bh = (unsigned)(B * H);
-    wkv6_bwd_dr_dv_kernel<IO><<<dim3(bh, kHeadSize / kHalf, with_dv ? 2 : 1), kThreads, 0, st>>>(
+    wkv6_bwd_dr_dv_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf, with_dv ? 2 : 1), kThreads, 0, st>>>(
         r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_dk_domega_kernel<IO><<<dim3(bh, kHeadSize / kHalf), kThreads, 0, st>>>(
+    wkv6_bwd_dk_domega_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf), kThreads, 0, st>>>(
         r_, k_, v_, o_, u, dy_, dstate_out, (IO*)dk, (IO*)domega, P, E, dstate_in, T, H);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (kC2) return cudaSuccess;   // no bonus u in this form
     wkv6_bwd_du_kernel<<<H, kHeadSize, 0, st>>>(du_part, du, B, H);
     return cudaGetLastError();
 }
@@ -556,13 +581,22 @@ cudaError_t launch_backward(const void* r, const void* k, const void* v, const v
                             const float* u, const float* state_in, const void* dy,
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
-                            int B, int T, int H, bool bf16, bool with_dv, cudaStream_t st) {
-    if (bf16)
-        return launch_typed<__nv_bfloat16>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
-                                           dv, domega, du, dstate_in, P, E, du_part, B, T, H,
-                                           with_dv, st);
-    return launch_typed<float>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv, domega,
-                               du, dstate_in, P, E, du_part, B, T, H, with_dv, st);
+                            int B, int T, int H, bool bf16, bool with_dv, bool c2,
+                            cudaStream_t st) {
+    using BF = __nv_bfloat16;
+    if (c2)
+        return bf16 ? launch_typed<BF, true>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
+                                            dv, domega, du, dstate_in, P, E, du_part, B, T, H,
+                                            with_dv, st)
+                    : launch_typed<float, true>(r, k, v, omega, u, state_in, dy, dstate_out, dr,
+                                                dk, dv, domega, du, dstate_in, P, E, du_part, B,
+                                                T, H, with_dv, st);
+    return bf16 ? launch_typed<BF, false>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv,
+                                          domega, du, dstate_in, P, E, du_part, B, T, H, with_dv,
+                                          st)
+                : launch_typed<float, false>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
+                                             dv, domega, du, dstate_in, P, E, du_part, B, T, H,
+                                             with_dv, st);
 }
 
 cudaError_t launch_reverse_tokens(const void* const* src, void* const* dst, int n, int B, int T,

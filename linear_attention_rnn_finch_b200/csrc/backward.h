@@ -10,11 +10,13 @@ namespace goldwkv {
 // accumulation type (fp64 for fp32 I/O, fp32 for bf16 I/O), du_part [B*H][64] fp32.
 // dstate_out / state_in may be null (zero); dstate_in may be null (not written).
 // with_dv == false: dv is computed elsewhere (the caller's tensor-core path); dv unused.
+// c2: Finch-C2's exact form (key k (1 - w), no bonus; u and du unused).
 cudaError_t launch_backward(const void* r, const void* k, const void* v, const void* omega,
                             const float* u, const float* state_in, const void* dy,
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
-                            int B, int T, int H, bool bf16, bool with_dv, cudaStream_t st);
+                            int B, int T, int H, bool bf16, bool with_dv, bool c2,
+                            cudaStream_t st);
 
 constexpr int kMaxReverse = 4;
 
