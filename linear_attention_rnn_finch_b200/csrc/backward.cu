@@ -374,6 +374,10 @@ __device__ __forceinline__ void row_sweep(RowSmem<Acc, kTile>& s, const IO* __re
 }
 
 // The dv sweep: columns of G, reverse in time (the forward recurrence with r <-> k, v -> dy).
+// Thread (g, c) = (tid / 16, tid % 16) keeps the 4 x 4 block of rows 4c..4c+3 and columns
+// 4g..4g+3 (of the CTA's 32): per token one 16-byte read each of its rows' k, r and w and of
+// its columns' dy; the column sums finish over the 16 lanes of a half-warp (reduce16x4),
+// and lane c % 4 == 0 of each group of four owns column f = c / 4.
 template <typename IO, bool kC2, int kTile = Prec<IO>::kTile>
 __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restrict__ r,
                                           const IO* __restrict__ k, const IO* __restrict__ omega,
@@ -384,22 +388,21 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh - (bh / H) * H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int qq = lane & 3;                    // row quarter: rows 16qq .. 16qq+15
-    const int jl = warp * 8 + (lane >> 2);      // local column 0..31
+    const int g = tid >> 4, c = tid & 15;
     const int colbase = blockIdx.y * kHalf;
-    const int j = colbase + jl;
+    const int fr = 2 * ((c >> 3) & 1) + ((c >> 2) & 1);   // column (of 4) this lane owns
+    const bool owner = (c & 3) == 0;
+    const int jl_own = 4 * g + fr;                        // its local column 0..31
 
     if (tid < D) s.u[tid] = kC2 ? 0.f : u[h * D + tid];
 
-    // G[4*m4 + e] is entry (row 16*m4 + 4*qq + e, column j): rows interleave in blocks of 4
-    // across the four threads of a column (bank-conflict-free 16-byte reads)
-    const size_t sbase = (size_t)bh * D * D;
-    float G[16];
+    // G[e][f]: entry (row 4c + e, column colbase + 4g + f)
+    const size_t sbase = (size_t)bh * D * D + (size_t)(4 * c) * D + colbase + 4 * g;
+    float G[4][4];
 #pragma unroll
-    for (int m4 = 0; m4 < 4; ++m4)
+    for (int e = 0; e < 4; ++e)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            G[4 * m4 + e] = dS_T ? dS_T[sbase + (size_t)(16 * m4 + 4 * qq + e) * D + j] : 0.f;
+        for (int f = 0; f < 4; ++f) G[e][f] = dS_T ? dS_T[sbase + (size_t)e * D + f] : 0.f;
 
     const size_t tstride = (size_t)H * D;
     const size_t xbase = ((size_t)b * T * H + h) * D;
@@ -413,14 +416,14 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
     auto fetch = [&](int it) {   // chunks of tile `it` (reverse order) into registers
         const int t0 = (ntile - 1 - it) * kTile, nt = min(kTile, T - t0);
 #pragma unroll
-        for (int c = 0; c < kFull; ++c) {
-            rr[c] = load_chunk(r, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
-            rk[c] = load_chunk(k, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
-            ro[c] = load_chunk(omega, xbase, tstride, t0, nt, 0, D, tid + c * kThreads);
+        for (int x = 0; x < kFull; ++x) {
+            rr[x] = load_chunk(r, xbase, tstride, t0, nt, 0, D, tid + x * kThreads);
+            rk[x] = load_chunk(k, xbase, tstride, t0, nt, 0, D, tid + x * kThreads);
+            ro[x] = load_chunk(omega, xbase, tstride, t0, nt, 0, D, tid + x * kThreads);
         }
 #pragma unroll
-        for (int c = 0; c < kCols; ++c)
-            rd[c] = load_chunk(dy, xbase, tstride, t0, nt, colbase, kHalf, tid + c * kThreads);
+        for (int x = 0; x < kCols; ++x)
+            rd[x] = load_chunk(dy, xbase, tstride, t0, nt, colbase, kHalf, tid + x * kThreads);
     };
     if (ntile > 0) fetch(0);
     for (int it = 0; it < ntile; ++it) {
@@ -428,22 +431,22 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
         const int nt = min(kTile, T - t0);
         __syncthreads();
 #pragma unroll
-        for (int c = 0; c < kFull; ++c) {
+        for (int x = 0; x < kFull; ++x) {
             constexpr int n = ChunkOf<IO>::n;
-            put_chunk<IO>(rr[c], &s.r[0][0], tid + c * kThreads);
+            put_chunk<IO>(rr[x], &s.r[0][0], tid + x * kThreads);
             float om[n], w[n], kv[n];
-            unpack(ro[c], om);
-            unpack(rk[c], kv);
+            unpack(ro[x], om);
+            unpack(rk[x], kv);
 #pragma unroll
-            for (int j = 0; j < n; ++j) {
-                w[j] = decay_from_logit(om[j]);
-                if (kC2) kv[j] *= -expm1f(-expf(om[j]));   // kn = k (1 - w)
+            for (int e = 0; e < n; ++e) {
+                w[e] = decay_from_logit(om[e]);
+                if (kC2) kv[e] *= -expm1f(-expf(om[e]));   // kn = k (1 - w)
             }
-            store_f32(&s.w[0][0] + (tid + c * kThreads) * n, w);
-            store_f32(&s.k[0][0] + (tid + c * kThreads) * n, kv);
+            store_f32(&s.w[0][0] + (tid + x * kThreads) * n, w);
+            store_f32(&s.k[0][0] + (tid + x * kThreads) * n, kv);
         }
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) put_chunk<IO>(rd[c], &s.dy[0][0], tid + c * kThreads);
+        for (int x = 0; x < kCols; ++x) put_chunk<IO>(rd[x], &s.dy[0][0], tid + x * kThreads);
         __syncthreads();
         if (it + 1 < ntile) fetch(it + 1);
         for (int tt = warp * (kTile / 4); tt < (warp + 1) * (kTile / 4); ++tt) {
@@ -455,32 +458,31 @@ __device__ __forceinline__ void col_sweep(ColSmem<kTile>& s, const IO* __restric
 
         for (int st = 0; st < nt; ++st) {
             const int tt = nt - 1 - st;
-            const float dyj = s.dy[tt][jl];
-            float acc0 = 0.f, acc1 = 0.f;
+            const float4 kv = *reinterpret_cast<const float4*>(&s.k[tt][4 * c]);
+            const float4 rv = *reinterpret_cast<const float4*>(&s.r[tt][4 * c]);
+            const float4 wv = *reinterpret_cast<const float4*>(&s.w[tt][4 * c]);
+            const float4 dv4 = *reinterpret_cast<const float4*>(&s.dy[tt][4 * g]);
+            const float ke[4] = {kv.x, kv.y, kv.z, kv.w}, re[4] = {rv.x, rv.y, rv.z, rv.w};
+            const float we[4] = {wv.x, wv.y, wv.z, wv.w}, df[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+            float part[4];
 #pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 kk = *reinterpret_cast<const float4*>(&s.k[tt][16 * m4 + 4 * qq]);
-                const float4 rr = *reinterpret_cast<const float4*>(&s.r[tt][16 * m4 + 4 * qq]);
-                const float4 ww = *reinterpret_cast<const float4*>(&s.w[tt][16 * m4 + 4 * qq]);
-                float* g = &G[4 * m4];
-                acc0 = fmaf(kk.x, g[0], acc0);
-                acc1 = fmaf(kk.y, g[1], acc1);
-                acc0 = fmaf(kk.z, g[2], acc0);
-                acc1 = fmaf(kk.w, g[3], acc1);
-                g[0] = fmaf(ww.x, g[0], rr.x * dyj);
-                g[1] = fmaf(ww.y, g[1], rr.y * dyj);
-                g[2] = fmaf(ww.z, g[2], rr.z * dyj);
-                g[3] = fmaf(ww.w, g[3], rr.w * dyj);
+            for (int f = 0; f < 4; ++f) {
+                float a0 = ke[0] * G[0][f], a1 = ke[1] * G[1][f];
+                a0 = fmaf(ke[2], G[2][f], a0);
+                a1 = fmaf(ke[3], G[3][f], a1);
+                part[f] = a0 + a1;
             }
-            float acc = acc0 + acc1;
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (qq == 0) s.o[tt][jl] = fmaf(s.rku[tt], dyj, acc);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) G[e][f] = fmaf(we[e], G[e][f], re[e] * df[f]);
+            reduce16x4(part, lane);
+            if (owner) s.o[tt][jl_own] = fmaf(s.rku[tt], s.dy[tt][jl_own], part[0]);
         }
         __syncthreads();
         for (int idx = tid; idx < nt * kHalf; idx += kThreads) {
-            const int tt = idx / kHalf, c = idx - (idx / kHalf) * kHalf;
-            dv[tok_index(xbase, t0 + tt, tstride, colbase + c)] = from_f32<IO>(s.o[tt][c]);
+            const int tt = idx / kHalf, cc = idx - (idx / kHalf) * kHalf;
+            dv[tok_index(xbase, t0 + tt, tstride, colbase + cc)] = from_f32<IO>(s.o[tt][cc]);
         }
     }
 }
