@@ -72,6 +72,33 @@ def test_workspace_queries():
     assert binding.prefill_workspace_bytes(2, 10, 3, 32, torch.bfloat16, True) == 0
 
 
+def test_backward_and_gold_workspace_queries():
+    import torch
+    r256 = lambda x: (x + 255) // 256 * 256
+    hand = lambda B, H: 256 + r256(B * H * 4) + B * H * 64 * 64 * 4
+    B, T, H = 2, 10, 3
+    x, bh = B * T * H * 64, B * H * 64
+    # P and E in the scans' accumulation type (fp64 with fp32 I/O), then the du parts
+    assert binding.load().wkv6_backward_workspace_bytes(B, T, H, 64, 0) == \
+        r256(8 * x) + r256(8 * bh) + r256(4 * bh)
+    assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 0) == \
+        r256(8 * x) + r256(8 * bh) + r256(4 * bh)
+    base16 = r256(4 * x) + r256(4 * bh) + r256(4 * bh)
+    # bf16 base form: + reversed k, r, dy, omega, dv and the chunked prefill's workspace
+    assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16) == \
+        base16 + 5 * r256(2 * x) + hand(B, H)
+    assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 1) == base16
+    assert binding.backward_workspace_bytes(B, 0, H, 64, torch.bfloat16) == 0
+    assert binding.load().wkv6_backward_workspace_bytes(B, T, H, 32, 1) == 0
+    # GOLD: cuBLASLt workspace (32 MiB); decompression adds the fp32 product and [x0 | c]
+    lt = 32 << 20
+    assert binding.load().gold_compress_workspace_bytes(1000, 256, 16) == lt
+    assert binding.load().gold_decompress_workspace_bytes(1000, 256, 16) == \
+        r256(1000 * 256 * 4) + r256(1000 * 272 * 2) + lt
+    assert binding.load().gold_compress_workspace_bytes(0, 256, 16) == 0
+    assert binding.load().gold_decompress_workspace_bytes(10, 100, 16) == 0    # D % 8 != 0
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 2, 1, 64)
