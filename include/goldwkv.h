@@ -234,7 +234,10 @@ wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, cons
  *   dstate_in   [B][H][D][D] fp32 output, or NULL (not computed)
  *   workspace   at least wkv6_backward_workspace_bytes(...) bytes; no initial contents needed.
  * No output may overlap an input, another output or the workspace.  T = 0: du = 0 and
- * dstate_in = dstate_out (or zero).
+ * dstate_in = dstate_out (or zero).  The bf16 dv pass uses the chunked prefill's bounded
+ * waits; if one expired (a device that stopped making progress for about a second), dv is
+ * invalid and the call does not report it (the chunked region's status word is internal to
+ * the workspace).
  */
 size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io);
 
