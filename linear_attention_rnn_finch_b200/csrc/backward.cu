@@ -27,10 +27,11 @@
 // bf16 path leaves it out of these scans and runs it through the chunked tensor-core
 // prefill on time-reversed copies (reverse_tokens_kernel moves them).
 //
-// Work split: a CTA owns one (b,h) and 32 of the 64 rows (or columns); thread (row, q)
-// keeps 16 state entries in registers, the sum over the other index is finished with two
-// xor-shuffles across the four q-threads of a row.  Tokens are staged through shared memory
-// in tiles of kTile; per-token outputs are staged too and written coalesced per tile.
+// Work split: a CTA owns one (b,h) and 32 of the 64 rows (dr, dk) or columns (dv); each
+// thread keeps a 4 x 4 block of the state in registers, and the sums over the other index
+// finish over the 16 lanes of a half-warp by a reduce-scatter (reduce16x4).  Tokens are
+// staged through shared memory in tiles of kTile (the next tile's 16-byte chunks held in
+// registers meanwhile); per-token outputs are staged too and written coalesced per tile.
 //
 // Finch-C2's exact form (kC2): the key enters the state as kn_t = k_t (1 - w_t) and there
 // is no bonus, so the dr and dv scans use kn in place of k (formed while staging), the dk
