@@ -16,6 +16,10 @@ with nvidia-smi during the timed region, an end-to-end figure through the public
 host buffers (pinned host -> device inputs, prefill, device -> host y and state inside the
 timed region), the fp64 oracle timed on the host cores on a bounded sample, and the decode
 step (B=256, H=32, 100 steps, state updated in place) in GB/s against the same roofline.
+Further lines, each with its own roofline: the long-context and decay-extreme (+ LayerNorm)
+prefill shapes, the 1.5B layer in Finch-C2's form and with base Finch's GroupNorm + gate,
+the backward of both forms (FP32 CUDA-core roofline), and GOLD compression + decompression
+(bf16 tensor roofline).  `--only backward|backward_c2|gold` prints one of those alone.
 
 `--impl reference` times the oracle (the only reference implementation of this path) on the
 host cores on the same workload, one bounded sample per step.

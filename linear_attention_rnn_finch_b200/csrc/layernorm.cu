@@ -3,7 +3,8 @@
 // GoldFinch review page, section 3.4 "Finch-C2 Time Mixing", output equation):
 //     out = (x - mean) / sqrt(var + eps) * gamma + beta,   var = biased variance.
 // Used as the second pass after a recurrence kernel has written fp32 rows; one CTA per
-// row, exact two-pass mean / variance from the fp32 values.
+// row, exact two-pass mean / variance from the fp32 values (held in registers when the row
+// has at most 8192 channels).  Base Finch's per-head GroupNorm + gate lives here too.
 #include "common.cuh"
 #include "internal.h"
 
