@@ -298,10 +298,8 @@ def backward_line(cfg, dev, world, steps, c2=False):
     dy = torch.randn(inp["r"].shape, generator=g, device=dev).to(cfg.dtype)
     dS = torch.randn(inp["state0"].shape, generator=g, device=dev) * 0.1
     B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
-    L = gw.load()
-    nbytes_ws = (L.wkv6c2_backward_workspace_bytes if c2 else L.wkv6_backward_workspace_bytes)(
-        B, T, H, D, 1)
-    ws = torch.empty(nbytes_ws, dtype=torch.uint8, device=dev)
+    ws = torch.empty(gw.backward_workspace_bytes(B, T, H, D, cfg.dtype, c2=c2), dtype=torch.uint8,
+                     device=dev)
     names = ("r", "k", "v", "omega", "state0") if c2 else ("r", "k", "v", "omega", "u", "state0")
     args_b = [inp[n] for n in names]
 

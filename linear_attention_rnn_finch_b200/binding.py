@@ -461,8 +461,11 @@ def wkv6_backward(r, k, v, omega, u, state_in, dy, dstate_out=None, *, want_dsta
     return dr, dk, dv, dom, du, ds_in
 
 
-def backward_workspace_bytes(B, T, H, D, io_dtype) -> int:
-    return int(load().wkv6_backward_workspace_bytes(B, T, H, D, _io(io_dtype)))
+def backward_workspace_bytes(B, T, H, D, io_dtype, c2=False) -> int:
+    """Bytes of workspace wkv6_backward (or, c2, wkv6c2_backward) needs for these sizes."""
+    L = load()
+    fn = L.wkv6c2_backward_workspace_bytes if c2 else L.wkv6_backward_workspace_bytes
+    return int(fn(B, T, H, D, _io(io_dtype)))
 
 
 def gold_compress(x, w_kd, *, c=None, workspace=None, stream=None):

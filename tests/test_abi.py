@@ -88,6 +88,7 @@ def test_backward_and_gold_workspace_queries():
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16) == \
         base16 + 5 * r256(2 * x) + hand(B, H)
     assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 1) == base16
+    assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16, c2=True) == base16
     assert binding.backward_workspace_bytes(B, 0, H, 64, torch.bfloat16) == 0
     assert binding.load().wkv6_backward_workspace_bytes(B, T, H, 32, 1) == 0
     # GOLD: cuBLASLt workspace (32 MiB); decompression adds the fp32 product and [x0 | c]
