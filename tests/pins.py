@@ -58,7 +58,10 @@ v, omega, u and the initial state):
 * c2_bwd_finite_diff- Finch-C2's backward against central differences through the C2
                       forward entry point (inputs r, k, v, omega, u', S_0);
 * c2_bwd_autograd   - Finch-C2's backward against torch autograd through an independent
-                      torch statement of the C2 explicit sum.
+                      torch statement of the C2 explicit sum;
+* c2_bwd_decay_identity - the pair identity with the normalised keys as sources
+                      (Q_s = kn_s dkn_s, dkn = dk / (1 - w)), plus kn's own dependence on w:
+                      domega_t = -exp(omega_t) (dlog w_t - dkn_t k_t w_t).
 
 GOLD key compression and TokenCat decompression (section 3.4 "GOLD Key Compression and
 TokenCat Decompression"):
@@ -529,6 +532,24 @@ def pin_c2_bwd_autograd(o):
     return ok
 
 
+def pin_c2_bwd_decay_identity(o):
+    r, k, v, om, _, S0, dy, dS = _bwd_inputs(39, 2, 6, 2, 4)
+    up = _rng(40).normal(0, 0.5, r.shape)
+    dr, dk, dv, dom, dup, dS0 = o.backward_c2(r, k, v, om, S0, dy, dS)
+    _, S_T = o.prefill_c2(r, k, v, om, up, S0)
+    w = np.exp(-np.exp(om))
+    dkn = dk / (1.0 - w)                 # omega in (-3, 1): 1 - w >= 0.049
+    P = r * dr
+    Q = k * (1.0 - w) * dkn
+    E = np.einsum("bhij,bhij->bhi", S_T, dS)
+    T = r.shape[1]
+    want = np.empty_like(r)
+    for t in range(T):
+        dlog = E + P[:, t + 1:].sum(axis=1) - Q[:, t:].sum(axis=1)
+        want[:, t] = -np.exp(om[:, t]) * (dlog - dkn[:, t] * k[:, t] * w[:, t])
+    return _close(dom, want, rtol=1e-10) and np.array_equal(dup, dy)
+
+
 def pin_bwd_empty(o):
     r, k, v, om, u, S0, dy, dS = _bwd_inputs(34, 2, 0, 3, 4)
     dr, dk, dv, dom, du, dS0 = o.backward(r, k, v, om, u, S0, dy, dS)
@@ -596,6 +617,7 @@ PINS = {
     "bwd_empty": pin_bwd_empty,
     "c2_bwd_finite_diff": pin_c2_bwd_finite_diff,
     "c2_bwd_autograd": pin_c2_bwd_autograd,
+    "c2_bwd_decay_identity": pin_c2_bwd_decay_identity,
     "gold_compress_matmul": pin_gold_compress_matmul,
     "gold_decompress_blocks": pin_gold_decompress_blocks,
     "gold_rmsnorm_torch": pin_gold_rmsnorm_torch,
