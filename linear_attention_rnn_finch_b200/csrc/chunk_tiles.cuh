@@ -58,15 +58,31 @@ __device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, uint32_t (&v)[16]) {
           "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
 }
+// The same shape repeated 8 times: columns col + 8k + 2(l%4) + {0,1}, k = 0..7.
+__device__ __forceinline__ void tmem_ld16x8(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+}
 // the (hi row + lo row) pair k of a 16x256b load: registers 4k, 4k+1 plus 4k+2, 4k+3
-__device__ __forceinline__ float2 rows_sum(const uint32_t (&v)[16], int k) {
+template <int N>
+__device__ __forceinline__ float2 rows_sum(const uint32_t (&v)[N], int k) {
     return __fadd2_rn(make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1])),
                       make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
 }
-__device__ __forceinline__ float2 lo_pair(const uint32_t (&v)[16], int k) {
+template <int N>
+__device__ __forceinline__ float2 lo_pair(const uint32_t (&v)[N], int k) {
     return make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]));
 }
-__device__ __forceinline__ float2 hi_pair(const uint32_t (&v)[16], int k) {
+template <int N>
+__device__ __forceinline__ float2 hi_pair(const uint32_t (&v)[N], int k) {
     return make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
 }
 
@@ -110,25 +126,52 @@ __device__ __forceinline__ float2 one_minus_exp_neg2(float2 x) {
     return make_float2(x.x < 0.25f ? p.x : d.x, x.y < 0.25f ? p.y : d.y);
 }
 
+// How long one try_wait of a bounded wait may sleep before the thread looks at the CTA's
+// abort / hand-over words and its budget again (nanoseconds; 0: poll without sleeping).  A
+// hand-over wakes the threads still waiting for chunks that will not come within about
+// this time.
+#ifndef GW_WAIT_SLEEP_NS
+#define GW_WAIT_SLEEP_NS 2000
+#endif
+constexpr uint32_t kWaitSleepNs = GW_WAIT_SLEEP_NS;
+
+// The dynamic shared memory rounded up to a 1024-byte boundary (the 128B-swizzle atom),
+// derived from the __shared__ array by pointer arithmetic only: the compiler then still
+// knows every access through it is to shared memory (32-bit addressed LDS / STS, not
+// generic loads and stores).
+template <class T>
+__device__ __forceinline__ T& smem_aligned(uint8_t* raw) {
+    const uint32_t pad = (1024u - (ptx::smem_addr(raw) & 1023u)) & 1023u;
+    return *reinterpret_cast<T*>(raw + pad);
+}
+
 // Bounded wait on an mbarrier phase.  `s` is the CTA's shared state with `abort` and
 // `stop_at` words: the wait gives up early once the CTA has aborted, and on expiry it aborts
 // the CTA.
 // Returns false if the caller should treat its data as invalid (abort).
-// With `or_stop`, also gives up (without aborting) once this (b,h) has been handed over.
+// With stop_chunk >= 0, also gives up (without aborting) once this (b,h) has been handed
+// over at or before chunk stop_chunk (stop_at <= stop_chunk).
 template <class Sm>
 __device__ __forceinline__ bool wait_soft(Sm& s, uint64_t* bar, uint32_t parity, long long budget,
-                                          bool or_stop = false) {
+                                          int stop_chunk = -1) {
     if (ptx::mbar_test_wait(bar, parity)) return true;
-    if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
+    if (stop_chunk >= 0 && ld_volatile(&s.stop_at) <= stop_chunk) return false;
     if (budget <= 0) {
         s.abort = 1;
         return false;
     }
     const long long t0 = clock64();
     for (;;) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
+#ifdef GW_CONTROL_SPIN
+        const bool sleep = kWaitSleepNs > 0 && threadIdx.x >= 96;
+#else
+        const bool sleep = kWaitSleepNs > 0;
+#endif
+        if (sleep ? ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)
+                  : ptx::mbar_try_wait(bar, parity))
+            return true;
         if (ld_volatile(&s.abort)) return false;
-        if (or_stop && ld_volatile(&s.stop_at) >= 0) return false;
+        if (stop_chunk >= 0 && ld_volatile(&s.stop_at) <= stop_chunk) return false;
         if (clock64() - t0 > budget) {
             s.abort = 1;
             return false;

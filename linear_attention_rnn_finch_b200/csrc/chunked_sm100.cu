@@ -135,8 +135,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                     const __nv_bfloat16* __restrict__ uprime, int T, int H, Segments seg, int* status, const int* start_chunk,
                     const float* handoff_state, long long spin_budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
-    Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                       ~uintptr_t(1023));
+    Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // unit: segment pseg of sequence bh, absolute chunks c_begin .. NC - 1
     const int unit = blockIdx.x, nbh = gridDim.x / seg.P;

@@ -55,7 +55,7 @@ struct __align__(1024) Smem {
     uint64_t prep_done[2], op_free[2], ep_free[2], gu_done[2], du_free[2];
     uint32_t tmem_base;
     int abort;
-    int stop_at;                     // unused here (no hand-over); read by wait_soft
+    int stop_at;                     // no hand-over here: never <= a chunk index
 };
 
 // kC2: Finch-C2's normalised key k (1 - w) enters the state.
@@ -65,8 +65,7 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                           const __grid_constant__ CUtensorMap tm_w, float* s_loc, float* log2g, int H,
                           int P, int seg_chunks, int* status, long long budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
-    Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                       ~uintptr_t(1023));
+    Smem& s = smem_aligned<Smem>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // unit: segment pseg (< P-1, so every chunk is full) of sequence bh
     const int unit = blockIdx.x, nbh = gridDim.x / (P - 1);
@@ -89,7 +88,7 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
         ptx::fence_mbar_init();
         s.abort = 0;
-        s.stop_at = -1;
+        s.stop_at = 0x7fffffff;
     }
     if (warp == kTmaWarp) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     ptx::tc_fence_before();
