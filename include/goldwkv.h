@@ -20,8 +20,9 @@
  *  - Pointers r, k, v, omega, u, state*, y, gamma, beta, workspace are DEVICE pointers on
  *    the current CUDA device; the caller owns every buffer.  The library never allocates
  *    device memory, keeps no global mutable state (one exception: the built-in scratch of
- *    wkv6_prefill_static) and, apart from wkv6_workspace_status, never synchronises, so
- *    calls on different streams with different workspaces are independent.
+ *    wkv6_prefill_static) and, apart from wkv6_workspace_status and
+ *    wkv6_prefill_static_status, never synchronises, so calls on different streams with
+ *    different workspaces are independent.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
  *    enqueued asynchronously; a device-side fault surfaces as a CUDA error at the caller's
  *    next synchronisation.
@@ -310,20 +311,28 @@ wkv_status gold_decompress(const void *x0, const void *c, const void *w_ku, cons
  * workspace arguments.  The workspace wkv6_prefill would need is taken instead from a
  * scratch array of WKV6_STATIC_SCRATCH_BYTES bytes compiled into the library (one per
  * device).  Neither this call nor anything it calls allocates memory.
- *   - Limit: sizes for which wkv6_prefill_workspace_bytes(B, T, H, D, io, ln != NULL,
- *     WKV_ALGO_AUTO) exceeds WKV6_STATIC_SCRATCH_BYTES return WKV_ERR_WORKSPACE with
- *     nothing launched.  On the chunked path (bf16 I/O) that is 16 KB per (b,h) plus a
- *     little, so up to 511 (b,h) pairs without LayerNorm; bf16 with LayerNorm also needs
- *     4 * B*T*H*D bytes and fits only for small problems.  fp32 I/O needs no scratch.
+ *   - Limit: on the chunked path (bf16 I/O) wkv6_prefill may cut each (b,h) sequence into
+ *     P segments, and its workspace grows with the number of (b,h,segment) units (about
+ *     32 KB per unit).  Here P is capped: the segment count wkv6_prefill would use if its
+ *     workspace fits the scratch, else the largest smaller one that fits, else P = 1 (no
+ *     split; about 16 KB per (b,h), so up to 511 (b,h) pairs without LayerNorm).  A smaller
+ *     P only leaves SMs idle on few-(b,h) problems; results are the same up to rounding.
+ *     Sizes that do not fit even at P = 1 return WKV_ERR_WORKSPACE with nothing launched;
+ *     bf16 with LayerNorm also needs 4 * B*T*H*D bytes and fits only for small problems.
+ *     fp32 I/O needs no scratch.
  *   - Set-up: the first call on each device, with that device current, looks up the
  *     scratch's device address (cudaGetSymbolAddress, which may load the library's device
- *     code) and caches it; a failed lookup returns WKV_ERR_CUDA.  Make that first call, on
- *     every device that will use it, before capturing a stream that will contain it.
- *   - Zero state: the scratch's first 4 bytes are the chunked path's status word, zero
- *     when the library's device code is loaded.  Nothing else in it has to start at zero:
- *     every other byte a call reads was written earlier in the same call.  A wait that
- *     expires sets the word; this entry point does not report it (there is no
- *     wkv6_workspace_status for it), and the word has no effect on any result.
+ *     code) and caches it with the current CUDA context; a later call in another context
+ *     (for example after cudaDeviceReset) looks it up again.  A failed lookup returns
+ *     WKV_ERR_CUDA.  Make that first call, on every device that will use it, before
+ *     capturing a stream that will contain it.
+ *   - Timeouts: the chunked kernels bound every wait; if one expires, its CTA returns early
+ *     and y and state_out of that call are UNDEFINED, although the call itself returned
+ *     WKV_OK (it returns before the kernels run).  The expiry is recorded in the scratch's
+ *     first 4 bytes (zero when the library's device code is loaded) and stays recorded
+ *     until wkv6_prefill_static_status reads and clears it.  Nothing else in the scratch
+ *     has to start at zero: every other byte a call reads was written earlier in the same
+ *     call.
  *   - Concurrency: all calls on one device share the one scratch.  Calls whose execution
  *     may overlap (different streams, or different host threads without ordering between
  *     them) race on it and can corrupt each other's outputs; order them (one stream, or
@@ -333,6 +342,15 @@ wkv_status wkv6_prefill_static(const void *r, const void *k, const void *v, cons
                                const float *u, const float *state_in, float *state_out, void *y,
                                int B, int T, int H, int D, wkv_dtype io, const wkv_ln *ln,
                                void *stream);
+
+/*
+ * Status of the calls to wkv6_prefill_static on the current device, as wkv6_workspace_status
+ * for a caller's workspace: synchronises `stream` (order it after those calls), returns
+ * WKV_ERR_TIMEOUT and clears the record if a bounded wait of one of them expired since the
+ * last query (their outputs are then undefined), WKV_OK otherwise.  WKV_ERR_CUDA if the
+ * scratch cannot be looked up or the copy fails.  Allocates nothing.
+ */
+wkv_status wkv6_prefill_static_status(void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *wkv6_status_string(wkv_status s);

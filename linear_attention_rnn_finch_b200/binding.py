@@ -61,6 +61,8 @@ def load(path: Path | str | None = None):
     L.wkv6_prefill_algo.restype = i
     L.wkv6_prefill_static.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp]
     L.wkv6_prefill_static.restype = i
+    L.wkv6_prefill_static_status.argtypes = [vp]
+    L.wkv6_prefill_static_status.restype = i
     L.wkv6c2_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
     L.wkv6c2_prefill.restype = i
     L.wkv6c2_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
@@ -233,6 +235,16 @@ def wkv6_prefill_static(r, k, v, omega, u, state_in=None, *, ln=None, y=None, st
     del ln_s
     _raise("wkv6_prefill_static", st)
     return y, state_out
+
+
+def prefill_static_status(device=None, stream=None) -> int:
+    """Synchronise the stream and read (then clear) the timeout record of the built-in
+    scratch of ``device`` (include/goldwkv.h, wkv6_prefill_static_status): WKV_OK, or
+    WKV_ERR_TIMEOUT if a bounded wait of a wkv6_prefill_static call expired since the last
+    query (that call's outputs are undefined)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(load().wkv6_prefill_static_status(_stream_ptr(dev, stream)))
 
 
 def wkv6c2_prefill(r, k, v, omega, uprime, state_in=None, *, ln=None, y=None, state_out=None,

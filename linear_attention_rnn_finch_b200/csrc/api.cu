@@ -156,10 +156,14 @@ long waves(long ctas, int per_sm = 1) {
 // pays when B*H alone leaves SMs idle: estimated time = waves of the main pass x chunks per
 // segment + the pre-pass over the first P-1 segments.  Every segment must be non-empty.
 // GOLDWKV_SEGMENTS=n forces n (tests of the split on small problems).
+bool segments_feasible(int nc, int P) {
+    return P >= 1 && (long)(P - 1) * ((nc + P - 1) / P) < nc;
+}
+
 int choose_segments(int B, int T, int H) {
     const long nbh = (long)B * H;
     const int nc = (T + kChunk - 1) / kChunk;
-    auto feasible = [&](int P) { return P >= 1 && (long)(P - 1) * ((nc + P - 1) / P) < nc; };
+    auto feasible = [&](int P) { return segments_feasible(nc, P); };
     if (const char* f = getenv("GOLDWKV_SEGMENTS")) {
         int P = atoi(f);
         while (P > 1 && !feasible(P)) --P;
@@ -194,6 +198,29 @@ size_t chunked_bytes(int B, int H, int P) {
            segment_bytes(B, H, P);
 }
 
+constexpr size_t kNoCap = ~(size_t)0;
+
+// Segment count and workspace bytes of one prefill (B, T, H > 0, valid io).  The segment
+// count is choose_segments' unless its workspace exceeds `cap`; then it is the largest
+// smaller feasible count whose workspace fits, or 1 when none does (bytes may then still
+// exceed cap: the caller rejects the call).
+struct PrefillPlan {
+    int P;
+    size_t bytes;
+};
+PrefillPlan prefill_plan(int B, int T, int H, wkv_dtype io, bool with_ln, wkv_algo algo,
+                         size_t cap) {
+    const bool chunked = use_chunked(io, algo);
+    // LayerNorm with bf16 output stages the fp32 rows; with fp32 output y itself does
+    const size_t ln = with_ln && io == WKV_BF16 ? (size_t)B * T * H * kHeadSizeApi * sizeof(float)
+                                                : 0;
+    if (!chunked) return {1, ln};
+    int P = algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
+    const int nc = (T + kChunk - 1) / kChunk;
+    while (P > 1 && (!segments_feasible(nc, P) || chunked_bytes(B, H, P) + ln > cap)) --P;
+    return {P, chunked_bytes(B, H, P) + ln};
+}
+
 }  // namespace
 
 extern "C" {
@@ -215,12 +242,7 @@ const char* wkv6_status_string(wkv_status s) {
 size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
                                     wkv_algo algo) {
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
-    const bool chunked = use_chunked(io, algo);
-    const int P = algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
-    size_t bytes = chunked ? chunked_bytes(B, H, P) : 0;
-    // LayerNorm with bf16 output stages the fp32 rows; with fp32 output y itself does
-    if (with_ln && io == WKV_BF16) bytes += (size_t)B * T * H * D * sizeof(float);
-    return bytes;
+    return prefill_plan(B, T, H, io, with_ln != 0, algo, kNoCap).bytes;
 }
 
 size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln) {
@@ -288,7 +310,7 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
                         const float* u, const void* uprime, const float* state_in,
                         float* state_out, void* y, int B, int T, int H, int D, wkv_dtype io,
                         const Norm& nm, wkv_algo algo, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+                        size_t workspace_bytes, void* stream, size_t seg_cap = kNoCap) {
     const bool c2 = uprime != nullptr;
     if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
     if (algo != WKV_ALGO_AUTO && algo != WKV_ALGO_RECURRENT && algo != WKV_ALGO_CHUNKED &&
@@ -333,7 +355,9 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     if (state_in && state_out && state_in != state_out && overlaps(sso, ins[5]))
         return WKV_ERR_INVALID_ARG;
 
-    const size_t need = wkv6_prefill_workspace_bytes(B, T, H, D, io, nm.on(), algo);
+    const PrefillPlan plan = tokens ? prefill_plan(B, T, H, io, nm.on(), algo, seg_cap)
+                                    : PrefillPlan{1, 0};
+    const size_t need = plan.bytes;
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
         const Span sw = span(workspace, need);
@@ -356,7 +380,7 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     const goldwkv::Variant var{uprime};
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
-    const int P = !chunked || algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
+    const int P = plan.P;
     const size_t raw_at = chunked ? chunked_bytes(B, H, P) : 0;
     if (nm.on()) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
@@ -746,3 +770,22 @@ wkv_status gold_decompress(const void* x0, const void* c, const void* w_ku, cons
 }
 
 }  // extern "C"
+
+namespace goldwkv {
+
+size_t prefill_bytes_within(int B, int T, int H, int D, wkv_dtype io, bool with_ln,
+                            size_t cap) {
+    if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
+    return prefill_plan(B, T, H, io, with_ln, WKV_ALGO_AUTO, cap).bytes;
+}
+
+wkv_status prefill_within(const void* r, const void* k, const void* v, const void* omega,
+                          const float* u, const float* state_in, float* state_out, void* y,
+                          int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    return prefill_impl(r, k, v, omega, u, nullptr, state_in, state_out, y, B, T, H, D, io,
+                        layer_norm(ln), WKV_ALGO_AUTO, workspace, workspace_bytes, stream,
+                        workspace_bytes);
+}
+
+}  // namespace goldwkv

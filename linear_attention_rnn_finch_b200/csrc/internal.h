@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include "goldwkv.h"
+
 namespace goldwkv {
 
 // Which form of the time mixing: base Finch / RWKV-6 (static bonus u) when uprime is null;
@@ -84,5 +86,17 @@ cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const
 size_t chunked_smem_bytes();
 size_t fast_smem_bytes();
 size_t segment_smem_bytes();
+
+// ---- prefill within a fixed workspace (the allocation-free entry point uses these)
+// Bytes wkv6_prefill (WKV_ALGO_AUTO) needs when its sequence split is capped so that the
+// workspace stays within `cap`: the split choose_segments makes if it fits, else the largest
+// smaller one that does, else none (the result may then still exceed cap).  0 = no workspace.
+size_t prefill_bytes_within(int B, int T, int H, int D, wkv_dtype io, bool with_ln, size_t cap);
+// wkv6_prefill (WKV_ALGO_AUTO) with the split capped by workspace_bytes as above; same
+// arguments, checks and results.  WKV_ERR_WORKSPACE when even the unsplit path does not fit.
+wkv_status prefill_within(const void* r, const void* k, const void* v, const void* omega,
+                          const float* u, const float* state_in, float* state_out, void* y,
+                          int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 }  // namespace goldwkv

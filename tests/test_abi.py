@@ -34,7 +34,8 @@ def test_headers_declare_entry_points():
     for must in ("wkv6_prefill", "wkv6_prefill_algo", "wkv6_decode_step",
                  "wkv6_prefill_workspace_bytes", "wkv6_decode_workspace_bytes",
                  "wkv6_status_string", "wkv6_abi_version", "wkv6_workspace_status",
-                 "wkv6_prefill_static", "wkv6c2_prefill", "wkv6c2_decode_step",
+                 "wkv6_prefill_static", "wkv6_prefill_static_status", "wkv6c2_prefill",
+                 "wkv6c2_decode_step",
                  "wkv6_prefill_gn", "wkv6_decode_step_gn", "wkv6_backward",
                  "wkv6_backward_workspace_bytes", "wkv6c2_backward",
                  "wkv6c2_backward_workspace_bytes", "gold_compress", "gold_decompress",

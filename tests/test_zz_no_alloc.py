@@ -3,7 +3,10 @@
 Called straight through the C ABI with raw device pointers and compared with wkv6_prefill
 (given a workspace of its own) on the same inputs, for two calls in a row that reuse the
 built-in scratch: the second call hands one sequence over to the level-factorised kernel
-through that scratch.  This file is named to be collected last, and passes on its own too.
+through that scratch.  Also: sequences long enough to be split into segments, one whose
+automatic split would not fit the scratch (served with a smaller split), and an expired
+bounded wait reported by wkv6_prefill_static_status.  This file is named to be collected
+last, and passes on its own too.
 """
 import ctypes
 
@@ -100,6 +103,49 @@ def test_sizes_beyond_the_scratch_are_rejected_untouched():
     y = torch.empty_like(inp["r"])
     s = torch.empty(1, H, 64, 64, device=DEV)
     assert call_static(inp, y, s) == bd.WKV_OK
+    y_ref, s_ref = call_with_workspace(inp)
+    torch.cuda.synchronize()
+    assert rel_err(y, f64(y_ref)) <= TOL[torch.bfloat16]
+    assert rel_err(s, f64(s_ref)) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 16384, 4), (1, 65536, 8)])
+def test_split_sequences_match_the_workspace_entry_point(B, T, H):
+    """Few (b,h) pairs and long sequences: the chunked path cuts each sequence into
+    segments.  At B=1, T=16384, H=4 the automatic split fits the scratch; at B=1, T=65536,
+    H=8 its workspace (about 9.2 MiB) does not, and the call takes a smaller split."""
+    auto = bd.prefill_workspace_bytes(B, T, H, 64, torch.bfloat16, False)
+    unsplit = bd.prefill_workspace_bytes(B, T, H, 64, torch.bfloat16, False,
+                                         algo="chunked_levels")
+    assert auto > unsplit   # wkv6_prefill splits this problem
+    if T == 65536:
+        assert auto > bd.STATIC_SCRATCH_BYTES
+    inp = problem(9305 + H, B=B, T=T, H=H)
+    y = torch.full_like(inp["r"], 3.0)
+    s = torch.full((B, H, 64, 64), 7.0, device=DEV)
+    assert call_static(inp, y, s) == bd.WKV_OK
+    assert bd.prefill_static_status() == bd.WKV_OK
+    y_ref, s_ref = call_with_workspace(inp)
+    torch.cuda.synchronize()
+    assert rel_err(y, f64(y_ref)) <= TOL[torch.bfloat16]
+    assert rel_err(s, f64(s_ref)) <= TOL[torch.bfloat16]
+
+
+def test_expired_wait_is_reported_once_and_the_next_call_is_correct(monkeypatch):
+    """A zero spin budget makes the first bounded wait of every CTA expire: the call still
+    returns WKV_OK, the status query reports the timeout once and clears it, and the next
+    call (normal budget) through the same scratch is correct."""
+    inp = problem(9310, B=2, T=200, H=8)
+    y = torch.empty_like(inp["r"])
+    s = torch.empty(2, 8, 64, 64, device=DEV)
+    assert bd.prefill_static_status() == bd.WKV_OK
+    monkeypatch.setenv("GOLDWKV_FAULT", "timeout0")
+    assert call_static(inp, y, s) == bd.WKV_OK
+    assert bd.prefill_static_status() == bd.WKV_ERR_TIMEOUT
+    assert bd.prefill_static_status() == bd.WKV_OK
+    monkeypatch.delenv("GOLDWKV_FAULT")
+    assert call_static(inp, y, s) == bd.WKV_OK
+    assert bd.prefill_static_status() == bd.WKV_OK
     y_ref, s_ref = call_with_workspace(inp)
     torch.cuda.synchronize()
     assert rel_err(y, f64(y_ref)) <= TOL[torch.bfloat16]
