@@ -33,22 +33,30 @@
 //   GA(n): [A_hi ; A_lo] x V (N=64), accumulated into Y's first 64 columns
 //                                                               A = masked scores + bonus.
 //
-// Roles (16 warps, no dedicated producer or issuer threads: the group that finishes a step
-// issues the copies and products that follow it, so no thread polls for another's work):
+// Roles (16 warps, no dedicated producer or issuer warps: a thread that has just finished
+// a step, or is between two steps of its own work, issues the copies and products that
+// follow, so no warp does nothing but poll):
 //   warps 0-7, prep: two groups of 4 warps taking alternate chunks (group g: n = g mod 2).
 //     A warp takes 16 tokens; a thread takes 8 channels (one 16-byte column of the tile) of
 //     4 consecutive tokens: exp(omega), the log-decay prefix (serial over its 4 tokens, a
 //     shuffle scan over the warp's 4 runs, a shared-memory sum over the group's warps), the
 //     range test, Rt / Kh hi/lo with 16-byte stores, the bonus (shuffle-reduced over the 8
-//     channel columns) and gamma.  Then the group's elected thread issues the r / k / omega
-//     copy of chunk n+3 into the stage just read, and GU(n), SC(n).
-//   warps 8-15, epilogue, per chunk n: the elected thread issues RO(n) as soon as GU(n) has
-//     landed; state(n) = gamma (S + DU), S_n hi/lo for RO(n+1); A(n); the elected thread
-//     issues GA(n); the output of chunk n-1 (Y -> y); the elected thread loads v of chunk
-//     n+3.
+//     channel columns) and gamma.  Lane 0 of three of the group's warps issues tensor-core
+//     work, so that one issuer's wait on the tensor pipe does not hold up the others:
+//       warp 0, after chunk n: the r / k / omega copy of chunk n+3, GU(n) and SC(n);
+//       warp 1, after chunk n: GA(n-1) (the other group's chunk), once the epilogue stored
+//               A(n-1) and RO(n-1) is complete;
+//       warp 2, between the two passes of chunk n: RO(n-2), once the epilogue stored S_{n-3}
+//               (before pass 2 rewrites the Rt buffer RO(n-2) reads).
+//   warps 8-15, epilogue, per chunk n: state(n) = gamma (S + DU); S_n hi/lo for RO(n+1);
+//     A(n); the output of chunk n-1 (Y -> y); its elected thread loads v of chunk n+3.
+//     The epilogue issues no tensor-core work.
 // The fp32 state stays in the epilogue's registers.  Handshakes are mbarriers (tensor-core
-// commits, copy completion, buffer releases) and named barriers inside a group; every
-// mbarrier wait is bounded.
+// commits, copy completion, epilogue arrivals) and named barriers inside a group; every
+// mbarrier wait is bounded.  A barrier phase is never completed while a waiter may still be
+// waiting for the phase before it (its parity wait would alias): commits follow from the
+// data dependencies, and a hand-over or give-up that could break that order skips its
+// commit or waits first.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <limits.h>
@@ -101,9 +109,13 @@ struct __align__(1024) Smem {
     float gamma[4][64];                 // gamma and bonus of chunk n in slot n % 4
     float bonus[4][64];
     uint64_t full_rkw[kStagesRkw], full_v[kStagesV];
-    uint64_t gu_done[2], sc_done[2];    // prep leaders' commits (GU and SC of parity n & 1)
-    uint64_t ya_done[2], op_free[2];    // epilogue leader's commits (RO + GA; Rt / Kh free)
-    uint64_t du_free[2], sc_free[2], ep_free[4];   // epilogue arrivals
+    // prep issuers' commits for chunk n in slot n & 1: mm_done after GU(n) + SC(n), op_free
+    // after RO(n), ya_done after GA(n); drain[g][i]: issuer i of group g's last commit
+    uint64_t mm_done[2], op_free[2], ya_done[2], drain[kPrepGroups][3];
+    // epilogue arrivals: du_free (DU read), ep_free[n % 4] (gamma / bonus of n read),
+    // a_ready[n & 1] (A(n) stored, SC(n) read), s_ready[n & 1] (S_{n-1} stored in sb[n & 1]
+    // and Y[n & 1] free: RO(n) may run)
+    uint64_t du_free, ep_free[4], a_ready[2], s_ready[2];
     int last_rkw[kStagesRkw], last_v[kStagesV];    // latest chunk loaded into each stage
     uint32_t tmem_base;
     int abort;
@@ -268,13 +280,15 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             s.last_v[i] = -1;
         }
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&s.gu_done[i], 1);
-            ptx::mbar_init(&s.sc_done[i], 1);
-            ptx::mbar_init(&s.ya_done[i], 1);
+            ptx::mbar_init(&s.mm_done[i], 1);
             ptx::mbar_init(&s.op_free[i], 1);
-            ptx::mbar_init(&s.du_free[i], kEpiThreads);
-            ptx::mbar_init(&s.sc_free[i], kEpiThreads);
+            ptx::mbar_init(&s.ya_done[i], 1);
+            ptx::mbar_init(&s.a_ready[i], kEpiThreads);
+            ptx::mbar_init(&s.s_ready[i], kEpiThreads);
         }
+        for (int i = 0; i < kPrepGroups; ++i)
+            for (int j = 0; j < 3; ++j) ptx::mbar_init(&s.drain[i][j], 1);
+        ptx::mbar_init(&s.du_free, kEpiThreads);
         for (int i = 0; i < 4; ++i) ptx::mbar_init(&s.ep_free[i], kEpiThreads);
         ptx::fence_mbar_init();
         s.abort = 0;
@@ -299,7 +313,10 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         // lane: channels 8cg .. 8cg+7 (cg = lane % 8) of tokens tb .. tb+3 (tb = 16wg + 4rr,
         // rr = lane / 8).  Log-decay sums are in log2 units.
         const int g = warp / kGroupWarps, wg = warp % kGroupWarps;
-        const bool leader = wg == 0 && lane == 0;   // issues the group's copies and products
+        // lane 0 of the group's warps 0, 1, 2 issues, for chunk n of the group: the r / k / omega
+        // copy of n+3, GU(n) and SC(n) (warp 0); GA(n-1) (warp 1); RO(n) (warp 2)
+        const bool leader = wg == 0 && lane == 0;
+        const bool ga_issuer = wg == 1 && lane == 0, ro_issuer = wg == 2 && lane == 0;
         const int cg = lane & 7, rr = lane >> 3;
         const int c0 = 8 * cg;
         const int tb = 16 * wg + 4 * rr;
@@ -312,16 +329,54 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         for (int p = 0; p < 4; ++p) toff[p] = (uint32_t)((tb + p) * 128 + ((cg ^ ((tb + p) & 7)) << 4));
         const float2 l2e = make_float2(kLog2e, kLog2e);
         const float2 nl2e = make_float2(-kLog2e, -kLog2e);
-        int last_mma = -1;   // the latest chunk whose products this thread (leader) issued
-        for (int n = g; n < NC; n += kPrepGroups) {
+        bool issued = false;   // the leader issued tensor-core work (drained before exit)
+        // GA(m) = Y[m & 1] += A(m) x V(m), issued by this group's leader for m = n - 1 (the other
+        // group's chunk) once the epilogue stored A(m) and RO(m) (the other leader's) is complete
+        auto issue_ga = [&](int m) {
+            const int mb = m & 1;
+            bool ok = wait_soft(s, &s.a_ready[mb], (uint32_t)((m >> 1) & 1), budget, m);
+            ok = ok && wait_soft(s, &s.op_free[mb], (uint32_t)((m >> 1) & 1), budget, m);
+            if (ok) {
+                ptx::tc_fence_after();
+                const uint32_t ycol = tmem + COL_Y + 128 * mb;
+                const uint32_t v_tile = ptx::smem_addr(s.vt[m % kStagesV]);
+                const uint32_t at = ptx::smem_addr(s.at);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)   // Y += [A] x V
+                    ptx::mma_bf16(ycol, ptx::desc_kmajor(at + 32 * kq),
+                                  ptx::desc_mnmajor(v_tile + 2048 * kq), IDESC_GA, 1);
+                issued = true;
+                ptx::mma_commit(&s.ya_done[mb]);
+            }
+            // after a give-up (hand-over at or before m, or abort) nothing waits for chunk m's
+            // phase, and completing it could alias an earlier phase a waiter has not seen
+        };
+        // RO(m) = Y[m & 1] = Rt(m) x S_{m-1}, for this group's chunk m, issued by warp 2 while
+        // the group works on chunk m+2 (between its two passes), once the epilogue has stored
+        // S_{m-1} in sb[m & 1] and read Y[m & 1] (end of its chunk m-1)
+        int ro_next = g;   // this group's next chunk whose RO is to be issued
+        auto issue_ro = [&](int m) {
+            const int mb = m & 1;
+            if (wait_soft(s, &s.s_ready[mb], (uint32_t)((m >> 1) & 1), budget, m)) {
+                ptx::tc_fence_after();
+                const uint32_t rtile = ptx::smem_addr(s.rt[mb]);
+                const uint32_t sbuf = ptx::smem_addr(s.sb[mb]);
+                const uint32_t ycol = tmem + COL_Y + 128 * mb;
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)   // Y = [Rt] x [S_hi^T ; S_lo^T]
+                    ptx::mma_bf16(ycol, ptx::desc_kmajor(rtile + 32 * kq),
+                                  ptx::desc_kmajor(sbuf + 32 * kq), IDESC_RO, kq > 0);
+                issued = true;
+                ptx::mma_commit(&s.op_free[mb]);
+            }
+            ro_next = m + kPrepGroups;
+        };
+        int n = g;
+        for (; n < NC; n += kPrepGroups) {
             const int pb = n & 1, st = n % kStagesRkw;
             const int valid = min(C, T - (cseg + n) * C);
-            // r / k / omega of chunk n; Rt / Kh of parity pb read by SC and RO of chunk n-2
-            // (the RO commit comes after the epilogue saw SC(n-2) complete); gamma / bonus
-            // slot n % 4 read by the epilogue for chunk n-4
+            // r / k / omega of chunk n; gamma / bonus slot n % 4, read by the epilogue for n-4
             bool ok_wait = wait_soft(s, &s.full_rkw[st], (uint32_t)((n / kStagesRkw) & 1), budget, n);
-            if (n >= 2)
-                ok_wait = ok_wait && wait_soft(s, &s.op_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget, n);
             if (n >= 4)
                 ok_wait = ok_wait && wait_soft(s, &s.ep_free[n & 3], (uint32_t)(((n - 4) >> 2) & 1), budget, n);
             if (named_bar_any(kBarPrep0 + g, kGroupThreads, !ok_wait || stopped_at(s, n))) break;
@@ -366,7 +421,12 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 dst[0] = make_float4(inc[0].x, inc[0].y, inc[1].x, inc[1].y);
                 dst[1] = make_float4(inc[2].x, inc[2].y, inc[3].x, inc[3].y);
             }
-            named_bar(kBarPrep0 + g, kGroupThreads);
+            // Rt / Kh of parity pb were read by GU, SC and RO of chunk n-2, which this group
+            // issued; RO(n-2) is issued now and committed on op_free[pb]
+            if (ro_issuer && n >= kPrepGroups) issue_ro(n - kPrepGroups);
+            __syncwarp();
+            const bool ok_free = n < 2 || wait_soft(s, &s.op_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget, n);
+            if (named_bar_any(kBarPrep0 + g, kGroupThreads, !ok_free)) break;
             float2 off[4], tot[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) off[q] = tot[q] = make_float2(0.f, 0.f);
@@ -390,10 +450,15 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 in_range = in_range && (tot[q].x >= -kMaxLog2Range) && (tot[q].y >= -kMaxLog2Range);
             if (!__all_sync(0xffffffffu, in_range)) {
                 // hand this (b,h) to the level kernel from chunk n on (the other group may
-                // have found a later chunk first: keep the earliest), and wake the epilogue
+                // have found a later chunk first: keep the earliest), and wake the epilogue.
+                // The arrive completes the phase of mm_done[pb] for chunk n; it waits until
+                // every epilogue thread is past its wait for chunk n-2 on the same barrier
+                // (they have read DU of chunk n-1), or a parity wait there could see two
+                // completed phases as none.  No arrive if the sequence stops earlier.
                 if (leader) {
                     atomicMin(&s.stop_at, n);
-                    mbar_arrive(&s.gu_done[pb]);
+                    const bool wake = n < 1 || wait_soft(s, &s.du_free, (uint32_t)((n - 1) & 1), budget, n - 1);
+                    if (wake) mbar_arrive(&s.mm_done[pb]);
                 }
                 break;
             }
@@ -466,13 +531,11 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             named_bar(kBarPrep0 + g, kGroupThreads);
             if (leader) {
                 if (n + kStagesRkw < NC) load_rkw(s, &tm_r, &tm_k, &tm_w, n + kStagesRkw, cseg, h, b);
-                // v of chunk n; DU / SC of parity pb read by the epilogue for chunk n-2
-                // (each gives up if the sequence was handed over at or before chunk n)
+                // GU(n), SC(n): v of chunk n; DU read by the epilogue for chunk n-1; the SC
+                // buffer of parity pb read by A(n-2) (GA(n-2) waited for that).  Every wait
+                // gives up if the sequence was handed over at or before the chunk it serves.
                 bool ok = wait_soft(s, &s.full_v[n % kStagesV], (uint32_t)((n / kStagesV) & 1), budget, n);
-                if (n >= 1)   // the single DU buffer read by the epilogue for chunk n-1
-                    ok = ok && wait_soft(s, &s.du_free[0], (uint32_t)((n - 1) & 1), budget, n);
-                if (n >= 2)
-                    ok = ok && wait_soft(s, &s.sc_free[pb], (uint32_t)(((n - 2) >> 1) & 1), budget, n);
+                if (n >= 1) ok = ok && wait_soft(s, &s.du_free, (uint32_t)((n - 1) & 1), budget, n);
                 if (ok) {
                     ptx::tc_fence_after();
                     const uint32_t v_tile = ptx::smem_addr(s.vt[n % kStagesV]);
@@ -482,19 +545,28 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     for (int kq = 0; kq < 4; ++kq)   // DU = V^T x [Kh_hi | Kh_lo]
                         ptx::mma_bf16(tmem + COL_DU, ptx::desc_mnmajor(v_tile + 2048 * kq),
                                       ptx::desc_sw128(kh + 2048 * kq, kTile), IDESC_GU, kq > 0);
-                    ptx::mma_commit(&s.gu_done[pb]);
 #pragma unroll
                     for (int kq = 0; kq < 4; ++kq)   // SC = [Rt] x Kh_hi^T
                         ptx::mma_bf16(tmem + COL_SC + 64 * pb, ptx::desc_kmajor(rtile + 32 * kq),
                                       ptx::desc_kmajor(kh + 32 * kq), IDESC_SC, kq > 0);
-                    ptx::mma_commit(&s.sc_done[pb]);
-                    last_mma = n;
+                    ptx::mma_commit(&s.mm_done[pb]);
+                    issued = true;
                 }
+            } else if (ga_issuer) {
+                if (n >= 1) issue_ga(n - 1);
             }
+            __syncwarp();
         }
+        // the chunk this group stopped at (or the first past the sequence): GA of the chunk
+        // before it is still this group's (it is the other group's chunk)
+        if (ga_issuer && n >= 1 && n <= NC) issue_ga(n - 1);
+        // RO of this group's last chunk whose products were issued
+        if (ro_issuer && ro_next <= n - kPrepGroups && ro_next < NC) issue_ro(ro_next);
         // drain: this thread's tensor-core work must be complete before TMEM is freed
-        if (leader && last_mma >= 0)
-            ptx::mbar_wait(&s.sc_done[last_mma & 1], (uint32_t)((last_mma >> 1) & 1), drain_budget);
+        if (issued) {   // one of the group's issuers
+            ptx::mma_commit(&s.drain[g][wg]);
+            ptx::mbar_wait(&s.drain[g][wg], 0, drain_budget);
+        }
     } else {
         // ------------------------------------------------------------ epilogue (8 warps)
         // warp (q, ch0): TMEM sub-partition q = warp % 4, columns 32ch0 .. 32ch0+31 of each
@@ -534,6 +606,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 }
             }
             ptx::fence_proxy_async_smem();
+            mbar_arrive(&s.s_ready[0]);   // RO(0) may run
         }
         uint32_t up0[kPairs], up1[kPairs];   // Finch-C2: u' of the next output
 #pragma unroll
@@ -545,33 +618,20 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             if (kC2 && n >= 1) load_uprime(uprime, n - 1, cseg, b, h, T, H, col0, cl, r0, r1, up0, up1);
             // ---- state(n): S <- gamma (S + DU), DU^T[j][i] accumulated on the tensor cores.
             // gamma and bonus of chunk n reach us through prep's named barrier -> its leader's
-            // MMA issue -> the commit on gu_done (or, at a hand-over, the leader's arrive).
+            // MMA issue -> the commit on mm_done (or, at a hand-over, the leader's arrive).
             {
-                const bool ok = wait_soft(s, &s.gu_done[pb], (uint32_t)((n >> 1) & 1), budget);
+                const bool ok = wait_soft(s, &s.mm_done[pb], (uint32_t)((n >> 1) & 1), budget);
                 // uniform over the epilogue: stop (hand-off) or abort
                 if (named_bar_any(kBarEpi, kEpiThreads, !ok || stopped_at(s, n))) break;
             }
             ptx::tc_fence_after();
-            // RO(n) needs only Rt(n), S_{n-1} (stored in the previous round) and Y[n & 1] (read
-            // by output(n-2) in the previous round): issue it first, so that the Rt / Kh
-            // buffer of parity pb is released to prep as early as possible
-            if (leader) {
-                const uint32_t rtile = ptx::smem_addr(s.rt[pb]);
-                const uint32_t sbuf = ptx::smem_addr(s.sb[pb]);
-                const uint32_t ycol = tmem + COL_Y + 128 * pb;
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // Y = [Rt] x [S_hi^T ; S_lo^T]
-                    ptx::mma_bf16(ycol, ptx::desc_kmajor(rtile + 32 * kq), ptx::desc_kmajor(sbuf + 32 * kq),
-                                  IDESC_RO, kq > 0);
-                ptx::mma_commit(&s.op_free[pb]);   // Rt / Kh of parity pb no longer read
-            }
             {
                 uint32_t ua[16], ub[16];
                 tmem_ld16x4(tmem + lane_h0 + COL_DU + col0, ua);
                 tmem_ld16x4(tmem + lane_h0 + COL_DU + 64 + col0, ub);
                 ptx::tmem_wait_ld();
                 ptx::tc_fence_before();
-                mbar_arrive(&s.du_free[0]);
+                mbar_arrive(&s.du_free);
                 const float* gam = s.gamma[n & 3] + col0 + cl;
 #pragma unroll
                 for (int j = 0; j < kPairs; ++j) {
@@ -585,9 +645,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             if (n >= 1 && !wait_soft(s, &s.ya_done[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), budget))
                 s.abort = 1;
             if (n + 1 < NC) store_state(s.sb[(n + 1) & 1], S0, S1, r0, r1, q0, cb);   // for RO(n+1)
-            // ---- A(n): masked scores with the bonus on the diagonal, hi / lo, for GA(n)
-            if (!wait_soft(s, &s.sc_done[pb], (uint32_t)((n >> 1) & 1), budget)) s.abort = 1;
-            ptx::tc_fence_after();
+            // ---- A(n): masked scores with the bonus on the diagonal, hi / lo, for GA(n).  SC(n)
+            // is complete: it was committed with GU(n) on mm_done.
             if (!a_zero) {
                 uint32_t p0[16], p1[16];
                 tmem_ld16x4(tmem + lane_h0 + COL_SC + 64 * pb + col0, p0);
@@ -613,23 +672,11 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     sts32(s.at, sw_off(hr1 + 8, q0 + k) + cb, lo);
                 }
             }
-            ptx::tc_fence_before();
-            mbar_arrive(&s.sc_free[pb]);
-            mbar_arrive(&s.ep_free[n & 3]);   // gamma / bonus of chunk n read
+            // A(n) (and S_n) stored, SC(n), gamma and bonus of chunk n read: GA(n) may run
             ptx::fence_proxy_async_smem();
-            // S_n and A(n) written in every thread
-            named_bar(kBarEpi, kEpiThreads);
-            if (leader && !ld_volatile(&s.abort)) {
-                ptx::tc_fence_after();
-                const uint32_t ycol = tmem + COL_Y + 128 * pb;
-                const uint32_t v_tile = ptx::smem_addr(s.vt[n % kStagesV]);
-                const uint32_t at = ptx::smem_addr(s.at);
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq)   // Y += [A] x V
-                    ptx::mma_bf16(ycol, ptx::desc_kmajor(at + 32 * kq),
-                                  ptx::desc_mnmajor(v_tile + 2048 * kq), IDESC_GA, 1);
-                ptx::mma_commit(&s.ya_done[pb]);
-            }
+            ptx::tc_fence_before();
+            mbar_arrive(&s.ep_free[n & 3]);
+            mbar_arrive(&s.a_ready[pb]);
             // ---- output of chunk n-1 (GA(n-1) is complete: waited above)
             if (n >= 1) {
                 ptx::tc_fence_after();
@@ -639,6 +686,9 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 if (leader && n + kStagesV - 1 < NC && !stopped_at(s, n + kStagesV - 1))
                     load_v(s, &tm_v, n + kStagesV - 1, cseg, h, b);
             }
+            // S_n is in sb[(n+1) & 1] and Y[(n+1) & 1] (output(n-1)) has been read: RO(n+1)
+            ptx::tc_fence_before();
+            mbar_arrive(&s.s_ready[(n + 1) & 1]);
         }
         // ---- leave: output of the last chunk done, final state (or the state entering the
         // chunk handed to the level kernel)
@@ -669,9 +719,6 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             }
             if (leader) handoff_chunk[unit] = stopped ? cseg + n : -1;
         }
-        // drain: the leader's last products must be complete before TMEM is freed
-        if (leader && n >= 1)
-            ptx::mbar_wait(&s.ya_done[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), drain_budget);
     }
 
     ptx::tc_fence_before();
