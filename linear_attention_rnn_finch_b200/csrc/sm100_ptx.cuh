@@ -154,30 +154,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
-// mma_bf16 executed by a whole warp with warp-uniform operands and issued by the one lane
-// whose `issue` is nonzero: the warp stays converged around the issue.
-__device__ __forceinline__ void mma_bf16_by(uint32_t issue, uint32_t d_tmem, uint64_t a_desc,
-                                            uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "setp.ne.b32 e, %5, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(issue)
-        : "memory");
-}
-
-// mma_commit by the lane whose `issue` is nonzero (the lane that issued the products).
-__device__ __forceinline__ void mma_commit_by(uint32_t issue, uint64_t* bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t"
-        "setp.ne.b32 e, %1, 0;\n\t"
-        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-            smem_addr(bar)), "r"(issue)
-        : "memory");
-}
-
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
