@@ -5,6 +5,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "goldwkv.h"
 #include "internal.h"
 #include "backward.h"
@@ -140,15 +142,34 @@ bool use_chunked(wkv_dtype io, wkv_algo algo) {
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 constexpr int kChunk = 64;          // tokens per chunk of the chunked kernels
-constexpr int kSmCount = 148;       // SMs of a B200: the unit of a wave of CTAs
+constexpr int kSmCountDefault = 148;   // SMs of a full B200, if the device cannot be asked
 constexpr int kMinSegChunks = 16;   // shortest segment worth a CTA
 // The state pre-pass runs two CTAs per SM; its time per chunk and wave of those slots,
 // relative to the main prefill's per chunk and wave (one CTA per SM), measured on B200.
 constexpr int kPrePassCtasPerSm = 2;
 constexpr double kPrePassCost = 0.62;
 
+// SMs of the current device (the unit of a wave of CTAs), asked once per device.
+int sm_count() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        (void)cudaGetLastError();
+        return kSmCountDefault;
+    }
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        return kSmCountDefault;
+    }
+    cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 long waves(long ctas, int per_sm = 1) {
-    const long slots = (long)kSmCount * per_sm;
+    const long slots = (long)sm_count() * per_sm;
     return (ctas + slots - 1) / slots;
 }
 
