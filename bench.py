@@ -14,12 +14,15 @@ The line also reports: the dominant kernel's roofline fraction (algorithmic byte
 launch / CUDA-event launch time vs. the measured HBM copy bandwidth), SM clocks sampled
 with nvidia-smi during the timed region, an end-to-end figure through the public API with
 host buffers (pinned host -> device inputs, prefill, device -> host y and state inside the
-timed region), the fp64 oracle timed on the host cores on a bounded sample, and the decode
-step (B=256, H=32, 100 steps, state updated in place) in GB/s against the same roofline.
-Further lines, each with its own roofline: the long-context and decay-extreme (+ LayerNorm)
-prefill shapes, the 1.5B layer in Finch-C2's form and with base Finch's GroupNorm + gate,
-the backward of both forms (FP32 CUDA-core roofline), and GOLD compression + decompression
-(bf16 tensor roofline).  `--only backward|backward_c2|gold` prints one of those alone.
+timed region) and the fp64 oracle timed on the host cores on a bounded sample.
+The other measurements go, one short record each, into the list `more` (workload with its
+sizes, ms per call, value and unit, roofline bound and fraction, and for decode also the
+fraction from the DRAM bytes ncu counted): the decode step, the long-context and
+decay-extreme (+ LayerNorm) prefill shapes, the 1.5B layer in Finch-C2's form and with base
+Finch's GroupNorm + gate, the backward of both forms (FP32 CUDA-core roofline), and GOLD
+compression + decompression (bf16 tensor roofline).  `--only backward|backward_c2|gold`
+prints one of those alone, in full.  Every API call in a timed loop sits in an NVTX range
+named after the entry point.
 
 `--impl reference` times the oracle (the only reference implementation of this path) on the
 host cores on the same workload, one bounded sample per step.
@@ -87,12 +90,10 @@ NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
                             "internal.h"),
                 "sha256_16": "70892a82047ac1bf", "bytes": 541468160 + 120561920,
-                "workload": (8, 4096, 32),
-                "profile": "profiles/wkv6_fast_kernel_prefill_B8_T4096_H32_bf16.md"},
+                "workload": (8, 4096, 32)},
     "decode": {"sources": ("decode.cu", "common.cuh"),
                "sha256_16": "8fb24cf16874f036", "bytes": 138433536 + 78408192,
-               "workload": (256, 32),
-               "profile": "profiles/wkv6_decode_kernel_B256_H32_bf16.md"},
+               "workload": (256, 32)},
 }
 
 
@@ -105,6 +106,32 @@ def ncu_traffic(kind: str, workload: tuple):
     if h.hexdigest()[:16] != rec["sha256_16"] or tuple(workload) != rec["workload"]:
         return None
     return rec["bytes"]
+
+
+def sig(x, digits=4):
+    """x rounded to `digits` significant figures (keeps the printed line short)."""
+    if x is None or x == 0 or not isinstance(x, float):
+        return x
+    from math import floor, log10
+    return round(x, max(0, digits - 1 - int(floor(log10(abs(x))))))
+
+
+def compact(line: dict) -> dict:
+    """One secondary measurement as a short record: workload, ms per call, value and unit,
+    the roofline bound and fraction, and (where an ncu capture of the same sources exists)
+    the fraction computed from the DRAM bytes ncu counted instead of the algorithmic ones."""
+    r = line["roofline"]
+    out = {"w": line["workload"], "ms": sig(line["ms_per_call"]),
+           "v": sig(float(line["value"])), "u": line["unit"],
+           "bound": r["bound"], "frac": sig(r["frac"], 3)}
+    if r.get("dram_frac") is not None:
+        out["dram_frac"] = sig(r["dram_frac"], 3)
+    return out
+
+
+def nvtx(name: str):
+    """NVTX range around one API call (visible in an nsys or ncu timeline)."""
+    return torch.cuda.nvtx.range(name)
 
 
 def peaks():
@@ -242,6 +269,10 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False, gn=False):
     args_p = [inp[n] for n in ("r", "k", "v", "omega")]
 
     def call():
+        with nvtx("wkv6_prefill_gn" if gn else "wkv6c2_prefill" if c2 else "wkv6_prefill"):
+            call_()
+
+    def call_():
         if gn:
             gw.wkv6_prefill_gn(*args_p, inp["u"], inp["state0"], gn=gn_args, y=y, state_out=s_out,
                                workspace=ws)
@@ -274,9 +305,9 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False, gn=False):
     form = ("Finch-C2 (normalised key, second value)" if c2 else
             "base Finch (static bonus), per-head GroupNorm and gate" if gn else
             "base Finch (static bonus)")
-    line = {"workload": name, "B": B, "T": T, "H": H, "D": D, "io": "bf16", "form": form,
-            "ln": bool(cfg.ln), "steps": steps, "ms_per_call": ms,
-            "tokens_per_s": world * B * T / (ms / 1e3),
+    line = {"workload": f"{name} B{B} T{T} H{H}", "B": B, "T": T, "H": H, "D": D, "io": "bf16",
+            "form": form, "ln": bool(cfg.ln), "steps": steps, "ms_per_call": ms,
+            "value": world * B * T / (ms / 1e3), "unit": "tokens/s",
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm,
                          "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm,
                          "algorithmic_bytes_per_call": nbytes}}
@@ -304,9 +335,10 @@ def backward_line(cfg, dev, world, steps, c2=False):
     args_b = [inp[n] for n in names]
 
     def call():
-        if c2:
-            return gw.wkv6c2_backward(*args_b, dy, dS, workspace=ws)
-        return gw.wkv6_backward(*args_b, dy, dS, workspace=ws)
+        with nvtx("wkv6c2_backward" if c2 else "wkv6_backward"):
+            if c2:
+                return gw.wkv6c2_backward(*args_b, dy, dS, workspace=ws)
+            return gw.wkv6_backward(*args_b, dy, dS, workspace=ws)
 
     for _ in range(3):
         call()
@@ -324,9 +356,9 @@ def backward_line(cfg, dev, world, steps, c2=False):
     # dr scan, dk scan, du sum; 2 reversals + fast + level kernels for dv (+ 2 segment
     # kernels when the sequence is split).  Finch-C2: the dr + dv scan launch and the dk scan
     launches_per_call = 2 if c2 else 3 + 4
-    line = {"workload": "wkv6c2_backward_1p5b_layer" if c2 else "wkv6_backward_1p5b_layer",
-            "B": B, "T": T, "H": H, "D": D, "io": "bf16",
-            "steps": steps, "ms_per_call": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+    line = {"workload": ("wkv6c2_backward" if c2 else "wkv6_backward") + f" B{B} T{T} H{H}",
+            "B": B, "T": T, "H": H, "D": D, "io": "bf16", "steps": steps, "ms_per_call": ms,
+            "value": world * B * T / (ms / 1e3), "unit": "tokens/s",
             "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
                          "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
                          "frac": flops / (ms / 1e3) / 1e12 / ALU_FP32_TFLOPS,
@@ -365,8 +397,10 @@ def gold_line(dev, world, steps, B=8, T=4096, D=2048, Dc=128):
     ws_d = torch.empty(L.gold_decompress_workspace_bytes(N, D, Dc), dtype=torch.uint8, device=dev)
 
     def call():
-        gw.gold_compress(x, w_kd, c=c, workspace=ws_c)
-        gw.gold_decompress(x0, c, w_ku, gamma, 1e-6, kd=kd, workspace=ws_d)
+        with nvtx("gold_compress"):
+            gw.gold_compress(x, w_kd, c=c, workspace=ws_c)
+        with nvtx("gold_decompress"):
+            gw.gold_decompress(x0, c, w_ku, gamma, 1e-6, kd=kd, workspace=ws_d)
 
     for _ in range(3):
         call()
@@ -382,9 +416,9 @@ def gold_line(dev, world, steps, B=8, T=4096, D=2048, Dc=128):
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
     flops = 2 * N * D * Dc + 2 * N * (D + Dc) * D
     peak = bf16_peak()
-    line = {"workload": "gold_compress_decompress_1p5b", "N_tokens": N, "D": D, "Dc": Dc,
-            "io": "bf16", "steps": steps, "ms_per_call": ms,
-            "tokens_per_s": world * N / (ms / 1e3),
+    line = {"workload": f"gold_compress_decompress N{N} D{D} Dc{Dc}", "N_tokens": N, "D": D,
+            "Dc": Dc, "io": "bf16", "steps": steps, "ms_per_call": ms,
+            "value": world * N / (ms / 1e3), "unit": "tokens/s",
             "roofline": {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": peak,
                          "unit": "TFLOP/s", "frac": flops / (ms / 1e3) / 1e12 / peak,
                          "peak_source": "measured bf16_tflops (cuBLAS burst)",
@@ -464,8 +498,9 @@ def run_ours(args, world, rank, local):
     algo = args.algo
 
     def step():
-        gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], y=y, state_out=s_out, algo=algo,
-                        workspace=ws)
+        with nvtx("wkv6_prefill"):
+            gw.wkv6_prefill(*args_p, inp["u"], inp["state0"], y=y, state_out=s_out, algo=algo,
+                            workspace=ws)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -515,17 +550,17 @@ def run_ours(args, world, rank, local):
         "config": {"workload": "wkv6_prefill_1p5b_layer" + ("" if args.batch is None else f"_B{B}"),
                    "B": B, "T": T, "H": H, "D": D,
                    "io": "bf16", "state": "fp32", "algo": algo,
-                   "parallelism": f"dp{world} (independent batches, no collective)",
-                   "l2": "inputs larger than L2 (537 MB in, 134 MB out per step)"},
+                   "parallelism": f"dp{world}, independent batches, no collective",
+                   "l2": "inputs (537 MB) larger than L2, no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm,
                      "traffic": ncu_traffic("prefill", (B, T, H)) if chunked else None,
-                     "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                     "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": bytes_launch,
-                     "kernel": "wkv6 prefill (algo=%s): wkv6_fast_kernel + level kernel, "
-                               "timed together per call" % algo},
+                     "kernel": "wkv6_fast_kernel + wkv6_chunked_kernel, per call"},
         "gpu_launches": launches_per_step * args.steps,
     }
+    more = []   # the other measurements, printed compactly under "more"
 
     # decode: 100 steps back to back, state in place; GB/s of algorithmic bytes
     if not args.no_decode:
@@ -537,7 +572,8 @@ def run_ours(args, world, rank, local):
         dargs = [[dinp[n][s] for n in ("r", "k", "v", "omega")] for s in range(dsteps)]
 
         def dstep(s):
-            gw.wkv6_decode_step(*dargs[s], dinp["u"], state, y=ybuf)
+            with nvtx("wkv6_decode_step"):
+                gw.wkv6_decode_step(*dargs[s], dinp["u"], state, y=ybuf)
 
         for s in range(dsteps):
             dstep(s)
@@ -553,31 +589,30 @@ def run_ours(args, world, rank, local):
         dms = max_over_ranks(e0.elapsed_time(e1), world) / dsteps
         dbytes = decode_bytes(dcfg.B, dcfg.H, dcfg.D)
         dgbs = dbytes / (dms / 1e3) / 1e9
-        out["decode"] = {"metric": "decode GB/s", "value": dgbs * world, "unit": "GB/s",
-                         "per_gpu_gbs": dgbs, "ms_per_step": dms, "steps": dsteps,
-                         "config": {"workload": "wkv6_decode_step", "B": dcfg.B, "H": dcfg.H,
-                                    "D": dcfg.D, "io": "bf16", "state": "fp32 in place",
-                                    "l2": "state 134 MB > L2"},
-                         "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm,
-                                      "unit": "GB/s", "frac": dgbs / hbm,
-                                      "traffic": ncu_traffic("decode", (dcfg.B, dcfg.H)),
-                                      "algorithmic_bytes_per_launch": dbytes},
-                         "gpu_launches": dsteps}
+        # DRAM-only rate: the bytes ncu counted at DRAM per step (part of the state round
+        # trip is served from L2 between back-to-back steps) over the same time
+        dtraffic = ncu_traffic("decode", (dcfg.B, dcfg.H))
+        more.append({"workload": f"wkv6_decode_step B{dcfg.B} H{dcfg.H}", "ms_per_call": dms,
+                     "value": dgbs * world, "unit": "GB/s",
+                     "roofline": {"bound": "hbm", "frac": dgbs / hbm,
+                                  "dram_frac": None if dtraffic is None else
+                                  dtraffic / (dms / 1e3) / 1e9 / hbm}})
+
         del dinp, dargs, state
 
     # the other prefill shapes: long context (one sequence per head; the library splits it
     # into segments across SMs), the decay-extreme stress with LayerNorm, and the 1.5B layer
     # in Finch-C2's form and with base Finch's GroupNorm + gate
     if not args.no_other:
-        out["other_prefill"] = [other_prefill(W.CONFIGS[2], dev, world, hbm, args.algo, steps=5),
-                                other_prefill(W.CONFIGS[4], dev, world, hbm, args.algo, steps=5),
-                                other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
-                                              c2=True),
-                                other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10,
-                                              gn=True)]
-        out["backward"] = backward_line(W.CONFIGS[1], dev, world, steps=5)
-        out["backward_c2"] = backward_line(W.CONFIGS[1], dev, world, steps=5, c2=True)
-        out["gold"] = gold_line(dev, world, steps=10)
+        more += [other_prefill(W.CONFIGS[2], dev, world, hbm, args.algo, steps=5),
+                 other_prefill(W.CONFIGS[4], dev, world, hbm, args.algo, steps=5),
+                 other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10, c2=True),
+                 other_prefill(W.CONFIGS[1], dev, world, hbm, args.algo, steps=10, gn=True),
+                 backward_line(W.CONFIGS[1], dev, world, steps=5),
+                 backward_line(W.CONFIGS[1], dev, world, steps=5, c2=True),
+                 gold_line(dev, world, steps=10)]
+    if more:
+        out["more"] = [compact(m) for m in more]
 
     # end to end through the public API with host buffers: every step copies its inputs in
     # from pinned host memory and reads y and the final state back.  Steps are pipelined over
@@ -641,8 +676,7 @@ def run_ours(args, world, rank, local):
         etok = sum_over_ranks(float(B * T * e2e_steps), world)
         out["e2e"] = {"value": etok / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                      "note": "steps pipelined over two buffer sets (copy in / compute / copy out "
-                              "on separate streams)"}
+                      "note": "copy in / compute / copy out streams, 2 buffer sets"}
         del dbuf, ybuf, sbuf, wsb
 
     sampler.stop()
@@ -658,9 +692,8 @@ def run_ours(args, world, rank, local):
             tps, cores, secs1 = time_oracle(cfg, b_rows, t_tok, reps=reps)
             secs = secs1 * reps
         out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                               "sample": f"{b_rows} batch rows x {t_tok} tokens x {H} heads of "
-                                         f"the same workload, best of {reps} "
-                                         f"({secs:.1f} s of fp64 work in total)"}
+                               "sample": f"{b_rows} rows x {t_tok} tokens x {H} heads, best of "
+                                         f"{reps} ({secs:.1f} s of fp64 work)"}
     return out
 
 
