@@ -89,7 +89,7 @@ CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
                             "internal.h"),
-                "sha256_16": "70892a82047ac1bf", "bytes": 541468160 + 120561920,
+                "sha256_16": "386acc0d0af256f9", "bytes": 541149696 + 121576192,
                 "workload": (8, 4096, 32)},
     "decode": {"sources": ("decode.cu", "common.cuh"),
                "sha256_16": "8fb24cf16874f036", "bytes": 138433536 + 78408192,
