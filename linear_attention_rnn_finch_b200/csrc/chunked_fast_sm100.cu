@@ -233,10 +233,22 @@ __device__ __forceinline__ void store_state(uint8_t* tile, const float2 (&S0)[kP
     }
 }
 
+// The CTA's unit and the bounds its copies must stay in (checked in debug builds only).
+struct Unit {
+    int h, b, cseg, NC, T, H, B;
+    int* status;
+};
+// chunk n of the unit is a valid copy source: in the segment, the sequence and the tensor
+__device__ __forceinline__ bool copy_ok(const Unit& u, int n) {
+    return gw_check(u.status, n >= 0 && n < u.NC && (u.cseg + n) * C < u.T && u.h >= 0 &&
+                                  u.h < u.H && u.b >= 0 && u.b < u.B);
+}
+
 // r, k, omega tiles of chunk n into stage n % 3 (one thread)
 __device__ __forceinline__ void load_rkw(Smem& s, const CUtensorMap* tm_r, const CUtensorMap* tm_k,
-                                         const CUtensorMap* tm_w, int n, int cseg, int h, int b) {
-    const int st = n % kStagesRkw;
+                                         const CUtensorMap* tm_w, int n, const Unit& u) {
+    if (!copy_ok(u, n)) return;
+    const int st = n % kStagesRkw, cseg = u.cseg, h = u.h, b = u.b;
     ptx::mbar_arrive_expect_tx(&s.full_rkw[st], 3 * kTile);
     ptx::tma_load_4d(s.rkw[st][0], tm_r, &s.full_rkw[st], 0, h, (cseg + n) * C, b);
     ptx::tma_load_4d(s.rkw[st][1], tm_k, &s.full_rkw[st], 0, h, (cseg + n) * C, b);
@@ -244,8 +256,9 @@ __device__ __forceinline__ void load_rkw(Smem& s, const CUtensorMap* tm_r, const
     s.last_rkw[st] = n;
 }
 // v tile of chunk n into stage n % 4 (one thread)
-__device__ __forceinline__ void load_v(Smem& s, const CUtensorMap* tm_v, int n, int cseg, int h, int b) {
-    const int st = n % kStagesV;
+__device__ __forceinline__ void load_v(Smem& s, const CUtensorMap* tm_v, int n, const Unit& u) {
+    if (!copy_ok(u, n)) return;
+    const int st = n % kStagesV, cseg = u.cseg, h = u.h, b = u.b;
     ptx::mbar_arrive_expect_tx(&s.full_v[st], kTile);
     ptx::tma_load_4d(s.vt[st], tm_v, &s.full_v[st], 0, h, (cseg + n) * C, b);
     s.last_v[st] = n;
@@ -269,6 +282,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
     const int bh = unit % nbh, pseg = unit / nbh, b = bh / H, h = bh - (bh / H) * H;
     const int cseg = pseg * seg.seg_chunks;
     const int NC = min((T + C - 1) / C, cseg + seg.seg_chunks) - cseg;
+    const Unit cu{h, b, cseg, NC, T, H, nbh / H, status};
 
     if (tid == 0) {
         for (int i = 0; i < kStagesRkw; ++i) {
@@ -298,8 +312,8 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         ptx::prefetch_tensormap(&tm_v);
         ptx::prefetch_tensormap(&tm_w);
         // the first chunks' copies; later ones are issued as stages are released
-        for (int n = 0; n < min(NC, kStagesRkw); ++n) load_rkw(s, &tm_r, &tm_k, &tm_w, n, cseg, h, b);
-        for (int n = 0; n < min(NC, kStagesV); ++n) load_v(s, &tm_v, n, cseg, h, b);
+        for (int n = 0; n < min(NC, kStagesRkw); ++n) load_rkw(s, &tm_r, &tm_k, &tm_w, n, cu);
+        for (int n = 0; n < min(NC, kStagesV); ++n) load_v(s, &tm_v, n, cu);
     }
     if (warp == 0) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     ptx::tc_fence_before();
@@ -320,6 +334,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         const int cg = lane & 7, rr = lane >> 3;
         const int c0 = 8 * cg;
         const int tb = 16 * wg + 4 * rr;
+        gw_check(status, tb + 3 < C && c0 + 8 <= 64);   // this thread's tokens / channels
         float2 uu[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -530,7 +545,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             // every thread of the group has read stage st and written its operands
             named_bar(kBarPrep0 + g, kGroupThreads);
             if (leader) {
-                if (n + kStagesRkw < NC) load_rkw(s, &tm_r, &tm_k, &tm_w, n + kStagesRkw, cseg, h, b);
+                if (n + kStagesRkw < NC) load_rkw(s, &tm_r, &tm_k, &tm_w, n + kStagesRkw, cu);
                 // GU(n), SC(n): v of chunk n; DU read by the epilogue for chunk n-1; the SC
                 // buffer of parity pb read by A(n-2) (GA(n-2) waited for that).  Every wait
                 // gives up if the sequence was handed over at or before the chunk it serves.
@@ -577,6 +592,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         const int col0 = 32 * ch0, q0 = 4 * ch0;
         const int r0 = 16 * q + (lane >> 2), r1 = r0 + 8;
         const int cl = 2 * (lane & 3);
+        gw_check(status, r1 < C && col0 + 8 * (kPairs - 1) + cl + 2 <= 64);   // rows, columns
         const uint32_t cb = (uint32_t)(lane & 3) * 4;
         const uint32_t lane_h0 = (uint32_t)(32 * q) << 16, lane_h1 = (uint32_t)(32 * q + 16) << 16;
         const int hr0 = hi_row(r0), hr1 = hi_row(r1);
@@ -684,7 +700,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                                   y_raw, up0, up1);
                 // v stage (n+3) % 4 held v(n-1), read by GU(n-1) and GA(n-1), both complete
                 if (leader && n + kStagesV - 1 < NC && !stopped_at(s, n + kStagesV - 1))
-                    load_v(s, &tm_v, n + kStagesV - 1, cseg, h, b);
+                    load_v(s, &tm_v, n + kStagesV - 1, cu);
             }
             // S_n is in sb[(n+1) & 1] and Y[(n+1) & 1] (output(n-1)) has been read: RO(n+1)
             ptx::tc_fence_before();

@@ -176,8 +176,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
 
     auto issue_load = [&](int chunk) {
         const int st = (chunk - n0) % kStages;
-        ptx::mbar_arrive_expect_tx(&s.full[st], 4 * kTile);
         const int t0 = chunk * C;
+        if (!gw_check(status, chunk >= n0 && chunk < NC && t0 < T && h < H && b < nbh / H)) return;
+        ptx::mbar_arrive_expect_tx(&s.full[st], 4 * kTile);
         ptx::tma_load_4d(s.in[st][0], &tm_r, &s.full[st], 0, h, t0, b);
         ptx::tma_load_4d(s.in[st][1], &tm_k, &s.full[st], 0, h, t0, b);
         ptx::tma_load_4d(s.in[st][2], &tm_v, &s.full[st], 0, h, t0, b);
@@ -512,7 +513,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
         __syncthreads();
         if (s.abort) { failed = true; break; }
         if (tid == 0) {
-            if (y_raw == nullptr) {
+            if (y_raw == nullptr && gw_check(status, t0 >= 0 && t0 < T && h < H && b < nbh / H)) {
                 ptx::tma_store_4d(&tm_y, y_tile, 0, h, t0, b);
                 ptx::bulk_commit();
             }

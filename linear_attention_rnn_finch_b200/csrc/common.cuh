@@ -24,6 +24,19 @@ __device__ __forceinline__ float decay_from_logit(float omega) {
     return expf(-expf(omega));
 }
 
+// Debug builds (-DGW_DEBUG, built as libgoldwkv_debug.so): device-side checks of the
+// indices a copy or a store is about to use.  A failed check sets bit 1 of the kernel's
+// status word (*status |= 2) and the guarded access is skipped; nothing traps.  In release
+// builds the check is the constant true and costs nothing.
+#ifdef GW_DEBUG
+__device__ __forceinline__ bool gw_check(int* status, bool ok) {
+    if (!ok) atomicOr(status, 2);
+    return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool gw_check(int*, bool) { return true; }
+#endif
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

@@ -106,6 +106,8 @@ wkv6_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             for (int n = 0; n < NC; ++n) {
                 const int st = n % kStages;
                 if (n >= kStages && !wait_soft(s, &s.empty[st], (uint32_t)((n / kStages - 1) & 1), budget)) break;
+                // every chunk of a segment before the last is inside the sequence
+                if (!gw_check(status, pseg < P - 1 && h < H && b < nbh / H)) break;
                 ptx::mbar_arrive_expect_tx(&s.full[st], 3 * kTile);
                 ptx::tma_load_4d(s.in[st][0], &tm_k, &s.full[st], 0, h, (cseg + n) * C, b);
                 ptx::tma_load_4d(s.in[st][1], &tm_v, &s.full[st], 0, h, (cseg + n) * C, b);
