@@ -589,6 +589,31 @@ def run_ours(args, world, rank, local):
         dms = max_over_ranks(e0.elapsed_time(e1), world) / dsteps
         dbytes = decode_bytes(dcfg.B, dcfg.H, dcfg.D)
         dgbs = dbytes / (dms / 1e3) / 1e9
+        # the same steps with Finch-C2's LayerNorm over each row's H*D outputs, fused into the
+        # decode kernel (one launch per step; one zero-filled workspace for all steps)
+        g = torch.Generator(device=dev).manual_seed(dcfg.seed + 3)
+        lnp = (1.0 + 0.1 * torch.randn(dcfg.H * dcfg.D, generator=g, device=dev),
+               0.1 * torch.randn(dcfg.H * dcfg.D, generator=g, device=dev), 1e-5)
+        lnws = gw.new_workspace(gw.decode_workspace_bytes(dcfg.B, dcfg.H, dcfg.D, dcfg.dtype, True), dev)
+
+        def dstep_ln(s):
+            with nvtx("wkv6_decode_step"):
+                gw.wkv6_decode_step(*dargs[s], dinp["u"], state, ln=lnp, y=ybuf, workspace=lnws)
+
+        for s in range(dsteps):
+            dstep_ln(s)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0.record(stream)
+        for s in range(dsteps):
+            dstep_ln(s)
+        e1.record(stream)
+        e1.synchronize()
+        barrier(world)
+        dms_ln = max_over_ranks(e0.elapsed_time(e1), world) / dsteps
+        # + gamma and beta read once per step
+        dbytes_ln = dbytes + 2 * dcfg.H * dcfg.D * 4
+        dgbs_ln = dbytes_ln / (dms_ln / 1e3) / 1e9
         # DRAM-only rate: the bytes ncu counted at DRAM per step (part of the state round
         # trip is served from L2 between back-to-back steps) over the same time
         dtraffic = ncu_traffic("decode", (dcfg.B, dcfg.H))
@@ -597,8 +622,11 @@ def run_ours(args, world, rank, local):
                      "roofline": {"bound": "hbm", "frac": dgbs / hbm,
                                   "dram_frac": None if dtraffic is None else
                                   dtraffic / (dms / 1e3) / 1e9 / hbm}})
+        more.append({"workload": f"wkv6_decode_step_layernorm B{dcfg.B} H{dcfg.H} (one kernel)",
+                     "ms_per_call": dms_ln, "value": dgbs_ln * world, "unit": "GB/s",
+                     "roofline": {"bound": "hbm", "frac": dgbs_ln / hbm}})
 
-        del dinp, dargs, state
+        del dinp, dargs, state, lnws
 
     # the other prefill shapes: long context (one sequence per head; the library splits it
     # into segments across SMs), the decay-extreme stress with LayerNorm, and the 1.5B layer

@@ -128,7 +128,8 @@ wkv_status wkv6_prefill_algo(const void *r, const void *k, const void *v, const 
  */
 wkv_status wkv6_workspace_status(void *workspace, void *stream);
 
-/* Bytes of device workspace wkv6_decode_step needs (non-zero only with LayerNorm). */
+/* Bytes of device workspace wkv6_decode_step needs (non-zero only with LayerNorm): a block
+ * of B row counters (256-byte aligned size), then, with bf16 I/O, B*H*D fp32 outputs. */
 size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln);
 
 /*
@@ -137,7 +138,11 @@ size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_l
  * (autoregressive generation) applied to the recurrence above.
  *   r, k, v, omega  [B][H][D] io;  u [H][D] fp32;  state [B][H][D][D] fp32 (read, then
  *   overwritten with the new state);  y [B][H][D] io (LayerNorm-ed when ln != NULL).
- *   workspace: at least wkv6_decode_workspace_bytes(...) bytes.
+ *   workspace: at least wkv6_decode_workspace_bytes(...) bytes (none without LayerNorm).
+ * One kernel launch, LayerNorm included: the last CTA of each batch row to finish
+ * normalises the row.  With LayerNorm the workspace's row counters (its first bytes) must
+ * be zero before the first call on it (zero-fill new workspace); every call leaves them
+ * zero, so one workspace serves any number of steps, in stream order.
  */
 wkv_status wkv6_decode_step(const void *r, const void *k, const void *v, const void *omega,
                             const float *u, float *state, void *y, int B, int H, int D,
@@ -204,8 +209,9 @@ wkv_status wkv6_prefill_gn(const void *r, const void *k, const void *v, const vo
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /* wkv6_decode_step_gn: as wkv6_decode_step with the GroupNorm + gate output stage (gn
- * required; gate [B][H][D] io or NULL).  Workspace: wkv6_decode_workspace_bytes(B, H, D,
- * io, 1). */
+ * required; gate [B][H][D] io or NULL), in the same kernel (each head is normalised by the
+ * CTA that computes it).  No workspace is needed (workspace may be NULL); one of
+ * wkv6_decode_workspace_bytes(B, H, D, io, 1) bytes is accepted. */
 wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, const void *omega,
                                const float *u, float *state, void *y, int B, int H, int D,
                                wkv_dtype io, const wkv_gn *gn, void *workspace,

@@ -304,7 +304,7 @@ def wkv6c2_decode_step(r, k, v, omega, uprime, state, *, ln=None, y=None, worksp
     ln_s, ln_p = _ln_struct(ln, H, D, dev)
     need = int(L.wkv6_decode_workspace_bytes(B, H, D, _io(dt), int(ln is not None)))
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = new_workspace(need, dev)   # zero: LayerNorm row counters
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         st = L.wkv6c2_decode_step(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(uprime), _ptr(state),
@@ -348,7 +348,7 @@ def wkv6_decode_step(r, k, v, omega, u, state, *, ln=None, y=None, workspace=Non
     ln_s, ln_p = _ln_struct(ln, H, D, dev)
     need = int(L.wkv6_decode_workspace_bytes(B, H, D, _io(dt), int(ln is not None)))
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = new_workspace(need, dev)   # zero: LayerNorm row counters
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         st = L.wkv6_decode_step(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state),
@@ -426,9 +426,7 @@ def wkv6_decode_step_gn(r, k, v, omega, u, state, *, gn, y=None, workspace=None,
         y = torch.empty((B, H, D), dtype=dt, device=dev)
     _check("y", y, dev, dt, (B, H, D))
     gn_s, gn_p = _gn_struct(gn, H, D, dev, dt, (B, H, D))
-    need = int(L.wkv6_decode_workspace_bytes(B, H, D, _io(dt), 1))
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    # the GroupNorm stage runs inside the decode kernel: no workspace
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         st = L.wkv6_decode_step_gn(_ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(state),

@@ -213,6 +213,13 @@ size_t handoff_state_bytes(long units) { return (size_t)units * 64 * 64 * sizeof
 size_t segment_bytes(int B, int H, int P) {
     return (size_t)B * H * (P - 1) * (64 * 64 + 64) * sizeof(float);
 }
+// LayerNorm decode workspace: the per-row counters (zero between calls), then, with bf16
+// output, the fp32 outputs of the step ([B][H][D]) that the row's last CTA normalises
+size_t decode_counter_bytes(int B) { return round256((size_t)B * sizeof(int)); }
+size_t decode_ln_bytes(int B, int H, wkv_dtype io) {
+    return decode_counter_bytes(B) + (io == WKV_BF16 ? (size_t)B * H * kHeadSizeApi * sizeof(float) : 0);
+}
+
 size_t chunked_bytes(int B, int H, int P) {
     const long units = (long)B * H * P;
     return kStatusBytes + handoff_ints_bytes(units) + handoff_state_bytes(units) +
@@ -267,9 +274,8 @@ size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, in
 }
 
 size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln) {
-    if (B <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
-    if (with_ln && io == WKV_BF16) return (size_t)B * H * D * sizeof(float);
-    return 0;
+    if (B <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io) || !with_ln) return 0;
+    return decode_ln_bytes(B, H, io);
 }
 
 }  // extern "C"
@@ -452,7 +458,8 @@ wkv_status decode_impl(const void* r, const void* k, const void* v, const void* 
     for (const Span& in : ins)
         if (overlaps(sy, in) || overlaps(ss, in)) return WKV_ERR_INVALID_ARG;
 
-    const size_t need = wkv6_decode_workspace_bytes(B, H, D, io, nm.on());
+    // LayerNorm needs the row counters (and bf16 staging); GroupNorm runs inside the kernel
+    const size_t need = nm.kind == Norm::kLayer ? decode_ln_bytes(B, H, io) : 0;
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
         const Span sw = span(workspace, need);
@@ -463,14 +470,15 @@ wkv_status decode_impl(const void* r, const void* k, const void* v, const void* 
     if (injected("launch")) return WKV_ERR_CUDA;
 
     const bool bf16 = io == WKV_BF16;
-    float* y_raw = nullptr;
-    if (nm.on()) y_raw = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(y);
-    cudaError_t e = goldwkv::launch_decode(r, k, v, omega, u, state, y, y_raw, B, H, bf16,
-                                           goldwkv::Variant{uprime}, st);
-    if (e != cudaSuccess) return WKV_ERR_CUDA;
-    if (nm.on() && launch_norm(nm, y_raw, y, (long)B, H, D, bf16, st) != cudaSuccess)
-        return WKV_ERR_CUDA;
-    return WKV_OK;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    goldwkv::DecodeOut out{nm.kind == Norm::kLayer ? 1 : nm.kind == Norm::kGroup ? 2 : 0,
+                           nm.gamma, nm.beta, nm.eps, nm.gate,
+                           nm.kind == Norm::kLayer ? reinterpret_cast<int*>(ws) : nullptr,
+                           nm.kind == Norm::kLayer && bf16
+                               ? reinterpret_cast<float*>(ws + decode_counter_bytes(B))
+                               : nullptr};
+    return from_cuda(goldwkv::launch_decode(r, k, v, omega, u, state, y, out, B, H, bf16,
+                                            goldwkv::Variant{uprime}, st));
 }
 
 }  // namespace

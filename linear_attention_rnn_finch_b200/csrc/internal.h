@@ -24,10 +24,24 @@ cudaError_t launch_recurrent(const void* r, const void* k, const void* v, const 
                              float* y_raw, int B, int T, int H, bool bf16, Variant var,
                              cudaStream_t st);
 
-// One decode step, state in place.  y_raw as above.
+// Output stage of a decode step: kind 0 none, 1 LayerNorm over each batch row's H*64
+// outputs, 2 per-head GroupNorm times an optional gate (dtype io, layout of y).  LayerNorm:
+// row_count [B] ints, zero before the call and left zero; y_raw [B][H][D] fp32 staging
+// (null: y itself, fp32 I/O).
+struct DecodeOut {
+    int kind;
+    const float* gamma;
+    const float* beta;
+    float eps;
+    const void* gate;
+    int* row_count;
+    float* y_raw;
+};
+
+// One decode step, state in place, with its output stage fused.
 cudaError_t launch_decode(const void* r, const void* k, const void* v, const void* omega,
-                          const float* u, float* state, void* y, float* y_raw, int B, int H,
-                          bool bf16, Variant var, cudaStream_t st);
+                          const float* u, float* state, void* y, const DecodeOut& out, int B,
+                          int H, bool bf16, Variant var, cudaStream_t st);
 
 // LayerNorm of `rows` rows of C fp32 values into `out` (fp32 or bf16); out may equal x.
 cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const float* beta,

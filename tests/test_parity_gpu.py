@@ -333,3 +333,29 @@ def test_layernorm_small_f32(oracle):
     yo, so = _oracle_full(oracle, inp, ln=True)
     assert rel_err(y, yo) <= TOL[torch.float32]
     assert rel_err(s, so) <= TOL[torch.float32]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_layernorm_one_kernel_reused_workspace(oracle, dtype):
+    """Decode with LayerNorm runs as one kernel: the last CTA of each batch row normalises
+    it and resets the row's counter.  One zero-filled workspace serves 6 steps in a row
+    (B=5 rows, H=12 heads, so rows do not fill a wave evenly), its counters are zero after
+    each step, and y and the state match the oracle at every step."""
+    cfg = W.CONFIGS[3].with_(seed=9500, B=5, H=12, io="f32" if dtype == torch.float32 else "bf16")
+    inp = W.make_decode_inputs(cfg, "cuda", steps=6)
+    B, H, D = 5, 12, 64
+    g = torch.Generator(device="cuda").manual_seed(9501)
+    gamma = 1.0 + 0.1 * torch.randn(H * D, generator=g, device="cuda")
+    beta = 0.1 * torch.randn(H * D, generator=g, device="cuda")
+    ws = gw.new_workspace(gw.decode_workspace_bytes(B, H, D, dtype, True), "cuda")
+    state = inp["state0"].clone()
+    st_o = f64(inp["state0"])
+    for t in range(6):
+        a = [inp[n][t] for n in ("r", "k", "v", "omega")]
+        y = gw.wkv6_decode_step(*a, inp["u"], state, ln=(gamma, beta, 1e-5), workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:4 * B].view(torch.int32).abs().sum()) == 0
+        yo, st_o = oracle.decode_step(*[f64(x) for x in a], f64(inp["u"]), st_o)
+        yo = oracle.layernorm(yo.reshape(B, H * D), f64(gamma), f64(beta), 1e-5).reshape(B, H, D)
+        assert rel_err(y, yo) <= TOL[dtype]
+        assert rel_err(state, st_o) <= TOL[dtype]
