@@ -286,11 +286,16 @@ wkv_status wkv6c2_backward(const void *r, const void *k, const void *v, const vo
  * each linear map (the layout of a linear layer's weight, [out][in]):
  *   x, x0 [N][D];  c [N][Dc];  kd [N][D];  w_kd [Dc][D] (w_kd[j][i] = W_KD[i][j]);
  *   w_ku [D][D + Dc] (w_ku[o][i] = W_KU[i][o]);  gamma [D] fp32 or NULL (= 1).
- * The products run on the tensor cores through cuBLASLt with fp32 accumulation (c is
- * rounded to bf16 once).  D and Dc must be multiples of 8 and D <= 16384 (else
- * WKV_ERR_UNSUPPORTED), N <= 2^31 - 1.  Outputs may not overlap inputs or the workspace.  Workspace: at least
- * gold_*_workspace_bytes(...) bytes, any contents; for decompression it holds the
- * concatenation [x0 | c] (bf16) and the fp32 product before RMSNorm.  eps must be > 0.
+ * The products run on the tensor cores in the library's own tcgen05 GEMM, with fp32
+ * accumulation (c is rounded to bf16 once); decompression reads x0 and c in place (no
+ * concatenated copy) and, for D <= 2048, applies RMSNorm to the fp32 product inside the
+ * same kernel (the CTAs of a row block exchange their partial sums of squares); wider D
+ * writes the fp32 product to the workspace and normalises it in a second kernel.  D and
+ * Dc must be multiples of 8 and D <= 16384 (else WKV_ERR_UNSUPPORTED), N <= 2^31 - 1.
+ * Outputs may not overlap inputs or the workspace.  Workspace: at least
+ * gold_*_workspace_bytes(...) bytes; its first 4 bytes are a status word that the kernel
+ * sets if one of its bounded waits expires (the outputs are then undefined), read and
+ * cleared by wkv6_workspace_status -- zero-fill new workspace to use it.  eps must be > 0.
  */
 size_t gold_compress_workspace_bytes(long N, int D, int Dc);
 wkv_status gold_compress(const void *x, const void *w_kd, void *c, long N, int D, int Dc,

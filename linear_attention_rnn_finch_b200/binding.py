@@ -494,7 +494,7 @@ def gold_compress(x, w_kd, *, c=None, workspace=None, stream=None):
     _check("c", c, dev, torch.bfloat16, (*x.shape[:-1], Dc))
     need = int(L.gold_compress_workspace_bytes(N, D, Dc))
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = new_workspace(need, dev)   # zero: status word
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         st = L.gold_compress(_ptr(x), _ptr(w_kd), _ptr(c), N, D, Dc, _ptr(workspace), ws_bytes,
@@ -523,7 +523,7 @@ def gold_decompress(x0, c, w_ku, gamma=None, eps=1e-6, *, kd=None, workspace=Non
     _check("kd", kd, dev, torch.bfloat16, tuple(x0.shape))
     need = int(L.gold_decompress_workspace_bytes(N, D, Dc))
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = new_workspace(need, dev)   # zero: status word
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         st = L.gold_decompress(_ptr(x0), _ptr(c), _ptr(w_ku), _ptr(gamma), float(eps), _ptr(kd),

@@ -78,8 +78,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
     with cf.ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 1)) as ex:
         objs = list(ex.map(lambda s: _compile(s, ptxas_info, verbose, debug), srcs))
     tmp = lib.with_suffix(".so.tmp")
-    # cuBLASLt serves the plain GEMMs of the GOLD compression entry points
-    cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *map(str, objs), "-lcublasLt"]
+    cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *map(str, objs)]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)

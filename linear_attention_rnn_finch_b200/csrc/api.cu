@@ -719,7 +719,9 @@ wkv_status wkv6c2_backward(const void* r, const void* k, const void* v, const vo
 
 namespace {
 
-constexpr size_t kLtWorkspace = (size_t)32 << 20;   // cuBLASLt workspace per call
+// GOLD workspaces start with the status word the tensor-core GEMM sets when a bounded wait
+// expires (read and cleared by wkv6_workspace_status)
+constexpr size_t kGoldStatusBytes = 256;
 
 // Sizes the GOLD entry points take: 16-byte rows of bf16 (D, Dc multiples of 8), N within
 // the GEMMs' int range.
@@ -735,14 +737,14 @@ extern "C" {
 
 size_t gold_compress_workspace_bytes(long N, int D, int Dc) {
     if (check_gold_sizes(N, D, Dc) != WKV_OK || N == 0) return 0;
-    return kLtWorkspace;
+    return kGoldStatusBytes;
 }
 
 size_t gold_decompress_workspace_bytes(long N, int D, int Dc) {
     if (check_gold_sizes(N, D, Dc) != WKV_OK || N == 0) return 0;
-    // fp32 product, the bf16 concatenation [x0 | c], cuBLASLt's workspace
-    return round256((size_t)N * D * sizeof(float)) + round256((size_t)N * (D + Dc) * 2) +
-           kLtWorkspace;
+    // status word; the fp32 product only when D is too wide for the fused RMSNorm
+    return kGoldStatusBytes +
+           (goldwkv::gold_rmsnorm_fusable(D) ? 0 : round256((size_t)N * D * sizeof(float)));
 }
 
 wkv_status gold_compress(const void* x, const void* w_kd, void* c, long N, int D, int Dc,
@@ -761,10 +763,10 @@ wkv_status gold_compress(const void* x, const void* w_kd, void* c, long N, int D
         overlaps(sw, span(x, xb)) || overlaps(sw, span(w_kd, wb)))
         return WKV_ERR_INVALID_ARG;
     if (injected("launch")) return WKV_ERR_CUDA;
-    return goldwkv::gold_gemm_compress(x, w_kd, c, N, D, Dc, workspace, need,
-                                       reinterpret_cast<cudaStream_t>(stream))
-               ? WKV_OK
-               : WKV_ERR_CUDA;
+    const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+    return from_cuda(goldwkv::gold_gemm(x, D, nullptr, 0, w_kd, Dc, N, goldwkv::GoldOut::kBf16, c,
+                                        nullptr, 0.f, static_cast<int*>(workspace), budget,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 wkv_status gold_decompress(const void* x0, const void* c, const void* w_ku, const float* gamma,
@@ -790,11 +792,17 @@ wkv_status gold_decompress(const void* x0, const void* c, const void* w_ku, cons
     if (injected("launch")) return WKV_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    float* z = reinterpret_cast<float*>(ws);
-    uint8_t* cat = ws + round256((size_t)N * D * sizeof(float));
-    void* lt = cat + round256((size_t)N * (D + Dc) * 2);
-    if (!goldwkv::gold_gemm_decompress(x0, c, w_ku, cat, z, N, D, Dc, lt, kLtWorkspace, st))
-        return WKV_ERR_CUDA;
+    int* status = reinterpret_cast<int*>(ws);
+    const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+    // one GEMM over [x0 | c] (the two are never concatenated in memory)
+    if (goldwkv::gold_rmsnorm_fusable(D))
+        return from_cuda(goldwkv::gold_gemm(x0, D, c, Dc, w_ku, D, N,
+                                            goldwkv::GoldOut::kRmsNormBf16, kd, gamma, eps,
+                                            status, budget, st));
+    float* z = reinterpret_cast<float*>(ws + kGoldStatusBytes);
+    cudaError_t e = goldwkv::gold_gemm(x0, D, c, Dc, w_ku, D, N, goldwkv::GoldOut::kF32, z,
+                                       nullptr, 0.f, status, budget, st);
+    if (e != cudaSuccess) return WKV_ERR_CUDA;
     return from_cuda(goldwkv::launch_rmsnorm_rows(z, gamma, eps, kd, N, D, st));
 }
 

@@ -586,6 +586,22 @@ bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H) {
            CUDA_SUCCESS;
 }
 
+// [rows][cols] bf16, row stride `row_bytes` (a multiple of 16); box = 64 columns x
+// box_rows rows, 128-byte swizzle.  Elements outside the matrix read as zeros.
+bool make_matrix_map(CUtensorMap* m, const void* base, long rows, long cols, long row_bytes,
+                     int box_rows) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 size_t chunked_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,

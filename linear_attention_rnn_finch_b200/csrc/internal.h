@@ -57,6 +57,10 @@ cudaError_t launch_groupnorm_gate(const float* x, const float* gamma, const floa
 // ---- chunked tensor-core prefill (bf16 I/O)
 // TMA descriptor of a [B][T][H][64] bf16 tensor: box 64 channels x 1 head x 64 tokens.
 bool make_token_map(CUtensorMap* m, const void* base, int B, int T, int H);
+// TMA descriptor of a [rows][cols] bf16 matrix, row stride row_bytes: box 64 columns x
+// box_rows rows, 128-byte swizzle, zeros outside the matrix.
+bool make_matrix_map(CUtensorMap* m, const void* base, long rows, long cols, long row_bytes,
+                     int box_rows);
 
 // Sequence split.  Every (b,h) sequence is cut into P segments of seg_chunks 64-token
 // chunks (the last one may be shorter); the kernels below run one CTA per unit

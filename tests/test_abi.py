@@ -94,11 +94,11 @@ def test_backward_and_gold_workspace_queries():
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16, c2=True) == base16
     assert binding.backward_workspace_bytes(B, 0, H, 64, torch.bfloat16) == 0
     assert binding.load().wkv6_backward_workspace_bytes(B, T, H, 32, 1) == 0
-    # GOLD: cuBLASLt workspace (32 MiB); decompression adds the fp32 product and [x0 | c]
-    lt = 32 << 20
-    assert binding.load().gold_compress_workspace_bytes(1000, 256, 16) == lt
-    assert binding.load().gold_decompress_workspace_bytes(1000, 256, 16) == \
-        r256(1000 * 256 * 4) + r256(1000 * 272 * 2) + lt
+    # GOLD: a 256-byte status block; decompression wider than one cluster of column tiles
+    # (D > 2048) adds the fp32 product
+    assert binding.load().gold_compress_workspace_bytes(1000, 256, 16) == 256
+    assert binding.load().gold_decompress_workspace_bytes(1000, 256, 16) == 256
+    assert binding.load().gold_decompress_workspace_bytes(1000, 4096, 256) == 256 + r256(1000 * 4096 * 4)
     assert binding.load().gold_compress_workspace_bytes(0, 256, 16) == 0
     assert binding.load().gold_decompress_workspace_bytes(10, 100, 16) == 0    # D % 8 != 0
 

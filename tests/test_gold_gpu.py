@@ -104,3 +104,37 @@ def test_gold_argument_checks():
     assert bool((kd == 3.0).all())
     assert dec(kd) == bd.WKV_OK
     assert L.gold_compress(vp(x0), vp(w_kd), vp(c), 0, D, Dc, None, 0, stream) == bd.WKV_OK
+
+
+@pytest.mark.parametrize("N,D,Dc", [(257, 1000, 40), (130, 4096, 256), (64, 136, 8)])
+def test_odd_widths(oracle, N, D, Dc):
+    """Widths that are not multiples of the GEMM's tiles: D = 1000 (a partial last column
+    tile, a 4-CTA cluster for the fused RMSNorm), Dc = 40 and 8 (a partial k-block of c, a
+    partial column tile of the compression), D = 4096 (wider than one cluster: the fp32
+    product and a separate RMSNorm), ragged N."""
+    w_kd, w_ku, g = _weights(10100 + D, D, Dc)
+    x, x0 = _acts(10101 + D, (N, D)), _acts(10102 + D, (N, D))
+    c = gw.gold_compress(x, w_kd)
+    kd = gw.gold_decompress(x0, c, w_ku, g, 1e-6)
+    torch.cuda.synchronize()
+    assert rel_err(c, oracle.gold_compress(f64(x), f64(w_kd))) <= TOL_BF16
+    want = oracle.gold_decompress(f64(x0), f64(c), f64(w_ku), f64(g), 1e-6)
+    assert rel_err(kd, want) <= TOL_BF16
+
+
+def test_gemm_wait_timeout_is_reported(monkeypatch):
+    """A zero spin budget makes the GEMM's bounded waits expire: the workspace status word
+    reports it once, and the next call (normal budget) is correct and reports nothing."""
+    N, D, Dc = 300, 512, 32
+    w_kd, w_ku, g = _weights(10200, D, Dc)
+    x0, c = _acts(10201, (N, D)), _acts(10202, (N, Dc))
+    ws = bd.new_workspace(bd.load().gold_decompress_workspace_bytes(N, D, Dc), DEV)
+    monkeypatch.setenv("GOLDWKV_FAULT", "timeout0")
+    gw.gold_decompress(x0, c, w_ku, g, 1e-6, workspace=ws)
+    assert bd.workspace_status(ws) == bd.WKV_ERR_TIMEOUT
+    monkeypatch.delenv("GOLDWKV_FAULT")
+    kd = gw.gold_decompress(x0, c, w_ku, g, 1e-6, workspace=ws)
+    assert bd.workspace_status(ws) == bd.WKV_OK
+    kd2 = gw.gold_decompress(x0, c, w_ku, g, 1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(kd, kd2)
