@@ -89,10 +89,10 @@ CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
                             "internal.h"),
-                "sha256_16": "386acc0d0af256f9", "bytes": 541149696 + 121576192,
+                "sha256_16": "e2abf82448988e28", "bytes": 541158912 + 118494464,
                 "workload": (8, 4096, 32)},
     "decode": {"sources": ("decode.cu", "common.cuh"),
-               "sha256_16": "8fb24cf16874f036", "bytes": 138433536 + 78408192,
+               "sha256_16": "0468671fdbdebeab", "bytes": 138433024 + 78395392,
                "workload": (256, 32)},
 }
 
