@@ -128,6 +128,41 @@ wkv_status wkv6_prefill_algo(const void *r, const void *k, const void *v, const 
  */
 wkv_status wkv6_workspace_status(void *workspace, void *stream);
 
+/*
+ * Splitting one sequence across devices (the state-passing form of the page's pre-fill,
+ * section 3.4 "Training and Inference Procedures": the state carried from one span of
+ * tokens to the next reproduces the single pass).  Rank p of P holds tokens
+ * [p*T, (p+1)*T) of every (b,h) sequence:
+ *   1. wkv6_segment_summary on its tokens: the state they build from a zero state, S_p,
+ *      and each channel's total log2 decay over them, g_p = sum_t log2 w_t;
+ *   2. exchange (S_p, g_p) between the ranks (one all-gather);
+ *   3. wkv6_segment_carry: the state entering every segment, s_in[p + 1] =
+ *      diag(2^g_p) s_in[p] + S_p from the sequence's initial state s_in[0];
+ *   4. wkv6_prefill of its tokens from s_in[p].
+ *
+ * wkv6_segment_summary: k, v, omega [B][T][H][D] bf16 (as for wkv6_prefill; c2 != 0 takes
+ * Finch-C2's normalised key k (1 - w)), T a multiple of 64 (chunk-aligned segments; else
+ * WKV_ERR_UNSUPPORTED).  Outputs s_loc [B][H][D][D] fp32 and log2_decay [B][H][D] fp32.
+ * Workspace: wkv6_segment_summary_workspace_bytes(...) bytes whose first word is the status
+ * word of wkv6_workspace_status (zero-fill new workspace).  Runs on the tensor cores with
+ * factors <= 1 only, so any decay is taken.  T == 0 writes the zero state and no decay.
+ */
+size_t wkv6_segment_summary_workspace_bytes(int B, int T, int H, int D);
+wkv_status wkv6_segment_summary(const void *k, const void *v, const void *omega, int c2,
+                                float *s_loc, float *log2_decay, int B, int T, int H, int D,
+                                wkv_dtype io, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
+ * wkv6_segment_carry: P segments' summaries laid out segment-major, s_loc [P][B][H][D][D]
+ * and log2_decay [P][B][H][D] (rank p's in slot p, as an all-gather leaves them), and the
+ * sequence's initial state state0 [B][H][D][D] (NULL: zero).  Writes s_in [P + 1][B][H][D][D]:
+ * s_in[0] = state0, s_in[p + 1] = 2^log2_decay[p] (rows) * s_in[p] + s_loc[p] -- the state
+ * entering segment p, and s_in[P] the state after the last.  fp32; no workspace.
+ */
+wkv_status wkv6_segment_carry(const float *state0, const float *s_loc, const float *log2_decay,
+                              float *s_in, int P, int B, int H, int D, void *stream);
+
 /* Bytes of device workspace wkv6_decode_step needs (non-zero only with LayerNorm): a block
  * of B row counters (256-byte aligned size), then, with bf16 I/O, B*H*D fp32 outputs. */
 size_t wkv6_decode_workspace_bytes(int B, int H, int D, wkv_dtype io, int with_ln);

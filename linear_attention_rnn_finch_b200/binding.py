@@ -63,6 +63,12 @@ def load(path: Path | str | None = None):
     L.wkv6_prefill_static.restype = i
     L.wkv6_prefill_static_status.argtypes = [vp]
     L.wkv6_prefill_static_status.restype = i
+    L.wkv6_segment_summary_workspace_bytes.argtypes = [i, i, i, i]
+    L.wkv6_segment_summary_workspace_bytes.restype = sz
+    L.wkv6_segment_summary.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, vp, sz, vp]
+    L.wkv6_segment_summary.restype = i
+    L.wkv6_segment_carry.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
+    L.wkv6_segment_carry.restype = i
     L.wkv6c2_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
     L.wkv6c2_prefill.restype = i
     L.wkv6c2_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
@@ -245,6 +251,53 @@ def prefill_static_status(device=None, stream=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         return int(load().wkv6_prefill_static_status(_stream_ptr(dev, stream)))
+
+
+def segment_summary(k, v, omega, *, c2=False, workspace=None, stream=None):
+    """State that k, v, omega [B, T, H, D] bf16 (T a multiple of 64) build from a zero state,
+    [B, H, D, D] fp32, and each channel's total log2 decay over them, [B, H, D] fp32
+    (include/goldwkv.h, wkv6_segment_summary)."""
+    L = load()
+    if k.dim() != 4:
+        raise ValueError("k must be [B, T, H, D]")
+    B, T, H, D = k.shape
+    dev = k.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (no CPU implementation)")
+    for name, t in (("k", k), ("v", v), ("omega", omega)):
+        _check(name, t, dev, torch.bfloat16, (B, T, H, D))
+    s_loc = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    g = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    need = int(L.wkv6_segment_summary_workspace_bytes(B, T, H, D))
+    if workspace is None and need > 0:
+        workspace = new_workspace(need, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = L.wkv6_segment_summary(_ptr(k), _ptr(v), _ptr(omega), int(bool(c2)), _ptr(s_loc),
+                                    _ptr(g), B, T, H, D, WKV_BF16, _ptr(workspace), ws_bytes,
+                                    _stream_ptr(dev, stream))
+    _raise("wkv6_segment_summary", st)
+    return s_loc, g
+
+
+def segment_carry(s_loc, log2_decay, state0=None, *, stream=None):
+    """States entering P segments from their summaries stacked segment-major, s_loc
+    [P, B, H, D, D] and log2_decay [P, B, H, D]: returns [P + 1, B, H, D, D], entry p the
+    state entering segment p and entry P the final state (include/goldwkv.h,
+    wkv6_segment_carry)."""
+    L = load()
+    P, B, H, D, _ = s_loc.shape
+    dev = s_loc.device
+    _check("s_loc", s_loc, dev, torch.float32, (P, B, H, D, D))
+    _check("log2_decay", log2_decay, dev, torch.float32, (P, B, H, D))
+    if state0 is not None:
+        _check("state0", state0, dev, torch.float32, (B, H, D, D))
+    s_in = torch.empty((P + 1, B, H, D, D), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = L.wkv6_segment_carry(_ptr(state0), _ptr(s_loc), _ptr(log2_decay), _ptr(s_in), P, B,
+                                  H, D, _stream_ptr(dev, stream))
+    _raise("wkv6_segment_carry", st)
+    return s_in
 
 
 def wkv6c2_prefill(r, k, v, omega, uprime, state_in=None, *, ln=None, y=None, state_out=None,

@@ -504,6 +504,78 @@ wkv_status wkv6c2_prefill(const void* r, const void* k, const void* v, const voi
                         layer_norm(ln), WKV_ALGO_AUTO, workspace, workspace_bytes, stream);
 }
 
+size_t wkv6_segment_summary_workspace_bytes(int B, int T, int H, int D) {
+    if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || T % kChunk != 0) return 0;
+    return kStatusBytes;
+}
+
+wkv_status wkv6_segment_summary(const void* k, const void* v, const void* omega, int c2,
+                                float* s_loc, float* log2_decay, int B, int T, int H, int D,
+                                wkv_dtype io, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    if (B < 0 || T < 0 || H < 0 || !valid_io(io)) return WKV_ERR_INVALID_ARG;
+    if (D != kHeadSizeApi || io != WKV_BF16 || T % kChunk != 0) return WKV_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return WKV_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t xbytes = (size_t)B * T * H * D * 2;
+    const size_t sbytes = (size_t)B * H * D * D * sizeof(float), gbytes = (size_t)B * H * D * sizeof(float);
+    const bool tokens = T > 0;
+    Buf bufs[] = {{k, xbytes, tokens}, {v, xbytes, tokens}, {omega, xbytes, tokens},
+                  {s_loc, sbytes, true}, {log2_decay, gbytes, true},
+                  {workspace, workspace_bytes, false}};
+    wkv_status s = check_bufs(bufs, 6);
+    if (s != WKV_OK) return s;
+    const size_t need = tokens ? wkv6_segment_summary_workspace_bytes(B, T, H, D) : 0;
+    const Span outs[] = {span(s_loc, sbytes), span(log2_decay, gbytes), span(workspace, need)};
+    const Span ins[] = {span(k, tokens ? xbytes : 0), span(v, tokens ? xbytes : 0),
+                        span(omega, tokens ? xbytes : 0)};
+    for (int a = 0; a < 3; ++a) {
+        for (const Span& in : ins)
+            if (overlaps(outs[a], in)) return WKV_ERR_INVALID_ARG;
+        for (int b2 = a + 1; b2 < 3; ++b2)
+            if (overlaps(outs[a], outs[b2])) return WKV_ERR_INVALID_ARG;
+    }
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return WKV_ERR_WORKSPACE;
+    if (injected("launch")) return WKV_ERR_CUDA;
+    if (!tokens) {   // no tokens: the zero state and no decay
+        if (cudaMemsetAsync(s_loc, 0, sbytes, st) != cudaSuccess ||
+            cudaMemsetAsync(log2_decay, 0, gbytes, st) != cudaSuccess)
+            return WKV_ERR_CUDA;
+        return WKV_OK;
+    }
+    CUtensorMap maps[4];
+    if (!goldwkv::make_token_map(&maps[1], k, B, T, H) ||
+        !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
+        !goldwkv::make_token_map(&maps[3], omega, B, T, H))
+        return WKV_ERR_CUDA;
+    maps[0] = maps[1];   // r is not read
+    const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+    // the whole sequence is "segment 0 of 2": its state from zero and its log2 decay
+    const goldwkv::Segments seg{2, T / kChunk, nullptr};
+    return from_cuda(goldwkv::launch_segment_states(maps, s_loc, log2_decay, B, T, H, seg,
+                                                    goldwkv::Variant{c2 ? k : nullptr},
+                                                    static_cast<int*>(workspace), budget, st));
+}
+
+wkv_status wkv6_segment_carry(const float* state0, const float* s_loc, const float* log2_decay,
+                              float* s_in, int P, int B, int H, int D, void* stream) {
+    if (P < 0 || B < 0 || H < 0) return WKV_ERR_INVALID_ARG;
+    if (D != kHeadSizeApi) return WKV_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return WKV_OK;
+    const size_t one = (size_t)B * H * D * D * sizeof(float), g1 = (size_t)B * H * D * sizeof(float);
+    Buf bufs[] = {{state0, one, false}, {s_loc, one * P, P > 0}, {log2_decay, g1 * P, P > 0},
+                  {s_in, one * (P + 1), true}};
+    wkv_status s = check_bufs(bufs, 4);
+    if (s != WKV_OK) return s;
+    const Span out = span(s_in, one * (P + 1));
+    if (overlaps(out, span(state0, state0 ? one : 0)) || overlaps(out, span(s_loc, one * P)) ||
+        overlaps(out, span(log2_decay, g1 * P)))
+        return WKV_ERR_INVALID_ARG;
+    if (injected("launch")) return WKV_ERR_CUDA;
+    return from_cuda(goldwkv::launch_segment_carry_ranks(state0, s_loc, log2_decay, s_in, B, H, P,
+                                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 wkv_status wkv6_workspace_status(void* workspace, void* stream) {
     if (workspace == nullptr || !aligned16(workspace)) return WKV_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

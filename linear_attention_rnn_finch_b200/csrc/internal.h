@@ -82,6 +82,12 @@ cudaError_t launch_segment_states(const CUtensorMap* maps, float* s_loc, float* 
 // s_in(0) = state_in (zero if null) and s_in(p) = s_mid[bh][p-1]; s_mid may alias s_loc.
 cudaError_t launch_segment_carry(const float* state_in, const float* s_loc, const float* log2g,
                                  float* s_mid, int B, int H, int P, cudaStream_t st);
+// The same chain over P segments laid out segment-major (s_loc [P][B*H][D][D], log2g
+// [P][B*H][D]): s_in [P + 1][B*H][D][D], s_in[0] = state0 (zero if null), s_in[p + 1] =
+// 2^log2g[p] (rows) * s_in[p] + s_loc[p].
+cudaError_t launch_segment_carry_ranks(const float* state0, const float* s_loc,
+                                       const float* log2g, float* s_in, int B, int H, int P,
+                                       cudaStream_t st);
 
 // Fast path (one-sided decay factorisation, warp-specialised pipeline).  maps: r, k, v,
 // omega.  For each unit it writes y (and, in the last segment, the final state), or stops at

@@ -295,7 +295,51 @@ wkv6_segment_carry_kernel(const float* state_in, const float* s_loc, const float
     }
 }
 
+// States entering P consecutive segments given each one's local state and log2 decay, laid
+// out segment-major ([p][bh]): s_in[0] = state0 (zero if null), s_in[p+1] = 2^g[p] (rows)
+// s_in[p] + s_loc[p], p = 0 .. P-1 (s_in has P + 1 entries).  One CTA per (b,h), a thread
+// per row i and 16 columns.
+__global__ void __launch_bounds__(256)
+wkv6_segment_carry_ranks_kernel(const float* state0, const float* s_loc, const float* log2g,
+                                float* s_in, int P, int nbh) {
+    const int bh = blockIdx.x, i = threadIdx.x >> 2, j0 = 16 * (threadIdx.x & 3);
+    float S[16];
+    const float* src = state0 ? state0 + (size_t)bh * 4096 + i * 64 + j0 : nullptr;
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+        const float4 x = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+    }
+    for (int p = 0; p <= P; ++p) {
+        float* out = s_in + ((size_t)p * nbh + bh) * 4096 + i * 64 + j0;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(out + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        if (p == P) break;
+        const size_t idx = (size_t)p * nbh + bh;
+        const float gi = exp2f(log2g[idx * 64 + i]);
+        const float* loc = s_loc + idx * 4096 + i * 64 + j0;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+            const float4 l = *reinterpret_cast<const float4*>(loc + j);
+            S[j] = fmaf(gi, S[j], l.x);
+            S[j + 1] = fmaf(gi, S[j + 1], l.y);
+            S[j + 2] = fmaf(gi, S[j + 2], l.z);
+            S[j + 3] = fmaf(gi, S[j + 3], l.w);
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_segment_carry_ranks(const float* state0, const float* s_loc,
+                                       const float* log2g, float* s_in, int B, int H, int P,
+                                       cudaStream_t st) {
+    if (B * H == 0) return cudaSuccess;
+    wkv6_segment_carry_ranks_kernel<<<(unsigned)(B * H), 256, 0, st>>>(state0, s_loc, log2g, s_in,
+                                                                      P, B * H);
+    return cudaGetLastError();
+}
 
 size_t segment_smem_bytes() { return sizeof(Smem) + 1024; }
 

@@ -35,6 +35,8 @@ def test_headers_declare_entry_points():
                  "wkv6_prefill_workspace_bytes", "wkv6_decode_workspace_bytes",
                  "wkv6_status_string", "wkv6_abi_version", "wkv6_workspace_status",
                  "wkv6_prefill_static", "wkv6_prefill_static_status", "wkv6c2_prefill",
+                 "wkv6_segment_summary", "wkv6_segment_summary_workspace_bytes",
+                 "wkv6_segment_carry",
                  "wkv6c2_decode_step",
                  "wkv6_prefill_gn", "wkv6_decode_step_gn", "wkv6_backward",
                  "wkv6_backward_workspace_bytes", "wkv6c2_backward",
