@@ -431,6 +431,48 @@ def gold_line(dev, world, steps, B=8, T=4096, D=2048, Dc=128):
     return line
 
 
+def seqpar_line(dev, world, rank, steps, hbm):
+    """The long-context shape (B1 T262144 H64) as ONE sequence split across the ranks
+    (linear_attention_rnn_finch_b200/seqpar.py): rank p holds tokens p*T/N .. (p+1)*T/N - 1;
+    per call: the span's summary, one all-gather of the summaries (NCCL), the carry, the
+    span's prefill.  Time is the slowest rank's (strong scaling: the work is fixed)."""
+    import torch.distributed as dist
+    import linear_attention_rnn_finch_b200 as gw
+    from linear_attention_rnn_finch_b200 import seqpar
+    cfg = W.CONFIGS[2]
+    B, T, H, D = cfg.B, cfg.T, cfg.H, cfg.D
+    if T % (64 * world):
+        raise ValueError("the sequence must split into chunk-aligned spans")
+    tp = T // world
+    full = W.make_prefill_inputs(cfg, dev)
+    a = [full[n][:, rank * tp:(rank + 1) * tp].contiguous() for n in ("r", "k", "v", "omega")]
+    u, s0 = full["u"], full["state0"]
+    del full
+    torch.cuda.empty_cache()
+
+    def call():
+        with nvtx("seqpar_prefill"):
+            return seqpar.prefill_sequence_parallel(*a, u, s0)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    dist.barrier()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    nbytes = prefill_bytes(B, T, H, D)
+    return {"workload": f"wkv6_prefill_long_ctx B{B} T{T} H{H} split over {world} rank(s)",
+            "ms_per_call": ms, "value": B * T / (ms / 1e3), "unit": "tokens/s",
+            "roofline": {"bound": "hbm", "frac": nbytes / (ms / 1e3) / 1e9 / (hbm * world)},
+            "note": "strong scaling of one sequence; frac against N GPUs' HBM bandwidth"}
+
+
 def bf16_peak():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -780,6 +822,9 @@ def main():
                          "decompression, on the 1.5B-layer shape; --batch and --seq-len "
                          "override B and T), for profiler runs")
     ap.add_argument("--seq-len", type=int, default=None, help="T of --only")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="print only the long-context shape as one sequence split across the "
+                         "ranks (NCCL exchange; a process group is set up even at one rank)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -795,7 +840,24 @@ def main():
 
     world, rank, local = dist_setup()
     try:
-        if args.only is not None:
+        if args.seqpar:
+            import torch.distributed as dist
+            from linear_attention_rnn_finch_b200 import binding
+            binding.load()
+            dev = torch.device("cuda", local)
+            if not dist.is_initialized():   # one rank: a one-member NCCL group
+                import datetime
+                import socket
+                with socket.socket() as sk:
+                    sk.bind(("127.0.0.1", 0))
+                    port = sk.getsockname()[1]
+                dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                        world_size=1, timeout=datetime.timedelta(seconds=120),
+                                        device_id=dev)
+                world = 1
+            hbm, _ = peaks()
+            out = seqpar_line(dev, world, rank, args.steps, hbm)
+        elif args.only is not None:
             from linear_attention_rnn_finch_b200 import binding
             binding.load()
             cfg = PREFILL_CFG.with_(**{k: v for k, v in (("B", args.batch), ("T", args.seq_len))
@@ -810,8 +872,8 @@ def main():
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)
     finally:
-        if world > 1:
-            import torch.distributed as dist
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
             dist.destroy_process_group()
 
 
