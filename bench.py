@@ -817,10 +817,12 @@ def main():
                     help="skip the ~1 s untimed warm-up loop (for profiler runs)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the prefill batch size (smaller profiler captures)")
-    ap.add_argument("--only", choices=["backward", "backward_c2", "gold"], default=None,
+    ap.add_argument("--only", choices=["backward", "backward_c2", "gold", "extreme_ln"],
+                    default=None,
                     help="print only that line (wkv6_backward, or GOLD compression + "
-                         "decompression, on the 1.5B-layer shape; --batch and --seq-len "
-                         "override B and T), for profiler runs")
+                         "decompression, on the 1.5B-layer shape; or the decay-extreme prefill "
+                         "with LayerNorm; --batch and --seq-len override B and T), for "
+                         "profiler runs")
     ap.add_argument("--seq-len", type=int, default=None, help="T of --only")
     ap.add_argument("--seqpar", action="store_true",
                     help="print only the long-context shape as one sequence split across the "
@@ -860,11 +862,15 @@ def main():
         elif args.only is not None:
             from linear_attention_rnn_finch_b200 import binding
             binding.load()
-            cfg = PREFILL_CFG.with_(**{k: v for k, v in (("B", args.batch), ("T", args.seq_len))
-                                       if v is not None})
+            base = W.CONFIGS[4] if args.only == "extreme_ln" else PREFILL_CFG
+            cfg = base.with_(**{k: v for k, v in (("B", args.batch), ("T", args.seq_len))
+                                if v is not None})
             dev = torch.device("cuda", local)
+            hbm, _ = peaks()
             out = (gold_line(dev, world, steps=args.steps, B=cfg.B, T=cfg.T)
                    if args.only == "gold" else
+                   other_prefill(cfg, dev, world, hbm, args.algo, steps=args.steps)
+                   if args.only == "extreme_ln" else
                    backward_line(cfg, dev, world, steps=args.steps,
                                  c2=args.only == "backward_c2"))
         else:

@@ -68,6 +68,7 @@ def test_workspace_queries():
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False, "recurrent") == 0
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.float32, True) == 0
     assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True) == hand(2, 3) + 2 * 10 * 3 * 64 * 4
+    assert binding.prefill_workspace_bytes(2, 130, 3, 64, torch.bfloat16, True) == hand(2, 3) + 2 * 130 * 3 * 64 * 4
     assert binding.prefill_workspace_bytes(2, 10, 3, 64, torch.bfloat16, True, "recurrent") == 2 * 10 * 3 * 64 * 4
     # 256-byte block of row counters, then the bf16 path's fp32 staging
     assert binding.decode_workspace_bytes(256, 32, 64, torch.bfloat16, True) == 1024 + 256 * 32 * 64 * 4
