@@ -236,7 +236,10 @@ typedef struct wkv_gn {
  * wkv6_prefill_gn: as wkv6_prefill (WKV_ALGO_AUTO; same layouts, aliasing rules and errors)
  * with the GroupNorm + gate output stage above in place of LayerNorm.  gn is required.
  * Workspace: wkv6_prefill_workspace_bytes(B, T, H, D, io, 1, WKV_ALGO_AUTO) -- the same as
- * with LayerNorm (an fp32 staging copy of y when io is bf16).
+ * with LayerNorm.  With bf16 I/O (the chunked path) the stage runs inside the recurrence
+ * kernels, as each chunk's output is formed (a head's 64 channels are one CTA's), and the
+ * workspace's LayerNorm staging area is left unused; the fp32 recurrence normalises in a
+ * second kernel over fp32 rows.
  */
 wkv_status wkv6_prefill_gn(const void *r, const void *k, const void *v, const void *omega,
                            const float *u, const float *state_in, float *state_out, void *y,

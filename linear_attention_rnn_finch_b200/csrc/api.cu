@@ -290,7 +290,8 @@ namespace {
 bool launch_chunked_path(const void* r, const void* k, const void* v, const void* omega,
                          const float* u, const goldwkv::Variant& var, const float* state_in,
                          float* state_out, void* y, float* y_raw, int B, int T, int H, int P,
-                         bool levels_only, uint8_t* ws, cudaStream_t st, cudaError_t* e) {
+                         bool levels_only, uint8_t* ws, cudaStream_t st, cudaError_t* e,
+                         const goldwkv::GnOut* gn = nullptr) {
     const long long budget = injected("timeout0") ? 0 : kSpinBudget;
     CUtensorMap maps[5];
     if (!goldwkv::make_token_map(&maps[0], r, B, T, H) ||
@@ -312,7 +313,7 @@ bool launch_chunked_path(const void* r, const void* k, const void* v, const void
     const goldwkv::Segments seg{P, (nc + P - 1) / P, s_mid};
     if (levels_only) {
         *e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg,
-                                            var, status, nullptr, nullptr, budget, st);
+                                            var, status, nullptr, nullptr, budget, st, gn);
         return true;
     }
     *e = cudaSuccess;
@@ -324,10 +325,10 @@ bool launch_chunked_path(const void* r, const void* k, const void* v, const void
     }
     if (*e == cudaSuccess)
         *e = goldwkv::launch_chunked_fast(maps, u, state_in, state_out, y, y_raw, B, T, H, seg,
-                                          var, status, h_chunk, h_state, budget, st);
+                                          var, status, h_chunk, h_state, budget, st, gn);
     if (*e == cudaSuccess)
         *e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg, var,
-                                            status, h_chunk, h_state, budget, st);
+                                            status, h_chunk, h_state, budget, st, gn);
     return true;
 }
 
@@ -409,18 +410,25 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     float* y_raw = nullptr;
     const int P = plan.P;
     const size_t raw_at = chunked ? chunked_bytes(B, H, P) : 0;
-    if (nm.on()) y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
+    // GroupNorm + gate runs inside the chunked kernels; LayerNorm (over all heads of a token)
+    // and the fp32 recurrence's output stages run as a second pass over fp32 rows
+    const bool fused_gn = chunked && nm.kind == Norm::kGroup;
+    const goldwkv::GnOut gn{nm.gamma, nm.beta, nm.eps, nm.gate};
+    if (nm.on() && !fused_gn)
+        y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
     if (chunked) {
         if (!launch_chunked_path(r, k, v, omega, u, var, state_in, state_out, y, y_raw, B, T, H,
-                                 P, algo == WKV_ALGO_CHUNKED_LEVELS, ws, st, &e))
+                                 P, algo == WKV_ALGO_CHUNKED_LEVELS, ws, st, &e,
+                                 fused_gn ? &gn : nullptr))
             return WKV_ERR_CUDA;
     } else {
         e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,
                                       H, bf16, var, st);
     }
     if (e != cudaSuccess) return WKV_ERR_CUDA;
-    if (nm.on() && launch_norm(nm, y_raw, y, (long)B * T, H, D, bf16, st) != cudaSuccess)
+    if (nm.on() && !fused_gn &&
+        launch_norm(nm, y_raw, y, (long)B * T, H, D, bf16, st) != cudaSuccess)
         return WKV_ERR_CUDA;
     return WKV_OK;
 }

@@ -89,8 +89,9 @@ constexpr uint32_t COL_DU = 0, COL_SC = 128, COL_Y = 256;
 // log2 of the largest factor exp(-L_s) allowed: ln range 60 -> log2 range 86.56
 constexpr float kMaxLog2Range = 86.5617f;
 constexpr float kLog2e = 1.4426950408889634f;
-// named barriers (id 0 is __syncthreads): one per prep group, one for the epilogue
-constexpr int kBarPrep0 = 1, kBarEpi = kBarPrep0 + kPrepGroups;
+// named barriers (id 0 is __syncthreads): one per prep group, one for the epilogue, and one
+// per pair of epilogue warps that hold the two column halves of the same rows (GroupNorm)
+constexpr int kBarPrep0 = 1, kBarEpi = kBarPrep0 + kPrepGroups, kBarPair0 = kBarEpi + 1;
 constexpr int kNoStop = INT_MAX;
 
 constexpr uint32_t IDESC_GU = ptx::idesc_bf16(64, 128, 1, 1);
@@ -120,6 +121,10 @@ struct __align__(1024) Smem {
     uint32_t tmem_base;
     int abort;
     int stop_at;                        // first chunk handed to the level kernel (kNoStop: none)
+    // GroupNorm output stage: the head's gamma / beta, and per output-chunk parity the
+    // (mean, M2) of each row's two 32-column halves
+    float gn_gamma[64], gn_beta[64];
+    float2 gn_mom[2][2][64];
 };
 
 __device__ __forceinline__ void sts128(uint8_t* base, uint32_t off, uint32_t a, uint32_t b,
@@ -151,13 +156,37 @@ __device__ __forceinline__ bool stopped_at(const Smem& s, int n) {
     return ld_volatile(&s.abort) != 0 || ld_volatile(&s.stop_at) <= n;
 }
 
+// (mean, M2) of the 8 values of a thread's 4 column pairs (two passes over the registers)
+__device__ __forceinline__ float2 moments8(const float2 (&v)[kPairs]) {
+    float sm = 0.f;
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) sm += v[j].x + v[j].y;
+    const float mean = sm * 0.125f;
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        const float d0 = v[j].x - mean, d1 = v[j].y - mean;
+        q = fmaf(d0, d0, fmaf(d1, d1, q));
+    }
+    return make_float2(mean, q);
+}
+// (mean, M2) of the union of two disjoint sets of n values each (Chan et al.'s update with
+// n_a = n_b = n: mean = (mean_a + mean_b) / 2, M2 = M2_a + M2_b + (mean_b - mean_a)^2 n / 2)
+__device__ __forceinline__ float2 merge_equal(float2 a, float2 b, float n) {
+    const float d = b.x - a.x;
+    return make_float2(0.5f * (a.x + b.x), a.y + b.y + 0.5f * n * d * d);
+}
+__device__ __forceinline__ float2 shfl_xor2(float2 v, int o) {
+    return make_float2(__shfl_xor_sync(0xffffffffu, v.x, o), __shfl_xor_sync(0xffffffffu, v.y, o));
+}
+
 // Output of chunk m (plus the second value u' of Finch-C2, whose words up0 / up1 for rows
 // r0 / r1 the caller loaded ahead of time): y = the hi and lo rows of both column blocks of
 // Y[m & 1], stored as bf16
 // (or fp32 rows to y_raw).  The caller has waited for GA(m).  col0: first column of this
 // thread's pairs (pair j at col0 + 8j).
-template <bool kC2>
-__device__ __forceinline__ void output_chunk(int m, int c0, uint32_t tmem, uint32_t lane_h0,
+template <bool kC2, bool kGN>
+__device__ __forceinline__ void output_chunk(Smem& s, float gn_eps, int m, int c0, uint32_t tmem, uint32_t lane_h0,
                                              uint32_t lane_h1, int col0, int cl, int r0, int r1,
                                              int b, int h, int T, int H, __nv_bfloat16* y,
                                              float* y_raw, const uint32_t (&up0)[kPairs],
@@ -182,6 +211,41 @@ __device__ __forceinline__ void output_chunk(int m, int c0, uint32_t tmem, uint3
     const int valid = min(C, T - tc);
     const size_t row0 = ((size_t)b * T + (size_t)tc + r0) * H + h;
     const size_t row1 = ((size_t)b * T + (size_t)tc + r1) * H + h;
+    if (kGN) {
+        // base Finch's output stage: GroupNorm of each (token, head) row of 64 channels, the
+        // head's affine, times the gate (words up0 / up1, loaded beforehand).  Mean and M2 of
+        // this thread's 8 values, merged over the 4 lanes of its 32-column half, then with
+        // the other half's (the partner warp, through shared memory)
+        const int half = col0 >> 5, slot = m & 1;
+        float2 mo0 = moments8(Y0), mo1 = moments8(Y1);   // (mean, M2) over 8 values
+        mo0 = merge_equal(mo0, shfl_xor2(mo0, 1), 8.f);   // 16 values
+        mo1 = merge_equal(mo1, shfl_xor2(mo1, 1), 8.f);
+        mo0 = merge_equal(mo0, shfl_xor2(mo0, 2), 16.f);  // 32: the half
+        mo1 = merge_equal(mo1, shfl_xor2(mo1, 2), 16.f);
+        if (cl == 0) {
+            s.gn_mom[slot][half][r0] = mo0;
+            s.gn_mom[slot][half][r1] = mo1;
+        }
+        named_bar(kBarPair0 + ((r0 >> 4) & 3), 64);
+        mo0 = merge_equal(mo0, s.gn_mom[slot][half ^ 1][r0], 32.f);   // 64: the row
+        mo1 = merge_equal(mo1, s.gn_mom[slot][half ^ 1][r1], 32.f);
+        const float inv0 = rsqrtf(mo0.y * (1.f / 64.f) + gn_eps);
+        const float inv1 = rsqrtf(mo1.y * (1.f / 64.f) + gn_eps);
+#pragma unroll
+        for (int jj = 0; jj < kPairs; ++jj) {
+            const int j = col0 + 8 * jj + cl;
+            const float2 g = *reinterpret_cast<const float2*>(&s.gn_gamma[j]);
+            const float2 be = *reinterpret_cast<const float2*>(&s.gn_beta[j]);
+            const float2 gt0 = unpack2(up0[jj]), gt1 = unpack2(up1[jj]);
+            const float2 a0 = make_float2(fmaf((Y0[jj].x - mo0.x) * inv0, g.x, be.x) * gt0.x,
+                                          fmaf((Y0[jj].y - mo0.x) * inv0, g.y, be.y) * gt0.y);
+            const float2 a1 = make_float2(fmaf((Y1[jj].x - mo1.x) * inv1, g.x, be.x) * gt1.x,
+                                          fmaf((Y1[jj].y - mo1.x) * inv1, g.y, be.y) * gt1.y);
+            if (r0 < valid) *reinterpret_cast<uint32_t*>(y + row0 * 64 + j) = pack2(a0.x, a0.y);
+            if (r1 < valid) *reinterpret_cast<uint32_t*>(y + row1 * 64 + j) = pack2(a1.x, a1.y);
+        }
+        return;
+    }
 #pragma unroll
     for (int jj = 0; jj < kPairs; ++jj) {
         const int j = col0 + 8 * jj + cl;
@@ -199,8 +263,9 @@ __device__ __forceinline__ void output_chunk(int m, int c0, uint32_t tmem, uint3
     }
 }
 
-// u' words of chunk (c0 + m) for this thread's rows r0, r1 and its column pairs; rows past T
-// read as zero.  Issued well before output_chunk needs them.
+// Words of a [B][T][H][64] bf16 tensor (u' of Finch-C2, or the GroupNorm gate) for chunk
+// (c0 + m), this thread's rows r0, r1 and its column pairs; rows past T read as zero, and a
+// null tensor as bf16 ones.  Issued well before output_chunk needs them.
 __device__ __forceinline__ void load_uprime(const __nv_bfloat16* __restrict__ uprime, int m, int c0,
                                             int b, int h, int T, int H, int col0, int cl, int r0, int r1,
                                             uint32_t (&up0)[kPairs], uint32_t (&up1)[kPairs]) {
@@ -208,9 +273,14 @@ __device__ __forceinline__ void load_uprime(const __nv_bfloat16* __restrict__ up
     const int valid = min(C, T - tc);
     const size_t row0 = ((size_t)b * T + (size_t)tc + r0) * H + h;
     const size_t row1 = ((size_t)b * T + (size_t)tc + r1) * H + h;
+    constexpr uint32_t kOnes = 0x3F803F80u;   // two bf16 1.0
 #pragma unroll
     for (int jj = 0; jj < kPairs; ++jj) {
         const int j = col0 + 8 * jj + cl;
+        if (uprime == nullptr) {
+            up0[jj] = up1[jj] = kOnes;
+            continue;
+        }
         up0[jj] = r0 < valid ? __ldg(reinterpret_cast<const unsigned int*>(uprime + row0 * 64 + j)) : 0u;
         up1[jj] = r1 < valid ? __ldg(reinterpret_cast<const unsigned int*>(uprime + row1 * 64 + j)) : 0u;
     }
@@ -265,13 +335,14 @@ __device__ __forceinline__ void load_v(Smem& s, const CUtensorMap* tm_v, int n, 
 }
 
 // kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
-template <bool kC2>
+// kGN: base form with the GroupNorm + gate output stage (gn).
+template <bool kC2, bool kGN>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                  const float* __restrict__ u, const float* s_in, float* s_out,
                  __nv_bfloat16* __restrict__ y, float* __restrict__ y_raw,
-                 const __nv_bfloat16* __restrict__ uprime, int T, int H,
+                 const __nv_bfloat16* __restrict__ uprime, const GnOut gn, int T, int H,
                  Segments seg, int* status, int* handoff_chunk, float* handoff_state,
                  long long budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
@@ -624,14 +695,21 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             ptx::fence_proxy_async_smem();
             mbar_arrive(&s.s_ready[0]);   // RO(0) may run
         }
-        uint32_t up0[kPairs], up1[kPairs];   // Finch-C2: u' of the next output
+        if (kGN && tid - kEpiLeader < 64) {   // read by output_chunk after the epilogue's barriers
+            s.gn_gamma[tid - kEpiLeader] = gn.gamma[h * 64 + tid - kEpiLeader];
+            s.gn_beta[tid - kEpiLeader] = gn.beta[h * 64 + tid - kEpiLeader];
+        }
+        uint32_t up0[kPairs], up1[kPairs];   // Finch-C2: u' (GroupNorm: the gate) of the next output
 #pragma unroll
         for (int j = 0; j < kPairs; ++j) up0[j] = up1[j] = 0u;
         int n = 0;
         for (; n < NC; ++n) {
             const int pb = n & 1;
             // Finch-C2: u' of chunk n-1 is read from HBM now and used by output(n-1) below
-            if (kC2 && n >= 1) load_uprime(uprime, n - 1, cseg, b, h, T, H, col0, cl, r0, r1, up0, up1);
+            // (GroupNorm: the gate of chunk n-1, the same way)
+            if ((kC2 || kGN) && n >= 1)
+                load_uprime(kGN ? static_cast<const __nv_bfloat16*>(gn.gate) : uprime, n - 1, cseg, b,
+                            h, T, H, col0, cl, r0, r1, up0, up1);
             // ---- state(n): S <- gamma (S + DU), DU^T[j][i] accumulated on the tensor cores.
             // gamma and bonus of chunk n reach us through prep's named barrier -> its leader's
             // MMA issue -> the commit on mm_done (or, at a hand-over, the leader's arrive).
@@ -696,7 +774,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             // ---- output of chunk n-1 (GA(n-1) is complete: waited above)
             if (n >= 1) {
                 ptx::tc_fence_after();
-                output_chunk<kC2>(n - 1, cseg, tmem, lane_h0, lane_h1, col0, cl, r0, r1, b, h, T, H, y,
+                output_chunk<kC2, kGN>(s, gn.eps, n - 1, cseg, tmem, lane_h0, lane_h1, col0, cl, r0, r1, b, h, T, H, y,
                                   y_raw, up0, up1);
                 // v stage (n+3) % 4 held v(n-1), read by GU(n-1) and GA(n-1), both complete
                 if (leader && n + kStagesV - 1 < NC && !stopped_at(s, n + kStagesV - 1))
@@ -710,10 +788,13 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         // chunk handed to the level kernel)
         if (n >= 1) {
             const bool ok = wait_soft(s, &s.ya_done[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), budget);
-            if (ok && !ld_volatile(&s.abort)) {
-                if (kC2) load_uprime(uprime, n - 1, cseg, b, h, T, H, col0, cl, r0, r1, up0, up1);
+            // uniform over the epilogue (the GroupNorm stage synchronises warp pairs)
+            if (!named_bar_any(kBarEpi, kEpiThreads, !ok || ld_volatile(&s.abort) != 0)) {
+                if (kC2 || kGN)
+                    load_uprime(kGN ? static_cast<const __nv_bfloat16*>(gn.gate) : uprime, n - 1, cseg,
+                                b, h, T, H, col0, cl, r0, r1, up0, up1);
                 ptx::tc_fence_after();
-                output_chunk<kC2>(n - 1, cseg, tmem, lane_h0, lane_h1, col0, cl, r0, r1, b, h, T, H, y,
+                output_chunk<kC2, kGN>(s, gn.eps, n - 1, cseg, tmem, lane_h0, lane_h1, col0, cl, r0, r1, b, h, T, H, y,
                                   y_raw, up0, up1);
             }
         }
@@ -765,14 +846,18 @@ size_t fast_smem_bytes() { return sizeof(Smem) + 1024; }
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
                                 float* s_out, void* y, float* y_raw, int B, int T, int H,
                                 Segments seg, Variant var, int* status, int* handoff_chunk,
-                                float* handoff_state, long long budget, cudaStream_t st) {
+                                float* handoff_state, long long budget, cudaStream_t st,
+                                const GnOut* gn) {
     const size_t smem = fast_smem_bytes();
-    auto kernel = var.uprime ? wkv6_fast_kernel<true> : wkv6_fast_kernel<false>;
+    auto kernel = var.uprime ? wkv6_fast_kernel<true, false>
+                  : gn       ? wkv6_fast_kernel<false, true>
+                             : wkv6_fast_kernel<false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    const GnOut g = gn ? *gn : GnOut{nullptr, nullptr, 0.f, nullptr};
     kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], u, s_in, s_out, static_cast<__nv_bfloat16*>(y),
-        y_raw, static_cast<const __nv_bfloat16*>(var.uprime), T, H, seg, status, handoff_chunk,
+        y_raw, static_cast<const __nv_bfloat16*>(var.uprime), g, T, H, seg, status, handoff_chunk,
         handoff_state, budget, 4000000000LL);
     return cudaGetLastError();
 }

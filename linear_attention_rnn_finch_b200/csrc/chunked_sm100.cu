@@ -84,6 +84,7 @@ struct __align__(1024) Smem {
     uint64_t mma1, mma2;
     uint32_t tmem_base;
     int abort;
+    float2 gn_mom[2][64];            // GroupNorm stage: (mean, M2) of each row's two halves
 };
 
 // byte offset of element (row, col) in a 64 x 64 bf16 tile with 128-byte rows, swizzled
@@ -126,13 +127,14 @@ __device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 
 }
 
 // kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
-template <bool kC2>
+// kGN: base form with the GroupNorm + gate output stage (gn).
+template <bool kC2, bool kGN>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
                     const float* s_in, float* s_out, float* __restrict__ y_raw,
-                    const __nv_bfloat16* __restrict__ uprime, int T, int H, Segments seg, int* status, const int* start_chunk,
+                    const __nv_bfloat16* __restrict__ uprime, const GnOut gn, int T, int H, Segments seg, int* status, const int* start_chunk,
                     const float* handoff_state, long long spin_budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
@@ -488,7 +490,54 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                     for (int e = 0; e < 8; ++e) Y[8 * cc + e] = __float_as_uint(__uint_as_float(Y[8 * cc + e]) + f[e]);
                 }
             }
-            if (row_lane && y_raw != nullptr) {
+            if (kGN) {
+                // base Finch's output stage: GroupNorm of the (token, head) row over its 64
+                // channels (this lane's 32, then the other half's from the partner warp),
+                // the head's affine, times the gate
+                float2 mo = make_float2(0.f, 0.f);
+                if (row_lane) {
+                    float sm = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sm += __uint_as_float(Y[j]);
+                    const float mean = sm * (1.f / 32.f);
+                    float q2 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float d = __uint_as_float(Y[j]) - mean;
+                        q2 = fmaf(d, d, q2);
+                    }
+                    mo = make_float2(mean, q2);
+                    s.gn_mom[hh][row] = mo;
+                }
+                __syncthreads();
+                if (row_lane) {
+                    const float2 ot = s.gn_mom[hh ^ 1][row];
+                    const float d = ot.x - mo.x;
+                    const float mean = 0.5f * (mo.x + ot.x);
+                    const float inv = rsqrtf((mo.y + ot.y + 16.f * d * d) * (1.f / 64.f) + gn.eps);
+                    const int c0 = h * 64 + 32 * hh;
+                    const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(gn.gate);
+                    const size_t gbase = (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float gt[8];
+                        if (gp != nullptr && row < valid) {
+                            unpack8(__ldg(reinterpret_cast<const uint4*>(gp + gbase + 8 * cc)), gt);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) gt[e] = 1.f;
+                        }
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = 8 * cc + e;
+                            f[e] = fmaf((__uint_as_float(Y[j]) - mean) * inv, __ldg(gn.gamma + c0 + j),
+                                        __ldg(gn.beta + c0 + j)) * gt[e];
+                        }
+                        st_shared_v4(y_tile, sw_chunk(row, 4 * hh + cc), pack8(f));
+                    }
+                }
+            } else if (row_lane && y_raw != nullptr) {
                 // fp32 rows for the LayerNorm pass: 128 contiguous bytes per lane
                 if (row < valid) {
                     float* dst = y_raw + (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
@@ -608,15 +657,18 @@ cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const
                                   float* s_out, float* y_raw, int B, int T, int H, Segments seg,
                                   Variant var, int* status, const int* start_chunk,
                                   const float* handoff_state, long long spin_budget,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, const GnOut* gn) {
     const size_t smem = chunked_smem_bytes();
-    auto kernel = var.uprime ? wkv6_chunked_kernel<true> : wkv6_chunked_kernel<false>;
+    auto kernel = var.uprime ? wkv6_chunked_kernel<true, false>
+                  : gn       ? wkv6_chunked_kernel<false, true>
+                             : wkv6_chunked_kernel<false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long drain = 4000000000LL;
     kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw,
-        static_cast<const __nv_bfloat16*>(var.uprime), T, H, seg, status, start_chunk,
+        static_cast<const __nv_bfloat16*>(var.uprime), gn ? *gn : GnOut{nullptr, nullptr, 0.f, nullptr},
+        T, H, seg, status, start_chunk,
         handoff_state, spin_budget, drain);
     return cudaGetLastError();
 }

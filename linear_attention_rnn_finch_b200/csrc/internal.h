@@ -89,24 +89,37 @@ cudaError_t launch_segment_carry_ranks(const float* state0, const float* s_loc,
                                        const float* log2g, float* s_in, int B, int H, int P,
                                        cudaStream_t st);
 
+// Base Finch's output stage fused into the chunked kernels: per (token, head) GroupNorm over
+// the head's 64 channels (biased variance, eps inside the square root), the per-channel
+// affine gamma / beta ([H*64] fp32), then times gate (bf16, layout of y; null: no gate).
+struct GnOut {
+    const float* gamma;
+    const float* beta;
+    float eps;
+    const void* gate;
+};
+
 // Fast path (one-sided decay factorisation, warp-specialised pipeline).  maps: r, k, v,
 // omega.  For each unit it writes y (and, in the last segment, the final state), or stops at
 // the first chunk whose decay range it cannot take and records that chunk (absolute index)
 // in handoff_chunk[u] (-1: done) with the state entering it in handoff_state[u].
-// y_raw != nullptr: fp32 y rows there instead of y.
+// y_raw != nullptr: fp32 y rows there instead of y.  gn != nullptr: y = GroupNorm + gate of
+// the rows (base form only; y_raw must then be null).
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
                                 float* s_out, void* y, float* y_raw, int B, int T, int H,
                                 Segments seg, Variant var, int* status, int* handoff_chunk,
-                                float* handoff_state, long long budget, cudaStream_t st);
+                                float* handoff_state, long long budget, cudaStream_t st,
+                                const GnOut* gn = nullptr);
 
 // Level-factorised path (any decay).  start_chunk == nullptr: every unit from its first
 // chunk with its incoming state; otherwise unit u resumes at chunk start_chunk[u] (skipped if
 // < 0) from handoff_state[u].  status: device word set to 1 if a bounded wait expired.
+// gn: as for the fast path.
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
                                   float* s_out, float* y_raw, int B, int T, int H, Segments seg,
                                   Variant var, int* status, const int* start_chunk,
                                   const float* handoff_state, long long spin_budget,
-                                  cudaStream_t st);
+                                  cudaStream_t st, const GnOut* gn = nullptr);
 size_t chunked_smem_bytes();
 size_t fast_smem_bytes();
 size_t segment_smem_bytes();
