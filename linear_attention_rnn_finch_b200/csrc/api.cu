@@ -655,7 +655,11 @@ size_t backward_bytes(int B, int T, int H, int D, wkv_dtype io, bool tc_dv) {
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     const size_t x = (size_t)B * T * H * D, bh = (size_t)B * H * D;
     size_t bytes = round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
-    if (tc_dv) bytes += 5 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H));
+    // tensor-core path: 5 time-reversed copies, the chunked prefill's workspace, and the dr
+    // kernel's fallback flag per (b,h)
+    if (tc_dv)
+        bytes += 5 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H)) +
+                 round256((size_t)B * H * sizeof(int));
     return bytes;
 }
 
@@ -728,6 +732,7 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     uint8_t* E = ws + round256((size_t)B * T * H * D * acc);
     uint8_t* dpart = E + round256((size_t)B * H * D * acc);
     float* du_part = reinterpret_cast<float*>(dpart);
+    int* dr_flags = nullptr;   // set on the tensor-core path: which (b,h) the dr scan redoes
     if (tc_dv) {
         // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
         // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.
@@ -754,11 +759,26 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         void* dst_dv[1] = {dv};
         if (goldwkv::launch_reverse_tokens(src_dv, dst_dv, 1, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
+        // dr (with P, E and du's parts) on the tensor cores; a (b,h) whose decay range the
+        // one-sided factorisation cannot take is flagged and left to the CUDA-core dr scan
+        dr_flags = reinterpret_cast<int*>(cws + chunked_bytes(B, H, choose_segments(B, T, H)));
+        CUtensorMap maps[5];
+        if (!goldwkv::make_token_map(&maps[0], dy, B, T, H) ||
+            !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
+            !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
+            !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
+            !goldwkv::make_token_map(&maps[4], dr, B, T, H))
+            return WKV_ERR_CUDA;
+        const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+        if (goldwkv::launch_bwd_dr_tc(maps, r, u, state_in, dstate_out, static_cast<float*>(P),
+                                      reinterpret_cast<float*>(E), du_part, dr_flags, B, T, H,
+                                      reinterpret_cast<int*>(cws), budget, st) != cudaSuccess)
+            return WKV_ERR_CUDA;
     }
     return from_cuda(goldwkv::launch_backward(r, k, v, omega, c2 ? nullptr : u, state_in, dy,
                                               dstate_out, dr, dk, dv, domega, du, dstate_in, P,
                                               E, du_part, B, T, H, bf16, /*with_dv=*/!tc_dv, c2,
-                                              st));
+                                              st, dr_flags));
 }
 
 }  // namespace

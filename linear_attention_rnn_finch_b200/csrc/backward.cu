@@ -503,9 +503,10 @@ wkv6_bwd_dr_dv_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                       const float* __restrict__ u, const float* state_in, const IO* __restrict__ dy,
                       const float* __restrict__ dS_T, IO* __restrict__ dr, IO* __restrict__ dv,
                       typename Prec<IO>::Acc* __restrict__ P, typename Prec<IO>::Acc* __restrict__ E,
-                      float* __restrict__ du_part, int T, int H) {
+                      float* __restrict__ du_part, int T, int H, const int* dr_only) {
     using Sm = SweepSmem<IO>;
     __shared__ __align__(16) unsigned char smem[Sm::kBytes];
+    if (blockIdx.z == 0 && dr_only != nullptr && dr_only[blockIdx.x] == 0) return;
     if (blockIdx.z == 0)
         row_sweep<IO, false, kC2>(*reinterpret_cast<typename Sm::Row*>(smem), k, r, v, dy, omega, u,
                              state_in, dr, P, nullptr, E, dS_T, du_part, nullptr, T, H);
@@ -560,14 +561,15 @@ cudaError_t launch_typed(const void* r, const void* k, const void* v, const void
                          const float* u, const float* state_in, const void* dy,
                          const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                          float* du, float* dstate_in, void* P_, void* E_, float* du_part, int B,
-                         int T, int H, bool with_dv, cudaStream_t st) {
+                         int T, int H, bool with_dv, cudaStream_t st, const int* dr_only) {
     using Acc = typename Prec<IO>::Acc;
     const IO *r_ = (const IO*)r, *k_ = (const IO*)k, *v_ = (const IO*)v, *o_ = (const IO*)omega,
              *dy_ = (const IO*)dy;
     Acc *P = static_cast<Acc*>(P_), *E = static_cast<Acc*>(E_);
     const unsigned bh = (unsigned)(B * H);
     wkv6_bwd_dr_dv_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf, with_dv ? 2 : 1), kThreads, 0, st>>>(
-        r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H);
+        r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H,
+        dr_only);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     wkv6_bwd_dk_domega_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf), kThreads, 0, st>>>(
@@ -585,21 +587,21 @@ cudaError_t launch_backward(const void* r, const void* k, const void* v, const v
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
                             int B, int T, int H, bool bf16, bool with_dv, bool c2,
-                            cudaStream_t st) {
+                            cudaStream_t st, const int* dr_only) {
     using BF = __nv_bfloat16;
     if (c2)
         return bf16 ? launch_typed<BF, true>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
                                             dv, domega, du, dstate_in, P, E, du_part, B, T, H,
-                                            with_dv, st)
+                                            with_dv, st, dr_only)
                     : launch_typed<float, true>(r, k, v, omega, u, state_in, dy, dstate_out, dr,
                                                 dk, dv, domega, du, dstate_in, P, E, du_part, B,
-                                                T, H, with_dv, st);
+                                                T, H, with_dv, st, dr_only);
     return bf16 ? launch_typed<BF, false>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv,
                                           domega, du, dstate_in, P, E, du_part, B, T, H, with_dv,
-                                          st)
+                                          st, dr_only)
                 : launch_typed<float, false>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
                                              dv, domega, du, dstate_in, P, E, du_part, B, T, H,
-                                             with_dv, st);
+                                             with_dv, st, dr_only);
 }
 
 cudaError_t launch_reverse_tokens(const void* const* src, void* const* dst, int n, int B, int T,

@@ -1,6 +1,7 @@
 // Launcher of the WKV6 backward kernels (csrc/backward.cu).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace goldwkv {
@@ -11,12 +12,24 @@ namespace goldwkv {
 // dstate_out / state_in may be null (zero); dstate_in may be null (not written).
 // with_dv == false: dv is computed elsewhere (the caller's tensor-core path); dv unused.
 // c2: Finch-C2's exact form (key k (1 - w), no bonus; u and du unused).
+// dr_only != nullptr: the dr scan runs only for the (b,h) with dr_only[bh] != 0 (the others'
+// dr, P, E and du_part were written by launch_bwd_dr_tc).
 cudaError_t launch_backward(const void* r, const void* k, const void* v, const void* omega,
                             const float* u, const float* state_in, const void* dy,
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
                             int B, int T, int H, bool bf16, bool with_dv, bool c2,
-                            cudaStream_t st);
+                            cudaStream_t st, const int* dr_only = nullptr);
+
+// dr of the base form (bf16 I/O) on the tensor cores (csrc/backward_tc_sm100.cu), one CTA per
+// (b,h): writes dr and, as the CUDA-core dr scan does, P, E and du_part.  maps: dy, k, v,
+// omega, dr ([B][T][H][64] bf16 token maps); r is read directly.  fallback[bh] = 1 for a
+// (b,h) with a chunk whose decay range the one-sided factorisation cannot take (its outputs
+// are then left to the scan), 0 otherwise.  status: set to 1 if a bounded wait expired.
+cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float* u,
+                             const float* state_in, const float* dS_T, float* P, float* E,
+                             float* du_part, int* fallback, int B, int T, int H, int* status,
+                             long long budget, cudaStream_t st);
 
 constexpr int kMaxReverse = 4;
 

@@ -1,0 +1,524 @@
+// dr of the WKV6 backward on the tensor cores (sm_100a): the chunked form of the readout of
+// the forward state with dy as the query.
+//
+// Forward (GoldFinch review page, section 3.4 "Recurrent state update and output"), per (b,h):
+//     S_t = diag(w_t) S_{t-1} + k_t^T v_t,   y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),
+// so dr_t[i] = sum_j S_{t-1}[i][j] dy_t[j] + u[i] k_t[i] (v_t . dy_t), the first term a
+// readout of the forward state in which the decay sits on the output index i.  For a chunk of
+// C = 64 tokens entering with state S, with L_t = sum_{tau<=t} log2 w_tau inside the chunk:
+//     S_{t-1}[i][j] = 2^(L_{t-1}[i]) S[i][j] + sum_{s<t} 2^(L_{t-1}[i] - L_s[i]) k_s[i] v_s[j]
+//     dr_t[i] = F[t][i] (Z[t][i] + sum_{s<t} A[t][s] Kh[s][i]) + u[i] k_t[i] A[t][t]
+// with  F[t][i] = 2^(L_{t-1}[i]) <= 1,  Kh[s][i] = k_s[i] 2^(-L_s[i]),  A = dy v^T (the scores,
+// no decay), Z = dy S^T.  The one-sided factor Kh is bounded by 2^86.56 when every channel's
+// log2 decay over the chunk is >= -86.56; a (b,h) with a chunk outside that range is flagged
+// and left to the CUDA-core scan (fallback[bh] = 1), which redoes its whole sequence.
+// The state itself advances with the suffix factors Kt_s = k_s 2^(L_{C-1} - L_s) <= 1 (any
+// decay): S <- diag(2^L_{C-1}) S + Kt^T V.
+//
+// Per chunk (one CTA per (b,h), 256 threads, all warps in lockstep):
+//   prep  : warp = 8 channels, lane = 2 tokens; log2 w, the prefix L by a warp scan, F (fp32),
+//           Kh and Kt^T as bf16 hi / lo tiles, gamma;
+//   MMA 1 : A = dy x v^T; Z = dy x S_hi^T + dy x S_lo^T; U = Kt_hi^T V + Kt_lo^T V;
+//   state : S <- gamma S + U in registers, S_hi / S_lo tiles for the next chunk;
+//   A     : strictly causal part, hi / lo tiles; the diagonal (v_t . dy_t) kept aside;
+//   MMA 2 : Z += A_hi Kh_hi + A_hi Kh_lo + A_lo Kh_hi;
+//   out   : dr = F Z + u k diag (bf16 tile, TMA store); for the decay gradient the pair
+//           terms ending at t, P_t = r_t (dr_t - bonus) (fp32), and du's per-(b,h) sums.
+// At the end: E[i] = sum_j S_T[i][j] dS_T[i][j] (with the dk scan's decay gradient) and du.
+// P, E and du_part have the layout and meaning of the CUDA-core dr scan's (csrc/backward.cu),
+// so the dk scan that follows reads them unchanged.  Every mbarrier wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "backward.h"
+#include "common.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace goldwkv {
+
+namespace {
+
+constexpr int C = 64;
+constexpr int kThreads = 256;
+constexpr int kStages = 2;
+constexpr int kTile = 64 * 64 * 2;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t COL_A = 0, COL_U = 64, COL_Z = 128;
+constexpr uint32_t IDESC_KK = ptx::idesc_bf16(64, 64, 0, 0);
+constexpr uint32_t IDESC_KM = ptx::idesc_bf16(64, 64, 0, 1);
+constexpr float kMaxLog2Range = 86.5617f;   // ln 60
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kFPitch = 68;                 // floats per row of F (padded against bank conflicts)
+
+struct __align__(1024) Smem {
+    uint8_t in[kStages][4][kTile];   // dy, k, v, omega tiles per stage (TMA, 128B swizzle)
+    uint8_t kh_hi[kTile], kh_lo[kTile];     // Kh [s][i]
+    uint8_t kt_hi[kTile], kt_lo[kTile];     // Kt^T [i][s]
+    uint8_t a_hi[kTile], a_lo[kTile];       // causal scores [t][s]
+    uint8_t s_hi[kTile], s_lo[kTile];       // S [i][j]
+    uint8_t ystage[2][kTile];               // dr tiles for the TMA store
+    float F[C][kFPitch];
+    float u[64];
+    float gamma[64];
+    float diag[64];                         // v_t . dy_t
+    float epart[2][64];                     // E halves
+    float dupart[4][64];                    // du sums per row quarter
+    uint64_t full[kStages];
+    uint64_t mma1, mma2;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t sw_chunk(int row, int chunk) {
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+// hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ void split8(const float (&f)[8], uint4& hi, uint4& lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = __bfloat162float(__float2bfloat16_rn(f[i]));
+        l[i] = f[i] - h[i];
+    }
+    hi = pack8(h);
+    lo = pack8(l);
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// the two bf16 of a transposed tile entry: channel row i, tokens (2 lane, 2 lane + 1)
+__device__ __forceinline__ uint32_t tr_off(int i, int lane) {
+    return (uint32_t)(i * 128 + ((((lane >> 2)) ^ (i & 7)) << 4) + (lane & 3) * 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+wkv6_bwd_dr_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                      const __grid_constant__ CUtensorMap tm_dr, const __nv_bfloat16* __restrict__ r,
+                      const float* __restrict__ u, const float* state_in, const float* dS_T,
+                      float* __restrict__ P, float* __restrict__ E, float* __restrict__ du_part,
+                      int* fallback, int T, int H, int* status, long long budget,
+                      long long drain_budget) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x, b = bh / H, h = bh - (bh / H) * H;
+    const int NC = (T + C - 1) / C;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) ptx::mbar_init(&s.full[i], 1);
+        ptx::mbar_init(&s.mma1, 1);
+        ptx::mbar_init(&s.mma2, 1);
+        ptx::fence_mbar_init();
+        s.abort = 0;
+        ptx::prefetch_tensormap(&tm_dy);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_w);
+        ptx::prefetch_tensormap(&tm_dr);
+    }
+    if (tid < 64) s.u[tid] = u[h * 64 + tid];
+    if (warp == 0) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+
+    auto issue_load = [&](int n) {
+        const int st = n % kStages, t0 = n * C;
+        if (!gw_check(status, n >= 0 && n < NC && t0 < T && h < H)) return;
+        ptx::mbar_arrive_expect_tx(&s.full[st], 4 * kTile);
+        ptx::tma_load_4d(s.in[st][0], &tm_dy, &s.full[st], 0, h, t0, b);
+        ptx::tma_load_4d(s.in[st][1], &tm_k, &s.full[st], 0, h, t0, b);
+        ptx::tma_load_4d(s.in[st][2], &tm_v, &s.full[st], 0, h, t0, b);
+        ptx::tma_load_4d(s.in[st][3], &tm_w, &s.full[st], 0, h, t0, b);
+    };
+    if (tid == 0)
+        for (int n = 0; n < kStages && n < NC; ++n) issue_load(n);
+
+    // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in lanes 0..15), column half hh
+    const int q = warp & 3, hh = warp >> 2;
+    const bool row_lane = lane < 16;
+    const int row = 16 * q + (lane & 15);        // state row i / token row t of this lane
+    const uint32_t tlane = (uint32_t)(32 * q) << 16;
+    float S[32];
+    {
+        const float* src = state_in ? state_in + (size_t)bh * 4096 + row * 64 + 32 * hh : nullptr;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (src && row_lane) x = *reinterpret_cast<const float4*>(src + j);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        if (row_lane) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                uint4 hi, lo;
+                split8(f, hi, lo);
+                *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, 4 * hh + cc)) = hi;
+                *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, 4 * hh + cc)) = lo;
+            }
+        }
+    }
+    float du_acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) du_acc[j] = 0.f;
+
+    bool failed = false, out_of_range = false;
+    int n = 0, issued1 = -1, issued2 = -1;
+    for (; n < NC; ++n) {
+        const int st = n % kStages;
+        const int t0 = n * C;
+        const int valid = min(C, T - t0);
+        uint8_t* dy_tile = s.in[st][0];
+        uint8_t* k_tile = s.in[st][1];
+        uint8_t* v_tile = s.in[st][2];
+        uint8_t* w_tile = s.in[st][3];
+        uint8_t* y_tile = s.ystage[n & 1];
+        if (tid == 0) ptx::bulk_wait_read<1>();   // the store that last used y_tile has read it
+        if (!ptx::mbar_wait(&s.full[st], (uint32_t)((n / kStages) & 1), budget)) s.abort = 1;
+
+        // -------------------------------------------------------- prep
+        bool in_range;
+        {
+            const int cg = warp;                    // channels 8cg .. 8cg+7
+            const int ta = 2 * lane, tb = ta + 1;   // tokens of this lane
+            float kv[2][8], lw[2][8];
+            {
+                float om[2][8];
+                unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(ta, cg)), kv[0]);
+                unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(tb, cg)), kv[1]);
+                unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(ta, cg)), om[0]);
+                unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(tb, cg)), om[1]);
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)   // log2 w = -exp(omega) log2(e); 0 past T
+                        lw[p][c] = (ta + p < valid) ? -ex2(om[p][c] * kLog2e) * kLog2e : 0.f;
+            }
+            // inclusive prefix over the chunk: this lane's pair, then a scan over the lanes
+            float inc[8], L63[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) inc[c] = lw[0][c] + lw[1][c];
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float o = __shfl_up_sync(0xffffffffu, inc[c], d);
+                    if (lane >= d) inc[c] += o;
+                }
+            }
+            in_range = true;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                L63[c] = __shfl_sync(0xffffffffu, inc[c], 31);
+                in_range = in_range && L63[c] >= -kMaxLog2Range;
+            }
+            // L of the two tokens (inclusive) and of the token before each (exclusive)
+            float Lt[2][8], Lx[2][8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                Lt[1][c] = inc[c];
+                Lt[0][c] = inc[c] - lw[1][c];
+                Lx[1][c] = Lt[0][c];
+                Lx[0][c] = Lt[0][c] - lw[0][c];
+            }
+            if (in_range) {
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    float kh[8], f[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        kh[c] = kv[p][c] * ex2(-Lt[p][c]);
+                        f[c] = ex2(Lx[p][c]);
+                    }
+                    uint4 hi, lo;
+                    split8(kh, hi, lo);
+                    *reinterpret_cast<uint4*>(s.kh_hi + sw_chunk(ta + p, cg)) = hi;
+                    *reinterpret_cast<uint4*>(s.kh_lo + sw_chunk(ta + p, cg)) = lo;
+                    float4* fd = reinterpret_cast<float4*>(&s.F[ta + p][8 * cg]);
+                    fd[0] = make_float4(f[0], f[1], f[2], f[3]);
+                    fd[1] = make_float4(f[4], f[5], f[6], f[7]);
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {   // Kt^T: channel row i, this lane's two tokens
+                    const int i = 8 * cg + c;
+                    const float x0 = kv[0][c] * ex2(L63[c] - Lt[0][c]);
+                    const float x1 = kv[1][c] * ex2(L63[c] - Lt[1][c]);
+                    const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+                    const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+                    *reinterpret_cast<uint32_t*>(s.kt_hi + tr_off(i, lane)) = pack2(h0, h1);
+                    *reinterpret_cast<uint32_t*>(s.kt_lo + tr_off(i, lane)) = pack2(x0 - h0, x1 - h1);
+                }
+                if (lane == 0)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) s.gamma[8 * cg + c] = ex2(L63[c]);
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        const bool stop = __syncthreads_or(!in_range || s.abort);
+        if (stop) {
+            if (s.abort) failed = true;
+            else out_of_range = true;
+            break;
+        }
+
+        // -------------------------------------------------------- MMA 1
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            const uint32_t a_dy = ptx::smem_addr(dy_tile), b_v = ptx::smem_addr(v_tile);
+            const uint32_t b_hi = ptx::smem_addr(s.s_hi), b_lo = ptx::smem_addr(s.s_lo);
+            const uint32_t a_kh = ptx::smem_addr(s.kt_hi), a_kl = ptx::smem_addr(s.kt_lo);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)   // A = dy v^T
+                ptx::mma_bf16(tmem + COL_A, ptx::desc_kmajor(a_dy + 32 * kq),
+                              ptx::desc_kmajor(b_v + 32 * kq), IDESC_KK, kq > 0);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)   // Z = dy S_hi^T
+                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(a_dy + 32 * kq),
+                              ptx::desc_kmajor(b_hi + 32 * kq), IDESC_KK, kq > 0);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)   // Z += dy S_lo^T
+                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(a_dy + 32 * kq),
+                              ptx::desc_kmajor(b_lo + 32 * kq), IDESC_KK, 1);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)   // U = Kt_hi^T V
+                ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kh + 32 * kq),
+                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, kq > 0);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)   // U += Kt_lo^T V
+                ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kl + 32 * kq),
+                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, 1);
+            ptx::mma_commit(&s.mma1);
+            issued1 = n;
+        }
+        if (!ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), budget)) s.abort = 1;
+        ptx::tc_fence_after();
+
+        // -------------------------------------------------------- state chain
+        {
+            uint32_t U[32];
+            ptx::tmem_ld32(tmem + tlane + COL_U + 32 * hh, U);
+            ptx::tmem_wait_ld();
+            if (row_lane) {
+                const float g = s.gamma[row];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                    uint4 hi, lo;
+                    split8(f, hi, lo);
+                    *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, 4 * hh + cc)) = hi;
+                    *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, 4 * hh + cc)) = lo;
+                }
+            }
+        }
+        // -------------------------------------------------------- causal scores
+        {
+            uint32_t A[32];
+            ptx::tmem_ld32(tmem + tlane + COL_A + 32 * hh, A);
+            ptx::tmem_wait_ld();
+            if (row_lane) {
+                const int t = row;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float a[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int sx = 32 * hh + 8 * cc + e;
+                        const float x = __uint_as_float(A[8 * cc + e]);
+                        if (sx == t) s.diag[t] = x;
+                        a[e] = sx < t ? x : 0.f;
+                    }
+                    uint4 hi, lo;
+                    split8(a, hi, lo);
+                    *reinterpret_cast<uint4*>(s.a_hi + sw_chunk(t, 4 * hh + cc)) = hi;
+                    *reinterpret_cast<uint4*>(s.a_lo + sw_chunk(t, 4 * hh + cc)) = lo;
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+        if (s.abort) { failed = true; break; }
+
+        // -------------------------------------------------------- MMA 2: Z += A Kh
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            const uint32_t ah = ptx::smem_addr(s.a_hi), al = ptx::smem_addr(s.a_lo);
+            const uint32_t bh_ = ptx::smem_addr(s.kh_hi), bl = ptx::smem_addr(s.kh_lo);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(ah + 32 * kq),
+                              ptx::desc_mnmajor(bh_ + 2048 * kq), IDESC_KM, 1);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(ah + 32 * kq),
+                              ptx::desc_mnmajor(bl + 2048 * kq), IDESC_KM, 1);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(al + 32 * kq),
+                              ptx::desc_mnmajor(bh_ + 2048 * kq), IDESC_KM, 1);
+            ptx::mma_commit(&s.mma2);
+            issued2 = n;
+        }
+        // r of this lane's row while the products run
+        const int t = row;
+        const bool live = row_lane && t < valid;
+        const size_t gx = (((size_t)b * T + t0 + t) * H + h) * 64 + 32 * hh;
+        float rv[32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            float f[8];
+            if (live) {
+                unpack8(__ldg(reinterpret_cast<const uint4*>(r + gx + 8 * cc)), f);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) rv[8 * cc + e] = f[e];
+        }
+        if (!ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), budget)) s.abort = 1;
+        ptx::tc_fence_after();
+
+        // -------------------------------------------------------- output
+        {
+            uint32_t Z[32];
+            ptx::tmem_ld32(tmem + tlane + COL_Z + 32 * hh, Z);
+            ptx::tmem_wait_ld();
+            if (row_lane) {
+                const float dg = s.diag[t];
+                float* pdst = P + gx;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float kx[8], o[8], pv[8];
+                    unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(t, 4 * hh + cc)), kx);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 8 * cc + e, i = 32 * hh + j;
+                        const float pair = s.F[t][i] * __uint_as_float(Z[j]);   // dr minus the bonus
+                        const float kd = kx[e] * dg;
+                        o[e] = fmaf(s.u[i], kd, pair);
+                        pv[e] = rv[j] * pair;
+                        du_acc[j] = fmaf(rv[j], kd, du_acc[j]);
+                    }
+                    *reinterpret_cast<uint4*>(y_tile + sw_chunk(t, 4 * hh + cc)) = pack8(o);
+                    if (live) {
+                        reinterpret_cast<float4*>(pdst + 8 * cc)[0] = make_float4(pv[0], pv[1], pv[2], pv[3]);
+                        reinterpret_cast<float4*>(pdst + 8 * cc)[1] = make_float4(pv[4], pv[5], pv[6], pv[7]);
+                    }
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+        if (s.abort) { failed = true; break; }
+        if (tid == 0) {
+            if (gw_check(status, t0 < T && h < H)) {
+                ptx::tma_store_4d(&tm_dr, y_tile, 0, h, t0, b);
+                ptx::bulk_commit();
+            }
+            // every thread is past its reads of this stage and the MMAs that read it are done
+            if (n + kStages < NC) {
+                ptx::fence_proxy_async_smem();
+                issue_load(n + kStages);
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ finish / drain
+    if (failed || out_of_range) {
+        if (tid == 0) {
+            if (failed) atomicExch(status, 1);
+            // copies still in flight: chunks n .. min(NC, n + kStages) - 1 may have been issued
+            for (int c = n; c < NC && c < n + kStages; ++c)
+                ptx::mbar_wait(&s.full[c % kStages], (uint32_t)((c / kStages) & 1), drain_budget);
+            if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), drain_budget);
+            if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), drain_budget);
+            fallback[bh] = 1;   // the CUDA-core scan redoes this (b,h)
+        }
+    } else {
+        // E[i] = sum_j S_T[i][j] dS_T[i][j]; du[i] = sum_t r_t[i] k_t[i] (v_t . dy_t)
+        float ev = 0.f;
+        if (dS_T && row_lane) {
+            const float* g = dS_T + (size_t)bh * 4096 + row * 64 + 32 * hh;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(g + j);
+                ev = fmaf(S[j], x.x, fmaf(S[j + 1], x.y, fmaf(S[j + 2], x.z, fmaf(S[j + 3], x.w, ev))));
+            }
+        }
+        if (row_lane) s.epart[hh][row] = ev;
+        // du: sum over the 16 row lanes of this warp, then over the 4 row quarters
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            float x = du_acc[j];
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            du_acc[j] = x;
+        }
+        if (lane == 0)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s.dupart[q][32 * hh + j] = du_acc[j];
+        __syncthreads();
+        if (tid < 64) {
+            E[(size_t)bh * 64 + tid] = s.epart[0][tid] + s.epart[1][tid];
+            du_part[(size_t)bh * 64 + tid] =
+                s.dupart[0][tid] + s.dupart[1][tid] + s.dupart[2][tid] + s.dupart[3][tid];
+        }
+        if (tid == 0) fallback[bh] = 0;
+    }
+    if (tid == 0) ptx::bulk_wait<0>();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+size_t bwd_dr_tc_smem_bytes() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float* u,
+                             const float* state_in, const float* dS_T, float* P, float* E,
+                             float* du_part, int* fallback, int B, int T, int H, int* status,
+                             long long budget, cudaStream_t st) {
+    const size_t smem = bwd_dr_tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_dr_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    wkv6_bwd_dr_tc_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(r), u,
+        state_in, dS_T, P, E, du_part, fallback, T, H, status, budget, 4000000000LL);
+    return cudaGetLastError();
+}
+
+}  // namespace goldwkv

@@ -90,9 +90,10 @@ def test_backward_and_gold_workspace_queries():
     assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 0) == \
         r256(8 * x) + r256(8 * bh) + r256(4 * bh)
     base16 = r256(4 * x) + r256(4 * bh) + r256(4 * bh)
-    # bf16 base form: + reversed k, r, dy, omega, dv and the chunked prefill's workspace
+    # bf16 base form: + reversed k, r, dy, omega, dv, the chunked prefill's workspace and
+    # the tensor-core dr kernel's fallback flag per (b,h)
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16) == \
-        base16 + 5 * r256(2 * x) + hand(B, H)
+        base16 + 5 * r256(2 * x) + hand(B, H) + r256(4 * B * H)
     assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 1) == base16
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16, c2=True) == base16
     assert binding.backward_workspace_bytes(B, 0, H, 64, torch.bfloat16) == 0

@@ -4,8 +4,9 @@ Every gradient (dr, dk, dv, domega, du, dS0) is compared element by element at s
 span several 32-token tiles and a ragged tail, for fp32 and bf16 I/O, with and without an
 initial state and a final-state gradient; the 1.5B-layer shape (B8 T4096 H32, bf16) is
 checked on sampled heads.  With bf16 I/O dv comes from the chunked tensor-core prefill run
-on time-reversed copies: extreme decays (hand-over to the level kernel) and a forced
-sequence split cover that path.  Also: the empty sequence, determinism and argument
+on time-reversed copies, and dr from the tensor-core dr kernel (a (b,h) whose decays it
+cannot take falls back to the CUDA-core scan): extreme decays (hand-over to the level
+kernel, dr fallback) and a forced sequence split cover those paths.  Also: the empty sequence, determinism and argument
 checks.
 """
 import ctypes
@@ -62,9 +63,26 @@ def test_backward_fp32(oracle, T):
     _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.float32])
 
 
-@pytest.mark.parametrize("T", [64, 513])
+@pytest.mark.parametrize("T", [1, 64, 65, 130, 513])
 def test_backward_bf16(oracle, T):
     inp = _problem(9850 + T, B=2, T=T, H=4, dtype=torch.bfloat16)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
+
+
+def test_backward_bf16_zero_state_no_state_gradient(oracle):
+    """The tensor-core dr pass with no initial state and no final-state gradient (E = 0)."""
+    inp = _problem(9871, B=3, T=200, H=2, dtype=torch.bfloat16, s0=False, ds=False)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
+
+
+def test_backward_bf16_some_heads_fall_back(oracle):
+    """bf16 dr runs on the tensor cores per (b,h) while every chunk's decay range fits the
+    one-sided factorisation; one batch row's head with decays near zero is redone by the
+    CUDA-core scan, the rest are not."""
+    inp = _problem(9872, B=3, T=300, H=3, dtype=torch.bfloat16)
+    om = inp["omega"].float()
+    om[1, 100:180, 2, ::2] = 3.0
+    inp["omega"] = om.to(torch.bfloat16)
     _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
 
 
