@@ -655,11 +655,13 @@ size_t backward_bytes(int B, int T, int H, int D, wkv_dtype io, bool tc_dv) {
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     const size_t x = (size_t)B * T * H * D, bh = (size_t)B * H * D;
     size_t bytes = round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
-    // tensor-core path: 5 time-reversed copies, the chunked prefill's workspace, and the dr
-    // kernel's fallback flag per (b,h)
+    // tensor-core path: 5 time-reversed copies and a reversed output, the chunked prefill's
+    // workspace, a fallback flag per (b,h) for dr and for dk, Q (fp32, reversed) and the
+    // decay gradient's per-chunk sums of P and Q
     if (tc_dv)
-        bytes += 5 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H)) +
-                 round256((size_t)B * H * sizeof(int));
+        bytes += 6 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H)) +
+                 2 * round256((size_t)B * H * sizeof(int)) + round256(x * sizeof(float)) +
+                 round256((size_t)B * H * ((T + kChunk - 1) / kChunk) * 128 * sizeof(float));
     return bytes;
 }
 
@@ -732,53 +734,95 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     uint8_t* E = ws + round256((size_t)B * T * H * D * acc);
     uint8_t* dpart = E + round256((size_t)B * H * D * acc);
     float* du_part = reinterpret_cast<float*>(dpart);
-    int* dr_flags = nullptr;   // set on the tensor-core path: which (b,h) the dr scan redoes
-    if (tc_dv) {
-        // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
-        // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.
-        // It runs through the chunked tensor-core prefill on time-reversed copies.
-        const size_t xr = round256(xbytes);
-        uint8_t* rev = dpart + round256((size_t)B * H * D * sizeof(float));
-        void* rk = rev;
-        void* rr = rev + xr;
-        void* rdy = rev + 2 * xr;
-        void* rom = rev + 3 * xr;
-        void* rdv = rev + 4 * xr;
-        uint8_t* cws = rev + 5 * xr;
-        const void* src[4] = {k, r, dy, omega};
-        void* dst[4] = {rk, rr, rdy, rom};
-        if (goldwkv::launch_reverse_tokens(src, dst, 4, B, T, H, st) != cudaSuccess)
-            return WKV_ERR_CUDA;
-        cudaError_t e = cudaSuccess;
-        if (!launch_chunked_path(rk, rr, rdy, rom, u, goldwkv::Variant{nullptr}, dstate_out,
-                                 nullptr, rdv, nullptr, B, T, H, choose_segments(B, T, H), false,
-                                 cws, st, &e) ||
-            e != cudaSuccess)
-            return WKV_ERR_CUDA;
-        const void* src_dv[1] = {rdv};
-        void* dst_dv[1] = {dv};
-        if (goldwkv::launch_reverse_tokens(src_dv, dst_dv, 1, B, T, H, st) != cudaSuccess)
-            return WKV_ERR_CUDA;
-        // dr (with P, E and du's parts) on the tensor cores; a (b,h) whose decay range the
-        // one-sided factorisation cannot take is flagged and left to the CUDA-core dr scan
-        dr_flags = reinterpret_cast<int*>(cws + chunked_bytes(B, H, choose_segments(B, T, H)));
-        CUtensorMap maps[5];
-        if (!goldwkv::make_token_map(&maps[0], dy, B, T, H) ||
-            !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
-            !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
-            !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
-            !goldwkv::make_token_map(&maps[4], dr, B, T, H))
-            return WKV_ERR_CUDA;
-        const long long budget = injected("timeout0") ? 0 : kSpinBudget;
-        if (goldwkv::launch_bwd_dr_tc(maps, r, u, state_in, dstate_out, static_cast<float*>(P),
-                                      reinterpret_cast<float*>(E), du_part, dr_flags, B, T, H,
-                                      reinterpret_cast<int*>(cws), budget, st) != cudaSuccess)
+    if (!tc_dv)
+        return from_cuda(goldwkv::launch_backward(r, k, v, omega, c2 ? nullptr : u, state_in, dy,
+                                                  dstate_out, dr, dk, dv, domega, du, dstate_in,
+                                                  P, E, du_part, B, T, H, bf16, /*with_dv=*/true,
+                                                  c2, st));
+    // Tensor-core path (bf16, base form).  Workspace after P, E and du_part: time-reversed
+    // copies of k, r, dy, omega and v, a reversed output (dv, then dk), the chunked
+    // prefill's workspace (its first word is the status word every tensor-core pass here
+    // reports an expired wait in), a fallback flag per (b,h) for each of dr and dk, the
+    // reversed Q and the decay gradient's chunk sums.
+    const int P_seg = choose_segments(B, T, H);
+    const size_t xr = round256(xbytes);
+    const size_t flags = round256((size_t)B * H * sizeof(int));
+    uint8_t* rev = dpart + round256((size_t)B * H * D * sizeof(float));
+    void* rk = rev;
+    void* rr = rev + xr;
+    void* rdy = rev + 2 * xr;
+    void* rom = rev + 3 * xr;
+    void* rv = rev + 4 * xr;
+    void* rout = rev + 5 * xr;
+    uint8_t* cws = rev + 6 * xr;
+    int* status = reinterpret_cast<int*>(cws);
+    int* dr_flags = reinterpret_cast<int*>(cws + chunked_bytes(B, H, P_seg));
+    int* dk_flags = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(dr_flags) + flags);
+    float* q_rev = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dk_flags) + flags);
+    float* sums = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(q_rev) +
+                                           round256((size_t)B * T * H * D * sizeof(float)));
+    const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+    const void* src[5] = {k, r, dy, omega, v};
+    void* dst[5] = {rk, rr, rdy, rom, rv};
+    if (goldwkv::launch_reverse_tokens(src, dst, 5, B, T, H, st) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r swapped
+    // and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.  It runs
+    // through the chunked tensor-core prefill on the reversed copies.
+    cudaError_t e = cudaSuccess;
+    if (!launch_chunked_path(rk, rr, rdy, rom, u, goldwkv::Variant{nullptr}, dstate_out, nullptr,
+                             rout, nullptr, B, T, H, P_seg, false, cws, st, &e) ||
+        e != cudaSuccess)
+        return WKV_ERR_CUDA;
+    {
+        const void* s1[1] = {rout};
+        void* d1[1] = {dv};
+        if (goldwkv::launch_reverse_tokens(s1, d1, 1, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
-    return from_cuda(goldwkv::launch_backward(r, k, v, omega, c2 ? nullptr : u, state_in, dy,
-                                              dstate_out, dr, dk, dv, domega, du, dstate_in, P,
-                                              E, du_part, B, T, H, bf16, /*with_dv=*/!tc_dv, c2,
-                                              st, dr_flags));
+    // dr (with P, E and du's parts) as the chunked readout of the forward state; a (b,h)
+    // whose decay range the one-sided factorisation cannot take is flagged and redone by the
+    // CUDA-core dr scan, so that P and E are complete before the decay gradient
+    CUtensorMap maps[5];
+    if (!goldwkv::make_token_map(&maps[0], dy, B, T, H) ||
+        !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
+        !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
+        !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
+        !goldwkv::make_token_map(&maps[4], dr, B, T, H))
+        return WKV_ERR_CUDA;
+    if (goldwkv::launch_bwd_dr_tc(maps, r, u, state_in, dstate_out, static_cast<float*>(P),
+                                  reinterpret_cast<float*>(E), du_part, dr_flags, B, T, H, status,
+                                  budget, st) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    if (goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv, domega,
+                                 du, dstate_in, P, E, du_part, B, T, H, bf16, false, false, st,
+                                 dr_flags, nullptr, goldwkv::kPhaseDr) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    // dk (and dS0, Q) as the same readout in reversed time: query v, key r, value dy
+    if (!goldwkv::make_token_map(&maps[0], rv, B, T, H) ||
+        !goldwkv::make_token_map(&maps[1], rr, B, T, H) ||
+        !goldwkv::make_token_map(&maps[2], rdy, B, T, H) ||
+        !goldwkv::make_token_map(&maps[3], rom, B, T, H) ||
+        !goldwkv::make_token_map(&maps[4], rout, B, T, H))
+        return WKV_ERR_CUDA;
+    if (goldwkv::launch_bwd_dk_tc(maps, rk, u, dstate_out, q_rev, dstate_in, dk_flags, B, T, H,
+                                  status, budget, st) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    {
+        const void* s1[1] = {rout};
+        void* d1[1] = {dk};
+        if (goldwkv::launch_reverse_tokens(s1, d1, 1, B, T, H, st) != cudaSuccess)
+            return WKV_ERR_CUDA;
+    }
+    if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_rev, sums,
+                                   reinterpret_cast<const float*>(E), omega, domega, B, T, H,
+                                   st) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    // the dk scan (with its decay gradient and dS0) for the flagged (b,h), then du
+    return from_cuda(goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
+                                              dv, domega, du, dstate_in, P, E, du_part, B, T, H,
+                                              bf16, false, false, st, nullptr, dk_flags,
+                                              goldwkv::kPhaseDk | goldwkv::kPhaseDu));
 }
 
 }  // namespace

@@ -522,7 +522,9 @@ wkv6_bwd_dk_domega_kernel(const IO* __restrict__ r, const IO* __restrict__ k,
                           const float* __restrict__ u, const IO* __restrict__ dy,
                           const float* __restrict__ dS_T, IO* __restrict__ dk,
                           IO* __restrict__ domega, typename Prec<IO>::Acc* __restrict__ P,
-                          typename Prec<IO>::Acc* __restrict__ E, float* dS_0, int T, int H) {
+                          typename Prec<IO>::Acc* __restrict__ E, float* dS_0, int T, int H,
+                          const int* dk_only) {
+    if (dk_only != nullptr && dk_only[blockIdx.x] == 0) return;
     __shared__ __align__(16) typename SweepSmem<IO>::Row s;
     row_sweep<IO, true, kC2>(s, r, k, dy, v, omega, u, dS_T, dk, P, domega, E, nullptr, nullptr, dS_0,
                         T, H);
@@ -561,21 +563,26 @@ cudaError_t launch_typed(const void* r, const void* k, const void* v, const void
                          const float* u, const float* state_in, const void* dy,
                          const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                          float* du, float* dstate_in, void* P_, void* E_, float* du_part, int B,
-                         int T, int H, bool with_dv, cudaStream_t st, const int* dr_only) {
+                         int T, int H, bool with_dv, cudaStream_t st, const int* dr_only,
+                         const int* dk_only, int phases) {
     using Acc = typename Prec<IO>::Acc;
     const IO *r_ = (const IO*)r, *k_ = (const IO*)k, *v_ = (const IO*)v, *o_ = (const IO*)omega,
              *dy_ = (const IO*)dy;
     Acc *P = static_cast<Acc*>(P_), *E = static_cast<Acc*>(E_);
     const unsigned bh = (unsigned)(B * H);
-    wkv6_bwd_dr_dv_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf, with_dv ? 2 : 1), kThreads, 0, st>>>(
-        r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H,
-        dr_only);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    wkv6_bwd_dk_domega_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf), kThreads, 0, st>>>(
-        r_, k_, v_, o_, u, dy_, dstate_out, (IO*)dk, (IO*)domega, P, E, dstate_in, T, H);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (kC2) return cudaSuccess;   // no bonus u in this form
+    cudaError_t e = cudaSuccess;
+    if (phases & kPhaseDr) {
+        wkv6_bwd_dr_dv_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf, with_dv ? 2 : 1), kThreads, 0, st>>>(
+            r_, k_, v_, o_, u, state_in, dy_, dstate_out, (IO*)dr, (IO*)dv, P, E, du_part, T, H,
+            dr_only);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (phases & kPhaseDk) {
+        wkv6_bwd_dk_domega_kernel<IO, kC2><<<dim3(bh, kHeadSize / kHalf), kThreads, 0, st>>>(
+            r_, k_, v_, o_, u, dy_, dstate_out, (IO*)dk, (IO*)domega, P, E, dstate_in, T, H, dk_only);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (kC2 || !(phases & kPhaseDu)) return cudaSuccess;   // (no bonus u in Finch-C2's form)
     wkv6_bwd_du_kernel<<<H, kHeadSize, 0, st>>>(du_part, du, B, H);
     return cudaGetLastError();
 }
@@ -587,21 +594,21 @@ cudaError_t launch_backward(const void* r, const void* k, const void* v, const v
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
                             int B, int T, int H, bool bf16, bool with_dv, bool c2,
-                            cudaStream_t st, const int* dr_only) {
+                            cudaStream_t st, const int* dr_only, const int* dk_only, int phases) {
     using BF = __nv_bfloat16;
     if (c2)
         return bf16 ? launch_typed<BF, true>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
                                             dv, domega, du, dstate_in, P, E, du_part, B, T, H,
-                                            with_dv, st, dr_only)
+                                            with_dv, st, dr_only, dk_only, phases)
                     : launch_typed<float, true>(r, k, v, omega, u, state_in, dy, dstate_out, dr,
                                                 dk, dv, domega, du, dstate_in, P, E, du_part, B,
-                                                T, H, with_dv, st, dr_only);
+                                                T, H, with_dv, st, dr_only, dk_only, phases);
     return bf16 ? launch_typed<BF, false>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv,
                                           domega, du, dstate_in, P, E, du_part, B, T, H, with_dv,
-                                          st, dr_only)
+                                          st, dr_only, dk_only, phases)
                 : launch_typed<float, false>(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
                                              dv, domega, du, dstate_in, P, E, du_part, B, T, H,
-                                             with_dv, st, dr_only);
+                                             with_dv, st, dr_only, dk_only, phases);
 }
 
 cudaError_t launch_reverse_tokens(const void* const* src, void* const* dst, int n, int B, int T,

@@ -6,6 +6,10 @@
 
 namespace goldwkv {
 
+// Phases of launch_backward: the dr (and dv) sweep, the dk sweep with the decay gradient, the
+// sum of du over the batch.
+constexpr int kPhaseDr = 1, kPhaseDk = 2, kPhaseDu = 4, kPhaseAll = 7;
+
 // Backward of the base recurrence: three token-by-token sweeps and a reduction of du over
 // the batch.  Scratch the caller provides: P [B][T][H][64] and E [B*H][64] of the scans
 // accumulation type (fp64 for fp32 I/O, fp32 for bf16 I/O), du_part [B*H][64] fp32.
@@ -13,13 +17,15 @@ namespace goldwkv {
 // with_dv == false: dv is computed elsewhere (the caller's tensor-core path); dv unused.
 // c2: Finch-C2's exact form (key k (1 - w), no bonus; u and du unused).
 // dr_only != nullptr: the dr scan runs only for the (b,h) with dr_only[bh] != 0 (the others'
-// dr, P, E and du_part were written by launch_bwd_dr_tc).
+// dr, P, E and du_part were written by launch_bwd_dr_tc); dk_only likewise for the dk scan
+// (dk, domega, dS_0 from launch_bwd_dk_tc and launch_bwd_domega).
 cudaError_t launch_backward(const void* r, const void* k, const void* v, const void* omega,
                             const float* u, const float* state_in, const void* dy,
                             const float* dstate_out, void* dr, void* dk, void* dv, void* domega,
                             float* du, float* dstate_in, void* P, void* E, float* du_part,
                             int B, int T, int H, bool bf16, bool with_dv, bool c2,
-                            cudaStream_t st, const int* dr_only = nullptr);
+                            cudaStream_t st, const int* dr_only = nullptr,
+                            const int* dk_only = nullptr, int phases = kPhaseAll);
 
 // dr of the base form (bf16 I/O) on the tensor cores (csrc/backward_tc_sm100.cu), one CTA per
 // (b,h): writes dr and, as the CUDA-core dr scan does, P, E and du_part.  maps: dy, k, v,
@@ -31,7 +37,22 @@ cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float
                              float* du_part, int* fallback, int B, int T, int H, int* status,
                              long long budget, cudaStream_t st);
 
-constexpr int kMaxReverse = 4;
+// dk of the base form on the tensor cores, the same readout on time-reversed copies: maps
+// v, r, dy, omega, dk (all reversed); k_rev read directly.  Writes dk (reversed), Q_rev (the
+// pair terms k_t (dk_t - bonus), reversed, fp32 [B][T][H][64]) and dS_0 (if non-null).
+// fallback / status as for launch_bwd_dr_tc.
+cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k_rev, const float* u,
+                             const float* dS_T, float* Q_rev, float* dS_0, int* fallback, int B,
+                             int T, int H, int* status, long long budget, cudaStream_t st);
+
+// domega (bf16) from P, Q_rev and E through the identity
+//     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,  domega_t = dlog w_t (-exp(omega_t));
+// sums: scratch of B*H*ceil(T/64)*128 floats.
+cudaError_t launch_bwd_domega(const float* P, const float* Q_rev, float* sums, const float* E,
+                              const void* omega, void* domega, int B, int T, int H,
+                              cudaStream_t st);
+
+constexpr int kMaxReverse = 5;
 
 // dst[i] = src[i] with the token axis reversed, for n <= kMaxReverse bf16 tensors
 // [B][T][H][64] (16-byte aligned, not overlapping).

@@ -25,8 +25,13 @@
 //   out   : dr = F Z + u k diag (bf16 tile, TMA store); for the decay gradient the pair
 //           terms ending at t, P_t = r_t (dr_t - bonus) (fp32), and du's per-(b,h) sums.
 // At the end: E[i] = sum_j S_T[i][j] dS_T[i][j] (with the dk scan's decay gradient) and du.
-// P, E and du_part have the layout and meaning of the CUDA-core dr scan's (csrc/backward.cu),
-// so the dk scan that follows reads them unchanged.  Every mbarrier wait is bounded.
+// P, E and du_part have the layout and meaning of the CUDA-core dr scan's (csrc/backward.cu).
+//
+// dk is the same computation in reversed time (kDk): with G_{t-1} = diag(w_t) G_t + r_t^T dy_t
+// the state gradient, dk_t[i] = sum_j G_t[i][j] v_t[j] + u[i] r_t[i] (v_t . dy_t), i.e. the
+// readout above on time-reversed copies with query v, key r, value dy, initial state dS_T;
+// its final state is dS_0, and its pair terms Q_t = k_t (dk_t - bonus) feed the decay
+// gradient (wkv6_bwd_domega kernels below).  Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -109,13 +114,17 @@ __device__ __forceinline__ uint32_t tr_off(int i, int lane) {
     return (uint32_t)(i * 128 + ((((lane >> 2)) ^ (i & 7)) << 4) + (lane & 3) * 4);
 }
 
+// kDk == false (dr): query dy, key k, value v, aux r, x0 = state_in; writes P, E, du_part.
+// kDk == true (dk, time-reversed inputs): query v, key r, value dy, aux k, x0 = dS_T; writes
+// Q (into P) and the final state (dS_0) to x_final.
+template <bool kDk>
 __global__ void __launch_bounds__(kThreads, 1)
-wkv6_bwd_dr_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_k,
+wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_dr, const __nv_bfloat16* __restrict__ r,
                       const float* __restrict__ u, const float* state_in, const float* dS_T,
                       float* __restrict__ P, float* __restrict__ E, float* __restrict__ du_part,
-                      int* fallback, int T, int H, int* status, long long budget,
+                      float* x_final, int* fallback, int T, int H, int* status, long long budget,
                       long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
@@ -463,6 +472,14 @@ wkv6_bwd_dr_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_co
             if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), drain_budget);
             fallback[bh] = 1;   // the CUDA-core scan redoes this (b,h)
         }
+    } else if (kDk) {
+        if (x_final != nullptr && row_lane) {   // dS_0
+            float* dst = x_final + (size_t)bh * 4096 + row * 64 + 32 * hh;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+        if (tid == 0) fallback[bh] = 0;
     } else {
         // E[i] = sum_j S_T[i][j] dS_T[i][j]; du[i] = sum_t r_t[i] k_t[i] (v_t . dy_t)
         float ev = 0.f;
@@ -505,19 +522,100 @@ wkv6_bwd_dr_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_co
 
 }  // namespace
 
-size_t bwd_dr_tc_smem_bytes() { return sizeof(Smem) + 1024; }
+size_t bwd_readout_tc_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float* u,
                              const float* state_in, const float* dS_T, float* P, float* E,
                              float* du_part, int* fallback, int B, int T, int H, int* status,
                              long long budget, cudaStream_t st) {
-    const size_t smem = bwd_dr_tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_dr_tc_kernel,
+    const size_t smem = bwd_readout_tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_readout_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_bwd_dr_tc_kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
+    wkv6_bwd_readout_tc_kernel<false><<<(unsigned)(B * H), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(r), u,
-        state_in, dS_T, P, E, du_part, fallback, T, H, status, budget, 4000000000LL);
+        state_in, dS_T, P, E, du_part, nullptr, fallback, T, H, status, budget, 4000000000LL);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k_rev, const float* u,
+                             const float* dS_T, float* Q_rev, float* dS_0, int* fallback, int B,
+                             int T, int H, int* status, long long budget, cudaStream_t st) {
+    const size_t smem = bwd_readout_tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_readout_tc_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    wkv6_bwd_readout_tc_kernel<true><<<(unsigned)(B * H), kThreads, smem, st>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(k_rev), u,
+        dS_T, nullptr, Q_rev, nullptr, nullptr, dS_0, fallback, T, H, status, budget,
+        4000000000LL);
+    return cudaGetLastError();
+}
+
+namespace {
+
+// Decay gradient from the pair terms (the identity of csrc/backward.cu):
+//     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,   domega_t = dlog w_t (-exp(omega_t)),
+// P in token order, Q in reversed token order (row T-1-s holds Q_s).  First the column sums
+// of P and Q over each 64-token chunk, then per chunk the sums over the later chunks and a
+// reverse scan over its own tokens.  One thread per channel, one CTA per (b,h,chunk).
+__global__ void __launch_bounds__(64)
+wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q_rev,
+                        float* __restrict__ sums, int T, int H) {
+    const int NC = (T + C - 1) / C;
+    const int n = blockIdx.x % NC, bh = blockIdx.x / NC, b = bh / H, h = bh - (bh / H) * H;
+    const int i = threadIdx.x, t0 = n * C, valid = min(C, T - t0);
+    float sp = 0.f, sq = 0.f;
+#pragma unroll 8
+    for (int tt = 0; tt < valid; ++tt) {
+        const int t = t0 + tt;
+        sp += P[(((size_t)b * T + t) * H + h) * 64 + i];
+        sq += Q_rev[(((size_t)b * T + (T - 1 - t)) * H + h) * 64 + i];
+    }
+    float* o = sums + ((size_t)bh * NC + n) * 128;
+    o[i] = sp;
+    o[64 + i] = sq;
+}
+
+__global__ void __launch_bounds__(64)
+wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q_rev,
+                       const float* __restrict__ sums, const float* __restrict__ E,
+                       const __nv_bfloat16* __restrict__ omega, __nv_bfloat16* __restrict__ domega,
+                       int T, int H) {
+    const int NC = (T + C - 1) / C;
+    const int n = blockIdx.x % NC, bh = blockIdx.x / NC, b = bh / H, h = bh - (bh / H) * H;
+    const int i = threadIdx.x, t0 = n * C, valid = min(C, T - t0);
+    // E + sum over the later chunks of (P - Q)
+    float acc = E[(size_t)bh * 64 + i];
+    for (int m = n + 1; m < NC; ++m) {
+        const float* o = sums + ((size_t)bh * NC + m) * 128;
+        acc += o[i] - o[64 + i];
+    }
+    // reverse over this chunk: dlog w_t = acc_after(t) - Q_t, with acc_after(t) = E + sum_{s>t}
+    // P_s - sum_{s>t} Q_s
+    for (int tt = valid - 1; tt >= 0; --tt) {
+        const int t = t0 + tt;
+        const size_t x = (((size_t)b * T + t) * H + h) * 64 + i;
+        const float q = Q_rev[(((size_t)b * T + (T - 1 - t)) * H + h) * 64 + i];
+        const float dl = acc - q;
+        domega[x] = __float2bfloat16_rn(dl * -__expf(__bfloat162float(omega[x])));
+        acc += P[x] - q;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_domega(const float* P, const float* Q_rev, float* sums, const float* E,
+                              const void* omega, void* domega, int B, int T, int H,
+                              cudaStream_t st) {
+    const unsigned blocks = (unsigned)((long)B * H * ((T + C - 1) / C));
+    if (blocks == 0) return cudaSuccess;
+    wkv6_bwd_pq_sums_kernel<<<blocks, 64, 0, st>>>(P, Q_rev, sums, T, H);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    wkv6_bwd_domega_kernel<<<blocks, 64, 0, st>>>(P, Q_rev, sums, E,
+                                                  static_cast<const __nv_bfloat16*>(omega),
+                                                  static_cast<__nv_bfloat16*>(domega), T, H);
     return cudaGetLastError();
 }
 

@@ -90,10 +90,13 @@ def test_backward_and_gold_workspace_queries():
     assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 0) == \
         r256(8 * x) + r256(8 * bh) + r256(4 * bh)
     base16 = r256(4 * x) + r256(4 * bh) + r256(4 * bh)
-    # bf16 base form: + reversed k, r, dy, omega, dv, the chunked prefill's workspace and
-    # the tensor-core dr kernel's fallback flag per (b,h)
+    # bf16 base form: + reversed k, r, dy, omega, v and a reversed output, the chunked
+    # prefill's workspace, a fallback flag per (b,h) for each of the tensor-core dr and dk
+    # passes, Q (fp32) and two per-chunk column sums per (b,h)
+    nc = (T + 63) // 64
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16) == \
-        base16 + 5 * r256(2 * x) + hand(B, H) + r256(4 * B * H)
+        base16 + 6 * r256(2 * x) + hand(B, H) + 2 * r256(4 * B * H) + r256(4 * x) + \
+        r256(B * H * nc * 128 * 4)
     assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 1) == base16
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16, c2=True) == base16
     assert binding.backward_workspace_bytes(B, 0, H, 64, torch.bfloat16) == 0
