@@ -740,10 +740,10 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
                                                   P, E, du_part, B, T, H, bf16, /*with_dv=*/true,
                                                   c2, st));
     // Tensor-core path (bf16, base form).  Workspace after P, E and du_part: time-reversed
-    // copies of k, r, dy, omega and v, a reversed output (dv, then dk), the chunked
+    // copies of k, r, dy, omega and v, the reversed dv, the chunked
     // prefill's workspace (its first word is the status word every tensor-core pass here
-    // reports an expired wait in), a fallback flag per (b,h) for each of dr and dk, the
-    // reversed Q and the decay gradient's chunk sums.
+    // reports an expired wait in), a fallback flag per (b,h) for each of dr and dk, Q and the
+    // decay gradient's chunk sums.
     const int P_seg = choose_segments(B, T, H);
     const size_t xr = round256(xbytes);
     const size_t flags = round256((size_t)B * H * sizeof(int));
@@ -758,8 +758,8 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     int* status = reinterpret_cast<int*>(cws);
     int* dr_flags = reinterpret_cast<int*>(cws + chunked_bytes(B, H, P_seg));
     int* dk_flags = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(dr_flags) + flags);
-    float* q_rev = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dk_flags) + flags);
-    float* sums = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(q_rev) +
+    float* q_tok = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dk_flags) + flags);
+    float* sums = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(q_tok) +
                                            round256((size_t)B * T * H * D * sizeof(float)));
     const long long budget = injected("timeout0") ? 0 : kSpinBudget;
     const void* src[5] = {k, r, dy, omega, v};
@@ -798,23 +798,18 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
                                  du, dstate_in, P, E, du_part, B, T, H, bf16, false, false, st,
                                  dr_flags, nullptr, goldwkv::kPhaseDr) != cudaSuccess)
         return WKV_ERR_CUDA;
-    // dk (and dS0, Q) as the same readout in reversed time: query v, key r, value dy
+    // dk (and dS0, Q) as the same readout in reversed time: query v, key r, value dy; dk and
+    // Q go straight to token order
     if (!goldwkv::make_token_map(&maps[0], rv, B, T, H) ||
         !goldwkv::make_token_map(&maps[1], rr, B, T, H) ||
         !goldwkv::make_token_map(&maps[2], rdy, B, T, H) ||
         !goldwkv::make_token_map(&maps[3], rom, B, T, H) ||
         !goldwkv::make_token_map(&maps[4], rout, B, T, H))
         return WKV_ERR_CUDA;
-    if (goldwkv::launch_bwd_dk_tc(maps, rk, u, dstate_out, q_rev, dstate_in, dk_flags, B, T, H,
+    if (goldwkv::launch_bwd_dk_tc(maps, k, u, dstate_out, dk, q_tok, dstate_in, dk_flags, B, T, H,
                                   status, budget, st) != cudaSuccess)
         return WKV_ERR_CUDA;
-    {
-        const void* s1[1] = {rout};
-        void* d1[1] = {dk};
-        if (goldwkv::launch_reverse_tokens(s1, d1, 1, B, T, H, st) != cudaSuccess)
-            return WKV_ERR_CUDA;
-    }
-    if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_rev, sums,
+    if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_tok, sums,
                                    reinterpret_cast<const float*>(E), omega, domega, B, T, H,
                                    st) != cudaSuccess)
         return WKV_ERR_CUDA;

@@ -38,17 +38,17 @@ cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float
                              long long budget, cudaStream_t st);
 
 // dk of the base form on the tensor cores, the same readout on time-reversed copies: maps
-// v, r, dy, omega, dk (all reversed); k_rev read directly.  Writes dk (reversed), Q_rev (the
-// pair terms k_t (dk_t - bonus), reversed, fp32 [B][T][H][64]) and dS_0 (if non-null).
-// fallback / status as for launch_bwd_dr_tc.
-cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k_rev, const float* u,
-                             const float* dS_T, float* Q_rev, float* dS_0, int* fallback, int B,
-                             int T, int H, int* status, long long budget, cudaStream_t st);
+// v, r, dy, omega (all reversed) and any valid token map (unused); k in token order.  Writes
+// dk and Q (the pair terms k_t (dk_t - bonus), fp32 [B][T][H][64]) in token order and dS_0
+// (if non-null).  fallback / status as for launch_bwd_dr_tc.
+cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k, const float* u,
+                             const float* dS_T, void* dk, float* Q, float* dS_0, int* fallback,
+                             int B, int T, int H, int* status, long long budget, cudaStream_t st);
 
-// domega (bf16) from P, Q_rev and E through the identity
+// domega (bf16) from P, Q (token order) and E through the identity
 //     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,  domega_t = dlog w_t (-exp(omega_t));
 // sums: scratch of B*H*ceil(T/64)*128 floats.
-cudaError_t launch_bwd_domega(const float* P, const float* Q_rev, float* sums, const float* E,
+cudaError_t launch_bwd_domega(const float* P, const float* Q, float* sums, const float* E,
                               const void* omega, void* domega, int B, int T, int H,
                               cudaStream_t st);
 

@@ -115,8 +115,9 @@ __device__ __forceinline__ uint32_t tr_off(int i, int lane) {
 }
 
 // kDk == false (dr): query dy, key k, value v, aux r, x0 = state_in; writes P, E, du_part.
-// kDk == true (dk, time-reversed inputs): query v, key r, value dy, aux k, x0 = dS_T; writes
-// Q (into P) and the final state (dS_0) to x_final.
+// kDk == true (dk, time-reversed inputs): query v, key r, value dy, aux k (in token order),
+// x0 = dS_T; writes dk to out_direct and Q (into P), both in token order, and the final state
+// (dS_0) to x_final.
 template <bool kDk>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_k,
@@ -124,8 +125,8 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
                       const __grid_constant__ CUtensorMap tm_dr, const __nv_bfloat16* __restrict__ r,
                       const float* __restrict__ u, const float* state_in, const float* dS_T,
                       float* __restrict__ P, float* __restrict__ E, float* __restrict__ du_part,
-                      float* x_final, int* fallback, int T, int H, int* status, long long budget,
-                      long long drain_budget) {
+                      float* x_final, __nv_bfloat16* __restrict__ out_direct, int* fallback, int T,
+                      int H, int* status, long long budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -206,6 +207,17 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         uint8_t* w_tile = s.in[st][3];
         uint8_t* y_tile = s.ystage[n & 1];
         if (tid == 0) ptx::bulk_wait_read<1>();   // the store that last used y_tile has read it
+        // the aux row (r, or k in reversed time) of this lane, read now for the output step
+        const int t = row;
+        const bool live = row_lane && t < valid;
+        // this row in the caller's token order: dk's inputs are time-reversed, its outputs
+        // (dk, Q) and its aux input (k) are not
+        const int tok = kDk ? T - 1 - (t0 + t) : t0 + t;
+        const size_t gx = (((size_t)b * T + tok) * H + h) * 64 + 32 * hh;
+        uint4 rw[4];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+            rw[cc] = live ? __ldg(reinterpret_cast<const uint4*>(r + gx + 8 * cc)) : make_uint4(0, 0, 0, 0);
         if (!ptx::mbar_wait(&s.full[st], (uint32_t)((n / kStages) & 1), budget)) s.abort = 1;
 
         // -------------------------------------------------------- prep
@@ -395,23 +407,6 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
             ptx::mma_commit(&s.mma2);
             issued2 = n;
         }
-        // r of this lane's row while the products run
-        const int t = row;
-        const bool live = row_lane && t < valid;
-        const size_t gx = (((size_t)b * T + t0 + t) * H + h) * 64 + 32 * hh;
-        float rv[32];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            float f[8];
-            if (live) {
-                unpack8(__ldg(reinterpret_cast<const uint4*>(r + gx + 8 * cc)), f);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) rv[8 * cc + e] = f[e];
-        }
         if (!ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), budget)) s.abort = 1;
         ptx::tc_fence_after();
 
@@ -425,18 +420,22 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
                 float* pdst = P + gx;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    float kx[8], o[8], pv[8];
+                    float kx[8], o[8], pv[8], rv[8];
                     unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(t, 4 * hh + cc)), kx);
+                    unpack8(rw[cc], rv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = 8 * cc + e, i = 32 * hh + j;
                         const float pair = s.F[t][i] * __uint_as_float(Z[j]);   // dr minus the bonus
                         const float kd = kx[e] * dg;
                         o[e] = fmaf(s.u[i], kd, pair);
-                        pv[e] = rv[j] * pair;
-                        du_acc[j] = fmaf(rv[j], kd, du_acc[j]);
+                        pv[e] = rv[e] * pair;
+                        du_acc[j] = fmaf(rv[e], kd, du_acc[j]);
                     }
-                    *reinterpret_cast<uint4*>(y_tile + sw_chunk(t, 4 * hh + cc)) = pack8(o);
+                    if (!kDk)
+                        *reinterpret_cast<uint4*>(y_tile + sw_chunk(t, 4 * hh + cc)) = pack8(o);
+                    else if (live)   // dk straight to its row in token order
+                        *reinterpret_cast<uint4*>(out_direct + gx + 8 * cc) = pack8(o);
                     if (live) {
                         reinterpret_cast<float4*>(pdst + 8 * cc)[0] = make_float4(pv[0], pv[1], pv[2], pv[3]);
                         reinterpret_cast<float4*>(pdst + 8 * cc)[1] = make_float4(pv[4], pv[5], pv[6], pv[7]);
@@ -449,7 +448,7 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         __syncthreads();
         if (s.abort) { failed = true; break; }
         if (tid == 0) {
-            if (gw_check(status, t0 < T && h < H)) {
+            if (!kDk && gw_check(status, t0 < T && h < H)) {
                 ptx::tma_store_4d(&tm_dr, y_tile, 0, h, t0, b);
                 ptx::bulk_commit();
             }
@@ -534,21 +533,22 @@ cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float
     if (e != cudaSuccess) return e;
     wkv6_bwd_readout_tc_kernel<false><<<(unsigned)(B * H), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(r), u,
-        state_in, dS_T, P, E, du_part, nullptr, fallback, T, H, status, budget, 4000000000LL);
+        state_in, dS_T, P, E, du_part, nullptr, nullptr, fallback, T, H, status, budget,
+        4000000000LL);
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k_rev, const float* u,
-                             const float* dS_T, float* Q_rev, float* dS_0, int* fallback, int B,
-                             int T, int H, int* status, long long budget, cudaStream_t st) {
+cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k, const float* u,
+                             const float* dS_T, void* dk, float* Q, float* dS_0, int* fallback,
+                             int B, int T, int H, int* status, long long budget, cudaStream_t st) {
     const size_t smem = bwd_readout_tc_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_readout_tc_kernel<true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     wkv6_bwd_readout_tc_kernel<true><<<(unsigned)(B * H), kThreads, smem, st>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(k_rev), u,
-        dS_T, nullptr, Q_rev, nullptr, nullptr, dS_0, fallback, T, H, status, budget,
-        4000000000LL);
+        maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(k), u,
+        dS_T, nullptr, Q, nullptr, nullptr, dS_0, static_cast<__nv_bfloat16*>(dk), fallback, T, H,
+        status, budget, 4000000000LL);
     return cudaGetLastError();
 }
 
@@ -556,11 +556,11 @@ namespace {
 
 // Decay gradient from the pair terms (the identity of csrc/backward.cu):
 //     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,   domega_t = dlog w_t (-exp(omega_t)),
-// P in token order, Q in reversed token order (row T-1-s holds Q_s).  First the column sums
+// P and Q in token order.  First the column sums
 // of P and Q over each 64-token chunk, then per chunk the sums over the later chunks and a
 // reverse scan over its own tokens.  One thread per channel, one CTA per (b,h,chunk).
 __global__ void __launch_bounds__(64)
-wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q_rev,
+wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q,
                         float* __restrict__ sums, int T, int H) {
     const int NC = (T + C - 1) / C;
     const int n = blockIdx.x % NC, bh = blockIdx.x / NC, b = bh / H, h = bh - (bh / H) * H;
@@ -570,7 +570,7 @@ wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q
     for (int tt = 0; tt < valid; ++tt) {
         const int t = t0 + tt;
         sp += P[(((size_t)b * T + t) * H + h) * 64 + i];
-        sq += Q_rev[(((size_t)b * T + (T - 1 - t)) * H + h) * 64 + i];
+        sq += Q[(((size_t)b * T + t) * H + h) * 64 + i];
     }
     float* o = sums + ((size_t)bh * NC + n) * 128;
     o[i] = sp;
@@ -578,7 +578,7 @@ wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q
 }
 
 __global__ void __launch_bounds__(64)
-wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q_rev,
+wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
                        const float* __restrict__ sums, const float* __restrict__ E,
                        const __nv_bfloat16* __restrict__ omega, __nv_bfloat16* __restrict__ domega,
                        int T, int H) {
@@ -596,7 +596,7 @@ wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q_
     for (int tt = valid - 1; tt >= 0; --tt) {
         const int t = t0 + tt;
         const size_t x = (((size_t)b * T + t) * H + h) * 64 + i;
-        const float q = Q_rev[(((size_t)b * T + (T - 1 - t)) * H + h) * 64 + i];
+        const float q = Q[x];
         const float dl = acc - q;
         domega[x] = __float2bfloat16_rn(dl * -__expf(__bfloat162float(omega[x])));
         acc += P[x] - q;
@@ -605,15 +605,15 @@ wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q_
 
 }  // namespace
 
-cudaError_t launch_bwd_domega(const float* P, const float* Q_rev, float* sums, const float* E,
+cudaError_t launch_bwd_domega(const float* P, const float* Q, float* sums, const float* E,
                               const void* omega, void* domega, int B, int T, int H,
                               cudaStream_t st) {
     const unsigned blocks = (unsigned)((long)B * H * ((T + C - 1) / C));
     if (blocks == 0) return cudaSuccess;
-    wkv6_bwd_pq_sums_kernel<<<blocks, 64, 0, st>>>(P, Q_rev, sums, T, H);
+    wkv6_bwd_pq_sums_kernel<<<blocks, 64, 0, st>>>(P, Q, sums, T, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_domega_kernel<<<blocks, 64, 0, st>>>(P, Q_rev, sums, E,
+    wkv6_bwd_domega_kernel<<<blocks, 64, 0, st>>>(P, Q, sums, E,
                                                   static_cast<const __nv_bfloat16*>(omega),
                                                   static_cast<__nv_bfloat16*>(domega), T, H);
     return cudaGetLastError();
