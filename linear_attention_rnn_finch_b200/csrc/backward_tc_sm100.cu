@@ -15,15 +15,18 @@
 // The state itself advances with the suffix factors Kt_s = k_s 2^(L_{C-1} - L_s) <= 1 (any
 // decay): S <- diag(2^L_{C-1}) S + Kt^T V.
 //
-// Per chunk (one CTA per (b,h), 256 threads, all warps in lockstep):
+// Steps of a chunk (one CTA per (b,h), 256 threads, all warps in lockstep):
 //   prep  : warp = 8 channels, lane = 2 tokens; log2 w, the prefix L by a warp scan, F (fp32),
 //           Kh and Kt^T as bf16 hi / lo tiles, gamma;
 //   MMA 1 : A = dy x v^T; Z = dy x S_hi^T + dy x S_lo^T; U = Kt_hi^T V + Kt_lo^T V;
-//   state : S <- gamma S + U in registers, S_hi / S_lo tiles for the next chunk;
 //   A     : strictly causal part, hi / lo tiles; the diagonal (v_t . dy_t) kept aside;
 //   MMA 2 : Z += A_hi Kh_hi + A_hi Kh_lo + A_lo Kh_hi;
+//   state : S <- gamma S + U in registers, S_hi / S_lo tiles for the next chunk;
 //   out   : dr = F Z + u k diag (bf16 tile, TMA store); for the decay gradient the pair
 //           terms ending at t, P_t = r_t (dr_t - bonus) (fp32), and du's per-(b,h) sums.
+// Pipelined over chunks: iteration n forms A(n), issues MMA 2(n), advances the state and
+// prepares chunk n+1 while MMA 2 runs, issues MMA 1(n+1), and forms the output of n while
+// MMA 1(n+1) runs (prep buffers, F, gamma and Z alternate by chunk parity).
 // At the end: E[i] = sum_j S_T[i][j] dS_T[i][j] (with the dk scan's decay gradient) and du.
 // P, E and du_part have the layout and meaning of the CUDA-core dr scan's (csrc/backward.cu).
 //
@@ -49,7 +52,7 @@ constexpr int kThreads = 256;
 constexpr int kStages = 2;
 constexpr int kTile = 64 * 64 * 2;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t COL_A = 0, COL_U = 64, COL_Z = 128;
+constexpr uint32_t COL_A = 0, COL_U = 64, COL_Z = 128;   // Z: 2 x 64 (chunk parity)
 constexpr uint32_t IDESC_KK = ptx::idesc_bf16(64, 64, 0, 0);
 constexpr uint32_t IDESC_KM = ptx::idesc_bf16(64, 64, 0, 1);
 constexpr float kMaxLog2Range = 86.5617f;   // ln 60
@@ -58,14 +61,14 @@ constexpr int kFPitch = 68;                 // floats per row of F (padded again
 
 struct __align__(1024) Smem {
     uint8_t in[kStages][4][kTile];   // dy, k, v, omega tiles per stage (TMA, 128B swizzle)
-    uint8_t kh_hi[kTile], kh_lo[kTile];     // Kh [s][i]
-    uint8_t kt_hi[kTile], kt_lo[kTile];     // Kt^T [i][s]
+    uint8_t kh_hi[2][kTile], kh_lo[2][kTile];   // Kh [s][i], per chunk parity
+    uint8_t kt_hi[2][kTile], kt_lo[2][kTile];   // Kt^T [i][s], per chunk parity
     uint8_t a_hi[kTile], a_lo[kTile];       // causal scores [t][s]
     uint8_t s_hi[kTile], s_lo[kTile];       // S [i][j]
     uint8_t ystage[2][kTile];               // dr tiles for the TMA store
-    float F[C][kFPitch];
+    float F[2][C][kFPitch];                 // per chunk parity
     float u[64];
-    float gamma[64];
+    float gamma[2][64];
     float diag[64];                         // v_t . dy_t
     float epart[2][64];                     // E halves
     float dupart[4][64];                    // du sums per row quarter
@@ -196,17 +199,145 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
     for (int j = 0; j < 32; ++j) du_acc[j] = 0.f;
 
     bool failed = false, out_of_range = false;
-    int n = 0, issued1 = -1, issued2 = -1;
-    for (; n < NC; ++n) {
-        const int st = n % kStages;
+    int issued1 = -1, issued2 = -1;
+    int last_load[kStages] = {-1, -1};   // latest chunk whose copy each stage received
+    if (tid == 0)
+        for (int m = 0; m < kStages && m < NC; ++m) last_load[m] = m;
+
+    // prep of chunk m into the buffers of parity m & 1 (all threads); false if a channel's
+    // log2 decay over the chunk is below -86.56
+    auto prep_chunk = [&](int m) -> bool {
+        const int st = m % kStages, pb = m & 1, valid = min(C, T - m * C);
+        const uint8_t* k_tile = s.in[st][1];
+        const uint8_t* w_tile = s.in[st][3];
+        const int cg = warp;                    // channels 8cg .. 8cg+7
+        const int ta = 2 * lane, tb = ta + 1;   // tokens of this lane
+        float kv[2][8], lw[2][8];
+        {
+            float om[2][8];
+            unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(ta, cg)), kv[0]);
+            unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(tb, cg)), kv[1]);
+            unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(ta, cg)), om[0]);
+            unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(tb, cg)), om[1]);
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)   // log2 w = -exp(omega) log2(e); 0 past T
+                    lw[q2][c] = (ta + q2 < valid) ? -ex2(om[q2][c] * kLog2e) * kLog2e : 0.f;
+        }
+        // inclusive prefix over the chunk: this lane's pair, then a scan over the lanes
+        float inc[8], L63[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) inc[c] = lw[0][c] + lw[1][c];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float o = __shfl_up_sync(0xffffffffu, inc[c], d);
+                if (lane >= d) inc[c] += o;
+            }
+        }
+        bool ok = true;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            L63[c] = __shfl_sync(0xffffffffu, inc[c], 31);
+            ok = ok && L63[c] >= -kMaxLog2Range;
+        }
+        if (!ok) return false;
+        // L of the two tokens (inclusive) and of the token before each (exclusive)
+        float Lt[2][8], Lx[2][8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            Lt[1][c] = inc[c];
+            Lt[0][c] = inc[c] - lw[1][c];
+            Lx[1][c] = Lt[0][c];
+            Lx[0][c] = Lt[0][c] - lw[0][c];
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            float kh[8], f[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                kh[c] = kv[q2][c] * ex2(-Lt[q2][c]);
+                f[c] = ex2(Lx[q2][c]);
+            }
+            uint4 hi, lo;
+            split8(kh, hi, lo);
+            *reinterpret_cast<uint4*>(s.kh_hi[pb] + sw_chunk(ta + q2, cg)) = hi;
+            *reinterpret_cast<uint4*>(s.kh_lo[pb] + sw_chunk(ta + q2, cg)) = lo;
+            float4* fd = reinterpret_cast<float4*>(&s.F[pb][ta + q2][8 * cg]);
+            fd[0] = make_float4(f[0], f[1], f[2], f[3]);
+            fd[1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {   // Kt^T: channel row i, this lane's two tokens
+            const int i = 8 * cg + c;
+            const float x0 = kv[0][c] * ex2(L63[c] - Lt[0][c]);
+            const float x1 = kv[1][c] * ex2(L63[c] - Lt[1][c]);
+            const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+            *reinterpret_cast<uint32_t*>(s.kt_hi[pb] + tr_off(i, lane)) = pack2(h0, h1);
+            *reinterpret_cast<uint32_t*>(s.kt_lo[pb] + tr_off(i, lane)) = pack2(x0 - h0, x1 - h1);
+        }
+        if (lane == 0)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) s.gamma[pb][8 * cg + c] = ex2(L63[c]);
+        return true;
+    };
+    // MMA 1 of chunk m (one thread): A = dy v^T, Z[m & 1] = dy S^T (S = the state entering m,
+    // in s_hi / s_lo), U = Kt^T V
+    auto issue_mma1 = [&](int m) {
+        const int st = m % kStages, pb = m & 1;
+        ptx::tc_fence_after();
+        const uint32_t a_dy = ptx::smem_addr(s.in[st][0]), b_v = ptx::smem_addr(s.in[st][2]);
+        const uint32_t b_hi = ptx::smem_addr(s.s_hi), b_lo = ptx::smem_addr(s.s_lo);
+        const uint32_t a_kh = ptx::smem_addr(s.kt_hi[pb]), a_kl = ptx::smem_addr(s.kt_lo[pb]);
+        const uint32_t zc = tmem + COL_Z + 64 * pb;
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq)   // A = dy v^T
+            ptx::mma_bf16(tmem + COL_A, ptx::desc_kmajor(a_dy + 32 * kq),
+                          ptx::desc_kmajor(b_v + 32 * kq), IDESC_KK, kq > 0);
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq)   // Z = dy S_hi^T
+            ptx::mma_bf16(zc, ptx::desc_kmajor(a_dy + 32 * kq), ptx::desc_kmajor(b_hi + 32 * kq),
+                          IDESC_KK, kq > 0);
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq)   // Z += dy S_lo^T
+            ptx::mma_bf16(zc, ptx::desc_kmajor(a_dy + 32 * kq), ptx::desc_kmajor(b_lo + 32 * kq),
+                          IDESC_KK, 1);
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq)   // U = Kt_hi^T V
+            ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kh + 32 * kq),
+                          ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, kq > 0);
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq)   // U += Kt_lo^T V
+            ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kl + 32 * kq),
+                          ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, 1);
+        ptx::mma_commit(&s.mma1);
+        issued1 = m;
+    };
+
+    // Software pipeline over chunks, all threads in lockstep: MMA 2 of chunk n runs while the
+    // state advances and chunk n+1 is prepared; MMA 1 of chunk n+1 runs while chunk n's
+    // output is formed.
+    int n = 0;
+    {
+        if (!ptx::mbar_wait(&s.full[0], 0, budget)) s.abort = 1;
+        const bool ok = NC > 0 && prep_chunk(0);
+        ptx::fence_proxy_async_smem();
+        if (__syncthreads_or(!ok || s.abort)) {
+            if (s.abort) failed = true;
+            else out_of_range = true;
+        } else if (tid == 0) {
+            issue_mma1(0);
+        }
+    }
+    if (!failed && !out_of_range) for (; n < NC; ++n) {
+        const int st = n % kStages, pb = n & 1;
         const int t0 = n * C;
         const int valid = min(C, T - t0);
-        uint8_t* dy_tile = s.in[st][0];
         uint8_t* k_tile = s.in[st][1];
-        uint8_t* v_tile = s.in[st][2];
-        uint8_t* w_tile = s.in[st][3];
-        uint8_t* y_tile = s.ystage[n & 1];
-        if (tid == 0) ptx::bulk_wait_read<1>();   // the store that last used y_tile has read it
+        uint8_t* y_tile = s.ystage[pb];
         // the aux row (r, or k in reversed time) of this lane, read now for the output step
         const int t = row;
         const bool live = row_lane && t < valid;
@@ -218,153 +349,17 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
             rw[cc] = live ? __ldg(reinterpret_cast<const uint4*>(r + gx + 8 * cc)) : make_uint4(0, 0, 0, 0);
-        if (!ptx::mbar_wait(&s.full[st], (uint32_t)((n / kStages) & 1), budget)) s.abort = 1;
+        // the store that last used y_tile (chunk n-2) has read it before this chunk rewrites it
+        if (!kDk && tid == 0) ptx::bulk_wait_read<1>();
 
-        // -------------------------------------------------------- prep
-        bool in_range;
-        {
-            const int cg = warp;                    // channels 8cg .. 8cg+7
-            const int ta = 2 * lane, tb = ta + 1;   // tokens of this lane
-            float kv[2][8], lw[2][8];
-            {
-                float om[2][8];
-                unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(ta, cg)), kv[0]);
-                unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(tb, cg)), kv[1]);
-                unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(ta, cg)), om[0]);
-                unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(tb, cg)), om[1]);
-#pragma unroll
-                for (int p = 0; p < 2; ++p)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)   // log2 w = -exp(omega) log2(e); 0 past T
-                        lw[p][c] = (ta + p < valid) ? -ex2(om[p][c] * kLog2e) * kLog2e : 0.f;
-            }
-            // inclusive prefix over the chunk: this lane's pair, then a scan over the lanes
-            float inc[8], L63[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) inc[c] = lw[0][c] + lw[1][c];
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float o = __shfl_up_sync(0xffffffffu, inc[c], d);
-                    if (lane >= d) inc[c] += o;
-                }
-            }
-            in_range = true;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                L63[c] = __shfl_sync(0xffffffffu, inc[c], 31);
-                in_range = in_range && L63[c] >= -kMaxLog2Range;
-            }
-            // L of the two tokens (inclusive) and of the token before each (exclusive)
-            float Lt[2][8], Lx[2][8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                Lt[1][c] = inc[c];
-                Lt[0][c] = inc[c] - lw[1][c];
-                Lx[1][c] = Lt[0][c];
-                Lx[0][c] = Lt[0][c] - lw[0][c];
-            }
-            if (in_range) {
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    float kh[8], f[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        kh[c] = kv[p][c] * ex2(-Lt[p][c]);
-                        f[c] = ex2(Lx[p][c]);
-                    }
-                    uint4 hi, lo;
-                    split8(kh, hi, lo);
-                    *reinterpret_cast<uint4*>(s.kh_hi + sw_chunk(ta + p, cg)) = hi;
-                    *reinterpret_cast<uint4*>(s.kh_lo + sw_chunk(ta + p, cg)) = lo;
-                    float4* fd = reinterpret_cast<float4*>(&s.F[ta + p][8 * cg]);
-                    fd[0] = make_float4(f[0], f[1], f[2], f[3]);
-                    fd[1] = make_float4(f[4], f[5], f[6], f[7]);
-                }
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {   // Kt^T: channel row i, this lane's two tokens
-                    const int i = 8 * cg + c;
-                    const float x0 = kv[0][c] * ex2(L63[c] - Lt[0][c]);
-                    const float x1 = kv[1][c] * ex2(L63[c] - Lt[1][c]);
-                    const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
-                    const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
-                    *reinterpret_cast<uint32_t*>(s.kt_hi + tr_off(i, lane)) = pack2(h0, h1);
-                    *reinterpret_cast<uint32_t*>(s.kt_lo + tr_off(i, lane)) = pack2(x0 - h0, x1 - h1);
-                }
-                if (lane == 0)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) s.gamma[8 * cg + c] = ex2(L63[c]);
-            }
-        }
-        ptx::fence_proxy_async_smem();
-        const bool stop = __syncthreads_or(!in_range || s.abort);
-        if (stop) {
-            if (s.abort) failed = true;
-            else out_of_range = true;
-            break;
-        }
-
-        // -------------------------------------------------------- MMA 1
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            const uint32_t a_dy = ptx::smem_addr(dy_tile), b_v = ptx::smem_addr(v_tile);
-            const uint32_t b_hi = ptx::smem_addr(s.s_hi), b_lo = ptx::smem_addr(s.s_lo);
-            const uint32_t a_kh = ptx::smem_addr(s.kt_hi), a_kl = ptx::smem_addr(s.kt_lo);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)   // A = dy v^T
-                ptx::mma_bf16(tmem + COL_A, ptx::desc_kmajor(a_dy + 32 * kq),
-                              ptx::desc_kmajor(b_v + 32 * kq), IDESC_KK, kq > 0);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)   // Z = dy S_hi^T
-                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(a_dy + 32 * kq),
-                              ptx::desc_kmajor(b_hi + 32 * kq), IDESC_KK, kq > 0);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)   // Z += dy S_lo^T
-                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(a_dy + 32 * kq),
-                              ptx::desc_kmajor(b_lo + 32 * kq), IDESC_KK, 1);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)   // U = Kt_hi^T V
-                ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kh + 32 * kq),
-                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, kq > 0);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)   // U += Kt_lo^T V
-                ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kl + 32 * kq),
-                              ptx::desc_mnmajor(b_v + 2048 * kq), IDESC_KM, 1);
-            ptx::mma_commit(&s.mma1);
-            issued1 = n;
-        }
         if (!ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), budget)) s.abort = 1;
         ptx::tc_fence_after();
-
-        // -------------------------------------------------------- state chain
-        {
-            uint32_t U[32];
-            ptx::tmem_ld32(tmem + tlane + COL_U + 32 * hh, U);
-            ptx::tmem_wait_ld();
-            if (row_lane) {
-                const float g = s.gamma[row];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
-                    uint4 hi, lo;
-                    split8(f, hi, lo);
-                    *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, 4 * hh + cc)) = hi;
-                    *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, 4 * hh + cc)) = lo;
-                }
-            }
-        }
-        // -------------------------------------------------------- causal scores
+        // -------------------------------------------------------- causal scores of chunk n
         {
             uint32_t A[32];
             ptx::tmem_ld32(tmem + tlane + COL_A + 32 * hh, A);
             ptx::tmem_wait_ld();
             if (row_lane) {
-                const int t = row;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     float a[8];
@@ -384,36 +379,69 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         }
         ptx::tc_fence_before();
         ptx::fence_proxy_async_smem();
-        __syncthreads();
-        if (s.abort) { failed = true; break; }
-
-        // -------------------------------------------------------- MMA 2: Z += A Kh
+        // (a vote, not a read after the barrier: a thread already past it may set abort)
+        if (__syncthreads_or(s.abort)) { failed = true; break; }
+        // -------------------------------------------------------- MMA 2: Z[n & 1] += A Kh
         if (tid == 0) {
             ptx::tc_fence_after();
             const uint32_t ah = ptx::smem_addr(s.a_hi), al = ptx::smem_addr(s.a_lo);
-            const uint32_t bh_ = ptx::smem_addr(s.kh_hi), bl = ptx::smem_addr(s.kh_lo);
+            const uint32_t bh_ = ptx::smem_addr(s.kh_hi[pb]), bl = ptx::smem_addr(s.kh_lo[pb]);
+            const uint32_t zc = tmem + COL_Z + 64 * pb;
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(ah + 32 * kq),
-                              ptx::desc_mnmajor(bh_ + 2048 * kq), IDESC_KM, 1);
+                ptx::mma_bf16(zc, ptx::desc_kmajor(ah + 32 * kq), ptx::desc_mnmajor(bh_ + 2048 * kq),
+                              IDESC_KM, 1);
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(ah + 32 * kq),
-                              ptx::desc_mnmajor(bl + 2048 * kq), IDESC_KM, 1);
+                ptx::mma_bf16(zc, ptx::desc_kmajor(ah + 32 * kq), ptx::desc_mnmajor(bl + 2048 * kq),
+                              IDESC_KM, 1);
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(tmem + COL_Z, ptx::desc_kmajor(al + 32 * kq),
-                              ptx::desc_mnmajor(bh_ + 2048 * kq), IDESC_KM, 1);
+                ptx::mma_bf16(zc, ptx::desc_kmajor(al + 32 * kq), ptx::desc_mnmajor(bh_ + 2048 * kq),
+                              IDESC_KM, 1);
             ptx::mma_commit(&s.mma2);
             issued2 = n;
         }
+        // -------------------------------------------------------- state chain (MMA 2 running)
+        {
+            uint32_t U[32];
+            ptx::tmem_ld32(tmem + tlane + COL_U + 32 * hh, U);
+            ptx::tmem_wait_ld();
+            if (row_lane) {
+                const float g = s.gamma[pb][row];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                    uint4 hi, lo;
+                    split8(f, hi, lo);
+                    *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, 4 * hh + cc)) = hi;
+                    *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, 4 * hh + cc)) = lo;
+                }
+            }
+        }
+        // -------------------------------------------------------- prep of chunk n+1
+        bool next_ok = true;
+        if (n + 1 < NC) {
+            if (!ptx::mbar_wait(&s.full[(n + 1) % kStages], (uint32_t)(((n + 1) / kStages) & 1), budget))
+                s.abort = 1;
+            next_ok = prep_chunk(n + 1);
+        }
+        ptx::tc_fence_before();
+        ptx::fence_proxy_async_smem();
+        const bool stop = __syncthreads_or(!next_ok || s.abort);
+        // MMA 1 of chunk n+1 (its inputs, the S tiles above and its operands, are in place;
+        // A and U of chunk n have been read)
+        if (!stop && tid == 0 && n + 1 < NC) issue_mma1(n + 1);
         if (!ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), budget)) s.abort = 1;
         ptx::tc_fence_after();
-
-        // -------------------------------------------------------- output
+        // -------------------------------------------------------- output of chunk n
         {
             uint32_t Z[32];
-            ptx::tmem_ld32(tmem + tlane + COL_Z + 32 * hh, Z);
+            ptx::tmem_ld32(tmem + tlane + COL_Z + 64 * pb + 32 * hh, Z);
             ptx::tmem_wait_ld();
             if (row_lane) {
                 const float dg = s.diag[t];
@@ -426,7 +454,7 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = 8 * cc + e, i = 32 * hh + j;
-                        const float pair = s.F[t][i] * __uint_as_float(Z[j]);   // dr minus the bonus
+                        const float pair = s.F[pb][t][i] * __uint_as_float(Z[j]);   // minus the bonus
                         const float kd = kx[e] * dg;
                         o[e] = fmaf(s.u[i], kd, pair);
                         pv[e] = rv[e] * pair;
@@ -445,18 +473,24 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         }
         ptx::tc_fence_before();
         ptx::fence_proxy_async_smem();
-        __syncthreads();
-        if (s.abort) { failed = true; break; }
+        const bool brk = __syncthreads_or(stop || s.abort);
         if (tid == 0) {
             if (!kDk && gw_check(status, t0 < T && h < H)) {
                 ptx::tma_store_4d(&tm_dr, y_tile, 0, h, t0, b);
                 ptx::bulk_commit();
             }
-            // every thread is past its reads of this stage and the MMAs that read it are done
-            if (n + kStages < NC) {
+            // every thread is past its reads of stage st and the MMAs that read it are done
+            if (!brk && n + kStages < NC) {
                 ptx::fence_proxy_async_smem();
                 issue_load(n + kStages);
+                last_load[st] = n + kStages;
             }
+        }
+        if (brk) {   // every abort write precedes the vote, so all threads read the same
+            if (s.abort) failed = true;
+            else out_of_range = true;
+            ++n;   // chunk n is complete; the drain below starts after it
+            break;
         }
     }
 
@@ -464,9 +498,11 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
     if (failed || out_of_range) {
         if (tid == 0) {
             if (failed) atomicExch(status, 1);
-            // copies still in flight: chunks n .. min(NC, n + kStages) - 1 may have been issued
-            for (int c = n; c < NC && c < n + kStages; ++c)
-                ptx::mbar_wait(&s.full[c % kStages], (uint32_t)((c / kStages) & 1), drain_budget);
+            // every issued copy must land (waiting again on a landed one returns at once),
+            // and the products of the chunk this CTA stopped at must be complete
+            for (int st = 0; st < kStages; ++st)
+                if (last_load[st] >= 0)
+                    ptx::mbar_wait(&s.full[st], (uint32_t)((last_load[st] / kStages) & 1), drain_budget);
             if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)(n & 1), drain_budget);
             if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)(n & 1), drain_budget);
             fallback[bh] = 1;   // the CUDA-core scan redoes this (b,h)
