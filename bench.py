@@ -353,9 +353,11 @@ def backward_line(cfg, dev, world, steps, c2=False):
     e1.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
     flops, nbytes = backward_flops(B, T, H, D), backward_bytes(B, T, H, D)
-    # dr scan, dk scan, du sum; 2 reversals + fast + level kernels for dv (+ 2 segment
-    # kernels when the sequence is split).  Finch-C2: the dr + dv scan launch and the dk scan
-    launches_per_call = 2 if c2 else 3 + 4
+    # base form: 2 reversals + fast + level kernels for dv (+ 2 segment kernels when the
+    # sequence is split), the tensor-core dr and dk readouts, the two decay-gradient kernels,
+    # the dr and dk scans (which exit at once unless a (b,h) fell back) and the du sum.
+    # Finch-C2: the dr + dv scan launch and the dk scan
+    launches_per_call = 2 if c2 else 11
     line = {"workload": ("wkv6c2_backward" if c2 else "wkv6_backward") + f" B{B} T{T} H{H}",
             "B": B, "T": T, "H": H, "D": D, "io": "bf16", "steps": steps, "ms_per_call": ms,
             "value": world * B * T / (ms / 1e3), "unit": "tokens/s",
@@ -368,12 +370,16 @@ def backward_line(cfg, dev, world, steps, c2=False):
             "gpu_launches": launches_per_call * steps,
             "kernels": ("dr and dv scans (wkv6_bwd_dr_dv_kernel), dk + decay-gradient scan "
                         "(wkv6_bwd_dk_domega_kernel), all on CUDA cores") if c2 else
-                       ("dr scan (wkv6_bwd_dr_dv_kernel), dk + decay-gradient scan "
-                        "(wkv6_bwd_dk_domega_kernel), du sum; dv through the chunked tensor-core "
-                        "prefill on time-reversed copies (reverse_tokens_kernel x2, "
-                        "wkv6_fast_kernel, wkv6_chunked_kernel)"),
+                       ("dr and dk as chunked tensor-core readouts of the forward and the "
+                        "reversed state (wkv6_bwd_readout_tc_kernel x2), the decay gradient from "
+                        "their pair terms (wkv6_bwd_pq_sums_kernel, wkv6_bwd_domega_kernel), dv "
+                        "through the chunked tensor-core prefill on time-reversed copies "
+                        "(reverse_tokens_kernel x2, wkv6_fast_kernel, wkv6_chunked_kernel); the "
+                        "CUDA-core scans run only for a (b,h) whose decays the one-sided factors "
+                        "cannot take"),
             "note": "algorithmic FLOPs are the three recurrences (dr, dk, dv) at 5 FLOPs per "
-                    "state entry per token" + ("" if c2 else "; dv runs on the tensor cores")}
+                    "state entry per token" + ("" if c2 else "; dr, dk and dv run on the tensor "
+                                                               "cores")}
     del inp, dy, dS, ws, args_b
     torch.cuda.empty_cache()
     return line

@@ -266,11 +266,14 @@ wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, cons
  *     dv_t = G^T k_t + (r_t . (u * k_t)) dy_t           du   = sum_{b,t} r_t * k_t (v_t . dy_t)
  *     domega_t[i] = (sum_j G[i][j] S_{t-1}[i][j]) * w_t[i] * (-exp(omega_t[i]))
  *     G <- diag(w_t) G + r_t^T dy_t,   dstate_in = G before the first token.
- * dr and dk (with the decay gradient, through the equivalent sum of the pair terms that
- * straddle each token) are token-by-token scans on CUDA cores in fp32.  dv is the forward
- * recurrence run in reversed time with r and k swapped and dy as the value; with bf16 I/O
- * it runs through the chunked tensor-core prefill on time-reversed copies, with fp32 I/O
- * as a third scan.
+ * With bf16 I/O all three run on the tensor cores, chunk by chunk: dr as the readout of the
+ * forward state S_{t-1} with dy as the query, dk as the same readout of G in reversed time
+ * (query v, key r, value dy), dv as the forward recurrence in reversed time with r and k
+ * swapped and dy as the value (the chunked prefill on time-reversed copies); the decay
+ * gradient is the equivalent sum of the pair terms that straddle each token.  A (b,h) with
+ * a chunk whose decays the dr or dk pass cannot factor (a channel's decay over 64 tokens
+ * below e^-60) is redone by token-by-token scans on CUDA cores in fp32, which also serve
+ * fp32 I/O (with dv as a third scan).
  *   r, k, v, omega, u, state_in   the forward call's inputs (state_in NULL = zeros)
  *   dy          [B][T][H][D] io   gradient of y
  *   dstate_out  [B][H][D][D] fp32 gradient of the final state, or NULL (zero)
@@ -279,10 +282,9 @@ wkv_status wkv6_decode_step_gn(const void *r, const void *k, const void *v, cons
  *   dstate_in   [B][H][D][D] fp32 output, or NULL (not computed)
  *   workspace   at least wkv6_backward_workspace_bytes(...) bytes; no initial contents needed.
  * No output may overlap an input, another output or the workspace.  T = 0: du = 0 and
- * dstate_in = dstate_out (or zero).  The bf16 dv pass uses the chunked prefill's bounded
- * waits; if one expired (a device that stopped making progress for about a second), dv is
- * invalid and the call does not report it (the chunked region's status word is internal to
- * the workspace).
+ * dstate_in = dstate_out (or zero).  The bf16 tensor-core passes use bounded waits; if one
+ * expired (a device that stopped making progress for about a second), the gradients are
+ * invalid and the call does not report it (the status word is internal to the workspace).
  */
 size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io);
 
