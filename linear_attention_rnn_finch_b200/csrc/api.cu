@@ -650,18 +650,20 @@ namespace {
 // Workspace of the backward: P and E in the row scans' accumulation type (fp64 for fp32
 // I/O, fp32 for bf16 I/O) and the per-(b,h) du parts; with tc_dv, also the time-reversed
 // k, r, dy, omega and dv and the chunked prefill's own workspace.
-size_t backward_bytes(int B, int T, int H, int D, wkv_dtype io, bool tc_dv) {
+size_t backward_bytes(int B, int T, int H, int D, wkv_dtype io, bool c2) {
+    const bool tc = io == WKV_BF16;   // the tensor-core path
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
     const size_t acc = io == WKV_F32 ? sizeof(double) : sizeof(float);
     const size_t x = (size_t)B * T * H * D, bh = (size_t)B * H * D;
     size_t bytes = round256(x * acc) + round256(bh * acc) + round256(bh * sizeof(float));
     // tensor-core path: 5 time-reversed copies and a reversed output, the chunked prefill's
-    // workspace, a fallback flag per (b,h) for dr and for dk, Q (fp32, reversed) and the
-    // decay gradient's per-chunk sums of P and Q
-    if (tc_dv)
+    // workspace, a fallback flag per (b,h) for dr and for dk, Q (fp32) and the decay
+    // gradient's per-chunk sums of P and Q; Finch-C2 also D (fp32)
+    if (tc)
         bytes += 6 * round256(x * 2) + chunked_bytes(B, H, choose_segments(B, T, H)) +
                  2 * round256((size_t)B * H * sizeof(int)) + round256(x * sizeof(float)) +
-                 round256((size_t)B * H * ((T + kChunk - 1) / kChunk) * 128 * sizeof(float));
+                 round256((size_t)B * H * ((T + kChunk - 1) / kChunk) * 128 * sizeof(float)) +
+                 (c2 ? round256(x * sizeof(float)) : 0);
     return bytes;
 }
 
@@ -706,8 +708,9 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
             if (overlaps(outs[a], outs[b2])) return WKV_ERR_INVALID_ARG;
     }
     const bool bf16 = io == WKV_BF16;
+    const bool tc = bf16;             // dr and dk on the tensor cores
     const bool tc_dv = bf16 && !c2;   // dv through the chunked tensor-core prefill
-    const size_t need = backward_bytes(B, T, H, D, io, tc_dv);
+    const size_t need = backward_bytes(B, T, H, D, io, c2);
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
         const Span sw = span(workspace, need);
@@ -734,16 +737,17 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     uint8_t* E = ws + round256((size_t)B * T * H * D * acc);
     uint8_t* dpart = E + round256((size_t)B * H * D * acc);
     float* du_part = reinterpret_cast<float*>(dpart);
-    if (!tc_dv)
+    if (!tc)
         return from_cuda(goldwkv::launch_backward(r, k, v, omega, c2 ? nullptr : u, state_in, dy,
                                                   dstate_out, dr, dk, dv, domega, du, dstate_in,
                                                   P, E, du_part, B, T, H, bf16, /*with_dv=*/true,
                                                   c2, st));
-    // Tensor-core path (bf16, base form).  Workspace after P, E and du_part: time-reversed
-    // copies of k, r, dy, omega and v, the reversed dv, the chunked
-    // prefill's workspace (its first word is the status word every tensor-core pass here
-    // reports an expired wait in), a fallback flag per (b,h) for each of dr and dk, Q and the
-    // decay gradient's chunk sums.
+    const float* ub = c2 ? nullptr : u;
+    // Tensor-core path (bf16).  Workspace after P, E and du_part: time-reversed copies of k,
+    // r, dy, omega and v, the reversed dv, the chunked prefill's workspace (its first word is
+    // the status word every tensor-core pass here reports an expired wait in), a fallback
+    // flag per (b,h) for each of dr and dk, Q, the decay gradient's chunk sums and, for
+    // Finch-C2, D.
     const int P_seg = choose_segments(B, T, H);
     const size_t xr = round256(xbytes);
     const size_t flags = round256((size_t)B * H * sizeof(int));
@@ -761,20 +765,29 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     float* q_tok = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dk_flags) + flags);
     float* sums = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(q_tok) +
                                            round256((size_t)B * T * H * D * sizeof(float)));
+    float* d_tok = c2 ? reinterpret_cast<float*>(
+                            reinterpret_cast<uint8_t*>(sums) +
+                            round256((size_t)B * H * ((T + kChunk - 1) / kChunk) * 128 * sizeof(float)))
+                      : nullptr;
     const long long budget = injected("timeout0") ? 0 : kSpinBudget;
-    const void* src[5] = {k, r, dy, omega, v};
-    void* dst[5] = {rk, rr, rdy, rom, rv};
-    if (goldwkv::launch_reverse_tokens(src, dst, 5, B, T, H, st) != cudaSuccess)
-        return WKV_ERR_CUDA;
-    // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r swapped
-    // and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.  It runs
-    // through the chunked tensor-core prefill on the reversed copies.
-    cudaError_t e = cudaSuccess;
-    if (!launch_chunked_path(rk, rr, rdy, rom, u, goldwkv::Variant{nullptr}, dstate_out, nullptr,
-                             rout, nullptr, B, T, H, P_seg, false, cws, st, &e) ||
-        e != cudaSuccess)
-        return WKV_ERR_CUDA;
+    // status word for the tensor-core passes (the chunked prefill's, when it runs)
+    if (!tc_dv && cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return WKV_ERR_CUDA;
     {
+        const void* src[5] = {r, dy, omega, v, k};
+        void* dst[5] = {rr, rdy, rom, rv, rk};
+        if (goldwkv::launch_reverse_tokens(src, dst, tc_dv ? 5 : 4, B, T, H, st) != cudaSuccess)
+            return WKV_ERR_CUDA;
+    }
+    if (tc_dv) {
+        // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
+        // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.
+        // It runs through the chunked tensor-core prefill on the reversed copies.  (Finch-C2's
+        // dv, whose query is k (1 - w), stays a CUDA-core scan, launched with the dr scan.)
+        cudaError_t e = cudaSuccess;
+        if (!launch_chunked_path(rk, rr, rdy, rom, u, goldwkv::Variant{nullptr}, dstate_out,
+                                 nullptr, rout, nullptr, B, T, H, P_seg, false, cws, st, &e) ||
+            e != cudaSuccess)
+            return WKV_ERR_CUDA;
         const void* s1[1] = {rout};
         void* d1[1] = {dv};
         if (goldwkv::launch_reverse_tokens(s1, d1, 1, B, T, H, st) != cudaSuccess)
@@ -790,13 +803,13 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         !goldwkv::make_token_map(&maps[3], omega, B, T, H) ||
         !goldwkv::make_token_map(&maps[4], dr, B, T, H))
         return WKV_ERR_CUDA;
-    if (goldwkv::launch_bwd_dr_tc(maps, r, u, state_in, dstate_out, static_cast<float*>(P),
+    if (goldwkv::launch_bwd_dr_tc(maps, r, ub, state_in, dstate_out, static_cast<float*>(P),
                                   reinterpret_cast<float*>(E), du_part, dr_flags, B, T, H, status,
-                                  budget, st) != cudaSuccess)
+                                  budget, st, c2) != cudaSuccess)
         return WKV_ERR_CUDA;
-    if (goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk, dv, domega,
-                                 du, dstate_in, P, E, du_part, B, T, H, bf16, false, false, st,
-                                 dr_flags, nullptr, goldwkv::kPhaseDr) != cudaSuccess)
+    if (goldwkv::launch_backward(r, k, v, omega, ub, state_in, dy, dstate_out, dr, dk, dv, domega,
+                                 du, dstate_in, P, E, du_part, B, T, H, bf16, /*with_dv=*/!tc_dv,
+                                 c2, st, dr_flags, nullptr, goldwkv::kPhaseDr) != cudaSuccess)
         return WKV_ERR_CUDA;
     // dk (and dS0, Q) as the same readout in reversed time: query v, key r, value dy; dk and
     // Q go straight to token order
@@ -806,17 +819,17 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         !goldwkv::make_token_map(&maps[3], rom, B, T, H) ||
         !goldwkv::make_token_map(&maps[4], rout, B, T, H))
         return WKV_ERR_CUDA;
-    if (goldwkv::launch_bwd_dk_tc(maps, k, u, dstate_out, dk, q_tok, dstate_in, dk_flags, B, T, H,
-                                  status, budget, st) != cudaSuccess)
+    if (goldwkv::launch_bwd_dk_tc(maps, k, ub, dstate_out, dk, q_tok, d_tok, dstate_in, dk_flags, B,
+                                  T, H, status, budget, st, c2) != cudaSuccess)
         return WKV_ERR_CUDA;
-    if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_tok, sums,
+    if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_tok, d_tok, sums,
                                    reinterpret_cast<const float*>(E), omega, domega, B, T, H,
                                    st) != cudaSuccess)
         return WKV_ERR_CUDA;
     // the dk scan (with its decay gradient and dS0) for the flagged (b,h), then du
-    return from_cuda(goldwkv::launch_backward(r, k, v, omega, u, state_in, dy, dstate_out, dr, dk,
+    return from_cuda(goldwkv::launch_backward(r, k, v, omega, ub, state_in, dy, dstate_out, dr, dk,
                                               dv, domega, du, dstate_in, P, E, du_part, B, T, H,
-                                              bf16, false, false, st, nullptr, dk_flags,
+                                              bf16, false, c2, st, nullptr, dk_flags,
                                               goldwkv::kPhaseDk | goldwkv::kPhaseDu));
 }
 
@@ -825,11 +838,11 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
 extern "C" {
 
 size_t wkv6_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
-    return backward_bytes(B, T, H, D, io, io == WKV_BF16);
+    return backward_bytes(B, T, H, D, io, false);
 }
 
 size_t wkv6c2_backward_workspace_bytes(int B, int T, int H, int D, wkv_dtype io) {
-    return backward_bytes(B, T, H, D, io, false);
+    return backward_bytes(B, T, H, D, io, true);
 }
 
 wkv_status wkv6_backward(const void* r, const void* k, const void* v, const void* omega,

@@ -32,23 +32,28 @@ cudaError_t launch_backward(const void* r, const void* k, const void* v, const v
 // omega, dr ([B][T][H][64] bf16 token maps); r is read directly.  fallback[bh] = 1 for a
 // (b,h) with a chunk whose decay range the one-sided factorisation cannot take (its outputs
 // are then left to the scan), 0 otherwise.  status: set to 1 if a bounded wait expired.
+// c2: Finch-C2's form (key k (1 - w), no bonus; u unused).
 cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float* u,
                              const float* state_in, const float* dS_T, float* P, float* E,
                              float* du_part, int* fallback, int B, int T, int H, int* status,
-                             long long budget, cudaStream_t st);
+                             long long budget, cudaStream_t st, bool c2 = false);
 
 // dk of the base form on the tensor cores, the same readout on time-reversed copies: maps
 // v, r, dy, omega (all reversed) and any valid token map (unused); k in token order.  Writes
 // dk and Q (the pair terms k_t (dk_t - bonus), fp32 [B][T][H][64]) in token order and dS_0
 // (if non-null).  fallback / status as for launch_bwd_dr_tc.
+// c2: Finch-C2's form: the readout is dkn, dk = dkn (1 - w), Q = k (1 - w) dkn, and D (fp32,
+// token order) = dkn k w, the direct dependence of kn on w (D unused otherwise).
 cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k, const float* u,
-                             const float* dS_T, void* dk, float* Q, float* dS_0, int* fallback,
-                             int B, int T, int H, int* status, long long budget, cudaStream_t st);
+                             const float* dS_T, void* dk, float* Q, float* D, float* dS_0,
+                             int* fallback, int B, int T, int H, int* status, long long budget,
+                             cudaStream_t st, bool c2 = false);
 
 // domega (bf16) from P, Q (token order) and E through the identity
-//     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,  domega_t = dlog w_t (-exp(omega_t));
-// sums: scratch of B*H*ceil(T/64)*128 floats.
-cudaError_t launch_bwd_domega(const float* P, const float* Q, float* sums, const float* E,
+//     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s - D_t,  domega_t = dlog w_t (-exp(omega_t));
+// D: Finch-C2's direct term, or null (zero).  sums: scratch of B*H*ceil(T/64)*128 floats.
+cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, float* sums,
+                              const float* E,
                               const void* omega, void* domega, int B, int T, int H,
                               cudaStream_t st);
 

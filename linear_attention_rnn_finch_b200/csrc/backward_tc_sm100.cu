@@ -34,7 +34,12 @@
 // the state gradient, dk_t[i] = sum_j G_t[i][j] v_t[j] + u[i] r_t[i] (v_t . dy_t), i.e. the
 // readout above on time-reversed copies with query v, key r, value dy, initial state dS_T;
 // its final state is dS_0, and its pair terms Q_t = k_t (dk_t - bonus) feed the decay
-// gradient (wkv6_bwd_domega kernels below).  Every mbarrier wait is bounded.
+// gradient (wkv6_bwd_domega kernels below).
+//
+// Finch-C2's exact form (kC2): the key enters the state as kn = k (1 - w) and there is no
+// bonus.  dr: the key is kn, formed in prep.  dk: the readout is dkn (the key of the reversed
+// recurrence is r, unchanged); dk = dkn (1 - w), Q_t = kn_t dkn_t, and kn's own dependence on
+// w adds D_t = dkn_t k_t w_t, subtracted from dlog w_t.  Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -121,14 +126,15 @@ __device__ __forceinline__ uint32_t tr_off(int i, int lane) {
 // kDk == true (dk, time-reversed inputs): query v, key r, value dy, aux k (in token order),
 // x0 = dS_T; writes dk to out_direct and Q (into P), both in token order, and the final state
 // (dS_0) to x_final.
-template <bool kDk>
+template <bool kDk, bool kC2>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_dr, const __nv_bfloat16* __restrict__ r,
                       const float* __restrict__ u, const float* state_in, const float* dS_T,
                       float* __restrict__ P, float* __restrict__ E, float* __restrict__ du_part,
-                      float* x_final, __nv_bfloat16* __restrict__ out_direct, int* fallback, int T,
+                      float* x_final, __nv_bfloat16* __restrict__ out_direct,
+                      float* __restrict__ Dw, int* fallback, int T,
                       int H, int* status, long long budget, long long drain_budget) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
@@ -148,7 +154,7 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         ptx::prefetch_tensormap(&tm_w);
         ptx::prefetch_tensormap(&tm_dr);
     }
-    if (tid < 64) s.u[tid] = u[h * 64 + tid];
+    if (tid < 64) s.u[tid] = kC2 ? 0.f : u[h * 64 + tid];
     if (warp == 0) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     ptx::tc_fence_before();
     __syncthreads();
@@ -224,6 +230,13 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
 #pragma unroll
                 for (int c = 0; c < 8; ++c)   // log2 w = -exp(omega) log2(e); 0 past T
                     lw[q2][c] = (ta + q2 < valid) ? -ex2(om[q2][c] * kLog2e) * kLog2e : 0.f;
+            if (kC2 && !kDk) {   // the state's key is kn = k (1 - w), 1 - w = -expm1(-exp(omega))
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        kv[q2][c] *= (ta + q2 < valid) ? -expm1f(-__expf(om[q2][c])) : 0.f;
+            }
         }
         // inclusive prefix over the chunk: this lane's pair, then a scan over the lanes
         float inc[8], L63[8];
@@ -448,17 +461,29 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
                 float* pdst = P + gx;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    float kx[8], o[8], pv[8], rv[8];
+                    float kx[8], o[8], pv[8], rv[8], dv8[8];
                     unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(t, 4 * hh + cc)), kx);
                     unpack8(rw[cc], rv);
+                    float om[8];
+                    if (kC2 && kDk)   // this token's omega (reversed-time tile, row t)
+                        unpack8(*reinterpret_cast<const uint4*>(s.in[st][3] + sw_chunk(t, 4 * hh + cc)), om);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = 8 * cc + e, i = 32 * hh + j;
                         const float pair = s.F[pb][t][i] * __uint_as_float(Z[j]);   // minus the bonus
-                        const float kd = kx[e] * dg;
-                        o[e] = fmaf(s.u[i], kd, pair);
-                        pv[e] = rv[e] * pair;
-                        du_acc[j] = fmaf(rv[e], kd, du_acc[j]);
+                        if (kC2 && kDk) {
+                            // pair = dkn; dk = dkn (1 - w); Q = kn dkn = k (1 - w) dkn; D = dkn k w
+                            const float ew = __expf(om[e]);
+                            const float omw = -expm1f(-ew), w = __expf(-ew);
+                            o[e] = pair * omw;
+                            pv[e] = rv[e] * omw * pair;
+                            dv8[e] = pair * rv[e] * w;
+                        } else {
+                            const float kd = kx[e] * dg;
+                            o[e] = fmaf(s.u[i], kd, pair);
+                            pv[e] = rv[e] * pair;
+                            du_acc[j] = fmaf(rv[e], kd, du_acc[j]);
+                        }
                     }
                     if (!kDk)
                         *reinterpret_cast<uint4*>(y_tile + sw_chunk(t, 4 * hh + cc)) = pack8(o);
@@ -467,6 +492,10 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
                     if (live) {
                         reinterpret_cast<float4*>(pdst + 8 * cc)[0] = make_float4(pv[0], pv[1], pv[2], pv[3]);
                         reinterpret_cast<float4*>(pdst + 8 * cc)[1] = make_float4(pv[4], pv[5], pv[6], pv[7]);
+                        if (kC2 && kDk) {
+                            reinterpret_cast<float4*>(Dw + gx + 8 * cc)[0] = make_float4(dv8[0], dv8[1], dv8[2], dv8[3]);
+                            reinterpret_cast<float4*>(Dw + gx + 8 * cc)[1] = make_float4(dv8[4], dv8[5], dv8[6], dv8[7]);
+                        }
                     }
                 }
             }
@@ -562,29 +591,30 @@ size_t bwd_readout_tc_smem_bytes() { return sizeof(Smem) + 1024; }
 cudaError_t launch_bwd_dr_tc(const CUtensorMap* maps, const void* r, const float* u,
                              const float* state_in, const float* dS_T, float* P, float* E,
                              float* du_part, int* fallback, int B, int T, int H, int* status,
-                             long long budget, cudaStream_t st) {
+                             long long budget, cudaStream_t st, bool c2) {
     const size_t smem = bwd_readout_tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_readout_tc_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kernel = c2 ? wkv6_bwd_readout_tc_kernel<false, true> : wkv6_bwd_readout_tc_kernel<false, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_bwd_readout_tc_kernel<false><<<(unsigned)(B * H), kThreads, smem, st>>>(
+    kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(r), u,
-        state_in, dS_T, P, E, du_part, nullptr, nullptr, fallback, T, H, status, budget,
+        state_in, dS_T, P, E, du_part, nullptr, nullptr, nullptr, fallback, T, H, status, budget,
         4000000000LL);
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k, const float* u,
-                             const float* dS_T, void* dk, float* Q, float* dS_0, int* fallback,
-                             int B, int T, int H, int* status, long long budget, cudaStream_t st) {
+                             const float* dS_T, void* dk, float* Q, float* D, float* dS_0,
+                             int* fallback, int B, int T, int H, int* status, long long budget,
+                             cudaStream_t st, bool c2) {
     const size_t smem = bwd_readout_tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_readout_tc_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kernel = c2 ? wkv6_bwd_readout_tc_kernel<true, true> : wkv6_bwd_readout_tc_kernel<true, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_bwd_readout_tc_kernel<true><<<(unsigned)(B * H), kThreads, smem, st>>>(
+    kernel<<<(unsigned)(B * H), kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], static_cast<const __nv_bfloat16*>(k), u,
-        dS_T, nullptr, Q, nullptr, nullptr, dS_0, static_cast<__nv_bfloat16*>(dk), fallback, T, H,
-        status, budget, 4000000000LL);
+        dS_T, nullptr, Q, nullptr, nullptr, dS_0, static_cast<__nv_bfloat16*>(dk), D, fallback, T,
+        H, status, budget, 4000000000LL);
     return cudaGetLastError();
 }
 
@@ -615,7 +645,8 @@ wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q
 
 __global__ void __launch_bounds__(64)
 wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
-                       const float* __restrict__ sums, const float* __restrict__ E,
+                       const float* __restrict__ Dw, const float* __restrict__ sums,
+                       const float* __restrict__ E,
                        const __nv_bfloat16* __restrict__ omega, __nv_bfloat16* __restrict__ domega,
                        int T, int H) {
     const int NC = (T + C - 1) / C;
@@ -633,7 +664,7 @@ wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
         const int t = t0 + tt;
         const size_t x = (((size_t)b * T + t) * H + h) * 64 + i;
         const float q = Q[x];
-        const float dl = acc - q;
+        const float dl = acc - q - (Dw != nullptr ? Dw[x] : 0.f);
         domega[x] = __float2bfloat16_rn(dl * -__expf(__bfloat162float(omega[x])));
         acc += P[x] - q;
     }
@@ -641,7 +672,8 @@ wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
 
 }  // namespace
 
-cudaError_t launch_bwd_domega(const float* P, const float* Q, float* sums, const float* E,
+cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, float* sums,
+                              const float* E,
                               const void* omega, void* domega, int B, int T, int H,
                               cudaStream_t st) {
     const unsigned blocks = (unsigned)((long)B * H * ((T + C - 1) / C));
@@ -649,7 +681,7 @@ cudaError_t launch_bwd_domega(const float* P, const float* Q, float* sums, const
     wkv6_bwd_pq_sums_kernel<<<blocks, 64, 0, st>>>(P, Q, sums, T, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_domega_kernel<<<blocks, 64, 0, st>>>(P, Q, sums, E,
+    wkv6_bwd_domega_kernel<<<blocks, 64, 0, st>>>(P, Q, D, sums, E,
                                                   static_cast<const __nv_bfloat16*>(omega),
                                                   static_cast<__nv_bfloat16*>(domega), T, H);
     return cudaGetLastError();

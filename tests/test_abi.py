@@ -97,8 +97,11 @@ def test_backward_and_gold_workspace_queries():
     assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16) == \
         base16 + 6 * r256(2 * x) + hand(B, H) + 2 * r256(4 * B * H) + r256(4 * x) + \
         r256(B * H * nc * 128 * 4)
-    assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 1) == base16
-    assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16, c2=True) == base16
+    # Finch-C2 (bf16): the same layout plus D (fp32), its direct decay term
+    c2_16 = base16 + 6 * r256(2 * x) + hand(B, H) + 2 * r256(4 * B * H) + 2 * r256(4 * x) + \
+        r256(B * H * nc * 128 * 4)
+    assert binding.load().wkv6c2_backward_workspace_bytes(B, T, H, 64, 1) == c2_16
+    assert binding.backward_workspace_bytes(B, T, H, 64, torch.bfloat16, c2=True) == c2_16
     assert binding.backward_workspace_bytes(B, 0, H, 64, torch.bfloat16) == 0
     assert binding.load().wkv6_backward_workspace_bytes(B, T, H, 32, 1) == 0
     # GOLD: a 256-byte status block; decompression wider than one cluster of column tiles

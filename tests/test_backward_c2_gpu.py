@@ -1,7 +1,9 @@
 """GPU parity of Finch-C2's backward pass (wkv6c2_backward) against the fp64 oracle's
 adjoint: every gradient (dr, dk, dv, domega, du', dS0) element by element, for fp32 and
 bf16 I/O, ragged tiles, strong decays, with and without the initial state and final-state
-gradient, and the 1.5B-layer shape on sampled heads."""
+gradient, and the 1.5B-layer shape on sampled heads.  With bf16 I/O dr and dk run on the
+tensor cores (a (b,h) whose decays the one-sided factors cannot take falls back to the
+scans: covered by a case that mixes both)."""
 import pytest
 import torch
 
@@ -63,6 +65,27 @@ def test_c2_backward_strong_decay_no_state(oracle):
     g = torch.Generator(device=DEV).manual_seed(10171)
     inp["omega"] = -9.0 + 13.0 * torch.rand(inp["omega"].shape, generator=g, device=DEV)
     _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.float32])
+
+
+@pytest.mark.parametrize("T", [1, 65, 130])
+def test_c2_backward_bf16_ragged(oracle, T):
+    inp = _problem(10160 + T, B=2, T=T, H=3, dtype=torch.bfloat16)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
+
+
+def test_c2_backward_bf16_no_state(oracle):
+    inp = _problem(10175, B=2, T=200, H=2, dtype=torch.bfloat16, s0=False, ds=False)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
+
+
+def test_c2_backward_bf16_some_heads_fall_back(oracle):
+    """bf16 dr and dk run on the tensor cores per (b,h); one batch row's head with decays
+    near zero is redone by the CUDA-core scans, the rest are not."""
+    inp = _problem(10176, B=3, T=300, H=3, dtype=torch.bfloat16)
+    om = inp["omega"].float()
+    om[1, 100:180, 2, ::2] = 3.0
+    inp["omega"] = om.to(torch.bfloat16)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
 
 
 def test_c2_backward_duprime_is_dy():
