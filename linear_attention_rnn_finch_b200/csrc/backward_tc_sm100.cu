@@ -18,9 +18,10 @@
 // Steps of a chunk (one CTA per (b,h), 256 threads, all warps in lockstep):
 //   prep  : warp = 8 channels, lane = 2 tokens; log2 w, the prefix L by a warp scan, F (fp32),
 //           Kh and Kt^T as bf16 hi / lo tiles, gamma;
-//   MMA 1 : A = dy x v^T; Z = dy x S_hi^T + dy x S_lo^T; U = Kt_hi^T V + Kt_lo^T V;
+//   MMA 1 : A = dy x v^T; Z = dy x [S_hi ; S_lo]^T (N = 128); U = Kt_hi^T V + Kt_lo^T V;
 //   A     : strictly causal part, hi / lo tiles; the diagonal (v_t . dy_t) kept aside;
-//   MMA 2 : Z += A_hi Kh_hi + A_hi Kh_lo + A_lo Kh_hi;
+//   MMA 2 : Z += A_hi [Kh_hi | Kh_lo] + A_lo [Kh_hi | Kh_lo] (N = 128); the output adds Z's
+//           two 64-column halves;
 //   state : S <- gamma S + U in registers, S_hi / S_lo tiles for the next chunk;
 //   out   : dr = F Z + u k diag (bf16 tile, TMA store); for the decay gradient the pair
 //           terms ending at t, P_t = r_t (dr_t - bonus) (fp32), and du's per-(b,h) sums.
@@ -56,17 +57,20 @@ constexpr int C = 64;
 constexpr int kThreads = 256;
 constexpr int kStages = 2;
 constexpr int kTile = 64 * 64 * 2;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t COL_A = 0, COL_U = 64, COL_Z = 128;   // Z: 2 x 64 (chunk parity)
+constexpr uint32_t kTmemCols = 512;
+// Z: 2 x 128 (chunk parity; the S_hi / Kh_hi part in the first 64 columns, the lo part next)
+constexpr uint32_t COL_A = 0, COL_U = 64, COL_Z = 128;
 constexpr uint32_t IDESC_KK = ptx::idesc_bf16(64, 64, 0, 0);
 constexpr uint32_t IDESC_KM = ptx::idesc_bf16(64, 64, 0, 1);
+constexpr uint32_t IDESC_KK2 = ptx::idesc_bf16(64, 128, 0, 0);   // B = two tiles side by side in N
+constexpr uint32_t IDESC_KM2 = ptx::idesc_bf16(64, 128, 0, 1);
 constexpr float kMaxLog2Range = 86.5617f;   // ln 60
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kFPitch = 68;                 // floats per row of F (padded against bank conflicts)
 
 struct __align__(1024) Smem {
     uint8_t in[kStages][4][kTile];   // dy, k, v, omega tiles per stage (TMA, 128B swizzle)
-    uint8_t kh_hi[2][kTile], kh_lo[2][kTile];   // Kh [s][i], per chunk parity
+    uint8_t kh[2][2][kTile];                // Kh [s][i] per chunk parity: hi tile, then lo tile
     uint8_t kt_hi[2][kTile], kt_lo[2][kTile];   // Kt^T [i][s], per chunk parity
     uint8_t a_hi[kTile], a_lo[kTile];       // causal scores [t][s]
     uint8_t s_hi[kTile], s_lo[kTile];       // S [i][j]
@@ -276,8 +280,8 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
             }
             uint4 hi, lo;
             split8(kh, hi, lo);
-            *reinterpret_cast<uint4*>(s.kh_hi[pb] + sw_chunk(ta + q2, cg)) = hi;
-            *reinterpret_cast<uint4*>(s.kh_lo[pb] + sw_chunk(ta + q2, cg)) = lo;
+            *reinterpret_cast<uint4*>(s.kh[pb][0] + sw_chunk(ta + q2, cg)) = hi;
+            *reinterpret_cast<uint4*>(s.kh[pb][1] + sw_chunk(ta + q2, cg)) = lo;
             float4* fd = reinterpret_cast<float4*>(&s.F[pb][ta + q2][8 * cg]);
             fd[0] = make_float4(f[0], f[1], f[2], f[3]);
             fd[1] = make_float4(f[4], f[5], f[6], f[7]);
@@ -303,21 +307,17 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         const int st = m % kStages, pb = m & 1;
         ptx::tc_fence_after();
         const uint32_t a_dy = ptx::smem_addr(s.in[st][0]), b_v = ptx::smem_addr(s.in[st][2]);
-        const uint32_t b_hi = ptx::smem_addr(s.s_hi), b_lo = ptx::smem_addr(s.s_lo);
+        const uint32_t b_s = ptx::smem_addr(s.s_hi);   // s_lo follows: [S_hi ; S_lo] in N
         const uint32_t a_kh = ptx::smem_addr(s.kt_hi[pb]), a_kl = ptx::smem_addr(s.kt_lo[pb]);
-        const uint32_t zc = tmem + COL_Z + 64 * pb;
+        const uint32_t zc = tmem + COL_Z + 128 * pb;
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq)   // A = dy v^T
             ptx::mma_bf16(tmem + COL_A, ptx::desc_kmajor(a_dy + 32 * kq),
                           ptx::desc_kmajor(b_v + 32 * kq), IDESC_KK, kq > 0);
 #pragma unroll
-        for (int kq = 0; kq < 4; ++kq)   // Z = dy S_hi^T
-            ptx::mma_bf16(zc, ptx::desc_kmajor(a_dy + 32 * kq), ptx::desc_kmajor(b_hi + 32 * kq),
-                          IDESC_KK, kq > 0);
-#pragma unroll
-        for (int kq = 0; kq < 4; ++kq)   // Z += dy S_lo^T
-            ptx::mma_bf16(zc, ptx::desc_kmajor(a_dy + 32 * kq), ptx::desc_kmajor(b_lo + 32 * kq),
-                          IDESC_KK, 1);
+        for (int kq = 0; kq < 4; ++kq)   // Z = dy [S_hi ; S_lo]^T (the two parts in N)
+            ptx::mma_bf16(zc, ptx::desc_kmajor(a_dy + 32 * kq), ptx::desc_kmajor(b_s + 32 * kq),
+                          IDESC_KK2, kq > 0);
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq)   // U = Kt_hi^T V
             ptx::mma_bf16(tmem + COL_U, ptx::desc_kmajor(a_kh + 32 * kq),
@@ -398,20 +398,16 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         if (tid == 0) {
             ptx::tc_fence_after();
             const uint32_t ah = ptx::smem_addr(s.a_hi), al = ptx::smem_addr(s.a_lo);
-            const uint32_t bh_ = ptx::smem_addr(s.kh_hi[pb]), bl = ptx::smem_addr(s.kh_lo[pb]);
-            const uint32_t zc = tmem + COL_Z + 64 * pb;
+            const uint32_t bk = ptx::smem_addr(s.kh[pb][0]);   // [Kh_hi | Kh_lo] in N
+            const uint32_t zc = tmem + COL_Z + 128 * pb;
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(zc, ptx::desc_kmajor(ah + 32 * kq), ptx::desc_mnmajor(bh_ + 2048 * kq),
-                              IDESC_KM, 1);
+            for (int kq = 0; kq < 4; ++kq)   // Z += A_hi [Kh_hi | Kh_lo]
+                ptx::mma_bf16(zc, ptx::desc_kmajor(ah + 32 * kq), ptx::desc_sw128(bk + 2048 * kq, kTile),
+                              IDESC_KM2, 1);
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(zc, ptx::desc_kmajor(ah + 32 * kq), ptx::desc_mnmajor(bl + 2048 * kq),
-                              IDESC_KM, 1);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(zc, ptx::desc_kmajor(al + 32 * kq), ptx::desc_mnmajor(bh_ + 2048 * kq),
-                              IDESC_KM, 1);
+            for (int kq = 0; kq < 4; ++kq)   // Z += A_lo [Kh_hi | Kh_lo]
+                ptx::mma_bf16(zc, ptx::desc_kmajor(al + 32 * kq), ptx::desc_sw128(bk + 2048 * kq, kTile),
+                              IDESC_KM2, 1);
             ptx::mma_commit(&s.mma2);
             issued2 = n;
         }
@@ -453,9 +449,12 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         ptx::tc_fence_after();
         // -------------------------------------------------------- output of chunk n
         {
-            uint32_t Z[32];
-            ptx::tmem_ld32(tmem + tlane + COL_Z + 64 * pb + 32 * hh, Z);
+            uint32_t Z[32], Z2[32];
+            ptx::tmem_ld32(tmem + tlane + COL_Z + 128 * pb + 32 * hh, Z);
+            ptx::tmem_ld32(tmem + tlane + COL_Z + 128 * pb + 64 + 32 * hh, Z2);
             ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) Z[j] = __float_as_uint(__uint_as_float(Z[j]) + __uint_as_float(Z2[j]));
             if (row_lane) {
                 const float dg = s.diag[t];
                 float* pdst = P + gx;
