@@ -356,10 +356,8 @@ def backward_line(cfg, dev, world, steps, c2=False):
     # base form: 2 reversals + fast + level kernels for dv (+ 2 segment kernels when the
     # sequence is split), the tensor-core dr and dk readouts, the two decay-gradient kernels,
     # the dr and dk scans (which exit at once unless a (b,h) fell back) and the du sum.
-    # Finch-C2: 1 reversal, the two tensor-core readouts, the two decay-gradient kernels and
-    # the dr + dv scan and dk scan launches (the scans' dr / dk parts exit unless a (b,h)
-    # fell back)
-    launches_per_call = 7 if c2 else 11
+    # (Finch-C2: the same launches; its dv prefill forms the query k (1 - w) inside)
+    launches_per_call = 11
     line = {"workload": ("wkv6c2_backward" if c2 else "wkv6_backward") + f" B{B} T{T} H{H}",
             "B": B, "T": T, "H": H, "D": D, "io": "bf16", "steps": steps, "ms_per_call": ms,
             "value": world * B * T / (ms / 1e3), "unit": "tokens/s",
@@ -372,9 +370,9 @@ def backward_line(cfg, dev, world, steps, c2=False):
             "gpu_launches": launches_per_call * steps,
             "kernels": ("dr and dk as chunked tensor-core readouts (wkv6_bwd_readout_tc_kernel "
                         "x2, kn = k (1 - w) formed in the dr pass), the decay gradient from "
-                        "their pair terms and kn's direct term, dv as a CUDA-core scan "
-                        "(wkv6_bwd_dr_dv_kernel); the CUDA-core dr / dk scans run only for a "
-                        "(b,h) that falls back") if c2 else
+                        "their pair terms and kn's direct term, dv through the chunked prefill "
+                        "on time-reversed copies with the query k (1 - w) formed inside; the "
+                        "CUDA-core scans run only for a (b,h) that falls back") if c2 else
                        ("dr and dk as chunked tensor-core readouts of the forward and the "
                         "reversed state (wkv6_bwd_readout_tc_kernel x2), the decay gradient from "
                         "their pair terms (wkv6_bwd_pq_sums_kernel, wkv6_bwd_domega_kernel), dv "
@@ -383,8 +381,7 @@ def backward_line(cfg, dev, world, steps, c2=False):
                         "CUDA-core scans run only for a (b,h) whose decays the one-sided factors "
                         "cannot take"),
             "note": "algorithmic FLOPs are the three recurrences (dr, dk, dv) at 5 FLOPs per "
-                    "state entry per token" + ("; dr and dk run on the tensor cores" if c2 else
-                                               "; dr, dk and dv run on the tensor cores")}
+                    "state entry per token; dr, dk and dv run on the tensor cores"}
     del inp, dy, dS, ws, args_b
     torch.cuda.empty_cache()
     return line

@@ -300,10 +300,11 @@ wkv_status wkv6_backward(const void *r, const void *k, const void *v, const void
  * dstate_out.  With kn_t = k_t (1 - w_t) and G as for wkv6_backward:
  *     dr_t = S_{t-1} dy_t;   dkn = G v_t, dk_t = dkn (1 - w_t);   dv_t = G^T kn_t;
  *     domega_t = (sum_j G[i][j] S_{t-1}[i][j] - dkn k_t) w_t (-exp(omega_t));   du'_t = dy_t
- * (no bonus; u' enters y additively).  With bf16 I/O dr and dk run on the tensor cores as
- * in wkv6_backward (kn formed in the dr pass; dk, Q and the direct term dkn k w from the dk
- * pass's readout dkn), with the same per-(b,h) fallback; dv, and everything with fp32 I/O,
- * are token-by-token scans on CUDA cores (fp32, fp64 row scans with fp32 I/O).  The decay
+ * (no bonus; u' enters y additively).  With bf16 I/O all three run on the tensor cores as
+ * in wkv6_backward: kn formed in the dr pass; dk, Q and the direct term dkn k w from the dk
+ * pass's readout dkn; dv through the chunked prefill on time-reversed copies with the query
+ * k (1 - w) formed inside; the same per-(b,h) fallback to token-by-token scans on CUDA
+ * cores, which also serve fp32 I/O (fp32, fp64 row scans with fp32 I/O).  The decay
  * gradient goes through the pair identity with the normalised keys.
  *   duprime  [B][T][H][D] io: output (a copy of dy), or NULL (not written).
  * Other arguments, layouts and errors as wkv6_backward; workspace: at least

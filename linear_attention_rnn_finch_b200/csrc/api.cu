@@ -648,8 +648,8 @@ wkv_status wkv6_decode_step_gn(const void* r, const void* k, const void* v, cons
 namespace {
 
 // Workspace of the backward: P and E in the row scans' accumulation type (fp64 for fp32
-// I/O, fp32 for bf16 I/O) and the per-(b,h) du parts; with tc_dv, also the time-reversed
-// k, r, dy, omega and dv and the chunked prefill's own workspace.
+// I/O, fp32 for bf16 I/O) and the per-(b,h) du parts; with bf16 I/O (the tensor-core path)
+// also the buffers listed below.
 size_t backward_bytes(int B, int T, int H, int D, wkv_dtype io, bool c2) {
     const bool tc = io == WKV_BF16;   // the tensor-core path
     if (B <= 0 || T <= 0 || H <= 0 || D != kHeadSizeApi || !valid_io(io)) return 0;
@@ -708,8 +708,7 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
             if (overlaps(outs[a], outs[b2])) return WKV_ERR_INVALID_ARG;
     }
     const bool bf16 = io == WKV_BF16;
-    const bool tc = bf16;             // dr and dk on the tensor cores
-    const bool tc_dv = bf16 && !c2;   // dv through the chunked tensor-core prefill
+    const bool tc = bf16;   // dr, dk and dv on the tensor cores
     const size_t need = backward_bytes(B, T, H, D, io, c2);
     if (need > 0) {
         if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
@@ -770,22 +769,22 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
                             round256((size_t)B * H * ((T + kChunk - 1) / kChunk) * 128 * sizeof(float)))
                       : nullptr;
     const long long budget = injected("timeout0") ? 0 : kSpinBudget;
-    // status word for the tensor-core passes (the chunked prefill's, when it runs)
-    if (!tc_dv && cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return WKV_ERR_CUDA;
     {
         const void* src[5] = {r, dy, omega, v, k};
         void* dst[5] = {rr, rdy, rom, rv, rk};
-        if (goldwkv::launch_reverse_tokens(src, dst, tc_dv ? 5 : 4, B, T, H, st) != cudaSuccess)
+        if (goldwkv::launch_reverse_tokens(src, dst, 5, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
-    if (tc_dv) {
+    {
         // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
-        // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = k_t . G.
-        // It runs through the chunked tensor-core prefill on the reversed copies.  (Finch-C2's
-        // dv, whose query is k (1 - w), stays a CUDA-core scan, launched with the dr scan.)
+        // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = q_t . G
+        // (+ the bonus), with the query q = k, or Finch-C2's kn = k (1 - w) (no bonus).  It
+        // runs through the chunked tensor-core prefill on the reversed copies.
+        goldwkv::Variant var{nullptr};
+        var.query_c2 = c2;
         cudaError_t e = cudaSuccess;
-        if (!launch_chunked_path(rk, rr, rdy, rom, u, goldwkv::Variant{nullptr}, dstate_out,
-                                 nullptr, rout, nullptr, B, T, H, P_seg, false, cws, st, &e) ||
+        if (!launch_chunked_path(rk, rr, rdy, rom, ub, var, dstate_out, nullptr, rout, nullptr, B,
+                                 T, H, P_seg, false, cws, st, &e) ||
             e != cudaSuccess)
             return WKV_ERR_CUDA;
         const void* s1[1] = {rout};
@@ -808,7 +807,7 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
                                   budget, st, c2) != cudaSuccess)
         return WKV_ERR_CUDA;
     if (goldwkv::launch_backward(r, k, v, omega, ub, state_in, dy, dstate_out, dr, dk, dv, domega,
-                                 du, dstate_in, P, E, du_part, B, T, H, bf16, /*with_dv=*/!tc_dv,
+                                 du, dstate_in, P, E, du_part, B, T, H, bf16, /*with_dv=*/false,
                                  c2, st, dr_flags, nullptr, goldwkv::kPhaseDr) != cudaSuccess)
         return WKV_ERR_CUDA;
     // dk (and dS0, Q) as the same readout in reversed time: query v, key r, value dy; dk and

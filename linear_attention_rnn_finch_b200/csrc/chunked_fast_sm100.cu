@@ -336,7 +336,8 @@ __device__ __forceinline__ void load_v(Smem& s, const CUtensorMap* tm_v, int n, 
 
 // kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
 // kGN: base form with the GroupNorm + gate output stage (gn).
-template <bool kC2, bool kGN>
+// kQ: no bonus, query r (1 - w) (Variant::query_c2).
+template <bool kC2, bool kGN, bool kQ>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
@@ -409,7 +410,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
         float2 uu[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            uu[q] = kC2 ? make_float2(0.f, 0.f) : make_float2(u[h * 64 + c0 + 2 * q], u[h * 64 + c0 + 2 * q + 1]);
+            uu[q] = (kC2 || kQ) ? make_float2(0.f, 0.f) : make_float2(u[h * 64 + c0 + 2 * q], u[h * 64 + c0 + 2 * q + 1]);
         uint32_t toff[4];   // byte offset of this thread's 16-byte column in token row tb + p
 #pragma unroll
         for (int p = 0; p < 4; ++p) toff[p] = (uint32_t)((tb + p) * 128 + ((cg ^ ((tb + p) & 7)) << 4));
@@ -582,12 +583,13 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                     const float2 fr = exp2_2(prev[q]);
                     const float2 fk = exp2_2(make_float2(-L[p][q].x, -L[p][q].y));
                     prev[q] = L[p][q];
-                    const float2 rr2 = unpack2(word(rv, q));
+                    float2 rr2 = unpack2(word(rv, q));
                     float2 kk = unpack2(word(kv, q));
-                    if (kC2) {   // k (1 - w), 1 - w = 1 - exp(-exp(omega)) without cancellation
+                    if (kC2 || kQ) {   // (1 - w), 1 - w = 1 - exp(-exp(omega)) without cancellation
                         float2 e = exp2_2(__fmul2_rn(unpack2(word(wv[p], q)), l2e));
                         if (t >= valid) e = make_float2(0.f, 0.f);
-                        kk = __fmul2_rn(kk, one_minus_exp_neg2(e));
+                        if (kC2) kk = __fmul2_rn(kk, one_minus_exp_neg2(e));   // key k (1 - w)
+                        else rr2 = __fmul2_rn(rr2, one_minus_exp_neg2(e));     // query r (1 - w)
                     }
                     split2(__fmul2_rn(rr2, fr), rh[q], rl[q]);
                     split2(__fmul2_rn(kk, fk), khv[q], klv[q]);
@@ -849,9 +851,10 @@ cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const f
                                 float* handoff_state, long long budget, cudaStream_t st,
                                 const GnOut* gn) {
     const size_t smem = fast_smem_bytes();
-    auto kernel = var.uprime ? wkv6_fast_kernel<true, false>
-                  : gn       ? wkv6_fast_kernel<false, true>
-                             : wkv6_fast_kernel<false, false>;
+    auto kernel = var.uprime     ? wkv6_fast_kernel<true, false, false>
+                  : gn           ? wkv6_fast_kernel<false, true, false>
+                  : var.query_c2 ? wkv6_fast_kernel<false, false, true>
+                                 : wkv6_fast_kernel<false, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const GnOut g = gn ? *gn : GnOut{nullptr, nullptr, 0.f, nullptr};

@@ -128,7 +128,8 @@ __device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 
 
 // kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
 // kGN: base form with the GroupNorm + gate output stage (gn).
-template <bool kC2, bool kGN>
+// kQ: no bonus, query r (1 - w) (Variant::query_c2).
+template <bool kC2, bool kGN, bool kQ>
 __global__ void __launch_bounds__(kThreads, 1)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
@@ -166,7 +167,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
         ptx::prefetch_tensormap(&tm_w);
         ptx::prefetch_tensormap(&tm_y);
     }
-    if (tid < 64) s.u[tid] = kC2 ? 0.f : u[h * 64 + tid];
+    if (tid < 64) s.u[tid] = (kC2 || kQ) ? 0.f : u[h * 64 + tid];
     if (warp == 0) ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     // zero the operand tiles once, so that rows an MMA reads but never uses hold finite data
     for (int i = tid; i < (int)(sizeof(s.q) + sizeof(s.kk)) / 16; i += kThreads)
@@ -263,6 +264,15 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                             kv[p][c] *= (ta + p < valid) ? -expm1f(-__expf(om[p][c])) : 0.f;
                     st_shared_v4(k_tile, sw_chunk(ta, cg), pack8(kv[0]));
                     st_shared_v4(k_tile, sw_chunk(tb, cg), pack8(kv[1]));
+                }
+                if (kQ) {   // query r (1 - w); level 0 reads the r tile itself: rewritten in place
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            rv[p][c] *= (ta + p < valid) ? -expm1f(-__expf(om[p][c])) : 0.f;
+                    st_shared_v4(r_tile, sw_chunk(ta, cg), pack8(rv[0]));
+                    st_shared_v4(r_tile, sw_chunk(tb, cg), pack8(rv[1]));
                 }
             }
             // bonus partials: sum over this lane's 8 channels of r u k
@@ -659,9 +669,10 @@ cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const
                                   const float* handoff_state, long long spin_budget,
                                   cudaStream_t st, const GnOut* gn) {
     const size_t smem = chunked_smem_bytes();
-    auto kernel = var.uprime ? wkv6_chunked_kernel<true, false>
-                  : gn       ? wkv6_chunked_kernel<false, true>
-                             : wkv6_chunked_kernel<false, false>;
+    auto kernel = var.uprime     ? wkv6_chunked_kernel<true, false, false>
+                  : gn           ? wkv6_chunked_kernel<false, true, false>
+                  : var.query_c2 ? wkv6_chunked_kernel<false, false, true>
+                                 : wkv6_chunked_kernel<false, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long drain = 4000000000LL;

@@ -15,6 +15,9 @@ namespace goldwkv {
 // readout before LayerNorm.
 struct Variant {
     const void* uprime;
+    // query_c2 (base form, no bonus): the query is r (1 - w) instead of r -- Finch-C2's dv,
+    // the forward recurrence in reversed time whose query is the normalised key k (1 - w)
+    bool query_c2 = false;
 };
 
 // Token-by-token recurrence (fp32 math).  y_raw != nullptr: write fp32 un-normalised y
