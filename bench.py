@@ -89,7 +89,7 @@ CSRC = ROOT / "linear_attention_rnn_finch_b200" / "csrc"
 NCU_TRAFFIC = {
     "prefill": {"sources": ("chunked_fast_sm100.cu", "chunk_tiles.cuh", "sm100_ptx.cuh", "common.cuh",
                             "internal.h"),
-                "sha256_16": "85a5d09a0f7ea761", "bytes": 541159680 + 118830080,
+                "sha256_16": "e07ae25d1780988a", "bytes": 541190912 + 118802176,
                 "workload": (8, 4096, 32)},
     "decode": {"sources": ("decode.cu", "common.cuh"),
                "sha256_16": "0468671fdbdebeab", "bytes": 138433024 + 78395392,

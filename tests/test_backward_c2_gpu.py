@@ -88,6 +88,20 @@ def test_c2_backward_bf16_some_heads_fall_back(oracle):
     _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
 
 
+@pytest.mark.parametrize("segments", [None, "3"])
+def test_c2_backward_bf16_extreme_decay_and_split(oracle, monkeypatch, segments):
+    """bf16: dv runs through the chunked prefill's query-(1 - w) variant on time-reversed
+    copies; decays near zero make it hand sequences to the level kernel, and a forced 3-way
+    sequence split runs the segment pre-pass on the reversed sequence."""
+    if segments:
+        monkeypatch.setenv("GOLDWKV_SEGMENTS", segments)
+    inp = _problem(10177, B=2, T=1100, H=2, dtype=torch.bfloat16)
+    om = inp["omega"].float()
+    om[:, 300:420, 1, ::3] = 3.5
+    inp["omega"] = om.to(torch.bfloat16)
+    _compare(_gpu(inp), _oracle(oracle, inp), TOL[torch.bfloat16])
+
+
 def test_c2_backward_duprime_is_dy():
     inp = _problem(10180, B=1, T=70, H=2, dtype=torch.bfloat16)
     out = _gpu(inp)
