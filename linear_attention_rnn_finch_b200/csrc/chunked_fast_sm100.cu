@@ -106,7 +106,9 @@ struct __align__(1024) Smem {
     uint8_t kh[2][2 * kTile];           // per parity: Kh_hi tile, then Kh_lo tile
     uint8_t sb[2][2 * kTile];           // S_hi^T tile, then S_lo^T tile; sb[m & 1] feeds RO(m)
     uint8_t at[2 * kTile];              // A hi/lo, 128 stacked rows
-    float qtot[kPrepGroups][kGroupWarps][64];   // prep: per-warp sums of log2 w
+    // prep: per-warp sums of log2 w, 8 channels per 16-byte pair of columns, rows padded to
+    // 12 floats so that the 8 column groups a quarter-warp reads fall in distinct banks
+    float qtot[kPrepGroups][kGroupWarps][8][12];
     float gamma[4][64];                 // gamma and bonus of chunk n in slot n % 4
     float bonus[4][64];
     uint64_t full_rkw[kStagesRkw], full_v[kStagesV];
@@ -504,7 +506,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
                 exc[q] = rr > 0 ? o : make_float2(0.f, 0.f);
             }
             if (rr == 3) {   // warp totals for channels c0 .. c0+7
-                float4* dst = reinterpret_cast<float4*>(&s.qtot[g][wg][c0]);
+                float4* dst = reinterpret_cast<float4*>(&s.qtot[g][wg][cg][0]);
                 dst[0] = make_float4(inc[0].x, inc[0].y, inc[1].x, inc[1].y);
                 dst[1] = make_float4(inc[2].x, inc[2].y, inc[3].x, inc[3].y);
             }
@@ -519,7 +521,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
             for (int q = 0; q < 4; ++q) off[q] = tot[q] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int w = 0; w < kGroupWarps; ++w) {
-                const float4* src = reinterpret_cast<const float4*>(&s.qtot[g][w][c0]);
+                const float4* src = reinterpret_cast<const float4*>(&s.qtot[g][w][cg][0]);
                 const float4 a0 = src[0], a1 = src[1];
                 const float2 v[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w),
                                      make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
@@ -844,6 +846,7 @@ wkv6_fast_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant
 }  // namespace
 
 size_t fast_smem_bytes() { return sizeof(Smem) + 1024; }
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "the fast kernel's shared memory exceeds a CTA's 227 KB");
 
 cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const float* s_in,
                                 float* s_out, void* y, float* y_raw, int B, int T, int H,
