@@ -23,8 +23,9 @@
 //       roles r <-> k, v -> dy run backwards
 //   dk  rows of G, reverse in time, with the decay-gradient scan fused (needs P and E).
 // The dr and dv sweeps run as one launch (blockIdx.z); the dk sweep follows; a small kernel
-// sums du over the batch.  Because dv is exactly a forward recurrence in reversed time, the
-// bf16 path leaves it out of these scans and runs it through the chunked tensor-core
+// sums du over the batch.  These scans are the whole fp32-I/O path.  With bf16 I/O they run
+// only for a (b,h) that the tensor-core readouts (backward_tc_sm100.cu) hand back, and dv,
+// exactly a forward recurrence in reversed time, runs through the chunked tensor-core
 // prefill on time-reversed copies (reverse_tokens_kernel moves them).
 //
 // Work split: a CTA owns one (b,h) and 32 of the 64 rows (dr, dk) or columns (dv); each
@@ -37,7 +38,8 @@
 // is no bonus, so the dr and dv scans use kn in place of k (formed while staging), the dk
 // scan yields dkn and returns dk = dkn (1 - w) with Q_t = kn_t dkn_t, and the decay gradient
 // gains the direct term of kn on w: domega += dkn k w exp(omega).  du' = dy is the caller's
-// copy.  dv stays a CUDA-core scan in this form (the chunked prefill would need kn in bf16).
+// copy.  With bf16 I/O dv goes through the chunked prefill here too, its query kn formed in
+// the prefill's own staging; with fp32 I/O it is the dv scan with kn.
 //
 // Precision.  The identity subtracts, at every token, the pair terms that start at or after
 // it; where w_t is tiny the result is tiny too and what is left is the rounding of those
@@ -536,16 +538,37 @@ struct ReverseArgs {
     uint4* dst[kMaxReverse];
 };
 
-__global__ void reverse_tokens_kernel(ReverseArgs a, int n, long B, int T, int H) {
-    const long per = (long)T * H * 8;               // 16-byte chunks per batch row
-    const long total = B * per;
-    for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-         e += (long)gridDim.x * blockDim.x) {
-        const long b = e / per;
-        const long rem = e - b * per;
-        const long t = rem / ((long)H * 8);
-        const long src_e = b * per + ((long)(T - 1 - t) * H * 8) + (rem - t * H * 8);
-        for (int i = 0; i < n; ++i) a.dst[i][e] = a.src[i][src_e];
+// A CTA moves kRows token rows (H*8 16-byte chunks each) of all kN tensors per step, every
+// load of the step issued before its first store: kRows * kN = 8-10 loads in flight per
+// thread, whatever the number of tensors (the destinations may not alias the sources, so
+// nothing else would let a store wait behind the next load).
+template <int kN>
+__global__ void __launch_bounds__(256) reverse_tokens_kernel(ReverseArgs a, long rows, int T,
+                                                             int row_chunks) {
+    constexpr int kRows = kN >= 4 ? 2 : 8 / kN;
+    for (long r0 = (long)blockIdx.x * kRows; r0 < rows; r0 += (long)gridDim.x * kRows) {
+        for (int c = threadIdx.x; c < row_chunks; c += blockDim.x) {
+            uint4 x[kRows][kN];
+            long dst[kRows];
+#pragma unroll
+            for (int j = 0; j < kRows; ++j) {
+                const long bt = r0 + j;
+                dst[j] = -1;
+                if (bt < rows) {
+                    const long b = bt / T, t = bt - b * T;
+                    const long src = (b * T + (T - 1 - t)) * row_chunks + c;
+                    dst[j] = bt * row_chunks + c;
+#pragma unroll
+                    for (int i = 0; i < kN; ++i) x[j][i] = a.src[i][src];
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kRows; ++j)
+                if (dst[j] >= 0) {
+#pragma unroll
+                    for (int i = 0; i < kN; ++i) a.dst[i][dst[j]] = x[j][i];
+                }
+        }
     }
 }
 
@@ -620,10 +643,18 @@ cudaError_t launch_reverse_tokens(const void* const* src, void* const* dst, int 
         a.src[i] = static_cast<const uint4*>(src[i]);
         a.dst[i] = static_cast<uint4*>(dst[i]);
     }
-    const long total = (long)B * T * H * 8;
-    const long blocks = (total + 255) / 256;
-    reverse_tokens_kernel<<<(unsigned)(blocks < 148L * 16 ? blocks : 148L * 16), 256, 0, st>>>(
-        a, n, B, T, H);
+    const long rows = (long)B * T;
+    const int row_chunks = H * 8;
+    const int per_cta = n >= 4 ? 2 : 8 / n;
+    const long need = (rows + per_cta - 1) / per_cta;
+    const unsigned grid = (unsigned)(need < 148L * 32 ? need : 148L * 32);
+    switch (n) {
+        case 1: reverse_tokens_kernel<1><<<grid, 256, 0, st>>>(a, rows, T, row_chunks); break;
+        case 2: reverse_tokens_kernel<2><<<grid, 256, 0, st>>>(a, rows, T, row_chunks); break;
+        case 3: reverse_tokens_kernel<3><<<grid, 256, 0, st>>>(a, rows, T, row_chunks); break;
+        case 4: reverse_tokens_kernel<4><<<grid, 256, 0, st>>>(a, rows, T, row_chunks); break;
+        default: reverse_tokens_kernel<5><<<grid, 256, 0, st>>>(a, rows, T, row_chunks); break;
+    }
     return cudaGetLastError();
 }
 

@@ -621,47 +621,60 @@ namespace {
 
 // Decay gradient from the pair terms (the identity of csrc/backward.cu):
 //     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,   domega_t = dlog w_t (-exp(omega_t)),
-// P and Q in token order.  First the column sums
-// of P and Q over each 64-token chunk, then per chunk the sums over the later chunks and a
-// reverse scan over its own tokens.  One thread per channel, one CTA per (b,h,chunk).
-__global__ void __launch_bounds__(64)
+// P and Q in token order.  First the column sums of P and Q over each 64-token chunk, then
+// per chunk the sums over the later chunks and a reverse scan over its own tokens.  One
+// thread per channel and chunk, kDomegaChunks chunks of one (b,h) per CTA.  (One CTA per
+// (b,h) walking its chunks backwards with a running total reads P and Q once instead of
+// twice, but at 256 CTAs each chunk's loads wait in line: it measured slower.)
+constexpr int kDomegaChunks = 4;
+
+__global__ void __launch_bounds__(64 * kDomegaChunks)
 wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q,
                         float* __restrict__ sums, int T, int H) {
-    const int NC = (T + C - 1) / C;
-    const int n = blockIdx.x % NC, bh = blockIdx.x / NC, b = bh / H, h = bh - (bh / H) * H;
-    const int i = threadIdx.x, t0 = n * C, valid = min(C, T - t0);
-    float sp = 0.f, sq = 0.f;
+    const int NC = (T + C - 1) / C, groups = (NC + kDomegaChunks - 1) / kDomegaChunks;
+    const int g = blockIdx.x % groups, bh = blockIdx.x / groups, b = bh / H, h = bh - b * H;
+    const int n = g * kDomegaChunks + (threadIdx.x >> 6), i = threadIdx.x & 63;
+    if (n >= NC) return;
+    const int t0 = n * C, valid = min(C, T - t0);
+    const size_t stride = (size_t)H * 64, x0 = (((size_t)b * T + t0) * H + h) * 64 + i;
+    // four partial sums: the loads of 8 tokens in flight, not one add chain
+    float sp[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
     for (int tt = 0; tt < valid; ++tt) {
-        const int t = t0 + tt;
-        sp += P[(((size_t)b * T + t) * H + h) * 64 + i];
-        sq += Q[(((size_t)b * T + t) * H + h) * 64 + i];
+        sp[tt & 3] += P[x0 + tt * stride];
+        sq[tt & 3] += Q[x0 + tt * stride];
     }
     float* o = sums + ((size_t)bh * NC + n) * 128;
-    o[i] = sp;
-    o[64 + i] = sq;
+    o[i] = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+    o[64 + i] = (sq[0] + sq[1]) + (sq[2] + sq[3]);
 }
 
-__global__ void __launch_bounds__(64)
+// CTAs run in the reverse of the sums kernel's order, so the first of them find the P and Q
+// that kernel read last still in L2.
+__global__ void __launch_bounds__(64 * kDomegaChunks)
 wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
                        const float* __restrict__ Dw, const float* __restrict__ sums,
                        const float* __restrict__ E,
                        const __nv_bfloat16* __restrict__ omega, __nv_bfloat16* __restrict__ domega,
                        int T, int H) {
-    const int NC = (T + C - 1) / C;
-    const int n = blockIdx.x % NC, bh = blockIdx.x / NC, b = bh / H, h = bh - (bh / H) * H;
-    const int i = threadIdx.x, t0 = n * C, valid = min(C, T - t0);
-    // E + sum over the later chunks of (P - Q)
-    float acc = E[(size_t)bh * 64 + i];
-    for (int m = n + 1; m < NC; ++m) {
-        const float* o = sums + ((size_t)bh * NC + m) * 128;
-        acc += o[i] - o[64 + i];
-    }
+    const int NC = (T + C - 1) / C, groups = (NC + kDomegaChunks - 1) / kDomegaChunks;
+    const int blk = gridDim.x - 1 - blockIdx.x;
+    const int g = blk % groups, bh = blk / groups, b = bh / H, h = bh - b * H;
+    const int n = g * kDomegaChunks + (threadIdx.x >> 6), i = threadIdx.x & 63;
+    if (n >= NC) return;
+    const int t0 = n * C, valid = min(C, T - t0);
+    // E + sum over the later chunks of (P - Q), four independent partial sums
+    const float* o = sums + (size_t)bh * NC * 128 + i;
+    float part[4] = {E[(size_t)bh * 64 + i], 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int m = n + 1; m < NC; ++m) part[(m - n) & 3] += o[(size_t)m * 128] - o[(size_t)m * 128 + 64];
+    float acc = (part[0] + part[1]) + (part[2] + part[3]);
     // reverse over this chunk: dlog w_t = acc_after(t) - Q_t, with acc_after(t) = E + sum_{s>t}
     // P_s - sum_{s>t} Q_s
+    const size_t stride = (size_t)H * 64, x0 = (((size_t)b * T + t0) * H + h) * 64 + i;
+#pragma unroll 8
     for (int tt = valid - 1; tt >= 0; --tt) {
-        const int t = t0 + tt;
-        const size_t x = (((size_t)b * T + t) * H + h) * 64 + i;
+        const size_t x = x0 + tt * stride;
         const float q = Q[x];
         const float dl = acc - q - (Dw != nullptr ? Dw[x] : 0.f);
         domega[x] = __float2bfloat16_rn(dl * -__expf(__bfloat162float(omega[x])));
@@ -675,12 +688,13 @@ cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, fl
                               const float* E,
                               const void* omega, void* domega, int B, int T, int H,
                               cudaStream_t st) {
-    const unsigned blocks = (unsigned)((long)B * H * ((T + C - 1) / C));
+    const long groups = ((T + C - 1) / C + kDomegaChunks - 1) / kDomegaChunks;
+    const unsigned blocks = (unsigned)((long)B * H * groups);
     if (blocks == 0) return cudaSuccess;
-    wkv6_bwd_pq_sums_kernel<<<blocks, 64, 0, st>>>(P, Q, sums, T, H);
+    wkv6_bwd_pq_sums_kernel<<<blocks, 64 * kDomegaChunks, 0, st>>>(P, Q, sums, T, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_domega_kernel<<<blocks, 64, 0, st>>>(P, Q, D, sums, E,
+    wkv6_bwd_domega_kernel<<<blocks, 64 * kDomegaChunks, 0, st>>>(P, Q, D, sums, E,
                                                   static_cast<const __nv_bfloat16*>(omega),
                                                   static_cast<__nv_bfloat16*>(domega), T, H);
     return cudaGetLastError();
