@@ -19,13 +19,16 @@
  * Conventions shared by every entry point
  *  - Pointers r, k, v, omega, u, state*, y, gamma, beta, workspace are DEVICE pointers on
  *    the current CUDA device; the caller owns every buffer.  The library never allocates
- *    device memory, keeps no global mutable state (one exception: the built-in scratch of
- *    wkv6_prefill_static) and, apart from wkv6_workspace_status and
+ *    device memory, keeps no global mutable state (two exceptions: the built-in scratch of
+ *    wkv6_prefill_static, and the two side streams per device that the bf16 backward
+ *    entry points create on first use) and, apart from wkv6_workspace_status and
  *    wkv6_prefill_static_status, never synchronises, so calls on different streams with
  *    different workspaces are independent.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
  *    enqueued asynchronously; a device-side fault surfaces as a CUDA error at the caller's
- *    next synchronisation.
+ *    next synchronisation.  The bf16 backward entry points fork part of their work onto
+ *    their side streams through events recorded on `stream` and join it back the same way
+ *    before they return: to the caller the call is ordered on `stream` like any other.
  *  - Arguments are validated before anything is launched; on any error nothing is
  *    launched and no output is touched.
  *  - Layouts are row-major and dense:

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "goldwkv.h"
 #include "internal.h"
@@ -167,6 +168,95 @@ int sm_count() {
     cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
+
+// Side streams per device, with a fork event and a join event each, for passes of one call
+// that depend on none of each other's work: kernels on several streams run side by side,
+// and the CTAs of one take the SMs another leaves idle in its last wave.  The mutex keeps
+// each record-and-wait sequence of a call together when several host threads call at once
+// (each join then follows that call's own work on its side stream: a stream runs in order).
+constexpr int kSideStreams = 2;
+struct SideStreams {
+    cudaStream_t s[kSideStreams] = {};
+    cudaEvent_t fork = nullptr;
+    cudaEvent_t join[kSideStreams] = {};
+};
+constexpr int kMaxSideDevices = 64;
+std::mutex g_side_mutex;
+SideStreams g_side[kMaxSideDevices];
+
+void destroy_side(SideStreams& n) {
+    for (int i = 0; i < kSideStreams; ++i) {
+        if (n.join[i]) cudaEventDestroy(n.join[i]);
+        if (n.s[i]) cudaStreamDestroy(n.s[i]);
+    }
+    if (n.fork) cudaEventDestroy(n.fork);
+}
+
+// The current device's side streams (created on first use, under g_side_mutex), or null: no
+// device, or creation failed, or st is being captured into a graph and the streams do not
+// exist yet (creating them then could invalidate the capture) -- the caller then queues
+// everything on st, in order.
+const SideStreams* side_streams_locked(cudaStream_t st) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    SideStreams& sd = g_side[dev];
+    if (sd.s[0] != nullptr) return &sd;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    SideStreams n;
+    bool ok = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < kSideStreams; ++i)
+        ok = cudaStreamCreateWithFlags(&n.s[i], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreateWithFlags(&n.join[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        (void)cudaGetLastError();
+        destroy_side(n);
+        return nullptr;
+    }
+    sd = n;
+    return &sd;
+}
+
+// Work queued on side(i) after the constructor runs after everything queued on st before
+// it; everything queued on st after join() (or the destructor) runs after that work.
+// Without side streams side(i) is st itself.
+class Fork {
+  public:
+    explicit Fork(cudaStream_t st) : st_(st) {
+        std::lock_guard<std::mutex> lock(g_side_mutex);
+        sd_ = side_streams_locked(st);
+        if (sd_ == nullptr) return;
+        ok_ = cudaEventRecord(sd_->fork, st) == cudaSuccess;
+        for (int i = 0; ok_ && i < kSideStreams; ++i)
+            ok_ = cudaStreamWaitEvent(sd_->s[i], sd_->fork, 0) == cudaSuccess;
+    }
+    Fork(const Fork&) = delete;
+    Fork& operator=(const Fork&) = delete;
+    ~Fork() { (void)join(); }
+    bool ok() const { return ok_; }
+    cudaStream_t side(int i) const { return sd_ != nullptr ? sd_->s[i] : st_; }
+    bool join() {
+        if (sd_ == nullptr || joined_) return ok_;
+        joined_ = true;
+        std::lock_guard<std::mutex> lock(g_side_mutex);
+        for (int i = 0; i < kSideStreams; ++i)
+            if (cudaEventRecord(sd_->join[i], sd_->s[i]) != cudaSuccess ||
+                cudaStreamWaitEvent(st_, sd_->join[i], 0) != cudaSuccess)
+                ok_ = false;
+        return ok_;
+    }
+
+  private:
+    cudaStream_t st_;
+    const SideStreams* sd_ = nullptr;
+    bool ok_ = true, joined_ = false;
+};
 
 long waves(long ctas, int per_sm = 1) {
     const long slots = (long)sm_count() * per_sm;
@@ -775,27 +865,48 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         if (goldwkv::launch_reverse_tokens(src, dst, 5, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
+    // The three passes after the reversal need only its copies and the inputs, and share no
+    // buffer: dk on st, dv (the prefill on the reversed copies, then its reversal) on one
+    // side stream, dr on the other, queued in that order (a readout's CTAs outlast the
+    // prefill's two to one: long ones first).  Each pass is 256 CTAs of one SM apiece, so
+    // alone it leaves SMs idle in its last wave; side by side, the other passes' CTAs take
+    // them.  The decay gradient, after the join, needs P and E of dr and Q of dk.
+    Fork fork(st);
+    if (!fork.ok()) return WKV_ERR_CUDA;
+    CUtensorMap maps[5];
+    // dk (and dS0, Q) as the readout of the forward state's adjoint in reversed time: query
+    // v, key r, value dy; dk and Q go straight to token order (the fifth map, the dr pass's
+    // store, is not used by this pass)
+    if (!goldwkv::make_token_map(&maps[0], rv, B, T, H) ||
+        !goldwkv::make_token_map(&maps[1], rr, B, T, H) ||
+        !goldwkv::make_token_map(&maps[2], rdy, B, T, H) ||
+        !goldwkv::make_token_map(&maps[3], rom, B, T, H) ||
+        !goldwkv::make_token_map(&maps[4], dk, B, T, H))
+        return WKV_ERR_CUDA;
+    if (goldwkv::launch_bwd_dk_tc(maps, k, ub, dstate_out, dk, q_tok, d_tok, dstate_in, dk_flags, B,
+                                  T, H, status, budget, st, c2) != cudaSuccess)
+        return WKV_ERR_CUDA;
     {
         // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
         // swapped and dy as the value: G_t = diag(w_t) G_{t+1} + r_t^T dy_t, dv_t = q_t . G
         // (+ the bonus), with the query q = k, or Finch-C2's kn = k (1 - w) (no bonus).  It
         // runs through the chunked tensor-core prefill on the reversed copies.
+        const cudaStream_t sd = fork.side(0);
         goldwkv::Variant var{nullptr};
         var.query_c2 = c2;
         cudaError_t e = cudaSuccess;
         if (!launch_chunked_path(rk, rr, rdy, rom, ub, var, dstate_out, nullptr, rout, nullptr, B,
-                                 T, H, P_seg, false, cws, st, &e) ||
+                                 T, H, P_seg, false, cws, sd, &e) ||
             e != cudaSuccess)
             return WKV_ERR_CUDA;
         const void* s1[1] = {rout};
         void* d1[1] = {dv};
-        if (goldwkv::launch_reverse_tokens(s1, d1, 1, B, T, H, st) != cudaSuccess)
+        if (goldwkv::launch_reverse_tokens(s1, d1, 1, B, T, H, sd) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
     // dr (with P, E and du's parts) as the chunked readout of the forward state; a (b,h)
     // whose decay range the one-sided factorisation cannot take is flagged and redone by the
     // CUDA-core dr scan, so that P and E are complete before the decay gradient
-    CUtensorMap maps[5];
     if (!goldwkv::make_token_map(&maps[0], dy, B, T, H) ||
         !goldwkv::make_token_map(&maps[1], k, B, T, H) ||
         !goldwkv::make_token_map(&maps[2], v, B, T, H) ||
@@ -804,23 +915,14 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         return WKV_ERR_CUDA;
     if (goldwkv::launch_bwd_dr_tc(maps, r, ub, state_in, dstate_out, static_cast<float*>(P),
                                   reinterpret_cast<float*>(E), du_part, dr_flags, B, T, H, status,
-                                  budget, st, c2) != cudaSuccess)
+                                  budget, fork.side(1), c2) != cudaSuccess)
         return WKV_ERR_CUDA;
     if (goldwkv::launch_backward(r, k, v, omega, ub, state_in, dy, dstate_out, dr, dk, dv, domega,
                                  du, dstate_in, P, E, du_part, B, T, H, bf16, /*with_dv=*/false,
-                                 c2, st, dr_flags, nullptr, goldwkv::kPhaseDr) != cudaSuccess)
+                                 c2, fork.side(1), dr_flags, nullptr, goldwkv::kPhaseDr) !=
+        cudaSuccess)
         return WKV_ERR_CUDA;
-    // dk (and dS0, Q) as the same readout in reversed time: query v, key r, value dy; dk and
-    // Q go straight to token order
-    if (!goldwkv::make_token_map(&maps[0], rv, B, T, H) ||
-        !goldwkv::make_token_map(&maps[1], rr, B, T, H) ||
-        !goldwkv::make_token_map(&maps[2], rdy, B, T, H) ||
-        !goldwkv::make_token_map(&maps[3], rom, B, T, H) ||
-        !goldwkv::make_token_map(&maps[4], rout, B, T, H))
-        return WKV_ERR_CUDA;
-    if (goldwkv::launch_bwd_dk_tc(maps, k, ub, dstate_out, dk, q_tok, d_tok, dstate_in, dk_flags, B,
-                                  T, H, status, budget, st, c2) != cudaSuccess)
-        return WKV_ERR_CUDA;
+    if (!fork.join()) return WKV_ERR_CUDA;
     if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_tok, d_tok, sums,
                                    reinterpret_cast<const float*>(E), omega, domega, B, T, H,
                                    st) != cudaSuccess)
