@@ -25,6 +25,9 @@
 //   state : S <- gamma S + U in registers, S_hi / S_lo tiles for the next chunk;
 //   out   : dr = F Z + u k diag (bf16 tile, TMA store); for the decay gradient the pair
 //           terms ending at t, P_t = r_t (dr_t - bonus) (fp32), and du's per-(b,h) sums.
+// The M = 64 accumulators (A, U, Z) keep their rows in lanes 0-15 of each TMEM
+// sub-partition; a two-half TMEM load gives every thread of a warp a row, 16 columns each,
+// so the A, state and out steps run on all 32 lanes (the state S too: 16 fp32 a thread).
 // Pipelined over chunks: iteration n forms A(n), issues MMA 2(n), advances the state and
 // prepares chunk n+1 while MMA 2 runs, issues MMA 1(n+1), and forms the output of n while
 // MMA 1(n+1) runs (prep buffers, F, gamma and Z alternate by chunk parity).
@@ -177,36 +180,37 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
     if (tid == 0)
         for (int n = 0; n < kStages && n < NC; ++n) issue_load(n);
 
-    // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in lanes 0..15), column half hh
+    // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in its lanes 0..15), columns
+    // 32 hh .. 32 hh + 31.  Lane l takes row 16q + (l & 15) and 16 of those columns, from
+    // cb = 32 hh + 16 (l >> 4): the two-half TMEM load gives every lane a row.
     const int q = warp & 3, hh = warp >> 2;
-    const bool row_lane = lane < 16;
     const int row = 16 * q + (lane & 15);        // state row i / token row t of this lane
+    const int cb = 32 * hh + 16 * (lane >> 4);   // its first column
+    const int cc0 = cb >> 3;                     // its first 16-byte chunk of a tile row
     const uint32_t tlane = (uint32_t)(32 * q) << 16;
-    float S[32];
+    float S[16];
     {
-        const float* src = state_in ? state_in + (size_t)bh * 4096 + row * 64 + 32 * hh : nullptr;
+        const float* src = state_in ? state_in + (size_t)bh * 4096 + row * 64 + cb : nullptr;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
+        for (int j = 0; j < 16; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (src && row_lane) x = *reinterpret_cast<const float4*>(src + j);
+            if (src) x = *reinterpret_cast<const float4*>(src + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        if (row_lane) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float f[8];
+        for (int cc = 0; cc < 2; ++cc) {
+            float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
-                uint4 hi, lo;
-                split8(f, hi, lo);
-                *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, 4 * hh + cc)) = hi;
-                *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, 4 * hh + cc)) = lo;
-            }
+            for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+            uint4 hi, lo;
+            split8(f, hi, lo);
+            *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, cc0 + cc)) = hi;
+            *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, cc0 + cc)) = lo;
         }
     }
-    float du_acc[32];
+    float du_acc[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) du_acc[j] = 0.f;
+    for (int j = 0; j < 16; ++j) du_acc[j] = 0.f;
 
     bool failed = false, out_of_range = false;
     int issued1 = -1, issued2 = -1;
@@ -353,14 +357,14 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         uint8_t* y_tile = s.ystage[pb];
         // the aux row (r, or k in reversed time) of this lane, read now for the output step
         const int t = row;
-        const bool live = row_lane && t < valid;
+        const bool live = t < valid;
         // this row in the caller's token order: dk's inputs are time-reversed, its outputs
         // (dk, Q) and its aux input (k) are not
         const int tok = kDk ? T - 1 - (t0 + t) : t0 + t;
-        const size_t gx = (((size_t)b * T + tok) * H + h) * 64 + 32 * hh;
-        uint4 rw[4];
+        const size_t gx = (((size_t)b * T + tok) * H + h) * 64 + cb;
+        uint4 rw[2];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
+        for (int cc = 0; cc < 2; ++cc)
             rw[cc] = live ? __ldg(reinterpret_cast<const uint4*>(r + gx + 8 * cc)) : make_uint4(0, 0, 0, 0);
         // the store that last used y_tile (chunk n-2) has read it before this chunk rewrites it
         if (!kDk && tid == 0) ptx::bulk_wait_read<1>();
@@ -369,25 +373,23 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         ptx::tc_fence_after();
         // -------------------------------------------------------- causal scores of chunk n
         {
-            uint32_t A[32];
-            ptx::tmem_ld32(tmem + tlane + COL_A + 32 * hh, A);
+            uint32_t A[16];
+            ptx::tmem_ld16x2(tmem + tlane + COL_A + 32 * hh, A);
             ptx::tmem_wait_ld();
-            if (row_lane) {
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float a[8];
+            for (int cc = 0; cc < 2; ++cc) {
+                float a[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int sx = 32 * hh + 8 * cc + e;
-                        const float x = __uint_as_float(A[8 * cc + e]);
-                        if (sx == t) s.diag[t] = x;
-                        a[e] = sx < t ? x : 0.f;
-                    }
-                    uint4 hi, lo;
-                    split8(a, hi, lo);
-                    *reinterpret_cast<uint4*>(s.a_hi + sw_chunk(t, 4 * hh + cc)) = hi;
-                    *reinterpret_cast<uint4*>(s.a_lo + sw_chunk(t, 4 * hh + cc)) = lo;
+                for (int e = 0; e < 8; ++e) {
+                    const int sx = cb + 8 * cc + e;
+                    const float x = __uint_as_float(A[8 * cc + e]);
+                    if (sx == t) s.diag[t] = x;
+                    a[e] = sx < t ? x : 0.f;
                 }
+                uint4 hi, lo;
+                split8(a, hi, lo);
+                *reinterpret_cast<uint4*>(s.a_hi + sw_chunk(t, cc0 + cc)) = hi;
+                *reinterpret_cast<uint4*>(s.a_lo + sw_chunk(t, cc0 + cc)) = lo;
             }
         }
         ptx::tc_fence_before();
@@ -413,23 +415,21 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         }
         // -------------------------------------------------------- state chain (MMA 2 running)
         {
-            uint32_t U[32];
-            ptx::tmem_ld32(tmem + tlane + COL_U + 32 * hh, U);
+            uint32_t U[16];
+            ptx::tmem_ld16x2(tmem + tlane + COL_U + 32 * hh, U);
             ptx::tmem_wait_ld();
-            if (row_lane) {
-                const float g = s.gamma[pb][row];
+            const float g = s.gamma[pb][row];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float f[8];
+            for (int cc = 0; cc < 2; ++cc) {
+                float f[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
-                    uint4 hi, lo;
-                    split8(f, hi, lo);
-                    *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, 4 * hh + cc)) = hi;
-                    *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, 4 * hh + cc)) = lo;
-                }
+                for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                uint4 hi, lo;
+                split8(f, hi, lo);
+                *reinterpret_cast<uint4*>(s.s_hi + sw_chunk(row, cc0 + cc)) = hi;
+                *reinterpret_cast<uint4*>(s.s_lo + sw_chunk(row, cc0 + cc)) = lo;
             }
         }
         // -------------------------------------------------------- prep of chunk n+1
@@ -449,26 +449,26 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         ptx::tc_fence_after();
         // -------------------------------------------------------- output of chunk n
         {
-            uint32_t Z[32], Z2[32];
-            ptx::tmem_ld32(tmem + tlane + COL_Z + 128 * pb + 32 * hh, Z);
-            ptx::tmem_ld32(tmem + tlane + COL_Z + 128 * pb + 64 + 32 * hh, Z2);
+            uint32_t Z[16], Z2[16];
+            ptx::tmem_ld16x2(tmem + tlane + COL_Z + 128 * pb + 32 * hh, Z);
+            ptx::tmem_ld16x2(tmem + tlane + COL_Z + 128 * pb + 64 + 32 * hh, Z2);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) Z[j] = __float_as_uint(__uint_as_float(Z[j]) + __uint_as_float(Z2[j]));
-            if (row_lane) {
+            for (int j = 0; j < 16; ++j) Z[j] = __float_as_uint(__uint_as_float(Z[j]) + __uint_as_float(Z2[j]));
+            {
                 const float dg = s.diag[t];
                 float* pdst = P + gx;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < 2; ++cc) {
                     float kx[8], o[8], pv[8], rv[8], dv8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(t, 4 * hh + cc)), kx);
+                    unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(t, cc0 + cc)), kx);
                     unpack8(rw[cc], rv);
                     float om[8];
                     if (kC2 && kDk)   // this token's omega (reversed-time tile, row t)
-                        unpack8(*reinterpret_cast<const uint4*>(s.in[st][3] + sw_chunk(t, 4 * hh + cc)), om);
+                        unpack8(*reinterpret_cast<const uint4*>(s.in[st][3] + sw_chunk(t, cc0 + cc)), om);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int j = 8 * cc + e, i = 32 * hh + j;
+                        const int j = 8 * cc + e, i = cb + j;
                         const float pair = s.F[pb][t][i] * __uint_as_float(Z[j]);   // minus the bonus
                         if (kC2 && kDk) {
                             // pair = dkn; dk = dkn (1 - w); Q = kn dkn = k (1 - w) dkn; D = dkn k w
@@ -485,7 +485,7 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
                         }
                     }
                     if (!kDk)
-                        *reinterpret_cast<uint4*>(y_tile + sw_chunk(t, 4 * hh + cc)) = pack8(o);
+                        *reinterpret_cast<uint4*>(y_tile + sw_chunk(t, cc0 + cc)) = pack8(o);
                     else if (live)   // dk straight to its row in token order
                         *reinterpret_cast<uint4*>(out_direct + gx + 8 * cc) = pack8(o);
                     if (live) {
@@ -536,36 +536,37 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
             fallback[bh] = 1;   // the CUDA-core scan redoes this (b,h)
         }
     } else if (kDk) {
-        if (x_final != nullptr && row_lane) {   // dS_0
-            float* dst = x_final + (size_t)bh * 4096 + row * 64 + 32 * hh;
+        if (x_final != nullptr) {   // dS_0
+            float* dst = x_final + (size_t)bh * 4096 + row * 64 + cb;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
+            for (int j = 0; j < 16; j += 4)
                 *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
         if (tid == 0) fallback[bh] = 0;
     } else {
         // E[i] = sum_j S_T[i][j] dS_T[i][j]; du[i] = sum_t r_t[i] k_t[i] (v_t . dy_t)
         float ev = 0.f;
-        if (dS_T && row_lane) {
-            const float* g = dS_T + (size_t)bh * 4096 + row * 64 + 32 * hh;
+        if (dS_T) {
+            const float* g = dS_T + (size_t)bh * 4096 + row * 64 + cb;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
+            for (int j = 0; j < 16; j += 4) {
                 const float4 x = *reinterpret_cast<const float4*>(g + j);
                 ev = fmaf(S[j], x.x, fmaf(S[j + 1], x.y, fmaf(S[j + 2], x.z, fmaf(S[j + 3], x.w, ev))));
             }
         }
-        if (row_lane) s.epart[hh][row] = ev;
-        // du: sum over the 16 row lanes of this warp, then over the 4 row quarters
+        ev += __shfl_xor_sync(0xffffffffu, ev, 16);   // the row's other 16 columns
+        if (lane < 16) s.epart[hh][row] = ev;
+        // du: sum over the 16 row lanes of each half-warp, then over the 4 row quarters
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
             float x = du_acc[j];
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
             du_acc[j] = x;
         }
-        if (lane == 0)
+        if ((lane & 15) == 0)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) s.dupart[q][32 * hh + j] = du_acc[j];
+            for (int j = 0; j < 16; ++j) s.dupart[q][cb + j] = du_acc[j];
         __syncthreads();
         if (tid < 64) {
             E[(size_t)bh * 64 + tid] = s.epart[0][tid] + s.epart[1][tid];
