@@ -40,8 +40,10 @@
 //   assemble: A from the level accumulators, hi/lo to smem;
 //   MMA 2   : Y += A_hi V + A_lo V;
 //   epilogue: Y -> bf16 -> smem -> TMA store (double-buffered).
-// An M=64 accumulator occupies TMEM lanes 16q..16q+15 of sub-partition q, so warp w reads
-// rows 16(w%4)..+15 with its lanes 0..15, columns split between warps w and w+4.
+// An M=64 accumulator occupies lanes 0..15 of TMEM sub-partition q for rows 16q..16q+15,
+// so warp w reads rows 16(w%4)..+15, columns split between warps w and w+4.  The state
+// chain and the epilogue read them with a two-half load (lanes 16..31 of the warp get the
+// same rows' next 16 columns): every lane holds a row, 16 columns; so does A's assembly.
 //
 // Every mbarrier wait is bounded (spin budget in SM cycles); on expiry the CTA records
 // an error word, drains its in-flight copies and MMAs with a second bounded wait, frees
@@ -191,31 +193,32 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
         for (int c = n0; c < n0 + kStages && c < NC; ++c) issue_load(c);
 
     // ------------------------------------------------------------ state in registers
-    // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in lanes 0..15), column half hh
+    // warp w: TMEM sub-partition q = w % 4 (rows 16q .. 16q+15 in its lanes 0..15), columns
+    // 32 hh .. 32 hh + 31.  The state and the output take a row on every lane: row
+    // 16q + (l & 15), 16 columns from cb = 32 hh + 16 (l >> 4) (the two-half TMEM load).
     const int q = warp & 3, hh = warp >> 2;
-    const bool row_lane = lane < 16;
     const int row = 16 * q + (lane & 15);          // state row i / token row t of this lane
+    const int cb = 32 * hh + 16 * (lane >> 4);     // its first state / output column
+    const int cc0 = cb >> 3;                       // its first 16-byte chunk of a tile row
     const uint32_t tlane = (uint32_t)(32 * q) << 16;
-    float S[32];
+    float S[16];
     {
-        const float* src = state0 ? state0 + row * 64 + 32 * hh : nullptr;
+        const float* src = state0 ? state0 + row * 64 + cb : nullptr;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
+        for (int j = 0; j < 16; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (src && row_lane) x = *reinterpret_cast<const float4*>(src + j);
+            if (src) x = *reinterpret_cast<const float4*>(src + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        if (row_lane) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float f[8];
+        for (int cc = 0; cc < 2; ++cc) {
+            float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
-                uint4 hi, lo;
-                split8(f, hi, lo);
-                st_shared_v4(s.s_hi, sw_chunk(row, 4 * hh + cc), hi);
-                st_shared_v4(s.s_lo, sw_chunk(row, 4 * hh + cc), lo);
-            }
+            for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+            uint4 hi, lo;
+            split8(f, hi, lo);
+            st_shared_v4(s.s_hi, sw_chunk(row, cc0 + cc), hi);
+            st_shared_v4(s.s_lo, sw_chunk(row, cc0 + cc), lo);
         }
     }
 
@@ -384,81 +387,94 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
 
         // -------------------------------------------------------- state chain
         {
-            uint32_t U[32];
-            ptx::tmem_ld32(tmem + tlane + COL_U + 32 * hh, U);
+            uint32_t U[16];
+            ptx::tmem_ld16x2(tmem + tlane + COL_U + 32 * hh, U);
             ptx::tmem_wait_ld();
-            if (row_lane) {
-                const float g = s.gamma[row];
+            const float g = s.gamma[row];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(g, S[j], __uint_as_float(U[j]));
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float f[8];
+            for (int cc = 0; cc < 2; ++cc) {
+                float f[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
-                    uint4 hi, lo;
-                    split8(f, hi, lo);
-                    st_shared_v4(s.s_hi, sw_chunk(row, 4 * hh + cc), hi);
-                    st_shared_v4(s.s_lo, sw_chunk(row, 4 * hh + cc), lo);
-                }
+                for (int e = 0; e < 8; ++e) f[e] = S[8 * cc + e];
+                uint4 hi, lo;
+                split8(f, hi, lo);
+                st_shared_v4(s.s_hi, sw_chunk(row, cc0 + cc), hi);
+                st_shared_v4(s.s_lo, sw_chunk(row, cc0 + cc), lo);
             }
         }
 
         // -------------------------------------------------------- assemble A
         {
-            const int t = row;               // token row (lanes 0..15)
+            // lane: token row t, key blocks g = gw + 2 hf (8 columns each) for gw = 4 hh + gg;
+            // the warp loads block gw, its half-warp hf = 1 receives block gw + 2.  The rows'
+            // block pair (2q, 2q+1) lies after all of the warp's 4 blocks, before all of them,
+            // or inside them (hh = q / 2): a warp-uniform choice of loads.
+            const int t = row;
             const int p = t & 7;
             const bool upper8 = (lane & 15) >= 8;  // t in block 2q+1 (else 2q)
+            const int hf = lane >> 4;
             float bonus = 0.f;
-            if (row_lane) {
 #pragma unroll
-                for (int g = 0; g < 8; ++g) bonus += s.bonus_part[g][t];
-            }
+            for (int g = 0; g < 8; ++g) bonus += s.bonus_part[g][t];
 #pragma unroll
-            for (int gg = 0; gg < 4; ++gg) {
-                const int g = 4 * hh + gg;   // key block of 8 columns
+            for (int gg = 0; gg < 2; ++gg) {
+                const int gw = 4 * hh + gg;
+                const int g = gw + 2 * hf;       // this lane's key block
                 float a[8];
-                if (g < 2 * q) {
-                    const int lvl = 3 + (31 - __clz((2 * q) ^ g));
+                if (4 * hh > 2 * q + 1) {        // every block after t's pair: no pairs
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) a[c] = 0.f;
+                } else if (4 * hh + 3 < 2 * q) {
+                    // every block before t's pair: one level, the same for both halves (gw and
+                    // gw + 2 differ in bit 1 only, below the highest bit where they leave 2q)
+                    const int lvl = 3 + (31 - __clz((2 * q) ^ gw));
                     uint32_t v[8];
-                    ptx::tmem_ld8(tmem + tlane + 64 * lvl + 8 * g, v);
+                    ptx::tmem_ld16x2_8(tmem + tlane + 64 * lvl + 8 * gw, v);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 8; ++c) a[c] = __uint_as_float(v[c]);
-                } else if (g <= 2 * q + 1) {
-                    uint32_t v0[8], v1[8], v2[8], v3[8];
-                    ptx::tmem_ld8(tmem + tlane + 0 + 8 * g, v0);
-                    ptx::tmem_ld8(tmem + tlane + 64 + 8 * g, v1);
-                    ptx::tmem_ld8(tmem + tlane + 128 + 8 * g, v2);
-                    ptx::tmem_ld8(tmem + tlane + 192 + 8 * g, v3);
-                    ptx::tmem_wait_ld();
-                    const bool diag = (g == 2 * q) ? !upper8 : upper8;  // s in t's own 8-block
-                    const bool below = (g == 2 * q) && upper8;           // whole block before t
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float x = 0.f;
-                        if (below) {
-                            x = __uint_as_float(v3[c]);
-                        } else if (diag) {
-                            if (c == p) {
-                                x = bonus;
-                            } else if (c < p) {
-                                const int lvl = 31 - __clz(p ^ c);
-                                x = __uint_as_float(lvl == 0 ? v0[c] : (lvl == 1 ? v1[c] : v2[c]));
-                            }
-                        }
-                        a[c] = x;
-                    }
                 } else {
+                    // t's pair among the warp's blocks: levels 0-3 for the pair's own blocks
+                    // and level 4 for a block before it (q odd: half-warp 0's blocks)
+                    uint32_t v0[8], v1[8], v2[8], v3[8], v4[8];
+                    ptx::tmem_ld16x2_8(tmem + tlane + 0 + 8 * gw, v0);
+                    ptx::tmem_ld16x2_8(tmem + tlane + 64 + 8 * gw, v1);
+                    ptx::tmem_ld16x2_8(tmem + tlane + 128 + 8 * gw, v2);
+                    ptx::tmem_ld16x2_8(tmem + tlane + 192 + 8 * gw, v3);
+                    ptx::tmem_ld16x2_8(tmem + tlane + 256 + 8 * gw, v4);
+                    ptx::tmem_wait_ld();
+                    if (g < 2 * q) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) a[c] = 0.f;
+                        for (int c = 0; c < 8; ++c) a[c] = __uint_as_float(v4[c]);
+                    } else if (g <= 2 * q + 1) {
+                        const bool diag = (g == 2 * q) ? !upper8 : upper8;  // s in t's own 8-block
+                        const bool below = (g == 2 * q) && upper8;           // whole block before t
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float x = 0.f;
+                            if (below) {
+                                x = __uint_as_float(v3[c]);
+                            } else if (diag) {
+                                if (c == p) {
+                                    x = bonus;
+                                } else if (c < p) {
+                                    const int lvl = 31 - __clz(p ^ c);
+                                    x = __uint_as_float(lvl == 0 ? v0[c] : (lvl == 1 ? v1[c] : v2[c]));
+                                }
+                            }
+                            a[c] = x;
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) a[c] = 0.f;
+                    }
                 }
-                if (row_lane) {
-                    uint4 hi, lo;
-                    split8(a, hi, lo);
-                    st_shared_v4(s.q[0], sw_chunk(t, g), hi);
-                    st_shared_v4(s.q[1], sw_chunk(t, g), lo);
-                }
+                uint4 hi, lo;
+                split8(a, hi, lo);
+                st_shared_v4(s.q[0], sw_chunk(t, g), hi);
+                st_shared_v4(s.q[1], sw_chunk(t, g), lo);
             }
         }
         ptx::tc_fence_before();
@@ -487,13 +503,13 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
 
         // -------------------------------------------------------- epilogue
         {
-            uint32_t Y[32];
-            ptx::tmem_ld32(tmem + tlane + COL_Y + 32 * hh, Y);
+            uint32_t Y[16];
+            ptx::tmem_ld16x2(tmem + tlane + COL_Y + 32 * hh, Y);
             ptx::tmem_wait_ld();
-            if (kC2 && row_lane && row < valid) {   // the second value u'_t joins the readout
-                const __nv_bfloat16* up = uprime + (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
+            if (kC2 && row < valid) {   // the second value u'_t joins the readout
+                const __nv_bfloat16* up = uprime + (((size_t)b * T + t0 + row) * H + h) * 64 + cb;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < 2; ++cc) {
                     float f[8];
                     unpack8(*reinterpret_cast<const uint4*>(up + 8 * cc), f);
 #pragma unroll
@@ -502,34 +518,35 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             }
             if (kGN) {
                 // base Finch's output stage: GroupNorm of the (token, head) row over its 64
-                // channels (this lane's 32, then the other half's from the partner warp),
-                // the head's affine, times the gate
-                float2 mo = make_float2(0.f, 0.f);
-                if (row_lane) {
-                    float sm = 0.f;
+                // channels (this lane's 16, the other half-warp's 16 by a shuffle, then the
+                // other 32 from the partner warp), the head's affine, times the gate
+                float sm = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) sm += __uint_as_float(Y[j]);
-                    const float mean = sm * (1.f / 32.f);
-                    float q2 = 0.f;
+                for (int j = 0; j < 16; ++j) sm += __uint_as_float(Y[j]);
+                const float mean16 = sm * (1.f / 16.f);
+                float q16 = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float d = __uint_as_float(Y[j]) - mean;
-                        q2 = fmaf(d, d, q2);
-                    }
-                    mo = make_float2(mean, q2);
-                    s.gn_mom[hh][row] = mo;
+                for (int j = 0; j < 16; ++j) {
+                    const float d = __uint_as_float(Y[j]) - mean16;
+                    q16 = fmaf(d, d, q16);
                 }
+                // merge two 16-value parts: (mean, M2) of the 32 columns, the same on both lanes
+                const float om16 = __shfl_xor_sync(0xffffffffu, mean16, 16);
+                const float oq16 = __shfl_xor_sync(0xffffffffu, q16, 16);
+                const float d16 = om16 - mean16;
+                const float2 mo = make_float2(0.5f * (mean16 + om16), q16 + oq16 + 8.f * d16 * d16);
+                if (lane < 16) s.gn_mom[hh][row] = mo;
                 __syncthreads();
-                if (row_lane) {
+                {
                     const float2 ot = s.gn_mom[hh ^ 1][row];
                     const float d = ot.x - mo.x;
                     const float mean = 0.5f * (mo.x + ot.x);
                     const float inv = rsqrtf((mo.y + ot.y + 16.f * d * d) * (1.f / 64.f) + gn.eps);
-                    const int c0 = h * 64 + 32 * hh;
+                    const int c0 = h * 64 + cb;
                     const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(gn.gate);
-                    const size_t gbase = (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
+                    const size_t gbase = (((size_t)b * T + t0 + row) * H + h) * 64 + cb;
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < 2; ++cc) {
                         float gt[8];
                         if (gp != nullptr && row < valid) {
                             unpack8(__ldg(reinterpret_cast<const uint4*>(gp + gbase + 8 * cc)), gt);
@@ -544,26 +561,26 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                             f[e] = fmaf((__uint_as_float(Y[j]) - mean) * inv, __ldg(gn.gamma + c0 + j),
                                         __ldg(gn.beta + c0 + j)) * gt[e];
                         }
-                        st_shared_v4(y_tile, sw_chunk(row, 4 * hh + cc), pack8(f));
+                        st_shared_v4(y_tile, sw_chunk(row, cc0 + cc), pack8(f));
                     }
                 }
-            } else if (row_lane && y_raw != nullptr) {
-                // fp32 rows for the LayerNorm pass: 128 contiguous bytes per lane
+            } else if (y_raw != nullptr) {
+                // fp32 rows for the LayerNorm pass: 64 contiguous bytes per lane
                 if (row < valid) {
-                    float* dst = y_raw + (((size_t)b * T + t0 + row) * H + h) * 64 + 32 * hh;
+                    float* dst = y_raw + (((size_t)b * T + t0 + row) * H + h) * 64 + cb;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
+                    for (int j = 0; j < 16; j += 4)
                         *reinterpret_cast<float4*>(dst + j) =
                             make_float4(__uint_as_float(Y[j]), __uint_as_float(Y[j + 1]),
                                         __uint_as_float(Y[j + 2]), __uint_as_float(Y[j + 3]));
                 }
-            } else if (row_lane) {
+            } else {
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < 2; ++cc) {
                     float f[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(Y[8 * cc + e]);
-                    st_shared_v4(y_tile, sw_chunk(row, 4 * hh + cc), pack8(f));
+                    st_shared_v4(y_tile, sw_chunk(row, cc0 + cc), pack8(f));
                 }
             }
         }
@@ -595,10 +612,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)((n - n0) & 1), drain_budget);
             if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)((n - n0) & 1), drain_budget);
         }
-    } else if (s_out != nullptr && row_lane) {
-        float* dst = s_out + (size_t)bh * 4096 + row * 64 + 32 * hh;
+    } else if (s_out != nullptr) {
+        float* dst = s_out + (size_t)bh * 4096 + row * 64 + cb;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
+        for (int j = 0; j < 16; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     if (tid == 0) ptx::bulk_wait<0>();
