@@ -35,8 +35,10 @@
 //   TMA loads of r, k, v, omega run two chunks ahead (2-stage ring, mbarrier tx-count);
 //   prep    : warp = 8 channels, lane = 2 tokens; w, block products (shuffle butterfly),
 //             operands Q^1..5, K^1..5, Rt, Kt^T written to 128B-swizzled smem;
-//   MMA 1   : L^0..L^5, U = Kt^T V, Y = Rt S_hi + Rt S_lo (thread 0 issues, commit);
-//   state   : S <- gamma S + U in registers; S_hi/S_lo for the next chunk;
+//   MMA 1   : U = Kt^T V, Y = Rt S_hi + Rt S_lo (thread 0 issues, commit), then L^0..L^5
+//             (commit);
+//   state   : S <- gamma S + U in registers; S_hi/S_lo for the next chunk (once U and Y are
+//             done, while the level products run);
 //   assemble: A from the level accumulators, hi/lo to smem;
 //   MMA 2   : Y += A_hi V + A_lo V;
 //   epilogue: Y -> bf16 -> smem -> TMA store (double-buffered).
@@ -83,7 +85,7 @@ struct __align__(1024) Smem {
     float gamma[64];
     float bonus_part[8][64];         // per channel group partial of sum_i r u k
     uint64_t full[kStages];
-    uint64_t mma1, mma2;
+    uint64_t mma1u, mma1, mma2;   // MMA 1's U and Y products; all of MMA 1; MMA 2
     uint32_t tmem_base;
     int abort;
     float2 gn_mom[2][64];            // GroupNorm stage: (mean, M2) of each row's two halves
@@ -159,6 +161,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) ptx::mbar_init(&s.full[i], 1);
+        ptx::mbar_init(&s.mma1u, 1);
         ptx::mbar_init(&s.mma1, 1);
         ptx::mbar_init(&s.mma2, 1);
         ptx::fence_mbar_init();
@@ -349,21 +352,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
         if (s.abort) { failed = true; break; }
 
         // -------------------------------------------------------- MMA 1
+        // U and Y first, with a commit of their own: the state chain needs only U, and may
+        // rewrite S_hi / S_lo once Y has read them, while the level products still run
         if (tid == 0) {
             ptx::tc_fence_after();
-            const uint32_t a_r = ptx::smem_addr(r_tile), b_k = ptx::smem_addr(k_tile);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq)
-                ptx::mma_bf16(tmem + COL_L0, ptx::desc_kmajor(a_r + 32 * kq),
-                              ptx::desc_kmajor(b_k + 32 * kq), IDESC_KK, kq > 0);
-#pragma unroll
-            for (int l = 1; l <= 5; ++l) {
-                const uint32_t a = ptx::smem_addr(s.q[l - 1]), bb = ptx::smem_addr(s.kk[l - 1]);
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq)
-                    ptx::mma_bf16(tmem + 64 * l, ptx::desc_kmajor(a + 32 * kq),
-                                  ptx::desc_kmajor(bb + 32 * kq), IDESC_KK, kq > 0);
-            }
             const uint32_t a_kt = ptx::smem_addr(s.ktT), b_v = ptx::smem_addr(v_tile);
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
@@ -379,10 +371,24 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             for (int kq = 0; kq < 4; ++kq)
                 ptx::mma_bf16(tmem + COL_Y, ptx::desc_kmajor(a_rt + 32 * kq),
                               ptx::desc_mnmajor(b_lo + 2048 * kq), IDESC_KM, 1);
+            ptx::mma_commit(&s.mma1u);
+            const uint32_t a_r = ptx::smem_addr(r_tile), b_k = ptx::smem_addr(k_tile);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                ptx::mma_bf16(tmem + COL_L0, ptx::desc_kmajor(a_r + 32 * kq),
+                              ptx::desc_kmajor(b_k + 32 * kq), IDESC_KK, kq > 0);
+#pragma unroll
+            for (int l = 1; l <= 5; ++l) {
+                const uint32_t a = ptx::smem_addr(s.q[l - 1]), bb = ptx::smem_addr(s.kk[l - 1]);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)
+                    ptx::mma_bf16(tmem + 64 * l, ptx::desc_kmajor(a + 32 * kq),
+                                  ptx::desc_kmajor(bb + 32 * kq), IDESC_KK, kq > 0);
+            }
             ptx::mma_commit(&s.mma1);
             issued1 = n;
         }
-        if (!ptx::mbar_wait(&s.mma1, (uint32_t)(m & 1), spin_budget)) s.abort = 1;
+        if (!ptx::mbar_wait(&s.mma1u, (uint32_t)(m & 1), spin_budget)) s.abort = 1;
         ptx::tc_fence_after();
 
         // -------------------------------------------------------- state chain
@@ -404,6 +410,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                 st_shared_v4(s.s_lo, sw_chunk(row, cc0 + cc), lo);
             }
         }
+
+        if (!ptx::mbar_wait(&s.mma1, (uint32_t)(m & 1), spin_budget)) s.abort = 1;
+        ptx::tc_fence_after();
 
         // -------------------------------------------------------- assemble A
         {
