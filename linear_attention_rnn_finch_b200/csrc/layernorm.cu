@@ -2,9 +2,9 @@
 // per-head GroupNorm of Finch with one LayerNorm across the full concatenated width;
 // GoldFinch review page, section 3.4 "Finch-C2 Time Mixing", output equation):
 //     out = (x - mean) / sqrt(var + eps) * gamma + beta,   var = biased variance.
-// Used as the second pass after a recurrence kernel has written fp32 rows; one CTA per
-// row, exact two-pass mean / variance from the fp32 values (held in registers when the row
-// has at most 8192 channels).  Base Finch's per-head GroupNorm + gate lives here too.
+// Used as the second pass after a recurrence kernel has written fp32 rows: a warp per row
+// for rows of 512-2048 channels, else one CTA per row; exact two-pass mean / variance from
+// the fp32 values (held in registers when the row has at most 8192 channels).  Base Finch's per-head GroupNorm + gate lives here too.
 #include "common.cuh"
 #include "internal.h"
 
@@ -100,6 +100,71 @@ layernorm_rows_vec_kernel(const float* x, const float* __restrict__ gamma,
             store8(orow + 8 * ch, v[m]);
         }
     }
+}
+
+// Rows of C = 128 * kV4 channels (at most 2048), one warp per row: lane l holds the row's
+// 16-byte pieces l, l + 32, ... in registers, so the row is read from memory once and both
+// moments are warp reductions (no block barrier between the steps of a row).  The CTAs are
+// persistent, 8 rows at a time, and stage gamma and beta in shared memory once.
+__device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    *reinterpret_cast<uint2*>(p) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+}
+
+constexpr int kRowsPerCta = kThreads / 32;
+
+template <typename IO, int kV4>
+__global__ void __launch_bounds__(kThreads)
+layernorm_rows_warp_kernel(const float* x, const float* __restrict__ gamma,
+                           const float* __restrict__ beta, float eps, IO* out, long rows) {
+    constexpr int C = 128 * kV4;
+    __shared__ float4 g4[C / 4], b4[C / 4];
+    for (int i = threadIdx.x; i < C / 4; i += kThreads) {
+        g4[i] = reinterpret_cast<const float4*>(gamma)[i];
+        b4[i] = reinterpret_cast<const float4*>(beta)[i];
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (long r = (long)blockIdx.x * kRowsPerCta + warp; r < rows;
+         r += (long)gridDim.x * kRowsPerCta) {
+        const float4* row = reinterpret_cast<const float4*>(x + r * C);
+        float4 v[kV4];
+#pragma unroll
+        for (int m = 0; m < kV4; ++m) v[m] = row[lane + 32 * m];
+        float sm = 0.f;
+#pragma unroll
+        for (int m = 0; m < kV4; ++m) sm += (v[m].x + v[m].y) + (v[m].z + v[m].w);
+        const float mean = warp_sum(sm) * (1.f / (float)C);
+        float q = 0.f;
+#pragma unroll
+        for (int m = 0; m < kV4; ++m) {
+            v[m].x -= mean; v[m].y -= mean; v[m].z -= mean; v[m].w -= mean;
+            q = fmaf(v[m].x, v[m].x, fmaf(v[m].y, v[m].y, fmaf(v[m].z, v[m].z, fmaf(v[m].w, v[m].w, q))));
+        }
+        const float inv = rsqrtf(warp_sum(q) * (1.f / (float)C) + eps);
+        // x and out may alias (fp32 in place): this warp read the whole row above
+        IO* orow = out + r * C;
+#pragma unroll
+        for (int m = 0; m < kV4; ++m) {
+            const int i = lane + 32 * m;
+            const float4 g = g4[i], b = b4[i];
+            store4(orow + 4 * i, fmaf(v[m].x * inv, g.x, b.x), fmaf(v[m].y * inv, g.y, b.y),
+                   fmaf(v[m].z * inv, g.z, b.z), fmaf(v[m].w * inv, g.w, b.w));
+        }
+    }
+}
+
+template <typename IO, int kV4>
+cudaError_t launch_ln_warp(const float* x, const float* gamma, const float* beta, float eps,
+                           IO* out, long rows, cudaStream_t st) {
+    const long need = (rows + kRowsPerCta - 1) / kRowsPerCta;
+    const unsigned grid = (unsigned)(need < 148L * 8 ? need : 148L * 8);
+    layernorm_rows_warp_kernel<IO, kV4><<<grid, kThreads, 0, st>>>(x, gamma, beta, eps, out, rows);
+    return cudaGetLastError();
 }
 
 template <typename IO>
@@ -199,6 +264,19 @@ cudaError_t launch_layernorm_rows(const float* x, const float* gamma, const floa
                                   float eps, void* out, long rows, int C, bool bf16,
                                   cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
+    // rows of 512, 1024 or 2048 channels (H = 8, 16, 32): a warp per row
+    if (C == 512 || C == 1024 || C == 2048) {
+        if (bf16) {
+            auto* o = (__nv_bfloat16*)out;
+            if (C == 512) return launch_ln_warp<__nv_bfloat16, 4>(x, gamma, beta, eps, o, rows, st);
+            if (C == 1024) return launch_ln_warp<__nv_bfloat16, 8>(x, gamma, beta, eps, o, rows, st);
+            return launch_ln_warp<__nv_bfloat16, 16>(x, gamma, beta, eps, o, rows, st);
+        }
+        auto* o = (float*)out;
+        if (C == 512) return launch_ln_warp<float, 4>(x, gamma, beta, eps, o, rows, st);
+        if (C == 1024) return launch_ln_warp<float, 8>(x, gamma, beta, eps, o, rows, st);
+        return launch_ln_warp<float, 16>(x, gamma, beta, eps, o, rows, st);
+    }
     // C = H * 64: whole 8-value chunks; rows of up to 8192 channels stay in registers
     const int per = (C / 8 + kThreads - 1) / kThreads;
     const unsigned grid = (unsigned)rows;
