@@ -354,10 +354,11 @@ def backward_line(cfg, dev, world, steps, c2=False):
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
     flops, nbytes = backward_flops(B, T, H, D), backward_bytes(B, T, H, D)
     # base form: 2 reversals + fast + level kernels for dv (+ 2 segment kernels when the
-    # sequence is split), the tensor-core dr and dk readouts, the two decay-gradient kernels,
-    # the dr and dk scans (which exit at once unless a (b,h) fell back) and the du sum.
+    # sequence is split), the tensor-core dr and dk readouts, the decay gradient's two
+    # column-sum kernels and its scan, the dr and dk scans (which exit at once unless a
+    # (b,h) fell back) and the du sum.
     # (Finch-C2: the same launches; its dv prefill forms the query k (1 - w) inside)
-    launches_per_call = 11
+    launches_per_call = 12
     line = {"workload": ("wkv6c2_backward" if c2 else "wkv6_backward") + f" B{B} T{T} H{H}",
             "B": B, "T": T, "H": H, "D": D, "io": "bf16", "steps": steps, "ms_per_call": ms,
             "value": world * B * T / (ms / 1e3), "unit": "tokens/s",
@@ -375,7 +376,7 @@ def backward_line(cfg, dev, world, steps, c2=False):
                         "CUDA-core scans run only for a (b,h) that falls back") if c2 else
                        ("dr and dk as chunked tensor-core readouts of the forward and the "
                         "reversed state (wkv6_bwd_readout_tc_kernel x2), the decay gradient from "
-                        "their pair terms (wkv6_bwd_pq_sums_kernel, wkv6_bwd_domega_kernel), dv "
+                        "their pair terms (wkv6_bwd_col_sums_kernel x2, wkv6_bwd_domega_kernel), dv "
                         "through the chunked tensor-core prefill on time-reversed copies "
                         "(reverse_tokens_kernel x2, wkv6_fast_kernel, wkv6_chunked_kernel); the "
                         "CUDA-core scans run only for a (b,h) whose decays the one-sided factors "

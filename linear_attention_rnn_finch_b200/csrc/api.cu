@@ -870,7 +870,8 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     // side stream, dr on the other, queued in that order (a readout's CTAs outlast the
     // prefill's two to one: long ones first).  Each pass is 256 CTAs of one SM apiece, so
     // alone it leaves SMs idle in its last wave; side by side, the other passes' CTAs take
-    // them.  The decay gradient, after the join, needs P and E of dr and Q of dk.
+    // them.  The chunk sums of Q and of P follow dk and dr on their streams; the rest of the
+    // decay gradient, after the join, needs P, E and Q.
     Fork fork(st);
     if (!fork.ok()) return WKV_ERR_CUDA;
     CUtensorMap maps[5];
@@ -884,7 +885,8 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         !goldwkv::make_token_map(&maps[4], dk, B, T, H))
         return WKV_ERR_CUDA;
     if (goldwkv::launch_bwd_dk_tc(maps, k, ub, dstate_out, dk, q_tok, d_tok, dstate_in, dk_flags, B,
-                                  T, H, status, budget, st, c2) != cudaSuccess)
+                                  T, H, status, budget, st, c2) != cudaSuccess ||
+        goldwkv::launch_bwd_col_sums(q_tok, sums, 1, B, T, H, st) != cudaSuccess)
         return WKV_ERR_CUDA;
     {
         // dv (and, unused, dS0) is the forward recurrence in reversed time with k and r
@@ -920,7 +922,9 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     if (goldwkv::launch_backward(r, k, v, omega, ub, state_in, dy, dstate_out, dr, dk, dv, domega,
                                  du, dstate_in, P, E, du_part, B, T, H, bf16, /*with_dv=*/false,
                                  c2, fork.side(1), dr_flags, nullptr, goldwkv::kPhaseDr) !=
-        cudaSuccess)
+            cudaSuccess ||
+        goldwkv::launch_bwd_col_sums(static_cast<const float*>(P), sums, 0, B, T, H,
+                                     fork.side(1)) != cudaSuccess)
         return WKV_ERR_CUDA;
     if (!fork.join()) return WKV_ERR_CUDA;
     if (goldwkv::launch_bwd_domega(static_cast<const float*>(P), q_tok, d_tok, sums,

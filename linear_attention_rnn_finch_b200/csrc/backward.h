@@ -49,13 +49,18 @@ cudaError_t launch_bwd_dk_tc(const CUtensorMap* maps, const void* k, const float
                              int* fallback, int B, int T, int H, int* status, long long budget,
                              cudaStream_t st, bool c2 = false);
 
-// domega (bf16) from P, Q (token order) and E through the identity
+// The column sums of X (P for half 0, Q for half 1; [B][T][H][64] fp32, token order) over
+// each 64-token chunk into sums, B*H*ceil(T/64)*128 floats: sums[bh][n][64 * half + i].
+cudaError_t launch_bwd_col_sums(const float* X, float* sums, int half, int B, int T, int H,
+                                cudaStream_t st);
+
+// domega (bf16) from P, Q (token order), their chunk sums (both halves) and E through the
+// identity
 //     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s - D_t,  domega_t = dlog w_t (-exp(omega_t));
-// D: Finch-C2's direct term, or null (zero).  sums: scratch of B*H*ceil(T/64)*128 floats.
-cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, float* sums,
-                              const float* E,
-                              const void* omega, void* domega, int B, int T, int H,
-                              cudaStream_t st);
+// D: Finch-C2's direct term, or null (zero).
+cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, const float* sums,
+                              const float* E, const void* omega, void* domega, int B, int T,
+                              int H, cudaStream_t st);
 
 constexpr int kMaxReverse = 5;
 

@@ -622,16 +622,19 @@ namespace {
 
 // Decay gradient from the pair terms (the identity of csrc/backward.cu):
 //     dlog w_t = E + sum_{s>t} P_s - sum_{s>=t} Q_s,   domega_t = dlog w_t (-exp(omega_t)),
-// P and Q in token order.  First the column sums of P and Q over each 64-token chunk, then
-// per chunk the sums over the later chunks and a reverse scan over its own tokens.  One
-// thread per channel and chunk, kDomegaChunks chunks of one (b,h) per CTA.  (One CTA per
-// (b,h) walking its chunks backwards with a running total reads P and Q once instead of
-// twice, but at 256 CTAs each chunk's loads wait in line: it measured slower.)
+// P and Q in token order.  First the column sums of P and of Q over each 64-token chunk (a
+// launch each, queued right after the pass that writes the array, so that it runs beside
+// the other pass), then per chunk the sums over the later chunks and a reverse scan over
+// its own tokens.  One thread per channel and chunk, kDomegaChunks chunks of one (b,h) per
+// CTA.  (One CTA per (b,h) walking its chunks backwards with a running total reads P and Q
+// once instead of twice, but at 256 CTAs each chunk's loads wait in line: it measured
+// slower.)
 constexpr int kDomegaChunks = 4;
 
+// sums[bh][n][64 * half + i] = sum over chunk n's tokens of X[t][i]
 __global__ void __launch_bounds__(64 * kDomegaChunks)
-wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q,
-                        float* __restrict__ sums, int T, int H) {
+wkv6_bwd_col_sums_kernel(const float* __restrict__ X, float* __restrict__ sums, int half, int T,
+                         int H) {
     const int NC = (T + C - 1) / C, groups = (NC + kDomegaChunks - 1) / kDomegaChunks;
     const int g = blockIdx.x % groups, bh = blockIdx.x / groups, b = bh / H, h = bh - b * H;
     const int n = g * kDomegaChunks + (threadIdx.x >> 6), i = threadIdx.x & 63;
@@ -639,19 +642,14 @@ wkv6_bwd_pq_sums_kernel(const float* __restrict__ P, const float* __restrict__ Q
     const int t0 = n * C, valid = min(C, T - t0);
     const size_t stride = (size_t)H * 64, x0 = (((size_t)b * T + t0) * H + h) * 64 + i;
     // four partial sums: the loads of 8 tokens in flight, not one add chain
-    float sp[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
+    float sx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-    for (int tt = 0; tt < valid; ++tt) {
-        sp[tt & 3] += P[x0 + tt * stride];
-        sq[tt & 3] += Q[x0 + tt * stride];
-    }
-    float* o = sums + ((size_t)bh * NC + n) * 128;
-    o[i] = (sp[0] + sp[1]) + (sp[2] + sp[3]);
-    o[64 + i] = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+    for (int tt = 0; tt < valid; ++tt) sx[tt & 3] += X[x0 + tt * stride];
+    sums[((size_t)bh * NC + n) * 128 + 64 * half + i] = (sx[0] + sx[1]) + (sx[2] + sx[3]);
 }
 
-// CTAs run in the reverse of the sums kernel's order, so the first of them find the P and Q
-// that kernel read last still in L2.
+// CTAs run from the last (b,h) to the first: the first of them find the P and Q the sums
+// kernels read last still in L2.
 __global__ void __launch_bounds__(64 * kDomegaChunks)
 wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
                        const float* __restrict__ Dw, const float* __restrict__ sums,
@@ -685,16 +683,21 @@ wkv6_bwd_domega_kernel(const float* __restrict__ P, const float* __restrict__ Q,
 
 }  // namespace
 
-cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, float* sums,
-                              const float* E,
-                              const void* omega, void* domega, int B, int T, int H,
-                              cudaStream_t st) {
+cudaError_t launch_bwd_col_sums(const float* X, float* sums, int half, int B, int T, int H,
+                                cudaStream_t st) {
     const long groups = ((T + C - 1) / C + kDomegaChunks - 1) / kDomegaChunks;
     const unsigned blocks = (unsigned)((long)B * H * groups);
     if (blocks == 0) return cudaSuccess;
-    wkv6_bwd_pq_sums_kernel<<<blocks, 64 * kDomegaChunks, 0, st>>>(P, Q, sums, T, H);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    wkv6_bwd_col_sums_kernel<<<blocks, 64 * kDomegaChunks, 0, st>>>(X, sums, half, T, H);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_domega(const float* P, const float* Q, const float* D, const float* sums,
+                              const float* E, const void* omega, void* domega, int B, int T,
+                              int H, cudaStream_t st) {
+    const long groups = ((T + C - 1) / C + kDomegaChunks - 1) / kDomegaChunks;
+    const unsigned blocks = (unsigned)((long)B * H * groups);
+    if (blocks == 0) return cudaSuccess;
     wkv6_bwd_domega_kernel<<<blocks, 64 * kDomegaChunks, 0, st>>>(P, Q, D, sums, E,
                                                   static_cast<const __nv_bfloat16*>(omega),
                                                   static_cast<__nv_bfloat16*>(domega), T, H);
