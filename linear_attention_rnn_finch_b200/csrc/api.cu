@@ -241,6 +241,15 @@ class Fork {
     ~Fork() { (void)join(); }
     bool ok() const { return ok_; }
     cudaStream_t side(int i) const { return sd_ != nullptr ? sd_->s[i] : st_; }
+    // work queued on side(i) from now on also runs after everything queued on st so far
+    bool sync(int i) {
+        if (sd_ == nullptr || !ok_) return ok_;
+        std::lock_guard<std::mutex> lock(g_side_mutex);
+        if (cudaEventRecord(sd_->fork, st_) != cudaSuccess ||
+            cudaStreamWaitEvent(sd_->s[i], sd_->fork, 0) != cudaSuccess)
+            ok_ = false;
+        return ok_;
+    }
     bool join() {
         if (sd_ == nullptr || joined_) return ok_;
         joined_ = true;
@@ -859,21 +868,23 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
                             round256((size_t)B * H * ((T + kChunk - 1) / kChunk) * 128 * sizeof(float)))
                       : nullptr;
     const long long budget = injected("timeout0") ? 0 : kSpinBudget;
+    // The passes: dk on st, dv (the prefill on the reversed copies, then its reversal) on one
+    // side stream, dr on the other, queued in that order after the reversal of the inputs (a
+    // readout's CTAs outlast the prefill's two to one: long ones first).  dr reads no
+    // reversed copy, so its stream waits only for the call's start; dv's waits for the
+    // reversal.  Each pass is 256 CTAs of one SM apiece, so alone it leaves SMs idle in its
+    // last wave; side by side, the other passes' CTAs take them.  The chunk sums of Q and of
+    // P follow dk and dr on their streams; the rest of the decay gradient, after the join,
+    // needs P, E and Q.
+    Fork fork(st);
+    if (!fork.ok()) return WKV_ERR_CUDA;
     {
         const void* src[5] = {r, dy, omega, v, k};
         void* dst[5] = {rr, rdy, rom, rv, rk};
         if (goldwkv::launch_reverse_tokens(src, dst, 5, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
-    // The three passes after the reversal need only its copies and the inputs, and share no
-    // buffer: dk on st, dv (the prefill on the reversed copies, then its reversal) on one
-    // side stream, dr on the other, queued in that order (a readout's CTAs outlast the
-    // prefill's two to one: long ones first).  Each pass is 256 CTAs of one SM apiece, so
-    // alone it leaves SMs idle in its last wave; side by side, the other passes' CTAs take
-    // them.  The chunk sums of Q and of P follow dk and dr on their streams; the rest of the
-    // decay gradient, after the join, needs P, E and Q.
-    Fork fork(st);
-    if (!fork.ok()) return WKV_ERR_CUDA;
+    if (!fork.sync(0)) return WKV_ERR_CUDA;
     CUtensorMap maps[5];
     // dk (and dS0, Q) as the readout of the forward state's adjoint in reversed time: query
     // v, key r, value dy; dk and Q go straight to token order (the fifth map, the dr pass's
