@@ -871,11 +871,11 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
     // The passes: dk on st, dv (the prefill on the reversed copies, then its reversal) on one
     // side stream, dr on the other, queued in that order after the reversal of the inputs (a
     // readout's CTAs outlast the prefill's two to one: long ones first).  dr reads no
-    // reversed copy, so its stream waits only for the call's start; dv's waits for the
-    // reversal.  Each pass is 256 CTAs of one SM apiece, so alone it leaves SMs idle in its
-    // last wave; side by side, the other passes' CTAs take them.  The chunk sums of Q and of
-    // P follow dk and dr on their streams; the rest of the decay gradient, after the join,
-    // needs P, E and Q.
+    // reversed copy, so its stream waits only for the call's start (base form); dv's waits
+    // for the reversal.  Each pass is 256 CTAs of one SM apiece, so alone it leaves SMs idle
+    // in its last wave; side by side, the other passes' CTAs take them.  The chunk sums of Q
+    // and of P follow dk and dr on their streams; the rest of the decay gradient, after the
+    // join, needs P, E and Q.
     Fork fork(st);
     if (!fork.ok()) return WKV_ERR_CUDA;
     {
@@ -884,7 +884,10 @@ wkv_status backward_impl(const void* r, const void* k, const void* v, const void
         if (goldwkv::launch_reverse_tokens(src, dst, 5, B, T, H, st) != cudaSuccess)
             return WKV_ERR_CUDA;
     }
-    if (!fork.sync(0)) return WKV_ERR_CUDA;
+    // (Finch-C2: dr waits for the reversal too.  Its dk readout's CTAs run longer, and with
+    // dr started early the chain dk -> decay gradient ended later: 2.105 against 2.087 ms at
+    // the 1.5B-layer shape, where the base form gains 1.669 -> 1.647 ms from the early start.)
+    if (!fork.sync(0) || (c2 && !fork.sync(1))) return WKV_ERR_CUDA;
     CUtensorMap maps[5];
     // dk (and dS0, Q) as the readout of the forward state's adjoint in reversed time: query
     // v, key r, value dy; dk and Q go straight to token order (the fifth map, the dr pass's
