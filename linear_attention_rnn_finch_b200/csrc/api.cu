@@ -176,6 +176,7 @@ int sm_count() {
 // (each join then follows that call's own work on its side stream: a stream runs in order).
 constexpr int kSideStreams = 2;
 struct SideStreams {
+    CUcontext ctx = nullptr;   // context the streams and events were made in
     cudaStream_t s[kSideStreams] = {};
     cudaEvent_t fork = nullptr;
     cudaEvent_t join[kSideStreams] = {};
@@ -195,7 +196,9 @@ void destroy_side(SideStreams& n) {
 // The current device's side streams (created on first use, under g_side_mutex), or null: no
 // device, or creation failed, or st is being captured into a graph and the streams do not
 // exist yet (creating them then could invalidate the capture) -- the caller then queues
-// everything on st, in order.
+// everything on st, in order.  They are made again when the current context is not the one
+// they were made in (a device reset makes a new primary context; the old handles died with
+// the old one and are dropped, not destroyed).
 const SideStreams* side_streams_locked(cudaStream_t st) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) {
@@ -203,7 +206,8 @@ const SideStreams* side_streams_locked(cudaStream_t st) {
         return nullptr;
     }
     SideStreams& sd = g_side[dev];
-    if (sd.s[0] != nullptr) return &sd;
+    const CUcontext ctx = goldwkv::current_context();
+    if (sd.s[0] != nullptr && (ctx == nullptr || ctx == sd.ctx)) return &sd;
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
         (void)cudaGetLastError();
@@ -219,6 +223,7 @@ const SideStreams* side_streams_locked(cudaStream_t st) {
         destroy_side(n);
         return nullptr;
     }
+    n.ctx = goldwkv::current_context();   // current now, whether or not it was before
     sd = n;
     return &sd;
 }

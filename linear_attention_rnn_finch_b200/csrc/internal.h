@@ -139,4 +139,8 @@ wkv_status prefill_within(const void* r, const void* k, const void* v, const voi
                           int B, int T, int H, int D, wkv_dtype io, const wkv_ln* ln,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+// The calling thread's current CUDA context, or null (none yet, or the driver entry point
+// could not be had).  Makes no context current and does not synchronise.
+CUcontext current_context();
+
 }  // namespace goldwkv

@@ -73,6 +73,17 @@ void* scratch_for_current_device() {
 
 }  // namespace
 
+namespace goldwkv {
+
+CUcontext current_context() {
+    CUcontext ctx = nullptr;
+    CtxGetCurrent get = ctx_get_current();
+    if (get == nullptr || get(&ctx) != CUDA_SUCCESS) return nullptr;
+    return ctx;
+}
+
+}  // namespace goldwkv
+
 extern "C" wkv_status wkv6_prefill_static(const void* r, const void* k, const void* v,
                                           const void* omega, const float* u,
                                           const float* state_in, float* state_out, void* y,
