@@ -274,27 +274,33 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
             Lx[1][c] = Lt[0][c];
             Lx[0][c] = Lt[0][c] - lw[0][c];
         }
+        float khf[2][8];   // Kh in fp32, kept for Kt below
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
-            float kh[8], f[8];
+            float f[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                kh[c] = kv[q2][c] * ex2(-Lt[q2][c]);
+                khf[q2][c] = kv[q2][c] * ex2(-Lt[q2][c]);
                 f[c] = ex2(Lx[q2][c]);
             }
             uint4 hi, lo;
-            split8(kh, hi, lo);
+            split8(khf[q2], hi, lo);
             *reinterpret_cast<uint4*>(s.kh[pb][0] + sw_chunk(ta + q2, cg)) = hi;
             *reinterpret_cast<uint4*>(s.kh[pb][1] + sw_chunk(ta + q2, cg)) = lo;
             float4* fd = reinterpret_cast<float4*>(&s.F[pb][ta + q2][8 * cg]);
             fd[0] = make_float4(f[0], f[1], f[2], f[3]);
             fd[1] = make_float4(f[4], f[5], f[6], f[7]);
         }
+        // Kt = k 2^(L63 - L) = Kh * gamma: both factors are within the range test's bounds
+        // (2^(-L) <= 2^86.56, gamma >= 2^-86.56), so the product is a normal fp32 number
+        float gam[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) gam[c] = ex2(L63[c]);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {   // Kt^T: channel row i, this lane's two tokens
             const int i = 8 * cg + c;
-            const float x0 = kv[0][c] * ex2(L63[c] - Lt[0][c]);
-            const float x1 = kv[1][c] * ex2(L63[c] - Lt[1][c]);
+            const float x0 = khf[0][c] * gam[c];
+            const float x1 = khf[1][c] * gam[c];
             const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
             const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
             *reinterpret_cast<uint32_t*>(s.kt_hi[pb] + tr_off(i, lane)) = pack2(h0, h1);
@@ -302,7 +308,7 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
         }
         if (lane == 0)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) s.gamma[pb][8 * cg + c] = ex2(L63[c]);
+            for (int c = 0; c < 8; ++c) s.gamma[pb][8 * cg + c] = gam[c];
         return true;
     };
     // MMA 1 of chunk m (one thread): A = dy v^T, Z[m & 1] = dy S^T (S = the state entering m,
