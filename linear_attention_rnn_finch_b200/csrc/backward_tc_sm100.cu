@@ -48,6 +48,7 @@
 #include <cuda_bf16.h>
 
 #include "backward.h"
+#include "chunk_tiles.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
@@ -233,17 +234,24 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
             unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(tb, cg)), kv[1]);
             unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(ta, cg)), om[0]);
             unpack8(*reinterpret_cast<const uint4*>(w_tile + sw_chunk(tb, cg)), om[1]);
+            float ew[2][8];   // exp(omega)
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
-                for (int c = 0; c < 8; ++c)   // log2 w = -exp(omega) log2(e); 0 past T
-                    lw[q2][c] = (ta + q2 < valid) ? -ex2(om[q2][c] * kLog2e) * kLog2e : 0.f;
-            if (kC2 && !kDk) {   // the state's key is kn = k (1 - w), 1 - w = -expm1(-exp(omega))
+                for (int c = 0; c < 8; ++c) {   // log2 w = -exp(omega) log2(e); 0 past T
+                    ew[q2][c] = ex2(om[q2][c] * kLog2e);
+                    lw[q2][c] = (ta + q2 < valid) ? -ew[q2][c] * kLog2e : 0.f;
+                }
+            if (kC2 && !kDk) {   // the state's key is kn = k (1 - w), 1 - w = 1 - exp(-exp(omega))
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        kv[q2][c] *= (ta + q2 < valid) ? -expm1f(-__expf(om[q2][c])) : 0.f;
+                    for (int c = 0; c < 8; c += 2) {
+                        const float2 f = tiles::one_minus_exp_neg2(make_float2(ew[q2][c], ew[q2][c + 1]));
+                        const bool in = ta + q2 < valid;
+                        kv[q2][c] *= in ? f.x : 0.f;
+                        kv[q2][c + 1] *= in ? f.y : 0.f;
+                    }
             }
         }
         // inclusive prefix over the chunk: this lane's pair, then a scan over the lanes
@@ -469,17 +477,26 @@ wkv6_bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __gr
                     float kx[8], o[8], pv[8], rv[8], dv8[8];
                     unpack8(*reinterpret_cast<const uint4*>(k_tile + sw_chunk(t, cc0 + cc)), kx);
                     unpack8(rw[cc], rv);
-                    float om[8];
-                    if (kC2 && kDk)   // this token's omega (reversed-time tile, row t)
+                    float om[8], omw8[8], w8[8];
+                    if (kC2 && kDk) {   // this token's omega (reversed-time tile, row t)
                         unpack8(*reinterpret_cast<const uint4*>(s.in[st][3] + sw_chunk(t, cc0 + cc)), om);
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {   // w and 1 - w of x = exp(omega)
+                            const float2 x = make_float2(ex2(om[e] * kLog2e), ex2(om[e + 1] * kLog2e));
+                            const float2 f = tiles::one_minus_exp_neg2(x);
+                            omw8[e] = f.x;
+                            omw8[e + 1] = f.y;
+                            w8[e] = ex2(-x.x * kLog2e);
+                            w8[e + 1] = ex2(-x.y * kLog2e);
+                        }
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = 8 * cc + e, i = cb + j;
                         const float pair = s.F[pb][t][i] * __uint_as_float(Z[j]);   // minus the bonus
                         if (kC2 && kDk) {
                             // pair = dkn; dk = dkn (1 - w); Q = kn dkn = k (1 - w) dkn; D = dkn k w
-                            const float ew = __expf(om[e]);
-                            const float omw = -expm1f(-ew), w = __expf(-ew);
+                            const float omw = omw8[e], w = w8[e];
                             o[e] = pair * omw;
                             pv[e] = rv[e] * omw * pair;
                             dv8[e] = pair * rv[e] * w;
