@@ -382,7 +382,8 @@ def backward_line(cfg, dev, world, steps, c2=False):
                         "CUDA-core scans run only for a (b,h) whose decays the one-sided factors "
                         "cannot take"),
             "note": "algorithmic FLOPs are the three recurrences (dr, dk, dv) at 5 FLOPs per "
-                    "state entry per token; dr, dk and dv run on the tensor cores"}
+                    "state entry per token; dr, dk and dv run on the tensor cores, on three "
+                    "streams forked from and joined to the caller's"}
     del inp, dy, dS, ws, args_b
     torch.cuda.empty_cache()
     return line
