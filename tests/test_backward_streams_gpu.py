@@ -5,8 +5,12 @@ own stream like any other.
 - on a stream of the caller's, with dy produced on that stream just before the call and the
   outputs reduced on it just after, the results equal a default-stream call bit for bit;
 - captured into a CUDA graph (after a first call has made the side streams), a replay gives
-  the same results as an eager call, bit for bit.
+  the same results as an eager call, bit for bit;
+- two host threads calling at once, each on a stream of its own (the side streams and
+  their events are shared per device), get the results of calls made one after another.
 """
+import threading
+
 import pytest
 import torch
 
@@ -77,3 +81,37 @@ def test_backward_graph_capture_replay(c2):
             continue
         assert torch.equal(g, w)
     del graph
+
+
+@pytest.mark.parametrize("c2", [False, True])
+def test_backward_two_host_threads(c2):
+    problems = [_inputs(7300 + i) for i in range(2)]
+    want = [_call(*p, c2) for p in problems]
+    torch.cuda.synchronize()
+    got, errors = [None, None], []
+
+    def run(i):
+        try:
+            s = torch.cuda.Stream()
+            outs = []
+            with torch.cuda.stream(s):
+                for _ in range(3):
+                    outs.append(_call(*problems[i], c2, stream=s))
+            s.synchronize()
+            got[i] = outs
+        except Exception as e:   # reported below, on the test's thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for i in range(2):
+        for outs in got[i]:
+            for g, w in zip(outs, want[i]):
+                if w is None:
+                    assert g is None
+                    continue
+                assert torch.equal(g, w)
