@@ -324,6 +324,12 @@ size_t decode_ln_bytes(int B, int H, wkv_dtype io) {
     return decode_counter_bytes(B) + (io == WKV_BF16 ? (size_t)B * H * kHeadSizeApi * sizeof(float) : 0);
 }
 
+// LayerNorm on the chunked path: a progress word per (b,h,segment) unit, which the level
+// kernel's fused LayerNorm reads (zeroed before each call)
+size_t ln_progress_bytes(int B, int H, int P) {
+    return round256((size_t)B * H * P * sizeof(int));
+}
+
 size_t chunked_bytes(int B, int H, int P) {
     const long units = (long)B * H * P;
     return kStatusBytes + handoff_ints_bytes(units) + handoff_state_bytes(units) +
@@ -347,10 +353,14 @@ PrefillPlan prefill_plan(int B, int T, int H, wkv_dtype io, bool with_ln, wkv_al
     const size_t ln = with_ln && io == WKV_BF16 ? (size_t)B * T * H * kHeadSizeApi * sizeof(float)
                                                 : 0;
     if (!chunked) return {1, ln};
+    // on the chunked path LayerNorm also keeps a progress word per (b,h,segment) unit
+    auto bytes = [&](int P) {
+        return chunked_bytes(B, H, P) + (with_ln ? ln_progress_bytes(B, H, P) : 0) + ln;
+    };
     int P = algo == WKV_ALGO_CHUNKED_LEVELS ? 1 : choose_segments(B, T, H);
     const int nc = (T + kChunk - 1) / kChunk;
-    while (P > 1 && (!segments_feasible(nc, P) || chunked_bytes(B, H, P) + ln > cap)) --P;
-    return {P, chunked_bytes(B, H, P) + ln};
+    while (P > 1 && (!segments_feasible(nc, P) || bytes(P) > cap)) --P;
+    return {P, bytes(P)};
 }
 
 }  // namespace
@@ -395,7 +405,9 @@ bool launch_chunked_path(const void* r, const void* k, const void* v, const void
                          const float* u, const goldwkv::Variant& var, const float* state_in,
                          float* state_out, void* y, float* y_raw, int B, int T, int H, int P,
                          bool levels_only, uint8_t* ws, cudaStream_t st, cudaError_t* e,
-                         const goldwkv::GnOut* gn = nullptr) {
+                         const goldwkv::GnOut* gn = nullptr,
+                         const goldwkv::LnFuse* ln = nullptr, bool* ln_done = nullptr) {
+    if (ln_done) *ln_done = false;
     const long long budget = injected("timeout0") ? 0 : kSpinBudget;
     CUtensorMap maps[5];
     if (!goldwkv::make_token_map(&maps[0], r, B, T, H) ||
@@ -417,7 +429,8 @@ bool launch_chunked_path(const void* r, const void* k, const void* v, const void
     const goldwkv::Segments seg{P, (nc + P - 1) / P, s_mid};
     if (levels_only) {
         *e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg,
-                                            var, status, nullptr, nullptr, budget, st, gn);
+                                            var, status, nullptr, nullptr, budget, st, gn, ln,
+                                            ln_done);
         return true;
     }
     *e = cudaSuccess;
@@ -432,7 +445,8 @@ bool launch_chunked_path(const void* r, const void* k, const void* v, const void
                                           var, status, h_chunk, h_state, budget, st, gn);
     if (*e == cudaSuccess)
         *e = goldwkv::launch_chunked_levels(maps, u, state_in, state_out, y_raw, B, T, H, seg, var,
-                                            status, h_chunk, h_state, budget, st, gn);
+                                            status, h_chunk, h_state, budget, st, gn, ln,
+                                            ln_done);
     return true;
 }
 
@@ -513,7 +527,13 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* y_raw = nullptr;
     const int P = plan.P;
-    const size_t raw_at = chunked ? chunked_bytes(B, H, P) : 0;
+    // chunked path with LayerNorm: the units' progress words, then the fp32 rows
+    int* ln_progress = chunked && nm.kind == Norm::kLayer
+                           ? reinterpret_cast<int*>(ws + chunked_bytes(B, H, P))
+                           : nullptr;
+    const size_t raw_at = chunked ? chunked_bytes(B, H, P) +
+                                        (ln_progress ? ln_progress_bytes(B, H, P) : 0)
+                                  : 0;
     // GroupNorm + gate runs inside the chunked kernels; LayerNorm (over all heads of a token)
     // and the fp32 recurrence's output stages run as a second pass over fp32 rows
     const bool fused_gn = chunked && nm.kind == Norm::kGroup;
@@ -521,17 +541,25 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
     if (nm.on() && !fused_gn)
         y_raw = bf16 ? reinterpret_cast<float*>(ws + raw_at) : static_cast<float*>(y);
     cudaError_t e;
+    bool ln_done = false;   // the level kernel's launch normalised the rows itself
     if (chunked) {
+        // (the level kernel's CTAs normalise the rows in the same launch when they fit)
+        const goldwkv::LnFuse lnf{ln_progress, nm.gamma, nm.beta, nm.eps,
+                                  static_cast<__nv_bfloat16*>(y)};
+        if (ln_progress != nullptr &&
+            cudaMemsetAsync(ln_progress, 0, (size_t)B * H * P * sizeof(int), st) != cudaSuccess)
+            return WKV_ERR_CUDA;
         if (!launch_chunked_path(r, k, v, omega, u, var, state_in, state_out, y, y_raw, B, T, H,
                                  P, algo == WKV_ALGO_CHUNKED_LEVELS, ws, st, &e,
-                                 fused_gn ? &gn : nullptr))
+                                 fused_gn ? &gn : nullptr, ln_progress ? &lnf : nullptr,
+                                 &ln_done))
             return WKV_ERR_CUDA;
     } else {
         e = goldwkv::launch_recurrent(r, k, v, omega, u, state_in, state_out, y, y_raw, B, T,
                                       H, bf16, var, st);
     }
     if (e != cudaSuccess) return WKV_ERR_CUDA;
-    if (nm.on() && !fused_gn &&
+    if (nm.on() && !fused_gn && !ln_done &&
         launch_norm(nm, y_raw, y, (long)B * T, H, D, bf16, st) != cudaSuccess)
         return WKV_ERR_CUDA;
     return WKV_OK;

@@ -52,6 +52,7 @@
 // its TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <limits.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -88,6 +89,7 @@ struct __align__(1024) Smem {
     uint64_t mma1u, mma1, mma2;   // MMA 1's U and Y products; all of MMA 1; MMA 2
     uint32_t tmem_base;
     int abort;
+    int ln_go;                       // LayerNorm CTAs: every head of the block is stored
     float2 gn_mom[2][64];            // GroupNorm stage: (mean, M2) of each row's two halves
 };
 
@@ -130,6 +132,103 @@ __device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 
     *reinterpret_cast<uint4*>(base + off) = v;
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// One warp: LayerNorm of a row of nf4 16-byte pieces (nf4 <= 512, i.e. H <= 32 heads) read
+// from L2 (the rows were written by other SMs during this launch), bf16 out.
+__device__ __forceinline__ void ln_row_warp(const float* row, __nv_bfloat16* orow,
+                                            const float* gamma, const float* beta, float eps,
+                                            int nf4, int lane) {
+    float4 v[16];
+    float sm = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        const int i = lane + 32 * m;
+        v[m] = i < nf4 ? __ldcg(reinterpret_cast<const float4*>(row) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sm += (v[m].x + v[m].y) + (v[m].z + v[m].w);
+    }
+    const float inv_n = 1.f / (4.f * (float)nf4);
+    const float mean = warp_sum(sm) * inv_n;
+    float q = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        if (lane + 32 * m < nf4) {
+            v[m].x -= mean; v[m].y -= mean; v[m].z -= mean; v[m].w -= mean;
+            q = fmaf(v[m].x, v[m].x, fmaf(v[m].y, v[m].y, fmaf(v[m].z, v[m].z, fmaf(v[m].w, v[m].w, q))));
+        }
+    }
+    const float inv = rsqrtf(warp_sum(q) * inv_n + eps);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        const int i = lane + 32 * m;
+        if (i < nf4) {
+            const float4 g = __ldg(reinterpret_cast<const float4*>(gamma) + i);
+            const float4 bb = __ldg(reinterpret_cast<const float4*>(beta) + i);
+            __nv_bfloat162 lo = __floats2bfloat162_rn(fmaf(v[m].x * inv, g.x, bb.x), fmaf(v[m].y * inv, g.y, bb.y));
+            __nv_bfloat162 hi = __floats2bfloat162_rn(fmaf(v[m].z * inv, g.z, bb.z), fmaf(v[m].w * inv, g.w, bb.w));
+            reinterpret_cast<uint2*>(orow)[i] =
+                make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+        }
+    }
+}
+
+// The LayerNorm CTAs of a fused launch (blockIdx.x >= units): 64-token blocks (b, chunk c)
+// in chunk-major order, CTA j taking blocks j, j + nctas, ...; warp 0 waits until every
+// head's unit owning chunk c has published a progress past c (bounded; a unit that gave up
+// publishes INT_MIN and the block is skipped), then each warp normalises rows.  Nothing
+// else waits for these CTAs, and the cooperative launch keeps them co-resident with the
+// units they wait for.
+__device__ void ln_blocks(Smem& s, const LnFuse& ln, const float* y_raw, int T, int H,
+                          const Segments& seg, int units, int* status, long long budget) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nbh = units / seg.P, B = nbh / H, NCt = (T + C - 1) / C;
+    const int nctas = gridDim.x - units, j = blockIdx.x - units;
+    const int nf4 = H * 16;
+    const long blocks = (long)B * NCt;
+    for (long rb = j; rb < blocks; rb += nctas) {
+        const int c = (int)(rb / B), b = (int)(rb - (long)c * B);
+        const int p = min(c / seg.seg_chunks, seg.P - 1);
+        if (warp == 0) {
+            bool ok = true;
+            for (int h = lane; h < H; h += 32) {
+                const int* w = ln.progress + (size_t)p * nbh + b * H + h;
+                const long long t0 = clock64();
+                int v = ld_acquire_gpu(w);
+                while (v >= 0 && v <= c) {
+                    if (clock64() - t0 > budget) {
+                        v = -1;
+                        break;
+                    }
+                    __nanosleep(500);
+                    v = ld_acquire_gpu(w);
+                }
+                ok = ok && v > c;
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (lane == 0) s.ln_go = ok ? 1 : 0;
+        }
+        __syncthreads();
+        const bool go = s.ln_go != 0;
+        __syncthreads();   // every warp has read the flag before warp 0 writes the next one
+        if (!go) {
+            if (tid == 0) atomicExch(status, 1);
+            continue;
+        }
+        const int t_end = min(T, (c + 1) * C);
+        for (int t = c * C + warp; t < t_end; t += kThreads / 32) {
+            const size_t at = ((size_t)b * T + t) * (size_t)(H * 64);
+            ln_row_warp(y_raw + at, ln.out + at, ln.gamma, ln.beta, ln.eps, nf4, lane);
+        }
+    }
+}
+
 // kC2: Finch-C2 exact form -- key k (1 - w), no static bonus, second value uprime added.
 // kGN: base form with the GroupNorm + gate output stage (gn).
 // kQ: no bonus, query r (1 - w) (Variant::query_c2).
@@ -140,17 +239,25 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
                     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ u,
                     const float* s_in, float* s_out, float* __restrict__ y_raw,
                     const __nv_bfloat16* __restrict__ uprime, const GnOut gn, int T, int H, Segments seg, int* status, const int* start_chunk,
-                    const float* handoff_state, long long spin_budget, long long drain_budget) {
+                    const float* handoff_state, long long spin_budget, long long drain_budget,
+                    const LnFuse ln, int units) {
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if ((int)blockIdx.x >= units) {   // a LayerNorm CTA of a fused launch
+        ln_blocks(s, ln, y_raw, T, H, seg, units, status, spin_budget);
+        return;
+    }
     // unit: segment pseg of sequence bh, absolute chunks c_begin .. NC - 1
-    const int unit = blockIdx.x, nbh = gridDim.x / seg.P;
+    const int unit = blockIdx.x, nbh = units / seg.P;
     const int bh = unit % nbh, pseg = unit / nbh, b = bh / H, h = bh - (bh / H) * H;
     const int c_begin = pseg * seg.seg_chunks;
     const int NC = min((T + C - 1) / C, c_begin + seg.seg_chunks);
     // resume point: chunks before n0 (and the state entering n0) came from the fast kernel
     const int n0 = start_chunk ? start_chunk[unit] : c_begin;
+    // LayerNorm fused: the rows before n0 (the fast kernel's, or another unit's) are stored
+    if (ln.progress != nullptr && tid == 0)
+        st_release_gpu(ln.progress + unit, (n0 < 0 || n0 >= NC) ? INT_MAX : n0);
     if (n0 < 0 || n0 >= NC) return;       // this unit is already complete
     const float* state0 = start_chunk ? handoff_state + (size_t)unit * 4096
                         : pseg > 0    ? seg.s_mid + ((size_t)bh * (seg.P - 1) + (pseg - 1)) * 4096
@@ -388,6 +495,14 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             ptx::mma_commit(&s.mma1);
             issued1 = n;
         }
+        // LayerNorm fused: the previous chunk's fp32 rows (stored before that chunk's last
+        // barrier) are published to the LayerNorm CTAs here, where every warp waits for the
+        // products anyway, so the fence's wait is off the chunk's critical path (warp 1:
+        // thread 0 issues the copies and products)
+        if (ln.progress != nullptr && tid == 32 && n > n0) {
+            __threadfence();
+            st_release_gpu(ln.progress + unit, n);
+        }
         if (!ptx::mbar_wait(&s.mma1u, (uint32_t)(m & 1), spin_budget)) s.abort = 1;
         ptx::tc_fence_after();
 
@@ -614,6 +729,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     if (failed) {
         if (tid == 0) {
             atomicExch(status, 1);
+            if (ln.progress != nullptr) st_release_gpu(ln.progress + unit, INT_MIN);
             // copies still in flight: chunks n .. min(NC, n + kStages) - 1 may have been issued
             for (int c = n; c < NC && c < n + kStages; ++c)
                 ptx::mbar_wait(&s.full[(c - n0) % kStages], (uint32_t)(((c - n0) / kStages) & 1),
@@ -621,11 +737,17 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
             if (issued1 == n) ptx::mbar_wait(&s.mma1, (uint32_t)((n - n0) & 1), drain_budget);
             if (issued2 == n) ptx::mbar_wait(&s.mma2, (uint32_t)((n - n0) & 1), drain_budget);
         }
-    } else if (s_out != nullptr) {
-        float* dst = s_out + (size_t)bh * 4096 + row * 64 + cb;
+    } else {
+        if (s_out != nullptr) {
+            float* dst = s_out + (size_t)bh * 4096 + row * 64 + cb;
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+        if (ln.progress != nullptr && tid == 32) {   // the last chunk's rows
+            __threadfence();
+            st_release_gpu(ln.progress + unit, INT_MAX);
+        }
     }
     if (tid == 0) ptx::bulk_wait<0>();
     ptx::tc_fence_before();
@@ -693,7 +815,9 @@ cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const
                                   float* s_out, float* y_raw, int B, int T, int H, Segments seg,
                                   Variant var, int* status, const int* start_chunk,
                                   const float* handoff_state, long long spin_budget,
-                                  cudaStream_t st, const GnOut* gn) {
+                                  cudaStream_t st, const GnOut* gn, const LnFuse* ln,
+                                  bool* ln_done) {
+    if (ln_done) *ln_done = false;
     const size_t smem = chunked_smem_bytes();
     auto kernel = var.uprime     ? wkv6_chunked_kernel<true, false, false>
                   : gn           ? wkv6_chunked_kernel<false, true, false>
@@ -702,11 +826,42 @@ cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long drain = 4000000000LL;
-    kernel<<<(unsigned)(B * H * seg.P), kThreads, smem, st>>>(
+    const int units = B * H * seg.P;
+    const GnOut g = gn ? *gn : GnOut{nullptr, nullptr, 0.f, nullptr};
+    // LayerNorm inside the launch: as many extra CTAs as stay co-resident with the units
+    // (at most one per 64-token block), under a cooperative launch that guarantees it
+    long ln_ctas = 0;
+    if (ln != nullptr && y_raw != nullptr && gn == nullptr && H <= 32 && T > 0) {
+        int dev = 0, nsm = 0, coop = 0, nb = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess &&
+            coop != 0 &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, kThreads, smem) == cudaSuccess) {
+            ln_ctas = (long)nb * nsm - units;
+            const long blocks = (long)B * ((T + C - 1) / C);
+            if (ln_ctas > blocks) ln_ctas = blocks;
+        } else {
+            (void)cudaGetLastError();
+        }
+    }
+    if (ln_ctas >= 1) {
+        const LnFuse lf = *ln;
+        void* args[] = {(void*)&maps[0], (void*)&maps[1], (void*)&maps[2], (void*)&maps[3],
+                        (void*)&maps[4], (void*)&u, (void*)&s_in, (void*)&s_out, (void*)&y_raw,
+                        (void*)&var.uprime, (void*)&g, (void*)&T, (void*)&H, (void*)&seg,
+                        (void*)&status, (void*)&start_chunk, (void*)&handoff_state,
+                        (void*)&spin_budget, (void*)&drain, (void*)&lf, (void*)&units};
+        e = cudaLaunchCooperativeKernel((const void*)kernel, dim3((unsigned)(units + ln_ctas)),
+                                        dim3(kThreads), args, smem, st);
+        if (e == cudaSuccess && ln_done) *ln_done = true;
+        return e;
+    }
+    const LnFuse none{nullptr, nullptr, nullptr, 0.f, nullptr};
+    kernel<<<(unsigned)units, kThreads, smem, st>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], u, s_in, s_out, y_raw,
-        static_cast<const __nv_bfloat16*>(var.uprime), gn ? *gn : GnOut{nullptr, nullptr, 0.f, nullptr},
-        T, H, seg, status, start_chunk,
-        handoff_state, spin_budget, drain);
+        static_cast<const __nv_bfloat16*>(var.uprime), g, T, H, seg, status, start_chunk,
+        handoff_state, spin_budget, drain, none, units);
     return cudaGetLastError();
 }
 

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stddef.h>
 
 #include "goldwkv.h"
@@ -114,15 +115,32 @@ cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const f
                                 float* handoff_state, long long budget, cudaStream_t st,
                                 const GnOut* gn = nullptr);
 
+// LayerNorm of the fp32 rows y_raw (a token's H heads) inside the level kernel's launch:
+// extra CTAs, co-resident with the recurrence's (a cooperative launch), normalise the
+// 64-token blocks of a batch row as soon as every head has published them.  progress: one
+// word per (b,h,segment) unit, zero before the launch; a unit stores, with release
+// semantics, the absolute index of the first chunk whose rows it has not yet stored
+// (INT_MAX: all; INT_MIN: it gave up).
+struct LnFuse {
+    int* progress;
+    const float* gamma;
+    const float* beta;
+    float eps;
+    __nv_bfloat16* out;   // y [B][T][H][64]
+};
+
 // Level-factorised path (any decay).  start_chunk == nullptr: every unit from its first
 // chunk with its incoming state; otherwise unit u resumes at chunk start_chunk[u] (skipped if
 // < 0) from handoff_state[u].  status: device word set to 1 if a bounded wait expired.
-// gn: as for the fast path.
+// gn: as for the fast path.  ln (y_raw != nullptr, H <= 32): LayerNorm into ln->out within
+// the launch if the recurrence's CTAs leave room for at least one more co-resident CTA;
+// *ln_done says whether it did (else the caller runs the LayerNorm pass).
 cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const float* s_in,
                                   float* s_out, float* y_raw, int B, int T, int H, Segments seg,
                                   Variant var, int* status, const int* start_chunk,
                                   const float* handoff_state, long long spin_budget,
-                                  cudaStream_t st, const GnOut* gn = nullptr);
+                                  cudaStream_t st, const GnOut* gn = nullptr,
+                                  const LnFuse* ln = nullptr, bool* ln_done = nullptr);
 size_t chunked_smem_bytes();
 size_t fast_smem_bytes();
 size_t segment_smem_bytes();
