@@ -297,10 +297,12 @@ def other_prefill(cfg, dev, world, hbm, algo, steps, c2=False, gn=False):
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
     # + u' read (C2) or + gate read (GroupNorm)
     nbytes = prefill_bytes(B, T, H, D) + (B * T * H * D * 2 if c2 or gn else 0)
-    # with LayerNorm / GroupNorm the library also writes and re-reads an fp32 copy of y; the
-    # roofline counts only the bytes the operation itself must move
-    nbytes_note = (("GroupNorm + gate" if gn else "LayerNorm") + " runs as a second pass over an "
-                   "fp32 copy of y, not counted in the algorithmic bytes") if cfg.ln or gn else None
+    # the roofline counts only the bytes the operation itself must move (LayerNorm's fp32
+    # staging of y is not counted)
+    nbytes_note = ("GroupNorm + gate runs in the recurrence kernels' output stage" if gn else
+                   "LayerNorm runs inside the level kernel's launch on co-resident CTAs when the "
+                   "recurrence's CTAs leave SMs free (else as a second pass) over an fp32 staging "
+                   "of y, not counted in the algorithmic bytes" if cfg.ln else None)
     name = ("wkv6c2_" + cfg.name[5:]) if c2 else (cfg.name + "_groupnorm_gate") if gn else cfg.name
     form = ("Finch-C2 (normalised key, second value)" if c2 else
             "base Finch (static bonus), per-head GroupNorm and gate" if gn else

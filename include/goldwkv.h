@@ -107,6 +107,11 @@ size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, in
  *                   new workspace; see wkv6_workspace_status); other bytes are scratch.
  *   Algorithm: WKV_ALGO_AUTO takes the chunked tensor-core kernel for bf16 I/O and the
  *   fp32 recurrence for fp32 I/O.
+ *   LayerNorm: the recurrence stages fp32 rows of y in the workspace.  On the chunked path
+ *   with H <= 32, when the level-factorised kernel's CTAs leave room on the device, extra
+ *   CTAs of the same (cooperative) launch normalise each 64-token block of a batch row as
+ *   soon as all H heads have stored it, and drop the consumed staging lines from L2;
+ *   otherwise (and for fp32 I/O) a second kernel normalises the staged rows.  Same results.
  * Returns WKV_OK, or an error with nothing launched (INVALID_ARG, UNSUPPORTED, WORKSPACE)
  * or WKV_ERR_CUDA if a launch failed.
  */

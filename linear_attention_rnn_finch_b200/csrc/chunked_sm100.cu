@@ -142,7 +142,10 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 }
 
 // One warp: LayerNorm of a row of nf4 16-byte pieces (nf4 <= 512, i.e. H <= 32 heads) read
-// from L2 (the rows were written by other SMs during this launch), bf16 out.
+// from L2 (the rows were written by other SMs during this launch), bf16 out.  The fp32 row
+// is scratch nobody reads again: once it is in registers its 128-byte L2 lines are dropped
+// (discard.global.L2: no write-back), so rows read soon after they were written never
+// reach DRAM.  Only for a 128-byte-aligned row (the instruction's requirement).
 __device__ __forceinline__ void ln_row_warp(const float* row, __nv_bfloat16* orow,
                                             const float* gamma, const float* beta, float eps,
                                             int nf4, int lane) {
@@ -164,7 +167,10 @@ __device__ __forceinline__ void ln_row_warp(const float* row, __nv_bfloat16* oro
             q = fmaf(v[m].x, v[m].x, fmaf(v[m].y, v[m].y, fmaf(v[m].z, v[m].z, fmaf(v[m].w, v[m].w, q))));
         }
     }
-    const float inv = rsqrtf(warp_sum(q) * inv_n + eps);
+    const float inv = rsqrtf(warp_sum(q) * inv_n + eps);   // every lane's loads are done
+    if ((reinterpret_cast<uintptr_t>(row) & 127u) == 0)
+        for (int li = lane; li < nf4 / 8; li += 32)           // 8 pieces per 128-byte line
+            asm volatile("discard.global.L2 [%0], 128;" ::"l"(row + 32 * li) : "memory");
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
         const int i = lane + 32 * m;
