@@ -1,7 +1,10 @@
 """Prefill with LayerNorm (bf16 chunked path), against the fp64 oracle.
 
-The recurrence kernels stage each token's fp32 rows and a second kernel normalises them
-over all H*64 channels.  These cases cover each way a token chunk's rows can be produced:
+The recurrence kernels stage each token's fp32 rows, normalised over all H*64 channels by
+extra CTAs of the level kernel's launch when the recurrence's CTAs leave room on the device
+and H <= 32, else by a second kernel (the last cases here force that: more (b,h) units than
+the device holds at once, or H > 32).  These cases cover each way a token chunk's rows can
+be produced:
 the fast kernel alone, the level-factorised kernel alone, a hand-over from one to the other
 in the middle of a sequence (so one chunk's heads come from both kernels), a forced sequence
 split, ragged tails, one head, odd head counts, Finch-C2's form, and repeated calls on one
@@ -108,3 +111,12 @@ def test_prefill_ln_reused_workspace_after_expired_wait(oracle, monkeypatch):
         assert bd.workspace_status(ws) == bd.WKV_OK
         assert torch.equal(y, y1) and torch.equal(s, s1)
     check(oracle, inp, y1, s1)
+
+
+@pytest.mark.parametrize("algo", ["chunked", "chunked_levels"])
+@pytest.mark.parametrize("B,H,T", [(5, 32, 130), (1, 40, 70)])
+def test_prefill_ln_second_pass(oracle, B, H, T, algo):
+    """160 (b,h) units fill every SM (no room for the normalising CTAs), or 40 heads (rows
+    wider than the in-launch LayerNorm takes): the staged rows go through the second kernel."""
+    inp = problem(9700 + B * H + T, B=B, T=T, H=H)
+    check(oracle, inp, *run(inp, algo))
