@@ -83,8 +83,8 @@ typedef struct wkv_ln {
  * on its arguments.  Layout on the chunked path: a 4-byte device status word at offset 0
  * (256 bytes reserved), then per (b,h) a hand-off record (chunk index, and a D x D fp32
  * state) used when a sequence moves from the fast to the level-factorised kernel;
- * LayerNorm with bf16 output adds a progress word per (b,h,segment) unit (256-byte aligned)
- * and an fp32 [B][T][H][D] staging buffer at the end. */
+ * LayerNorm with bf16 output adds a progress word per (b,h,segment) unit and one counter
+ * (256-byte aligned) and an fp32 [B][T][H][D] staging buffer at the end. */
 size_t wkv6_prefill_workspace_bytes(int B, int T, int H, int D, wkv_dtype io, int with_ln,
                                     wkv_algo algo);
 

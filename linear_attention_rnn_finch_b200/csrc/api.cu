@@ -324,10 +324,11 @@ size_t decode_ln_bytes(int B, int H, wkv_dtype io) {
     return decode_counter_bytes(B) + (io == WKV_BF16 ? (size_t)B * H * kHeadSizeApi * sizeof(float) : 0);
 }
 
-// LayerNorm on the chunked path: a progress word per (b,h,segment) unit, which the level
-// kernel's fused LayerNorm reads (zeroed before each call)
+// LayerNorm on the chunked path: a progress word per (b,h,segment) unit and a block counter,
+// which the level kernel's fused LayerNorm uses (zeroed before each call)
+size_t ln_progress_words(int B, int H, int P) { return (size_t)B * H * P + 1; }
 size_t ln_progress_bytes(int B, int H, int P) {
-    return round256((size_t)B * H * P * sizeof(int));
+    return round256(ln_progress_words(B, H, P) * sizeof(int));
 }
 
 size_t chunked_bytes(int B, int H, int P) {
@@ -547,7 +548,8 @@ wkv_status prefill_impl(const void* r, const void* k, const void* v, const void*
         const goldwkv::LnFuse lnf{ln_progress, nm.gamma, nm.beta, nm.eps,
                                   static_cast<__nv_bfloat16*>(y)};
         if (ln_progress != nullptr &&
-            cudaMemsetAsync(ln_progress, 0, (size_t)B * H * P * sizeof(int), st) != cudaSuccess)
+            cudaMemsetAsync(ln_progress, 0, ln_progress_words(B, H, P) * sizeof(int), st) !=
+                cudaSuccess)
             return WKV_ERR_CUDA;
         if (!launch_chunked_path(r, k, v, omega, u, var, state_in, state_out, y, y_raw, B, T, H,
                                  P, algo == WKV_ALGO_CHUNKED_LEVELS, ws, st, &e,

@@ -90,6 +90,7 @@ struct __align__(1024) Smem {
     uint32_t tmem_base;
     int abort;
     int ln_go;                       // LayerNorm CTAs: every head of the block is stored
+    int ln_rb;                       // LayerNorm CTAs: the block taken
     float2 gn_mom[2][64];            // GroupNorm stage: (mean, M2) of each row's two halves
 };
 
@@ -185,25 +186,29 @@ __device__ __forceinline__ void ln_row_warp(const float* row, __nv_bfloat16* oro
     }
 }
 
-// The LayerNorm CTAs of a fused launch (blockIdx.x >= units): 64-token blocks (b, chunk c)
-// in chunk-major order, CTA j taking blocks j, j + nctas, ...; warp 0 waits until every
-// head's unit owning chunk c has published a progress past c (bounded; a unit that gave up
-// publishes INT_MIN and the block is skipped), then each warp normalises rows.  Nothing
-// else waits for these CTAs, and the cooperative launch keeps them co-resident with the
-// units they wait for.
+// The LayerNorm workers of a fused launch: the extra CTAs (blockIdx.x >= units) and the CTA
+// of every unit that is already complete (the fast kernel finished it), so that when the
+// fast kernel did most of the work most of the device normalises.  A worker takes the next
+// 64-token block (b, chunk c), in chunk-major order, from a counter after the progress
+// words; warp 0 waits until every head's unit owning chunk c has published a progress past
+// c (bounded; a unit that gave up publishes INT_MIN and the block is skipped), then each
+// warp normalises rows.  Nothing waits for the workers, and the cooperative launch keeps
+// them co-resident with the units they wait for.
 __device__ void ln_blocks(Smem& s, const LnFuse& ln, const float* y_raw, int T, int H,
                           const Segments& seg, int units, int* status, long long budget) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nbh = units / seg.P, B = nbh / H, NCt = (T + C - 1) / C;
-    const int nctas = gridDim.x - units, j = blockIdx.x - units;
     const int nf4 = H * 16;
-    const long blocks = (long)B * NCt;
-    for (long rb = j; rb < blocks; rb += nctas) {
-        const int c = (int)(rb / B), b = (int)(rb - (long)c * B);
-        const int p = min(c / seg.seg_chunks, seg.P - 1);
+    const int blocks = B * NCt;
+    for (;;) {
         if (warp == 0) {
+            int rb = 0;
+            if (lane == 0) rb = atomicAdd(ln.progress + units, 1);
+            rb = __shfl_sync(0xffffffffu, rb, 0);
             bool ok = true;
-            for (int h = lane; h < H; h += 32) {
+            const int c = rb / B, b = rb - (rb / B) * B;
+            const int p = min(c / seg.seg_chunks, seg.P - 1);
+            for (int h = lane; rb < blocks && h < H; h += 32) {
                 const int* w = ln.progress + (size_t)p * nbh + b * H + h;
                 const long long t0 = clock64();
                 int v = ld_acquire_gpu(w);
@@ -218,15 +223,21 @@ __device__ void ln_blocks(Smem& s, const LnFuse& ln, const float* y_raw, int T, 
                 ok = ok && v > c;
             }
             ok = __all_sync(0xffffffffu, ok);
-            if (lane == 0) s.ln_go = ok ? 1 : 0;
+            if (lane == 0) {
+                s.ln_rb = rb;
+                s.ln_go = ok ? 1 : 0;
+            }
         }
         __syncthreads();
+        const int rb = s.ln_rb;
         const bool go = s.ln_go != 0;
-        __syncthreads();   // every warp has read the flag before warp 0 writes the next one
+        __syncthreads();   // every warp has read the block before warp 0 takes the next one
+        if (rb >= blocks) break;
         if (!go) {
             if (tid == 0) atomicExch(status, 1);
             continue;
         }
+        const int c = rb / B, b = rb - (rb / B) * B;
         const int t_end = min(T, (c + 1) * C);
         for (int t = c * C + warp; t < t_end; t += kThreads / 32) {
             const size_t at = ((size_t)b * T + t) * (size_t)(H * 64);
@@ -264,7 +275,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_const
     // LayerNorm fused: the rows before n0 (the fast kernel's, or another unit's) are stored
     if (ln.progress != nullptr && tid == 0)
         st_release_gpu(ln.progress + unit, (n0 < 0 || n0 >= NC) ? INT_MAX : n0);
-    if (n0 < 0 || n0 >= NC) return;       // this unit is already complete
+    if (n0 < 0 || n0 >= NC) {             // this unit is already complete
+        if (ln.progress != nullptr)       // its CTA normalises instead
+            ln_blocks(s, ln, y_raw, T, H, seg, units, status, spin_budget);
+        return;
+    }
     const float* state0 = start_chunk ? handoff_state + (size_t)unit * 4096
                         : pseg > 0    ? seg.s_mid + ((size_t)bh * (seg.P - 1) + (pseg - 1)) * 4096
                         : s_in        ? s_in + (size_t)bh * 4096

@@ -117,8 +117,9 @@ cudaError_t launch_chunked_fast(const CUtensorMap* maps, const float* u, const f
 
 // LayerNorm of the fp32 rows y_raw (a token's H heads) inside the level kernel's launch:
 // extra CTAs, co-resident with the recurrence's (a cooperative launch), normalise the
-// 64-token blocks of a batch row as soon as every head has published them.  progress: one
-// word per (b,h,segment) unit, zero before the launch; a unit stores, with release
+// 64-token blocks of a batch row as soon as every head has published them (so do the CTAs
+// of units the fast kernel already finished).  progress: one word per (b,h,segment) unit
+// and a block counter after them, all zero before the launch; a unit stores, with release
 // semantics, the absolute index of the first chunk whose rows it has not yet stored
 // (INT_MAX: all; INT_MIN: it gave up).
 struct LnFuse {

@@ -62,10 +62,11 @@ def test_workspace_queries():
     import torch
     # the chunked path keeps a 256-byte status block and a hand-off record per (b,h)
     # (chunk index, rounded up to 256 bytes in total, and a 16 KB state); LayerNorm with bf16
-    # output adds a progress word per (b,h) unit (rounded up to 256 bytes; the fused
-    # LayerNorm reads it) and an fp32 staging buffer of y; the fp32 recurrence needs nothing
+    # output adds a progress word per (b,h) unit and a block counter (rounded up to 256
+    # bytes; the fused LayerNorm uses them) and an fp32 staging buffer of y; the fp32
+    # recurrence needs nothing
     hand = lambda B, H: 256 + ((B * H * 4 + 255) // 256) * 256 + B * H * 64 * 64 * 4
-    prog = lambda B, H: ((B * H * 4 + 255) // 256) * 256
+    prog = lambda B, H: ((B * H * 4 + 4 + 255) // 256) * 256
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False) == hand(4, 32)
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.bfloat16, False, "recurrent") == 0
     assert binding.prefill_workspace_bytes(4, 16384, 32, 64, torch.float32, True) == 0
