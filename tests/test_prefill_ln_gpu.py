@@ -120,3 +120,25 @@ def test_prefill_ln_second_pass(oracle, B, H, T, algo):
     wider than the in-launch LayerNorm takes): the staged rows go through the second kernel."""
     inp = problem(9700 + B * H + T, B=B, T=T, H=H)
     check(oracle, inp, *run(inp, algo))
+
+
+def test_prefill_ln_graph_capture():
+    """The in-launch LayerNorm is a cooperative launch: captured into a CUDA graph and replayed,
+    the call gives what an eager call gives, bit for bit."""
+    inp = problem(9800, B=2, T=200, H=4)
+    want, _ = run(inp)
+    args = [inp[n] for n in ("r", "k", "v", "omega")]
+    ln = (inp["gamma"], inp["beta"], inp["eps"])
+    warm = torch.cuda.Stream()
+    warm.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(warm):
+        gw.wkv6_prefill(*args, inp["u"], inp["state0"], ln=ln)
+    torch.cuda.current_stream().wait_stream(warm)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        got, _ = gw.wkv6_prefill(*args, inp["u"], inp["state0"], ln=ln)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+    del graph
