@@ -41,7 +41,12 @@
 //             done, while the level products run);
 //   assemble: A from the level accumulators, hi/lo to smem;
 //   MMA 2   : Y += A_hi V + A_lo V;
-//   epilogue: Y -> bf16 -> smem -> TMA store (double-buffered).
+//   epilogue: Y -> bf16 -> smem -> TMA store (double-buffered), or fp32 rows for the
+//             LayerNorm (y_raw).
+// LayerNorm over a token's H heads (the page's final output) can run in the same launch:
+// extra CTAs, and the CTAs of units the fast kernel already finished, normalise 64-token
+// blocks of a batch row once every head has published them (ln_blocks below; a cooperative
+// launch keeps them co-resident with the units they wait for).
 // An M=64 accumulator occupies lanes 0..15 of TMEM sub-partition q for rows 16q..16q+15,
 // so warp w reads rows 16(w%4)..+15, columns split between warps w and w+4.  The state
 // chain and the epilogue read them with a two-half load (lanes 16..31 of the warp get the
