@@ -880,8 +880,13 @@ cudaError_t launch_chunked_levels(const CUtensorMap* maps, const float* u, const
                         (void*)&spin_budget, (void*)&drain, (void*)&lf, (void*)&units};
         e = cudaLaunchCooperativeKernel((const void*)kernel, dim3((unsigned)(units + ln_ctas)),
                                         dim3(kThreads), args, smem, st);
-        if (e == cudaSuccess && ln_done) *ln_done = true;
-        return e;
+        if (e != cudaErrorCooperativeLaunchTooLarge) {
+            if (e == cudaSuccess && ln_done) *ln_done = true;
+            return e;
+        }
+        // fewer slots than the occupancy query promised (another context holds SMs): the
+        // refused launch queued nothing; run the units alone, the caller's pass normalises
+        (void)cudaGetLastError();
     }
     const LnFuse none{nullptr, nullptr, nullptr, 0.f, nullptr};
     kernel<<<(unsigned)units, kThreads, smem, st>>>(
